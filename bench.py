@@ -1,0 +1,507 @@
+"""Benchmark of the KDA operator on B200 (one JSON line on stdout, rank 0).
+
+Default: one GPU, the prefill workload B=4, H=32, T=8192, D_k=D_v=128, C=64
+(BF16 q/k/v, FP32 g/beta/state, zero initial state) as the headline, plus the
+decode workload (512 sequences x 32 heads, 256 steps captured in one CUDA
+graph, FP32 state N(0, 0.02)) as a second object on the same line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload prefill|decode|append_varlen|long] [--no-decode]
+
+For N > 1 it is launched by torchrun, one rank per GPU; every rank runs its
+own copy of the workload (the operator's (sequence, head) units are
+independent, so nothing is exchanged on the data path) and the job time is
+the maximum over ranks.  ``--impl reference`` times the FP64 CPU oracle on a
+bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from linear_attention_08_b200 import inputs as kin  # noqa: E402
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------------------
+# Algorithmic counts ("Kimi K3 architecture" summary, Methods 1: prefill costs
+# 12C^3 + 8C^2 D + 6 C D^2 FLOPs per chunk; decode about 7 D^2 FLOPs and 8 D^2 bytes
+# of FP32 state traffic per head per token).
+# --------------------------------------------------------------------------------------
+def prefill_flops_per_chunk(C: int, D: int) -> int:
+    return 12 * C ** 3 + 8 * C ** 2 * D + 6 * C * D ** 2
+
+
+def prefill_io_bytes_per_token_head(Dk: int, Dv: int, qkv_bytes: int) -> int:
+    # q, k (Dk each) and v (Dv) in the qkv dtype; g (Dk) and beta FP32; o (Dv) in the qkv dtype
+    return qkv_bytes * (2 * Dk + Dv) + 4 * Dk + 4 + qkv_bytes * Dv
+
+
+def decode_state_bytes_per_token_head(Dk: int, Dv: int) -> int:
+    return 8 * Dk * Dv           # FP32 state read + write
+
+
+def decode_flops_per_token_head(D: int) -> int:
+    return 7 * D * D
+
+
+def prefill_algorithmic(lengths, H, Dk, Dv, C, qkv_bytes, interval, has_init):
+    T = sum(lengths)
+    chunks = sum(-(-n // C) for n in lengths)
+    flops = chunks * H * prefill_flops_per_chunk(C, Dk)
+    state = Dk * Dv * 4 * H * len(lengths)
+    n_ck = sum(n // interval for n in lengths) if interval else 0
+    byts = T * H * prefill_io_bytes_per_token_head(Dk, Dv, qkv_bytes) + state \
+        + (state if has_init else 0) + n_ck * H * Dk * Dv * 4
+    return flops, byts
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            p = json.load(fh)
+        return p, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_attention_08_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as fh:
+                h.update(name.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh).get(kernel)
+    if not rec or rec.get("source_sha") != kernel_source_sha():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+# --------------------------------------------------------------------------------------
+# Clocks during the timed region
+# --------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.proc = None
+        self.index = index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.result = None
+        if self.proc is None:
+            return False
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 7]
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[0]))
+                mx = max(mx, float(r[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, r[4:8]):
+                if val.strip().lower() == "active":
+                    reasons.add(name)
+        if sm:
+            busy = [x for x in sm if x > 0.5 * mx] or sm
+            self.result = {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx,
+                           "reasons": sorted(reasons), "samples": len(sm)}
+        return False
+
+
+# --------------------------------------------------------------------------------------
+# Distributed plumbing
+# --------------------------------------------------------------------------------------
+def dist_setup(gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------------------
+# Our arm
+# --------------------------------------------------------------------------------------
+def time_prefill(name, steps, warmup, world, local):
+    from linear_attention_08_b200 import kda
+    w = kin.WORKLOADS[name]
+    d = kin.make_workload(name, device="cuda", seed=local)
+    lengths, cu = d["lengths"], d["cu_seqlens"]
+    cu_dev = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    C, H, Dk, Dv = w["chunk"], w["H"], w["Dk"], w["Dv"]
+    interval = w["ckpt_interval"]
+    init = d["init_state"] if w["state_std"] > 0 else None
+    out = torch.empty_like(d["v"])
+    fin = torch.empty(len(lengths), H, Dk, Dv, device="cuda")
+    n_ck = kda.kda_ckpt_count(cu, interval) if interval else 0
+    ck = torch.empty(max(n_ck, 1), H, Dk, Dv, device="cuda") if interval else None
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], cu_dev, init_state=init,
+                        chunk=C, ckpt_interval=interval, out=out, final_state=fin,
+                        ckpt_states=ck, cu_seqlens_host=cu, stream=stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        barrier(world)
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(steps):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    total_ms = t0.elapsed_time(t1)
+    launch_ms = sum(a.elapsed_time(b) for a, b in ev) / steps
+    barrier(world)
+    total_ms = max_over_ranks(total_ms, world)
+    launch_ms = max_over_ranks(launch_ms, world)
+
+    # End to end through the public API: pinned host inputs -> device -> kernel -> host.
+    host = {x: d[x].to("cpu").pin_memory() for x in ("q", "k", "v", "g", "beta")}
+    h_init = init.to("cpu").pin_memory() if init is not None else None
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_fin = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    dev = {x: torch.empty_like(d[x]) for x in host}
+    d_init = torch.empty_like(init) if init is not None else None
+    bi = sum(t.numel() * t.element_size() for t in host.values()) + \
+        (h_init.numel() * 4 if h_init is not None else 0)
+    bo = h_out.numel() * h_out.element_size() + h_fin.numel() * 4
+    e2e_steps = max(1, min(steps, 5))
+
+    def e2e_step():
+        for x in host:
+            dev[x].copy_(host[x], non_blocking=True)
+        if d_init is not None:
+            d_init.copy_(h_init, non_blocking=True)
+        kda.kda_prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu_dev,
+                        init_state=d_init, chunk=C, ckpt_interval=interval, out=out,
+                        final_state=fin, ckpt_states=ck, cu_seqlens_host=cu, stream=stream)
+        h_out.copy_(out, non_blocking=True)
+        h_fin.copy_(fin, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
+
+    tokens = sum(lengths)
+    flops, byts = prefill_algorithmic(lengths, H, Dk, Dv, C, 2 if w["dtype"] == "bf16" else 4,
+                                      interval, init is not None)
+    path = kda.kda_prefill_path(kda.make_shape(len(lengths), tokens, H, Dk, Dv, C,
+                                               1 if w["dtype"] == "bf16" else 0))
+    return dict(tokens=tokens, steps=steps, total_ms=total_ms, launch_ms=launch_ms,
+                e2e_ms=e2e_ms, bi=bi, bo=bo, flops=flops, bytes=byts, clocks=clk.result,
+                kernel="prefill_tc" if path == 1 else "prefill_simt", w=w, lengths=lengths)
+
+
+def time_decode(steps_graph, warmup, world, local):
+    from linear_attention_08_b200 import kda
+    w = kin.WORKLOADS["decode"]
+    d = kin.make_workload("decode", device="cuda", seed=local)
+    S, N, H, Dk, Dv = w["steps"], w["num_seqs"], w["H"], w["Dk"], w["Dv"]
+    state = d["init_state"].clone()
+    outs = torch.empty_like(d["v"])
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        for t in range(S):   # warm the kernels before capture
+            kda.kda_decode(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], state,
+                           out=outs[t], stream=side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for t in range(S):
+            kda.kda_decode(d["q"][t], d["k"][t], d["v"][t], d["g"][t], d["beta"][t], state,
+                           out=outs[t], stream=side)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(warmup, 1)):
+        graph.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    with ClockSampler(local) as clk:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps_graph):
+            graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / steps_graph, world)
+    # end to end: per-step host inputs in, per-step outputs out (state stays resident)
+    hq = {x: d[x].to("cpu").pin_memory() for x in ("q", "k", "v", "g", "beta")}
+    h_out = torch.empty(outs.shape, dtype=outs.dtype).pin_memory()
+    bi = sum(t.numel() * t.element_size() for t in hq.values())
+    bo = h_out.numel() * h_out.element_size()
+
+    def e2e():
+        for x in hq:
+            d[x].copy_(hq[x], non_blocking=True)
+        graph.replay()
+        h_out.copy_(outs, non_blocking=True)
+
+    e2e()
+    torch.cuda.synchronize()
+    a2, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a2.record(stream)
+    e2e()
+    b2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a2.elapsed_time(b2), world)
+    del graph
+    token_heads = S * N * H
+    byts = token_heads * (decode_state_bytes_per_token_head(Dk, Dv)
+                          + prefill_io_bytes_per_token_head(Dk, Dv, 2))
+    return dict(tokens=S * N, ms=ms, launches=S, e2e_ms=e2e_ms, bi=bi, bo=bo, bytes=byts,
+                flops=token_heads * decode_flops_per_token_head(Dk), clocks=clk.result)
+
+
+def run_ours(args, rank, world, local):
+    peaks, peaks_src = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tflops = peaks["bf16_tflops"]
+    name = args.workload
+    res = time_prefill(name, args.steps, args.warmup, world, local) if name != "decode" else None
+    dec = None
+    if name == "decode" or not args.no_decode:
+        dec = time_decode(max(1, args.steps // 2) if name != "decode" else args.steps,
+                          args.warmup, world, local)
+    if rank != 0:
+        return None
+    if res is not None:
+        r = res
+        w = r["w"]
+        ms_step = r["total_ms"] / r["steps"]
+        value = world * r["tokens"] / (ms_step / 1e3)
+        gbs = r["bytes"] / (r["launch_ms"] / 1e3) / 1e9
+        tfs = r["flops"] / (r["launch_ms"] / 1e3) / 1e12
+        traffic = ncu_traffic(r["kernel"])
+        line = {
+            "metric": "KDA prefill tokens/s", "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": r["steps"], "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if w["dtype"] == "bf16" else "f32",
+            "data": "synthetic",
+            "config": {"workload": name, "num_seqs": w["num_seqs"], "seq_lens": sorted(set(r["lengths"]))[:4],
+                       "total_tokens": r["tokens"], "heads": w["H"], "d_k": w["Dk"], "d_v": w["Dv"],
+                       "chunk": w["chunk"], "ckpt_interval": w["ckpt_interval"],
+                       "state": "fp32", "parallelism": f"replicas{world}",
+                       "l2": "inputs larger than L2 (%.2f GB per step)" % (r["bytes"] / 1e9)},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": gbs / hbm, "traffic": traffic,
+                         "kernel": r["kernel"], "peak_source": peaks_src,
+                         "tensor_tflops": tfs, "tensor_frac": tfs * 1e12 / (tflops * 1e12),
+                         "algorithmic_bytes_per_launch": r["bytes"],
+                         "algorithmic_flops_per_launch": r["flops"]},
+            "e2e": {"value": world * r["tokens"] / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["bi"], "d2h_bytes_per_step": r["bo"]},
+            "gpu_launches": r["steps"],
+            "clocks": r["clocks"],
+        }
+    if dec is not None:
+        dgbs = dec["bytes"] / (dec["ms"] / dec["launches"] / 1e3) / 1e9 / dec["launches"]
+        dobj = {
+            "metric": "KDA decode tokens/s", "value": world * dec["tokens"] / (dec["ms"] / 1e3),
+            "unit": "tokens/s", "ms_per_step": dec["ms"], "steps_per_graph": dec["launches"],
+            "config": {"workload": "decode", "num_seqs": 512, "heads": 32, "d": 128,
+                       "steps": dec["launches"], "l2": "state 2.1 GB > L2"},
+            "roofline": {"bound": "hbm", "achieved": dgbs, "peak": hbm, "unit": "GB/s",
+                         "frac": dgbs / hbm, "traffic": ncu_traffic("decode"),
+                         "kernel": "decode", "peak_source": peaks_src},
+            "e2e": {"value": world * dec["tokens"] / (dec["e2e_ms"] / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": dec["bi"], "d2h_bytes_per_step": dec["bo"]},
+            "gpu_launches": dec["launches"], "clocks": dec["clocks"],
+        }
+        if res is None:
+            line = dict(dobj)
+            line.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                         "dtype": "bf16", "data": "synthetic"})
+        else:
+            line["decode"] = dobj
+    return line
+
+
+# --------------------------------------------------------------------------------------
+# CPU baseline: the FP64 oracle on a bounded sample of the same workload
+# --------------------------------------------------------------------------------------
+def oracle_sample(name, budget_s=12.0):
+    """Time the oracle on the first tokens of a few (sequence, head) units of the
+    workload, growing the sample until about budget_s seconds of CPU work."""
+    import oracle
+    w = kin.WORKLOADS[name]
+    threads = oracle.max_threads()
+    H = w["H"]
+    units = max(threads, 1)
+    tokens = 256
+    if name == "decode":
+        d = kin.make_inputs((w["steps"], 1), units, w["Dk"], w["Dv"], kin.torch_dtype(w["dtype"]),
+                            0, num_states=1, state_std=w["state_std"])
+    while True:
+        if name == "decode":
+            n_steps = min(tokens, w["steps"])
+            sl = lambda x: x[:n_steps]
+            t0 = time.perf_counter()
+            oracle.decode(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["g"]), sl(d["beta"]),
+                          d["init_state"], nthreads=threads)
+            dt = time.perf_counter() - t0
+            token_heads = n_steps * units
+        else:
+            L = tokens
+            di = kin.make_inputs((L,), units, w["Dk"], w["Dv"], kin.torch_dtype(w["dtype"]), 0,
+                                 num_states=1, state_std=w["state_std"])
+            t0 = time.perf_counter()
+            oracle.prefill(di["q"], di["k"], di["v"], di["g"], di["beta"], [0, L],
+                           di["init_state"], 0, 0, threads)
+            dt = time.perf_counter() - t0
+            token_heads = L * units
+        if dt > budget_s / 4 or (name == "decode" and tokens >= w["steps"]):
+            break
+        if name != "decode" and tokens * 2 > max(kin.workload_lengths(name)):
+            units *= 2          # longer than a sequence of the workload: add heads instead
+        else:
+            tokens *= 2
+    tok_per_s = token_heads / dt / H   # a token is H token-heads
+    return {"value": tok_per_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{token_heads} token-heads ({units} heads x {token_heads // units} tokens) "
+                      f"of the {name} workload, FP64 recurrence, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    name = args.workload
+    per_step = []
+    for _ in range(args.warmup):
+        oracle_sample(name, budget_s=2.0)
+    base = None
+    for _ in range(args.steps):
+        base = oracle_sample(name, budget_s=8.0)
+        per_step.append(base["value"])
+    value = statistics.median(per_step)
+    base["value"] = value
+    return {"metric": "KDA decode tokens/s" if name == "decode" else "KDA prefill tokens/s",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference", "config": {"workload": name},
+            "cpu_baseline": base,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill",
+                    choices=["prefill", "decode", "append_varlen", "long"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        line = run_reference(args, rank, int(os.environ.get("WORLD_SIZE", "1")))
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    rank, world, local = dist_setup(args.gpus)
+    line = run_ours(args, rank, world, local)
+    if rank == 0 and line is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(args.workload)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,141 @@
+/*
+ * kda.h -- C ABI of a B200 (sm_100a) implementation of Kimi Delta Attention.
+ *
+ * KDA is a gated delta-rule linear attention with one forget gate per key
+ * channel ("Kimi K3 architecture" summary, charstring.tistory.com/2557,
+ * Background: Gated DeltaNet's scalar gate widened to a diagonal matrix).
+ * For one (sequence, head), with a D_k x D_v FP32 state S (row = key channel):
+ *
+ *     alpha_t = exp(g_t)                           (natural log-decay, per channel)
+ *     S_t     = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t     = S_t^T q_t
+ *
+ * Preconditions on the data (not checked on the device): g in [-5, 0] (the
+ * lower-bounded decay of the Kimi-K3 deep dive, fiv.co.kr, section 4-1),
+ * beta in [0, 1], finite inputs.  No 1/sqrt(D) scale is applied to q, and q,
+ * k, beta, g are used as given (no normalisation, sigmoid or clamp inside).
+ *
+ * Layouts (all dense, row-major, no padding):
+ *   q, k, g : [T_tot, H, D_k]     v, out : [T_tot, H, D_v]     beta : [T_tot, H]
+ *   states  : [N, H, D_k, D_v] FP32
+ *   checkpoints : [n_ckpt, H, D_k, D_v] FP32, packed sequence by sequence.
+ * q, k, v and out share one dtype (FP32 or BF16); g, beta and states are FP32.
+ *
+ * Ownership and streams: the caller owns every buffer; all pointers are
+ * device pointers unless a comment says "host".  Every call is asynchronous
+ * on the given stream and never synchronises.  The library keeps no device
+ * allocation of its own between calls.
+ *
+ * Errors: argument problems return KDA_ERR_INVALID_ARGUMENT or
+ * KDA_ERR_UNSUPPORTED before anything is launched.  A failed launch returns
+ * KDA_ERR_CUDA; kda_last_cuda_error() gives the cudaError_t value.  Kernels
+ * with bounded waits write KDA_ERR_TIMEOUT to shape->dev_status (when it is
+ * not NULL) instead of hanging; the caller reads it after synchronising.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st *kda_stream_t;
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misalignment          */
+  KDA_ERR_UNSUPPORTED = 2,      /* a head size or chunk size this build lacks    */
+  KDA_ERR_CUDA = 3,             /* a CUDA call failed; see kda_last_cuda_error() */
+  KDA_ERR_TIMEOUT = 4           /* written to dev_status by a bounded wait       */
+} kda_status;
+
+typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
+
+typedef struct {
+  int32_t num_seqs;     /* N >= 1                                                  */
+  int64_t total_tokens; /* T_tot = cu_seqlens[N] (prefill); N (decode)             */
+  int32_t num_heads;    /* H >= 1                                                  */
+  int32_t head_dim_k;   /* D_k in {32, 64, 128}                                    */
+  int32_t head_dim_v;   /* D_v in {32, 64, 128}                                    */
+  int32_t chunk;        /* C in {16, 64} (prefill); ignored by decode              */
+  int32_t qkv_dtype;    /* kda_dtype of q, k, v and out                            */
+  int32_t *dev_status;  /* optional device int32, 0 = fine, else a kda_status      */
+} kda_shape;
+
+/*
+ * Chunked prefill ("Kimi K3 architecture" summary, Methods 1, FlashKDA: the
+ * recurrence unrolled over chunks into matrix products; deep dive section
+ * 4-1: 16-token tiles with a recurrence between tiles) and state
+ * checkpoints for prefix caching (summary, Methods 3: the state is kept only
+ * at coarse positions such as every 32K tokens).
+ *
+ *   q, k, v, g, beta : inputs in the layouts above (beta needs 4-byte alignment).
+ *   init_state       : [N, H, D_k, D_v] or NULL for zeros (append-prefill
+ *                      after a cached prefix passes the cached state here).
+ *   cu_seqlens       : device int32[N+1], cu_seqlens[0] = 0, non-decreasing,
+ *                      cu_seqlens[N] = total_tokens.  Not checked on the device.
+ *   out              : [T_tot, H, D_v], written for every token.
+ *   final_state      : [N, H, D_k, D_v] or NULL; may alias init_state.
+ *   ckpt_interval    : 0 = no checkpoints; else a positive multiple of chunk.
+ *                      Sequence i stores its state after every ckpt_interval
+ *                      of its own tokens (counted from its first token, the
+ *                      end included when T_i is a multiple).
+ *   ckpt_states      : [kda_ckpt_count(...), H, D_k, D_v]; NULL iff interval 0.
+ * Every other pointer must be 16-byte aligned; out must not overlap any input.
+ */
+kda_status kda_prefill(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                       void *out, float *final_state, int64_t ckpt_interval,
+                       float *ckpt_states, const kda_shape *shape, kda_stream_t stream);
+
+/*
+ * One decode step for N sequences (summary, Methods 1: decode runs the
+ * recurrence directly; about 7 D^2 FLOPs and 8 D^2 bytes of FP32 state
+ * traffic per head per token).
+ *
+ *   q, k, v, g : [N, H, D]   beta : [N, H]   out : [N, H, D_v]
+ *   state_inout: [N, H, D_k, D_v], read and overwritten in place.
+ * shape->total_tokens must equal shape->num_seqs; shape->chunk is ignored.
+ */
+kda_status kda_decode(const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, float *state_inout, void *out,
+                      const kda_shape *shape, kda_stream_t stream);
+
+/* Host helper: sum_i floor(T_i / ckpt_interval) for host int32 cu_seqlens[N+1]
+ * (0 when ckpt_interval <= 0; -1 on a bad argument). */
+int64_t kda_ckpt_count(const int32_t *host_cu_seqlens, int32_t num_seqs, int64_t ckpt_interval);
+
+/* Bytes of device scratch kda_prefill needs for this shape beyond its
+ * arguments.  The prefill kernels in this build carry the state on chip and
+ * need none, so this is 0 for every valid shape and (size_t)-1 for an
+ * invalid one. */
+size_t kda_prefill_workspace_bytes(const kda_shape *shape);
+
+/* Which prefill kernel a shape runs on: 1 = tcgen05 tensor-core kernel,
+ * 0 = SIMT FP32 kernel, -1 = invalid shape. */
+int kda_prefill_path(const kda_shape *shape);
+
+/* Bounded-wait self-test: launches one CTA that waits on an mbarrier that
+ * nothing arrives at, with the same bounded wait the tensor-core kernel
+ * uses, giving up after max_polls polls.  The kernel writes
+ * KDA_ERR_TIMEOUT to *dev_status and exits, so the context stays usable. */
+kda_status kda_selftest_bounded_wait(int32_t *dev_status, int64_t max_polls,
+                                     kda_stream_t stream);
+
+/* The cudaError_t of the last KDA_ERR_CUDA on this thread. */
+int kda_last_cuda_error(void);
+
+const char *kda_status_string(kda_status status);
+
+/* Library version as an integer: major * 10000 + minor * 100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

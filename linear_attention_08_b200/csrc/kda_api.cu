@@ -1,0 +1,188 @@
+// C ABI of the KDA library: argument checks, kernel choice and launch.
+#include <stdint.h>
+#include <stdio.h>
+
+#include "kda_common.cuh"
+
+namespace kda {
+cudaError_t launch_decode(int dtype, int dk, int dv, const void *q, const void *k, const void *v,
+                          const float *g, const float *beta, float *state, void *out,
+                          int64_t units, int H, cudaStream_t stream);
+cudaError_t launch_prefill_simt(int dtype, int dk, int dv, const void *q, const void *k,
+                                const void *v, const float *g, const float *beta,
+                                const float *init, const int32_t *cu, void *out, float *fin,
+                                int64_t interval, float *ck, int N, int H, cudaStream_t stream);
+bool prefill_tc_supported(int dtype, int dk, int dv, int chunk);
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *init, const int32_t *cu,
+                              void *out, float *fin, int64_t interval, float *ck, int N, int H,
+                              int64_t total_tokens, int32_t *dev_status, cudaStream_t stream);
+
+static thread_local int g_last_cuda_error = 0;
+
+static kda_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return KDA_OK;
+  g_last_cuda_error = (int)e;
+  return KDA_ERR_CUDA;
+}
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+static size_t elem_size(int dtype) { return dtype == KDA_DTYPE_BF16 ? 2 : 4; }
+
+// Byte ranges [a, a + na) and [b, b + nb) overlap.
+static bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+// Common shape checks; returns KDA_OK or the status to report.
+static kda_status check_shape(const kda_shape *s, bool prefill) {
+  if (!s) return KDA_ERR_INVALID_ARGUMENT;
+  if (s->num_seqs < 1 || s->num_heads < 1 || s->total_tokens < 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (s->qkv_dtype != KDA_DTYPE_F32 && s->qkv_dtype != KDA_DTYPE_BF16)
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (!head_dim_ok(s->head_dim_k) || !head_dim_ok(s->head_dim_v)) return KDA_ERR_UNSUPPORTED;
+  if (prefill && s->chunk != 16 && s->chunk != 64) return KDA_ERR_UNSUPPORTED;
+  if ((int64_t)s->num_seqs * s->num_heads > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  if (s->dev_status && (reinterpret_cast<uintptr_t>(s->dev_status) & 3u))
+    return KDA_ERR_INVALID_ARGUMENT;
+  return KDA_OK;
+}
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+int kda_version(void) { return 100; }
+
+int kda_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *kda_status_string(kda_status s) {
+  switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_INVALID_ARGUMENT: return "invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "unsupported shape";
+    case KDA_ERR_CUDA: return "CUDA error";
+    case KDA_ERR_TIMEOUT: return "bounded wait timed out on the device";
+  }
+  return "unknown status";
+}
+
+int64_t kda_ckpt_count(const int32_t *host_cu_seqlens, int32_t num_seqs, int64_t ckpt_interval) {
+  if (ckpt_interval <= 0) return 0;
+  if (!host_cu_seqlens || num_seqs < 0) return -1;
+  int64_t n = 0;
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    const int64_t len = (int64_t)host_cu_seqlens[i + 1] - host_cu_seqlens[i];
+    if (len < 0) return -1;
+    n += len / ckpt_interval;
+  }
+  return n;
+}
+
+size_t kda_prefill_workspace_bytes(const kda_shape *shape) {
+  return check_shape(shape, true) == KDA_OK ? 0 : (size_t)-1;
+}
+
+int kda_prefill_path(const kda_shape *s) {
+  if (check_shape(s, true) != KDA_OK) return -1;
+  return prefill_tc_supported(s->qkv_dtype, s->head_dim_k, s->head_dim_v, s->chunk) ? 1 : 0;
+}
+
+kda_status kda_prefill(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                       void *out, float *final_state, int64_t ckpt_interval,
+                       float *ckpt_states, const kda_shape *s, kda_stream_t stream) {
+  kda_status st = check_shape(s, true);
+  if (st != KDA_OK) return st;
+  const int N = s->num_seqs, H = s->num_heads, DK = s->head_dim_k, DV = s->head_dim_v;
+  const int64_t T = s->total_tokens;
+  if (!cu_seqlens || !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARGUMENT;
+  if (T > INT32_MAX) return KDA_ERR_UNSUPPORTED;  // cu_seqlens are int32
+  if (T > 0) {
+    const void *ptrs[] = {q, k, v, g, out};
+    for (const void *p : ptrs)
+      if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    if (!beta || (reinterpret_cast<uintptr_t>(beta) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
+  }
+  if (init_state && !aligned16(init_state)) return KDA_ERR_INVALID_ARGUMENT;
+  if (final_state && !aligned16(final_state)) return KDA_ERR_INVALID_ARGUMENT;
+  if (ckpt_interval < 0 || ckpt_interval % s->chunk != 0) return KDA_ERR_INVALID_ARGUMENT;
+  if ((ckpt_interval > 0) != (ckpt_states != nullptr)) return KDA_ERR_INVALID_ARGUMENT;
+  if (ckpt_states && !aligned16(ckpt_states)) return KDA_ERR_INVALID_ARGUMENT;
+  const size_t es = elem_size(s->qkv_dtype);
+  const size_t n_out = (size_t)T * H * DV * es;
+  const size_t n_qk = (size_t)T * H * DK * es, n_v = (size_t)T * H * DV * es;
+  const size_t n_g = (size_t)T * H * DK * 4, n_b = (size_t)T * H * 4;
+  const size_t n_state = (size_t)N * H * DK * DV * 4;
+  if (overlaps(out, n_out, q, n_qk) || overlaps(out, n_out, k, n_qk) ||
+      overlaps(out, n_out, v, n_v) || overlaps(out, n_out, g, n_g) ||
+      overlaps(out, n_out, beta, n_b) || overlaps(out, n_out, init_state, n_state) ||
+      overlaps(out, n_out, final_state, n_state))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (final_state && init_state && final_state != init_state &&
+      overlaps(final_state, n_state, init_state, n_state))
+    return KDA_ERR_INVALID_ARGUMENT;  // exact aliasing is fine, partial overlap is not
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (prefill_tc_supported(s->qkv_dtype, DK, DV, s->chunk))
+    e = launch_prefill_tc(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
+                          ckpt_interval, ckpt_states, N, H, T, s->dev_status, cs);
+  else
+    e = launch_prefill_simt(s->qkv_dtype, DK, DV, q, k, v, g, beta, init_state, cu_seqlens, out,
+                            final_state, ckpt_interval, ckpt_states, N, H, cs);
+  return cuda_status(e);
+}
+
+kda_status kda_decode(const void *q, const void *k, const void *v, const float *g,
+                      const float *beta, float *state_inout, void *out, const kda_shape *s,
+                      kda_stream_t stream) {
+  kda_status st = check_shape(s, false);
+  if (st != KDA_OK) return st;
+  if (s->total_tokens != s->num_seqs) return KDA_ERR_INVALID_ARGUMENT;
+  const void *ptrs[] = {q, k, v, g, state_inout, out};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!beta || (reinterpret_cast<uintptr_t>(beta) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
+  const int64_t units = (int64_t)s->num_seqs * s->num_heads;
+  const size_t es = elem_size(s->qkv_dtype);
+  const size_t n_out = (size_t)units * s->head_dim_v * es;
+  const size_t n_state = (size_t)units * s->head_dim_k * s->head_dim_v * 4;
+  if (overlaps(out, n_out, state_inout, n_state) ||
+      overlaps(out, n_out, q, (size_t)units * s->head_dim_k * es) ||
+      overlaps(out, n_out, k, (size_t)units * s->head_dim_k * es) ||
+      overlaps(out, n_out, v, n_out) || overlaps(out, n_out, g, (size_t)units * s->head_dim_k * 4))
+    return KDA_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_decode(s->qkv_dtype, s->head_dim_k, s->head_dim_v, q, k, v, g, beta,
+                                   state_inout, out, units, s->num_heads,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+namespace kda {
+__global__ void selftest_wait_kernel(int32_t *dev_status, int64_t max_polls) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  // Nothing ever arrives: the wait must give up and report.
+  if (threadIdx.x == 0 && !mbar_wait_bounded(&bar, 0, max_polls)) report(dev_status, KDA_ERR_TIMEOUT);
+}
+}  // namespace kda
+
+extern "C" kda_status kda_selftest_bounded_wait(int32_t *dev_status, int64_t max_polls,
+                                                kda_stream_t stream) {
+  if (!dev_status || max_polls < 0 || max_polls > (int64_t(1) << 24)) return KDA_ERR_INVALID_ARGUMENT;
+  kda::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(dev_status,
+                                                                                  max_polls);
+  return kda::cuda_status(cudaGetLastError());
+}

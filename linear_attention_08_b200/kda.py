@@ -1,0 +1,170 @@
+"""Thin ctypes binding of libkda.so (the C ABI declared in include/kda.h).
+
+Argument marshalling only: every step of the operator runs in the CUDA
+kernels behind the C ABI.  PyTorch provides device memory and streams.  There
+is no fallback: if the library is missing or a call fails, this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARGUMENT, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
+KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
+
+EXPORTED = ("kda_prefill", "kda_decode", "kda_ckpt_count", "kda_prefill_workspace_bytes",
+            "kda_prefill_path", "kda_selftest_bounded_wait", "kda_last_cuda_error",
+            "kda_status_string", "kda_version")
+
+
+class KdaShape(ctypes.Structure):
+    _fields_ = [("num_seqs", ctypes.c_int32), ("total_tokens", ctypes.c_int64),
+                ("num_heads", ctypes.c_int32), ("head_dim_k", ctypes.c_int32),
+                ("head_dim_v", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("qkv_dtype", ctypes.c_int32), ("dev_status", ctypes.c_void_p)]
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = _lib_or_none().kda_status_string(status).decode() if _lib_or_none() else str(status)
+        if status == KDA_ERR_CUDA and _lib_or_none():
+            msg += f" (cudaError {_lib_or_none().kda_last_cuda_error()})"
+        super().__init__(f"{what}: {msg}")
+
+
+_lib = None
+
+
+def _lib_or_none():
+    return _lib
+
+
+def load(path: str | None = None):
+    """Load libkda.so (cached); raises if it has not been built.  An explicit
+    ``path`` loads that file without touching the cache."""
+    global _lib
+    if path is None and _lib is not None:
+        return _lib
+    explicit = path is not None
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m linear_attention_08_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, I64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+    SP = ctypes.POINTER(KdaShape)
+    lib.kda_prefill.argtypes = [P, P, P, P, P, P, P, P, P, I64, P, SP, P]
+    lib.kda_prefill.restype = ctypes.c_int
+    lib.kda_decode.argtypes = [P, P, P, P, P, P, P, SP, P]
+    lib.kda_decode.restype = ctypes.c_int
+    lib.kda_ckpt_count.argtypes = [P, I32, I64]
+    lib.kda_ckpt_count.restype = I64
+    lib.kda_prefill_workspace_bytes.argtypes = [SP]
+    lib.kda_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_prefill_path.argtypes = [SP]
+    lib.kda_prefill_path.restype = ctypes.c_int
+    lib.kda_selftest_bounded_wait.argtypes = [P, I64, P]
+    lib.kda_selftest_bounded_wait.restype = ctypes.c_int
+    lib.kda_last_cuda_error.restype = ctypes.c_int
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_version.restype = ctypes.c_int
+    if not explicit:
+        _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_DTYPE_BF16
+    if t.dtype == torch.float32:
+        return KDA_DTYPE_F32
+    raise TypeError(f"q/k/v must be float32 or bfloat16, got {t.dtype}")
+
+
+def make_shape(num_seqs, total_tokens, H, Dk, Dv, chunk, dtype_code, dev_status=None) -> KdaShape:
+    return KdaShape(int(num_seqs), int(total_tokens), int(H), int(Dk), int(Dv), int(chunk),
+                    int(dtype_code), None if dev_status is None else dev_status.data_ptr())
+
+
+def kda_ckpt_count(cu_seqlens_host, ckpt_interval: int) -> int:
+    cu = (ctypes.c_int32 * len(cu_seqlens_host))(*[int(x) for x in cu_seqlens_host])
+    n = load().kda_ckpt_count(cu, len(cu_seqlens_host) - 1, int(ckpt_interval))
+    if n < 0:
+        raise ValueError("bad cu_seqlens")
+    return int(n)
+
+
+def kda_prefill_path(shape: KdaShape) -> int:
+    return int(load().kda_prefill_path(ctypes.byref(shape)))
+
+
+def kda_prefill(q, k, v, g, beta, cu_seqlens, *, init_state=None, chunk: int = 64,
+                ckpt_interval: int = 0, cu_seqlens_host=None, out=None, final_state=None,
+                ckpt_states=None, dev_status=None, stream=None, want_final: bool = True):
+    """Chunked KDA prefill over a packed batch (see kda_prefill in include/kda.h).
+
+    q, k, g: [T, H, Dk]; v: [T, H, Dv]; beta: [T, H]; cu_seqlens: int32 device
+    [N+1]; init_state: [N, H, Dk, Dv] FP32 or None.  Outputs are allocated
+    with torch when not given.  ``cu_seqlens_host`` (a list) avoids a device
+    read when checkpoints are requested.  Returns (out, final_state, ckpt_states).
+    """
+    lib = load()
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty(T, H, Dv, dtype=q.dtype, device=q.device)
+    if final_state is None and want_final:
+        final_state = torch.empty(N, H, Dk, Dv, dtype=torch.float32, device=q.device)
+    if ckpt_interval > 0 and ckpt_states is None:
+        host = cu_seqlens_host if cu_seqlens_host is not None else cu_seqlens.tolist()
+        n = kda_ckpt_count(host, ckpt_interval)
+        ckpt_states = torch.empty(max(n, 1), H, Dk, Dv, dtype=torch.float32, device=q.device)[:n]
+    shape = make_shape(N, T, H, Dk, Dv, chunk, _dtype_code(q), dev_status)
+    ck_ptr = _ptr(ckpt_states) if ckpt_interval > 0 else None
+    if ckpt_interval > 0 and ckpt_states.numel() == 0:
+        ck_ptr = ctypes.c_void_p(ckpt_states.untyped_storage().data_ptr())
+    st = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init_state),
+                         _ptr(cu_seqlens), _ptr(out), _ptr(final_state), int(ckpt_interval),
+                         ck_ptr, ctypes.byref(shape), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_prefill")
+    return out, final_state, ckpt_states
+
+
+def kda_decode(q, k, v, g, beta, state, *, out=None, dev_status=None, stream=None):
+    """One decode step: q, k, g [N, H, Dk]; v [N, H, Dv]; beta [N, H]; state
+    [N, H, Dk, Dv] FP32 updated in place.  Returns out [N, H, Dv]."""
+    lib = load()
+    N, H, Dk = q.shape
+    Dv = v.shape[2]
+    if out is None:
+        out = torch.empty(N, H, Dv, dtype=q.dtype, device=q.device)
+    shape = make_shape(N, N, H, Dk, Dv, 0, _dtype_code(q), dev_status)
+    st = lib.kda_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state), _ptr(out),
+                        ctypes.byref(shape), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode")
+    return out
+
+
+def kda_selftest_bounded_wait(dev_status, max_polls: int, stream=None) -> None:
+    st = load().kda_selftest_bounded_wait(_ptr(dev_status), int(max_polls), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_selftest_bounded_wait")

@@ -1,0 +1,114 @@
+"""Host-side checks of the C ABI that need no GPU: exports and argument validation."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from linear_attention_08_b200 import kda
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    text = open(os.path.join(ROOT, "include", "kda.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_function():
+    lib = kda.load()
+    names = header_functions()
+    assert "kda_prefill" in names and "kda_decode" in names
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/kda.h but not exported"
+    assert set(kda.EXPORTED) <= set(names)
+
+
+def test_version_and_strings():
+    lib = kda.load()
+    assert lib.kda_version() >= 100
+    for s in range(5):
+        assert lib.kda_status_string(s)
+
+
+def test_ckpt_count():
+    assert kda.kda_ckpt_count([0, 5000, 9000, 9000], 4096) == 1
+    assert kda.kda_ckpt_count([0, 8192, 16384], 4096) == 4
+    assert kda.kda_ckpt_count([0, 100], 0) == 0
+    # the 1M-token workload with 32K snapshots stores 32 of them
+    assert kda.kda_ckpt_count([0, 1 << 20], 32768) == 32
+
+
+def _shape(**kw):
+    base = dict(num_seqs=2, total_tokens=64, H=2, Dk=32, Dv=32, chunk=16, dtype_code=0)
+    base.update(kw)
+    return kda.make_shape(base["num_seqs"], base["total_tokens"], base["H"], base["Dk"],
+                          base["Dv"], base["chunk"], base["dtype_code"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(Dk=48), kda.KDA_ERR_UNSUPPORTED),
+    (dict(Dv=256), kda.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=32), kda.KDA_ERR_UNSUPPORTED),
+    (dict(num_seqs=0), kda.KDA_ERR_INVALID_ARGUMENT),
+    (dict(H=0), kda.KDA_ERR_INVALID_ARGUMENT),
+    (dict(dtype_code=7), kda.KDA_ERR_INVALID_ARGUMENT),
+    (dict(total_tokens=-1), kda.KDA_ERR_INVALID_ARGUMENT),
+])
+def test_prefill_rejects_bad_shapes_before_launch(kw, status):
+    lib = kda.load()
+    s = _shape(**kw)
+    fake = ctypes.c_void_p(1 << 20)  # never dereferenced: validation fails first
+    st = lib.kda_prefill(fake, fake, fake, fake, fake, None, fake, fake, None, 0, None,
+                         ctypes.byref(s), None)
+    assert st == status
+
+
+def test_prefill_rejects_bad_pointers_and_intervals():
+    lib = kda.load()
+    s = _shape()
+    a = ctypes.c_void_p(1 << 20)
+    b = ctypes.c_void_p(1 << 24)
+    c = ctypes.c_void_p(1 << 28)
+    mis = ctypes.c_void_p((1 << 20) + 4)
+    call = lambda *args: lib.kda_prefill(*args, ctypes.byref(s), None)
+    # null cu_seqlens / null q
+    assert call(a, a, a, a, a, None, None, b, None, 0, None) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert call(None, a, a, a, a, None, a, b, None, 0, None) == kda.KDA_ERR_INVALID_ARGUMENT
+    # misaligned q
+    assert call(mis, a, a, a, a, None, a, b, None, 0, None) == kda.KDA_ERR_INVALID_ARGUMENT
+    # interval not a multiple of the chunk; interval without a buffer; buffer without interval
+    assert call(a, a, a, a, a, None, a, b, None, 24, c) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert call(a, a, a, a, a, None, a, b, None, 32, None) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert call(a, a, a, a, a, None, a, b, None, 0, c) == kda.KDA_ERR_INVALID_ARGUMENT
+    # out overlapping an input
+    assert call(a, a, a, a, a, None, c, a, None, 0, None) == kda.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_decode_rejects_bad_arguments():
+    lib = kda.load()
+    a = ctypes.c_void_p(1 << 20)
+    b = ctypes.c_void_p(1 << 26)
+    s = kda.make_shape(4, 5, 2, 32, 32, 0, 1)   # total_tokens != num_seqs
+    assert lib.kda_decode(a, a, a, a, a, b, ctypes.c_void_p(1 << 28), ctypes.byref(s),
+                          None) == kda.KDA_ERR_INVALID_ARGUMENT
+    s = kda.make_shape(4, 4, 2, 32, 32, 0, 1)
+    # out aliasing the state
+    assert lib.kda_decode(a, a, a, a, a, b, b, ctypes.byref(s), None) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_decode(a, a, a, a, a, b, ctypes.c_void_p(1 << 28), None,
+                          None) == kda.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_workspace_and_path_queries():
+    lib = kda.load()
+    s = _shape()
+    assert lib.kda_prefill_workspace_bytes(ctypes.byref(s)) == 0
+    assert kda.kda_prefill_path(s) == 0            # FP32 runs on the SIMT kernel
+    bad = _shape(Dk=12)
+    assert kda.kda_prefill_path(bad) == -1
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    with pytest.raises(ImportError):
+        kda.load(str(tmp_path / "missing.so"))

@@ -1,0 +1,221 @@
+"""Prefill parity: the CUDA path through the C ABI against the FP64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+from linear_attention_08_b200 import inputs as kin
+from linear_attention_08_b200 import kda
+from parity import (TOL, ckpt_base, gpu_prefill, make_case, oracle_full, oracle_unit, rel_l2,
+                    to_device)
+
+pytestmark = pytest.mark.gpu
+
+
+def check_full(d, chunk, interval=0, use_init=True, tol=None, **kw):
+    dd = to_device(d)
+    out, fin, ck = gpu_prefill(dd, chunk, interval, use_init, **kw)
+    torch.cuda.synchronize()
+    ro, rf, rc = oracle_full(d, interval, use_init)
+    tol = tol or TOL[d["q"].dtype]
+    errs = {"o": rel_l2(out, ro), "S": rel_l2(fin, rf)}
+    if interval > 0:
+        assert ck.shape[0] == rc.shape[0]
+        if rc.shape[0]:
+            errs["ckpt"] = rel_l2(ck, rc)
+    for name, e in errs.items():
+        assert e <= tol, f"{name}: rel-L2 {e:.3e} > {tol:.0e}"
+    return errs
+
+
+def test_tiny_workload_fp32():
+    """B=1, H=2, T=64, D=32, FP32, C=16, zero initial state: o and final state within 1e-4."""
+    d = kin.make_workload("tiny")
+    assert d["q"].dtype == torch.float32
+    check_full(d, chunk=16, use_init=False, tol=1e-4)
+    check_full(d, chunk=64, use_init=False, tol=1e-4)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dims", [(32, 32), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("chunk", [16, 64])
+def test_ragged_varlen(dtype, dims, chunk):
+    """Several sequences with ragged tails around the tile size, nonzero initial state,
+    checkpoints every two chunks."""
+    Dk, Dv = dims
+    lengths = [1, chunk - 1, chunk, chunk + 1, 3 * chunk + 5, 130]
+    d = make_case(lengths, 3, Dk, Dv, dtype, seed=1, state_std=0.1)
+    check_full(d, chunk, interval=2 * chunk)
+
+
+@pytest.mark.parametrize("chunk", [16, 64])
+def test_decay_at_floor_and_extremes(chunk):
+    """g = -5 everywhere (the floor), g = 0, beta in {0, 1}."""
+    lengths = [200, 77]
+    for gval, bval in [(-5.0, None), (0.0, None), (None, 0.0), (None, 1.0), (-5.0, 1.0)]:
+        d = make_case(lengths, 2, 128, 128, torch.bfloat16, seed=2, state_std=0.5)
+        if gval is not None:
+            d["g"].fill_(gval)
+        if bval is not None:
+            d["beta"].fill_(bval)
+        check_full(d, chunk, interval=chunk)
+
+
+def test_identity_tokens_keep_state():
+    """beta = 0 and g = 0: the final state is the initial one and o_t = S0^T q_t."""
+    d = make_case([50, 13], 2, 64, 32, torch.float32, seed=3, state_std=1.0)
+    d["beta"].zero_()
+    d["g"].zero_()
+    dd = to_device(d)
+    out, fin, _ = gpu_prefill(dd, 16)
+    torch.cuda.synchronize()
+    assert torch.allclose(fin.cpu(), d["init_state"], rtol=0, atol=1e-6)
+
+
+def test_empty_sequences_and_empty_batch():
+    d = make_case([0, 40, 0, 17, 0], 2, 32, 32, torch.float32, seed=4, state_std=0.3)
+    check_full(d, 16, interval=16)
+    # an all-empty batch only copies init to final
+    d0 = make_case([0, 0], 2, 32, 32, torch.float32, seed=5, state_std=0.3)
+    dd = to_device(d0)
+    out, fin, _ = gpu_prefill(dd, 16)
+    torch.cuda.synchronize()
+    assert out.numel() == 0 and torch.equal(fin.cpu(), d0["init_state"])
+
+
+def test_null_init_is_zero_and_final_aliases_init():
+    d = make_case([90, 33], 2, 128, 128, torch.bfloat16, seed=6, state_std=0.0)
+    dd = to_device(d)
+    o1, f1, _ = gpu_prefill(dd, 64, use_init=False)
+    o2, f2, _ = gpu_prefill(dd, 64, use_init=True)          # explicit zeros
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(f1, f2)
+    d2 = make_case([90, 33], 2, 128, 128, torch.bfloat16, seed=6, state_std=0.2)
+    dd2 = to_device(d2)
+    o3, f3, _ = gpu_prefill(dd2, 64)
+    st = dd2["init_state"].clone()
+    o4, f4, _ = kda.kda_prefill(dd2["q"], dd2["k"], dd2["v"], dd2["g"], dd2["beta"], dd2["cu_dev"],
+                                init_state=st, final_state=st, chunk=64)
+    torch.cuda.synchronize()
+    assert torch.equal(o3, o4) and torch.equal(f3, st)
+
+
+def test_deterministic():
+    d = make_case([300, 129], 4, 128, 128, torch.bfloat16, seed=7)
+    dd = to_device(d)
+    a = gpu_prefill(dd, 64, 128)
+    b = gpu_prefill(dd, 64, 128)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
+
+
+def test_varlen_equals_separate_calls():
+    lengths = [70, 5, 129]
+    d = make_case(lengths, 2, 128, 128, torch.bfloat16, seed=8)
+    dd = to_device(d)
+    out, fin, _ = gpu_prefill(dd, 64)
+    cu = d["cu_seqlens"]
+    for n in range(len(lengths)):
+        a, b = cu[n], cu[n + 1]
+        o_n, f_n, _ = kda.kda_prefill(dd["q"][a:b].contiguous(), dd["k"][a:b].contiguous(),
+                                      dd["v"][a:b].contiguous(), dd["g"][a:b].contiguous(),
+                                      dd["beta"][a:b].contiguous(),
+                                      torch.tensor([0, b - a], dtype=torch.int32, device="cuda"),
+                                      init_state=dd["init_state"][n:n + 1].contiguous(), chunk=64)
+        torch.cuda.synchronize()
+        assert torch.equal(o_n, out[a:b]) and torch.equal(f_n[0], fin[n])
+
+
+def test_checkpoint_resume():
+    """Resuming from checkpoint j reproduces the rest of the sequence."""
+    L, interval = 640, 128
+    d = make_case([L], 2, 128, 128, torch.bfloat16, seed=9)
+    dd = to_device(d)
+    out, fin, ck = gpu_prefill(dd, 64, interval)
+    assert ck.shape[0] == L // interval
+    for j in (1, 3):
+        n = j * interval
+        o_r, f_r, _ = kda.kda_prefill(dd["q"][n:].contiguous(), dd["k"][n:].contiguous(),
+                                      dd["v"][n:].contiguous(), dd["g"][n:].contiguous(),
+                                      dd["beta"][n:].contiguous(),
+                                      torch.tensor([0, L - n], dtype=torch.int32, device="cuda"),
+                                      init_state=ck[j - 1:j].contiguous(), chunk=64)
+        torch.cuda.synchronize()
+        assert rel_l2(o_r, out[n:].double().cpu().numpy()) < 1e-5
+        assert rel_l2(f_r, fin.double().cpu().numpy()) < 1e-5
+
+
+# ---------------------------------------------------------------------------------------
+# The full-size workloads, in the launch configuration the benchmark times, compared on
+# sampled (sequence, head) units.
+# ---------------------------------------------------------------------------------------
+def sampled_units(N, H, count, seed):
+    rng = np.random.default_rng(seed)
+    picks = {(0, 0), (N - 1, H - 1)}
+    while len(picks) < count:
+        picks.add((int(rng.integers(N)), int(rng.integers(H))))
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("name", ["prefill", "append_varlen"])
+def test_full_workload_sampled(name):
+    w = kin.WORKLOADS[name]
+    d = kin.make_workload(name, device="cuda")
+    d["cu_dev"] = torch.tensor(d["cu_seqlens"], dtype=torch.int32, device="cuda")
+    interval = w["ckpt_interval"]
+    use_init = w["state_std"] > 0
+    out, fin, ck = kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_dev"],
+                                   init_state=d["init_state"] if use_init else None,
+                                   chunk=w["chunk"], ckpt_interval=interval,
+                                   cu_seqlens_host=d["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all() and torch.isfinite(fin).all()
+    cu = d["cu_seqlens"]
+    for seq, h in sampled_units(len(d["lengths"]), w["H"], 4, seed=len(name)):
+        ro, rf, rc = oracle_unit(d, seq, h, interval, use_init)
+        a, b = cu[seq], cu[seq + 1]
+        assert rel_l2(out[a:b, h:h + 1], ro) <= 1e-2
+        assert rel_l2(fin[seq:seq + 1, h:h + 1], rf) <= 1e-2
+        if interval > 0 and rc.shape[0]:
+            base = ckpt_base(d["lengths"], seq, interval)
+            assert rel_l2(ck[base:base + rc.shape[0], h:h + 1], rc) <= 1e-2
+
+
+def test_long_context_segments():
+    """T = 1,048,576 with snapshots every 32,768 tokens.  The oracle replays sampled
+    32K-token segments of sampled heads from the GPU's own snapshot before each one
+    (a property that holds at any length), plus the first segment from zero."""
+    w = kin.WORKLOADS["long"]
+    d = kin.make_workload("long", device="cuda")
+    cu_dev = torch.tensor(d["cu_seqlens"], dtype=torch.int32, device="cuda")
+    I = w["ckpt_interval"]
+    out, fin, ck = kda.kda_prefill(d["q"], d["k"], d["v"], d["g"], d["beta"], cu_dev,
+                                   init_state=None, chunk=w["chunk"], ckpt_interval=I,
+                                   cu_seqlens_host=d["cu_seqlens"])
+    torch.cuda.synchronize()
+    T = d["cu_seqlens"][-1]
+    assert ck.shape[0] == T // I == 32
+    assert torch.equal(ck[-1], fin[0])
+    import oracle
+    for seg, h in [(0, 0), (17, 5), (31, 31)]:
+        a, b = seg * I, (seg + 1) * I
+        cpu = lambda t: t[a:b, h:h + 1].to("cpu")
+        init = None if seg == 0 else ck[seg - 1:seg, h:h + 1].to("cpu")
+        ro, rf, _ = oracle.prefill(cpu(d["q"]), cpu(d["k"]), cpu(d["v"]), cpu(d["g"]),
+                                   cpu(d["beta"]), [0, I], init, 0, 0, 1)
+        assert rel_l2(out[a:b, h:h + 1], ro) <= 1e-2
+        assert rel_l2(ck[seg:seg + 1, h:h + 1], rf) <= 1e-2
+
+
+def test_bounded_wait_reports_timeout():
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    kda.kda_selftest_bounded_wait(status, 0)
+    torch.cuda.synchronize()
+    assert int(status[0]) == kda.KDA_ERR_TIMEOUT
+    status.zero_()
+    kda.kda_selftest_bounded_wait(status, 1000)
+    torch.cuda.synchronize()
+    assert int(status[0]) == kda.KDA_ERR_TIMEOUT
+    # the context is still usable afterwards
+    x = torch.ones(8, device="cuda")
+    assert float(x.sum()) == 8.0
