@@ -1,11 +1,630 @@
-// KDA chunked prefill on the tcgen05 tensor cores (placeholder until the kernel lands).
+// KDA chunked prefill on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// Covers BF16 q/k/v/out with D_k = D_v = 128 and 64-token chunks; the FP32
+// state never leaves the chip between chunks.  The method: prefill groups the
+// tokens into chunks, unrolls the recurrence inside a chunk into dense matrix
+// products and carries the state between chunks ("Kimi K3 architecture"
+// summary, Methods 1, FlashKDA; Kimi-K3 deep dive section 4-1, chunk-parallel
+// tiles with a recurrence between them).
+//
+// One CTA owns one (sequence, head, slice of DVS value columns) and walks its
+// sequence chunk by chunk.  For a chunk of 64 tokens starting from S0, with
+// Gam_r = sum_{s<=r} g_s (inclusive, per channel):
+//
+//   M_ri = beta_r sum_c k_rc k_ic exp(Gam_rc - Gam_ic)   (i < r)  gated Gram of k
+//   P_ri = sum_c q_rc k_ic exp(Gam_rc - Gam_ic)          (i <= r) gated q.k^T
+//   T    = (I + M)^-1 diag(beta)                          UT transform
+//   What = T Ktilde, Utilde = T V      (Ktilde_r = k_r exp(Gam_r))   WY form
+//   U    = Utilde - What S0                               delta-rule corrections
+//   O    = Qtilde S0 + P U             (Qtilde_r = q_r exp(Gam_r))
+//   S    = Diag(exp(Gam_63)) S0 + Khat^T U   (Khat_r = k_r exp(Gam_63 - Gam_r))
+//
+// Gate numerics: exp(Gam_r - Gam_i) is split into a factor on each operand
+// so that both stay inside the FP32/BF16 exponent range.  With g >= -5 a
+// factor exp(+-(Gam - ref)) is at most e^80 when the reference sits in the
+// middle of a 32-token half.  The Gram products are therefore formed on three
+// 32x32 block pairs of the 64x64 matrices: the two diagonal pairs use the
+// middle of their half as reference, the off-diagonal pair uses the boundary
+// between the halves (both factors <= 1; an underflow there only loses
+// products below e^-87).
+//
+// Tensor-core work per chunk (BF16 operands in 128-byte-swizzled shared
+// tiles, FP32 accumulators in tensor memory):
+//   Gram:   3 x [64 x 32 x 128]    (rows: k-part and q-part of a half)
+//   T-prod: [T;P] (128x64) x [Ktilde | V]           -> What, Utilde
+//   MMA1:   [What; Qtilde] (128x128) x S0_bf16      -> What S0, Qtilde S0
+//   MMA2:   [T;P] x U accumulated onto MMA1 (rows 64..127 become O),
+//           Khat^T (128x64) x U                     -> state increment
+// The triangular solve, the gates and the FP32 state update run on the SIMT
+// pipes.  The FP32 state of the CTA's slice stays in registers: row c of the
+// state belongs to TMEM lane c.
 #include "kda_common.cuh"
+#include "kda_tc_util.cuh"
 
 namespace kda {
-bool prefill_tc_supported(int, int, int, int) { return false; }
-cudaError_t launch_prefill_tc(const void *, const void *, const void *, const float *,
-                              const float *, const float *, const int32_t *, void *, float *,
-                              int64_t, float *, int, int, int64_t, int32_t *, cudaStream_t) {
-  return cudaErrorNotSupported;
+namespace {
+
+constexpr int kC = 64;      // chunk length
+constexpr int kDK = 128;    // key head size
+constexpr int kDV = 128;    // value head size (full)
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr int kLd = 65;     // row stride of the FP32 64x64 scratch matrices
+
+template <int DVS>
+struct Layout {
+  static constexpr uint32_t S_T = 0;                              // [128][DVS]  state, MN-major B
+  static constexpr uint32_t WQ_T = S_T + 128 * DVS * 2;           // [128][128]  What;Qtilde, K-major A
+  static constexpr uint32_t TP_T = WQ_T + 32768;                  // [128][64]   T;P, K-major A
+  static constexpr uint32_t KH_T = TP_T + 16384;                  // [64][128]   Khat, MN-major A
+  static constexpr uint32_t KV_T = KH_T + 16384;                  // [64][128+DVS] Ktilde|V, MN-major B
+  static constexpr uint32_t G = KV_T + 64 * (128 + DVS) * 2;      // 72 KB region
+  static constexpr uint32_t A00 = G, A11 = G + 16384, A10 = G + 32768;   // [64][128] K-major
+  static constexpr uint32_t B00 = G + 49152, B11 = G + 57344, B10 = G + 65536;  // [32][128]
+  static constexpr uint32_t MM = G;                                // float [64][65] (after Gram)
+  static constexpr uint32_t PM = G + 16640;
+  static constexpr uint32_t XM = G + 33280;
+  static constexpr uint32_t YS = G + 49920;                        // float [3][16][17]
+  static constexpr uint32_t U_T = G + 57344;                       // [64][DVS] U, MN-major B
+  static constexpr uint32_t SMALL = G + 73728;
+  static constexpr uint32_t BETA = SMALL;                          // float [64]
+  static constexpr uint32_t DVEC = SMALL + 256;                    // float [128]
+  static constexpr uint32_t RED = SMALL + 768;                     // float [16][128]
+  static constexpr uint32_t GREF = RED + 8192;                     // float [4][128]
+  static constexpr uint32_t BAR = GREF + 2048;                     // mbarrier
+  static constexpr uint32_t TMEM_SLOT = BAR + 8;
+  static constexpr uint32_t TOTAL = BAR + 64;
+  static_assert(YS + 3 * 16 * 17 * 4 <= U_T, "scratch overlaps U");
+  static_assert(U_T + 64 * DVS * 2 <= SMALL, "U overflows its region");
+};
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
 }
+
+// Wait for an mbarrier phase for at most limit_ns nanoseconds.
+__device__ __forceinline__ bool wait_timed(uint64_t *bar, uint32_t phase, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, phase)) return true;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, phase))
+    if (globaltimer() - t0 > limit_ns) return false;
+  return true;
+}
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float *x) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __bfloat1622float2(h[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+}
+
+template <int DVS>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                  const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
+                  const float *__restrict__ beta, const float *__restrict__ init,
+                  const int32_t *__restrict__ cu, __nv_bfloat16 *__restrict__ out,
+                  float *__restrict__ fin, int64_t interval, float *__restrict__ ck, int H,
+                  int32_t *dev_status, uint64_t wait_ns) {
+  using Lay = Layout<DVS>;
+  constexpr int NCOL = DVS / 2;           // state columns per thread
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sb = (sraw + 1023u) & ~1023u;
+  uint8_t *sp = smem_raw + (sb - sraw);
+  float *s_beta = reinterpret_cast<float *>(sp + Lay::BETA);
+  float *s_dvec = reinterpret_cast<float *>(sp + Lay::DVEC);
+  float *s_red = reinterpret_cast<float *>(sp + Lay::RED);
+  float *s_gref = reinterpret_cast<float *>(sp + Lay::GREF);
+  float *s_M = reinterpret_cast<float *>(sp + Lay::MM);
+  float *s_P = reinterpret_cast<float *>(sp + Lay::PM);
+  float *s_X = reinterpret_cast<float *>(sp + Lay::XM);
+  float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sp + Lay::BAR);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hw = warp >> 2;      // TMEM lane quadrant, column half
+  const int unit = blockIdx.x, seq = unit / H, h = unit % H;
+  const int col0 = blockIdx.y * DVS;            // first value column of the slice
+  const int crow = 32 * qd + lane;              // state row (key channel) owned
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
+  const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);   // this warp's lane base
+
+  // FP32 state slice in registers: row crow, columns [hw*NCOL, hw*NCOL + NCOL).
+  float S[NCOL];
+  const size_t soff = ((size_t)unit * kDK + crow) * kDV + col0 + hw * NCOL;
+#pragma unroll
+  for (int j = 0; j < NCOL; j += 4) {
+    float4 x = init ? *reinterpret_cast<const float4 *>(init + soff + j) : make_float4(0, 0, 0, 0);
+    S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
+  }
+#pragma unroll
+  for (int j = 0; j < NCOL; j += 8)
+    tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + j) >> 3), S + j);
+
+  const int64_t t_begin = cu[seq], t_end = cu[seq + 1];
+  int64_t ck_slot = 0;
+  if (interval > 0)
+    for (int j = 0; j < seq; ++j) ck_slot += (int64_t)(cu[j + 1] - cu[j]) / interval;
+  uint32_t phase = 0;
+  bool aborted = false;
+
+  for (int64_t t0 = t_begin; t0 < t_end; t0 += kC) {
+    const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
+
+    // ---------------- gate prep: cumulative decay and scaled operands ----------------
+    {
+      const int rg = tid >> 4, jc = tid & 15;   // rows 4rg..4rg+3, channels 8jc..8jc+7
+      float gm[4][8], kk[4][8], qq[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * rg + i;
+        if (r < L) {
+          const size_t off = ((size_t)(t0 + r) * H + h) * kDK + 8 * jc;
+          unpack8(__ldcs(reinterpret_cast<const uint4 *>(q + off)), qq[i]);
+          unpack8(__ldcs(reinterpret_cast<const uint4 *>(k + off)), kk[i]);
+          const float4 a = __ldcs(reinterpret_cast<const float4 *>(g + off));
+          const float4 b = __ldcs(reinterpret_cast<const float4 *>(g + off + 4));
+          gm[i][0] = a.x; gm[i][1] = a.y; gm[i][2] = a.z; gm[i][3] = a.w;
+          gm[i][4] = b.x; gm[i][5] = b.y; gm[i][6] = b.z; gm[i][7] = b.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) gm[i][e] = kk[i][e] = qq[i][e] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int i = 1; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gm[i][e] += gm[i - 1][e];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_red[rg * 128 + 8 * jc + e] = gm[3][e];
+      if (tid < kC) s_beta[tid] = tid < L ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
+      // V slice into the right part of the [Ktilde | V] tile (columns 128..).
+      for (int e = tid; e < kC * DVS / 8; e += kThreads) {
+        const int r = e / (DVS / 8), cj = e % (DVS / 8);
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (r < L)
+          val = __ldcs(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + r) * H + h) * kDV + col0 + 8 * cj));
+        tc::st_shared_v4(sb + Lay::KV_T + tc::tile_offset(64, r, 16 + cj), val.x, val.y, val.z, val.w);
+      }
+      __syncthreads();
+      float base[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) base[e] = 0.f;
+      for (int p = 0; p < rg; ++p)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) base[e] += s_red[p * 128 + 8 * jc + e];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gm[i][e] += base[e];
+      if ((rg & 3) == 3)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s_gref[(rg >> 2) * 128 + 8 * jc + e] = gm[3][e];
+      __syncthreads();
+      float G15[8], G31[8], G47[8], G63[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        G15[e] = s_gref[0 * 128 + 8 * jc + e];
+        G31[e] = s_gref[1 * 128 + 8 * jc + e];
+        G47[e] = s_gref[2 * 128 + 8 * jc + e];
+        G63[e] = s_gref[3 * 128 + 8 * jc + e];
+      }
+      if (rg == 0)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s_dvec[8 * jc + e] = __expf(G63[e]);
+
+      if (rg < 8) {   // first half: reference Gam_15 for the diagonal pair
+        float c1[8], e15[8], c12[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c1[e] = __expf(G31[e] - G15[e]);            // in [e^-80, 1]
+          e15[e] = __expf(G15[e]);                    // in [e^-80, 1]
+          c12[e] = c1[e] * __expf(G63[e] - G31[e]);   // may underflow: harmless
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 4 * rg + i;
+          float x[8], y[8], t[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            x[e] = __expf(gm[i][e] - G15[e]);
+            y[e] = __expf(G15[e] - gm[i][e]);
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * x[e];
+          tc::st_chunk(sb + Lay::A00 + tc::tile_offset(64, r, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * x[e];
+          tc::st_chunk(sb + Lay::A00 + tc::tile_offset(64, 32 + r, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * y[e];
+          tc::st_chunk(sb + Lay::B00 + tc::tile_offset(32, r, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (y[e] * c1[e]);
+          tc::st_chunk(sb + Lay::B10 + tc::tile_offset(32, r, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (x[e] * e15[e]);
+          tc::st_chunk(sb + Lay::KV_T + tc::tile_offset(64, r, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * (x[e] * e15[e]);
+          tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, 64 + r, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (y[e] * c12[e]);
+          tc::st_chunk(sb + Lay::KH_T + tc::tile_offset(64, r, jc), t);
+        }
+      } else {        // second half: reference Gam_47 (diagonal), Gam_31 (off-diagonal)
+        float c3[8], e31[8], c4[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          c3[e] = __expf(G47[e] - G31[e]);            // in [e^-80, 1]
+          e31[e] = __expf(G31[e]);                    // may underflow: harmless
+          c4[e] = __expf(G63[e] - G47[e]);            // in [e^-80, 1]
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = 4 * rg + i, rl = r - 32;
+          float x[8], y[8], xo[8], t[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            x[e] = __expf(gm[i][e] - G47[e]);
+            y[e] = __expf(G47[e] - gm[i][e]);
+            xo[e] = x[e] * c3[e];                     // exp(Gam_r - Gam_31) <= 1
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * x[e];
+          tc::st_chunk(sb + Lay::A11 + tc::tile_offset(64, rl, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * x[e];
+          tc::st_chunk(sb + Lay::A11 + tc::tile_offset(64, 32 + rl, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * y[e];
+          tc::st_chunk(sb + Lay::B11 + tc::tile_offset(32, rl, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * xo[e];
+          tc::st_chunk(sb + Lay::A10 + tc::tile_offset(64, rl, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * xo[e];
+          tc::st_chunk(sb + Lay::A10 + tc::tile_offset(64, 32 + rl, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (xo[e] * e31[e]);
+          tc::st_chunk(sb + Lay::KV_T + tc::tile_offset(64, r, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * (xo[e] * e31[e]);
+          tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, 64 + r, jc), t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (y[e] * c4[e]);
+          tc::st_chunk(sb + Lay::KH_T + tc::tile_offset(64, r, jc), t);
+        }
+      }
+      tc::fence_smem_to_async();
+      __syncthreads();
+    }
+
+    // ---------------- gated Gram products on the tensor cores ----------------
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(64, 32, 0, 0);
+      const uint32_t A[3] = {sb + Lay::A00, sb + Lay::A11, sb + Lay::A10};
+      const uint32_t B[3] = {sb + Lay::B00, sb + Lay::B11, sb + Lay::B10};
+#pragma unroll
+      for (int p = 0; p < 3; ++p)
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          tc::mma_bf16(tmem + 32 * p, tc::desc_kmajor(A[p], 64, s), tc::desc_kmajor(B[p], 32, s),
+                       id, s > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
+    phase ^= 1;
+    tc::fence_after_sync();
+
+    // Read the three 64x32 blocks (M=64 layout: row m in lane (m%16) + 32*(m/16)).
+    if (warp < 4) {
+      float a[32];
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        tc::tmem_ld32(tl + 32 * p, a);
+        tc::tmem_wait_ld();
+        if (lane < 16) {
+          const int m = 16 * warp + lane, part = m >> 5, rl = m & 31;
+          const int r = p == 0 ? rl : 32 + rl;
+          const int cbase = p == 1 ? 32 : 0;
+          float *dst = (part == 0 ? s_M : s_P) + r * kLd + cbase;
+          const float br = part == 0 ? s_beta[r] : 1.f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const bool valid = p == 2 || (part == 0 ? j < rl : j <= rl);
+            dst[j] = valid ? br * a[j] : 0.f;
+          }
+          if (p == 0) {
+            float *z = (part == 0 ? s_M : s_P) + r * kLd + 32;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) z[j] = 0.f;
+          }
+        }
+      }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+
+    // ---------------- UT transform: X = (I + M)^-1, blockwise on 16x16 blocks ----------------
+    if (tid < 64) {
+      const int b = tid >> 4, ci = tid & 15, o = 16 * b;
+      float x[16];
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) {
+        float acc = 0.f;
+#pragma unroll
+        for (int s = 0; s < rr; ++s) acc += s_M[(o + rr) * kLd + o + s] * x[s];
+        x[rr] = rr < ci ? 0.f : (rr == ci ? 1.f : -acc);
+      }
+#pragma unroll
+      for (int rr = 0; rr < 16; ++rr) s_X[(o + rr) * kLd + o + ci] = x[rr];
+    }
+    __syncthreads();
+    // distance 1: (1,0), (2,1), (3,2)
+    for (int e = tid; e < 768; e += kThreads) {
+      const int pi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, b = pi + 1, a = pi;
+      float acc = 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; ++s) acc += s_M[(16 * b + rr) * kLd + 16 * a + s] * s_X[(16 * a + s) * kLd + 16 * a + cc];
+      s_Y[(pi * 16 + rr) * 17 + cc] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < 768; e += kThreads) {
+      const int pi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, b = pi + 1, a = pi;
+      float acc = 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; ++s) acc += s_X[(16 * b + rr) * kLd + 16 * b + s] * s_Y[(pi * 16 + s) * 17 + cc];
+      s_X[(16 * b + rr) * kLd + 16 * a + cc] = -acc;
+    }
+    __syncthreads();
+    // distance 2: (2,0), (3,1)
+    for (int e = tid; e < 512; e += kThreads) {
+      const int pi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, b = pi + 2, a = pi;
+      float acc = 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; ++s)
+        acc += s_M[(16 * b + rr) * kLd + 16 * a + s] * s_X[(16 * a + s) * kLd + 16 * a + cc] +
+               s_M[(16 * b + rr) * kLd + 16 * (a + 1) + s] * s_X[(16 * (a + 1) + s) * kLd + 16 * a + cc];
+      s_Y[(pi * 16 + rr) * 17 + cc] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < 512; e += kThreads) {
+      const int pi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, b = pi + 2, a = pi;
+      float acc = 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; ++s) acc += s_X[(16 * b + rr) * kLd + 16 * b + s] * s_Y[(pi * 16 + s) * 17 + cc];
+      s_X[(16 * b + rr) * kLd + 16 * a + cc] = -acc;
+    }
+    __syncthreads();
+    // distance 3: (3,0)
+    {
+      const int rr = tid >> 4, cc = tid & 15;
+      float acc = 0.f;
+#pragma unroll
+      for (int c3 = 0; c3 < 3; ++c3)
+#pragma unroll
+        for (int s = 0; s < 16; ++s)
+          acc += s_M[(48 + rr) * kLd + 16 * c3 + s] * s_X[(16 * c3 + s) * kLd + cc];
+      s_Y[rr * 17 + cc] = acc;
+    }
+    __syncthreads();
+    {
+      const int rr = tid >> 4, cc = tid & 15;
+      float acc = 0.f;
+#pragma unroll
+      for (int s = 0; s < 16; ++s) acc += s_X[(48 + rr) * kLd + 48 + s] * s_Y[s * 17 + cc];
+      s_X[(48 + rr) * kLd + cc] = -acc;
+    }
+    __syncthreads();
+    // [T; P] operand: T_ri = X_ri beta_i (i <= r), P as read.
+    for (int e = tid; e < 128 * 8; e += kThreads) {
+      const int row = e >> 3, ch = e & 7;
+      float val[8];
+      if (row < 64) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = 8 * ch + u;
+          val[u] = i <= row ? s_X[row * kLd + i] * s_beta[i] : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) val[u] = s_P[(row - 64) * kLd + 8 * ch + u];
+      }
+      tc::st_chunk(sb + Lay::TP_T + tc::tile_offset(128, row, ch), val);
+    }
+    tc::fence_smem_to_async();
+    __syncthreads();
+
+    // ---------------- WY products: [T;P] x [Ktilde | V] ----------------
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 128 + DVS, 0, 1);
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::TP_T, 128, s),
+                     tc::desc_mnmajor(sb + Lay::KV_T, 64, s), id, s > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
+    phase ^= 1;
+    tc::fence_after_sync();
+    if (qd < 2) {   // What rows 0..63 -> bf16 operand rows 0..63 of [What; Qtilde]
+      const int r = 32 * qd + lane;
+      float a[32];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        tc::tmem_ld32(tl + 64 * hw + 32 * u, a);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, r, 8 * hw + 4 * u + cc), a + 8 * cc);
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+
+    // ---------------- MMA1: [What; Qtilde] x S0 ----------------
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, DVS, 0, 1);
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::WQ_T, 128, s),
+                     tc::desc_mnmajor(sb + Lay::S_T, 128, s), id, s > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
+    phase ^= 1;
+    tc::fence_after_sync();
+    if (qd < 2) {   // U = Utilde - What S0 -> bf16 operand
+      const int r = 32 * qd + lane;
+      float a[32], b[32];
+#pragma unroll
+      for (int u = 0; u < NCOL / 32; ++u) {
+        const int col = hw * NCOL + 32 * u;
+        tc::tmem_ld32(tl + 256 + col, a);
+        tc::tmem_ld32(tl + 128 + col, b);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) b[i] -= a[i];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          tc::st_chunk(sb + Lay::U_T + tc::tile_offset(64, r, (col >> 3) + cc), b + 8 * cc);
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+
+    // ---------------- MMA2: O += P U, dS = Khat^T U ----------------
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t ida = tc::idesc_bf16(128, DVS, 0, 1);
+      constexpr uint32_t idb = tc::idesc_bf16(128, DVS, 1, 1);
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::TP_T, 128, s),
+                     tc::desc_mnmajor(sb + Lay::U_T, 64, s), ida, 1);
+#pragma unroll
+      for (int s = 0; s < 4; ++s)
+        tc::mma_bf16(tmem + 256 + DVS, tc::desc_mnmajor(sb + Lay::KH_T, 64, s),
+                     tc::desc_mnmajor(sb + Lay::U_T, 64, s), idb, s > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
+    phase ^= 1;
+    tc::fence_after_sync();
+    {
+      float a[32];
+      if (qd >= 2) {   // rows 64..127 hold O for tokens 0..63
+        const int r = 32 * (qd - 2) + lane;
+#pragma unroll
+        for (int u = 0; u < NCOL / 32; ++u) {
+          const int col = hw * NCOL + 32 * u;
+          tc::tmem_ld32(tl + 256 + col, a);
+          tc::tmem_wait_ld();
+          if (r < L) {
+            uint4 *dst = reinterpret_cast<uint4 *>(out + ((size_t)(t0 + r) * H + h) * kDV + col0 + col);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              dst[cc] = make_uint4(tc::pack_bf16(a[8 * cc], a[8 * cc + 1]),
+                                   tc::pack_bf16(a[8 * cc + 2], a[8 * cc + 3]),
+                                   tc::pack_bf16(a[8 * cc + 4], a[8 * cc + 5]),
+                                   tc::pack_bf16(a[8 * cc + 6], a[8 * cc + 7]));
+          }
+        }
+      }
+      const float d = s_dvec[crow];
+#pragma unroll
+      for (int u = 0; u < NCOL / 32; ++u) {
+        tc::tmem_ld32(tl + 256 + DVS + hw * NCOL + 32 * u, a);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) S[32 * u + i] = fmaf(d, S[32 * u + i], a[i]);
+      }
+#pragma unroll
+      for (int j = 0; j < NCOL; j += 8)
+        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + j) >> 3), S + j);
+      if (interval > 0 && L == kC && (t0 + kC - t_begin) % interval == 0) {
+        float *dst = ck + ((size_t)ck_slot * H + h) * kDK * kDV + (size_t)crow * kDV + col0 + hw * NCOL;
+#pragma unroll
+        for (int j = 0; j < NCOL; j += 4)
+          *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+        ++ck_slot;
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+  }
+
+  if (aborted) {
+    report(dev_status, KDA_ERR_TIMEOUT);
+    // Give the tensor core a last bounded chance to finish what it was given.
+    wait_timed(bar, phase, wait_ns);
+  } else if (fin) {
+    float *dst = fin + soff;
+#pragma unroll
+    for (int j = 0; j < NCOL; j += 4)
+      *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int DVS>
+cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *init, const int32_t *cu, void *out,
+                        float *fin, int64_t interval, float *ck, int N, int H,
+                        int32_t *dev_status, cudaStream_t stream) {
+  const size_t smem = Layout<DVS>::TOTAL + 1024;
+  auto kern = prefill_tc_kernel<DVS>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  dim3 grid((unsigned)((int64_t)N * H), (unsigned)(kDV / DVS));
+  kern<<<grid, kThreads, smem, stream>>>(
+      (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g, beta, init,
+      cu, (__nv_bfloat16 *)out, fin, interval, ck, H, dev_status, 2000000000ull);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool prefill_tc_supported(int dtype, int dk, int dv, int chunk) {
+  return dtype == KDA_DTYPE_BF16 && dk == kDK && dv == kDV && chunk == kC;
+}
+
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const float *init, const int32_t *cu, void *out,
+                              float *fin, int64_t interval, float *ck, int N, int H,
+                              int64_t total_tokens, int32_t *dev_status, cudaStream_t stream) {
+  (void)total_tokens;
+  // Few (sequence, head) units: split the value columns in two to fill the SMs.
+  if ((int64_t)N * H * 2 <= 148)
+    return launch_tc_t<64>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N, H, dev_status, stream);
+  return launch_tc_t<128>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N, H, dev_status, stream);
+}
+
 }  // namespace kda
