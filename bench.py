@@ -77,25 +77,32 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def kernel_source_sha() -> str:
+KERNEL_SOURCES = {
+    "decode": ("kda_decode.cu", "kda_common.cuh"),
+    "prefill_tc": ("kda_prefill_tc.cu", "kda_tc_util.cuh", "kda_common.cuh"),
+    "prefill_simt": ("kda_prefill_simt.cu", "kda_common.cuh"),
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
+    """Hash of the source files a kernel is built from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_attention_08_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as fh:
-                h.update(name.encode() + fh.read())
+    for name in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(csrc, name), "rb") as fh:
+            h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
 
 
 def ncu_traffic(kernel: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    the current sources of that kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as fh:
         rec = json.load(fh).get(kernel)
-    if not rec or rec.get("source_sha") != kernel_source_sha():
+    if not rec or rec.get("source_sha") != kernel_source_sha(kernel):
         return None
     return rec.get("bytes_per_launch")
 
@@ -279,10 +286,14 @@ def time_prefill(name, steps, warmup, world, local):
                 kernel="prefill_tc" if path == 1 else "prefill_simt", w=w, lengths=lengths)
 
 
-def time_decode(steps_graph, warmup, world, local):
+def time_decode(steps_graph, warmup, world, local, decode_steps=None):
     from linear_attention_08_b200 import kda
-    w = kin.WORKLOADS["decode"]
-    d = kin.make_workload("decode", device="cuda", seed=local)
+    w = dict(kin.WORKLOADS["decode"])
+    if decode_steps:
+        w["steps"] = decode_steps
+    d = kin.make_inputs((w["steps"], w["num_seqs"]), w["H"], w["Dk"], w["Dv"],
+                        kin.torch_dtype(w["dtype"]), local, num_states=w["num_seqs"],
+                        state_std=w["state_std"], device="cuda")
     S, N, H, Dk, Dv = w["steps"], w["num_seqs"], w["H"], w["Dk"], w["Dv"]
     state = d["init_state"].clone()
     outs = torch.empty_like(d["v"])
@@ -348,7 +359,7 @@ def run_ours(args, rank, world, local):
     dec = None
     if name == "decode" or not args.no_decode:
         dec = time_decode(max(1, args.steps // 2) if name != "decode" else args.steps,
-                          args.warmup, world, local)
+                          args.warmup, world, local, args.decode_steps)
     if rank != 0:
         return None
     if res is not None:
@@ -482,6 +493,8 @@ def main():
     ap.add_argument("--workload", default="prefill",
                     choices=["prefill", "decode", "append_varlen", "long"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=0,
+                    help="decode steps per graph (default: the workload's 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
