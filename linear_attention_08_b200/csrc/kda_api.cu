@@ -131,7 +131,7 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
     return KDA_ERR_INVALID_ARGUMENT;  // exact aliasing is fine, partial overlap is not
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (prefill_tc_supported(s->qkv_dtype, DK, DV, s->chunk))
+  if (T > 0 && prefill_tc_supported(s->qkv_dtype, DK, DV, s->chunk))
     e = launch_prefill_tc(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
                           ckpt_interval, ckpt_states, N, H, T, s->dev_status, cs);
   else

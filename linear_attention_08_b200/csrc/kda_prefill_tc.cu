@@ -38,6 +38,8 @@
 // The triangular solve, the gates and the FP32 state update run on the SIMT
 // pipes.  The FP32 state of the CTA's slice stays in registers: row c of the
 // state belongs to TMEM lane c.
+#include <cuda.h>
+
 #include "kda_common.cuh"
 #include "kda_tc_util.cuh"
 
@@ -58,24 +60,27 @@ struct Layout {
   static constexpr uint32_t TP_T = WQ_T + 32768;                  // [128][64]   T;P, K-major A
   static constexpr uint32_t KH_T = TP_T + 16384;                  // [64][128]   Khat, MN-major A
   static constexpr uint32_t KV_T = KH_T + 16384;                  // [64][128+DVS] Ktilde|V, MN-major B
-  static constexpr uint32_t G = KV_T + 64 * (128 + DVS) * 2;      // 72 KB region
-  static constexpr uint32_t A00 = G, A11 = G + 16384, A10 = G + 32768;   // [64][128] K-major
-  static constexpr uint32_t B00 = G + 49152, B11 = G + 57344, B10 = G + 65536;  // [32][128]
-  static constexpr uint32_t MM = G;                                // float [64][65] (after Gram)
-  static constexpr uint32_t PM = G + 16640;
-  static constexpr uint32_t XM = G + 33280;
-  static constexpr uint32_t YS = G + 49920;                        // float [3][16][17]
-  static constexpr uint32_t U_T = G + 57344;                       // [64][DVS] U, MN-major B
+  static constexpr uint32_t U_T = KV_T;                           // [64][DVS] U, MN-major B, reuses
+                                                                  //   the Ktilde slot after the WY product
+  static constexpr uint32_t G = KV_T + 64 * (128 + DVS) * 2;      // 72 KB region, used in turn for:
+  static constexpr uint32_t STG_Q = G, STG_K = G + 16384;         //  next chunk's q, k [64][128] bf16
+  static constexpr uint32_t STG_G = G + 32768;                    //  next chunk's g [64][128] fp32
+  static constexpr uint32_t RED = G + 65536;                      //  float [16][128] scan partials
+  static constexpr uint32_t A00 = G, A11 = G + 16384, A10 = G + 32768;          // Gram A [64][128]
+  static constexpr uint32_t B00 = G + 49152, B11 = G + 57344, B10 = G + 65536;  // Gram B [32][128]
+  static constexpr uint32_t MM = G;                               //  float [64][65] M
+  static constexpr uint32_t XM = G + 16640;                       //  float [64][65] (I + M)^-1
+  static constexpr uint32_t YS = G + 33280;                       //  float [3][16][17]
   static constexpr uint32_t SMALL = G + 73728;
-  static constexpr uint32_t BETA = SMALL;                          // float [64]
-  static constexpr uint32_t DVEC = SMALL + 256;                    // float [128]
-  static constexpr uint32_t RED = SMALL + 768;                     // float [16][128]
-  static constexpr uint32_t GREF = RED + 8192;                     // float [4][128]
-  static constexpr uint32_t BAR = GREF + 2048;                     // mbarrier
-  static constexpr uint32_t TMEM_SLOT = BAR + 8;
+  static constexpr uint32_t BETA = SMALL;                         // float [64]
+  static constexpr uint32_t DVEC = SMALL + 256;                   // float [128]
+  static constexpr uint32_t GREF = SMALL + 768;                   // float [4][128]
+  static constexpr uint32_t BAR = GREF + 2048;                    // mbarrier: MMA completion
+  static constexpr uint32_t TBAR = BAR + 8;                       // mbarrier: TMA loads landed
+  static constexpr uint32_t TMEM_SLOT = BAR + 16;
   static constexpr uint32_t TOTAL = BAR + 64;
-  static_assert(YS + 3 * 16 * 17 * 4 <= U_T, "scratch overlaps U");
-  static_assert(U_T + 64 * DVS * 2 <= SMALL, "U overflows its region");
+  static_assert(YS + 3 * 16 * 17 * 4 <= G + 73728, "solve scratch overflows");
+  static_assert(64 * DVS * 2 <= 16384, "U must fit the Ktilde slot");
 };
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -93,6 +98,66 @@ __device__ __forceinline__ bool wait_timed(uint64_t *bar, uint32_t phase, uint64
   return true;
 }
 
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, bool valid) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+               "r"(valid ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Tensor maps of the inputs (3-D views [T_tot][H][D] of the token-major
+// tensors; box = 64 tokens of one head):
+//   q, k : bf16, box (128, 1, 64), no swizzle   -> staging rows of 256 bytes
+//   g    : fp32, box (128, 1, 64), no swizzle   -> staging rows of 512 bytes
+//   v    : bf16, box (64, 1, 64), 128-byte swizzle -> one column block of the
+//          [Ktilde | V] operand tile, already in the MMA layout.
+// Tokens past T_tot read as zeros; tokens of the next sequence are masked by
+// the consumer (q, k, g) or cancel exactly (v: beta is 0 there).
+struct TmaMaps {
+  CUtensorMap q, k, g, v;
+};
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+// Start loading the raw inputs of the chunk [t0, t0 + L): q, k, g into the
+// staging area and v into its operand slot (one elected thread, TMA); beta
+// into s_beta (64 threads, 4-byte async copies, zero past L).
+template <int DVS>
+__device__ __forceinline__ void prefetch_chunk(uint32_t sb, const TmaMaps &maps, const float *beta,
+                                               int64_t t0, int L, int H, int h, int col0,
+                                               int tid) {
+  using Lay = Layout<DVS>;
+  if (tid == 0) {
+    const uint32_t bar = sb + Lay::TBAR;
+    mbar_expect_tx(bar, 64 * (256 + 256 + 512) + 64 * DVS * 2);
+    const int z = (int)t0;
+    tma_load_3d(sb + Lay::STG_Q, &maps.q, 0, h, z, bar);
+    tma_load_3d(sb + Lay::STG_K, &maps.k, 0, h, z, bar);
+    tma_load_3d(sb + Lay::STG_G, &maps.g, 0, h, z, bar);
+#pragma unroll
+    for (int j = 0; j < DVS / 64; ++j)
+      tma_load_3d(sb + Lay::KV_T + (2 + j) * 8192, &maps.v, col0 + 64 * j, h, z, bar);
+  }
+  if (tid < kC) {
+    const bool ok = tid < L;
+    cp_async4(sb + Lay::BETA + 4 * tid, beta + (ok ? (size_t)(t0 + tid) * H + h : 0), ok);
+  }
+  cp_async_commit();
+}
+
 __device__ __forceinline__ void unpack8(const uint4 &u, float *x) {
   const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
 #pragma unroll
@@ -105,9 +170,7 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float *x) {
 
 template <int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
-prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                  const __nv_bfloat16 *__restrict__ v, const float *__restrict__ g,
-                  const float *__restrict__ beta, const float *__restrict__ init,
+prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ beta, const float *__restrict__ init,
                   const int32_t *__restrict__ cu, __nv_bfloat16 *__restrict__ out,
                   float *__restrict__ fin, int64_t interval, float *__restrict__ ck, int H,
                   int32_t *dev_status, uint64_t wait_ns) {
@@ -122,7 +185,6 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
   float *s_red = reinterpret_cast<float *>(sp + Lay::RED);
   float *s_gref = reinterpret_cast<float *>(sp + Lay::GREF);
   float *s_M = reinterpret_cast<float *>(sp + Lay::MM);
-  float *s_P = reinterpret_cast<float *>(sp + Lay::PM);
   float *s_X = reinterpret_cast<float *>(sp + Lay::XM);
   float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
   uint64_t *bar = reinterpret_cast<uint64_t *>(sp + Lay::BAR);
@@ -135,7 +197,10 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
 
   if (tid == 0) {
     mbar_init(bar, 1);
+    mbar_init(reinterpret_cast<uint64_t *>(sp + Lay::TBAR), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.g)) : "memory");
   }
   if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, kTmemCols);
   tc::fence_before_sync();
@@ -160,11 +225,18 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
   int64_t ck_slot = 0;
   if (interval > 0)
     for (int j = 0; j < seq; ++j) ck_slot += (int64_t)(cu[j + 1] - cu[j]) / interval;
-  uint32_t phase = 0;
+  uint32_t phase = 0, tphase = 0;
   bool aborted = false;
+  uint64_t *tbar = reinterpret_cast<uint64_t *>(sp + Lay::TBAR);
+  if (t_begin < t_end)
+    prefetch_chunk<DVS>(sb, maps, beta, t_begin,
+                        (int)((t_end - t_begin) < kC ? (t_end - t_begin) : kC), H, h, col0, tid);
 
   for (int64_t t0 = t_begin; t0 < t_end; t0 += kC) {
     const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
+    cp_async_wait_all();
+    if (__syncthreads_or(!wait_timed(tbar, tphase, wait_ns))) { aborted = true; break; }
+    tphase ^= 1;
 
     // ---------------- gate prep: cumulative decay and scaled operands ----------------
     {
@@ -173,18 +245,17 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = 4 * rg + i;
-        if (r < L) {
-          const size_t off = ((size_t)(t0 + r) * H + h) * kDK + 8 * jc;
-          unpack8(__ldcs(reinterpret_cast<const uint4 *>(q + off)), qq[i]);
-          unpack8(__ldcs(reinterpret_cast<const uint4 *>(k + off)), kk[i]);
-          const float4 a = __ldcs(reinterpret_cast<const float4 *>(g + off));
-          const float4 b = __ldcs(reinterpret_cast<const float4 *>(g + off + 4));
-          gm[i][0] = a.x; gm[i][1] = a.y; gm[i][2] = a.z; gm[i][3] = a.w;
-          gm[i][4] = b.x; gm[i][5] = b.y; gm[i][6] = b.z; gm[i][7] = b.w;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) gm[i][e] = kk[i][e] = qq[i][e] = 0.f;
-        }
+        const bool in = r < L;
+        const uint4 z4 = make_uint4(0, 0, 0, 0);
+        const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
+        const uint4 qv = in ? *reinterpret_cast<const uint4 *>(sp + Lay::STG_Q + r * 256 + jc * 16) : z4;
+        const uint4 kv = in ? *reinterpret_cast<const uint4 *>(sp + Lay::STG_K + r * 256 + jc * 16) : z4;
+        const float4 a = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + jc * 32) : zf;
+        const float4 b = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + jc * 32 + 16) : zf;
+        unpack8(qv, qq[i]);
+        unpack8(kv, kk[i]);
+        gm[i][0] = a.x; gm[i][1] = a.y; gm[i][2] = a.z; gm[i][3] = a.w;
+        gm[i][4] = b.x; gm[i][5] = b.y; gm[i][6] = b.z; gm[i][7] = b.w;
       }
 #pragma unroll
       for (int i = 1; i < 4; ++i)
@@ -192,15 +263,6 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         for (int e = 0; e < 8; ++e) gm[i][e] += gm[i - 1][e];
 #pragma unroll
       for (int e = 0; e < 8; ++e) s_red[rg * 128 + 8 * jc + e] = gm[3][e];
-      if (tid < kC) s_beta[tid] = tid < L ? beta[(size_t)(t0 + tid) * H + h] : 0.f;
-      // V slice into the right part of the [Ktilde | V] tile (columns 128..).
-      for (int e = tid; e < kC * DVS / 8; e += kThreads) {
-        const int r = e / (DVS / 8), cj = e % (DVS / 8);
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (r < L)
-          val = __ldcs(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + r) * H + h) * kDV + col0 + 8 * cj));
-        tc::st_shared_v4(sb + Lay::KV_T + tc::tile_offset(64, r, 16 + cj), val.x, val.y, val.z, val.w);
-      }
       __syncthreads();
       float base[8];
 #pragma unroll
@@ -333,28 +395,42 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     phase ^= 1;
     tc::fence_after_sync();
 
-    // Read the three 64x32 blocks (M=64 layout: row m in lane (m%16) + 32*(m/16)).
-    if (warp < 4) {
+    // Read the Gram blocks (M=64 layout: row m in lane (m%16) + 32*(m/16)).  Warps 0-3
+    // take pairs 00 and 11, warps 4-7 pair 10.  k-part rows become rows of the FP32
+    // matrix M (scaled by beta_r, strictly lower); q-part rows become rows of P,
+    // written straight into rows 64..127 of the bf16 [T; P] operand.
+    {
       float a[32];
 #pragma unroll
-      for (int p = 0; p < 3; ++p) {
+      for (int pp = 0; pp < 2; ++pp) {
+        const int p = hw == 0 ? pp : 2;
+        if (hw == 1 && pp == 1) break;
         tc::tmem_ld32(tl + 32 * p, a);
         tc::tmem_wait_ld();
         if (lane < 16) {
-          const int m = 16 * warp + lane, part = m >> 5, rl = m & 31;
+          const int m = 16 * qd + lane, part = m >> 5, rl = m & 31;
           const int r = p == 0 ? rl : 32 + rl;
           const int cbase = p == 1 ? 32 : 0;
-          float *dst = (part == 0 ? s_M : s_P) + r * kLd + cbase;
-          const float br = part == 0 ? s_beta[r] : 1.f;
+          if (part == 0) {
+            float *dst = s_M + r * kLd + cbase;
+            const float br = s_beta[r];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const bool valid = p == 2 || (part == 0 ? j < rl : j <= rl);
-            dst[j] = valid ? br * a[j] : 0.f;
-          }
-          if (p == 0) {
-            float *z = (part == 0 ? s_M : s_P) + r * kLd + 32;
+            for (int j = 0; j < 32; ++j) dst[j] = (p == 2 || j < rl) ? br * a[j] : 0.f;
+            if (p == 0)
 #pragma unroll
-            for (int j = 0; j < 32; ++j) z[j] = 0.f;
+              for (int j = 32; j < 64; ++j) s_M[r * kLd + j] = 0.f;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) a[j] = (p == 2 || j <= rl) ? a[j] : 0.f;
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+              tc::st_chunk(sb + Lay::TP_T + tc::tile_offset(128, 64 + r, (cbase >> 3) + cc), a + 8 * cc);
+            if (p == 0) {
+              float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int cc = 4; cc < 8; ++cc)
+                tc::st_chunk(sb + Lay::TP_T + tc::tile_offset(128, 64 + r, cc), z);
+            }
           }
         }
       }
@@ -363,18 +439,25 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     __syncthreads();
 
     // ---------------- UT transform: X = (I + M)^-1, blockwise on 16x16 blocks ----------------
-    if (tid < 64) {
-      const int b = tid >> 4, ci = tid & 15, o = 16 * b;
-      float x[16];
+    // Diagonal blocks: warp b inverts block b by a column sweep; lane = (column c,
+    // half hf) holds rows 8hf..8hf+7 of column c; row s is broadcast by shuffle.
+    if (warp < 4) {
+      const int o = 16 * warp, c = lane & 15, hf = lane >> 4;
+      float x[8];
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) {
-        float acc = 0.f;
+      for (int i = 0; i < 8; ++i) x[i] = (8 * hf + i == c) ? 1.f : 0.f;
+      const float *mrow = s_M + (o + 8 * hf) * kLd + o;
 #pragma unroll
-        for (int s = 0; s < rr; ++s) acc += s_M[(o + rr) * kLd + o + s] * x[s];
-        x[rr] = rr < ci ? 0.f : (rr == ci ? 1.f : -acc);
+      for (int sidx = 0; sidx < 15; ++sidx) {
+        float m[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = mrow[i * kLd + sidx];   // 0 on and above the diagonal
+        const float xs = __shfl_sync(0xffffffffu, x[sidx & 7], c + 16 * (sidx >> 3));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = fmaf(-m[i], xs, x[i]);
       }
 #pragma unroll
-      for (int rr = 0; rr < 16; ++rr) s_X[(o + rr) * kLd + o + ci] = x[rr];
+      for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * kLd + o + c] = x[i];
     }
     __syncthreads();
     // distance 1: (1,0), (2,1), (3,2)
@@ -433,19 +516,14 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
       s_X[(48 + rr) * kLd + cc] = -acc;
     }
     __syncthreads();
-    // [T; P] operand: T_ri = X_ri beta_i (i <= r), P as read.
-    for (int e = tid; e < 128 * 8; e += kThreads) {
+    // T rows of the [T; P] operand: T_ri = X_ri beta_i (i <= r).
+    for (int e = tid; e < 64 * 8; e += kThreads) {
       const int row = e >> 3, ch = e & 7;
       float val[8];
-      if (row < 64) {
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int i = 8 * ch + u;
-          val[u] = i <= row ? s_X[row * kLd + i] * s_beta[i] : 0.f;
-        }
-      } else {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) val[u] = s_P[(row - 64) * kLd + 8 * ch + u];
+      for (int u = 0; u < 8; ++u) {
+        const int i = 8 * ch + u;
+        val[u] = i <= row ? s_X[row * kLd + i] * s_beta[i] : 0.f;
       }
       tc::st_chunk(sb + Lay::TP_T + tc::tile_offset(128, row, ch), val);
     }
@@ -465,6 +543,9 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
     phase ^= 1;
     tc::fence_after_sync();
+    if (t0 + kC < t_end)
+      prefetch_chunk<DVS>(sb, maps, beta, t0 + kC,
+                          (int)((t_end - t0 - kC) < kC ? (t_end - t0 - kC) : kC), H, h, col0, tid);
     if (qd < 2) {   // What rows 0..63 -> bf16 operand rows 0..63 of [What; Qtilde]
       const int r = 32 * qd + lane;
       float a[32];
@@ -576,10 +657,13 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     __syncthreads();
   }
 
+  cp_async_wait_all();
   if (aborted) {
     report(dev_status, KDA_ERR_TIMEOUT);
-    // Give the tensor core a last bounded chance to finish what it was given.
+    // Give the tensor core and the copy engine a last bounded chance to finish
+    // what they were given before the CTA releases its memory.
     wait_timed(bar, phase, wait_ns);
+    wait_timed(tbar, tphase, wait_ns);
   } else if (fin) {
     float *dst = fin + soff;
 #pragma unroll
@@ -594,19 +678,55 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
   }
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3-D map over a token-major tensor [T][H][D]: dims (D, H, T), box (box_d, 1, 64).
+static bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes,
+                     int D, int H, int64_t T, int box_d, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * elem_bytes, (cuuint64_t)D * elem_bytes * H};
+  const cuuint32_t box[3] = {(cuuint32_t)box_d, 1, (cuuint32_t)kC};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int DVS>
 cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const float *g,
                         const float *beta, const float *init, const int32_t *cu, void *out,
-                        float *fin, int64_t interval, float *ck, int N, int H,
+                        float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
                         int32_t *dev_status, cudaStream_t stream) {
+  TmaMaps maps;
+  if (!make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, H, T, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, H, T, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&maps.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, H, T, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   const size_t smem = Layout<DVS>::TOTAL + 1024;
   auto kern = prefill_tc_kernel<DVS>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)((int64_t)N * H), (unsigned)(kDV / DVS));
-  kern<<<grid, kThreads, smem, stream>>>(
-      (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, g, beta, init,
-      cu, (__nv_bfloat16 *)out, fin, interval, ck, H, dev_status, 2000000000ull);
+  kern<<<grid, kThreads, smem, stream>>>(maps, beta, init, cu, (__nv_bfloat16 *)out, fin, interval,
+                                         ck, H, dev_status, 2000000000ull);
   return cudaGetLastError();
 }
 
@@ -620,11 +740,12 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                               const float *beta, const float *init, const int32_t *cu, void *out,
                               float *fin, int64_t interval, float *ck, int N, int H,
                               int64_t total_tokens, int32_t *dev_status, cudaStream_t stream) {
-  (void)total_tokens;
   // Few (sequence, head) units: split the value columns in two to fill the SMs.
   if ((int64_t)N * H * 2 <= 148)
-    return launch_tc_t<64>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N, H, dev_status, stream);
-  return launch_tc_t<128>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N, H, dev_status, stream);
+    return launch_tc_t<64>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N, H, total_tokens,
+                           dev_status, stream);
+  return launch_tc_t<128>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N, H, total_tokens,
+                          dev_status, stream);
 }
 
 }  // namespace kda
