@@ -21,16 +21,19 @@
 //
 // Gate numerics: exp(Gam_r - Gam_i) is split into a factor on each operand
 // so that both stay inside the FP32/BF16 exponent range.  With g >= -5 a
-// factor exp(+-(Gam - ref)) is at most e^80 when the reference sits in the
-// middle of a 32-token half.  The Gram products are therefore formed on three
-// 32x32 block pairs of the 64x64 matrices: the two diagonal pairs use the
-// middle of their half as reference, the off-diagonal pair uses the boundary
-// between the halves (both factors <= 1; an underflow there only loses
-// products below e^-87).
+// factor exp(+-(Gam_r - ref)) is at most e^80 when the reference sits in the
+// middle of a 32-token half, so each row r is scaled against the middle of
+// its own half (Gam_15 or Gam_47).  The key operand then comes in two
+// versions: k_i exp(Gam_15 - Gam_i) (i < 32) for rows of the first half and
+// k_i exp(Gam_47 - Gam_i) (i < 64) for rows of the second; one MMA with
+// N = 32 + 64 forms every needed product (the cross products are never
+// read).  In the second version a factor for i < 32 can underflow; the
+// product it belongs to is then below e^-12 (the other factor is at most
+// e^75), far below the BF16 rounding of the operands.
 //
 // Tensor-core work per chunk (BF16 operands in 128-byte-swizzled shared
 // tiles, FP32 accumulators in tensor memory):
-//   Gram:   3 x [64 x 32 x 128]    (rows: k-part and q-part of a half)
+//   Gram:   [k x; q x] (128x128) x [B^(0) | B^(1)] (96x128)^T -> M, P
 //   T-prod: [T;P] (128x64) x [Ktilde | V]           -> What, Utilde
 //   MMA1:   [What; Qtilde] (128x128) x S0_bf16      -> What S0, Qtilde S0
 //   MMA2:   [T;P] x U accumulated onto MMA1 (rows 64..127 become O),
@@ -51,7 +54,7 @@ constexpr int kDK = 128;    // key head size
 constexpr int kDV = 128;    // value head size (full)
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kLd = 65;     // row stride of the FP32 64x64 scratch matrices
+constexpr int kLd = 68;     // row stride of the FP32 64x64 scratch matrices (16-byte rows)
 
 template <int DVS>
 struct Layout {
@@ -66,11 +69,12 @@ struct Layout {
   static constexpr uint32_t STG_Q = G, STG_K = G + 16384;         //  next chunk's q, k [64][128] bf16
   static constexpr uint32_t STG_G = G + 32768;                    //  next chunk's g [64][128] fp32
   static constexpr uint32_t RED = G + 65536;                      //  float [16][128] scan partials
-  static constexpr uint32_t A00 = G, A11 = G + 16384, A10 = G + 32768;          // Gram A [64][128]
-  static constexpr uint32_t B00 = G + 49152, B11 = G + 57344, B10 = G + 65536;  // Gram B [32][128]
-  static constexpr uint32_t MM = G;                               //  float [64][65] M
-  static constexpr uint32_t XM = G + 16640;                       //  float [64][65] (I + M)^-1
-  static constexpr uint32_t YS = G + 33280;                       //  float [3][16][17]
+  static constexpr uint32_t GA = G;                               //  Gram A [128][128] K-major
+  static constexpr uint32_t GB = G + 32768;                       //  Gram B [96][128] K-major
+  static constexpr uint32_t MM = G;                               //  float [64][68] M
+  static constexpr uint32_t XM = G + 17408;                       //  float [64][68] (I + M)^-1
+  static constexpr uint32_t YS = G + 34816;                       //  float [2][16][17]
+  static constexpr uint32_t ZS = G + 36992;                       //  float [32][36]
   static constexpr uint32_t SMALL = G + 73728;
   static constexpr uint32_t BETA = SMALL;                         // float [64]
   static constexpr uint32_t DVEC = SMALL + 256;                   // float [128]
@@ -79,7 +83,7 @@ struct Layout {
   static constexpr uint32_t TBAR = BAR + 8;                       // mbarrier: TMA loads landed
   static constexpr uint32_t TMEM_SLOT = BAR + 16;
   static constexpr uint32_t TOTAL = BAR + 64;
-  static_assert(YS + 3 * 16 * 17 * 4 <= G + 73728, "solve scratch overflows");
+  static_assert(ZS + 32 * 36 * 4 <= G + 65536, "solve scratch overflows");
   static_assert(64 * DVS * 2 <= 16384, "U must fit the Ktilde slot");
 };
 
@@ -187,6 +191,7 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   float *s_M = reinterpret_cast<float *>(sp + Lay::MM);
   float *s_X = reinterpret_cast<float *>(sp + Lay::XM);
   float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
+  float *s_Z = reinterpret_cast<float *>(sp + Lay::ZS);
   uint64_t *bar = reinterpret_cast<uint64_t *>(sp + Lay::BAR);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -239,8 +244,9 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     tphase ^= 1;
 
     // ---------------- gate prep: cumulative decay and scaled operands ----------------
+    // Thread (rg, jc) owns rows 4rg..4rg+3 and channels 8jc..8jc+7 of the chunk.
     {
-      const int rg = tid >> 4, jc = tid & 15;   // rows 4rg..4rg+3, channels 8jc..8jc+7
+      const int rg = tid >> 4, jc = tid & 15, hf = rg >> 3;
       float gm[4][8], kk[4][8], qq[4][8];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -264,23 +270,31 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
 #pragma unroll
       for (int e = 0; e < 8; ++e) s_red[rg * 128 + 8 * jc + e] = gm[3][e];
       __syncthreads();
-      float base[8];
+      // Exclusive scan of the 16 row-group totals, channel by channel: warp w scans
+      // channels 16w..16w+15; lane (ch, half) holds row groups 8*half..8*half+7.
+      {
+        const int ch = 16 * warp + (lane & 15), half = lane >> 4;
+        float t[8], run = 0.f;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) base[e] = 0.f;
-      for (int p = 0; p < rg; ++p)
+        for (int i = 0; i < 8; ++i) t[i] = s_red[(8 * half + i) * 128 + ch];
+        float incl[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) base[e] += s_red[p * 128 + 8 * jc + e];
+        for (int i = 0; i < 8; ++i) { run += t[i]; incl[i] = run; }
+        const float lower = __shfl_sync(0xffffffffu, run, lane & 15);   // half 0's total
+        const float off = half ? lower : 0.f;
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) gm[i][e] += base[e];
-      if ((rg & 3) == 3)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s_gref[(rg >> 2) * 128 + 8 * jc + e] = gm[3][e];
+        for (int i = 0; i < 8; ++i) s_red[(8 * half + i) * 128 + ch] = off + incl[i] - t[i];
+        // cumulative decay at rows 15, 31, 47, 63 = ends of row groups 3, 7, 11, 15
+        s_gref[(2 * half + 0) * 128 + ch] = off + incl[3];
+        s_gref[(2 * half + 1) * 128 + ch] = off + incl[7];
+      }
       __syncthreads();
       float G15[8], G31[8], G47[8], G63[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
+        const float base = s_red[rg * 128 + 8 * jc + e];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) gm[i][e] += base;
         G15[e] = s_gref[0 * 128 + 8 * jc + e];
         G31[e] = s_gref[1 * 128 + 8 * jc + e];
         G47[e] = s_gref[2 * 128 + 8 * jc + e];
@@ -290,149 +304,114 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
 #pragma unroll
         for (int e = 0; e < 8; ++e) s_dvec[8 * jc + e] = __expf(G63[e]);
 
-      if (rg < 8) {   // first half: reference Gam_15 for the diagonal pair
-        float c1[8], e15[8], c12[8];
+      // Per-channel factors.  Row r of half hf is scaled against ref = Gam_15 (hf 0)
+      // or Gam_47 (hf 1): x = exp(Gam_r - ref), y = 1/x, both within [e^-80, e^80].
+      // Products are grouped so that an intermediate can only underflow when the
+      // exact value is itself below e^-87 (or, for the B^(1) rows of the first
+      // half and Ktilde of the second, below e^-12 times a unit-norm product).
+      float ref[8], fk[8], fk2[8], fh[8], fh2[8], cb[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (hf == 0) {
+          ref[e] = G15[e];
+          fk[e] = 1.f;                              // Ktilde: x * exp(Gam_15)
+          fk2[e] = __expf(G15[e]);                  //   exp(Gam_15) >= e^-80
+          fh[e] = __expf(G31[e] - G15[e]);          // Khat: (y * exp(Gam_31 - Gam_15))
+          fh2[e] = __expf(G63[e] - G31[e]);         //        * exp(Gam_63 - Gam_31)
+          cb[e] = __expf(G47[e] - G15[e]);          // B^(1) rows of the first half
+        } else {
+          ref[e] = G47[e];
+          fk[e] = __expf(G47[e] - G31[e]);          // Ktilde: (x * exp(Gam_47 - Gam_31))
+          fk2[e] = __expf(G31[e]);                  //          * exp(Gam_31)
+          fh[e] = __expf(G63[e] - G47[e]);          // Khat: y * exp(Gam_63 - Gam_47)
+          fh2[e] = 1.f;
+          cb[e] = 0.f;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * rg + i;
+        float x[8], y[8], t[8], kt[8], kh[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          c1[e] = __expf(G31[e] - G15[e]);            // in [e^-80, 1]
-          e15[e] = __expf(G15[e]);                    // in [e^-80, 1]
-          c12[e] = c1[e] * __expf(G63[e] - G31[e]);   // may underflow: harmless
+          x[e] = __expf(gm[i][e] - ref[e]);
+          // reciprocal by two Newton steps from the bit-level initial guess
+          float r0 = __int_as_float(0x7EF311C3 - __float_as_int(x[e]));
+          r0 = r0 * fmaf(-x[e], r0, 2.f);
+          y[e] = r0 * fmaf(-x[e], r0, 2.f);
+          kt[e] = (x[e] * fk[e]) * fk2[e];          // exp(Gam_r)
+          kh[e] = (y[e] * fh[e]) * fh2[e];          // exp(Gam_63 - Gam_r)
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = 4 * rg + i;
-          float x[8], y[8], t[8];
+        for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * x[e];
+        tc::st_chunk(sb + Lay::GA + tc::tile_offset(128, r, jc), t);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            x[e] = __expf(gm[i][e] - G15[e]);
-            y[e] = __expf(G15[e] - gm[i][e]);
-          }
+        for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * x[e];
+        tc::st_chunk(sb + Lay::GA + tc::tile_offset(128, 64 + r, jc), t);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * x[e];
-          tc::st_chunk(sb + Lay::A00 + tc::tile_offset(64, r, jc), t);
+        for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * y[e];
+        tc::st_chunk(sb + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, jc), t);
+        if (!hf) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * x[e];
-          tc::st_chunk(sb + Lay::A00 + tc::tile_offset(64, 32 + r, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * y[e];
-          tc::st_chunk(sb + Lay::B00 + tc::tile_offset(32, r, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (y[e] * c1[e]);
-          tc::st_chunk(sb + Lay::B10 + tc::tile_offset(32, r, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (x[e] * e15[e]);
-          tc::st_chunk(sb + Lay::KV_T + tc::tile_offset(64, r, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * (x[e] * e15[e]);
-          tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, 64 + r, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (y[e] * c12[e]);
-          tc::st_chunk(sb + Lay::KH_T + tc::tile_offset(64, r, jc), t);
-        }
-      } else {        // second half: reference Gam_47 (diagonal), Gam_31 (off-diagonal)
-        float c3[8], e31[8], c4[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          c3[e] = __expf(G47[e] - G31[e]);            // in [e^-80, 1]
-          e31[e] = __expf(G31[e]);                    // may underflow: harmless
-          c4[e] = __expf(G63[e] - G47[e]);            // in [e^-80, 1]
+          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (y[e] * cb[e]);
+          tc::st_chunk(sb + Lay::GB + tc::tile_offset(96, 32 + r, jc), t);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = 4 * rg + i, rl = r - 32;
-          float x[8], y[8], xo[8], t[8];
+        for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * kt[e];
+        tc::st_chunk(sb + Lay::KV_T + tc::tile_offset(64, r, jc), t);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            x[e] = __expf(gm[i][e] - G47[e]);
-            y[e] = __expf(G47[e] - gm[i][e]);
-            xo[e] = x[e] * c3[e];                     // exp(Gam_r - Gam_31) <= 1
-          }
+        for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * kt[e];
+        tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, 64 + r, jc), t);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * x[e];
-          tc::st_chunk(sb + Lay::A11 + tc::tile_offset(64, rl, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * x[e];
-          tc::st_chunk(sb + Lay::A11 + tc::tile_offset(64, 32 + rl, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * y[e];
-          tc::st_chunk(sb + Lay::B11 + tc::tile_offset(32, rl, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * xo[e];
-          tc::st_chunk(sb + Lay::A10 + tc::tile_offset(64, rl, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * xo[e];
-          tc::st_chunk(sb + Lay::A10 + tc::tile_offset(64, 32 + rl, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (xo[e] * e31[e]);
-          tc::st_chunk(sb + Lay::KV_T + tc::tile_offset(64, r, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * (xo[e] * e31[e]);
-          tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, 64 + r, jc), t);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (y[e] * c4[e]);
-          tc::st_chunk(sb + Lay::KH_T + tc::tile_offset(64, r, jc), t);
-        }
+        for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * kh[e];
+        tc::st_chunk(sb + Lay::KH_T + tc::tile_offset(64, r, jc), t);
       }
       tc::fence_smem_to_async();
       __syncthreads();
     }
 
-    // ---------------- gated Gram products on the tensor cores ----------------
+    // ---------------- gated Gram products: one [128 x 96 x 128] MMA ----------------
+    // A = [k_r x_r ; q_r x_r] (rows 0..63 k, 64..127 q), B = [k_i exp(Gam_15 - Gam_i), i < 32 |
+    // k_i exp(Gam_47 - Gam_i), i < 64].  Rows of the first half use columns 0..31, rows of
+    // the second half columns 32..95; the other products are never read.
     if (tid == 0) {
       tc::fence_after_sync();
-      constexpr uint32_t id = tc::idesc_bf16(64, 32, 0, 0);
-      const uint32_t A[3] = {sb + Lay::A00, sb + Lay::A11, sb + Lay::A10};
-      const uint32_t B[3] = {sb + Lay::B00, sb + Lay::B11, sb + Lay::B10};
+      constexpr uint32_t id = tc::idesc_bf16(128, 96, 0, 0);
 #pragma unroll
-      for (int p = 0; p < 3; ++p)
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          tc::mma_bf16(tmem + 32 * p, tc::desc_kmajor(A[p], 64, s), tc::desc_kmajor(B[p], 32, s),
-                       id, s > 0);
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::GA, 128, s2), tc::desc_kmajor(sb + Lay::GB, 96, s2),
+                     id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
     if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
     phase ^= 1;
     tc::fence_after_sync();
 
-    // Read the Gram blocks (M=64 layout: row m in lane (m%16) + 32*(m/16)).  Warps 0-3
-    // take pairs 00 and 11, warps 4-7 pair 10.  k-part rows become rows of the FP32
-    // matrix M (scaled by beta_r, strictly lower); q-part rows become rows of P,
-    // written straight into rows 64..127 of the bf16 [T; P] operand.
+    // Read the Gram rows: lane m = row m.  k-part rows become rows of the FP32 matrix M
+    // (scaled by beta_r, strictly lower); q-part rows become rows of P, written straight
+    // into rows 64..127 of the bf16 [T; P] operand.
     {
+      const int m = 32 * qd + lane, part = m >> 6, r = m & 63, second = r >> 5;
+      // first-half rows: hw 0 reads columns 0..31, hw 1 writes the zero half;
+      // second-half rows: hw 0 reads i = 0..31 (columns 32..63), hw 1 i = 32..63.
+      const int i0 = second ? 32 * hw : (hw ? 32 : 0);
       float a[32];
-#pragma unroll
-      for (int pp = 0; pp < 2; ++pp) {
-        const int p = hw == 0 ? pp : 2;
-        if (hw == 1 && pp == 1) break;
-        tc::tmem_ld32(tl + 32 * p, a);
+      if (second || hw == 0) {
+        tc::tmem_ld32(tl + (second ? 32 + 32 * hw : 0), a);
         tc::tmem_wait_ld();
-        if (lane < 16) {
-          const int m = 16 * qd + lane, part = m >> 5, rl = m & 31;
-          const int r = p == 0 ? rl : 32 + rl;
-          const int cbase = p == 1 ? 32 : 0;
-          if (part == 0) {
-            float *dst = s_M + r * kLd + cbase;
-            const float br = s_beta[r];
+      }
+      const bool zero = !second && hw;
+      if (part == 0) {
+        const float br = s_beta[r];
+        float *dst = s_M + r * kLd + i0;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) dst[j] = (p == 2 || j < rl) ? br * a[j] : 0.f;
-            if (p == 0)
+        for (int j = 0; j < 32; ++j) dst[j] = (!zero && i0 + j < r) ? br * a[j] : 0.f;
+      } else {
 #pragma unroll
-              for (int j = 32; j < 64; ++j) s_M[r * kLd + j] = 0.f;
-          } else {
+        for (int j = 0; j < 32; ++j) a[j] = (!zero && i0 + j <= r) ? a[j] : 0.f;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) a[j] = (p == 2 || j <= rl) ? a[j] : 0.f;
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc)
-              tc::st_chunk(sb + Lay::TP_T + tc::tile_offset(128, 64 + r, (cbase >> 3) + cc), a + 8 * cc);
-            if (p == 0) {
-              float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-              for (int cc = 4; cc < 8; ++cc)
-                tc::st_chunk(sb + Lay::TP_T + tc::tile_offset(128, 64 + r, cc), z);
-            }
-          }
-        }
+        for (int cc = 0; cc < 4; ++cc)
+          tc::st_chunk(sb + Lay::TP_T + tc::tile_offset(128, 64 + r, (i0 >> 3) + cc), a + 8 * cc);
       }
     }
     tc::fence_before_sync();
@@ -458,64 +437,60 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * kLd + o + c] = x[i];
-    }
-    __syncthreads();
-    // distance 1: (1,0), (2,1), (3,2)
-    for (int e = tid; e < 768; e += kThreads) {
-      const int pi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, b = pi + 1, a = pi;
-      float acc = 0.f;
+      if ((warp & 1) == 0)   // block above the diagonal inside the 32-row half
 #pragma unroll
-      for (int s = 0; s < 16; ++s) acc += s_M[(16 * b + rr) * kLd + 16 * a + s] * s_X[(16 * a + s) * kLd + 16 * a + cc];
-      s_Y[(pi * 16 + rr) * 17 + cc] = acc;
+        for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * kLd + o + 16 + c] = 0.f;
     }
     __syncthreads();
-    for (int e = tid; e < 768; e += kThreads) {
-      const int pi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, b = pi + 1, a = pi;
-      float acc = 0.f;
-#pragma unroll
-      for (int s = 0; s < 16; ++s) acc += s_X[(16 * b + rr) * kLd + 16 * b + s] * s_Y[(pi * 16 + s) * 17 + cc];
-      s_X[(16 * b + rr) * kLd + 16 * a + cc] = -acc;
-    }
-    __syncthreads();
-    // distance 2: (2,0), (3,1)
-    for (int e = tid; e < 512; e += kThreads) {
-      const int pi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, b = pi + 2, a = pi;
-      float acc = 0.f;
-#pragma unroll
-      for (int s = 0; s < 16; ++s)
-        acc += s_M[(16 * b + rr) * kLd + 16 * a + s] * s_X[(16 * a + s) * kLd + 16 * a + cc] +
-               s_M[(16 * b + rr) * kLd + 16 * (a + 1) + s] * s_X[(16 * (a + 1) + s) * kLd + 16 * a + cc];
-      s_Y[(pi * 16 + rr) * 17 + cc] = acc;
-    }
-    __syncthreads();
-    for (int e = tid; e < 512; e += kThreads) {
-      const int pi = e >> 8, rr = (e >> 4) & 15, cc = e & 15, b = pi + 2, a = pi;
-      float acc = 0.f;
-#pragma unroll
-      for (int s = 0; s < 16; ++s) acc += s_X[(16 * b + rr) * kLd + 16 * b + s] * s_Y[(pi * 16 + s) * 17 + cc];
-      s_X[(16 * b + rr) * kLd + 16 * a + cc] = -acc;
-    }
-    __syncthreads();
-    // distance 3: (3,0)
+    // Level 1: the 32x32 inverse of each half, X_(2h+1,2h) = -X_(2h+1,2h+1) M_(2h+1,2h) X_(2h,2h).
     {
-      const int rr = tid >> 4, cc = tid & 15;
-      float acc = 0.f;
+      const int hh = tid >> 7, rr = (tid >> 3) & 15, c0 = (tid & 7) * 2;
+      const int ro = 32 * hh + 16, co = 32 * hh;
+      float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-      for (int c3 = 0; c3 < 3; ++c3)
+      for (int s2 = 0; s2 < 16; ++s2) {
+        const float m = s_M[(ro + rr) * kLd + co + s2];
+        const float2 xv = *reinterpret_cast<const float2 *>(s_X + (co + s2) * kLd + co + c0);
+        y0 = fmaf(m, xv.x, y0);
+        y1 = fmaf(m, xv.y, y1);
+      }
+      s_Y[(hh * 16 + rr) * 17 + c0] = y0;
+      s_Y[(hh * 16 + rr) * 17 + c0 + 1] = y1;
+      __syncthreads();
+      float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-        for (int s = 0; s < 16; ++s)
-          acc += s_M[(48 + rr) * kLd + 16 * c3 + s] * s_X[(16 * c3 + s) * kLd + cc];
-      s_Y[rr * 17 + cc] = acc;
+      for (int s2 = 0; s2 < 16; ++s2) {
+        const float a = s_X[(ro + rr) * kLd + ro + s2];
+        x0 = fmaf(a, s_Y[(hh * 16 + s2) * 17 + c0], x0);
+        x1 = fmaf(a, s_Y[(hh * 16 + s2) * 17 + c0 + 1], x1);
+      }
+      *reinterpret_cast<float2 *>(s_X + (ro + rr) * kLd + co + c0) = make_float2(-x0, -x1);
+      __syncthreads();
     }
-    __syncthreads();
+    // Level 2: X_(1,0) = -H1 M_(1,0) H0 on the 32x32 halves (H0, H1 lower triangular).
     {
-      const int rr = tid >> 4, cc = tid & 15;
-      float acc = 0.f;
-#pragma unroll
-      for (int s = 0; s < 16; ++s) acc += s_X[(48 + rr) * kLd + 48 + s] * s_Y[s * 17 + cc];
-      s_X[(48 + rr) * kLd + cc] = -acc;
+      const int rr = tid >> 3, cq = (tid & 7) * 4;
+      float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+      for (int s2 = 0; s2 < 32; ++s2) {
+        const float m = s_M[(32 + rr) * kLd + s2];
+        const float4 xv = *reinterpret_cast<const float4 *>(s_X + s2 * kLd + cq);
+        z.x = fmaf(m, xv.x, z.x); z.y = fmaf(m, xv.y, z.y);
+        z.z = fmaf(m, xv.z, z.z); z.w = fmaf(m, xv.w, z.w);
+      }
+      *reinterpret_cast<float4 *>(s_Z + rr * 36 + cq) = z;
+      __syncthreads();
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+      for (int s2 = 0; s2 < 32; ++s2) {
+        const float a = s_X[(32 + rr) * kLd + 32 + s2];
+        const float4 zv = *reinterpret_cast<const float4 *>(s_Z + s2 * 36 + cq);
+        w.x = fmaf(a, zv.x, w.x); w.y = fmaf(a, zv.y, w.y);
+        w.z = fmaf(a, zv.z, w.z); w.w = fmaf(a, zv.w, w.w);
+      }
+      *reinterpret_cast<float4 *>(s_X + (32 + rr) * kLd + cq) = make_float4(-w.x, -w.y, -w.z, -w.w);
+      __syncthreads();
     }
-    __syncthreads();
     // T rows of the [T; P] operand: T_ri = X_ri beta_i (i <= r).
     for (int e = tid; e < 64 * 8; e += kThreads) {
       const int row = e >> 3, ch = e & 7;

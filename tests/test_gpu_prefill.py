@@ -60,6 +60,25 @@ def test_decay_at_floor_and_extremes(chunk):
         check_full(d, chunk, interval=chunk)
 
 
+@pytest.mark.parametrize("pattern", ["strong_16_32", "strong_32_48", "strong_first_half",
+                                     "strong_last_16", "alternate_8"])
+def test_decay_patterns_inside_a_chunk(pattern):
+    """Strong decay (g = -5) confined to parts of each 64-token chunk and none elsewhere:
+    the cumulative decay then spans the full exponent range inside one chunk, which is
+    where a factored exp(Gam_r - Gam_i) could overflow or lose non-negligible terms."""
+    lengths = [256, 130]
+    d = make_case(lengths, 2, 128, 128, torch.bfloat16, seed=21, state_std=0.3)
+    pos = torch.cat([torch.arange(n) for n in lengths]) % 64
+    mask = {"strong_16_32": (pos >= 16) & (pos < 32),
+            "strong_32_48": (pos >= 32) & (pos < 48),
+            "strong_first_half": pos < 32,
+            "strong_last_16": pos >= 48,
+            "alternate_8": (pos // 8) % 2 == 0}[pattern]
+    d["g"] = torch.where(mask[:, None, None], torch.full_like(d["g"], -5.0),
+                         torch.zeros_like(d["g"])).contiguous()
+    check_full(d, 64, interval=64)
+
+
 def test_identity_tokens_keep_state():
     """beta = 0 and g = 0: the final state is the initial one and o_t = S0^T q_t."""
     d = make_case([50, 13], 2, 64, 32, torch.float32, seed=3, state_std=1.0)
