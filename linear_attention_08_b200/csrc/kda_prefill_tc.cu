@@ -3,9 +3,10 @@
 // Covers BF16 q/k/v/out with D_k = D_v = 128 and 64-token chunks; the FP32
 // state never leaves the chip between chunks.  The method: prefill groups the
 // tokens into chunks, unrolls the recurrence inside a chunk into dense matrix
-// products and carries the state between chunks ("Kimi K3 architecture"
-// summary, Methods 1, FlashKDA; Kimi-K3 deep dive section 4-1, chunk-parallel
-// tiles with a recurrence between them).
+// products and carries the state between chunks
+// ("LLM - Semianalysis, Kimi K3 아키텍처" (charstring.tistory.com/2557),
+// Methods 1, FlashKDA; "MoonshotAI/Kimi-K3 딥다이브" (fiv.co.kr/repos/kimi-k3-deep-dive.html),
+// section 4-1, chunk-parallel tiles with a recurrence between them).
 //
 // One CTA owns one (sequence, head, slice of DVS value columns) and walks its
 // sequence chunk by chunk.  For a chunk of 64 tokens starting from S0, with

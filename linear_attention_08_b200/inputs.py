@@ -11,8 +11,8 @@ Distributions (one value per token-head unless noted):
 * v ~ N(0, 1), cast to the compute dtype;
 * beta = sigmoid(N(0, 1)) in FP32;
 * g = max(-softplus(N(0, 1)), -5) in FP32 per key channel: a natural-log decay
-  with the lower bound of -5 that the Kimi K3 deep dive (section 4-1,
-  "lower-bounded decay") asks for;
+  with the lower bound of -5 for the lower-bounded decay that
+  "MoonshotAI/Kimi-K3 딥다이브" (fiv.co.kr/repos/kimi-k3-deep-dive.html), section 4-1, describes;
 * the initial state, when requested, ~ N(0, std^2) in FP32.
 
 Draw order from one generator: q, k, v, beta-logits, g-logits, init_state.
