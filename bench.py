@@ -351,12 +351,46 @@ def time_decode(steps_graph, warmup, world, local, decode_steps=None):
                 flops=token_heads * decode_flops_per_token_head(Dk), clocks=clk.result)
 
 
+def time_spec_decode(steps, warmup, world, local, T_new=8):
+    """Multi-token decode: 512 sequences x 32 heads, T_new draft tokens each, all
+    accepted.  One call moves the FP32 state once for T_new tokens."""
+    from linear_attention_08_b200 import kda
+    N, H, D = 512, 32, 128
+    d = kin.make_inputs((N, T_new), H, D, D, torch.bfloat16, local, num_states=N,
+                        state_std=0.02, device="cuda")
+    state = d["init_state"].clone()
+    out = torch.empty_like(d["v"])
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.kda_decode_multi(d["q"], d["k"], d["v"], d["g"], d["beta"], state, out=out,
+                             stream=stream)
+
+    for _ in range(max(warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    byts = N * H * (decode_state_bytes_per_token_head(D, D)
+                    + T_new * prefill_io_bytes_per_token_head(D, D, 2))
+    return dict(tokens=N * T_new, ms=ms, bytes=byts, T_new=T_new)
+
+
 def run_ours(args, rank, world, local):
     peaks, peaks_src = load_peaks()
     hbm = peaks["hbm_gbs"]
     tflops = peaks["bf16_tflops"]
     name = args.workload
     res = time_prefill(name, args.steps, args.warmup, world, local) if name != "decode" else None
+    spec = None
+    if not args.no_decode:
+        spec = time_spec_decode(max(args.steps, 5), args.warmup, world, local)
     dec = None
     if name == "decode" or not args.no_decode:
         dec = time_decode(max(1, args.steps // 2) if name != "decode" else args.steps,
@@ -407,6 +441,16 @@ def run_ours(args, rank, world, local):
                     "h2d_bytes_per_step": dec["bi"], "d2h_bytes_per_step": dec["bo"]},
             "gpu_launches": dec["launches"], "clocks": dec["clocks"],
         }
+        if spec is not None:
+            sgbs = spec["bytes"] / (spec["ms"] / 1e3) / 1e9
+            dobj["spec_decode"] = {
+                "metric": "KDA multi-token decode tokens/s",
+                "value": world * spec["tokens"] / (spec["ms"] / 1e3), "unit": "tokens/s",
+                "ms_per_call": spec["ms"],
+                "config": {"num_seqs": 512, "heads": 32, "d": 128, "tokens_per_seq": spec["T_new"],
+                           "accepted": "all"},
+                "roofline": {"bound": "hbm", "achieved": sgbs, "peak": hbm, "unit": "GB/s",
+                             "frac": sgbs / hbm, "kernel": "decode_multi"}}
         if res is None:
             line = dict(dobj)
             line.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -108,6 +108,28 @@ kda_status kda_decode(const void *q, const void *k, const void *v, const float *
                       const float *beta, float *state_inout, void *out,
                       const kda_shape *shape, kda_stream_t stream);
 
+/*
+ * Multi-token decode for speculative-decoding verification: every sequence
+ * brings tokens_per_seq new tokens (a draft), all of them run through the
+ * recurrence from state_inout, the output of every token is written, and
+ * state_inout is then replaced by the state reached after the first
+ * accept_len[n] tokens of sequence n (0 leaves it unchanged).  accept_len
+ * may be NULL: all tokens are accepted.  The state crosses HBM once per call.
+ *
+ *   q, k, g : [N, tokens_per_seq, H, D_k]   v, out : [N, tokens_per_seq, H, D_v]
+ *   beta    : [N, tokens_per_seq, H]         accept_len : device int32[N] or NULL
+ *   state_inout : [N, H, D_k, D_v]
+ * shape->total_tokens must equal N * tokens_per_seq; 1 <= tokens_per_seq <= 64.
+ * Values of accept_len outside [0, tokens_per_seq] are clamped.  This is the
+ * recurrence of the decode step applied token by token (the first page,
+ * Methods 1: decode runs the recurrence directly); the serving side that
+ * decides acceptance is not part of this library.
+ */
+kda_status kda_decode_multi(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float *state_inout, void *out,
+                            const int32_t *accept_len, int32_t tokens_per_seq,
+                            const kda_shape *shape, kda_stream_t stream);
+
 /* Host helper: sum_i floor(T_i / ckpt_interval) for host int32 cu_seqlens[N+1]
  * (0 when ckpt_interval <= 0; -1 on a bad argument). */
 int64_t kda_ckpt_count(const int32_t *host_cu_seqlens, int32_t num_seqs, int64_t ckpt_interval);

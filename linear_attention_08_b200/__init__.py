@@ -5,7 +5,7 @@ include/kda.h (libkda.so, built in-tree by ``linear_attention_08_b200.build``).
 ``linear_attention_08_b200.kda`` is the ctypes binding; ``inputs`` draws the
 seeded synthetic workloads.
 """
-from .kda import (kda_ckpt_count, kda_decode, kda_prefill, kda_prefill_path,  # noqa: F401
-                  kda_selftest_bounded_wait, load)
+from .kda import (kda_ckpt_count, kda_decode, kda_decode_multi,  # noqa: F401
+                  kda_prefill, kda_prefill_path, kda_selftest_bounded_wait, load)
 
 __version__ = "0.1.0"

@@ -12,6 +12,10 @@ cudaError_t launch_prefill_simt(int dtype, int dk, int dv, const void *q, const 
                                 const void *v, const float *g, const float *beta,
                                 const float *init, const int32_t *cu, void *out, float *fin,
                                 int64_t interval, float *ck, int N, int H, cudaStream_t stream);
+cudaError_t launch_decode_multi(int dtype, int dk, int dv, const void *q, const void *k,
+                                const void *v, const float *g, const float *beta, float *state,
+                                void *out, const int32_t *accept_len, int T_new, int64_t units,
+                                int H, cudaStream_t stream);
 bool prefill_tc_supported(int dtype, int dk, int dv, int chunk);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *init, const int32_t *cu,
@@ -162,6 +166,35 @@ kda_status kda_decode(const void *q, const void *k, const void *v, const float *
   return cuda_status(launch_decode(s->qkv_dtype, s->head_dim_k, s->head_dim_v, q, k, v, g, beta,
                                    state_inout, out, units, s->num_heads,
                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_decode_multi(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, float *state_inout, void *out,
+                            const int32_t *accept_len, int32_t tokens_per_seq,
+                            const kda_shape *s, kda_stream_t stream) {
+  kda_status st = check_shape(s, false);
+  if (st != KDA_OK) return st;
+  if (tokens_per_seq < 1 || tokens_per_seq > 64) return KDA_ERR_INVALID_ARGUMENT;
+  if (s->total_tokens != (int64_t)s->num_seqs * tokens_per_seq) return KDA_ERR_INVALID_ARGUMENT;
+  const void *ptrs[] = {q, k, v, g, state_inout, out};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+  if (!beta || (reinterpret_cast<uintptr_t>(beta) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
+  if (accept_len && (reinterpret_cast<uintptr_t>(accept_len) & 3u)) return KDA_ERR_INVALID_ARGUMENT;
+  const int64_t units = (int64_t)s->num_seqs * s->num_heads;
+  const int64_t T = s->total_tokens, H = s->num_heads;
+  const size_t es = elem_size(s->qkv_dtype);
+  const size_t n_out = (size_t)T * H * s->head_dim_v * es;
+  const size_t n_state = (size_t)units * s->head_dim_k * s->head_dim_v * 4;
+  if (overlaps(out, n_out, state_inout, n_state) ||
+      overlaps(out, n_out, q, (size_t)T * H * s->head_dim_k * es) ||
+      overlaps(out, n_out, k, (size_t)T * H * s->head_dim_k * es) ||
+      overlaps(out, n_out, v, n_out) || overlaps(out, n_out, g, (size_t)T * H * s->head_dim_k * 4))
+    return KDA_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_decode_multi(s->qkv_dtype, s->head_dim_k, s->head_dim_v, q, k, v, g,
+                                         beta, state_inout, out, accept_len, tokens_per_seq,
+                                         units, s->num_heads,
+                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

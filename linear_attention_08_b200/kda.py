@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 KDA_OK, KDA_ERR_INVALID_ARGUMENT, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 
-EXPORTED = ("kda_prefill", "kda_decode", "kda_ckpt_count", "kda_prefill_workspace_bytes",
+EXPORTED = ("kda_prefill", "kda_decode", "kda_decode_multi", "kda_ckpt_count", "kda_prefill_workspace_bytes",
             "kda_prefill_path", "kda_selftest_bounded_wait", "kda_last_cuda_error",
             "kda_status_string", "kda_version")
 
@@ -62,6 +62,8 @@ def load(path: str | None = None):
     lib.kda_prefill.restype = ctypes.c_int
     lib.kda_decode.argtypes = [P, P, P, P, P, P, P, SP, P]
     lib.kda_decode.restype = ctypes.c_int
+    lib.kda_decode_multi.argtypes = [P, P, P, P, P, P, P, P, I32, SP, P]
+    lib.kda_decode_multi.restype = ctypes.c_int
     lib.kda_ckpt_count.argtypes = [P, I32, I64]
     lib.kda_ckpt_count.restype = I64
     lib.kda_prefill_workspace_bytes.argtypes = [SP]
@@ -161,6 +163,26 @@ def kda_decode(q, k, v, g, beta, state, *, out=None, dev_status=None, stream=Non
                         ctypes.byref(shape), _stream(stream))
     if st != KDA_OK:
         raise KdaError(st, "kda_decode")
+    return out
+
+
+def kda_decode_multi(q, k, v, g, beta, state, *, accept_len=None, out=None, dev_status=None,
+                     stream=None):
+    """Multi-token decode: q, k, g [N, T_new, H, Dk]; v [N, T_new, H, Dv]; beta
+    [N, T_new, H]; state [N, H, Dk, Dv] FP32, replaced by the state after the
+    first accept_len[n] tokens (int32 device tensor, or None for all).
+    Returns out [N, T_new, H, Dv]."""
+    lib = load()
+    N, T_new, H, Dk = q.shape
+    Dv = v.shape[3]
+    if out is None:
+        out = torch.empty(N, T_new, H, Dv, dtype=q.dtype, device=q.device)
+    shape = make_shape(N, N * T_new, H, Dk, Dv, 0, _dtype_code(q), dev_status)
+    st = lib.kda_decode_multi(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state),
+                              _ptr(out), _ptr(accept_len), int(T_new), ctypes.byref(shape),
+                              _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_decode_multi")
     return out
 
 

@@ -112,3 +112,20 @@ def test_workspace_and_path_queries():
 def test_binding_fails_loudly_without_library(tmp_path):
     with pytest.raises(ImportError):
         kda.load(str(tmp_path / "missing.so"))
+
+
+def test_decode_multi_rejects_bad_arguments():
+    lib = kda.load()
+    a = ctypes.c_void_p(1 << 20)
+    st = ctypes.c_void_p(1 << 26)
+    o = ctypes.c_void_p(1 << 28)
+    good = kda.make_shape(4, 4 * 8, 2, 32, 32, 0, 1)
+    for tokens in (0, 65):
+        assert lib.kda_decode_multi(a, a, a, a, a, st, o, None, tokens, ctypes.byref(good),
+                                    None) == kda.KDA_ERR_INVALID_ARGUMENT
+    bad = kda.make_shape(4, 4 * 8 + 1, 2, 32, 32, 0, 1)       # total_tokens != N * T_new
+    assert lib.kda_decode_multi(a, a, a, a, a, st, o, None, 8, ctypes.byref(bad),
+                                None) == kda.KDA_ERR_INVALID_ARGUMENT
+    mis = ctypes.c_void_p((1 << 20) + 2)                        # misaligned accept_len
+    assert lib.kda_decode_multi(a, a, a, a, a, st, o, mis, 8, ctypes.byref(good),
+                                None) == kda.KDA_ERR_INVALID_ARGUMENT
