@@ -79,8 +79,8 @@ struct Layout {
   static constexpr uint32_t SMALL = G + 73728;
   static constexpr uint32_t BETA = SMALL;                         // float [64]
   static constexpr uint32_t DVEC = SMALL + 256;                   // float [128]
-  static constexpr uint32_t GREF = SMALL + 768;                   // float [4][128]
-  static constexpr uint32_t BAR = GREF + 2048;                    // mbarrier: MMA completion
+  static constexpr uint32_t CST = SMALL + 768;                    // float [2][6][128] gate factors
+  static constexpr uint32_t BAR = CST + 6144;                     // mbarrier: MMA completion
   static constexpr uint32_t TBAR = BAR + 8;                       // mbarrier: TMA loads landed
   static constexpr uint32_t TMEM_SLOT = BAR + 16;
   static constexpr uint32_t TOTAL = BAR + 64;
@@ -188,7 +188,7 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   float *s_beta = reinterpret_cast<float *>(sp + Lay::BETA);
   float *s_dvec = reinterpret_cast<float *>(sp + Lay::DVEC);
   float *s_red = reinterpret_cast<float *>(sp + Lay::RED);
-  float *s_gref = reinterpret_cast<float *>(sp + Lay::GREF);
+  float *s_cst = reinterpret_cast<float *>(sp + Lay::CST);
   float *s_M = reinterpret_cast<float *>(sp + Lay::MM);
   float *s_X = reinterpret_cast<float *>(sp + Lay::XM);
   float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
@@ -276,6 +276,7 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
       __syncthreads();
       // Exclusive scan of the 16 row-group totals, channel by channel: warp w scans
       // channels 16w..16w+15; lane (ch, half) holds row groups 8*half..8*half+7.
+      // The same lanes form each channel's gate factors once (for both halves).
       {
         const int ch = 16 * warp + (lane & 15), half = lane >> 4;
         float t[8], run = 0.f;
@@ -288,12 +289,39 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
         const float off = half ? lower : 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) s_red[(8 * half + i) * 128 + ch] = off + incl[i] - t[i];
-        // cumulative decay at rows 15, 31, 47, 63 = ends of row groups 3, 7, 11, 15
-        s_gref[(2 * half + 0) * 128 + ch] = off + incl[3];
-        s_gref[(2 * half + 1) * 128 + ch] = off + incl[7];
+        // cumulative decay at rows 15, 31 (half 0) and 47, 63 (half 1)
+        const float ga = off + incl[3], gb = off + incl[7];
+        const float G15 = __shfl_sync(0xffffffffu, ga, lane & 15);
+        const float G31 = __shfl_sync(0xffffffffu, gb, lane & 15);
+        const float G47 = __shfl_sync(0xffffffffu, ga, (lane & 15) + 16);
+        const float G63 = __shfl_sync(0xffffffffu, gb, (lane & 15) + 16);
+        // Row r of half hf is scaled against ref = Gam_15 (hf 0) or Gam_47 (hf 1):
+        // x = exp(Gam_r - ref), y = 1/x, both within [e^-80, e^80].  Products are
+        // grouped so that an intermediate can only underflow when the exact value
+        // is itself below e^-87 (or, for the B^(1) rows of the first half and
+        // Ktilde of the second, below e^-12 times a unit-norm product).
+        float f[6];
+        if (half == 0) {
+          f[0] = G15;                       // ref
+          f[1] = 1.f;                       // Ktilde: (x * 1) * exp(Gam_15)
+          f[2] = __expf(G15);
+          f[3] = __expf(G31 - G15);         // Khat: (y * exp(Gam_31 - Gam_15)) * exp(Gam_63 - Gam_31)
+          f[4] = __expf(G63 - G31);
+          f[5] = __expf(G47 - G15);         // B^(1) rows of the first half
+        } else {
+          f[0] = G47;
+          f[1] = __expf(G47 - G31);         // Ktilde: (x * exp(Gam_47 - Gam_31)) * exp(Gam_31)
+          f[2] = __expf(G31);
+          f[3] = __expf(G63 - G47);         // Khat: y * exp(Gam_63 - Gam_47)
+          f[4] = 1.f;
+          f[5] = 0.f;
+          s_dvec[ch] = __expf(G63);
+        }
+#pragma unroll
+        for (int j = 0; j < 6; ++j) s_cst[(half * 6 + j) * 128 + ch] = f[j];
       }
       __syncthreads();
-      float G15[8], G31[8], G47[8], G63[8], base[8];
+      float base[8], ref[8], fk[8], fk2[8], fh[8], fh2[8], cb[8];
       {
         // 128-bit reads: 16 threads cover 512 contiguous bytes, no bank conflicts
         auto ld8 = [&](const float *src, float *d8) {
@@ -302,46 +330,19 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
           d8[0] = a.x; d8[1] = a.y; d8[2] = a.z; d8[3] = a.w;
           d8[4] = b.x; d8[5] = b.y; d8[6] = b.z; d8[7] = b.w;
         };
+        const float *c = s_cst + hf * 6 * 128 + 8 * jc;
         ld8(s_red + rg * 128 + 8 * jc, base);
-        ld8(s_gref + 0 * 128 + 8 * jc, G15);
-        ld8(s_gref + 1 * 128 + 8 * jc, G31);
-        ld8(s_gref + 2 * 128 + 8 * jc, G47);
-        ld8(s_gref + 3 * 128 + 8 * jc, G63);
+        ld8(c + 0 * 128, ref);
+        ld8(c + 1 * 128, fk);
+        ld8(c + 2 * 128, fk2);
+        ld8(c + 3 * 128, fh);
+        ld8(c + 4 * 128, fh2);
+        ld8(c + 5 * 128, cb);
       }
 #pragma unroll
       for (int e = 0; e < 8; ++e)
 #pragma unroll
         for (int i = 0; i < 4; ++i) gm[i][e] += base[e];
-      if (rg == 0) {
-        float4 *dv = reinterpret_cast<float4 *>(s_dvec + 8 * jc);
-        dv[0] = make_float4(__expf(G63[0]), __expf(G63[1]), __expf(G63[2]), __expf(G63[3]));
-        dv[1] = make_float4(__expf(G63[4]), __expf(G63[5]), __expf(G63[6]), __expf(G63[7]));
-      }
-
-      // Per-channel factors.  Row r of half hf is scaled against ref = Gam_15 (hf 0)
-      // or Gam_47 (hf 1): x = exp(Gam_r - ref), y = 1/x, both within [e^-80, e^80].
-      // Products are grouped so that an intermediate can only underflow when the
-      // exact value is itself below e^-87 (or, for the B^(1) rows of the first
-      // half and Ktilde of the second, below e^-12 times a unit-norm product).
-      float ref[8], fk[8], fk2[8], fh[8], fh2[8], cb[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if (hf == 0) {
-          ref[e] = G15[e];
-          fk[e] = 1.f;                              // Ktilde: x * exp(Gam_15)
-          fk2[e] = __expf(G15[e]);                  //   exp(Gam_15) >= e^-80
-          fh[e] = __expf(G31[e] - G15[e]);          // Khat: (y * exp(Gam_31 - Gam_15))
-          fh2[e] = __expf(G63[e] - G31[e]);         //        * exp(Gam_63 - Gam_31)
-          cb[e] = __expf(G47[e] - G15[e]);          // B^(1) rows of the first half
-        } else {
-          ref[e] = G47[e];
-          fk[e] = __expf(G47[e] - G31[e]);          // Ktilde: (x * exp(Gam_47 - Gam_31))
-          fk2[e] = __expf(G31[e]);                  //          * exp(Gam_31)
-          fh[e] = __expf(G63[e] - G47[e]);          // Khat: y * exp(Gam_63 - Gam_47)
-          fh2[e] = 1.f;
-          cb[e] = 0.f;
-        }
-      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = 4 * rg + i;
