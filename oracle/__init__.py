@@ -48,6 +48,8 @@ def _bind(lib):
     lib.kda_oracle_recurrent.restype = ctypes.c_int
     lib.kda_oracle_chunked.argtypes = common + [I64]
     lib.kda_oracle_chunked.restype = ctypes.c_int
+    lib.kda_oracle_recurrent_pos.argtypes = common + [P, P, P]
+    lib.kda_oracle_recurrent_pos.restype = ctypes.c_int
     lib.kda_oracle_max_threads.restype = ctypes.c_int
     return lib
 
@@ -76,14 +78,16 @@ def ckpt_count(lengths, interval: int) -> int:
 
 
 def prefill(q, k, v, g, beta, cu_seqlens, init_state=None, ckpt_interval: int = 0,
-            chunk: int = 0, nthreads: int = 0, lib=None):
+            chunk: int = 0, nthreads: int = 0, lib=None, positions=None):
     """Run the oracle over a packed batch.
 
     q, k, g: [T_tot, H, Dk]; v: [T_tot, H, Dv]; beta: [T_tot, H];
     cu_seqlens: N+1 offsets; init_state: [N, H, Dk, Dv] or None (zeros).
     ``chunk`` = 0 runs the token-by-token recurrence, > 0 the chunked form.
     Returns (out [T_tot, H, Dv], final_state [N, H, Dk, Dv],
-    checkpoints [n_ckpt, H, Dk, Dv]) as float64 numpy arrays.
+    checkpoints [n_ckpt, H, Dk, Dv]) as float64 numpy arrays.  With
+    ``positions`` (one list of token counts per sequence) a fourth array
+    [n_pos, H, Dk, Dv] holds the states after those counts.
     """
     lib = lib or load()
     q, k, v, g, beta = (_f64(a) for a in (q, k, v, g, beta))
@@ -102,6 +106,19 @@ def prefill(q, k, v, g, beta, cu_seqlens, init_state=None, ckpt_interval: int = 
     ck = np.zeros((max(nck, 1), H, Dk, Dv))
     args = [N, _ptr(cu), H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init),
             int(ckpt_interval), _ptr(out), _ptr(fin), _ptr(ck), int(nthreads)]
+    if positions is not None:
+        if chunk != 0:
+            raise ValueError("explicit positions are supported by the recurrent form only")
+        pos_cu = np.zeros(N + 1, dtype=np.int64)
+        for i, lst in enumerate(positions):
+            pos_cu[i + 1] = pos_cu[i] + len(lst)
+        pos = np.ascontiguousarray(np.concatenate([np.asarray(l, dtype=np.int64) for l in positions])
+                                   if pos_cu[-1] else np.zeros(1, dtype=np.int64))
+        ps = np.zeros((max(int(pos_cu[-1]), 1), H, Dk, Dv))
+        rc = lib.kda_oracle_recurrent_pos(*args, _ptr(pos_cu), _ptr(pos), _ptr(ps))
+        if rc != 0:
+            raise ValueError(f"oracle rejected its arguments (status {rc})")
+        return out, fin, ck[:nck], ps[:int(pos_cu[-1])]
     if chunk == 0:
         rc = lib.kda_oracle_recurrent(*args)
     else:

@@ -280,6 +280,32 @@ def pin_varlen(lib):
     return float(err)
 
 
+# --- explicit positions: the state after j tokens is the final state of the first j ---
+def pin_positions(lib):
+    rng = np.random.default_rng(22)
+    lengths = [19, 7, 12]
+    p = rand_problem(rng, lengths, 2, 3, 4)
+    positions = [[1, 5, 5, 13, 19, 30], [0, 7], []]
+    o, f, ck, ps = oracle.prefill(p["q"], p["k"], p["v"], p["g"], p["beta"], p["cu_seqlens"],
+                                  p["init_state"], 0, 0, 2, lib, positions)
+    if ps.shape[0] != sum(len(x) for x in positions):
+        return float("inf")
+    err, j = 0.0, 0
+    cu = p["cu_seqlens"]
+    for n, lst in enumerate(positions):
+        for pos in lst:
+            m = max(0, min(pos, lengths[n]))
+            a = cu[n]
+            pn = {key: (val[a:a + m] if key in ("q", "k", "v", "g", "beta") else val)
+                  for key, val in p.items()}
+            pn["init_state"] = p["init_state"][n:n + 1]
+            pn["cu_seqlens"] = np.array([0, m], dtype=np.int64)
+            _, fn, _ = _run(lib, pn)
+            err = max(err, np.abs(ps[j] - fn[0]).max())
+            j += 1
+    return float(err)
+
+
 # name -> (function, bound)
 PINS = {
     "identity_tokens": (pin_identity_tokens, 1e-15),
@@ -297,4 +323,5 @@ PINS = {
     "column_split": (pin_column_split, 1e-14),
     "checkpoint_resume": (pin_checkpoint_resume, 1e-12),
     "varlen": (pin_varlen, 1e-14),
+    "positions": (pin_positions, 1e-14),
 }
