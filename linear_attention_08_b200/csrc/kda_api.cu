@@ -11,7 +11,9 @@ cudaError_t launch_decode(int dtype, int dk, int dv, const void *q, const void *
 cudaError_t launch_prefill_simt(int dtype, int dk, int dv, const void *q, const void *k,
                                 const void *v, const float *g, const float *beta,
                                 const float *init, const int32_t *cu, void *out, float *fin,
-                                int64_t interval, float *ck, int N, int H, cudaStream_t stream);
+                                int64_t interval, float *ck, const int32_t *pos_cu,
+                                const int32_t *positions, float *pos_states, int N, int H,
+                                cudaStream_t stream);
 cudaError_t launch_decode_multi(int dtype, int dk, int dv, const void *q, const void *k,
                                 const void *v, const float *g, const float *beta, float *state,
                                 void *out, const int32_t *accept_len, int T_new, int64_t units,
@@ -19,8 +21,10 @@ cudaError_t launch_decode_multi(int dtype, int dk, int dv, const void *q, const 
 bool prefill_tc_supported(int dtype, int dk, int dv, int chunk);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *init, const int32_t *cu,
-                              void *out, float *fin, int64_t interval, float *ck, int N, int H,
-                              int64_t total_tokens, int32_t *dev_status, cudaStream_t stream);
+                              void *out, float *fin, int64_t interval, float *ck,
+                              const int32_t *pos_cu, const int32_t *positions, float *pos_states,
+                              int N, int H, int64_t total_tokens, int32_t *dev_status,
+                              cudaStream_t stream);
 
 static thread_local int g_last_cuda_error = 0;
 
@@ -103,6 +107,15 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
                        const float *beta, const float *init_state, const int32_t *cu_seqlens,
                        void *out, float *final_state, int64_t ckpt_interval,
                        float *ckpt_states, const kda_shape *s, kda_stream_t stream) {
+  return kda_prefill_at(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
+                        ckpt_interval, ckpt_states, nullptr, nullptr, nullptr, s, stream);
+}
+
+kda_status kda_prefill_at(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                          void *out, float *final_state, int64_t ckpt_interval,
+                          float *ckpt_states, const int32_t *pos_cu, const int32_t *positions,
+                          float *pos_states, const kda_shape *s, kda_stream_t stream) {
   kda_status st = check_shape(s, true);
   if (st != KDA_OK) return st;
   const int N = s->num_seqs, H = s->num_heads, DK = s->head_dim_k, DV = s->head_dim_v;
@@ -120,6 +133,11 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
   if (ckpt_interval < 0 || ckpt_interval % s->chunk != 0) return KDA_ERR_INVALID_ARGUMENT;
   if ((ckpt_interval > 0) != (ckpt_states != nullptr)) return KDA_ERR_INVALID_ARGUMENT;
   if (ckpt_states && !aligned16(ckpt_states)) return KDA_ERR_INVALID_ARGUMENT;
+  if ((positions != nullptr) != (pos_cu != nullptr) || (positions != nullptr) != (pos_states != nullptr))
+    return KDA_ERR_INVALID_ARGUMENT;
+  if (positions && ((reinterpret_cast<uintptr_t>(positions) & 3u) ||
+                    (reinterpret_cast<uintptr_t>(pos_cu) & 3u) || !aligned16(pos_states)))
+    return KDA_ERR_INVALID_ARGUMENT;
   const size_t es = elem_size(s->qkv_dtype);
   const size_t n_out = (size_t)T * H * DV * es;
   const size_t n_qk = (size_t)T * H * DK * es, n_v = (size_t)T * H * DV * es;
@@ -137,10 +155,12 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
   cudaError_t e;
   if (T > 0 && prefill_tc_supported(s->qkv_dtype, DK, DV, s->chunk))
     e = launch_prefill_tc(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
-                          ckpt_interval, ckpt_states, N, H, T, s->dev_status, cs);
+                          ckpt_interval, ckpt_states, pos_cu, positions, pos_states, N, H, T,
+                          s->dev_status, cs);
   else
     e = launch_prefill_simt(s->qkv_dtype, DK, DV, q, k, v, g, beta, init_state, cu_seqlens, out,
-                            final_state, ckpt_interval, ckpt_states, N, H, cs);
+                            final_state, ckpt_interval, ckpt_states, pos_cu, positions,
+                            pos_states, N, H, cs);
   return cuda_status(e);
 }
 

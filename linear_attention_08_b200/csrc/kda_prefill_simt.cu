@@ -52,7 +52,9 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                     const float *__restrict__ beta, const float *__restrict__ init_state,
                     const int32_t *__restrict__ cu_seqlens, TIn *__restrict__ out,
                     float *__restrict__ final_state, int64_t ckpt_interval,
-                    float *__restrict__ ckpt_states, int H, int DV) {
+                    float *__restrict__ ckpt_states, const int32_t *__restrict__ pos_cu,
+                    const int32_t *__restrict__ positions, float *__restrict__ pos_states,
+                    int H, int DV) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SimtSmem<DK> &sm = *reinterpret_cast<SimtSmem<DK> *>(smem_raw);
   constexpr int T = kSimtTile, W = kSimtSlice, NT = kSimtThreads;
@@ -61,19 +63,43 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
   const int col0 = blockIdx.y * W;             // first value column of this slice
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  const int64_t t_begin = cu_seqlens[seq], t_end = cu_seqlens[seq + 1];
+  const int64_t t_begin = cu_seqlens[seq], t_end = cu_seqlens[seq + 1], T_seq = t_end - t_begin;
   int64_t ck_slot = 0;
   if (ckpt_interval > 0)
     for (int j = 0; j < seq; ++j) ck_slot += (cu_seqlens[j + 1] - cu_seqlens[j]) / ckpt_interval;
+  int pi = positions ? pos_cu[seq] : 0;
+  const int pe = positions ? pos_cu[seq + 1] : 0;
 
   const size_t state_off = (size_t)unit * DK * DV;
   for (int e = tid; e < DK * W; e += NT) {
     const int c = e / W, j = e % W;
     sm.S[c][j] = init_state ? init_state[state_off + (size_t)c * DV + col0 + j] : 0.f;
   }
+  // Copy the state slice into a [.., H, DK, DV] array (after a barrier).
+  auto store_state = [&](float *base_ptr, int64_t slot) {
+    __syncthreads();
+    float *dst = base_ptr + ((size_t)slot * H + h) * DK * DV;
+    for (int e = tid; e < DK * W; e += NT) {
+      const int c = e / W, j = e % W;
+      dst[(size_t)c * DV + col0 + j] = sm.S[c][j];
+    }
+  };
+  while (pi < pe && positions[pi] <= 0) store_state(pos_states, pi++);   // initial state
 
-  for (int64_t c0 = t_begin; c0 < t_end; c0 += T) {
-    const int L = (int)(t_end - c0 < T ? t_end - c0 : T);
+  // Tiles end at the next checkpoint boundary or explicit position, so every
+  // stored state is the state at a tile end (tiling does not change the result).
+  for (int64_t done = 0; done < T_seq;) {
+    const int64_t c0 = t_begin + done;
+    int64_t m = T_seq - done < T ? T_seq - done : T;
+    if (ckpt_interval > 0) {
+      const int64_t to_ck = ckpt_interval - done % ckpt_interval;
+      m = to_ck < m ? to_ck : m;
+    }
+    if (pi < pe) {
+      const int64_t to_pos = (int64_t)positions[pi] - done;
+      m = to_pos < m ? to_pos : m;
+    }
+    const int L = (int)m;
     __syncthreads();  // previous tile fully consumed
     for (int e = tid; e < T * DK; e += NT) {
       const int r = e / DK, c = e % DK;
@@ -175,17 +201,11 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
       sm.S[c][j] = s;
     }
 
-    const int64_t done = c0 + L - t_begin;
-    if (ckpt_interval > 0 && L == T && done % ckpt_interval == 0) {
-      __syncthreads();
-      float *dst = ckpt_states + ((size_t)ck_slot * H + h) * DK * DV;
-      for (int e = tid; e < DK * W; e += NT) {
-        const int c = e / W, j = e % W;
-        dst[(size_t)c * DV + col0 + j] = sm.S[c][j];
-      }
-      ++ck_slot;
-    }
+    done += L;
+    if (ckpt_interval > 0 && done % ckpt_interval == 0) store_state(ckpt_states, ck_slot++);
+    while (pi < pe && positions[pi] <= done) store_state(pos_states, pi++);
   }
+  while (pi < pe) store_state(pos_states, pi++);   // positions past the end: final state
   __syncthreads();
   if (final_state)
     for (int e = tid; e < DK * W; e += NT) {
@@ -197,8 +217,9 @@ prefill_simt_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 template <int DK, typename TIn>
 static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const float *init, const int32_t *cu,
-                                 void *out, float *fin, int64_t interval, float *ck, int N,
-                                 int H, int DV, cudaStream_t stream) {
+                                 void *out, float *fin, int64_t interval, float *ck,
+                                 const int32_t *pos_cu, const int32_t *positions,
+                                 float *pos_states, int N, int H, int DV, cudaStream_t stream) {
   const size_t smem = sizeof(SimtSmem<DK>);
   auto kern = prefill_simt_kernel<DK, TIn>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -206,24 +227,26 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)((int64_t)N * H), (unsigned)(DV / kSimtSlice));
   kern<<<grid, kSimtThreads, smem, stream>>>((const TIn *)q, (const TIn *)k, (const TIn *)v, g,
-                                             beta, init, cu, (TIn *)out, fin, interval, ck, H,
-                                             DV);
+                                             beta, init, cu, (TIn *)out, fin, interval, ck,
+                                             pos_cu, positions, pos_states, H, DV);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_simt(int dtype, int dk, int dv, const void *q, const void *k,
                                 const void *v, const float *g, const float *beta,
                                 const float *init, const int32_t *cu, void *out, float *fin,
-                                int64_t interval, float *ck, int N, int H,
+                                int64_t interval, float *ck, const int32_t *pos_cu,
+                                const int32_t *positions, float *pos_states, int N, int H,
                                 cudaStream_t stream) {
   if (dv % kSimtSlice != 0) return cudaErrorInvalidValue;
 #define KDA_SIMT(DK_)                                                                        \
   if (dk == DK_) {                                                                           \
     if (dtype == KDA_DTYPE_BF16)                                                             \
       return launch_simt_t<DK_, __nv_bfloat16>(q, k, v, g, beta, init, cu, out, fin,         \
-                                               interval, ck, N, H, dv, stream);             \
-    return launch_simt_t<DK_, float>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N,  \
-                                     H, dv, stream);                                         \
+                                               interval, ck, pos_cu, positions, pos_states,  \
+                                               N, H, dv, stream);                            \
+    return launch_simt_t<DK_, float>(q, k, v, g, beta, init, cu, out, fin, interval, ck,     \
+                                     pos_cu, positions, pos_states, N, H, dv, stream);       \
   }
   KDA_SIMT(32) KDA_SIMT(64) KDA_SIMT(128)
 #undef KDA_SIMT

@@ -177,8 +177,9 @@ template <int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ beta, const float *__restrict__ init,
                   const int32_t *__restrict__ cu, __nv_bfloat16 *__restrict__ out,
-                  float *__restrict__ fin, int64_t interval, float *__restrict__ ck, int H,
-                  int32_t *dev_status, uint64_t wait_ns) {
+                  float *__restrict__ fin, int64_t interval, float *__restrict__ ck,
+                  const int32_t *__restrict__ pos_cu, const int32_t *__restrict__ positions,
+                  float *__restrict__ pos_states, int H, int32_t *dev_status, uint64_t wait_ns) {
   using Lay = Layout<DVS>;
   constexpr int NCOL = DVS / 2;           // state columns per thread
   extern __shared__ uint8_t smem_raw[];
@@ -227,19 +228,46 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   for (int j = 0; j < NCOL; j += 8)
     tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + j) >> 3), S + j);
 
-  const int64_t t_begin = cu[seq], t_end = cu[seq + 1];
+  const int64_t t_begin = cu[seq], t_end = cu[seq + 1], T_seq = t_end - t_begin;
   int64_t ck_slot = 0;
   if (interval > 0)
     for (int j = 0; j < seq; ++j) ck_slot += (int64_t)(cu[j + 1] - cu[j]) / interval;
+  // Explicit state positions of this sequence (token counts), if any.
+  int pi = positions ? pos_cu[seq] : 0;
+  const int pe = positions ? pos_cu[seq + 1] : 0;
+  // Store the FP32 state slice of this thread into a [.., H, D_k, D_v] array.
+  auto store_state = [&](float *base_ptr, int64_t slot) {
+    float *dst = base_ptr + ((size_t)slot * H + h) * kDK * kDV + (size_t)crow * kDV + col0 + hw * NCOL;
+#pragma unroll
+    for (int j = 0; j < NCOL; j += 4)
+      *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+  };
+  // Length of the chunk that starts after `done` tokens: at most 64, and it ends
+  // at the next checkpoint boundary or explicit position (chunking does not
+  // change the result, so every stored state is the state at a chunk end).
+  auto chunk_len = [&](int64_t done, int p) -> int {
+    int64_t m = T_seq - done < kC ? T_seq - done : kC;
+    if (interval > 0) {
+      const int64_t to_ck = interval - done % interval;
+      m = to_ck < m ? to_ck : m;
+    }
+    if (p < pe) {
+      const int64_t to_pos = (int64_t)positions[p] - done;
+      m = to_pos < m ? to_pos : m;
+    }
+    return (int)m;
+  };
+  while (pi < pe && positions[pi] <= 0) store_state(pos_states, pi++);   // initial state
+
   uint32_t phase = 0, tphase = 0;
   bool aborted = false;
   uint64_t *tbar = reinterpret_cast<uint64_t *>(sp + Lay::TBAR);
-  if (t_begin < t_end)
-    prefetch_chunk<DVS>(sb, maps, beta, t_begin,
-                        (int)((t_end - t_begin) < kC ? (t_end - t_begin) : kC), H, h, col0, tid);
+  int64_t done = 0;
+  int L = T_seq > 0 ? chunk_len(0, pi) : 0;
+  if (T_seq > 0) prefetch_chunk<DVS>(sb, maps, beta, t_begin, L, H, h, col0, tid);
 
-  for (int64_t t0 = t_begin; t0 < t_end; t0 += kC) {
-    const int L = (int)((t_end - t0) < kC ? (t_end - t0) : kC);
+  while (done < T_seq) {
+    const int64_t t0 = t_begin + done;
     cp_async_wait_all();
     if (__syncthreads_or(!wait_timed(tbar, tphase, wait_ns))) { aborted = true; break; }
     tphase ^= 1;
@@ -533,9 +561,12 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
     phase ^= 1;
     tc::fence_after_sync();
-    if (t0 + kC < t_end)
-      prefetch_chunk<DVS>(sb, maps, beta, t0 + kC,
-                          (int)((t_end - t0 - kC) < kC ? (t_end - t0 - kC) : kC), H, h, col0, tid);
+    const int64_t done_next = done + L;
+    int p_next = pi;
+    while (p_next < pe && positions[p_next] <= done_next) ++p_next;
+    const int L_next = done_next < T_seq ? chunk_len(done_next, p_next) : 0;
+    if (done_next < T_seq)
+      prefetch_chunk<DVS>(sb, maps, beta, t_begin + done_next, L_next, H, h, col0, tid);
     if (qd < 2) {   // What rows 0..63 -> bf16 operand rows 0..63 of [What; Qtilde]
       const int r = 32 * qd + lane;
       float a[32];
@@ -634,13 +665,10 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
 #pragma unroll
       for (int j = 0; j < NCOL; j += 8)
         tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + j) >> 3), S + j);
-      if (interval > 0 && L == kC && (t0 + kC - t_begin) % interval == 0) {
-        float *dst = ck + ((size_t)ck_slot * H + h) * kDK * kDV + (size_t)crow * kDV + col0 + hw * NCOL;
-#pragma unroll
-        for (int j = 0; j < NCOL; j += 4)
-          *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-        ++ck_slot;
-      }
+      done += L;
+      if (interval > 0 && done % interval == 0) store_state(ck, ck_slot++);
+      while (pi < pe && positions[pi] <= done) store_state(pos_states, pi++);
+      L = L_next;
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -654,11 +682,14 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     // what they were given before the CTA releases its memory.
     wait_timed(bar, phase, wait_ns);
     wait_timed(tbar, tphase, wait_ns);
-  } else if (fin) {
-    float *dst = fin + soff;
+  } else {
+    while (pi < pe) store_state(pos_states, pi++);   // positions past the end: final state
+    if (fin) {
+      float *dst = fin + soff;
 #pragma unroll
-    for (int j = 0; j < NCOL; j += 4)
-      *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+      for (int j = 0; j < NCOL; j += 4)
+        *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    }
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -702,7 +733,8 @@ static bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, i
 template <int DVS>
 cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const float *g,
                         const float *beta, const float *init, const int32_t *cu, void *out,
-                        float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
+                        float *fin, int64_t interval, float *ck, const int32_t *pos_cu,
+                        const int32_t *positions, float *pos_states, int N, int H, int64_t T,
                         int32_t *dev_status, cudaStream_t stream) {
   TmaMaps maps;
   if (!make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, H, T, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
@@ -716,7 +748,8 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const float
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)((int64_t)N * H), (unsigned)(kDV / DVS));
   kern<<<grid, kThreads, smem, stream>>>(maps, beta, init, cu, (__nv_bfloat16 *)out, fin, interval,
-                                         ck, H, dev_status, 2000000000ull);
+                                         ck, pos_cu, positions, pos_states, H, dev_status,
+                                         2000000000ull);
   return cudaGetLastError();
 }
 
@@ -728,14 +761,15 @@ bool prefill_tc_supported(int dtype, int dk, int dv, int chunk) {
 
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *init, const int32_t *cu, void *out,
-                              float *fin, int64_t interval, float *ck, int N, int H,
+                              float *fin, int64_t interval, float *ck, const int32_t *pos_cu,
+                              const int32_t *positions, float *pos_states, int N, int H,
                               int64_t total_tokens, int32_t *dev_status, cudaStream_t stream) {
   // Few (sequence, head) units: split the value columns in two to fill the SMs.
   if ((int64_t)N * H * 2 <= 148)
-    return launch_tc_t<64>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N, H, total_tokens,
-                           dev_status, stream);
-  return launch_tc_t<128>(q, k, v, g, beta, init, cu, out, fin, interval, ck, N, H, total_tokens,
-                          dev_status, stream);
+    return launch_tc_t<64>(q, k, v, g, beta, init, cu, out, fin, interval, ck, pos_cu, positions,
+                           pos_states, N, H, total_tokens, dev_status, stream);
+  return launch_tc_t<128>(q, k, v, g, beta, init, cu, out, fin, interval, ck, pos_cu, positions,
+                          pos_states, N, H, total_tokens, dev_status, stream);
 }
 
 }  // namespace kda

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 KDA_OK, KDA_ERR_INVALID_ARGUMENT, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 
-EXPORTED = ("kda_prefill", "kda_decode", "kda_decode_multi", "kda_ckpt_count", "kda_prefill_workspace_bytes",
+EXPORTED = ("kda_prefill", "kda_prefill_at", "kda_decode", "kda_decode_multi", "kda_ckpt_count", "kda_prefill_workspace_bytes",
             "kda_prefill_path", "kda_selftest_bounded_wait", "kda_last_cuda_error",
             "kda_status_string", "kda_version")
 
@@ -60,6 +60,8 @@ def load(path: str | None = None):
     SP = ctypes.POINTER(KdaShape)
     lib.kda_prefill.argtypes = [P, P, P, P, P, P, P, P, P, I64, P, SP, P]
     lib.kda_prefill.restype = ctypes.c_int
+    lib.kda_prefill_at.argtypes = [P, P, P, P, P, P, P, P, P, I64, P, P, P, P, SP, P]
+    lib.kda_prefill_at.restype = ctypes.c_int
     lib.kda_decode.argtypes = [P, P, P, P, P, P, P, SP, P]
     lib.kda_decode.restype = ctypes.c_int
     lib.kda_decode_multi.argtypes = [P, P, P, P, P, P, P, P, I32, SP, P]
@@ -118,13 +120,17 @@ def kda_prefill_path(shape: KdaShape) -> int:
 
 def kda_prefill(q, k, v, g, beta, cu_seqlens, *, init_state=None, chunk: int = 64,
                 ckpt_interval: int = 0, cu_seqlens_host=None, out=None, final_state=None,
-                ckpt_states=None, dev_status=None, stream=None, want_final: bool = True):
+                ckpt_states=None, dev_status=None, stream=None, want_final: bool = True,
+                positions=None, pos_states=None):
     """Chunked KDA prefill over a packed batch (see kda_prefill in include/kda.h).
 
     q, k, g: [T, H, Dk]; v: [T, H, Dv]; beta: [T, H]; cu_seqlens: int32 device
     [N+1]; init_state: [N, H, Dk, Dv] FP32 or None.  Outputs are allocated
     with torch when not given.  ``cu_seqlens_host`` (a list) avoids a device
-    read when checkpoints are requested.  Returns (out, final_state, ckpt_states).
+    read when checkpoints are requested.  ``positions`` (one list of token
+    counts per sequence) also stores the states after those counts
+    (kda_prefill_at).  Returns (out, final_state, ckpt_states), plus
+    pos_states when positions are given.
     """
     lib = load()
     T, H, Dk = q.shape
@@ -142,12 +148,32 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, *, init_state=None, chunk: int = 6
     ck_ptr = _ptr(ckpt_states) if ckpt_interval > 0 else None
     if ckpt_interval > 0 and ckpt_states.numel() == 0:
         ck_ptr = ctypes.c_void_p(ckpt_states.untyped_storage().data_ptr())
-    st = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init_state),
-                         _ptr(cu_seqlens), _ptr(out), _ptr(final_state), int(ckpt_interval),
-                         ck_ptr, ctypes.byref(shape), _stream(stream))
+    if positions is None:
+        st = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init_state),
+                             _ptr(cu_seqlens), _ptr(out), _ptr(final_state), int(ckpt_interval),
+                             ck_ptr, ctypes.byref(shape), _stream(stream))
+        if st != KDA_OK:
+            raise KdaError(st, "kda_prefill")
+        return out, final_state, ckpt_states
+    counts = [0]
+    for lst in positions:
+        counts.append(counts[-1] + len(lst))
+    assert len(counts) == N + 1, "one list of positions per sequence"
+    pos_cu = torch.tensor(counts, dtype=torch.int32, device=q.device)
+    flat = [int(x) for lst in positions for x in lst]
+    pos = torch.tensor(flat or [0], dtype=torch.int32, device=q.device)
+    if pos_states is None:
+        pos_states = torch.empty(max(counts[-1], 1), H, Dk, Dv, dtype=torch.float32,
+                                 device=q.device)[:counts[-1]]
+    ps_ptr = ctypes.c_void_p(pos_states.untyped_storage().data_ptr()) if counts[-1] == 0 \
+        else _ptr(pos_states)
+    st = lib.kda_prefill_at(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init_state),
+                            _ptr(cu_seqlens), _ptr(out), _ptr(final_state), int(ckpt_interval),
+                            ck_ptr, _ptr(pos_cu), _ptr(pos), ps_ptr, ctypes.byref(shape),
+                            _stream(stream))
     if st != KDA_OK:
-        raise KdaError(st, "kda_prefill")
-    return out, final_state, ckpt_states
+        raise KdaError(st, "kda_prefill_at")
+    return out, final_state, ckpt_states, pos_states
 
 
 def kda_decode(q, k, v, g, beta, state, *, out=None, dev_status=None, stream=None):

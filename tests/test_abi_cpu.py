@@ -129,3 +129,20 @@ def test_decode_multi_rejects_bad_arguments():
     mis = ctypes.c_void_p((1 << 20) + 2)                        # misaligned accept_len
     assert lib.kda_decode_multi(a, a, a, a, a, st, o, mis, 8, ctypes.byref(good),
                                 None) == kda.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_prefill_at_requires_all_position_pointers():
+    lib = kda.load()
+    s = _shape()
+    a = ctypes.c_void_p(1 << 20)
+    b = ctypes.c_void_p(1 << 24)
+    c = ctypes.c_void_p(1 << 28)
+    # positions without pos_cu / pos_states
+    assert lib.kda_prefill_at(a, a, a, a, a, None, a, b, None, 0, None, None, a, None,
+                              ctypes.byref(s), None) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_prefill_at(a, a, a, a, a, None, a, b, None, 0, None, a, a, None,
+                              ctypes.byref(s), None) == kda.KDA_ERR_INVALID_ARGUMENT
+    # misaligned pos_states
+    assert lib.kda_prefill_at(a, a, a, a, a, None, a, b, None, 0, None, a, a,
+                              ctypes.c_void_p((1 << 28) + 4), ctypes.byref(s),
+                              None) == kda.KDA_ERR_INVALID_ARGUMENT
