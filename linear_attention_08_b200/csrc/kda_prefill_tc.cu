@@ -15,8 +15,8 @@
 //   M_ri = beta_r sum_c k_rc k_ic exp(Gam_rc - Gam_ic)   (i < r)  gated Gram of k
 //   P_ri = sum_c q_rc k_ic exp(Gam_rc - Gam_ic)          (i <= r) gated q.k^T
 //   T    = (I + M)^-1 diag(beta)                          UT transform
-//   What = T Ktilde, Utilde = T V      (Ktilde_r = k_r exp(Gam_r))   WY form
-//   U    = Utilde - What S0                               delta-rule corrections
+//   X    = V - Ktilde S0               (Ktilde_r = k_r exp(Gam_r))
+//   U    = T X                                            delta-rule corrections
 //   O    = Qtilde S0 + P U             (Qtilde_r = q_r exp(Gam_r))
 //   S    = Diag(exp(Gam_63)) S0 + Khat^T U   (Khat_r = k_r exp(Gam_63 - Gam_r))
 //
@@ -35,10 +35,12 @@
 // Tensor-core work per chunk (BF16 operands in 128-byte-swizzled shared
 // tiles, FP32 accumulators in tensor memory):
 //   Gram:   [k x; q x] (128x128) x [B^(0) | B^(1)] (96x128)^T -> M, P
-//   T-prod: [T;P] (128x64) x [Ktilde | V]           -> What, Utilde
-//   MMA1:   [What; Qtilde] (128x128) x S0_bf16      -> What S0, Qtilde S0
+//   MMA1:   [Ktilde; Qtilde] (128x128) x S0_bf16   -> Ktilde S0, Qtilde S0
+//           (issued with the Gram product: it needs only the gates and S0)
+//   MMA-U:  [T;P] (128x64) x X (64xDVS)            -> U (rows 0..63)
 //   MMA2:   [T;P] x U accumulated onto MMA1 (rows 64..127 become O),
 //           Khat^T (128x64) x U                     -> state increment
+// The state-dependent chain per chunk is MMA1 -> X -> MMA-U -> MMA2.
 // The triangular solve, the gates and the FP32 state update run on the SIMT
 // pipes.  The FP32 state of the CTA's slice stays in registers: row c of the
 // state belongs to TMEM lane c.
@@ -60,12 +62,11 @@ constexpr int kLd = 68;     // row stride of the FP32 64x64 scratch matrices (16
 template <int DVS>
 struct Layout {
   static constexpr uint32_t S_T = 0;                              // [128][DVS]  state, MN-major B
-  static constexpr uint32_t WQ_T = S_T + 128 * DVS * 2;           // [128][128]  What;Qtilde, K-major A
+  static constexpr uint32_t WQ_T = S_T + 128 * DVS * 2;           // [128][128]  Ktilde;Qtilde, K-major A
   static constexpr uint32_t TP_T = WQ_T + 32768;                  // [128][64]   T;P, K-major A
   static constexpr uint32_t KH_T = TP_T + 16384;                  // [64][128]   Khat, MN-major A
-  static constexpr uint32_t KV_T = KH_T + 16384;                  // [64][128+DVS] Ktilde|V, MN-major B
-  static constexpr uint32_t U_T = KV_T;                           // [64][DVS] U, MN-major B, reuses
-                                                                  //   the Ktilde slot after the WY product
+  static constexpr uint32_t KV_T = KH_T + 16384;                  // [64][128+DVS]: X then U | V
+  static constexpr uint32_t U_T = KV_T;                           // [64][DVS] X, then U, MN-major B
   static constexpr uint32_t G = KV_T + 64 * (128 + DVS) * 2;      // 72 KB region, used in turn for:
   static constexpr uint32_t STG_Q = G, STG_K = G + 16384;         //  next chunk's q, k [64][128] bf16
   static constexpr uint32_t STG_G = G + 32768;                    //  next chunk's g [64][128] fp32
@@ -82,7 +83,8 @@ struct Layout {
   static constexpr uint32_t CST = SMALL + 768;                    // float [2][6][128] gate factors
   static constexpr uint32_t BAR = CST + 6144;                     // mbarrier: MMA completion
   static constexpr uint32_t TBAR = BAR + 8;                       // mbarrier: TMA loads landed
-  static constexpr uint32_t TMEM_SLOT = BAR + 16;
+  static constexpr uint32_t SBAR = BAR + 16;                      // mbarrier: state product done
+  static constexpr uint32_t TMEM_SLOT = BAR + 24;
   static constexpr uint32_t TOTAL = BAR + 64;
   static_assert(ZS + 32 * 36 * 4 <= G + 65536, "solve scratch overflows");
   static_assert(64 * DVS * 2 <= 16384, "U must fit the Ktilde slot");
@@ -116,7 +118,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 //   q, k : bf16, box (128, 1, 64), no swizzle   -> staging rows of 256 bytes
 //   g    : fp32, box (128, 1, 64), no swizzle   -> staging rows of 512 bytes
 //   v    : bf16, box (64, 1, 64), 128-byte swizzle -> one column block of the
-//          [Ktilde | V] operand tile, already in the MMA layout.
+//          [X/U | V] tile, already in the MMA layout.
 // Tokens past T_tot read as zeros; tokens of the next sequence are masked by
 // the consumer (q, k, g) or cancel exactly (v: beta is 0 there).
 struct TmaMaps {
@@ -145,7 +147,7 @@ __device__ __forceinline__ void prefetch_chunk(uint32_t sb, const TmaMaps &maps,
                                                int64_t t0, int L, int H, int h, int col0,
                                                int tid) {
   using Lay = Layout<DVS>;
-  if (tid == 0) {
+  if (tid == 32) {   // not thread 0, which issues the tensor-core work
     const uint32_t bar = sb + Lay::TBAR;
     mbar_expect_tx(bar, 64 * (256 + 256 + 512) + 64 * DVS * 2);
     const int z = (int)t0;
@@ -205,6 +207,7 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(reinterpret_cast<uint64_t *>(sp + Lay::TBAR), 1);
+    mbar_init(reinterpret_cast<uint64_t *>(sp + Lay::SBAR), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.g)) : "memory");
@@ -259,9 +262,10 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   };
   while (pi < pe && positions[pi] <= 0) store_state(pos_states, pi++);   // initial state
 
-  uint32_t phase = 0, tphase = 0;
+  uint32_t phase = 0, tphase = 0, sphase = 0;
   bool aborted = false;
   uint64_t *tbar = reinterpret_cast<uint64_t *>(sp + Lay::TBAR);
+  uint64_t *sbar = reinterpret_cast<uint64_t *>(sp + Lay::SBAR);
   int64_t done = 0;
   int L = T_seq > 0 ? chunk_len(0, pi) : 0;
   if (T_seq > 0) prefetch_chunk<DVS>(sb, maps, beta, t_begin, L, H, h, col0, tid);
@@ -401,7 +405,7 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * kt[e];
-        tc::st_chunk(sb + Lay::KV_T + tc::tile_offset(64, r, jc), t);
+        tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, r, jc), t);
 #pragma unroll
         for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * kt[e];
         tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, 64 + r, jc), t);
@@ -425,6 +429,14 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
         tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::GA, 128, s2), tc::desc_kmajor(sb + Lay::GB, 96, s2),
                      id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
+      // The state product needs only prep's output and S0: [Ktilde; Qtilde] S0 -> acc1.
+      // It completes on its own barrier, while the Gram rows are read and inverted.
+      constexpr uint32_t id1 = tc::idesc_bf16(128, DVS, 0, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::WQ_T, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::S_T, 128, s2), id1, s2 > 0);
+      tc::mma_commit(sb + Lay::SBAR);
     }
     if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
     phase ^= 1;
@@ -463,8 +475,9 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     // ---------------- UT transform: X = (I + M)^-1, blockwise on 16x16 blocks ----------------
     // Diagonal blocks: warp b inverts block b by a column sweep; lane = (column c,
     // half hf) holds rows 8hf..8hf+7 of column c; row s is broadcast by shuffle.
-    if (warp < 4) {
-      const int o = 16 * warp, c = lane & 15, hf = lane >> 4;
+    if (qd >= 2) {   // warps 2, 3, 6, 7 invert the diagonal blocks 0, 1, 2, 3
+      const int blk = (qd - 2) + 2 * hw;
+      const int o = 16 * blk, c = lane & 15, hf = lane >> 4;
       float x[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) x[i] = (8 * hf + i == c) ? 1.f : 0.f;
@@ -480,11 +493,38 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
       }
 #pragma unroll
       for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * kLd + o + c] = x[i];
-      if ((warp & 1) == 0)   // block above the diagonal inside the 32-row half
+      if ((blk & 1) == 0)   // block above the diagonal inside the 32-row half
 #pragma unroll
         for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * kLd + o + 16 + c] = 0.f;
     }
-    __syncthreads();
+    // Meanwhile warps 0, 1, 4, 5 (TMEM lanes 0..63) form X = V - Ktilde S0 for tokens
+    // 0..63 from the state product and write it as the bf16 operand of U = T X.
+    bool s_late = false;
+    if (qd < 2) {
+      s_late = !wait_timed(sbar, sphase, wait_ns);
+      tc::fence_after_sync();
+      const int r = 32 * qd + lane;
+#pragma unroll
+      for (int col = hw * NCOL; col < hw * NCOL + NCOL; col += 32) {
+        float a[32];
+        tc::tmem_ld32(tl + 256 + col, a);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint4 vv = *reinterpret_cast<const uint4 *>(
+              sp + Lay::KV_T + tc::tile_offset(64, r, 16 + (col >> 3) + cc));
+          float xv[8];
+          unpack8(vv, xv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xv[e] -= a[8 * cc + e];
+          tc::st_chunk(sb + Lay::U_T + tc::tile_offset(64, r, (col >> 3) + cc), xv);
+        }
+      }
+      tc::fence_smem_to_async();
+      tc::fence_before_sync();
+    }
+    if (__syncthreads_or(s_late)) { aborted = true; break; }
+    sphase ^= 1;
     // Level 1: the 32x32 inverse of each half, X_(2h+1,2h) = -X_(2h+1,2h+1) M_(2h+1,2h) X_(2h,2h).
     {
       const int hh = tid >> 7, rr = (tid >> 3) & 15, c0 = (tid & 7) * 2;
@@ -548,68 +588,38 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     tc::fence_smem_to_async();
     __syncthreads();
 
-    // ---------------- WY products: [T;P] x [Ktilde | V] ----------------
-    if (tid == 0) {
-      tc::fence_after_sync();
-      constexpr uint32_t id = tc::idesc_bf16(128, 128 + DVS, 0, 1);
-#pragma unroll
-      for (int s = 0; s < 4; ++s)
-        tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::TP_T, 128, s),
-                     tc::desc_mnmajor(sb + Lay::KV_T, 64, s), id, s > 0);
-      tc::mma_commit(sb + Lay::BAR);
-    }
-    if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
-    phase ^= 1;
-    tc::fence_after_sync();
+    // Prefetch the next chunk: the staging area and the V slot are free now.
     const int64_t done_next = done + L;
     int p_next = pi;
     while (p_next < pe && positions[p_next] <= done_next) ++p_next;
     const int L_next = done_next < T_seq ? chunk_len(done_next, p_next) : 0;
     if (done_next < T_seq)
       prefetch_chunk<DVS>(sb, maps, beta, t_begin + done_next, L_next, H, h, col0, tid);
-    if (qd < 2) {   // What rows 0..63 -> bf16 operand rows 0..63 of [What; Qtilde]
-      const int r = 32 * qd + lane;
-      float a[32];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        tc::tmem_ld32(tl + 64 * hw + 32 * u, a);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, r, 8 * hw + 4 * u + cc), a + 8 * cc);
-      }
-    }
-    tc::fence_smem_to_async();
-    tc::fence_before_sync();
-    __syncthreads();
 
-    // ---------------- MMA1: [What; Qtilde] x S0 ----------------
+    // ---------------- U = T X (rows 0..63 of [T; P] X) ----------------
     if (tid == 0) {
       tc::fence_after_sync();
       constexpr uint32_t id = tc::idesc_bf16(128, DVS, 0, 1);
 #pragma unroll
-      for (int s = 0; s < 8; ++s)
-        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::WQ_T, 128, s),
-                     tc::desc_mnmajor(sb + Lay::S_T, 128, s), id, s > 0);
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::TP_T, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::U_T, 64, s2), id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
     if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
     phase ^= 1;
     tc::fence_after_sync();
-    if (qd < 2) {   // U = Utilde - What S0 -> bf16 operand
+    if (qd < 2) {   // U -> bf16 operand (replaces X, which the MMA has consumed)
       const int r = 32 * qd + lane;
-      float a[32], b[32];
+      float a[32];
 #pragma unroll
       for (int u = 0; u < NCOL / 32; ++u) {
         const int col = hw * NCOL + 32 * u;
-        tc::tmem_ld32(tl + 256 + col, a);
-        tc::tmem_ld32(tl + 128 + col, b);
+        tc::tmem_ld32(tl + col, a);
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) b[i] -= a[i];
-#pragma unroll
         for (int cc = 0; cc < 4; ++cc)
-          tc::st_chunk(sb + Lay::U_T + tc::tile_offset(64, r, (col >> 3) + cc), b + 8 * cc);
+          tc::st_chunk(sb + Lay::U_T + tc::tile_offset(64, r, (col >> 3) + cc), a + 8 * cc);
       }
     }
     tc::fence_smem_to_async();
@@ -681,6 +691,7 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     // Give the tensor core and the copy engine a last bounded chance to finish
     // what they were given before the CTA releases its memory.
     wait_timed(bar, phase, wait_ns);
+    wait_timed(sbar, sphase, wait_ns);
     wait_timed(tbar, tphase, wait_ns);
   } else {
     while (pi < pe) store_state(pos_states, pi++);   // positions past the end: final state
