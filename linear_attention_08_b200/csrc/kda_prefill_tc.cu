@@ -77,6 +77,7 @@ struct Layout {
   static constexpr uint32_t XM = G + 17408;                       //  float [64][68] (I + M)^-1
   static constexpr uint32_t YS = G + 34816;                       //  float [2][16][17]
   static constexpr uint32_t ZS = G + 36992;                       //  float [32][36]
+  static constexpr uint32_t MT = G + 41600;                       //  float [32][33] M_(1,0)^T
   static constexpr uint32_t SMALL = G + 73728;
   static constexpr uint32_t BETA = SMALL;                         // float [64]
   static constexpr uint32_t DVEC = SMALL + 256;                   // float [128]
@@ -86,7 +87,7 @@ struct Layout {
   static constexpr uint32_t SBAR = BAR + 16;                      // mbarrier: state product done
   static constexpr uint32_t TMEM_SLOT = BAR + 24;
   static constexpr uint32_t TOTAL = BAR + 64;
-  static_assert(ZS + 32 * 36 * 4 <= G + 65536, "solve scratch overflows");
+  static_assert(MT + 32 * 33 * 4 <= G + 65536, "solve scratch overflows");
   static_assert(64 * DVS * 2 <= 16384, "U must fit the Ktilde slot");
 };
 
@@ -158,9 +159,10 @@ __device__ __forceinline__ void prefetch_chunk(uint32_t sb, const TmaMaps &maps,
     for (int j = 0; j < DVS / 64; ++j)
       tma_load_3d(sb + Lay::KV_T + (2 + j) * 8192, &maps.v, col0 + 64 * j, h, z, bar);
   }
-  if (tid < kC) {
-    const bool ok = tid < L;
-    cp_async4(sb + Lay::BETA + 4 * tid, beta + (ok ? (size_t)(t0 + tid) * H + h : 0), ok);
+  if (tid >= 64 && tid < 64 + kC) {   // warps 2-3: thread 0 is left free for the MMAs
+    const int r = tid - 64;
+    const bool ok = r < L;
+    cp_async4(sb + Lay::BETA + 4 * r, beta + (ok ? (size_t)(t0 + r) * H + h : 0), ok);
   }
   cp_async_commit();
 }
@@ -196,6 +198,7 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   float *s_X = reinterpret_cast<float *>(sp + Lay::XM);
   float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
   float *s_Z = reinterpret_cast<float *>(sp + Lay::ZS);
+  float *s_MT = reinterpret_cast<float *>(sp + Lay::MT);
   uint64_t *bar = reinterpret_cast<uint64_t *>(sp + Lay::BAR);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -386,8 +389,9 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
           float r0 = __int_as_float(0x7EF311C3 - __float_as_int(x[e]));
           r0 = r0 * fmaf(-x[e], r0, 2.f);
           y[e] = r0 * fmaf(-x[e], r0, 2.f);
-          kt[e] = (x[e] * fk[e]) * fk2[e];          // exp(Gam_r)
-          kh[e] = (y[e] * fh[e]) * fh2[e];          // exp(Gam_63 - Gam_r)
+          // exp(Gam_r) and exp(Gam_63 - Gam_r); fk = 1 in the first half, fh2 = 1 in the second
+          kt[e] = hf ? (x[e] * fk[e]) * fk2[e] : x[e] * fk2[e];
+          kh[e] = hf ? y[e] * fh[e] : (y[e] * fh[e]) * fh2[e];
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * x[e];
@@ -461,6 +465,9 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
         float *dst = s_M + r * kLd + i0;
 #pragma unroll
         for (int j = 0; j < 32; ++j) dst[j] = (!zero && i0 + j < r) ? br * a[j] : 0.f;
+        if (second && i0 == 0)   // the block M_(1,0), also transposed for the solve
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s_MT[j * 33 + (r - 32)] = br * a[j];
       } else {
 #pragma unroll
         for (int j = 0; j < 32; ++j) a[j] = (!zero && i0 + j <= r) ? a[j] : 0.f;
@@ -550,28 +557,30 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
       *reinterpret_cast<float2 *>(s_X + (ro + rr) * kLd + co + c0) = make_float2(-x0, -x1);
       __syncthreads();
     }
-    // Level 2: X_(1,0) = -H1 M_(1,0) H0 on the 32x32 halves (H0, H1 lower triangular).
+    // Level 2: X_(1,0) = -H1 M_(1,0) H0 on the 32x32 halves.  H0 and H1 are lower
+    // triangular, so each warp's trip count skips the zero half of the product.
     {
-      const int rr = tid >> 3, cq = (tid & 7) * 4;
+      // Z = M_(1,0) H0: warp w computes columns 4w..4w+3, lane = row; H0[s][c] = 0 for s < c.
+      const int rr = lane, cq = 4 * warp;
       float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-      for (int s2 = 0; s2 < 32; ++s2) {
-        const float m = s_M[(32 + rr) * kLd + s2];
+      for (int s2 = cq; s2 < 32; ++s2) {
+        const float m = s_MT[s2 * 33 + rr];
         const float4 xv = *reinterpret_cast<const float4 *>(s_X + s2 * kLd + cq);
         z.x = fmaf(m, xv.x, z.x); z.y = fmaf(m, xv.y, z.y);
         z.z = fmaf(m, xv.z, z.z); z.w = fmaf(m, xv.w, z.w);
       }
       *reinterpret_cast<float4 *>(s_Z + rr * 36 + cq) = z;
       __syncthreads();
+      // X_(1,0) = -H1 Z: warp w computes rows 4w..4w+3; H1[r][s] = 0 for s > r.
+      const int r2 = 4 * warp + (lane >> 3), c2 = 4 * (lane & 7);
       float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-      for (int s2 = 0; s2 < 32; ++s2) {
-        const float a = s_X[(32 + rr) * kLd + 32 + s2];
-        const float4 zv = *reinterpret_cast<const float4 *>(s_Z + s2 * 36 + cq);
+      for (int s2 = 0; s2 < 4 * warp + 4; ++s2) {
+        const float a = s_X[(32 + r2) * kLd + 32 + s2];
+        const float4 zv = *reinterpret_cast<const float4 *>(s_Z + s2 * 36 + c2);
         w.x = fmaf(a, zv.x, w.x); w.y = fmaf(a, zv.y, w.y);
         w.z = fmaf(a, zv.z, w.z); w.w = fmaf(a, zv.w, w.w);
       }
-      *reinterpret_cast<float4 *>(s_X + (32 + rr) * kLd + cq) = make_float4(-w.x, -w.y, -w.z, -w.w);
+      *reinterpret_cast<float4 *>(s_X + (32 + r2) * kLd + c2) = make_float4(-w.x, -w.y, -w.z, -w.w);
       __syncthreads();
     }
     // T rows of the [T; P] operand: T_ri = X_ri beta_i (i <= r).
