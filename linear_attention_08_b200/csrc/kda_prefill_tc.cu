@@ -222,17 +222,25 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
   const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);   // this warp's lane base
 
-  // FP32 state slice in registers: row crow, columns [hw*NCOL, hw*NCOL + NCOL).
-  float S[NCOL];
+  // The FP32 state slice lives in tensor memory, columns [128, 128 + DVS): lane c holds
+  // state row c.  This thread owns row crow, columns [hw*NCOL, hw*NCOL + NCOL).
+  const uint32_t s_tm = tl + 128 + hw * NCOL;
   const size_t soff = ((size_t)unit * kDK + crow) * kDV + col0 + hw * NCOL;
 #pragma unroll
-  for (int j = 0; j < NCOL; j += 4) {
-    float4 x = init ? *reinterpret_cast<const float4 *>(init + soff + j) : make_float4(0, 0, 0, 0);
-    S[j] = x.x; S[j + 1] = x.y; S[j + 2] = x.z; S[j + 3] = x.w;
-  }
+  for (int u = 0; u < NCOL / 32; ++u) {
+    float x[32];
 #pragma unroll
-  for (int j = 0; j < NCOL; j += 8)
-    tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + j) >> 3), S + j);
+    for (int j = 0; j < 32; j += 4) {
+      const float4 v4 = init ? *reinterpret_cast<const float4 *>(init + soff + 32 * u + j)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[j] = v4.x; x[j + 1] = v4.y; x[j + 2] = v4.z; x[j + 3] = v4.w;
+    }
+    tc::tmem_st32(s_tm + 32 * u, x);
+#pragma unroll
+    for (int j = 0; j < 32; j += 8)
+      tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + 32 * u + j) >> 3), x + j);
+  }
+  tc::tmem_wait_st();
 
   const int64_t t_begin = cu[seq], t_end = cu[seq + 1], T_seq = t_end - t_begin;
   int64_t ck_slot = 0;
@@ -241,20 +249,28 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   // Explicit state positions of this sequence (token counts), if any.
   int pi = positions ? pos_cu[seq] : 0;
   const int pe = positions ? pos_cu[seq + 1] : 0;
-  // Store the FP32 state slice of this thread into a [.., H, D_k, D_v] array.
+  // Store the FP32 state slice of this thread (read back from tensor memory) into
+  // a [.., H, D_k, D_v] array.
   auto store_state = [&](float *base_ptr, int64_t slot) {
     float *dst = base_ptr + ((size_t)slot * H + h) * kDK * kDV + (size_t)crow * kDV + col0 + hw * NCOL;
 #pragma unroll
-    for (int j = 0; j < NCOL; j += 4)
-      *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
+    for (int u = 0; u < NCOL / 32; ++u) {
+      float x[32];
+      tc::tmem_ld32(s_tm + 32 * u, x);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4 *>(dst + 32 * u + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+    }
   };
   // Length of the chunk that starts after `done` tokens: at most 64, and it ends
   // at the next checkpoint boundary or explicit position (chunking does not
   // change the result, so every stored state is the state at a chunk end).
-  auto chunk_len = [&](int64_t done, int p) -> int {
+  // since_ck = done % interval is tracked incrementally (no 64-bit division in the loop).
+  auto chunk_len = [&](int64_t done, int64_t since_ck, int p) -> int {
     int64_t m = T_seq - done < kC ? T_seq - done : kC;
     if (interval > 0) {
-      const int64_t to_ck = interval - done % interval;
+      const int64_t to_ck = interval - since_ck;
       m = to_ck < m ? to_ck : m;
     }
     if (p < pe) {
@@ -269,8 +285,8 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   bool aborted = false;
   uint64_t *tbar = reinterpret_cast<uint64_t *>(sp + Lay::TBAR);
   uint64_t *sbar = reinterpret_cast<uint64_t *>(sp + Lay::SBAR);
-  int64_t done = 0;
-  int L = T_seq > 0 ? chunk_len(0, pi) : 0;
+  int64_t done = 0, since_ck = 0;
+  int L = T_seq > 0 ? chunk_len(0, 0, pi) : 0;
   if (T_seq > 0) prefetch_chunk<DVS>(sb, maps, beta, t_begin, L, H, h, col0, tid);
 
   while (done < T_seq) {
@@ -601,7 +617,9 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     const int64_t done_next = done + L;
     int p_next = pi;
     while (p_next < pe && positions[p_next] <= done_next) ++p_next;
-    const int L_next = done_next < T_seq ? chunk_len(done_next, p_next) : 0;
+    int64_t since_next = since_ck + L;
+    if (since_next == interval) since_next = 0;
+    const int L_next = done_next < T_seq ? chunk_len(done_next, since_next, p_next) : 0;
     if (done_next < T_seq)
       prefetch_chunk<DVS>(sb, maps, beta, t_begin + done_next, L_next, H, h, col0, tid);
 
@@ -676,16 +694,24 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
       const float d = s_dvec[crow];
 #pragma unroll
       for (int u = 0; u < NCOL / 32; ++u) {
-        tc::tmem_ld32(tl + 256 + DVS + hw * NCOL + 32 * u, a);
+        float sv[32];
+        tc::tmem_ld32(tl + 256 + DVS + hw * NCOL + 32 * u, a);   // state increment
+        tc::tmem_ld32(s_tm + 32 * u, sv);                          // state
         tc::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) S[32 * u + i] = fmaf(d, S[32 * u + i], a[i]);
-      }
+        for (int i = 0; i < 32; ++i) sv[i] = fmaf(d, sv[i], a[i]);
+        tc::tmem_st32(s_tm + 32 * u, sv);
 #pragma unroll
-      for (int j = 0; j < NCOL; j += 8)
-        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + j) >> 3), S + j);
+        for (int j = 0; j < 32; j += 8)
+          tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + 32 * u + j) >> 3), sv + j);
+      }
+      tc::tmem_wait_st();
       done += L;
-      if (interval > 0 && done % interval == 0) store_state(ck, ck_slot++);
+      since_ck += L;
+      if (interval > 0 && since_ck == interval) {
+        store_state(ck, ck_slot++);
+        since_ck = 0;
+      }
       while (pi < pe && positions[pi] <= done) store_state(pos_states, pi++);
       L = L_next;
     }
@@ -704,12 +730,7 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     wait_timed(tbar, tphase, wait_ns);
   } else {
     while (pi < pe) store_state(pos_states, pi++);   // positions past the end: final state
-    if (fin) {
-      float *dst = fin + soff;
-#pragma unroll
-      for (int j = 0; j < NCOL; j += 4)
-        *reinterpret_cast<float4 *>(dst + j) = make_float4(S[j], S[j + 1], S[j + 2], S[j + 3]);
-    }
+    if (fin) store_state(fin, seq);
   }
   tc::fence_before_sync();
   __syncthreads();
