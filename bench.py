@@ -80,9 +80,12 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "decode": ("kda_decode.cu", "kda_common.cuh"),
-    "prefill_tc": ("kda_prefill_tc.cu", "kda_tc_util.cuh", "kda_common.cuh"),
+    "prefill_tc": ("kda_prefill_tc.cu", "kda_tc_util.cuh", "kda_tma.cuh", "kda_common.cuh"),
+    # two-pass path: intra-chunk pass + chain pass, one prefill call = one launch of each
+    "prefill_split": ("kda_prefill_split.cu", "kda_tc_util.cuh", "kda_tma.cuh", "kda_common.cuh"),
     "prefill_simt": ("kda_prefill_simt.cu", "kda_common.cuh"),
 }
+PATH_KERNEL = {2: "prefill_split", 1: "prefill_tc", 0: "prefill_simt"}
 
 
 def kernel_source_sha(kernel: str) -> str:
@@ -284,7 +287,7 @@ def time_prefill(name, steps, warmup, world, local):
                                                1 if w["dtype"] == "bf16" else 0))
     return dict(tokens=tokens, steps=steps, total_ms=total_ms, launch_ms=launch_ms,
                 e2e_ms=e2e_ms, bi=bi, bo=bo, flops=flops, bytes=byts, clocks=clk.result,
-                kernel="prefill_tc" if path == 1 else "prefill_simt", w=w, lengths=lengths)
+                kernel=PATH_KERNEL[path], w=w, lengths=lengths)
 
 
 def time_decode(steps_graph, warmup, world, local, decode_steps=None):

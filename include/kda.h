@@ -95,6 +95,26 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
                        float *ckpt_states, const kda_shape *shape, kda_stream_t stream);
 
 /*
+ * kda_prefill with a caller-owned device workspace.  Shapes on the two-pass
+ * tensor-core path (kda_prefill_path = 2) store one packet of intra-chunk
+ * products per (chunk, head) in the workspace, then run the inter-chunk
+ * chain over them.  workspace_bytes >= kda_prefill_workspace_bytes(shape)
+ * runs the whole batch in one window; a smaller workspace (at least
+ * kda_prefill_workspace_min_bytes) runs it in several windows of chunks.
+ * A NULL or too small workspace, or a shape off the two-pass path, runs the
+ * single-pass kernels, which need none.  The workspace must be 16-byte
+ * aligned (256 is best), must not overlap any argument, and is free again
+ * when the work queued on `stream` completes.  kda_prefill itself takes its
+ * workspace from a memory pool the library keeps per device (released by
+ * kda_release_workspace_pool).
+ */
+kda_status kda_prefill_ws(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                          void *out, float *final_state, int64_t ckpt_interval,
+                          float *ckpt_states, void *workspace, size_t workspace_bytes,
+                          const kda_shape *shape, kda_stream_t stream);
+
+/*
  * kda_prefill with states also stored at explicit positions, such as the
  * boundaries of cached prompts (the first page, Conclusion table: prefix
  * caching keeps the state every 32K tokens "+ prompt boundaries").
@@ -157,14 +177,24 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const f
  * (0 when ckpt_interval <= 0; -1 on a bad argument). */
 int64_t kda_ckpt_count(const int32_t *host_cu_seqlens, int32_t num_seqs, int64_t ckpt_interval);
 
-/* Bytes of device scratch kda_prefill needs for this shape beyond its
- * arguments.  The prefill kernels in this build carry the state on chip and
- * need none, so this is 0 for every valid shape and (size_t)-1 for an
- * invalid one. */
+/* Workspace that lets kda_prefill_ws run this shape in a single window:
+ * 74240 bytes per (chunk, head) packet for an upper bound of the chunk count
+ * (every sequence may end in a partial chunk), plus one FP32 state per
+ * (sequence, head) for the case without final_state.  0 for shapes off the
+ * two-pass path, (size_t)-1 for an invalid shape. */
 size_t kda_prefill_workspace_bytes(const kda_shape *shape);
 
-/* Which prefill kernel a shape runs on: 1 = tcgen05 tensor-core kernel,
- * 0 = SIMT FP32 kernel, -1 = invalid shape. */
+/* Smallest workspace the two-pass path accepts (windows of one chunk);
+ * 0 off that path, (size_t)-1 for an invalid shape. */
+size_t kda_prefill_workspace_min_bytes(const kda_shape *shape);
+
+/* Frees the memory cached by the library's per-device workspace pools. */
+kda_status kda_release_workspace_pool(void);
+
+/* Which prefill kernel a shape runs on without explicit positions:
+ * 2 = two-pass tcgen05 tensor-core kernels (intra-chunk pass + chain),
+ * 1 = single-pass tcgen05 kernel (also used with explicit positions and
+ *     without a workspace), 0 = SIMT FP32 kernel, -1 = invalid shape. */
 int kda_prefill_path(const kda_shape *shape);
 
 /* Bounded-wait self-test: launches one CTA that waits on an mbarrier that

@@ -2,6 +2,8 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "kda_common.cuh"
 
 namespace kda {
@@ -26,7 +28,61 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                               int N, int H, int64_t total_tokens, int32_t *dev_status,
                               cudaStream_t stream);
 
+bool prefill_split_supported(int N);
+size_t split_packet_bytes();
+size_t split_workspace_full(int N, int H, int64_t T, bool have_final);
+cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *init, const int32_t *cu, void *out,
+                                 float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
+                                 void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 cudaStream_t stream, int num_sms);
+
 static thread_local int g_last_cuda_error = 0;
+
+// Largest workspace kda_prefill takes from its pool (longer inputs run in windows).
+static const size_t kPoolCap = (size_t)8 << 30;
+static const int kMaxDevices = 64;
+static std::mutex g_pool_mu;
+static cudaMemPool_t g_pools[kMaxDevices];
+static int g_num_sms[kMaxDevices];
+
+static cudaError_t device_pool(int dev, cudaMemPool_t *out) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_pool_mu);
+  if (!g_pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaError_t e = cudaMemPoolCreate(&g_pools[dev], &props);
+    if (e != cudaSuccess) { g_pools[dev] = nullptr; return e; }
+    uint64_t keep = UINT64_MAX;   // keep freed blocks for the next call
+    cudaMemPoolSetAttribute(g_pools[dev], cudaMemPoolAttrReleaseThreshold, &keep);
+  }
+  *out = g_pools[dev];
+  return cudaSuccess;
+}
+
+static int device_sms(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  if (!g_num_sms[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    g_num_sms[dev] = v;
+  }
+  return g_num_sms[dev];
+}
+
+static bool split_path(const kda_shape *s) {
+  return prefill_tc_supported(s->qkv_dtype, s->head_dim_k, s->head_dim_v, s->chunk) &&
+         prefill_split_supported(s->num_seqs);
+}
+
+static size_t split_min_bytes(const kda_shape *s, bool have_final) {
+  return (size_t)s->num_seqs * s->num_heads * split_packet_bytes() +
+         (have_final ? 0 : (size_t)s->num_seqs * s->num_heads * 128 * 128 * 4) + 256;
+}
 
 static kda_status cuda_status(cudaError_t e) {
   if (e == cudaSuccess) return KDA_OK;
@@ -94,28 +150,43 @@ int64_t kda_ckpt_count(const int32_t *host_cu_seqlens, int32_t num_seqs, int64_t
   return n;
 }
 
-size_t kda_prefill_workspace_bytes(const kda_shape *shape) {
-  return check_shape(shape, true) == KDA_OK ? 0 : (size_t)-1;
+size_t kda_prefill_workspace_bytes(const kda_shape *s) {
+  if (check_shape(s, true) != KDA_OK) return (size_t)-1;
+  if (!split_path(s)) return 0;
+  return split_workspace_full(s->num_seqs, s->num_heads, s->total_tokens, false);
+}
+
+size_t kda_prefill_workspace_min_bytes(const kda_shape *s) {
+  if (check_shape(s, true) != KDA_OK) return (size_t)-1;
+  return split_path(s) ? split_min_bytes(s, false) : 0;
+}
+
+kda_status kda_release_workspace_pool(void) {
+  std::lock_guard<std::mutex> lock(g_pool_mu);
+  for (int d = 0; d < kMaxDevices; ++d)
+    if (g_pools[d]) {
+      cudaError_t e = cudaMemPoolTrimTo(g_pools[d], 0);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+  return KDA_OK;
 }
 
 int kda_prefill_path(const kda_shape *s) {
   if (check_shape(s, true) != KDA_OK) return -1;
+  if (split_path(s)) return 2;
   return prefill_tc_supported(s->qkv_dtype, s->head_dim_k, s->head_dim_v, s->chunk) ? 1 : 0;
 }
 
-kda_status kda_prefill(const void *q, const void *k, const void *v, const float *g,
-                       const float *beta, const float *init_state, const int32_t *cu_seqlens,
-                       void *out, float *final_state, int64_t ckpt_interval,
-                       float *ckpt_states, const kda_shape *s, kda_stream_t stream) {
-  return kda_prefill_at(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
-                        ckpt_interval, ckpt_states, nullptr, nullptr, nullptr, s, stream);
-}
+// Workspace modes of prefill_impl.
+enum { WS_NONE = 0, WS_CALLER = 1, WS_POOL = 2 };
 
-kda_status kda_prefill_at(const void *q, const void *k, const void *v, const float *g,
-                          const float *beta, const float *init_state, const int32_t *cu_seqlens,
-                          void *out, float *final_state, int64_t ckpt_interval,
-                          float *ckpt_states, const int32_t *pos_cu, const int32_t *positions,
-                          float *pos_states, const kda_shape *s, kda_stream_t stream) {
+static kda_status prefill_impl(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *init_state,
+                               const int32_t *cu_seqlens, void *out, float *final_state,
+                               int64_t ckpt_interval, float *ckpt_states, const int32_t *pos_cu,
+                               const int32_t *positions, float *pos_states, int ws_mode,
+                               void *workspace, size_t ws_bytes, const kda_shape *s,
+                               kda_stream_t stream) {
   kda_status st = check_shape(s, true);
   if (st != KDA_OK) return st;
   const int N = s->num_seqs, H = s->num_heads, DK = s->head_dim_k, DV = s->head_dim_v;
@@ -151,8 +222,44 @@ kda_status kda_prefill_at(const void *q, const void *k, const void *v, const flo
   if (final_state && init_state && final_state != init_state &&
       overlaps(final_state, n_state, init_state, n_state))
     return KDA_ERR_INVALID_ARGUMENT;  // exact aliasing is fine, partial overlap is not
+  if (ws_mode == WS_CALLER && workspace) {
+    if (!aligned16(workspace)) return KDA_ERR_INVALID_ARGUMENT;
+    if (overlaps(workspace, ws_bytes, out, n_out) || overlaps(workspace, ws_bytes, q, n_qk) ||
+        overlaps(workspace, ws_bytes, k, n_qk) || overlaps(workspace, ws_bytes, v, n_v) ||
+        overlaps(workspace, ws_bytes, g, n_g) || overlaps(workspace, ws_bytes, beta, n_b) ||
+        overlaps(workspace, ws_bytes, init_state, n_state) ||
+        overlaps(workspace, ws_bytes, final_state, n_state) ||
+        overlaps(workspace, ws_bytes, ckpt_states, ckpt_states ? 16 : 0))
+      return KDA_ERR_INVALID_ARGUMENT;
+  }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+  if (T > 0 && !positions && ws_mode != WS_NONE && split_path(s)) {
+    // Two-pass path when a large enough workspace is at hand.
+    const size_t need_min = split_min_bytes(s, final_state != nullptr);
+    if (ws_mode == WS_CALLER && workspace && ws_bytes >= need_min)
+      return cuda_status(launch_prefill_split(q, k, v, g, beta, init_state, cu_seqlens, out,
+                                              final_state, ckpt_interval, ckpt_states, N, H, T,
+                                              workspace, ws_bytes, s->dev_status, cs,
+                                              device_sms(dev)));
+    if (ws_mode == WS_POOL) {
+      cudaMemPool_t pool;
+      size_t want = split_workspace_full(N, H, T, final_state != nullptr);
+      if (want > kPoolCap) want = kPoolCap > need_min ? kPoolCap : need_min;
+      void *ws = nullptr;
+      if (device_pool(dev, &pool) == cudaSuccess &&
+          cudaMallocFromPoolAsync(&ws, want, pool, cs) == cudaSuccess) {
+        e = launch_prefill_split(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
+                                 ckpt_interval, ckpt_states, N, H, T, ws, want, s->dev_status, cs,
+                                 device_sms(dev));
+        const cudaError_t f = cudaFreeAsync(ws, cs);
+        return cuda_status(e != cudaSuccess ? e : f);
+      }
+      cudaGetLastError();   // an allocation that failed falls back to the single pass
+    }
+  }
   if (T > 0 && prefill_tc_supported(s->qkv_dtype, DK, DV, s->chunk))
     e = launch_prefill_tc(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
                           ckpt_interval, ckpt_states, pos_cu, positions, pos_states, N, H, T,
@@ -162,6 +269,34 @@ kda_status kda_prefill_at(const void *q, const void *k, const void *v, const flo
                             final_state, ckpt_interval, ckpt_states, pos_cu, positions,
                             pos_states, N, H, cs);
   return cuda_status(e);
+}
+
+kda_status kda_prefill(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                       void *out, float *final_state, int64_t ckpt_interval,
+                       float *ckpt_states, const kda_shape *s, kda_stream_t stream) {
+  return prefill_impl(q, k, v, g, beta, init_state, cu_seqlens, out, final_state, ckpt_interval,
+                      ckpt_states, nullptr, nullptr, nullptr, WS_POOL, nullptr, 0, s, stream);
+}
+
+kda_status kda_prefill_ws(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                          void *out, float *final_state, int64_t ckpt_interval,
+                          float *ckpt_states, void *workspace, size_t workspace_bytes,
+                          const kda_shape *s, kda_stream_t stream) {
+  return prefill_impl(q, k, v, g, beta, init_state, cu_seqlens, out, final_state, ckpt_interval,
+                      ckpt_states, nullptr, nullptr, nullptr, WS_CALLER, workspace,
+                      workspace_bytes, s, stream);
+}
+
+kda_status kda_prefill_at(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                          void *out, float *final_state, int64_t ckpt_interval,
+                          float *ckpt_states, const int32_t *pos_cu, const int32_t *positions,
+                          float *pos_states, const kda_shape *s, kda_stream_t stream) {
+  return prefill_impl(q, k, v, g, beta, init_state, cu_seqlens, out, final_state, ckpt_interval,
+                      ckpt_states, pos_cu, positions, pos_states, positions ? WS_NONE : WS_POOL,
+                      nullptr, 0, s, stream);
 }
 
 kda_status kda_decode(const void *q, const void *k, const void *v, const float *g,

@@ -1,0 +1,980 @@
+// KDA chunked prefill in two passes on the 5th-generation tensor cores (sm_100a).
+//
+// The chunked form ("LLM - Semianalysis, Kimi K3 아키텍처", Methods 1, FlashKDA;
+// "MoonshotAI/Kimi-K3 딥다이브", section 4-1) splits every chunk's work into a
+// part that depends only on the chunk's own inputs and a short part that
+// needs the state entering the chunk.  With Gam_r = sum_{s<=r} g_s and
+// T = (I + M)^-1 diag(beta) as in the fused kernel:
+//
+//   W = T Ktilde,  U = T V                              (state-free)
+//   V_new = U - W S0                                    (per chunk, serial)
+//   O     = Qtilde S0 + P V_new
+//   S     = Diag(exp(Gam_last)) S0 + Khat^T V_new
+//
+// (W S0 = T Ktilde S0, so V_new = T (V - Ktilde S0) is the fused kernel's U.)
+//
+// Pass 1 (intra_kernel) runs every (chunk, head) pair independently: gates,
+// the gated Gram products, the UT transform and the products T Ktilde and
+// T V; it writes one "packet" per pair to a workspace in global memory, its
+// MMA operands already in the 128-byte-swizzled shared-memory tile layout.
+// Two CTAs share an SM, so one's tensor-core and load waits overlap the
+// other's SIMT work.
+//
+// Pass 2 (chain_kernel) walks each (sequence, head, value slice) chunk by
+// chunk.  Per chunk it bulk-copies the packet (double or triple buffered) and
+// runs two tensor-core steps and two epilogues:
+//   [W; Qtilde] S0 -> acc1         V_new = U - (acc1 rows 0..63)
+//   acc1 += [*; P] V_new,  acc2 = Khat^T V_new,  S = d * S + acc2 (FP32, TMEM)
+// The FP32 state lives in tensor memory; its BF16 copy is the MMA operand.
+//
+// Long inputs are processed in windows of chunks so that the workspace stays
+// within the size the caller grants; the state is carried between windows in
+// FP32 through global memory.
+#include <cuda.h>
+
+#include "kda_common.cuh"
+#include "kda_tc_util.cuh"
+#include "kda_tma.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kC = 64;
+constexpr int kDK = 128;
+constexpr int kDV = 128;
+constexpr int kThreads = 256;
+constexpr int kLd = 68;
+constexpr int kMaxSeqs = 1024;   // sequences per call on this path
+
+// One packet: what the chain needs from one (chunk, head).
+struct Packet {
+  static constexpr uint32_t WQ = 0;        // [128][128] bf16 tile: W rows 0..63, Qtilde rows 64..127
+  static constexpr uint32_t KH = 32768;    // [64][128] bf16 tile: Khat (tokens x key channels)
+  static constexpr uint32_t U = 49152;     // [64][128] bf16 tile: U = T V (tokens x value columns)
+  static constexpr uint32_t P = 65536;     // [64][64] bf16 tile: P (lower triangle, diagonal included)
+  static constexpr uint32_t D = 73728;     // float[128]: exp(Gam) at the chunk's last token
+  static constexpr uint32_t BYTES = 74240;
+};
+
+// ---------------------------------------------------------------------------
+// Pass 1: intra-chunk products
+// ---------------------------------------------------------------------------
+struct IntraLayout {
+  // 64 KB region used in turn for: the raw inputs (k and q land by TMA in the
+  // rows of the Gram A tile that their scaled versions replace; g, fp32, in
+  // the upper half); the Gram operands and the gate factors; the solve
+  // scratch and the V tile.
+  static constexpr uint32_t STG_G = 32768;
+  static constexpr uint32_t GA = 0;          // [128][128] Gram A, K-major: k rows 0..63, q rows 64..127
+  static constexpr uint32_t GB = 32768;      // [96][128]  Gram B, K-major
+  static constexpr uint32_t CST = 57344;     // float [2][6][128] gate factors
+  static constexpr uint32_t MM = 0;          // float [64][68] M
+  static constexpr uint32_t XM = 17408;      // float [64][68] (I + M)^-1
+  static constexpr uint32_t YS = 34816;      // float [2][16][17]
+  static constexpr uint32_t ZS = 36992;      // float [32][36]
+  static constexpr uint32_t MT = 41600;      // float [32][33] M_(1,0)^T
+  static constexpr uint32_t VT = 49152;      // [64][128] V tile (MN-major B), loaded after the Gram MMA
+  static constexpr uint32_t KT = 65536;      // [64][128] Ktilde tile (MN-major B)
+  static constexpr uint32_t TP = 81920;      // [128][64] T (rows 0..63) as K-major A
+  static constexpr uint32_t RED = TP;        // float [16][128] scan partials (before T exists)
+  static constexpr uint32_t BETA = 98304;    // float [64]
+  static constexpr uint32_t PREF = BETA + 256;                    // int [kMaxSeqs + 1]
+  static constexpr uint32_t BAR = (PREF + 4 * (kMaxSeqs + 1) + 7) & ~7u;   // MMA completion
+  static constexpr uint32_t TBAR = BAR + 8;                       // q, k, g landed
+  static constexpr uint32_t VBAR = BAR + 16;                      // v landed
+  static constexpr uint32_t TMEM_SLOT = BAR + 24;
+  static constexpr uint32_t TOTAL = BAR + 32;
+  static_assert(MT + 32 * 33 * 4 <= VT, "solve scratch overlaps the V tile");
+  static_assert(CST + 6144 <= 65536, "gate factors overflow the staging region");
+  static_assert(GB + 96 * 256 <= CST, "Gram B overlaps the gate factors");
+};
+
+// 16-byte store of 8 floats as bf16 into global memory.
+__device__ __forceinline__ void st_global_chunk(uint8_t *dst, const float *x) {
+  *reinterpret_cast<uint4 *>(dst) = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                                               tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+}
+
+// Chunks of sequence n that fall in the window [jw0, jw0 + wc).
+__device__ __forceinline__ int64_t window_chunks(const int32_t *cu, int n, int64_t jw0, int64_t wc) {
+  const int64_t nch = ((int64_t)cu[n + 1] - cu[n] + kC - 1) / kC;
+  const int64_t c = nch - jw0;
+  return c <= 0 ? 0 : (c < wc ? c : wc);
+}
+
+// q and k come through maps with the v layout (box 64 x 64, 128-byte swizzle):
+// each box is one 64-row column block, i.e. rows 0..63 (k) or 64..127 (q) of a
+// column block of the Gram A tile.
+__device__ __forceinline__ void intra_issue_loads(uint32_t sb, const TmaMaps &maps,
+                                                  const float *beta, int64_t t0, int L, int H,
+                                                  int h, int tid) {
+  using Lay = IntraLayout;
+  if (tid == 32) {
+    const uint32_t bar = sb + Lay::TBAR;
+    mbar_expect_tx(bar, 64 * (256 + 256 + 512));
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h, (int)t0, bar);
+      tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h, (int)t0, bar);
+    }
+    tma_load_3d(sb + Lay::STG_G, &maps.g, 0, h, (int)t0, bar);
+  }
+  if (tid >= 64 && tid < 64 + kC) {
+    const int r = tid - 64;
+    const bool ok = r < L;
+    cp_async4(sb + Lay::BETA + 4 * r, beta + (ok ? (size_t)(t0 + r) * H + h : 0), ok);
+  }
+  cp_async_commit();
+}
+
+// Work item p of the window -> (sequence, head, chunk); see the packet order
+// in launch_prefill_split.
+struct Item {
+  int n, h, L;
+  int64_t j, t0;
+};
+
+__device__ __forceinline__ Item decode_item(int p, const int32_t *s_pref, const int32_t *cu, int N,
+                                            int H, int64_t jw0) {
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {   // last sequence whose first packet is at or before p
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_pref[mid] <= p) lo = mid; else hi = mid - 1;
+  }
+  Item it;
+  it.n = lo;
+  const int cnt = (s_pref[lo + 1] - s_pref[lo]) / H;
+  const int r = p - s_pref[lo];
+  it.h = r / cnt;
+  it.j = jw0 + (r - it.h * cnt);
+  const int64_t T_n = (int64_t)cu[lo + 1] - cu[lo];
+  it.t0 = cu[lo] + kC * it.j;
+  const int64_t rem = T_n - kC * it.j;
+  it.L = (int)(rem < kC ? rem : kC);
+  return it;
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ beta,
+             const int32_t *__restrict__ cu, int N, int H, int64_t jw0, int64_t wc,
+             uint8_t *__restrict__ ws, int32_t *dev_status, uint64_t wait_ns) {
+  using Lay = IntraLayout;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sb = (sraw + 1023u) & ~1023u;
+  uint8_t *sp = smem_raw + (sb - sraw);
+  float *s_beta = reinterpret_cast<float *>(sp + Lay::BETA);
+  float *s_red = reinterpret_cast<float *>(sp + Lay::RED);
+  float *s_cst = reinterpret_cast<float *>(sp + Lay::CST);
+  float *s_M = reinterpret_cast<float *>(sp + Lay::MM);
+  float *s_X = reinterpret_cast<float *>(sp + Lay::XM);
+  float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
+  float *s_Z = reinterpret_cast<float *>(sp + Lay::ZS);
+  float *s_MT = reinterpret_cast<float *>(sp + Lay::MT);
+  int32_t *s_pref = reinterpret_cast<int32_t *>(sp + Lay::PREF);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sp + Lay::BAR);
+  uint64_t *tbar = reinterpret_cast<uint64_t *>(sp + Lay::TBAR);
+  uint64_t *vbar = reinterpret_cast<uint64_t *>(sp + Lay::VBAR);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hw = warp >> 2;
+
+  // Packets of the window, sequence by sequence: s_pref[n] = first packet of n.
+  for (int n = tid; n < N; n += kThreads) s_pref[n + 1] = (int32_t)(window_chunks(cu, n, jw0, wc) * H);
+  if (tid == 0) s_pref[0] = 0;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t carry = 0;
+    for (int base = 1; base <= N; base += 32) {
+      const int i = base + lane;
+      int32_t v = i <= N ? s_pref[i] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+      }
+      if (i <= N) s_pref[i] = v + carry;
+      carry += __shfl_sync(0xffffffffu, v, 31);
+    }
+  }
+  __syncthreads();
+  const int total = s_pref[N];
+  if ((int)blockIdx.x >= total) return;
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(tbar, 1);
+    mbar_init(vbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.g)) : "memory");
+  }
+  if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, 256);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
+  const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+
+  uint32_t phase = 0, tphase = 0, vphase = 0;
+  bool aborted = false;
+  int p = blockIdx.x;
+  {
+    const Item it = decode_item(p, s_pref, cu, N, H, jw0);
+    intra_issue_loads(sb, maps, beta, it.t0, it.L, H, it.h, tid);
+  }
+
+  for (; p < total; p += gridDim.x) {
+    const Item it = decode_item(p, s_pref, cu, N, H, jw0);
+    const int L = it.L, h = it.h;
+    uint8_t *pk = ws + (size_t)p * Packet::BYTES;
+
+    cp_async_wait_all();
+    if (__syncthreads_or(!wait_timed(tbar, tphase, wait_ns))) { aborted = true; break; }
+    tphase ^= 1;
+
+    // ---------------- gate prep (as in the fused kernel) ----------------
+    // Thread (rg, jc) owns rows 4rg..4rg+3 and channels 8jc..8jc+7.
+    {
+      const int rg = tid >> 4, jc = tid & 15, hf = rg >> 3;
+      float gm[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * rg + i;
+        const bool in = r < L;
+        const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 a = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + jc * 32) : zf;
+        const float4 b = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + jc * 32 + 16) : zf;
+        gm[i][0] = a.x; gm[i][1] = a.y; gm[i][2] = a.z; gm[i][3] = a.w;
+        gm[i][4] = b.x; gm[i][5] = b.y; gm[i][6] = b.z; gm[i][7] = b.w;
+      }
+#pragma unroll
+      for (int i = 1; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gm[i][e] += gm[i - 1][e];
+      {
+        float4 *dst = reinterpret_cast<float4 *>(s_red + rg * 128 + 8 * jc);
+        dst[0] = make_float4(gm[3][0], gm[3][1], gm[3][2], gm[3][3]);
+        dst[1] = make_float4(gm[3][4], gm[3][5], gm[3][6], gm[3][7]);
+      }
+      __syncthreads();
+      // Exclusive scan of the 16 row-group totals per channel (warp w: channels
+      // 16w..16w+15; lane (ch, half) holds row groups 8 half .. 8 half + 7), and the
+      // per-channel gate factors, formed once.
+      {
+        const int ch = 16 * warp + (lane & 15), half = lane >> 4;
+        float t[8], run = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) t[i] = s_red[(8 * half + i) * 128 + ch];
+        float incl[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { run += t[i]; incl[i] = run; }
+        const float lower = __shfl_sync(0xffffffffu, run, lane & 15);
+        const float off = half ? lower : 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s_red[(8 * half + i) * 128 + ch] = off + incl[i] - t[i];
+        const float ga = off + incl[3], gb = off + incl[7];
+        const float G15 = __shfl_sync(0xffffffffu, ga, lane & 15);
+        const float G31 = __shfl_sync(0xffffffffu, gb, lane & 15);
+        const float G47 = __shfl_sync(0xffffffffu, ga, (lane & 15) + 16);
+        const float G63 = __shfl_sync(0xffffffffu, gb, (lane & 15) + 16);
+        // Row r of half hf is scaled against ref = Gam_15 (hf 0) or Gam_47 (hf 1);
+        // the products are grouped exactly as in the fused kernel (no intermediate
+        // underflows unless the exact value is itself far below the BF16 rounding).
+        float f[6];
+        if (half == 0) {
+          f[0] = G15; f[1] = 1.f; f[2] = __expf(G15);
+          f[3] = __expf(G31 - G15); f[4] = __expf(G63 - G31); f[5] = __expf(G47 - G15);
+        } else {
+          f[0] = G47; f[1] = __expf(G47 - G31); f[2] = __expf(G31);
+          f[3] = __expf(G63 - G47); f[4] = 1.f; f[5] = 0.f;
+          reinterpret_cast<float *>(pk + Packet::D)[ch] = __expf(G63);
+        }
+#pragma unroll
+        for (int j = 0; j < 6; ++j) s_cst[(half * 6 + j) * 128 + ch] = f[j];
+      }
+      __syncthreads();
+      auto ld8 = [&](const float *src, float *d8) {
+        const float4 a = reinterpret_cast<const float4 *>(src)[0];
+        const float4 b = reinterpret_cast<const float4 *>(src)[1];
+        d8[0] = a.x; d8[1] = a.y; d8[2] = a.z; d8[3] = a.w;
+        d8[4] = b.x; d8[5] = b.y; d8[6] = b.z; d8[7] = b.w;
+      };
+      {
+        float base[8];
+        ld8(s_red + rg * 128 + 8 * jc, base);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) gm[i][e] += base[e];
+      }
+      const float *c = s_cst + hf * 6 * 128 + 8 * jc;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = 4 * rg + i;
+        float ref[8], kk[8], qq[8], x[8], y[8], t[8];
+        ld8(c, ref);
+        {   // raw k and q of this row and channel group, replaced below by k x and q x
+          const uint4 z4 = make_uint4(0, 0, 0, 0);
+          const bool in = r < L;
+          const uint4 kv = in ? *reinterpret_cast<const uint4 *>(sp + Lay::GA + tc::tile_offset(128, r, jc)) : z4;
+          const uint4 qv = in ? *reinterpret_cast<const uint4 *>(sp + Lay::GA + tc::tile_offset(128, 64 + r, jc)) : z4;
+          unpack8(kv, kk);
+          unpack8(qv, qq);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          x[e] = __expf(gm[i][e] - ref[e]);
+          float r0 = __int_as_float(0x7EF311C3 - __float_as_int(x[e]));
+          r0 = r0 * fmaf(-x[e], r0, 2.f);
+          y[e] = r0 * fmaf(-x[e], r0, 2.f);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = kk[e] * x[e];
+        tc::st_chunk(sb + Lay::GA + tc::tile_offset(128, r, jc), t);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = qq[e] * x[e];
+        tc::st_chunk(sb + Lay::GA + tc::tile_offset(128, 64 + r, jc), t);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = kk[e] * y[e];
+        tc::st_chunk(sb + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, jc), t);
+        float fa[8], fb[8];
+        if (!hf) {
+          ld8(c + 5 * 128, fa);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t[e] = kk[e] * (y[e] * fa[e]);
+          tc::st_chunk(sb + Lay::GB + tc::tile_offset(96, 32 + r, jc), t);
+        }
+        // Ktilde, Qtilde: exp(Gam_r) = (x fk) fk2; fk = 1 in the first half.
+        ld8(c + 1 * 128, fa);
+        ld8(c + 2 * 128, fb);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = hf ? (x[e] * fa[e]) * fb[e] : x[e] * fb[e];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = kk[e] * x[e];
+        tc::st_chunk(sb + Lay::KT + tc::tile_offset(64, r, jc), t);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = qq[e] * x[e];
+        st_global_chunk(pk + Packet::WQ + tc::tile_offset(128, 64 + r, jc), t);
+        // Khat: exp(Gam_last - Gam_r) = (y fh) fh2; fh2 = 1 in the second half.
+        ld8(c + 3 * 128, fa);
+        ld8(c + 4 * 128, fb);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = kk[e] * (hf ? y[e] * fa[e] : (y[e] * fa[e]) * fb[e]);
+        st_global_chunk(pk + Packet::KH + tc::tile_offset(64, r, jc), t);
+      }
+      tc::fence_smem_to_async();
+      __syncthreads();
+    }
+
+    // ---------------- gated Gram products: one [128 x 96 x 128] MMA ----------------
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 96, 0, 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::GA, 128, s2), tc::desc_kmajor(sb + Lay::GB, 96, s2),
+                     id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
+    phase ^= 1;
+    tc::fence_after_sync();
+    // The Gram operands are consumed: load this chunk's V tile into their place.
+    if (tid == 32) {
+      const uint32_t vb = sb + Lay::VBAR;
+      mbar_expect_tx(vb, 64 * 256);
+      tma_load_3d(sb + Lay::VT, &maps.v, 0, h, (int)it.t0, vb);
+      tma_load_3d(sb + Lay::VT + 8192, &maps.v, 64, h, (int)it.t0, vb);
+    }
+
+    // Gram rows: lane m = row m.  k rows -> FP32 M (scaled by beta_r, strictly
+    // lower); q rows -> P (lower with diagonal), straight to the packet.
+    {
+      const int m = 32 * qd + lane, part = m >> 6, r = m & 63, second = r >> 5;
+      const int i0 = second ? 32 * hw : (hw ? 32 : 0);
+      float a[32];
+      if (second || hw == 0) {
+        tc::tmem_ld32(tl + (second ? 32 + 32 * hw : 0), a);
+        tc::tmem_wait_ld();
+      }
+      const bool zero = !second && hw;
+      if (part == 0) {
+        const float br = s_beta[r];
+        float *dst = s_M + r * kLd + i0;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dst[j] = (!zero && i0 + j < r) ? br * a[j] : 0.f;
+        if (second && i0 == 0)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) s_MT[j * 33 + (r - 32)] = br * a[j];
+      } else {   // P rows go to rows 64..127 of the TP tile, then to the packet in one bulk copy
+#pragma unroll
+        for (int j = 0; j < 32; ++j) a[j] = (!zero && i0 + j <= r) ? a[j] : 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          tc::st_chunk(sb + Lay::TP + tc::tile_offset(128, 64 + r, (i0 >> 3) + cc), a + 8 * cc);
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+      bulk_store(pk + Packet::P, sb + Lay::TP + 8192, 8192);
+      bulk_commit();
+    }
+
+    // ---------------- UT transform: (I + M)^-1 on 16x16 diagonal blocks ----------------
+    if (qd >= 2) {
+      const int blk = (qd - 2) + 2 * hw;
+      const int o = 16 * blk, c = lane & 15, hf = lane >> 4;
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = (8 * hf + i == c) ? 1.f : 0.f;
+      const float *mrow = s_M + (o + 8 * hf) * kLd + o;
+#pragma unroll
+      for (int sidx = 0; sidx < 15; ++sidx) {
+        float m[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = mrow[i * kLd + sidx];
+        const float xs = __shfl_sync(0xffffffffu, x[sidx & 7], c + 16 * (sidx >> 3));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = fmaf(-m[i], xs, x[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * kLd + o + c] = x[i];
+      if ((blk & 1) == 0)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * kLd + o + 16 + c] = 0.f;
+    }
+    __syncthreads();
+    // Level 1: the 32x32 inverse of each half.
+    {
+      const int hh = tid >> 7, rr = (tid >> 3) & 15, c0 = (tid & 7) * 2;
+      const int ro = 32 * hh + 16, co = 32 * hh;
+      float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) {
+        const float m = s_M[(ro + rr) * kLd + co + s2];
+        const float2 xv = *reinterpret_cast<const float2 *>(s_X + (co + s2) * kLd + co + c0);
+        y0 = fmaf(m, xv.x, y0);
+        y1 = fmaf(m, xv.y, y1);
+      }
+      s_Y[(hh * 16 + rr) * 17 + c0] = y0;
+      s_Y[(hh * 16 + rr) * 17 + c0 + 1] = y1;
+      __syncthreads();
+      float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) {
+        const float a = s_X[(ro + rr) * kLd + ro + s2];
+        x0 = fmaf(a, s_Y[(hh * 16 + s2) * 17 + c0], x0);
+        x1 = fmaf(a, s_Y[(hh * 16 + s2) * 17 + c0 + 1], x1);
+      }
+      *reinterpret_cast<float2 *>(s_X + (ro + rr) * kLd + co + c0) = make_float2(-x0, -x1);
+      __syncthreads();
+    }
+    // Level 2: X_(1,0) = -H1 M_(1,0) H0 with triangular trip counts.
+    {
+      const int rr = lane, cq = 4 * warp;
+      float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s2 = cq; s2 < 32; ++s2) {
+        const float m = s_MT[s2 * 33 + rr];
+        const float4 xv = *reinterpret_cast<const float4 *>(s_X + s2 * kLd + cq);
+        z.x = fmaf(m, xv.x, z.x); z.y = fmaf(m, xv.y, z.y);
+        z.z = fmaf(m, xv.z, z.z); z.w = fmaf(m, xv.w, z.w);
+      }
+      *reinterpret_cast<float4 *>(s_Z + rr * 36 + cq) = z;
+      __syncthreads();
+      const int r2 = 4 * warp + (lane >> 3), c2 = 4 * (lane & 7);
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s2 = 0; s2 < 4 * warp + 4; ++s2) {
+        const float a = s_X[(32 + r2) * kLd + 32 + s2];
+        const float4 zv = *reinterpret_cast<const float4 *>(s_Z + s2 * 36 + c2);
+        w.x = fmaf(a, zv.x, w.x); w.y = fmaf(a, zv.y, w.y);
+        w.z = fmaf(a, zv.z, w.z); w.w = fmaf(a, zv.w, w.w);
+      }
+      *reinterpret_cast<float4 *>(s_X + (32 + r2) * kLd + c2) = make_float4(-w.x, -w.y, -w.z, -w.w);
+      __syncthreads();
+    }
+    // T_ri = X_ri beta_i (i <= r) as rows 0..63 of the K-major A tile.
+    for (int e = tid; e < 64 * 8; e += kThreads) {
+      const int row = e >> 3, ch = e & 7;
+      float val[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = 8 * ch + u;
+        val[u] = i <= row ? s_X[row * kLd + i] * s_beta[i] : 0.f;
+      }
+      tc::st_chunk(sb + Lay::TP + tc::tile_offset(128, row, ch), val);
+    }
+    tc::fence_smem_to_async();
+    if (__syncthreads_or(!wait_timed(vbar, vphase, wait_ns))) { aborted = true; break; }
+    vphase ^= 1;
+
+    // ---------------- W = T Ktilde (columns 0..127), U = T V (128..255) ----------------
+    // Rows 64..127 of the A tile hold P, not T; the rows they produce are never read.
+    if (tid == 0) {
+      tc::fence_after_sync();
+      bulk_wait_read();   // the P copy has left TP (the epilogue stages U there)
+      constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::TP, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::KT, 64, s2), id, s2 > 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + 128, tc::desc_kmajor(sb + Lay::TP, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::VT, 64, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
+    phase ^= 1;
+    tc::fence_after_sync();
+    // The staging region is free again: start the next item's loads.
+    if (p + (int)gridDim.x < total) {
+      const Item nx = decode_item(p + gridDim.x, s_pref, cu, N, H, jw0);
+      intra_issue_loads(sb, maps, beta, nx.t0, nx.L, H, nx.h, tid);
+    }
+    if (qd < 2) {   // TMEM lanes 0..63 = tokens; hw 0: W -> KT tile, hw 1: U -> TP tile
+      const int r = 32 * qd + lane;
+      const uint32_t dst = sb + (hw ? Lay::TP : Lay::KT);
+      float a[32];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        tc::tmem_ld32(tl + 128 * hw + 32 * u, a);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tc::st_chunk(dst + tc::tile_offset(64, r, 4 * u + cc), a + 8 * cc);
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {   // W: rows 0..63 of both column blocks of the [W; Qtilde] tile; U: whole tile
+      bulk_store(pk + Packet::WQ, sb + Lay::KT, 8192);
+      bulk_store(pk + Packet::WQ + 16384, sb + Lay::KT + 8192, 8192);
+      bulk_store(pk + Packet::U, sb + Lay::TP, 16384);
+      bulk_commit();
+      bulk_wait_read();   // KT and TP are rewritten by the next item's prep
+    }
+    __syncthreads();
+  }
+  if (tid == 0) bulk_wait_all();
+
+  cp_async_wait_all();
+  if (aborted) {
+    report(dev_status, KDA_ERR_TIMEOUT);
+    wait_timed(bar, phase, wait_ns);
+    wait_timed(tbar, tphase, wait_ns);
+    wait_timed(vbar, vphase, wait_ns);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 256);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Pass 2: the inter-chunk chain
+// ---------------------------------------------------------------------------
+template <int DVS>
+struct ChainLayout {
+  static constexpr int NST = 2;                                   // packet buffers
+  static constexpr uint32_t S_T = 0;                              // [128][DVS] bf16 state, MN-major B
+  static constexpr uint32_t VN = S_T + 128 * DVS * 2;             // [64][DVS] bf16 V_new, MN-major B
+  static constexpr uint32_t OBUF = VN + 64 * DVS * 2;             // [64][DVS] bf16 O, rows of DVS*2 bytes
+  static constexpr uint32_t STAGE0 = OBUF + 64 * DVS * 2;
+  // inside a stage
+  static constexpr uint32_t WQ = 0;                               // [128][128] [W; Qtilde], K-major A
+  static constexpr uint32_t KH = 32768;                           // [64][128] Khat, MN-major A
+  static constexpr uint32_t U = 49152;                            // [64][DVS] U slice
+  static constexpr uint32_t P = U + 64 * DVS * 2;                 // [64][64] P = rows 64..127 of the A tile at P - 8192
+  static constexpr uint32_t D = P + 8192;                         // float[128]
+  static constexpr uint32_t STAGE = (D + 512 + 1023) & ~1023u;
+  static constexpr uint32_t BAR = STAGE0 + NST * STAGE;           // first product done
+  static constexpr uint32_t SBAR = BAR + 8;                       // state increment done
+  static constexpr uint32_t OBAR = BAR + 16;                      // O accumulation done
+  static constexpr uint32_t FULL = BAR + 24;                      // [NST] packet landed
+  static constexpr uint32_t SCAL = FULL + 8 * NST;                // int64 [2]: first packet, checkpoint slot
+  static constexpr uint32_t TMEM_SLOT = SCAL + 16;
+  static constexpr uint32_t TOTAL = TMEM_SLOT + 8;
+  static constexpr uint32_t TMEM_COLS = DVS == 128 ? 512 : 256;
+  // TMEM columns: acc1 in two buffers (chunk parity), acc2, the FP32 state
+  static constexpr uint32_t ACC1 = 0, ACC2 = DVS, SCOL = 2 * DVS, ACC1B = 3 * DVS;
+  static constexpr uint32_t TX_BYTES = 49152 + 64 * DVS * 2 + 8704;
+};
+
+template <int DVS>
+__global__ void __launch_bounds__(kThreads, 1)
+chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *__restrict__ cu,
+             __nv_bfloat16 *__restrict__ out, float *carry, int64_t interval, float *__restrict__ ck,
+             int N, int H, int64_t jw0, int64_t wc, int first_window, int32_t *dev_status,
+             uint64_t wait_ns) {
+  using Lay = ChainLayout<DVS>;
+  constexpr int NCOL = DVS / 2;
+  constexpr int NST = Lay::NST;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sb = (sraw + 1023u) & ~1023u;
+  uint8_t *sp = smem_raw + (sb - sraw);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sp + Lay::BAR);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hw = warp >> 2;
+  const int unit = blockIdx.x, n = unit / H, h = unit % H;
+  const int y = blockIdx.y, col0 = y * DVS;
+  const int crow = 32 * qd + lane;
+
+  const int64_t T_n = (int64_t)cu[n + 1] - cu[n];
+  const int64_t nch = (T_n + kC - 1) / kC;
+  if (!first_window && nch <= jw0) return;   // finished in an earlier window
+  const int64_t cnt = window_chunks(cu, n, jw0, wc);
+
+  // First packet of sequence n in this window, and its checkpoint slot.
+  if (warp == 0) {
+    int64_t before = 0, cks = 0;
+    for (int m = lane; m < n; m += 32) {
+      before += window_chunks(cu, m, jw0, wc);
+      if (interval > 0) cks += ((int64_t)cu[m + 1] - cu[m]) / interval;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+      cks += __shfl_xor_sync(0xffffffffu, cks, o);
+    }
+    if (lane == 0) {
+      reinterpret_cast<int64_t *>(sp + Lay::SCAL)[0] = before;
+      if (interval > 0) {
+        const int64_t done0 = kC * jw0 < T_n ? kC * jw0 : T_n;
+        cks += done0 / interval;
+      }
+      reinterpret_cast<int64_t *>(sp + Lay::SCAL)[1] = cks;
+    }
+  }
+  uint64_t *sbar = reinterpret_cast<uint64_t *>(sp + Lay::SBAR);
+  uint64_t *obar = reinterpret_cast<uint64_t *>(sp + Lay::OBAR);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(sbar, 1);
+    mbar_init(obar, 1);
+    for (int s = 0; s < NST; ++s) mbar_init(reinterpret_cast<uint64_t *>(sp + Lay::FULL + 8 * s), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, Lay::TMEM_COLS);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
+  const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+  const int64_t before = reinterpret_cast<const int64_t *>(sp + Lay::SCAL)[0];
+  int64_t ck_slot = reinterpret_cast<const int64_t *>(sp + Lay::SCAL)[1];
+
+  const uint8_t *pk0 = ws + ((size_t)before * H + (size_t)h * cnt) * Packet::BYTES;
+  auto issue = [&](int64_t jl, int s) {
+    const uint8_t *pk = pk0 + (size_t)jl * Packet::BYTES;
+    const uint32_t st = sb + Lay::STAGE0 + s * Lay::STAGE;
+    const uint32_t fb = sb + Lay::FULL + 8 * s;
+    mbar_expect_tx(fb, Lay::TX_BYTES);
+    bulk_load(st + Lay::WQ, pk + Packet::WQ, 49152, fb);                    // [W; Qtilde] and Khat
+    bulk_load(st + Lay::U, pk + Packet::U + (DVS == 64 ? 8192 * y : 0), 64 * DVS * 2, fb);
+    bulk_load(st + Lay::P, pk + Packet::P, 8704, fb);                       // P and d
+  };
+  if (tid == 32)
+    for (int s = 0; s < NST && s < cnt; ++s) issue(s, s);
+
+  // FP32 state slice in tensor memory (lane c = state row c), BF16 copy in S_T.
+  const uint32_t s_tm = tl + Lay::SCOL + hw * NCOL;
+  const float *src = first_window ? init : carry;
+  {
+    const size_t soff = ((size_t)unit * kDK + crow) * kDV + col0 + hw * NCOL;
+#pragma unroll
+    for (int u = 0; u < NCOL / 32; ++u) {
+      float x[32];
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 v4 = src ? *reinterpret_cast<const float4 *>(src + soff + 32 * u + j)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[j] = v4.x; x[j + 1] = v4.y; x[j + 2] = v4.z; x[j + 3] = v4.w;
+      }
+      tc::tmem_st32(s_tm + 32 * u, x);
+#pragma unroll
+      for (int j = 0; j < 32; j += 8)
+        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + 32 * u + j) >> 3), x + j);
+    }
+    tc::tmem_wait_st();
+  }
+  auto store_state = [&](float *base_ptr, int64_t slot) {
+    float *dst = base_ptr + ((size_t)slot * H + h) * kDK * kDV + (size_t)crow * kDV + col0 + hw * NCOL;
+#pragma unroll
+    for (int u = 0; u < NCOL / 32; ++u) {
+      float x[32];
+      tc::tmem_ld32(s_tm + 32 * u, x);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4 *>(dst + 32 * u + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+    }
+  };
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+
+  int64_t since_ck = interval > 0 ? (kC * jw0) % interval : 0;
+  uint32_t phase = 0, sphase = 0, ophase = 0, fphase = 0;   // fphase: bit s = parity of stage s
+  bool aborted = false;
+  // O of a chunk leaves TMEM while the next chunk's first product runs.
+  // Only the four warps on TMEM lanes 64..127 call it: they stage O (bf16) in
+  // OBUF, 16-byte chunks of row r permuted by r % 8, then write whole rows.
+  constexpr int CH = DVS / 8;   // 16-byte chunks per O row
+  auto write_o = [&](uint32_t acc, int64_t t0, int L) {
+    tc::fence_after_sync();
+    const int r = 32 * (qd - 2) + lane;
+    float a[NCOL];
+#pragma unroll
+    for (int u = 0; u < NCOL / 32; ++u)
+      tc::tmem_ld32(tl + acc + hw * NCOL + 32 * u, *reinterpret_cast<float(*)[32]>(a + 32 * u));
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int cc = 0; cc < NCOL / 8; ++cc) {
+      const int c = hw * (NCOL / 8) + cc;
+      tc::st_chunk(sb + Lay::OBUF + r * (DVS * 2) + ((c ^ (r & 7)) << 4), a + 8 * cc);
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");   // the four O warps
+    const int t = 32 * ((qd - 2) + 2 * hw) + lane;
+#pragma unroll
+    for (int e = t; e < 64 * CH; e += 128) {
+      const int row = e / CH, c = e % CH;
+      if (row < L) {
+        const uint4 v4 = *reinterpret_cast<const uint4 *>(sp + Lay::OBUF + row * (DVS * 2) + ((c ^ (row & 7)) << 4));
+        *reinterpret_cast<uint4 *>(out + ((size_t)(t0 + row) * H + h) * kDV + col0 + 8 * c) = v4;
+      }
+    }
+  };
+  int64_t t0_prev = 0;
+  int L_prev = 0;
+  for (int64_t jl = 0; jl < cnt; ++jl) {
+    const int s = (int)(jl % NST);
+    const uint32_t st = sb + Lay::STAGE0 + s * Lay::STAGE;
+    const uint32_t acc1 = (jl & 1) ? Lay::ACC1B : Lay::ACC1;
+    const int64_t j = jw0 + jl;
+    const int64_t t0 = cu[n] + kC * j;
+    const int L = (int)(T_n - kC * j < kC ? T_n - kC * j : kC);
+    if (__syncthreads_or(!wait_timed(reinterpret_cast<uint64_t *>(sp + Lay::FULL + 8 * s),
+                                     (fphase >> s) & 1u, wait_ns))) { aborted = true; break; }
+    fphase ^= 1u << s;
+
+    // acc1 = [W; Qtilde] S0
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, DVS, 0, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + acc1, tc::desc_kmajor(st + Lay::WQ, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::S_T, 128, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (jl > 0) {
+      // The previous chunk's O accumulation is done: its packet buffer may be
+      // refilled and its O written out.
+      if (__syncthreads_or(!wait_timed(obar, ophase, wait_ns))) { aborted = true; break; }
+      ophase ^= 1;
+      if (tid == 32 && jl - 1 + NST < cnt) issue(jl - 1 + NST, (int)((jl - 1) % NST));
+    }
+    // Warps on TMEM lanes 64..127 write the previous chunk's O while the others
+    // wait for the first product and form V_new.
+    bool late = false;
+    if (qd >= 2) {
+      if (jl > 0) write_o((jl & 1) ? Lay::ACC1 : Lay::ACC1B, t0_prev, L_prev);
+    } else {
+      late = !wait_timed(bar, phase, wait_ns);
+      tc::fence_after_sync();
+      // V_new = U - W S0 (TMEM lanes 0..63), as the bf16 B operand.
+      const int r = 32 * qd + lane;
+      float a[NCOL];
+#pragma unroll
+      for (int u = 0; u < NCOL / 32; ++u)
+        tc::tmem_ld32(tl + acc1 + hw * NCOL + 32 * u, *reinterpret_cast<float(*)[32]>(a + 32 * u));
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int cc = 0; cc < NCOL / 8; ++cc) {
+        const int chunk = hw * (NCOL / 8) + cc;
+        const uint4 uu = *reinterpret_cast<const uint4 *>(sp + (st - sb) + Lay::U + tc::tile_offset(64, r, chunk));
+        float xv[8];
+        unpack8(uu, xv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xv[e] -= a[8 * cc + e];
+        tc::st_chunk(sb + Lay::VN + tc::tile_offset(64, r, chunk), xv);
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    if (__syncthreads_or(late)) { aborted = true; break; }
+    phase ^= 1;
+
+    // acc1 += [*; P] V_new (rows 64..127 become O), acc2 = Khat^T V_new
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t ida = tc::idesc_bf16(128, DVS, 0, 1);
+      constexpr uint32_t idb = tc::idesc_bf16(128, DVS, 1, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + Lay::ACC2, tc::desc_mnmajor(st + Lay::KH, 64, s2),
+                     tc::desc_mnmajor(sb + Lay::VN, 64, s2), idb, s2 > 0);
+      tc::mma_commit(sb + Lay::SBAR);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + acc1, tc::desc_kmajor(st + Lay::P - 8192, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::VN, 64, s2), ida, 1);
+      tc::mma_commit(sb + Lay::OBAR);
+    }
+    const float d = reinterpret_cast<const float *>(sp + (st - sb) + Lay::D)[crow];
+    if (__syncthreads_or(!wait_timed(sbar, sphase, wait_ns))) { aborted = true; break; }
+    sphase ^= 1;
+    tc::fence_after_sync();
+    {
+      float a[NCOL], sv[NCOL];
+#pragma unroll
+      for (int u = 0; u < NCOL / 32; ++u) {
+        tc::tmem_ld32(tl + Lay::ACC2 + hw * NCOL + 32 * u, *reinterpret_cast<float(*)[32]>(a + 32 * u));
+        tc::tmem_ld32(s_tm + 32 * u, *reinterpret_cast<float(*)[32]>(sv + 32 * u));
+      }
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < NCOL; ++i) sv[i] = fmaf(d, sv[i], a[i]);
+#pragma unroll
+      for (int u = 0; u < NCOL / 32; ++u)
+        tc::tmem_st32(s_tm + 32 * u, *reinterpret_cast<float(*)[32]>(sv + 32 * u));
+#pragma unroll
+      for (int jj = 0; jj < NCOL; jj += 8)
+        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + jj) >> 3), sv + jj);
+      tc::tmem_wait_st();
+      since_ck += L;
+      if (interval > 0 && since_ck == interval) {
+        store_state(ck, ck_slot++);
+        since_ck = 0;
+      }
+    }
+    t0_prev = t0;
+    L_prev = L;
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+  }
+  if (!aborted && cnt > 0) {
+    if (__syncthreads_or(!wait_timed(obar, ophase, wait_ns))) aborted = true;
+    else {
+      ophase ^= 1;
+      if (qd >= 2) write_o(((cnt - 1) & 1) ? Lay::ACC1B : Lay::ACC1, t0_prev, L_prev);
+    }
+  }
+
+  if (aborted) {
+    report(dev_status, KDA_ERR_TIMEOUT);
+    wait_timed(bar, phase, wait_ns);
+    wait_timed(sbar, sphase, wait_ns);
+    wait_timed(obar, ophase, wait_ns);
+    for (int s = 0; s < NST; ++s)
+      wait_timed(reinterpret_cast<uint64_t *>(sp + Lay::FULL + 8 * s), (fphase >> s) & 1u, wait_ns);
+  } else if (carry) {
+    store_state(carry, n);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Lay::TMEM_COLS);
+  }
+}
+
+template <int DVS>
+cudaError_t launch_chain(const uint8_t *ws, const float *init, const int32_t *cu, void *out,
+                         float *carry, int64_t interval, float *ck, int N, int H, int64_t jw0,
+                         int64_t wc, int first, int32_t *dev_status, cudaStream_t stream) {
+  const size_t smem = ChainLayout<DVS>::TOTAL + 1024;
+  auto kern = chain_kernel<DVS>;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  dim3 grid((unsigned)((int64_t)N * H), (unsigned)(kDV / DVS));
+  kern<<<grid, kThreads, smem, stream>>>(ws, init, cu, (__nv_bfloat16 *)out, carry, interval, ck, N,
+                                         H, jw0, wc, first, dev_status, 2000000000ull);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Bytes of one packet (one chunk of one head).
+size_t split_packet_bytes() { return Packet::BYTES; }
+
+bool prefill_split_supported(int N) { return N >= 1 && N <= kMaxSeqs; }
+
+// Workspace that runs the whole batch as a single window (an upper bound:
+// every sequence may end in a partial chunk), plus the FP32 state carried
+// between windows when the caller keeps no final state.
+size_t split_workspace_full(int N, int H, int64_t T, bool have_final) {
+  const size_t packets = (size_t)H * (size_t)((T + (int64_t)(kC - 1) * N) / kC);
+  return packets * Packet::BYTES + (have_final ? 0 : (size_t)N * H * kDK * kDV * 4) + 256;
+}
+
+// Two-pass prefill over windows of chunks.  Packets of a window are stored
+// sequence by sequence, head by head, chunk by chunk: packet (n, h, j) sits at
+// index H * sum_{m<n} c_m + h * c_n + (j - jw0), c_m = chunks of m in the window.
+cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *init, const int32_t *cu, void *out,
+                                 float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
+                                 void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 cudaStream_t stream, int num_sms) {
+  if (!prefill_split_supported(N)) return cudaErrorNotSupported;
+  uintptr_t base = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~(uintptr_t)255;
+  const size_t lost = base - reinterpret_cast<uintptr_t>(workspace);
+  if (!workspace || ws_bytes < lost) return cudaErrorInvalidValue;
+  size_t avail = ws_bytes - lost;
+  const size_t state_bytes = (size_t)N * H * kDK * kDV * 4;
+  const int64_t max_chunks = (T + kC - 1) / kC;            // no sequence has more
+  const size_t all_packets = (size_t)H * (size_t)((T + (int64_t)(kC - 1) * N) / kC);
+  int64_t wc;
+  float *carry = fin;
+  uint8_t *ws = reinterpret_cast<uint8_t *>(base);
+  if (all_packets * Packet::BYTES <= avail) {
+    wc = max_chunks > 0 ? max_chunks : 1;                   // one window
+  } else {
+    if (!fin) {                                             // keep the carried state in the workspace
+      if (avail < state_bytes) return cudaErrorInvalidValue;
+      avail -= state_bytes;
+      carry = reinterpret_cast<float *>(ws + avail);
+    }
+    wc = (int64_t)(avail / ((size_t)N * H * Packet::BYTES));
+    if (wc < 1) return cudaErrorInvalidValue;
+  }
+  TmaMaps maps;
+  if (!make_input_maps(&maps, q, k, v, g, H, T) ||
+      !make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, H, T, 64, 64,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, H, T, 64, 64,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const size_t smem1 = IntraLayout::TOTAL + 1024;
+  cudaError_t err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  if (err != cudaSuccess) return err;
+  const bool narrow = (int64_t)N * H * 2 <= num_sms;       // few units: split the value columns
+  const int64_t windows = max_chunks > 0 ? (max_chunks + wc - 1) / wc : 1;
+  for (int64_t w = 0; w < windows; ++w) {
+    const int64_t jw0 = w * wc;
+    if (max_chunks > 0) {
+      intra_kernel<<<2 * num_sms, kThreads, smem1, stream>>>(maps, beta, cu, N, H, jw0, wc, ws,
+                                                            dev_status, 2000000000ull);
+      err = cudaGetLastError();
+      if (err != cudaSuccess) return err;
+    }
+    // One window: no carry needed unless the caller wants the final state.
+    float *c = (windows == 1) ? fin : carry;
+    err = narrow ? launch_chain<64>(ws, init, cu, out, c, interval, ck, N, H, jw0, wc, w == 0,
+                                    dev_status, stream)
+                 : launch_chain<128>(ws, init, cu, out, c, interval, ck, N, H, jw0, wc, w == 0,
+                                     dev_status, stream);
+    if (err != cudaSuccess) return err;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace kda

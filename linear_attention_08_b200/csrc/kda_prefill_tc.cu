@@ -48,6 +48,7 @@
 
 #include "kda_common.cuh"
 #include "kda_tc_util.cuh"
+#include "kda_tma.cuh"
 
 namespace kda {
 namespace {
@@ -91,55 +92,6 @@ struct Layout {
   static_assert(64 * DVS * 2 <= 16384, "U must fit the Ktilde slot");
 };
 
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Wait for an mbarrier phase for at most limit_ns nanoseconds.
-__device__ __forceinline__ bool wait_timed(uint64_t *bar, uint32_t phase, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, phase)) return true;
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try_wait(bar, phase))
-    if (globaltimer() - t0 > limit_ns) return false;
-  return true;
-}
-
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, bool valid) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
-               "r"(valid ? 4 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-
-// Tensor maps of the inputs (3-D views [T_tot][H][D] of the token-major
-// tensors; box = 64 tokens of one head):
-//   q, k : bf16, box (128, 1, 64), no swizzle   -> staging rows of 256 bytes
-//   g    : fp32, box (128, 1, 64), no swizzle   -> staging rows of 512 bytes
-//   v    : bf16, box (64, 1, 64), 128-byte swizzle -> one column block of the
-//          [X/U | V] tile, already in the MMA layout.
-// Tokens past T_tot read as zeros; tokens of the next sequence are masked by
-// the consumer (q, k, g) or cancel exactly (v: beta is 0 there).
-struct TmaMaps {
-  CUtensorMap q, k, g, v;
-};
-
-__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap *map, int x, int y,
-                                            int z, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-
 // Start loading the raw inputs of the chunk [t0, t0 + L): q, k, g into the
 // staging area and v into its operand slot (one elected thread, TMA); beta
 // into s_beta (64 threads, 4-byte async copies, zero past L).
@@ -165,16 +117,6 @@ __device__ __forceinline__ void prefetch_chunk(uint32_t sb, const TmaMaps &maps,
     cp_async4(sb + Lay::BETA + 4 * r, beta + (ok ? (size_t)(t0 + r) * H + h : 0), ok);
   }
   cp_async_commit();
-}
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float *x) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __bfloat1622float2(h[i]);
-    x[2 * i] = f.x;
-    x[2 * i + 1] = f.y;
-  }
 }
 
 template <int DVS>
@@ -740,37 +682,6 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
   }
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 3-D map over a token-major tensor [T][H][D]: dims (D, H, T), box (box_d, 1, 64).
-static bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes,
-                     int D, int H, int64_t T, int box_d, CUtensorMapSwizzle swz) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
-  const cuuint64_t strides[2] = {(cuuint64_t)D * elem_bytes, (cuuint64_t)D * elem_bytes * H};
-  const cuuint32_t box[3] = {(cuuint32_t)box_d, 1, (cuuint32_t)kC};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int DVS>
 cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const float *g,
                         const float *beta, const float *init, const int32_t *cu, void *out,
@@ -778,11 +689,7 @@ cudaError_t launch_tc_t(const void *q, const void *k, const void *v, const float
                         const int32_t *positions, float *pos_states, int N, int H, int64_t T,
                         int32_t *dev_status, cudaStream_t stream) {
   TmaMaps maps;
-  if (!make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, H, T, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDK, H, T, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&maps.g, g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK, H, T, kDK, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_map(&maps.v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kDV, H, T, 64, CU_TENSOR_MAP_SWIZZLE_128B))
-    return cudaErrorInvalidValue;
+  if (!make_input_maps(&maps, q, k, v, g, H, T)) return cudaErrorInvalidValue;
   const size_t smem = Layout<DVS>::TOTAL + 1024;
   auto kern = prefill_tc_kernel<DVS>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -17,9 +17,14 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 KDA_OK, KDA_ERR_INVALID_ARGUMENT, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(5)
 KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 
-EXPORTED = ("kda_prefill", "kda_prefill_at", "kda_decode", "kda_decode_multi", "kda_ckpt_count", "kda_prefill_workspace_bytes",
-            "kda_prefill_path", "kda_selftest_bounded_wait", "kda_last_cuda_error",
-            "kda_status_string", "kda_version")
+EXPORTED = ("kda_prefill", "kda_prefill_ws", "kda_prefill_at", "kda_decode", "kda_decode_multi",
+            "kda_ckpt_count", "kda_prefill_workspace_bytes", "kda_prefill_workspace_min_bytes",
+            "kda_release_workspace_pool", "kda_prefill_path", "kda_selftest_bounded_wait",
+            "kda_last_cuda_error", "kda_status_string", "kda_version")
+
+# Largest workspace the binding allocates for the two-pass prefill; longer
+# inputs run in windows of chunks.
+WORKSPACE_CAP = int(os.environ.get("KDA_WORKSPACE_CAP", 8 << 30))
 
 
 class KdaShape(ctypes.Structure):
@@ -60,6 +65,8 @@ def load(path: str | None = None):
     SP = ctypes.POINTER(KdaShape)
     lib.kda_prefill.argtypes = [P, P, P, P, P, P, P, P, P, I64, P, SP, P]
     lib.kda_prefill.restype = ctypes.c_int
+    lib.kda_prefill_ws.argtypes = [P, P, P, P, P, P, P, P, P, I64, P, P, ctypes.c_size_t, SP, P]
+    lib.kda_prefill_ws.restype = ctypes.c_int
     lib.kda_prefill_at.argtypes = [P, P, P, P, P, P, P, P, P, I64, P, P, P, P, SP, P]
     lib.kda_prefill_at.restype = ctypes.c_int
     lib.kda_decode.argtypes = [P, P, P, P, P, P, P, SP, P]
@@ -70,6 +77,9 @@ def load(path: str | None = None):
     lib.kda_ckpt_count.restype = I64
     lib.kda_prefill_workspace_bytes.argtypes = [SP]
     lib.kda_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_prefill_workspace_min_bytes.argtypes = [SP]
+    lib.kda_prefill_workspace_min_bytes.restype = ctypes.c_size_t
+    lib.kda_release_workspace_pool.restype = ctypes.c_int
     lib.kda_prefill_path.argtypes = [SP]
     lib.kda_prefill_path.restype = ctypes.c_int
     lib.kda_selftest_bounded_wait.argtypes = [P, I64, P]
@@ -118,10 +128,30 @@ def kda_prefill_path(shape: KdaShape) -> int:
     return int(load().kda_prefill_path(ctypes.byref(shape)))
 
 
+def kda_prefill_workspace_bytes(shape: KdaShape) -> int:
+    return int(load().kda_prefill_workspace_bytes(ctypes.byref(shape)))
+
+
+def kda_prefill_workspace_min_bytes(shape: KdaShape) -> int:
+    return int(load().kda_prefill_workspace_min_bytes(ctypes.byref(shape)))
+
+
+def workspace_for(shape: KdaShape, device, cap: int | None = None):
+    """A torch-owned workspace for the two-pass prefill of ``shape`` (None when
+    the shape runs on a single-pass kernel): the single-window size, capped
+    at ``cap`` bytes (but never below the minimum)."""
+    full = kda_prefill_workspace_bytes(shape)
+    if full in (0, (1 << 64) - 1):
+        return None
+    cap = WORKSPACE_CAP if cap is None else int(cap)
+    nbytes = max(min(full, cap), kda_prefill_workspace_min_bytes(shape))
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
 def kda_prefill(q, k, v, g, beta, cu_seqlens, *, init_state=None, chunk: int = 64,
                 ckpt_interval: int = 0, cu_seqlens_host=None, out=None, final_state=None,
                 ckpt_states=None, dev_status=None, stream=None, want_final: bool = True,
-                positions=None, pos_states=None):
+                positions=None, pos_states=None, workspace="auto"):
     """Chunked KDA prefill over a packed batch (see kda_prefill in include/kda.h).
 
     q, k, g: [T, H, Dk]; v: [T, H, Dv]; beta: [T, H]; cu_seqlens: int32 device
@@ -129,7 +159,9 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, *, init_state=None, chunk: int = 6
     with torch when not given.  ``cu_seqlens_host`` (a list) avoids a device
     read when checkpoints are requested.  ``positions`` (one list of token
     counts per sequence) also stores the states after those counts
-    (kda_prefill_at).  Returns (out, final_state, ckpt_states), plus
+    (kda_prefill_at).  ``workspace``: "auto" allocates one with torch
+    (``workspace_for``), a uint8 device tensor is used as given, None runs
+    the single-pass kernels.  Returns (out, final_state, ckpt_states), plus
     pos_states when positions are given.
     """
     lib = load()
@@ -149,11 +181,16 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, *, init_state=None, chunk: int = 6
     if ckpt_interval > 0 and ckpt_states.numel() == 0:
         ck_ptr = ctypes.c_void_p(ckpt_states.untyped_storage().data_ptr())
     if positions is None:
-        st = lib.kda_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init_state),
-                             _ptr(cu_seqlens), _ptr(out), _ptr(final_state), int(ckpt_interval),
-                             ck_ptr, ctypes.byref(shape), _stream(stream))
+        if isinstance(workspace, str):
+            assert workspace == "auto"
+            workspace = workspace_for(shape, q.device)
+        nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        st = lib.kda_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init_state),
+                                _ptr(cu_seqlens), _ptr(out), _ptr(final_state),
+                                int(ckpt_interval), ck_ptr, _ptr(workspace), nbytes,
+                                ctypes.byref(shape), _stream(stream))
         if st != KDA_OK:
-            raise KdaError(st, "kda_prefill")
+            raise KdaError(st, "kda_prefill_ws")
         return out, final_state, ckpt_states
     counts = [0]
     for lst in positions:

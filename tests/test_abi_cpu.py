@@ -107,6 +107,29 @@ def test_workspace_and_path_queries():
     assert kda.kda_prefill_path(s) == 0            # FP32 runs on the SIMT kernel
     bad = _shape(Dk=12)
     assert kda.kda_prefill_path(bad) == -1
+    assert lib.kda_prefill_workspace_bytes(ctypes.byref(bad)) == (1 << 64) - 1
+    # BF16, D = 128, C = 64: the two-pass path, 74240 bytes per (chunk, head) packet
+    s2 = kda.make_shape(2, 1000, 4, 128, 128, 64, kda.KDA_DTYPE_BF16)
+    assert kda.kda_prefill_path(s2) == 2
+    chunks_bound = (1000 + 63 * 2) // 64
+    state = 2 * 4 * 128 * 128 * 4
+    assert lib.kda_prefill_workspace_bytes(ctypes.byref(s2)) == 4 * chunks_bound * 74240 + state + 256
+    assert lib.kda_prefill_workspace_min_bytes(ctypes.byref(s2)) == 2 * 4 * 74240 + state + 256
+    s3 = kda.make_shape(2000, 4000, 4, 128, 128, 64, kda.KDA_DTYPE_BF16)
+    assert kda.kda_prefill_path(s3) == 1          # too many sequences for the two-pass path
+    assert lib.kda_prefill_workspace_bytes(ctypes.byref(s3)) == 0
+
+
+def test_prefill_ws_rejects_bad_workspace():
+    lib = kda.load()
+    s = kda.make_shape(2, 1000, 4, 128, 128, 64, kda.KDA_DTYPE_BF16)
+    a = ctypes.c_void_p(1 << 20)
+    b = ctypes.c_void_p(1 << 30)
+    call = lambda ws, nbytes: lib.kda_prefill_ws(a, a, a, a, a, None, a, b, None, 0, None, ws,
+                                                 nbytes, ctypes.byref(s), None)
+    # misaligned workspace; workspace overlapping out
+    assert call(ctypes.c_void_p((1 << 34) + 8), 1 << 20) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert call(ctypes.c_void_p((1 << 30) - 4096), 1 << 20) == kda.KDA_ERR_INVALID_ARGUMENT
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

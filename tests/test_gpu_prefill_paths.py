@@ -1,0 +1,114 @@
+"""Prefill routes against the FP64 oracle: the two-pass tensor-core path in one
+and in several windows of chunks (caller workspace), the single-pass kernel
+(no workspace), and the plain C entry that takes its workspace from the
+library's pool."""
+import ctypes
+
+import pytest
+import torch
+
+from linear_attention_08_b200 import kda
+from parity import TOL, make_case, oracle_full, rel_l2, to_device
+
+pytestmark = pytest.mark.gpu
+
+LENGTHS = [200, 64, 1, 130, 257]
+
+
+def run(dd, interval, workspace, want_final=True, use_init=True):
+    return kda.kda_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu_dev"],
+                           init_state=dd["init_state"] if use_init else None, chunk=64,
+                           ckpt_interval=interval, cu_seqlens_host=dd["cu_seqlens"],
+                           want_final=want_final, workspace=workspace)
+
+
+def shape_of(dd):
+    T, H, Dk = dd["q"].shape
+    return kda.make_shape(len(dd["cu_seqlens"]) - 1, T, H, Dk, dd["v"].shape[2], 64,
+                          kda.KDA_DTYPE_BF16)
+
+
+def check(d, out, fin, ck, interval, use_init=True, tol=TOL[torch.bfloat16]):
+    ro, rf, rc = oracle_full(d, interval, use_init)
+    assert rel_l2(out, ro) <= tol
+    if fin is not None:
+        assert rel_l2(fin, rf) <= tol
+    if interval > 0 and rc.shape[0]:
+        assert rel_l2(ck, rc) <= tol
+
+
+def test_path_query():
+    d = to_device(make_case(LENGTHS, 3, 128, 128, torch.bfloat16, seed=3))
+    assert kda.kda_prefill_path(shape_of(d)) == 2
+    s = shape_of(d)
+    s.chunk = 16
+    assert kda.kda_prefill_path(s) == 0
+    s = shape_of(d)
+    s.num_seqs = 4096   # too many sequences for the two-pass path
+    assert kda.kda_prefill_path(s) == 1
+    assert kda.kda_prefill_workspace_bytes(shape_of(d)) >= kda.kda_prefill_workspace_min_bytes(shape_of(d)) > 0
+
+
+@pytest.mark.parametrize("windows_of", [1, 2, 3, None])
+@pytest.mark.parametrize("want_final", [True, False])
+def test_two_pass_windows(windows_of, want_final):
+    """Workspace for windows of 1, 2 or 3 chunks (None: one window), checkpoints every two
+    chunks, nonzero initial state; without final_state the carried state lives in the
+    workspace."""
+    d = make_case(LENGTHS, 3, 128, 128, torch.bfloat16, seed=4, state_std=0.1)
+    dd = to_device(d)
+    shape = shape_of(dd)
+    if windows_of is None:
+        nbytes = kda.kda_prefill_workspace_bytes(shape)
+    else:
+        N, H = len(LENGTHS), 3
+        nbytes = (kda.kda_prefill_workspace_min_bytes(shape)
+                  + (windows_of - 1) * N * H * 74240)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    out, fin, ck = run(dd, 128, ws, want_final=want_final)
+    torch.cuda.synchronize()
+    check(d, out, fin if want_final else None, ck, 128)
+
+
+def test_single_pass_and_two_pass_agree():
+    d = make_case(LENGTHS, 4, 128, 128, torch.bfloat16, seed=5, state_std=0.05)
+    dd = to_device(d)
+    o1, f1, c1 = run(dd, 64, None)
+    o2, f2, c2 = run(dd, 64, "auto")
+    torch.cuda.synchronize()
+    check(d, o1, f1, c1, 64)
+    check(d, o2, f2, c2, 64)
+    assert rel_l2(o1, o2.double().cpu().numpy()) <= 1e-2
+    assert rel_l2(f1, f2.double().cpu().numpy()) <= 1e-2
+
+
+def test_plain_entry_uses_pool():
+    """kda_prefill (no workspace argument) twice, then the pool is released."""
+    d = make_case(LENGTHS, 3, 128, 128, torch.bfloat16, seed=6, state_std=0.02)
+    dd = to_device(d)
+    lib = kda.load()
+    T, H, Dk = dd["q"].shape
+    N = len(LENGTHS)
+    out = torch.empty(T, H, 128, dtype=torch.bfloat16, device="cuda")
+    fin = torch.empty(N, H, 128, 128, device="cuda")
+    shape = shape_of(dd)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for _ in range(2):
+        st = lib.kda_prefill(P(dd["q"]), P(dd["k"]), P(dd["v"]), P(dd["g"]), P(dd["beta"]),
+                             P(dd["init_state"]), P(dd["cu_dev"]), P(out), P(fin), 0, None,
+                             ctypes.byref(shape), stream)
+        assert st == kda.KDA_OK
+    torch.cuda.synchronize()
+    check(d, out, fin, None, 0)
+    assert lib.kda_release_workspace_pool() == kda.KDA_OK
+
+
+def test_many_sequences_single_pass():
+    """More sequences than the two-pass path takes: the single-pass kernel runs."""
+    lengths = [3, 70] * 520
+    d = make_case(lengths, 1, 128, 128, torch.bfloat16, seed=7, state_std=0.02)
+    dd = to_device(d)
+    out, fin, _ = run(dd, 0, "auto")
+    torch.cuda.synchronize()
+    check(d, out, fin, None, 0)
