@@ -43,17 +43,20 @@ def test_positions_against_oracle(dtype, dims, chunk):
 
 
 def test_position_state_resumes_exactly():
-    """Resuming from the state stored at an unaligned prompt boundary reproduces the rest."""
+    """Resuming from the state stored at an unaligned prompt boundary reproduces the rest:
+    to rounding when the resumed call runs the same single-pass kernel (no workspace),
+    within the parity tolerance when it runs the two-pass kernels."""
     L, cut = 500, 173
     d = make_case([L], 2, 128, 128, torch.bfloat16, seed=42, state_std=0.1)
     dd = to_device(d)
     out, fin, _, ps = kda.kda_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu_dev"],
                                       init_state=dd["init_state"], chunk=64, positions=[[cut]])
-    o_r, f_r, _ = kda.kda_prefill(dd["q"][cut:].contiguous(), dd["k"][cut:].contiguous(),
-                                  dd["v"][cut:].contiguous(), dd["g"][cut:].contiguous(),
-                                  dd["beta"][cut:].contiguous(),
-                                  torch.tensor([0, L - cut], dtype=torch.int32, device="cuda"),
-                                  init_state=ps[0:1].contiguous(), chunk=64)
-    torch.cuda.synchronize()
-    assert rel_l2(o_r, out[cut:].double().cpu().numpy()) <= 1e-5
-    assert rel_l2(f_r, fin.double().cpu().numpy()) <= 1e-5
+    for ws, tol in ((None, 1e-5), ("auto", 1e-2)):
+        o_r, f_r, _ = kda.kda_prefill(dd["q"][cut:].contiguous(), dd["k"][cut:].contiguous(),
+                                      dd["v"][cut:].contiguous(), dd["g"][cut:].contiguous(),
+                                      dd["beta"][cut:].contiguous(),
+                                      torch.tensor([0, L - cut], dtype=torch.int32, device="cuda"),
+                                      init_state=ps[0:1].contiguous(), chunk=64, workspace=ws)
+        torch.cuda.synchronize()
+        assert rel_l2(o_r, out[cut:].double().cpu().numpy()) <= tol
+        assert rel_l2(f_r, fin.double().cpu().numpy()) <= tol
