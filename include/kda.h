@@ -114,6 +114,37 @@ kda_status kda_prefill_ws(const void *q, const void *k, const void *v, const flo
                           float *ckpt_states, void *workspace, size_t workspace_bytes,
                           const kda_shape *shape, kda_stream_t stream);
 
+/* Size of the fixed device array behind kda_prefill_noalloc. */
+#define KDA_NOALLOC_SCRATCH_BYTES ((size_t)128 << 20)
+
+/*
+ * kda_prefill for callers that cannot allocate device memory when they call
+ * it: a serving engine that has already handed all free memory to its own
+ * pool (a KV cache sized to what was left), or a runtime whose allocator this
+ * library cannot reach.  It runs the two-pass prefill with its workspace in
+ * a fixed array of KDA_NOALLOC_SCRATCH_BYTES compiled into the library (every
+ * GPU that loads the library holds it until the process exits) and calls no
+ * allocator.  No part of the methods on the pages this library follows
+ * corresponds to it; it is a deployment aid.
+ *
+ * Arguments as for kda_prefill.  Only shapes on the two-pass path
+ * (kda_prefill_path = 2) are accepted, and only when one chunk of every
+ * (sequence, head) fits the array: num_seqs * num_heads * 74240 bytes, plus
+ * num_seqs * num_heads * 65536 when final_state is NULL, plus 256, at most
+ * KDA_NOALLOC_SCRATCH_BYTES; longer batches run in windows of chunks.  Other
+ * shapes return KDA_ERR_UNSUPPORTED before any work is queued.
+ * The first call on a device looks up the array's device address, so make
+ * that first call before any stream capture.  All calls share the one array
+ * and nothing in it needs to start at zero (each call writes every byte it
+ * reads), but calls whose work overlaps on the GPU (other streams, other
+ * threads) race on it: order them on one stream or synchronise between them.
+ */
+kda_status kda_prefill_noalloc(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *init_state,
+                               const int32_t *cu_seqlens, void *out, float *final_state,
+                               int64_t ckpt_interval, float *ckpt_states,
+                               const kda_shape *shape, kda_stream_t stream);
+
 /*
  * kda_prefill with states also stored at explicit positions, such as the
  * boundaries of cached prompts (the first page, Conclusion table: prefix

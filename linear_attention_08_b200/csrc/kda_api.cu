@@ -39,6 +39,13 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
 
 static thread_local int g_last_cuda_error = 0;
 
+// For entry points defined in other files of the library.
+kda_status record_cuda_error(cudaError_t e) {
+  if (e == cudaSuccess) return KDA_OK;
+  g_last_cuda_error = (int)e;
+  return KDA_ERR_CUDA;
+}
+
 // Largest workspace kda_prefill takes from its pool (longer inputs run in windows).
 static const size_t kPoolCap = (size_t)8 << 30;
 static const int kMaxDevices = 64;
