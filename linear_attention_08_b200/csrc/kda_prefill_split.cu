@@ -76,10 +76,11 @@ struct IntraLayout {
   static constexpr uint32_t VT = 49152;      // [64][128] V tile (MN-major B), loaded after the Gram MMA
   static constexpr uint32_t KT = 65536;      // [64][128] Ktilde tile (MN-major B)
   static constexpr uint32_t TP = 81920;      // [128][64] T (rows 0..63) as K-major A
-  static constexpr uint32_t RED = TP;        // float [16][128] scan partials (before T exists)
+  static constexpr uint32_t RED = TP;        // float [8][128] scan partials (before T exists)
   static constexpr uint32_t BETA = 98304;    // float [64]
   static constexpr uint32_t PREF = BETA + 256;                    // int [kMaxSeqs + 1]
-  static constexpr uint32_t BAR = (PREF + 4 * (kMaxSeqs + 1) + 7) & ~7u;   // MMA completion
+  static constexpr uint32_t CUS = PREF + 4 * (kMaxSeqs + 1);      // int [kMaxSeqs + 1] cu_seqlens
+  static constexpr uint32_t BAR = (CUS + 4 * (kMaxSeqs + 1) + 7) & ~7u;    // MMA completion
   static constexpr uint32_t TBAR = BAR + 8;                       // q, k, g landed
   static constexpr uint32_t VBAR = BAR + 16;                      // v landed
   static constexpr uint32_t TMEM_SLOT = BAR + 24;
@@ -88,6 +89,14 @@ struct IntraLayout {
   static_assert(CST + 6144 <= 65536, "gate factors overflow the staging region");
   static_assert(GB + 96 * 256 <= CST, "Gram B overlaps the gate factors");
 };
+
+// 16-byte store of 8 floats as bf16 into shared memory, as a plain C++ store
+// (the compiler may schedule loads around it; the proxy fences that publish
+// the tiles to the tensor core are ordered after it).
+__device__ __forceinline__ void st_chunk_s(uint8_t *dst, const float *x) {
+  *reinterpret_cast<uint4 *>(dst) = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                                               tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+}
 
 // 16-byte store of 8 floats as bf16 into global memory.
 __device__ __forceinline__ void st_global_chunk(uint8_t *dst, const float *x) {
@@ -179,6 +188,8 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, hw = warp >> 2;
 
+  int32_t *s_cu = reinterpret_cast<int32_t *>(sp + Lay::CUS);
+  for (int n = tid; n <= N; n += kThreads) s_cu[n] = cu[n];
   // Packets of the window, sequence by sequence: s_pref[n] = first packet of n.
   for (int n = tid; n < N; n += kThreads) s_pref[n + 1] = (int32_t)(window_chunks(cu, n, jw0, wc) * H);
   if (tid == 0) s_pref[0] = 0;
@@ -220,148 +231,136 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
   bool aborted = false;
   int p = blockIdx.x;
   {
-    const Item it = decode_item(p, s_pref, cu, N, H, jw0);
+    const Item it = decode_item(p, s_pref, s_cu, N, H, jw0);
     intra_issue_loads(sb, maps, beta, it.t0, it.L, H, it.h, tid);
   }
 
   for (; p < total; p += gridDim.x) {
-    const Item it = decode_item(p, s_pref, cu, N, H, jw0);
+    const Item it = decode_item(p, s_pref, s_cu, N, H, jw0);
     const int L = it.L, h = it.h;
     uint8_t *pk = ws + (size_t)p * Packet::BYTES;
 
     cp_async_wait_all();
+    if (tid == 0) bulk_wait_read();   // the previous item's W and U have left KT and TP
     if (__syncthreads_or(!wait_timed(tbar, tphase, wait_ns))) { aborted = true; break; }
     tphase ^= 1;
 
-    // ---------------- gate prep (as in the fused kernel) ----------------
-    // Thread (rg, jc) owns rows 4rg..4rg+3 and channels 8jc..8jc+7.
+    // ---------------- gate prep ----------------
+    // Warp w owns rows 8w..8w+7 (half hf = w / 4), lane l owns channels 4l..4l+3:
+    // per row one 8-byte piece of each 16-byte tile chunk, and the gate factors
+    // of the lane's channels stay in registers for all its rows.
     {
-      const int rg = tid >> 4, jc = tid & 15, hf = rg >> 3;
-      float gm[4][8];
+      const int hf = warp >> 2, cq = lane >> 1, sub = (lane & 1) * 8;
+      float gm[8][4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 4 * rg + i;
-        const bool in = r < L;
-        const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
-        const float4 a = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + jc * 32) : zf;
-        const float4 b = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + jc * 32 + 16) : zf;
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * warp + i;
+        const float4 a = r < L ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + lane * 16)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
         gm[i][0] = a.x; gm[i][1] = a.y; gm[i][2] = a.z; gm[i][3] = a.w;
-        gm[i][4] = b.x; gm[i][5] = b.y; gm[i][6] = b.z; gm[i][7] = b.w;
       }
 #pragma unroll
-      for (int i = 1; i < 4; ++i)
+      for (int i = 1; i < 8; ++i)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) gm[i][e] += gm[i - 1][e];
-      {
-        float4 *dst = reinterpret_cast<float4 *>(s_red + rg * 128 + 8 * jc);
-        dst[0] = make_float4(gm[3][0], gm[3][1], gm[3][2], gm[3][3]);
-        dst[1] = make_float4(gm[3][4], gm[3][5], gm[3][6], gm[3][7]);
-      }
+        for (int e = 0; e < 4; ++e) gm[i][e] += gm[i - 1][e];
+      *reinterpret_cast<float4 *>(s_red + warp * 128 + 4 * lane) =
+          make_float4(gm[7][0], gm[7][1], gm[7][2], gm[7][3]);
       __syncthreads();
-      // Exclusive scan of the 16 row-group totals per channel (warp w: channels
-      // 16w..16w+15; lane (ch, half) holds row groups 8 half .. 8 half + 7), and the
-      // per-channel gate factors, formed once.
-      {
-        const int ch = 16 * warp + (lane & 15), half = lane >> 4;
-        float t[8], run = 0.f;
+      // One lane per channel: exclusive scan of the 8 row-group totals, the cumulative
+      // decay at rows 15, 31, 47, 63, and the channel's gate factors for both halves.
+      if (tid < 128) {
+        const int ch = tid;
+        float t[8], run = 0.f, incl[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = s_red[(8 * half + i) * 128 + ch];
-        float incl[8];
+        for (int i = 0; i < 8; ++i) t[i] = s_red[i * 128 + ch];
 #pragma unroll
         for (int i = 0; i < 8; ++i) { run += t[i]; incl[i] = run; }
-        const float lower = __shfl_sync(0xffffffffu, run, lane & 15);
-        const float off = half ? lower : 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s_red[(8 * half + i) * 128 + ch] = off + incl[i] - t[i];
-        const float ga = off + incl[3], gb = off + incl[7];
-        const float G15 = __shfl_sync(0xffffffffu, ga, lane & 15);
-        const float G31 = __shfl_sync(0xffffffffu, gb, lane & 15);
-        const float G47 = __shfl_sync(0xffffffffu, ga, (lane & 15) + 16);
-        const float G63 = __shfl_sync(0xffffffffu, gb, (lane & 15) + 16);
+        for (int i = 0; i < 8; ++i) s_red[i * 128 + ch] = incl[i] - t[i];
+        const float G15 = incl[1], G31 = incl[3], G47 = incl[5], G63 = incl[7];
         // Row r of half hf is scaled against ref = Gam_15 (hf 0) or Gam_47 (hf 1);
         // the products are grouped exactly as in the fused kernel (no intermediate
         // underflows unless the exact value is itself far below the BF16 rounding).
-        float f[6];
-        if (half == 0) {
-          f[0] = G15; f[1] = 1.f; f[2] = __expf(G15);
-          f[3] = __expf(G31 - G15); f[4] = __expf(G63 - G31); f[5] = __expf(G47 - G15);
-        } else {
-          f[0] = G47; f[1] = __expf(G47 - G31); f[2] = __expf(G31);
-          f[3] = __expf(G63 - G47); f[4] = 1.f; f[5] = 0.f;
-          reinterpret_cast<float *>(pk + Packet::D)[ch] = __expf(G63);
-        }
+        float f[12];
+        f[0] = G15; f[1] = 1.f; f[2] = __expf(G15);
+        f[3] = __expf(G31 - G15); f[4] = __expf(G63 - G31); f[5] = __expf(G47 - G15);
+        f[6] = G47; f[7] = __expf(G47 - G31); f[8] = __expf(G31);
+        f[9] = __expf(G63 - G47); f[10] = 1.f; f[11] = 0.f;
 #pragma unroll
-        for (int j = 0; j < 6; ++j) s_cst[(half * 6 + j) * 128 + ch] = f[j];
+        for (int j = 0; j < 12; ++j) s_cst[j * 128 + ch] = f[j];
+        reinterpret_cast<float *>(pk + Packet::D)[ch] = __expf(G63);
       }
       __syncthreads();
-      auto ld8 = [&](const float *src, float *d8) {
-        const float4 a = reinterpret_cast<const float4 *>(src)[0];
-        const float4 b = reinterpret_cast<const float4 *>(src)[1];
-        d8[0] = a.x; d8[1] = a.y; d8[2] = a.z; d8[3] = a.w;
-        d8[4] = b.x; d8[5] = b.y; d8[6] = b.z; d8[7] = b.w;
-      };
+      float ref[4], fk[4], fk2[4], fh[4], fh2[4], cb[4];
       {
-        float base[8];
-        ld8(s_red + rg * 128 + 8 * jc, base);
+        auto ld4 = [&](int j, float *d4) {
+          const float4 v = *reinterpret_cast<const float4 *>(s_cst + (hf * 6 + j) * 128 + 4 * lane);
+          d4[0] = v.x; d4[1] = v.y; d4[2] = v.z; d4[3] = v.w;
+        };
+        float base[4];
+        const float4 bv = *reinterpret_cast<const float4 *>(s_red + warp * 128 + 4 * lane);
+        base[0] = bv.x; base[1] = bv.y; base[2] = bv.z; base[3] = bv.w;
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+        for (int i = 0; i < 8; ++i)
 #pragma unroll
-          for (int i = 0; i < 4; ++i) gm[i][e] += base[e];
+          for (int e = 0; e < 4; ++e) gm[i][e] += base[e];
+        ld4(0, ref); ld4(1, fk); ld4(2, fk2); ld4(3, fh); ld4(4, fh2); ld4(5, cb);
       }
-      const float *c = s_cst + hf * 6 * 128 + 8 * jc;
+      auto st4 = [&](uint8_t *dst, const float *x) {
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]));
+      };
+      auto un4 = [&](const uint2 &u, float *x) {
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+      };
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 4 * rg + i;
-        float ref[8], kk[8], qq[8], x[8], y[8], t[8];
-        ld8(c, ref);
-        {   // raw k and q of this row and channel group, replaced below by k x and q x
-          const uint4 z4 = make_uint4(0, 0, 0, 0);
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * warp + i;
+        float kk[4], qq[4], x[4], y[4], t[4];
+        {   // raw k and q of this row, replaced below by k x and q x
           const bool in = r < L;
-          const uint4 kv = in ? *reinterpret_cast<const uint4 *>(sp + Lay::GA + tc::tile_offset(128, r, jc)) : z4;
-          const uint4 qv = in ? *reinterpret_cast<const uint4 *>(sp + Lay::GA + tc::tile_offset(128, 64 + r, jc)) : z4;
-          unpack8(kv, kk);
-          unpack8(qv, qq);
+          const uint2 z2 = make_uint2(0, 0);
+          const uint2 kv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub) : z2;
+          const uint2 qv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub) : z2;
+          un4(kv, kk);
+          un4(qv, qq);
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           x[e] = __expf(gm[i][e] - ref[e]);
+          // reciprocal by two Newton steps from the bit-level initial guess
           float r0 = __int_as_float(0x7EF311C3 - __float_as_int(x[e]));
           r0 = r0 * fmaf(-x[e], r0, 2.f);
           y[e] = r0 * fmaf(-x[e], r0, 2.f);
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = kk[e] * x[e];
-        tc::st_chunk(sb + Lay::GA + tc::tile_offset(128, r, jc), t);
+        for (int e = 0; e < 4; ++e) t[e] = kk[e] * x[e];
+        st4(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = qq[e] * x[e];
-        tc::st_chunk(sb + Lay::GA + tc::tile_offset(128, 64 + r, jc), t);
+        for (int e = 0; e < 4; ++e) t[e] = qq[e] * x[e];
+        st4(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = kk[e] * y[e];
-        tc::st_chunk(sb + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, jc), t);
-        float fa[8], fb[8];
+        for (int e = 0; e < 4; ++e) t[e] = kk[e] * y[e];
+        st4(sp + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, cq) + sub, t);
         if (!hf) {
-          ld8(c + 5 * 128, fa);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[e] * (y[e] * fa[e]);
-          tc::st_chunk(sb + Lay::GB + tc::tile_offset(96, 32 + r, jc), t);
+          for (int e = 0; e < 4; ++e) t[e] = kk[e] * (y[e] * cb[e]);
+          st4(sp + Lay::GB + tc::tile_offset(96, 32 + r, cq) + sub, t);
         }
         // Ktilde, Qtilde: exp(Gam_r) = (x fk) fk2; fk = 1 in the first half.
-        ld8(c + 1 * 128, fa);
-        ld8(c + 2 * 128, fb);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = hf ? (x[e] * fa[e]) * fb[e] : x[e] * fb[e];
+        for (int e = 0; e < 4; ++e) x[e] = hf ? (x[e] * fk[e]) * fk2[e] : x[e] * fk2[e];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = kk[e] * x[e];
-        tc::st_chunk(sb + Lay::KT + tc::tile_offset(64, r, jc), t);
+        for (int e = 0; e < 4; ++e) t[e] = kk[e] * x[e];
+        st4(sp + Lay::KT + tc::tile_offset(64, r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = qq[e] * x[e];
-        st_global_chunk(pk + Packet::WQ + tc::tile_offset(128, 64 + r, jc), t);
+        for (int e = 0; e < 4; ++e) t[e] = qq[e] * x[e];
+        st4(pk + Packet::WQ + tc::tile_offset(128, 64 + r, cq) + sub, t);
         // Khat: exp(Gam_last - Gam_r) = (y fh) fh2; fh2 = 1 in the second half.
-        ld8(c + 3 * 128, fa);
-        ld8(c + 4 * 128, fb);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = kk[e] * (hf ? y[e] * fa[e] : (y[e] * fa[e]) * fb[e]);
-        st_global_chunk(pk + Packet::KH + tc::tile_offset(64, r, jc), t);
+        for (int e = 0; e < 4; ++e) t[e] = kk[e] * (hf ? y[e] * fh[e] : (y[e] * fh[e]) * fh2[e]);
+        st4(pk + Packet::KH + tc::tile_offset(64, r, cq) + sub, t);
       }
       tc::fence_smem_to_async();
       __syncthreads();
@@ -412,7 +411,7 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
         for (int j = 0; j < 32; ++j) a[j] = (!zero && i0 + j <= r) ? a[j] : 0.f;
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
-          tc::st_chunk(sb + Lay::TP + tc::tile_offset(128, 64 + r, (i0 >> 3) + cc), a + 8 * cc);
+          st_chunk_s(sp + Lay::TP + tc::tile_offset(128, 64 + r, (i0 >> 3) + cc), a + 8 * cc);
       }
     }
     tc::fence_smem_to_async();
@@ -493,9 +492,11 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
         w.z = fmaf(a, zv.z, w.z); w.w = fmaf(a, zv.w, w.w);
       }
       *reinterpret_cast<float4 *>(s_X + (32 + r2) * kLd + c2) = make_float4(-w.x, -w.y, -w.z, -w.w);
+      if (tid == 0) bulk_wait_read();   // the P copy has left rows 64..127 of TP
       __syncthreads();
     }
-    // T_ri = X_ri beta_i (i <= r) as rows 0..63 of the K-major A tile.
+    // T_ri = X_ri beta_i (i <= r), in rows 0..63 and again in rows 64..127 of the
+    // K-major A tile, so that the product rows reach all four TMEM lane quadrants.
     for (int e = tid; e < 64 * 8; e += kThreads) {
       const int row = e >> 3, ch = e & 7;
       float val[8];
@@ -504,17 +505,17 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
         const int i = 8 * ch + u;
         val[u] = i <= row ? s_X[row * kLd + i] * s_beta[i] : 0.f;
       }
-      tc::st_chunk(sb + Lay::TP + tc::tile_offset(128, row, ch), val);
+      st_chunk_s(sp + Lay::TP + tc::tile_offset(128, row, ch), val);
+      st_chunk_s(sp + Lay::TP + tc::tile_offset(128, 64 + row, ch), val);
     }
     tc::fence_smem_to_async();
     if (__syncthreads_or(!wait_timed(vbar, vphase, wait_ns))) { aborted = true; break; }
     vphase ^= 1;
 
     // ---------------- W = T Ktilde (columns 0..127), U = T V (128..255) ----------------
-    // Rows 64..127 of the A tile hold P, not T; the rows they produce are never read.
+    // Rows 64..127 of the A tile repeat T: TMEM lanes 64..127 get a copy of the product.
     if (tid == 0) {
       tc::fence_after_sync();
-      bulk_wait_read();   // the P copy has left TP (the epilogue stages U there)
       constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 1);
 #pragma unroll
       for (int s2 = 0; s2 < 4; ++s2)
@@ -531,20 +532,19 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
     tc::fence_after_sync();
     // The staging region is free again: start the next item's loads.
     if (p + (int)gridDim.x < total) {
-      const Item nx = decode_item(p + gridDim.x, s_pref, cu, N, H, jw0);
+      const Item nx = decode_item(p + gridDim.x, s_pref, s_cu, N, H, jw0);
       intra_issue_loads(sb, maps, beta, nx.t0, nx.L, H, nx.h, tid);
     }
-    if (qd < 2) {   // TMEM lanes 0..63 = tokens; hw 0: W -> KT tile, hw 1: U -> TP tile
-      const int r = 32 * qd + lane;
-      const uint32_t dst = sb + (hw ? Lay::TP : Lay::KT);
-      float a[32];
+    {   // Each warp takes one 64-column quarter of [W | U] (W -> KT tile, U -> TP tile)
+        // for 32 tokens: quadrants 0, 1 read lanes 0..63, quadrants 2, 3 the copy.
+      const int r = 32 * (qd & 1) + lane, quarter = 2 * (qd >> 1) + hw;
+      const uint32_t dst = sb + (quarter >= 2 ? Lay::TP : Lay::KT) + (quarter & 1) * 8192;
+      float a[64];
+      tc::tmem_ld32(tl + 64 * quarter, *reinterpret_cast<float(*)[32]>(a));
+      tc::tmem_ld32(tl + 64 * quarter + 32, *reinterpret_cast<float(*)[32]>(a + 32));
+      tc::tmem_wait_ld();
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        tc::tmem_ld32(tl + 128 * hw + 32 * u, a);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) tc::st_chunk(dst + tc::tile_offset(64, r, 4 * u + cc), a + 8 * cc);
-      }
+      for (int cc = 0; cc < 8; ++cc) st_chunk_s(sp + (dst - sb) + tc::tile_offset(64, r, cc), a + 8 * cc);
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
@@ -554,9 +554,7 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
       bulk_store(pk + Packet::WQ + 16384, sb + Lay::KT + 8192, 8192);
       bulk_store(pk + Packet::U, sb + Lay::TP, 16384);
       bulk_commit();
-      bulk_wait_read();   // KT and TP are rewritten by the next item's prep
     }
-    __syncthreads();
   }
   if (tid == 0) bulk_wait_all();
 
@@ -700,7 +698,7 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
       tc::tmem_st32(s_tm + 32 * u, x);
 #pragma unroll
       for (int j = 0; j < 32; j += 8)
-        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + 32 * u + j) >> 3), x + j);
+        st_chunk_s(sp + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + 32 * u + j) >> 3), x + j);
     }
     tc::tmem_wait_st();
   }
@@ -738,7 +736,7 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
 #pragma unroll
     for (int cc = 0; cc < NCOL / 8; ++cc) {
       const int c = hw * (NCOL / 8) + cc;
-      tc::st_chunk(sb + Lay::OBUF + r * (DVS * 2) + ((c ^ (r & 7)) << 4), a + 8 * cc);
+      st_chunk_s(sp + Lay::OBUF + r * (DVS * 2) + ((c ^ (r & 7)) << 4), a + 8 * cc);
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");   // the four O warps
     const int t = 32 * ((qd - 2) + 2 * hw) + lane;
@@ -804,7 +802,7 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
         unpack8(uu, xv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) xv[e] -= a[8 * cc + e];
-        tc::st_chunk(sb + Lay::VN + tc::tile_offset(64, r, chunk), xv);
+        st_chunk_s(sp + Lay::VN + tc::tile_offset(64, r, chunk), xv);
       }
     }
     tc::fence_smem_to_async();
@@ -847,7 +845,7 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
         tc::tmem_st32(s_tm + 32 * u, *reinterpret_cast<float(*)[32]>(sv + 32 * u));
 #pragma unroll
       for (int jj = 0; jj < NCOL; jj += 8)
-        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + jj) >> 3), sv + jj);
+        st_chunk_s(sp + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + jj) >> 3), sv + jj);
       tc::tmem_wait_st();
       since_ck += L;
       if (interval > 0 && since_ck == interval) {
