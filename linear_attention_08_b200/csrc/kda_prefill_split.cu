@@ -64,10 +64,10 @@ struct IntraLayout {
   // rows of the Gram A tile that their scaled versions replace; g, fp32, in
   // the upper half); the Gram operands and the gate factors; the solve
   // scratch and the V tile.
-  static constexpr uint32_t STG_G = 32768;
-  static constexpr uint32_t GA = 0;          // [128][128] Gram A, K-major: k rows 0..63, q rows 64..127
-  static constexpr uint32_t GB = 32768;      // [96][128]  Gram B, K-major
-  static constexpr uint32_t CST = 57344;     // float [2][6][128] gate factors
+  static constexpr uint32_t STG_G = 0;       // float [64][128] g
+  static constexpr uint32_t GA = 32768;      // [128][128] Gram A, K-major: k rows 0..63, q rows 64..127
+  static constexpr uint32_t GB = 0;          // [96][128]  Gram B, K-major (over the consumed g)
+  static constexpr uint32_t CST = 24576;     // float [2][6][128] gate factors
   static constexpr uint32_t MM = 0;          // float [64][68] M
   static constexpr uint32_t XM = 17408;      // float [64][68] (I + M)^-1
   static constexpr uint32_t YS = 34816;      // float [2][16][17]
@@ -81,12 +81,15 @@ struct IntraLayout {
   static constexpr uint32_t PREF = BETA + 256;                    // int [kMaxSeqs + 1]
   static constexpr uint32_t CUS = PREF + 4 * (kMaxSeqs + 1);      // int [kMaxSeqs + 1] cu_seqlens
   static constexpr uint32_t BAR = (CUS + 4 * (kMaxSeqs + 1) + 7) & ~7u;    // MMA completion
-  static constexpr uint32_t TBAR = BAR + 8;                       // q, k, g landed
+  static constexpr uint32_t TBAR = BAR + 8;                       // q, k landed
   static constexpr uint32_t VBAR = BAR + 16;                      // v landed
-  static constexpr uint32_t TMEM_SLOT = BAR + 24;
-  static constexpr uint32_t TOTAL = BAR + 32;
+  static constexpr uint32_t GBAR = BAR + 24;                      // g landed
+  static constexpr uint32_t TMEM_SLOT = BAR + 32;
+  static constexpr uint32_t TOTAL = BAR + 40;
   static_assert(MT + 32 * 33 * 4 <= VT, "solve scratch overlaps the V tile");
-  static_assert(CST + 6144 <= 65536, "gate factors overflow the staging region");
+  static_assert(VT >= GA && VT + 16384 <= GA + 32768, "the V tile must lie in the consumed Gram A tile");
+  static_assert(MT + 32 * 33 * 4 <= 65536 && STG_G + 32768 <= GA, "g staging and the solve scratch");
+  static_assert(CST + 6144 <= GA, "gate factors overflow into the Gram A tile");
   static_assert(GB + 96 * 256 <= CST, "Gram B overlaps the gate factors");
 };
 
@@ -111,21 +114,15 @@ __device__ __forceinline__ int64_t window_chunks(const int32_t *cu, int n, int64
   return c <= 0 ? 0 : (c < wc ? c : wc);
 }
 
-// q and k come through maps with the v layout (box 64 x 64, 128-byte swizzle):
-// each box is one 64-row column block, i.e. rows 0..63 (k) or 64..127 (q) of a
-// column block of the Gram A tile.
-__device__ __forceinline__ void intra_issue_loads(uint32_t sb, const TmaMaps &maps,
-                                                  const float *beta, int64_t t0, int L, int H,
-                                                  int h, int tid) {
+// g (fp32, staging rows of 512 bytes) and beta (4-byte async copies, zero
+// past L): needed first by the next chunk, and their space is free once T is
+// formed.
+__device__ __forceinline__ void intra_issue_g(uint32_t sb, const TmaMaps &maps, const float *beta,
+                                              int64_t t0, int L, int H, int h, int tid) {
   using Lay = IntraLayout;
   if (tid == 32) {
-    const uint32_t bar = sb + Lay::TBAR;
-    mbar_expect_tx(bar, 64 * (256 + 256 + 512));
-#pragma unroll
-    for (int b = 0; b < 2; ++b) {
-      tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h, (int)t0, bar);
-      tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h, (int)t0, bar);
-    }
+    const uint32_t bar = sb + Lay::GBAR;
+    mbar_expect_tx(bar, 64 * 512);
     tma_load_3d(sb + Lay::STG_G, &maps.g, 0, h, (int)t0, bar);
   }
   if (tid >= 64 && tid < 64 + kC) {
@@ -134,6 +131,24 @@ __device__ __forceinline__ void intra_issue_loads(uint32_t sb, const TmaMaps &ma
     cp_async4(sb + Lay::BETA + 4 * r, beta + (ok ? (size_t)(t0 + r) * H + h : 0), ok);
   }
   cp_async_commit();
+}
+
+// q and k come through maps with the v layout (box 64 x 64, 128-byte swizzle):
+// each box is one 64-row column block, i.e. rows 0..63 (k) or 64..127 (q) of a
+// column block of the Gram A tile, whose space holds the V tile until the last
+// product of the previous chunk is done.
+__device__ __forceinline__ void intra_issue_qk(uint32_t sb, const TmaMaps &maps, int64_t t0,
+                                               int h, int tid) {
+  using Lay = IntraLayout;
+  if (tid == 32) {
+    const uint32_t bar = sb + Lay::TBAR;
+    mbar_expect_tx(bar, 64 * 512);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h, (int)t0, bar);
+      tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h, (int)t0, bar);
+    }
+  }
 }
 
 // Work item p of the window -> (sequence, head, chunk); see the packet order
@@ -212,10 +227,12 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
   const int total = s_pref[N];
   if ((int)blockIdx.x >= total) return;
 
+  uint64_t *gbar = reinterpret_cast<uint64_t *>(sp + Lay::GBAR);
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(tbar, 1);
     mbar_init(vbar, 1);
+    mbar_init(gbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.q)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.g)) : "memory");
@@ -227,44 +244,49 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
   const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
 
-  uint32_t phase = 0, tphase = 0, vphase = 0;
+  uint32_t phase = 0, tphase = 0, vphase = 0, gphase = 0;
   bool aborted = false;
   int p = blockIdx.x;
   {
     const Item it = decode_item(p, s_pref, s_cu, N, H, jw0);
-    intra_issue_loads(sb, maps, beta, it.t0, it.L, H, it.h, tid);
+    intra_issue_g(sb, maps, beta, it.t0, it.L, H, it.h, tid);
+    intra_issue_qk(sb, maps, it.t0, it.h, tid);
   }
 
   for (; p < total; p += gridDim.x) {
     const Item it = decode_item(p, s_pref, s_cu, N, H, jw0);
+    const bool more = p + (int)gridDim.x < total;
+    const Item nx = decode_item(more ? p + (int)gridDim.x : p, s_pref, s_cu, N, H, jw0);
     const int L = it.L, h = it.h;
     uint8_t *pk = ws + (size_t)p * Packet::BYTES;
 
     cp_async_wait_all();
     if (tid == 0) bulk_wait_read();   // the previous item's W and U have left KT and TP
-    if (__syncthreads_or(!wait_timed(tbar, tphase, wait_ns))) { aborted = true; break; }
-    tphase ^= 1;
+    if (__syncthreads_or(!wait_timed(gbar, gphase, wait_ns))) { aborted = true; break; }
+    gphase ^= 1;
 
     // ---------------- gate prep ----------------
-    // Warp w owns rows 8w..8w+7 (half hf = w / 4), lane l owns channels 4l..4l+3:
-    // per row one 8-byte piece of each 16-byte tile chunk, and the gate factors
-    // of the lane's channels stay in registers for all its rows.
+    // Warp w owns rows 8w..8w+7 (half hf = w / 4), lane l owns channels 4l..4l+3
+    // (two pairs, handled by the paired FP32 instructions, each lane of which
+    // rounds like the scalar one): per row one 8-byte piece of each 16-byte tile
+    // chunk; the gate factors of the lane's channels stay in registers.
     {
       const int hf = warp >> 2, cq = lane >> 1, sub = (lane & 1) * 8;
-      float gm[8][4];
+      float2 gm[8][2];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = 8 * warp + i;
         const float4 a = r < L ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + lane * 16)
                                : make_float4(0.f, 0.f, 0.f, 0.f);
-        gm[i][0] = a.x; gm[i][1] = a.y; gm[i][2] = a.z; gm[i][3] = a.w;
+        gm[i][0] = make_float2(a.x, a.y);
+        gm[i][1] = make_float2(a.z, a.w);
       }
 #pragma unroll
       for (int i = 1; i < 8; ++i)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) gm[i][e] += gm[i - 1][e];
+        for (int j = 0; j < 2; ++j) gm[i][j] = __fadd2_rn(gm[i][j], gm[i - 1][j]);
       *reinterpret_cast<float4 *>(s_red + warp * 128 + 4 * lane) =
-          make_float4(gm[7][0], gm[7][1], gm[7][2], gm[7][3]);
+          make_float4(gm[7][0].x, gm[7][0].y, gm[7][1].x, gm[7][1].y);
       __syncthreads();
       // One lane per channel: exclusive scan of the 8 row-group totals, the cumulative
       // decay at rows 15, 31, 47, 63, and the channel's gate factors for both halves.
@@ -281,43 +303,53 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
         // Row r of half hf is scaled against ref = Gam_15 (hf 0) or Gam_47 (hf 1);
         // the products are grouped exactly as in the fused kernel (no intermediate
         // underflows unless the exact value is itself far below the BF16 rounding).
+        // Slots: -ref, fk, fk2, fh, fh2, cb; fk = 1 in the first half and fh2 = 1 in
+        // the second, so (x fk) fk2 and (y fh) fh2 serve both halves exactly.
         float f[12];
-        f[0] = G15; f[1] = 1.f; f[2] = __expf(G15);
+        f[0] = -G15; f[1] = 1.f; f[2] = __expf(G15);
         f[3] = __expf(G31 - G15); f[4] = __expf(G63 - G31); f[5] = __expf(G47 - G15);
-        f[6] = G47; f[7] = __expf(G47 - G31); f[8] = __expf(G31);
+        f[6] = -G47; f[7] = __expf(G47 - G31); f[8] = __expf(G31);
         f[9] = __expf(G63 - G47); f[10] = 1.f; f[11] = 0.f;
 #pragma unroll
         for (int j = 0; j < 12; ++j) s_cst[j * 128 + ch] = f[j];
         reinterpret_cast<float *>(pk + Packet::D)[ch] = __expf(G63);
       }
-      __syncthreads();
-      float ref[4], fk[4], fk2[4], fh[4], fh2[4], cb[4];
+      // q and k must have landed too before the rows are scaled.
+      if (__syncthreads_or(!wait_timed(tbar, tphase, wait_ns))) { aborted = true; break; }
+      tphase ^= 1;
+      float2 nref[2], fk[2], fk2[2], fh[2], fh2[2], cb[2];
       {
-        auto ld4 = [&](int j, float *d4) {
+        auto ld4 = [&](int j, float2 *d) {
           const float4 v = *reinterpret_cast<const float4 *>(s_cst + (hf * 6 + j) * 128 + 4 * lane);
-          d4[0] = v.x; d4[1] = v.y; d4[2] = v.z; d4[3] = v.w;
+          d[0] = make_float2(v.x, v.y);
+          d[1] = make_float2(v.z, v.w);
         };
-        float base[4];
+        float2 base[2];
         const float4 bv = *reinterpret_cast<const float4 *>(s_red + warp * 128 + 4 * lane);
-        base[0] = bv.x; base[1] = bv.y; base[2] = bv.z; base[3] = bv.w;
+        base[0] = make_float2(bv.x, bv.y);
+        base[1] = make_float2(bv.z, bv.w);
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) gm[i][e] += base[e];
-        ld4(0, ref); ld4(1, fk); ld4(2, fk2); ld4(3, fh); ld4(4, fh2); ld4(5, cb);
+          for (int j = 0; j < 2; ++j) gm[i][j] = __fadd2_rn(gm[i][j], base[j]);
+        ld4(0, nref); ld4(1, fk); ld4(2, fk2); ld4(3, fh); ld4(4, fh2); ld4(5, cb);
       }
-      auto st4 = [&](uint8_t *dst, const float *x) {
-        *reinterpret_cast<uint2 *>(dst) = make_uint2(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]));
+      auto st4 = [&](uint8_t *dst, const float2 *x) {
+        *reinterpret_cast<uint2 *>(dst) = make_uint2(tc::pack_bf16(x[0].x, x[0].y), tc::pack_bf16(x[1].x, x[1].y));
       };
-      auto un4 = [&](const uint2 &u, float *x) {
-        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-        x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+      auto un4 = [&](const uint2 &u, float2 *x) {
+        x[0] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        x[1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+      };
+      auto rcp = [](float v) {   // hardware reciprocal approximation; v is normal here
+        float r;
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+        return r;
       };
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int r = 8 * warp + i;
-        float kk[4], qq[4], x[4], y[4], t[4];
+        float2 kk[2], qq[2], x[2], y[2], t[2];
         {   // raw k and q of this row, replaced below by k x and q x
           const bool in = r < L;
           const uint2 z2 = make_uint2(0, 0);
@@ -327,39 +359,37 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
           un4(qv, qq);
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[e] = __expf(gm[i][e] - ref[e]);
-          // reciprocal by two Newton steps from the bit-level initial guess
-          float r0 = __int_as_float(0x7EF311C3 - __float_as_int(x[e]));
-          r0 = r0 * fmaf(-x[e], r0, 2.f);
-          y[e] = r0 * fmaf(-x[e], r0, 2.f);
+        for (int j = 0; j < 2; ++j) {
+          const float2 d = __fadd2_rn(gm[i][j], nref[j]);
+          x[j] = make_float2(__expf(d.x), __expf(d.y));   // exp(Gam_r - ref), within [e^-80, e^80]
+          y[j] = make_float2(rcp(x[j].x), rcp(x[j].y));   // exp(ref - Gam_r)
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) t[e] = kk[e] * x[e];
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], x[j]);
         st4(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) t[e] = qq[e] * x[e];
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(qq[j], x[j]);
         st4(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) t[e] = kk[e] * y[e];
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], y[j]);
         st4(sp + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, cq) + sub, t);
         if (!hf) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) t[e] = kk[e] * (y[e] * cb[e]);
+          for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], __fmul2_rn(y[j], cb[j]));
           st4(sp + Lay::GB + tc::tile_offset(96, 32 + r, cq) + sub, t);
         }
-        // Ktilde, Qtilde: exp(Gam_r) = (x fk) fk2; fk = 1 in the first half.
+        // Ktilde, Qtilde: exp(Gam_r) = (x fk) fk2.
 #pragma unroll
-        for (int e = 0; e < 4; ++e) x[e] = hf ? (x[e] * fk[e]) * fk2[e] : x[e] * fk2[e];
+        for (int j = 0; j < 2; ++j) x[j] = __fmul2_rn(__fmul2_rn(x[j], fk[j]), fk2[j]);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) t[e] = kk[e] * x[e];
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], x[j]);
         st4(sp + Lay::KT + tc::tile_offset(64, r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) t[e] = qq[e] * x[e];
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(qq[j], x[j]);
         st4(pk + Packet::WQ + tc::tile_offset(128, 64 + r, cq) + sub, t);
-        // Khat: exp(Gam_last - Gam_r) = (y fh) fh2; fh2 = 1 in the second half.
+        // Khat: exp(Gam_last - Gam_r) = (y fh) fh2.
 #pragma unroll
-        for (int e = 0; e < 4; ++e) t[e] = kk[e] * (hf ? y[e] * fh[e] : (y[e] * fh[e]) * fh2[e]);
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], __fmul2_rn(__fmul2_rn(y[j], fh[j]), fh2[j]));
         st4(pk + Packet::KH + tc::tile_offset(64, r, cq) + sub, t);
       }
       tc::fence_smem_to_async();
@@ -398,11 +428,12 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
         tc::tmem_wait_ld();
       }
       const bool zero = !second && hw;
-      if (part == 0) {
+      if (part == 0) {   // 16-byte stores: rows are 272 bytes apart, so 8 lanes hit 8 distinct slots
         const float br = s_beta[r];
-        float *dst = s_M + r * kLd + i0;
+        float4 *dst = reinterpret_cast<float4 *>(s_M + r * kLd + i0);
+        auto mv = [&](int j) { return (!zero && i0 + j < r) ? br * a[j] : 0.f; };
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dst[j] = (!zero && i0 + j < r) ? br * a[j] : 0.f;
+        for (int j = 0; j < 32; j += 4) dst[j >> 2] = make_float4(mv(j), mv(j + 1), mv(j + 2), mv(j + 3));
         if (second && i0 == 0)
 #pragma unroll
           for (int j = 0; j < 32; ++j) s_MT[j * 33 + (r - 32)] = br * a[j];
@@ -511,6 +542,8 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
     tc::fence_smem_to_async();
     if (__syncthreads_or(!wait_timed(vbar, vphase, wait_ns))) { aborted = true; break; }
     vphase ^= 1;
+    // The solve scratch and beta are consumed: the next item's g and beta may land.
+    if (more) intra_issue_g(sb, maps, beta, nx.t0, nx.L, H, nx.h, tid);
 
     // ---------------- W = T Ktilde (columns 0..127), U = T V (128..255) ----------------
     // Rows 64..127 of the A tile repeat T: TMEM lanes 64..127 get a copy of the product.
@@ -530,11 +563,8 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
     if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
     phase ^= 1;
     tc::fence_after_sync();
-    // The staging region is free again: start the next item's loads.
-    if (p + (int)gridDim.x < total) {
-      const Item nx = decode_item(p + gridDim.x, s_pref, s_cu, N, H, jw0);
-      intra_issue_loads(sb, maps, beta, nx.t0, nx.L, H, nx.h, tid);
-    }
+    // The V tile is consumed: the next item's q and k may land in the Gram A tile.
+    if (more) intra_issue_qk(sb, maps, nx.t0, nx.h, tid);
     {   // Each warp takes one 64-column quarter of [W | U] (W -> KT tile, U -> TP tile)
         // for 32 tokens: quadrants 0, 1 read lanes 0..63, quadrants 2, 3 the copy.
       const int r = 32 * (qd & 1) + lane, quarter = 2 * (qd >> 1) + hw;
@@ -564,6 +594,7 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
     wait_timed(bar, phase, wait_ns);
     wait_timed(tbar, tphase, wait_ns);
     wait_timed(vbar, vphase, wait_ns);
+    wait_timed(gbar, gphase, wait_ns);
   }
   tc::fence_before_sync();
   __syncthreads();
