@@ -6,7 +6,7 @@ decode workload (512 sequences x 32 heads, 256 steps captured in one CUDA
 graph, FP32 state N(0, 0.02)) as a second object on the same line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload prefill|decode|append_varlen|long] [--no-decode]
+                  [--workload prefill|decode|append_varlen|long|prefill_small] [--no-decode]
 
 For N > 1 it is launched by torchrun, one rank per GPU; every rank runs its
 own copy of the workload (the operator's (sequence, head) units are
@@ -283,11 +283,27 @@ def time_prefill(name, steps, warmup, world, local):
     tokens = sum(lengths)
     flops, byts = prefill_algorithmic(lengths, H, Dk, Dv, C, 2 if w["dtype"] == "bf16" else 4,
                                       interval, init is not None)
-    path = kda.kda_prefill_path(kda.make_shape(len(lengths), tokens, H, Dk, Dv, C,
-                                               1 if w["dtype"] == "bf16" else 0))
+    shape = kda.make_shape(len(lengths), tokens, H, Dk, Dv, C, 1 if w["dtype"] == "bf16" else 0)
+    path = kda.kda_prefill_path(shape)
+    launches = 1
+    if path == 2:   # one intra-chunk pass and one chain pass per window of chunks
+        ws = kda.workspace_for(shape, "meta")
+        launches = 2 * prefill_windows(len(lengths), H, tokens, ws.numel(),
+                                       kda.kda_prefill_workspace_bytes(shape))
     return dict(tokens=tokens, steps=steps, total_ms=total_ms, launch_ms=launch_ms,
+                launches_per_step=launches,
                 e2e_ms=e2e_ms, bi=bi, bo=bo, flops=flops, bytes=byts, clocks=clk.result,
                 kernel=PATH_KERNEL[path], w=w, lengths=lengths)
+
+
+def prefill_windows(N, H, T, ws_bytes, full_bytes, packet=74240, chunk=64):
+    """Windows of chunks the two-pass prefill runs for a workspace of ws_bytes
+    (with a final-state buffer, as the benchmark passes one)."""
+    if ws_bytes >= full_bytes:
+        return 1
+    wc = (ws_bytes - 256) // (N * H * packet)
+    max_chunks = -(-T // chunk)
+    return -(-max_chunks // wc)
 
 
 def time_decode(steps_graph, warmup, world, local, decode_steps=None):
@@ -427,7 +443,7 @@ def run_ours(args, rank, world, local):
                          "algorithmic_flops_per_launch": r["flops"]},
             "e2e": {"value": world * r["tokens"] / (r["e2e_ms"] / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["bi"], "d2h_bytes_per_step": r["bo"]},
-            "gpu_launches": r["steps"],
+            "gpu_launches": r["steps"] * r["launches_per_step"],
             "clocks": r["clocks"],
         }
     if dec is not None:
@@ -539,7 +555,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill",
-                    choices=["prefill", "decode", "append_varlen", "long"])
+                    choices=["prefill", "decode", "append_varlen", "long", "prefill_small"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=0,
                     help="decode steps per graph (default: the workload's 256)")
