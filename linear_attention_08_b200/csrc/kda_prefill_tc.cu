@@ -71,7 +71,7 @@ struct Layout {
   static constexpr uint32_t G = KV_T + 64 * (128 + DVS) * 2;      // 72 KB region, used in turn for:
   static constexpr uint32_t STG_Q = G, STG_K = G + 16384;         //  next chunk's q, k [64][128] bf16
   static constexpr uint32_t STG_G = G + 32768;                    //  next chunk's g [64][128] fp32
-  static constexpr uint32_t RED = G + 65536;                      //  float [16][128] scan partials
+  static constexpr uint32_t RED = G + 65536;                      //  float [8][128] scan partials
   static constexpr uint32_t GA = G;                               //  Gram A [128][128] K-major
   static constexpr uint32_t GB = G + 32768;                       //  Gram B [96][128] K-major
   static constexpr uint32_t MM = G;                               //  float [64][68] M
@@ -238,142 +238,128 @@ prefill_tc_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict_
     tphase ^= 1;
 
     // ---------------- gate prep: cumulative decay and scaled operands ----------------
-    // Thread (rg, jc) owns rows 4rg..4rg+3 and channels 8jc..8jc+7 of the chunk.
+    // Warp w owns rows 8w..8w+7 (half hf = w / 4), lane l owns channels 4l..4l+3
+    // (two pairs, on the paired FP32 instructions, each lane of which rounds like
+    // the scalar one): per row one 8-byte piece of each 16-byte tile chunk; the
+    // gate factors of the lane's channels stay in registers for all its rows.
     {
-      const int rg = tid >> 4, jc = tid & 15, hf = rg >> 3;
-      float gm[4][8], kk[4][8], qq[4][8];
+      const int hf = warp >> 2, cq = lane >> 1, sub = (lane & 1) * 8;
+      float2 gm[8][2];
+      uint2 kv[8], qv[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 4 * rg + i;
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * warp + i;
         const bool in = r < L;
-        const uint4 z4 = make_uint4(0, 0, 0, 0);
-        const float4 zf = make_float4(0.f, 0.f, 0.f, 0.f);
-        const uint4 qv = in ? *reinterpret_cast<const uint4 *>(sp + Lay::STG_Q + r * 256 + jc * 16) : z4;
-        const uint4 kv = in ? *reinterpret_cast<const uint4 *>(sp + Lay::STG_K + r * 256 + jc * 16) : z4;
-        const float4 a = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + jc * 32) : zf;
-        const float4 b = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + jc * 32 + 16) : zf;
-        unpack8(qv, qq[i]);
-        unpack8(kv, kk[i]);
-        gm[i][0] = a.x; gm[i][1] = a.y; gm[i][2] = a.z; gm[i][3] = a.w;
-        gm[i][4] = b.x; gm[i][5] = b.y; gm[i][6] = b.z; gm[i][7] = b.w;
+        const float4 a = in ? *reinterpret_cast<const float4 *>(sp + Lay::STG_G + r * 512 + lane * 16)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        gm[i][0] = make_float2(a.x, a.y);
+        gm[i][1] = make_float2(a.z, a.w);
+        const uint2 z2 = make_uint2(0, 0);
+        kv[i] = in ? *reinterpret_cast<const uint2 *>(sp + Lay::STG_K + r * 256 + lane * 8) : z2;
+        qv[i] = in ? *reinterpret_cast<const uint2 *>(sp + Lay::STG_Q + r * 256 + lane * 8) : z2;
       }
 #pragma unroll
-      for (int i = 1; i < 4; ++i)
+      for (int i = 1; i < 8; ++i)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) gm[i][e] += gm[i - 1][e];
-      {
-        float4 *dst = reinterpret_cast<float4 *>(s_red + rg * 128 + 8 * jc);
-        dst[0] = make_float4(gm[3][0], gm[3][1], gm[3][2], gm[3][3]);
-        dst[1] = make_float4(gm[3][4], gm[3][5], gm[3][6], gm[3][7]);
-      }
+        for (int j = 0; j < 2; ++j) gm[i][j] = __fadd2_rn(gm[i][j], gm[i - 1][j]);
+      *reinterpret_cast<float4 *>(s_red + warp * 128 + 4 * lane) =
+          make_float4(gm[7][0].x, gm[7][0].y, gm[7][1].x, gm[7][1].y);
       __syncthreads();
-      // Exclusive scan of the 16 row-group totals, channel by channel: warp w scans
-      // channels 16w..16w+15; lane (ch, half) holds row groups 8*half..8*half+7.
-      // The same lanes form each channel's gate factors once (for both halves).
-      {
-        const int ch = 16 * warp + (lane & 15), half = lane >> 4;
-        float t[8], run = 0.f;
+      // One lane per channel: exclusive scan of the 8 row-group totals, the cumulative
+      // decay at rows 15, 31, 47, 63 and the channel's gate factors for both halves.
+      if (tid < 128) {
+        const int ch = tid;
+        float t[8], run = 0.f, incl[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) t[i] = s_red[(8 * half + i) * 128 + ch];
-        float incl[8];
+        for (int i = 0; i < 8; ++i) t[i] = s_red[i * 128 + ch];
 #pragma unroll
         for (int i = 0; i < 8; ++i) { run += t[i]; incl[i] = run; }
-        const float lower = __shfl_sync(0xffffffffu, run, lane & 15);   // half 0's total
-        const float off = half ? lower : 0.f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) s_red[(8 * half + i) * 128 + ch] = off + incl[i] - t[i];
-        // cumulative decay at rows 15, 31 (half 0) and 47, 63 (half 1)
-        const float ga = off + incl[3], gb = off + incl[7];
-        const float G15 = __shfl_sync(0xffffffffu, ga, lane & 15);
-        const float G31 = __shfl_sync(0xffffffffu, gb, lane & 15);
-        const float G47 = __shfl_sync(0xffffffffu, ga, (lane & 15) + 16);
-        const float G63 = __shfl_sync(0xffffffffu, gb, (lane & 15) + 16);
+        for (int i = 0; i < 8; ++i) s_red[i * 128 + ch] = incl[i] - t[i];
+        const float G15 = incl[1], G31 = incl[3], G47 = incl[5], G63 = incl[7];
         // Row r of half hf is scaled against ref = Gam_15 (hf 0) or Gam_47 (hf 1):
         // x = exp(Gam_r - ref), y = 1/x, both within [e^-80, e^80].  Products are
         // grouped so that an intermediate can only underflow when the exact value
         // is itself below e^-87 (or, for the B^(1) rows of the first half and
         // Ktilde of the second, below e^-12 times a unit-norm product).
-        float f[6];
-        if (half == 0) {
-          f[0] = G15;                       // ref
-          f[1] = 1.f;                       // Ktilde: (x * 1) * exp(Gam_15)
-          f[2] = __expf(G15);
-          f[3] = __expf(G31 - G15);         // Khat: (y * exp(Gam_31 - Gam_15)) * exp(Gam_63 - Gam_31)
-          f[4] = __expf(G63 - G31);
-          f[5] = __expf(G47 - G15);         // B^(1) rows of the first half
-        } else {
-          f[0] = G47;
-          f[1] = __expf(G47 - G31);         // Ktilde: (x * exp(Gam_47 - Gam_31)) * exp(Gam_31)
-          f[2] = __expf(G31);
-          f[3] = __expf(G63 - G47);         // Khat: y * exp(Gam_63 - Gam_47)
-          f[4] = 1.f;
-          f[5] = 0.f;
-          s_dvec[ch] = __expf(G63);
-        }
+        // Slots: -ref, fk, fk2, fh, fh2, cb; fk = 1 in the first half and fh2 = 1 in
+        // the second, so (x fk) fk2 and (y fh) fh2 serve both halves exactly.
+        float f[12];
+        f[0] = -G15; f[1] = 1.f; f[2] = __expf(G15);
+        f[3] = __expf(G31 - G15); f[4] = __expf(G63 - G31); f[5] = __expf(G47 - G15);
+        f[6] = -G47; f[7] = __expf(G47 - G31); f[8] = __expf(G31);
+        f[9] = __expf(G63 - G47); f[10] = 1.f; f[11] = 0.f;
 #pragma unroll
-        for (int j = 0; j < 6; ++j) s_cst[(half * 6 + j) * 128 + ch] = f[j];
+        for (int j = 0; j < 12; ++j) s_cst[j * 128 + ch] = f[j];
+        s_dvec[ch] = __expf(G63);
       }
       __syncthreads();
-      float base[8], ref[8], fk[8], fk2[8], fh[8], fh2[8], cb[8];
+      float2 nref[2], fk[2], fk2[2], fh[2], fh2[2], cb[2];
       {
-        // 128-bit reads: 16 threads cover 512 contiguous bytes, no bank conflicts
-        auto ld8 = [&](const float *src, float *d8) {
-          const float4 a = reinterpret_cast<const float4 *>(src)[0];
-          const float4 b = reinterpret_cast<const float4 *>(src)[1];
-          d8[0] = a.x; d8[1] = a.y; d8[2] = a.z; d8[3] = a.w;
-          d8[4] = b.x; d8[5] = b.y; d8[6] = b.z; d8[7] = b.w;
+        auto ld4 = [&](int j, float2 *d) {
+          const float4 v = *reinterpret_cast<const float4 *>(s_cst + (hf * 6 + j) * 128 + 4 * lane);
+          d[0] = make_float2(v.x, v.y);
+          d[1] = make_float2(v.z, v.w);
         };
-        const float *c = s_cst + hf * 6 * 128 + 8 * jc;
-        ld8(s_red + rg * 128 + 8 * jc, base);
-        ld8(c + 0 * 128, ref);
-        ld8(c + 1 * 128, fk);
-        ld8(c + 2 * 128, fk2);
-        ld8(c + 3 * 128, fh);
-        ld8(c + 4 * 128, fh2);
-        ld8(c + 5 * 128, cb);
+        const float4 bv = *reinterpret_cast<const float4 *>(s_red + warp * 128 + 4 * lane);
+        const float2 base[2] = {make_float2(bv.x, bv.y), make_float2(bv.z, bv.w)};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) gm[i][j] = __fadd2_rn(gm[i][j], base[j]);
+        ld4(0, nref); ld4(1, fk); ld4(2, fk2); ld4(3, fh); ld4(4, fh2); ld4(5, cb);
       }
+      auto st4 = [&](uint32_t off, const float2 *x) {
+        *reinterpret_cast<uint2 *>(sp + off) = make_uint2(tc::pack_bf16(x[0].x, x[0].y), tc::pack_bf16(x[1].x, x[1].y));
+      };
+      auto un4 = [&](const uint2 &u, float2 *x) {
+        x[0] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+        x[1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+      };
+      auto rcp = [](float v) {   // hardware reciprocal approximation; v is normal here
+        float r;
+        asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+        return r;
+      };
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
+      for (int i = 0; i < 8; ++i) {
+        const int r = 8 * warp + i;
+        float2 kk[2], qq[2], x[2], y[2], t[2];
+        un4(kv[i], kk);
+        un4(qv[i], qq);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) gm[i][e] += base[e];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = 4 * rg + i;
-        float x[8], y[8], t[8], kt[8], kh[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          x[e] = __expf(gm[i][e] - ref[e]);
-          // reciprocal by two Newton steps from the bit-level initial guess
-          float r0 = __int_as_float(0x7EF311C3 - __float_as_int(x[e]));
-          r0 = r0 * fmaf(-x[e], r0, 2.f);
-          y[e] = r0 * fmaf(-x[e], r0, 2.f);
-          // exp(Gam_r) and exp(Gam_63 - Gam_r); fk = 1 in the first half, fh2 = 1 in the second
-          kt[e] = hf ? (x[e] * fk[e]) * fk2[e] : x[e] * fk2[e];
-          kh[e] = hf ? y[e] * fh[e] : (y[e] * fh[e]) * fh2[e];
+        for (int j = 0; j < 2; ++j) {
+          const float2 d = __fadd2_rn(gm[i][j], nref[j]);
+          x[j] = make_float2(__expf(d.x), __expf(d.y));
+          y[j] = make_float2(rcp(x[j].x), rcp(x[j].y));
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * x[e];
-        tc::st_chunk(sb + Lay::GA + tc::tile_offset(128, r, jc), t);
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], x[j]);
+        st4(Lay::GA + tc::tile_offset(128, r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * x[e];
-        tc::st_chunk(sb + Lay::GA + tc::tile_offset(128, 64 + r, jc), t);
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(qq[j], x[j]);
+        st4(Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * y[e];
-        tc::st_chunk(sb + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, jc), t);
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], y[j]);
+        st4(Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, cq) + sub, t);
         if (!hf) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * (y[e] * cb[e]);
-          tc::st_chunk(sb + Lay::GB + tc::tile_offset(96, 32 + r, jc), t);
+          for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], __fmul2_rn(y[j], cb[j]));
+          st4(Lay::GB + tc::tile_offset(96, 32 + r, cq) + sub, t);
         }
+        // Ktilde, Qtilde: exp(Gam_r) = (x fk) fk2.
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * kt[e];
-        tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, r, jc), t);
+        for (int j = 0; j < 2; ++j) x[j] = __fmul2_rn(__fmul2_rn(x[j], fk[j]), fk2[j]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = qq[i][e] * kt[e];
-        tc::st_chunk(sb + Lay::WQ_T + tc::tile_offset(128, 64 + r, jc), t);
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], x[j]);
+        st4(Lay::WQ_T + tc::tile_offset(128, r, cq) + sub, t);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = kk[i][e] * kh[e];
-        tc::st_chunk(sb + Lay::KH_T + tc::tile_offset(64, r, jc), t);
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(qq[j], x[j]);
+        st4(Lay::WQ_T + tc::tile_offset(128, 64 + r, cq) + sub, t);
+        // Khat: exp(Gam_63 - Gam_r) = (y fh) fh2.
+#pragma unroll
+        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], __fmul2_rn(__fmul2_rn(y[j], fh[j]), fh2[j]));
+        st4(Lay::KH_T + tc::tile_offset(64, r, cq) + sub, t);
       }
       tc::fence_smem_to_async();
       __syncthreads();
