@@ -51,6 +51,9 @@ def _bind(lib):
     lib.kda_oracle_recurrent_pos.argtypes = common + [P, P, P]
     lib.kda_oracle_recurrent_pos.restype = ctypes.c_int
     lib.kda_oracle_max_threads.restype = ctypes.c_int
+    lib.kda_oracle_backward.argtypes = [I64, P, I64, I64, I64, P, P, P, P, P, P, P, P, P, P, P, P,
+                                        P, P, ctypes.c_int]
+    lib.kda_oracle_backward.restype = ctypes.c_int
     return lib
 
 
@@ -148,3 +151,30 @@ def decode(q, k, v, g, beta, init_state, nthreads: int = 0, lib=None):
                           seq_major(beta), cu, init_state, 0, 0, nthreads, lib)
     out = np.ascontiguousarray(np.swapaxes(out.reshape(N, steps, H, Dv), 0, 1))
     return out, fin
+
+
+def backward(q, k, v, g, beta, cu_seqlens, d_out, init_state=None, d_final=None,
+             nthreads: int = 0, lib=None):
+    """Gradients of the recurrence (FP64) for an upstream gradient d_out
+    [T_tot, H, Dv] on the outputs and d_final [N, H, Dk, Dv] on the final
+    states (None = 0).  Returns (dq, dk, dv, dg, dbeta, d_init) as float64
+    numpy arrays with the shapes of the inputs."""
+    lib = lib or load()
+    q, k, v, g, beta, d_out = (_f64(a) for a in (q, k, v, g, beta, d_out))
+    init = _f64(init_state)
+    dfin = _f64(d_final)
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = len(cu) - 1
+    dq, dk, dg = (np.zeros((T, H, Dk)) for _ in range(3))
+    dv = np.zeros((T, H, Dv))
+    dbeta = np.zeros((T, H))
+    dinit = np.zeros((N, H, Dk, Dv))
+    rc = lib.kda_oracle_backward(N, _ptr(cu), H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                 _ptr(beta), _ptr(init), _ptr(d_out), _ptr(dfin), _ptr(dq),
+                                 _ptr(dk), _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(dinit),
+                                 int(nthreads))
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (status {rc})")
+    return dq, dk, dv, dg, dbeta, dinit

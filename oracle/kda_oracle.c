@@ -302,6 +302,151 @@ int kda_oracle_chunked(int64_t num_seqs, const int64_t *cu_seqlens, int64_t H, i
                out, final_state, ckpt_states, nthreads, chunk, NULL, NULL, NULL);
 }
 
+/*
+ * Backward pass of the recurrence (the training direction; the pages give no
+ * detail of it, so it is derived here from the forward definition above and
+ * pinned in the tests against central finite differences of the forward).
+ *
+ * Per token, with P_t = Diag(alpha_t) S_{t-1}, y_t = P_t^T k_t,
+ * u_t = beta_t (v_t - y_t), S_t = P_t + k_t u_t^T and o_t = S_t^T q_t, and
+ * dS the gradient of the loss with respect to S_t coming from later tokens
+ * (d_final_state for the last one):
+ *
+ *   dS    += q_t do_t^T                 dq_t   = S_t do_t
+ *   du     = dS^T k_t                   dk_t   = dS u_t - beta_t P_t du
+ *   dbeta_t = du . (v_t - y_t)          dv_t   = beta_t du
+ *   dP     = dS - beta_t k_t du^T       dg_t,c = alpha_t,c sum_j dP_cj S_{t-1,cj}
+ *   dS    <- Diag(alpha_t) dP           (the gradient with respect to S_{t-1})
+ *
+ * After the first token of a sequence dS is the gradient with respect to its
+ * initial state.  Arrays as for the forward (d_out [T_tot, H, Dv],
+ * d_final_state and d_init_state [N, H, Dk, Dv], either may be NULL).
+ */
+static void backward_unit(int64_t H, int64_t Dk, int64_t Dv, const double *q, const double *k,
+                          const double *v, const double *g, const double *beta,
+                          const double *init, const double *dout, const double *dfin,
+                          double *dq, double *dk, double *dv, double *dg, double *dbeta,
+                          double *dinit, const int64_t *cu, int64_t seq, int64_t h,
+                          double *states, double *dS, double *vec) {
+    const int64_t t0 = cu[seq], T = cu[seq + 1] - cu[seq], DD = Dk * Dv;
+    double *y = vec, *u = vec + Dv, *du = vec + 2 * Dv, *alpha = vec + 3 * Dv;
+    /* forward, keeping S_{t} for t = -1 .. T-1 (states[t + 1]) */
+    if (init) memcpy(states, init + (seq * H + h) * DD, sizeof(double) * (size_t)DD);
+    else memset(states, 0, sizeof(double) * (size_t)DD);
+    for (int64_t t = 0; t < T; ++t) {
+        const int64_t tt = t0 + t;
+        const double *kt = k + (tt * H + h) * Dk, *gt = g + (tt * H + h) * Dk;
+        const double *vt = v + (tt * H + h) * Dv;
+        const double bt = beta[tt * H + h];
+        const double *Sp = states + t * DD;
+        double *Sn = states + (t + 1) * DD;
+        for (int64_t c = 0; c < Dk; ++c) {
+            const double a = exp(gt[c]);
+            for (int64_t j = 0; j < Dv; ++j) Sn[c * Dv + j] = a * Sp[c * Dv + j];
+        }
+        for (int64_t j = 0; j < Dv; ++j) y[j] = 0.0;
+        for (int64_t c = 0; c < Dk; ++c)
+            for (int64_t j = 0; j < Dv; ++j) y[j] += Sn[c * Dv + j] * kt[c];
+        for (int64_t c = 0; c < Dk; ++c)
+            for (int64_t j = 0; j < Dv; ++j) Sn[c * Dv + j] += bt * kt[c] * (vt[j] - y[j]);
+    }
+    /* backward */
+    if (dfin) memcpy(dS, dfin + (seq * H + h) * DD, sizeof(double) * (size_t)DD);
+    else memset(dS, 0, sizeof(double) * (size_t)DD);
+    for (int64_t t = T - 1; t >= 0; --t) {
+        const int64_t tt = t0 + t;
+        const double *qt = q + (tt * H + h) * Dk, *kt = k + (tt * H + h) * Dk;
+        const double *gt = g + (tt * H + h) * Dk, *vt = v + (tt * H + h) * Dv;
+        const double *dot = dout + (tt * H + h) * Dv;
+        const double bt = beta[tt * H + h];
+        const double *Sp = states + t * DD, *Sn = states + (t + 1) * DD;
+        for (int64_t c = 0; c < Dk; ++c) alpha[c] = exp(gt[c]);
+        /* y and u of this token, from P = Diag(alpha) S_{t-1} */
+        for (int64_t j = 0; j < Dv; ++j) y[j] = 0.0;
+        for (int64_t c = 0; c < Dk; ++c)
+            for (int64_t j = 0; j < Dv; ++j) y[j] += alpha[c] * Sp[c * Dv + j] * kt[c];
+        for (int64_t j = 0; j < Dv; ++j) u[j] = bt * (vt[j] - y[j]);
+        /* o_t = S_t^T q_t */
+        double *dqt = dq + (tt * H + h) * Dk;
+        for (int64_t c = 0; c < Dk; ++c) {
+            double a = 0.0;
+            for (int64_t j = 0; j < Dv; ++j) a += Sn[c * Dv + j] * dot[j];
+            dqt[c] = a;
+        }
+        for (int64_t c = 0; c < Dk; ++c)
+            for (int64_t j = 0; j < Dv; ++j) dS[c * Dv + j] += qt[c] * dot[j];
+        /* S_t = P + k u^T */
+        for (int64_t j = 0; j < Dv; ++j) du[j] = 0.0;
+        for (int64_t c = 0; c < Dk; ++c)
+            for (int64_t j = 0; j < Dv; ++j) du[j] += dS[c * Dv + j] * kt[c];
+        double db = 0.0;
+        double *dvt = dv + (tt * H + h) * Dv;
+        for (int64_t j = 0; j < Dv; ++j) {
+            db += du[j] * (vt[j] - y[j]);
+            dvt[j] = bt * du[j];
+        }
+        dbeta[tt * H + h] = db;
+        double *dkt = dk + (tt * H + h) * Dk, *dgt = dg + (tt * H + h) * Dk;
+        for (int64_t c = 0; c < Dk; ++c) {
+            double a = 0.0, b = 0.0, da = 0.0;
+            for (int64_t j = 0; j < Dv; ++j) {
+                a += dS[c * Dv + j] * u[j];
+                b += alpha[c] * Sp[c * Dv + j] * du[j];
+                da += (dS[c * Dv + j] - bt * kt[c] * du[j]) * Sp[c * Dv + j];
+            }
+            dkt[c] = a - bt * b;
+            dgt[c] = alpha[c] * da;
+        }
+        /* the gradient with respect to S_{t-1} */
+        for (int64_t c = 0; c < Dk; ++c)
+            for (int64_t j = 0; j < Dv; ++j)
+                dS[c * Dv + j] = alpha[c] * (dS[c * Dv + j] - bt * kt[c] * du[j]);
+    }
+    if (dinit) memcpy(dinit + (seq * H + h) * DD, dS, sizeof(double) * (size_t)DD);
+}
+
+int kda_oracle_backward(int64_t num_seqs, const int64_t *cu, int64_t H, int64_t Dk, int64_t Dv,
+                        const double *q, const double *k, const double *v, const double *g,
+                        const double *beta, const double *init_state, const double *d_out,
+                        const double *d_final_state, double *dq, double *dk, double *dv,
+                        double *dg, double *dbeta, double *d_init_state, int nthreads) {
+    if (num_seqs < 0 || H <= 0 || Dk <= 0 || Dv <= 0 || !cu || cu[0] != 0) return -1;
+    int64_t maxT = 0;
+    for (int64_t i = 0; i < num_seqs; ++i) {
+        if (cu[i + 1] < cu[i]) return -1;
+        if (cu[i + 1] - cu[i] > maxT) maxT = cu[i + 1] - cu[i];
+    }
+    if (cu[num_seqs] > 0 && (!q || !k || !v || !g || !beta || !d_out || !dq || !dk || !dv ||
+                             !dg || !dbeta))
+        return -1;
+    const size_t per_unit = (size_t)((maxT + 2) * Dk * Dv + 3 * Dv + Dk);
+#ifdef _OPENMP
+    if (nthreads <= 0) nthreads = omp_get_max_threads();
+#else
+    nthreads = 1;
+#endif
+    int failed = 0;
+    const int64_t units = num_seqs * H;
+#pragma omp parallel num_threads(nthreads)
+    {
+        double *buf = (double *)malloc(sizeof(double) * per_unit);
+        if (!buf) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t w = 0; w < units; ++w) {
+            if (!buf) continue;
+            const int64_t DD = Dk * Dv;
+            backward_unit(H, Dk, Dv, q, k, v, g, beta, init_state, d_out, d_final_state, dq, dk, dv,
+                          dg, dbeta, d_init_state, cu, w / H, w % H, buf, buf + (maxT + 1) * DD,
+                          buf + (maxT + 2) * DD);
+        }
+        free(buf);
+    }
+    return failed ? -2 : 0;
+}
+
 int kda_oracle_max_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
