@@ -14,9 +14,10 @@ from oracle_pins import PINS
 
 MUTATIONS = {
     "drop_decay": ("S[c * Dv + j] *= a;", "S[c * Dv + j] *= 1.0;"),
-    "delta_sign": ("(vt[j] - y[j])", "(vt[j] + y[j])"),
+    "delta_sign": ("S[c * Dv + j] += bt * kt[c] * (vt[j] - y[j]);",
+                   "S[c * Dv + j] += bt * kt[c] * (vt[j] + y[j]);"),
     "retrieve_with_q": ("y[j] += S[c * Dv + j] * kt[c];", "y[j] += S[c * Dv + j] * qt[c];"),
-    "drop_beta": ("+= bt * kt[c] * (vt[j] - y[j])", "+= kt[c] * (vt[j] - y[j])"),
+    "drop_beta": ("S[c * Dv + j] += bt * kt[c] * (vt[j] - y[j])", "S[c * Dv + j] += kt[c] * (vt[j] - y[j])"),
     "output_with_k": ("ot[j] += S[c * Dv + j] * qt[c];", "ot[j] += S[c * Dv + j] * kt[c];"),
     "ckpt_off_by_one": ("(t + 1 - t0) % p->ckpt_interval", "(t + 2 - t0) % p->ckpt_interval"),
     "gate_transposed": ("exp(Gam[r * Dk + c] - Gam[i * Dk + c])",
