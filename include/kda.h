@@ -204,6 +204,29 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const f
                             const int32_t *accept_len, int32_t tokens_per_seq,
                             const kda_shape *shape, kda_stream_t stream);
 
+/*
+ * Backward pass of the recurrence, for training (the pages name training work
+ * but give no detail; the gradients follow from the forward definition above
+ * by reverse-mode differentiation, token by token in FP32).
+ *
+ *   q, k, v, g, beta, init_state, cu_seqlens : the forward call's inputs
+ *   d_out         : [T_tot, H, D_v] FP32, gradient of the loss w.r.t. out
+ *   d_final_state : [N, H, D_k, D_v] FP32 or NULL (zero), w.r.t. the final state
+ *   dq, dk, dg    : [T_tot, H, D_k] FP32 outputs     dv : [T_tot, H, D_v] FP32
+ *   dbeta         : [T_tot, H] FP32                 d_init_state : [N, H, D_k, D_v] or NULL
+ *   workspace     : at least kda_backward_workspace_bytes(shape) bytes (the
+ *                   state at every 16th token of every unit)
+ * q, k, v are BF16 or FP32 (shape->qkv_dtype); D_k, D_v in {32, 64, 128};
+ * shape->chunk is ignored.  Every pointer 16-byte aligned; outputs must not
+ * overlap inputs or each other.
+ */
+size_t kda_backward_workspace_bytes(const kda_shape *shape);
+kda_status kda_backward(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                        const float *d_out, const float *d_final_state, float *dq, float *dk,
+                        float *dv, float *dg, float *dbeta, float *d_init_state, void *workspace,
+                        size_t workspace_bytes, const kda_shape *shape, kda_stream_t stream);
+
 /* Host helper: sum_i floor(T_i / ckpt_interval) for host int32 cu_seqlens[N+1]
  * (0 when ckpt_interval <= 0; -1 on a bad argument). */
 int64_t kda_ckpt_count(const int32_t *host_cu_seqlens, int32_t num_seqs, int64_t ckpt_interval);

@@ -37,6 +37,13 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  void *workspace, size_t ws_bytes, int32_t *dev_status,
                                  cudaStream_t stream, int num_sms);
 
+size_t backward_workspace_bytes(int N, int H, int64_t T, int Dk, int Dv);
+cudaError_t launch_backward(int dtype, const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const float *init, const int32_t *cu,
+                            const float *dout, const float *dfin, float *dq, float *dk, float *dv,
+                            float *dg, float *dbeta, float *dinit, float *ws, int N, int H, int Dk,
+                            int Dv, cudaStream_t stream);
+
 static thread_local int g_last_cuda_error = 0;
 
 // For entry points defined in other files of the library.
@@ -304,6 +311,54 @@ kda_status kda_prefill_at(const void *q, const void *k, const void *v, const flo
   return prefill_impl(q, k, v, g, beta, init_state, cu_seqlens, out, final_state, ckpt_interval,
                       ckpt_states, pos_cu, positions, pos_states, positions ? WS_NONE : WS_POOL,
                       nullptr, 0, s, stream);
+}
+
+size_t kda_backward_workspace_bytes(const kda_shape *s) {
+  if (check_shape(s, false) != KDA_OK) return (size_t)-1;
+  return backward_workspace_bytes(s->num_seqs, s->num_heads, s->total_tokens, s->head_dim_k,
+                                  s->head_dim_v);
+}
+
+kda_status kda_backward(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, const float *init_state, const int32_t *cu_seqlens,
+                        const float *d_out, const float *d_final_state, float *dq, float *dk,
+                        float *dv, float *dg, float *dbeta, float *d_init_state, void *workspace,
+                        size_t workspace_bytes, const kda_shape *s, kda_stream_t stream) {
+  kda_status st = check_shape(s, false);
+  if (st != KDA_OK) return st;
+  const int N = s->num_seqs, H = s->num_heads, DK = s->head_dim_k, DV = s->head_dim_v;
+  const int64_t T = s->total_tokens;
+  if (!cu_seqlens || !aligned16(cu_seqlens)) return KDA_ERR_INVALID_ARGUMENT;
+  if (T > INT32_MAX) return KDA_ERR_UNSUPPORTED;
+  const size_t es = elem_size(s->qkv_dtype);
+  const size_t n_qk = (size_t)T * H * DK * es, n_v = (size_t)T * H * DV * es;
+  const size_t n_k4 = (size_t)T * H * DK * 4, n_v4 = (size_t)T * H * DV * 4, n_b = (size_t)T * H * 4;
+  const size_t n_state = (size_t)N * H * DK * DV * 4;
+  if (T > 0) {
+    const void *ptrs[] = {q, k, v, g, beta, d_out, dq, dk, dv, dg, dbeta};
+    for (const void *p : ptrs)
+      if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    const size_t need = backward_workspace_bytes(N, H, T, DK, DV);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return KDA_ERR_INVALID_ARGUMENT;
+  }
+  const void *sp[] = {init_state, d_final_state, d_init_state};
+  for (const void *p : sp)
+    if (p && !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+  // outputs must overlap no input and no other output
+  const void *outs[] = {dq, dk, dv, dg, dbeta, d_init_state, workspace};
+  const size_t out_n[] = {n_k4, n_k4, n_v4, n_k4, n_b, n_state, workspace_bytes};
+  const void *ins[] = {q, k, v, g, beta, init_state, d_out, d_final_state, cu_seqlens};
+  const size_t in_n[] = {n_qk, n_qk, n_v, n_k4, n_b, n_state, n_v4, n_state, (size_t)(N + 1) * 4};
+  for (int i = 0; i < 7; ++i) {
+    for (int j = 0; j < 9; ++j)
+      if (overlaps(outs[i], out_n[i], ins[j], in_n[j])) return KDA_ERR_INVALID_ARGUMENT;
+    for (int j = i + 1; j < 7; ++j)
+      if (overlaps(outs[i], out_n[i], outs[j], out_n[j])) return KDA_ERR_INVALID_ARGUMENT;
+  }
+  return cuda_status(launch_backward(s->qkv_dtype, q, k, v, g, beta, init_state, cu_seqlens, d_out,
+                                     d_final_state, dq, dk, dv, dg, dbeta, d_init_state,
+                                     reinterpret_cast<float *>(workspace), N, H, DK, DV,
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 kda_status kda_decode(const void *q, const void *k, const void *v, const float *g,

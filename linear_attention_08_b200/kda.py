@@ -20,7 +20,8 @@ KDA_DTYPE_F32, KDA_DTYPE_BF16 = 0, 1
 EXPORTED = ("kda_prefill", "kda_prefill_ws", "kda_prefill_at", "kda_decode", "kda_decode_multi",
             "kda_ckpt_count", "kda_prefill_workspace_bytes", "kda_prefill_workspace_min_bytes",
             "kda_release_workspace_pool", "kda_prefill_path", "kda_selftest_bounded_wait",
-            "kda_last_cuda_error", "kda_status_string", "kda_version")
+            "kda_last_cuda_error", "kda_status_string", "kda_version", "kda_backward",
+            "kda_backward_workspace_bytes")
 
 # Largest workspace the binding allocates for the two-pass prefill; longer
 # inputs run in windows of chunks.
@@ -77,6 +78,10 @@ def load(path: str | None = None):
     lib.kda_ckpt_count.restype = I64
     lib.kda_prefill_workspace_bytes.argtypes = [SP]
     lib.kda_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_backward.argtypes = [P] * 16 + [ctypes.c_size_t, SP, P]
+    lib.kda_backward.restype = ctypes.c_int
+    lib.kda_backward_workspace_bytes.argtypes = [SP]
+    lib.kda_backward_workspace_bytes.restype = ctypes.c_size_t
     lib.kda_prefill_workspace_min_bytes.argtypes = [SP]
     lib.kda_prefill_workspace_min_bytes.restype = ctypes.c_size_t
     lib.kda_release_workspace_pool.restype = ctypes.c_int
@@ -211,6 +216,36 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, *, init_state=None, chunk: int = 6
     if st != KDA_OK:
         raise KdaError(st, "kda_prefill_at")
     return out, final_state, ckpt_states, pos_states
+
+
+def kda_backward(q, k, v, g, beta, cu_seqlens, d_out, *, init_state=None, d_final=None,
+                 want_d_init: bool = True, workspace=None, stream=None):
+    """Gradients of the recurrence (see kda_backward in include/kda.h) for the
+    upstream gradient d_out [T, H, Dv] (FP32) and d_final [N, H, Dk, Dv] (FP32
+    or None).  Returns (dq, dk, dv, dg, dbeta, d_init) as FP32 tensors; d_init
+    is None unless want_d_init."""
+    lib = load()
+    T, H, Dk = q.shape
+    Dv = v.shape[2]
+    N = cu_seqlens.numel() - 1
+    dev = q.device
+    dq = torch.empty(T, H, Dk, dtype=torch.float32, device=dev)
+    dk = torch.empty_like(dq)
+    dg = torch.empty_like(dq)
+    dv = torch.empty(T, H, Dv, dtype=torch.float32, device=dev)
+    dbeta = torch.empty(T, H, dtype=torch.float32, device=dev)
+    d_init = torch.empty(N, H, Dk, Dv, dtype=torch.float32, device=dev) if want_d_init else None
+    shape = make_shape(N, T, H, Dk, Dv, 0, _dtype_code(q))
+    if workspace is None:
+        nbytes = int(lib.kda_backward_workspace_bytes(ctypes.byref(shape)))
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    st = lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init_state),
+                          _ptr(cu_seqlens), _ptr(d_out), _ptr(d_final), _ptr(dq), _ptr(dk),
+                          _ptr(dv), _ptr(dg), _ptr(dbeta), _ptr(d_init), _ptr(workspace),
+                          workspace.numel(), ctypes.byref(shape), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_backward")
+    return dq, dk, dv, dg, dbeta, d_init
 
 
 def kda_decode(q, k, v, g, beta, state, *, out=None, dev_status=None, stream=None):

@@ -1,0 +1,53 @@
+"""Backward pass on the GPU against the FP64 backward oracle (which is pinned to
+finite differences of the forward oracle in test_oracle_backward.py)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from linear_attention_08_b200 import kda
+from parity import make_case, rel_l2, to_device
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("dq", "dk", "dv", "dg", "dbeta", "d_init")
+
+
+def run_both(lengths, H, Dk, Dv, dtype, seed, use_init=True, use_dfin=True, tol=1e-4):
+    d = make_case(lengths, H, Dk, Dv, dtype, seed=seed, state_std=0.1)
+    dd = to_device(d)
+    rng = np.random.default_rng(seed + 100)
+    T = sum(lengths)
+    d_out = torch.tensor(rng.normal(size=(T, H, Dv)), dtype=torch.float32)
+    d_fin = torch.tensor(rng.normal(size=(len(lengths), H, Dk, Dv)) * 0.5, dtype=torch.float32)
+    init = dd["init_state"] if use_init else None
+    got = kda.kda_backward(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu_dev"],
+                           d_out.cuda(), init_state=init,
+                           d_final=d_fin.cuda() if use_dfin else None)
+    torch.cuda.synchronize()
+    ref = oracle.backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], d_out,
+                          init_state=d["init_state"] if use_init else None,
+                          d_final=d_fin if use_dfin else None)
+    errs = {n: rel_l2(x, r) for n, x, r in zip(NAMES, got, ref)}
+    for n, e in errs.items():
+        assert e <= tol, f"{n}: rel-L2 {e:.3e} > {tol:.0e} ({errs})"
+    return errs
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("dims", [(32, 32), (64, 128), (128, 64), (128, 128)])
+def test_backward_matches_oracle(dtype, dims):
+    """Ragged sequences around the 16-token replay blocks, nonzero initial state and
+    final-state gradient.  The GPU reads the same bits as the oracle, so the bound is
+    the FP32 one for both input dtypes."""
+    Dk, Dv = dims
+    run_both([1, 15, 16, 17, 40], 2, Dk, Dv, dtype, seed=5)
+
+
+def test_backward_without_init_or_final_gradient():
+    run_both([33, 7], 2, 128, 128, torch.bfloat16, seed=6, use_init=False, use_dfin=False)
+
+
+def test_backward_empty_sequence_passes_final_gradient_through():
+    errs = run_both([0, 20, 0], 1, 32, 32, torch.float32, seed=7)
+    assert errs["d_init"] <= 1e-6
