@@ -6,7 +6,7 @@ decode workload (512 sequences x 32 heads, 256 steps captured in one CUDA
 graph, FP32 state N(0, 0.02)) as a second object on the same line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload prefill|decode|append_varlen|long|prefill_small] [--no-decode]
+                  [--workload prefill|decode|append_varlen|long|prefill_small] [--no-decode] [--no-backward]
 
 For N > 1 it is launched by torchrun, one rank per GPU; every rank runs its
 own copy of the workload (the operator's (sequence, head) units are
@@ -401,6 +401,44 @@ def time_spec_decode(steps, warmup, world, local, T_new=8):
     return dict(tokens=N * T_new, ms=ms, bytes=byts, T_new=T_new)
 
 
+def time_backward(steps, warmup, world, local, N=4, H=32, T=1024, D=128):
+    """Backward pass: B=4 x 1024 tokens, 32 heads, D=128, BF16 inputs, random
+    upstream gradients on the outputs and the final states."""
+    from linear_attention_08_b200 import kda
+    lengths = [T] * N
+    d = kin.make_inputs((N * T,), H, D, D, torch.bfloat16, local, num_states=N, state_std=0.02,
+                        device="cuda")
+    cu = torch.tensor(kin.cu_seqlens_of(lengths), dtype=torch.int32, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(1000 + local)
+    d_out = torch.randn(N * T, H, D, device="cuda", generator=gen)
+    d_fin = torch.randn(N, H, D, D, device="cuda", generator=gen)
+    shape = kda.make_shape(N, N * T, H, D, D, 0, kda.KDA_DTYPE_BF16)
+    ws = torch.empty(kda.load().kda_backward_workspace_bytes(kda.ctypes.byref(shape)),
+                     dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.kda_backward(d["q"], d["k"], d["v"], d["g"], d["beta"], cu, d_out,
+                         init_state=d["init_state"], d_final=d_fin, workspace=ws, stream=stream)
+
+    for _ in range(max(warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    # algorithmic bytes per token-head: q, k, v (BF16), g, d_out, the five
+    # FP32 gradients and beta; plus three states per unit (init, d_final, d_init)
+    per_th = 3 * D * 2 + D * 4 + D * 4 + 4 + 3 * D * 4 + D * 4 + 4
+    byts = N * T * H * per_th + 3 * N * H * D * D * 4
+    return dict(tokens=N * T, ms=ms, bytes=byts, N=N, H=H, T=T, D=D)
+
+
 def run_ours(args, rank, world, local):
     peaks, peaks_src = load_peaks()
     hbm = peaks["hbm_gbs"]
@@ -410,6 +448,9 @@ def run_ours(args, rank, world, local):
     spec = None
     if not args.no_decode:
         spec = time_spec_decode(max(args.steps, 5), args.warmup, world, local)
+    bwd = None
+    if not args.no_backward and name == "prefill":
+        bwd = time_backward(max(1, min(args.steps, 3)), args.warmup, world, local)
     dec = None
     if name == "decode" or not args.no_decode:
         dec = time_decode(max(1, args.steps // 2) if name != "decode" else args.steps,
@@ -446,6 +487,17 @@ def run_ours(args, rank, world, local):
             "gpu_launches": r["steps"] * r["launches_per_step"],
             "clocks": r["clocks"],
         }
+        if bwd is not None:
+            bgbs = bwd["bytes"] / (bwd["ms"] / 1e3) / 1e9
+            line["backward"] = {
+                "metric": "KDA backward tokens/s",
+                "value": world * bwd["tokens"] / (bwd["ms"] / 1e3), "unit": "tokens/s",
+                "ms_per_call": bwd["ms"],
+                "config": {"num_seqs": bwd["N"], "seq_len": bwd["T"], "heads": bwd["H"],
+                           "d": bwd["D"], "dtype": "bf16 inputs, fp32 gradients"},
+                "roofline": {"bound": "latency", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
+                             "frac": bgbs / hbm, "kernel": "backward",
+                             "note": "SIMT, replays up to 7 forward steps per token"}}
     if dec is not None:
         dgbs = dec["bytes"] / (dec["ms"] / dec["launches"] / 1e3) / 1e9 / dec["launches"]
         dobj = {
@@ -557,6 +609,7 @@ def main():
     ap.add_argument("--workload", default="prefill",
                     choices=["prefill", "decode", "append_varlen", "long", "prefill_small"])
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=0,
                     help="decode steps per graph (default: the workload's 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

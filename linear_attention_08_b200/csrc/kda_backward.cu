@@ -14,8 +14,8 @@
 //   dS   <- Diag(alpha_t) (dS - beta_t k_t du^T)       (gradient w.r.t. S_{t-1})
 //
 // One CTA (256 threads) per (sequence, head).  A forward sweep stores the
-// state at every 16th token in the workspace; the reverse sweep rebuilds
-// S_{t-1} for each token from the nearest stored state (at most 15 forward
+// state at every 8th token in the workspace; the reverse sweep rebuilds
+// S_{t-1} for each token from the nearest stored state (at most 7 forward
 // steps) and applies the step above.  The state, its copy at the block start
 // and dS live in shared memory with a padded row stride (D_v + 1 floats), so
 // that both row-wise and column-wise passes are free of bank conflicts.
@@ -27,7 +27,7 @@ namespace kda {
 namespace {
 
 constexpr int kBThreads = 256;
-constexpr int kBlk = 16;      // tokens between stored states
+constexpr int kBlk = 8;       // tokens between stored states
 constexpr int kMaxD = 128;
 
 struct BwdArgs {
@@ -37,7 +37,7 @@ struct BwdArgs {
   const float *dout, *dfin;
   float *dq, *dk, *dv, *dg, *dbeta, *dinit;
   float *ws;
-  int H, Dk, Dv;
+  int H;
 };
 
 template <typename TIn>
@@ -45,10 +45,11 @@ __device__ __forceinline__ float ld_in(const void *p, size_t i) {
   return to_f32(reinterpret_cast<const TIn *>(p)[i]);
 }
 
-template <typename TIn>
+template <typename TIn, int Dk, int Dv>
 __global__ void __launch_bounds__(kBThreads, 1) backward_kernel(const BwdArgs a) {
   extern __shared__ float smem[];
-  const int Dk = a.Dk, Dv = a.Dv, H = a.H, ld = Dv + 1;
+  const int H = a.H;
+  constexpr int ld = Dv + 1;
   float *S = smem;                        // [Dk][Dv+1] working state (S_{t-1} after the replay)
   float *dS = S + Dk * ld;                // [Dk][Dv+1]
   float *S0 = dS + Dk * ld;               // [Dk][Dv]  stored state of the current block
@@ -71,13 +72,14 @@ __global__ void __launch_bounds__(kBThreads, 1) backward_kernel(const BwdArgs a)
   int64_t before = 0;
   for (int m = 0; m < n; ++m) before += ((int64_t)a.cu[m + 1] - a.cu[m] + kBlk - 1) / kBlk;
   float *wsu = a.ws + ((size_t)before * H + (size_t)h * nb) * Dk * Dv;
-  const int DD = Dk * Dv;
+  constexpr int DD = Dk * Dv;
 
-  // Column passes: thread (j, part) sums over rows c = part, part + cp, ...
-  const int cp = kBThreads / Dv;          // parts per column (2, 4 or 8)
+  // Column passes and elementwise passes: thread (j, part) takes column j of
+  // rows c = part, part + cp, ...; row passes: thread (c, part) takes row c
+  // at columns j = part, part + rp, ...
+  constexpr int cp = kBThreads / Dv;      // 2, 4 or 8
   const int cj = tid % Dv, cpart = tid / Dv;
-  // Row passes: thread (c, part) sums over columns j = part, part + rp, ...
-  const int rp = kBThreads / Dk;
+  constexpr int rp = kBThreads / Dk;
   const int rc = tid % Dk, rpart = tid / Dk;
 
   auto load_token = [&](int64_t t, bool full) {
@@ -112,47 +114,41 @@ __global__ void __launch_bounds__(kBThreads, 1) backward_kernel(const BwdArgs a)
     load_token(t, false);
     __syncthreads();
     form_y_u();
-    for (int e = tid; e < DD; e += kBThreads) {
-      const int c = e / Dv, j = e - c * Dv;
-      S[c * ld + j] = fmaf(va[c], S[c * ld + j], vk[c] * vu[j]);
-    }
+    const float uj = vu[cj];
+#pragma unroll
+    for (int c = cpart; c < Dk; c += cp) S[c * ld + cj] = fmaf(va[c], S[c * ld + cj], vk[c] * uj);
     __syncthreads();
   };
 
-  // ---------------- forward sweep: states at every 16th token ----------------
-  for (int e = tid; e < DD; e += kBThreads) {
-    const int c = e / Dv, j = e - c * Dv;
-    S[c * ld + j] = a.init ? a.init[(size_t)unit * DD + e] : 0.f;
-  }
+  // ---------------- forward sweep: states at every 8th token ----------------
+#pragma unroll
+  for (int c = cpart; c < Dk; c += cp)
+    S[c * ld + cj] = a.init ? a.init[(size_t)unit * DD + c * Dv + cj] : 0.f;
   __syncthreads();
   for (int64_t t = 0; t < T; ++t) {
     if (t % kBlk == 0) {
       float *dst = wsu + (size_t)(t / kBlk) * DD;
-      for (int e = tid; e < DD; e += kBThreads) {
-        const int c = e / Dv, j = e - c * Dv;
-        dst[e] = S[c * ld + j];
-      }
+#pragma unroll
+      for (int c = cpart; c < Dk; c += cp) dst[c * Dv + cj] = S[c * ld + cj];
     }
     forward_step(t);
   }
 
   // ---------------- reverse sweep ----------------
-  for (int e = tid; e < DD; e += kBThreads) {
-    const int c = e / Dv, j = e - c * Dv;
-    dS[c * ld + j] = a.dfin ? a.dfin[(size_t)unit * DD + e] : 0.f;
-  }
+#pragma unroll
+  for (int c = cpart; c < Dk; c += cp)
+    dS[c * ld + cj] = a.dfin ? a.dfin[(size_t)unit * DD + c * Dv + cj] : 0.f;
   __syncthreads();
   for (int64_t b = nb - 1; b >= 0; --b) {
     const int64_t t_lo = b * kBlk, t_hi = (t_lo + kBlk < T) ? t_lo + kBlk : T;
     const float *src = wsu + (size_t)b * DD;
-    for (int e = tid; e < DD; e += kBThreads) S0[e] = src[e];
+#pragma unroll
+    for (int c = cpart; c < Dk; c += cp) S0[c * Dv + cj] = src[c * Dv + cj];
     __syncthreads();
     for (int64_t t = t_hi - 1; t >= t_lo; --t) {
       // rebuild S_{t-1} from the block's stored state
-      for (int e = tid; e < DD; e += kBThreads) {
-        const int c = e / Dv, j = e - c * Dv;
-        S[c * ld + j] = S0[e];
-      }
+#pragma unroll
+      for (int c = cpart; c < Dk; c += cp) S[c * ld + cj] = S0[c * Dv + cj];
       __syncthreads();
       for (int64_t r = t_lo; r < t; ++r) forward_step(r);
       // ---- backward step of token t ----
@@ -160,9 +156,10 @@ __global__ void __launch_bounds__(kBThreads, 1) backward_kernel(const BwdArgs a)
       __syncthreads();
       form_y_u();
       // dS += q do^T
-      for (int e = tid; e < DD; e += kBThreads) {
-        const int c = e / Dv, j = e - c * Dv;
-        dS[c * ld + j] = fmaf(vq[c], vdo[j], dS[c * ld + j]);
+      {
+        const float doj = vdo[cj];
+#pragma unroll
+        for (int c = cpart; c < Dk; c += cp) dS[c * ld + cj] = fmaf(vq[c], doj, dS[c * ld + cj]);
       }
       __syncthreads();
       // du_j = sum_c k_c dS_cj
@@ -229,18 +226,18 @@ __global__ void __launch_bounds__(kBThreads, 1) backward_kernel(const BwdArgs a)
         a.dg[o] = al * (r4 - bt * kc * r3);
       }
       // dS <- Diag(alpha) (dS - beta k du^T)
-      for (int e = tid; e < DD; e += kBThreads) {
-        const int c = e / Dv, j = e - c * Dv;
-        dS[c * ld + j] = va[c] * fmaf(-bt * vk[c], vdu[j], dS[c * ld + j]);
+      {
+        const float duj = vdu[cj];
+#pragma unroll
+        for (int c = cpart; c < Dk; c += cp)
+          dS[c * ld + cj] = va[c] * fmaf(-bt * vk[c], duj, dS[c * ld + cj]);
       }
       __syncthreads();
     }
   }
   if (a.dinit)
-    for (int e = tid; e < DD; e += kBThreads) {
-      const int c = e / Dv, j = e - c * Dv;
-      a.dinit[(size_t)unit * DD + e] = dS[c * ld + j];
-    }
+#pragma unroll
+    for (int c = cpart; c < Dk; c += cp) a.dinit[(size_t)unit * DD + c * Dv + cj] = dS[c * ld + cj];
 }
 
 }  // namespace
@@ -253,27 +250,37 @@ size_t backward_workspace_bytes(int N, int H, int64_t T, int Dk, int Dv) {
   return sizeof(float) * (size_t)((T + (int64_t)(kBlk - 1) * N) / kBlk) * H * Dk * Dv;
 }
 
+template <typename TIn, int DK, int DV>
+static cudaError_t launch_backward_t(const BwdArgs &args, unsigned grid, cudaStream_t stream) {
+  const size_t smem = backward_smem_bytes(DK, DV);
+  cudaError_t e = cudaFuncSetAttribute(backward_kernel<TIn, DK, DV>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  backward_kernel<TIn, DK, DV><<<grid, kBThreads, smem, stream>>>(args);
+  return cudaGetLastError();
+}
+
+template <typename TIn>
+static cudaError_t launch_backward_d(const BwdArgs &args, int Dk, int Dv, unsigned grid,
+                                     cudaStream_t stream) {
+#define KDA_BWD(DK_, DV_) \
+  if (Dk == DK_ && Dv == DV_) return launch_backward_t<TIn, DK_, DV_>(args, grid, stream);
+  KDA_BWD(32, 32) KDA_BWD(32, 64) KDA_BWD(32, 128)
+  KDA_BWD(64, 32) KDA_BWD(64, 64) KDA_BWD(64, 128)
+  KDA_BWD(128, 32) KDA_BWD(128, 64) KDA_BWD(128, 128)
+#undef KDA_BWD
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_backward(int dtype, const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const float *init, const int32_t *cu,
                             const float *dout, const float *dfin, float *dq, float *dk, float *dv,
                             float *dg, float *dbeta, float *dinit, float *ws, int N, int H, int Dk,
                             int Dv, cudaStream_t stream) {
-  const BwdArgs args{q, k, v, g, beta, init, cu, dout, dfin, dq, dk, dv, dg, dbeta, dinit, ws,
-                     H, Dk, Dv};
-  const size_t smem = backward_smem_bytes(Dk, Dv);
+  const BwdArgs args{q, k, v, g, beta, init, cu, dout, dfin, dq, dk, dv, dg, dbeta, dinit, ws, H};
   const unsigned grid = (unsigned)((int64_t)N * H);
-  if (dtype == KDA_DTYPE_BF16) {
-    cudaError_t e = cudaFuncSetAttribute(backward_kernel<__nv_bfloat16>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    backward_kernel<__nv_bfloat16><<<grid, kBThreads, smem, stream>>>(args);
-  } else {
-    cudaError_t e = cudaFuncSetAttribute(backward_kernel<float>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    backward_kernel<float><<<grid, kBThreads, smem, stream>>>(args);
-  }
-  return cudaGetLastError();
+  if (dtype == KDA_DTYPE_BF16) return launch_backward_d<__nv_bfloat16>(args, Dk, Dv, grid, stream);
+  return launch_backward_d<float>(args, Dk, Dv, grid, stream);
 }
 
 }  // namespace kda
