@@ -101,12 +101,6 @@ __device__ __forceinline__ void st_chunk_s(uint8_t *dst, const float *x) {
                                                tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
 }
 
-// 16-byte store of 8 floats as bf16 into global memory.
-__device__ __forceinline__ void st_global_chunk(uint8_t *dst, const float *x) {
-  *reinterpret_cast<uint4 *>(dst) = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
-                                               tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
-}
-
 // Chunks of sequence n that fall in the window [jw0, jw0 + wc).
 __device__ __forceinline__ int64_t window_chunks(const int32_t *cu, int n, int64_t jw0, int64_t wc) {
   const int64_t nch = ((int64_t)cu[n + 1] - cu[n] + kC - 1) / kC;

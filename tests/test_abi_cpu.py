@@ -169,3 +169,30 @@ def test_prefill_at_requires_all_position_pointers():
     assert lib.kda_prefill_at(a, a, a, a, a, None, a, b, None, 0, None, a, a,
                               ctypes.c_void_p((1 << 28) + 4), ctypes.byref(s),
                               None) == kda.KDA_ERR_INVALID_ARGUMENT
+
+
+def test_backward_workspace_and_validation():
+    lib = kda.load()
+    s = kda.make_shape(2, 1000, 4, 128, 64, 0, kda.KDA_DTYPE_BF16)
+    need = lib.kda_backward_workspace_bytes(ctypes.byref(s))
+    assert need == ((1000 + 7 * 2) // 8) * 4 * 128 * 64 * 4   # a state every 8 tokens, bound
+    P = ctypes.c_void_p
+    base = 1 << 30
+    ptr = lambda i: P(base + i * (1 << 26))   # distinct, non-overlapping fake device addresses
+    args = [ptr(i) for i in range(5)] + [None, ptr(5), ptr(6), None] + [ptr(7 + i) for i in range(5)] + [None]
+    lib.kda_backward.argtypes = [P] * 16 + [ctypes.c_size_t, ctypes.POINTER(kda.KdaShape), P]
+    ws = ptr(12)
+    # workspace too small; null d_out; misaligned dq; dq overlapping q
+    assert lib.kda_backward(*args, ws, need - 16, ctypes.byref(s), None) == kda.KDA_ERR_INVALID_ARGUMENT
+    bad = list(args)
+    bad[7] = None
+    assert lib.kda_backward(*bad, ws, need, ctypes.byref(s), None) == kda.KDA_ERR_INVALID_ARGUMENT
+    bad = list(args)
+    bad[9] = P(base + 7 * (1 << 26) + 4)
+    assert lib.kda_backward(*bad, ws, need, ctypes.byref(s), None) == kda.KDA_ERR_INVALID_ARGUMENT
+    bad = list(args)
+    bad[9] = ptr(0)
+    assert lib.kda_backward(*bad, ws, need, ctypes.byref(s), None) == kda.KDA_ERR_INVALID_ARGUMENT
+    # head size outside {32, 64, 128}
+    s_bad = kda.make_shape(2, 1000, 4, 96, 64, 0, kda.KDA_DTYPE_BF16)
+    assert lib.kda_backward(*args, ws, need, ctypes.byref(s_bad), None) == kda.KDA_ERR_UNSUPPORTED
