@@ -49,7 +49,7 @@ typedef struct CUstream_st *kda_stream_t;
 typedef enum {
   KDA_OK = 0,
   KDA_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misalignment          */
-  KDA_ERR_UNSUPPORTED = 2,      /* a head size or chunk size this build lacks    */
+  KDA_ERR_UNSUPPORTED = 2,      /* a head size or chunk size the library lacks   */
   KDA_ERR_CUDA = 3,             /* a CUDA call failed; see kda_last_cuda_error() */
   KDA_ERR_TIMEOUT = 4           /* written to dev_status by a bounded wait       */
 } kda_status;
