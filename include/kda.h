@@ -227,6 +227,29 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const float
                         float *dv, float *dg, float *dbeta, float *d_init_state, void *workspace,
                         size_t workspace_bytes, const kda_shape *shape, kda_stream_t stream);
 
+/*
+ * Affine state maps for context (sequence) parallelism.  The pages name KDA
+ * context parallelism ("MoonshotAI/Kimi-K3 딥다이브", section 4-1) without
+ * detail.  The recurrence is affine in its starting state: over a segment,
+ * S_out = A S_in + B, with A the state of the segment run with v = 0 from the
+ * identity and B its state from zero; token by token the outputs from S_in
+ * are o_t(B) + S_in^T (A_t^T q_t), where A_t^T q_t is the output of the
+ * v = 0, identity-start run.  (linear_attention_08_b200/cp.py combines the
+ * segments of several ranks with these two calls.)
+ *
+ * kda_affine_rows:  y[r, h, :] = x[r, h, :] M[h]  (+ y when accumulate != 0)
+ *   x : [rows, H, D_k]  y : [rows, H, D_v]  (shape->qkv_dtype, BF16 or FP32)
+ *   M : [H, D_k, D_v] FP32.  y must not overlap x or M.
+ * kda_affine_state: S_out[h] = A[h] S_in[h] + B[h]
+ *   A : [H, D_k, D_k]  S_in, B, S_out : [H, D_k, D_v], all FP32; B may be NULL
+ *   (zero); S_out may alias S_in or B but not A.
+ * Only num_heads, head_dim_k, head_dim_v and qkv_dtype of the shape are used.
+ */
+kda_status kda_affine_rows(const void *x, const float *M, void *y, int64_t rows, int32_t accumulate,
+                           const kda_shape *shape, kda_stream_t stream);
+kda_status kda_affine_state(const float *A, const float *S_in, const float *B, float *S_out,
+                            const kda_shape *shape, kda_stream_t stream);
+
 /* Host helper: sum_i floor(T_i / ckpt_interval) for host int32 cu_seqlens[N+1]
  * (0 when ckpt_interval <= 0; -1 on a bad argument). */
 int64_t kda_ckpt_count(const int32_t *host_cu_seqlens, int32_t num_seqs, int64_t ckpt_interval);

@@ -37,6 +37,10 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  void *workspace, size_t ws_bytes, int32_t *dev_status,
                                  cudaStream_t stream, int num_sms);
 
+cudaError_t launch_affine_rows(int dtype, const void *x, const float *M, void *y, int64_t rows,
+                               int H, int Dk, int Dv, int accumulate, cudaStream_t stream);
+cudaError_t launch_affine_state(const float *A, const float *S, const float *B, float *S_out, int H,
+                                int Dk, int Dv, cudaStream_t stream);
 size_t backward_workspace_bytes(int N, int H, int64_t T, int Dk, int Dv);
 cudaError_t launch_backward(int dtype, const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const float *init, const int32_t *cu,
@@ -311,6 +315,38 @@ kda_status kda_prefill_at(const void *q, const void *k, const void *v, const flo
   return prefill_impl(q, k, v, g, beta, init_state, cu_seqlens, out, final_state, ckpt_interval,
                       ckpt_states, pos_cu, positions, pos_states, positions ? WS_NONE : WS_POOL,
                       nullptr, 0, s, stream);
+}
+
+kda_status kda_affine_rows(const void *x, const float *M, void *y, int64_t rows, int32_t accumulate,
+                           const kda_shape *s, kda_stream_t stream) {
+  if (!s || s->num_heads < 1 || rows < 0) return KDA_ERR_INVALID_ARGUMENT;
+  if (s->qkv_dtype != KDA_DTYPE_F32 && s->qkv_dtype != KDA_DTYPE_BF16) return KDA_ERR_INVALID_ARGUMENT;
+  if (!head_dim_ok(s->head_dim_k) || !head_dim_ok(s->head_dim_v)) return KDA_ERR_UNSUPPORTED;
+  const int H = s->num_heads, DK = s->head_dim_k, DV = s->head_dim_v;
+  if (rows == 0) return KDA_OK;
+  const void *ptrs[] = {x, M, y};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+  const size_t es = elem_size(s->qkv_dtype);
+  const size_t ny = (size_t)rows * H * DV * es;
+  if (overlaps(y, ny, x, (size_t)rows * H * DK * es) || overlaps(y, ny, M, (size_t)H * DK * DV * 4))
+    return KDA_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_affine_rows(s->qkv_dtype, x, M, y, rows, H, DK, DV, accumulate != 0,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_affine_state(const float *A, const float *S_in, const float *B, float *S_out,
+                            const kda_shape *s, kda_stream_t stream) {
+  if (!s || s->num_heads < 1) return KDA_ERR_INVALID_ARGUMENT;
+  if (!head_dim_ok(s->head_dim_k) || !head_dim_ok(s->head_dim_v)) return KDA_ERR_UNSUPPORTED;
+  const int H = s->num_heads, DK = s->head_dim_k, DV = s->head_dim_v;
+  const void *ptrs[] = {A, S_in, S_out};
+  for (const void *p : ptrs)
+    if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+  if (B && !aligned16(B)) return KDA_ERR_INVALID_ARGUMENT;
+  if (overlaps(S_out, (size_t)H * DK * DV * 4, A, (size_t)H * DK * DK * 4)) return KDA_ERR_INVALID_ARGUMENT;
+  return cuda_status(launch_affine_state(A, S_in, B, S_out, H, DK, DV,
+                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t kda_backward_workspace_bytes(const kda_shape *s) {

@@ -21,7 +21,7 @@ EXPORTED = ("kda_prefill", "kda_prefill_ws", "kda_prefill_at", "kda_decode", "kd
             "kda_ckpt_count", "kda_prefill_workspace_bytes", "kda_prefill_workspace_min_bytes",
             "kda_release_workspace_pool", "kda_prefill_path", "kda_selftest_bounded_wait",
             "kda_last_cuda_error", "kda_status_string", "kda_version", "kda_backward",
-            "kda_backward_workspace_bytes")
+            "kda_backward_workspace_bytes", "kda_affine_rows", "kda_affine_state")
 
 # Largest workspace the binding allocates for the two-pass prefill; longer
 # inputs run in windows of chunks.
@@ -78,6 +78,10 @@ def load(path: str | None = None):
     lib.kda_ckpt_count.restype = I64
     lib.kda_prefill_workspace_bytes.argtypes = [SP]
     lib.kda_prefill_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_affine_rows.argtypes = [P, P, P, I64, I32, SP, P]
+    lib.kda_affine_rows.restype = ctypes.c_int
+    lib.kda_affine_state.argtypes = [P, P, P, P, SP, P]
+    lib.kda_affine_state.restype = ctypes.c_int
     lib.kda_backward.argtypes = [P] * 16 + [ctypes.c_size_t, SP, P]
     lib.kda_backward.restype = ctypes.c_int
     lib.kda_backward_workspace_bytes.argtypes = [SP]
@@ -246,6 +250,32 @@ def kda_backward(q, k, v, g, beta, cu_seqlens, d_out, *, init_state=None, d_fina
     if st != KDA_OK:
         raise KdaError(st, "kda_backward")
     return dq, dk, dv, dg, dbeta, d_init
+
+
+def kda_affine_rows(x, M, y, *, accumulate: bool = False, stream=None):
+    """y[r, h, :] = x[r, h, :] @ M[h] (+ y when accumulate): x [rows, H, Dk],
+    y [rows, H, Dv] (same dtype, BF16 or FP32), M [H, Dk, Dv] FP32."""
+    rows, H, Dk = x.shape
+    Dv = y.shape[2]
+    shape = make_shape(1, rows, H, Dk, Dv, 0, _dtype_code(x))
+    st = load().kda_affine_rows(_ptr(x), _ptr(M), _ptr(y), int(rows), int(bool(accumulate)),
+                                ctypes.byref(shape), _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_affine_rows")
+    return y
+
+
+def kda_affine_state(A, S_in, B=None, S_out=None, *, stream=None):
+    """S_out[h] = A[h] @ S_in[h] + B[h] (FP32): A [H, Dk, Dk], S_in, B [H, Dk, Dv]."""
+    H, Dk, Dv = S_in.shape
+    if S_out is None:
+        S_out = torch.empty_like(S_in)
+    shape = make_shape(1, 1, H, Dk, Dv, 0, KDA_DTYPE_F32)
+    st = load().kda_affine_state(_ptr(A), _ptr(S_in), _ptr(B), _ptr(S_out), ctypes.byref(shape),
+                                 _stream(stream))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_affine_state")
+    return S_out
 
 
 def kda_decode(q, k, v, g, beta, state, *, out=None, dev_status=None, stream=None):
