@@ -497,7 +497,7 @@ def run_ours(args, rank, world, local):
                            "d": bwd["D"], "dtype": "bf16 inputs, fp32 gradients"},
                 "roofline": {"bound": "latency", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
                              "frac": bgbs / hbm, "kernel": "backward",
-                             "note": "SIMT, replays up to 7 forward steps per token"}}
+                             "note": "SIMT, one CTA per (sequence, head, 32 value columns), one replay per 4-token block"}}
     if dec is not None:
         dgbs = dec["bytes"] / (dec["ms"] / dec["launches"] / 1e3) / 1e9 / dec["launches"]
         dobj = {

@@ -215,7 +215,8 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const f
  *   dq, dk, dg    : [T_tot, H, D_k] FP32 outputs     dv : [T_tot, H, D_v] FP32
  *   dbeta         : [T_tot, H] FP32                 d_init_state : [N, H, D_k, D_v] or NULL
  *   workspace     : at least kda_backward_workspace_bytes(shape) bytes (the
- *                   state at every 8th token of every unit)
+ *                   state at every 4th token of every unit and, for D_v > 32,
+ *                   the dq, dk, dg, dbeta parts of value-column slices 2..)
  * q, k, v are BF16 or FP32 (shape->qkv_dtype); D_k, D_v in {32, 64, 128};
  * shape->chunk is ignored.  Every pointer 16-byte aligned; outputs must not
  * overlap inputs or each other.

@@ -46,7 +46,7 @@ cudaError_t launch_backward(int dtype, const void *q, const void *k, const void 
                             const float *beta, const float *init, const int32_t *cu,
                             const float *dout, const float *dfin, float *dq, float *dk, float *dv,
                             float *dg, float *dbeta, float *dinit, float *ws, int N, int H, int Dk,
-                            int Dv, cudaStream_t stream);
+                            int Dv, int64_t T, cudaStream_t stream);
 
 static thread_local int g_last_cuda_error = 0;
 
@@ -393,7 +393,7 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const float
   }
   return cuda_status(launch_backward(s->qkv_dtype, q, k, v, g, beta, init_state, cu_seqlens, d_out,
                                      d_final_state, dq, dk, dv, dg, dbeta, d_init_state,
-                                     reinterpret_cast<float *>(workspace), N, H, DK, DV,
+                                     reinterpret_cast<float *>(workspace), N, H, DK, DV, T,
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
