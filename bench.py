@@ -613,6 +613,9 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=0,
                     help="decode steps per graph (default: the workload's 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward-only", type=int, default=0, metavar="SEQ_LEN",
+                    help="time only the backward pass on 4 sequences of SEQ_LEN tokens "
+                         "(a small case for profiling); prints its object alone")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
@@ -622,6 +625,19 @@ def main():
             print(json.dumps(line), flush=True)
         return
     rank, world, local = dist_setup(args.gpus)
+    if args.backward_only > 0:
+        bwd = time_backward(args.steps, args.warmup, world, local, T=args.backward_only)
+        if rank == 0:
+            print(json.dumps({"metric": "KDA backward tokens/s", "unit": "tokens/s",
+                              "value": world * bwd["tokens"] / (bwd["ms"] / 1e3),
+                              "ms_per_call": bwd["ms"], "n_gpus": world,
+                              "config": {"num_seqs": bwd["N"], "seq_len": bwd["T"],
+                                         "heads": bwd["H"], "d": bwd["D"]}}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     line = run_ours(args, rank, world, local)
     if rank == 0 and line is not None:
         if world == 1 and not args.no_cpu_baseline:

@@ -59,15 +59,18 @@ __device__ __forceinline__ float ld_in(const void *p, size_t i) {
   return to_f32(reinterpret_cast<const TIn *>(p)[i]);
 }
 
-// Sum of v[i] over the 32 lanes for every i < M, scattered: on return, lane L
-// holds the sum for row i = L >> (5 - log2 M).  Recursive halving: at each
-// level a lane keeps one half of its values and adds its partner's copy of
-// that half, so a level of m values costs m/2 shuffles.
-template <int M>
+// Reduce-scatter across lanes: v[i] (i < M) is summed over the lanes that
+// differ in the lane bits OHI, OHI/2, ..., OLO; on return the lane holds the
+// sum for one i, i = the lane's bits OHI .. (OHI >> (log2 M - 1)) read as a
+// binary number (highest first).  Recursive halving: at each level a lane
+// keeps one half of its values and adds its partner's copy of that half, so
+// a level of m values costs m/2 shuffles; bits below the halving levels are
+// summed by plain butterflies.
+template <int M, int OHI, int OLO>
 __device__ __forceinline__ float reduce_scatter(float (&v)[M], int lane) {
 #pragma unroll
   for (int lvl = 0; (M >> lvl) > 1; ++lvl) {
-    const int half = M >> (lvl + 1), o = 16 >> lvl;
+    const int half = M >> (lvl + 1), o = OHI >> lvl;
     const bool up = (lane & o) != 0;
 #pragma unroll
     for (int i = 0; i < half; ++i) {
@@ -78,17 +81,47 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[M], int lane) {
   }
   float r = v[0];
 #pragma unroll
-  for (int o = 16 / M; o >= 1; o >>= 1) r += __shfl_xor_sync(kFull, r, o);
+  for (int o = OHI / M; o >= OLO; o >>= 1) r += __shfl_xor_sync(kFull, r, o);
   return r;
 }
 
 template <int M> struct Log2 { static constexpr int value = 1 + Log2<M / 2>::value; };
 template <> struct Log2<1> { static constexpr int value = 0; };
 
+// RT consecutive floats from shared memory (RT in {2, 4, 8}, aligned to RT floats).
+template <int RT>
+__device__ __forceinline__ void lds_rows(const float *p, float (&o)[RT]) {
+  if constexpr (RT % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < RT; i += 4) {
+      const float4 x = *reinterpret_cast<const float4 *>(p + i);
+      o[i] = x.x;
+      o[i + 1] = x.y;
+      o[i + 2] = x.z;
+      o[i + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < RT; i += 2) {
+      const float2 x = *reinterpret_cast<const float2 *>(p + i);
+      o[i] = x.x;
+      o[i + 1] = x.y;
+    }
+  }
+}
+
+__device__ __forceinline__ void lds4(const float *p, float (&o)[4]) {
+  const float4 x = *reinterpret_cast<const float4 *>(p);
+  o[0] = x.x;
+  o[1] = x.y;
+  o[2] = x.z;
+  o[3] = x.w;
+}
+
 // Shared memory, in floats.
 template <int Dk>
 struct BwdSmem {
-  static constexpr int RPW = Dk / 4;
+  static constexpr int PER_THREAD = Dk / 4;           // state entries per thread
   static constexpr int TK = 0;                        // k        [kBlk][Dk]
   static constexpr int TA = TK + kBlk * Dk;           // alpha    [kBlk][Dk]
   static constexpr int TQ = TA + kBlk * Dk;           // q        [kBlk][Dk]
@@ -97,21 +130,28 @@ struct BwdSmem {
   static constexpr int TB = TD + kBlk * kCols;        // beta     [kBlk] (padded to 4)
   static constexpr int PY = TB + 4;                   // y parts  [2][4][32]
   static constexpr int PD = PY + 2 * 4 * kCols;       // du parts [2][4][32]
-  static constexpr int ST = PD + 2 * 4 * kCols;       // states   [kBlk-2][RPW][128]
-  static constexpr int TOTAL = ST + (kBlk - 2) * RPW * kBThreads;
+  static constexpr int ST = PD + 2 * 4 * kCols;       // states   [kBlk-2][PER_THREAD][128]
+  static constexpr int TOTAL = ST + (kBlk - 2) * PER_THREAD * kBThreads;
 };
 
+// Thread layout: warp w owns rows [w Dk/4, (w+1) Dk/4) of the slice; lane
+// (rg, cg) = (lane >> 3, lane & 7) owns the RT = Dk/16 rows starting at
+// w Dk/4 + rg RT and the 4 columns starting at 4 cg.  Column sums over a
+// warp's rows reduce-scatter across rg (lane bits 16, 8), row sums over the
+// slice's columns across cg (lane bits 4, 2, 1).
 template <typename TIn, int Dk, int Dv>
 __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a) {
   using L = BwdSmem<Dk>;
-  constexpr int RPW = L::RPW, NS = Dv / kCols, DD = Dk * Dv;
-  constexpr int SHIFT = 5 - Log2<RPW>::value;
+  constexpr int RPW = Dk / 4, RT = Dk / 16, NS = Dv / kCols, DD = Dk * Dv;
+  constexpr int RSH = 3 - Log2<RT>::value;   // row sums: lanes sharing a row differ in cg's low RSH bits
   extern __shared__ __align__(16) float smem[];
-  const int tid = threadIdx.x, w = tid >> 5, j = tid & 31;
+  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  const int cg = lane & 7, rg = lane >> 3;
   const int H = a.H;
   const int slice = blockIdx.x % NS, unit = blockIdx.x / NS, n = unit / H, h = unit % H;
-  const int col = slice * kCols + j;
-  const int row0 = w * RPW;
+  const int c4 = cg * 4;                       // first column of the thread within the slice
+  const int col = slice * kCols + c4;          // ... within the head
+  const int rbase = w * RPW + rg * RT;         // first row of the thread
   const int64_t t_begin = a.cu[n], T = (int64_t)a.cu[n + 1] - t_begin;
   const int64_t nb = (T + kBlk - 1) / kBlk;
   int64_t before = 0;   // stored states of all earlier sequences, per head
@@ -133,7 +173,7 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     ob = a.part + 3 * (NS - 1) * n_k + s1 * (size_t)a.T * H;
   }
 
-  float S[RPW], dS[RPW];
+  float S[RT][4], dS[RT][4];
   int par = 0;
 
   auto load_tokens = [&](int64_t t_lo, int cnt, bool full) {
@@ -152,100 +192,136 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     }
     if (tid < cnt) tb[tid] = a.beta[(size_t)(t_begin + t_lo + tid) * H + h];
   };
-  auto load_state = [&](int64_t b) {
-    const float *src = ck + (size_t)b * DD;
+  // a [Dk][Dv] FP32 matrix in global memory <-> the thread's tile
+  auto ld_tile = [&](const float *src, float (&X)[RT][4]) {
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) S[i] = src[(row0 + i) * Dv + col];
+    for (int r = 0; r < RT; ++r) {
+      const float4 x = *reinterpret_cast<const float4 *>(src + (size_t)(rbase + r) * Dv + col);
+      X[r][0] = x.x;
+      X[r][1] = x.y;
+      X[r][2] = x.z;
+      X[r][3] = x.w;
+    }
   };
-  // One forward step of token slot s: S <- Diag(alpha) S + k u^T.  The warps'
-  // parts of y_j = sum_c alpha_c k_c S_cj meet in py.
-  auto fwd_step = [&](int s) {
-    const float *k_s = tk + s * Dk + row0, *a_s = ta + s * Dk + row0;
-    float pa = 0.f;
+  auto st_tile = [&](float *dst, const float (&X)[RT][4]) {
 #pragma unroll
-    for (int i = 0; i < RPW; i += 4) {
-      const float4 k4 = *reinterpret_cast<const float4 *>(k_s + i);
-      const float4 a4 = *reinterpret_cast<const float4 *>(a_s + i);
-      pa = fmaf(a4.x * k4.x, S[i], pa);
-      pa = fmaf(a4.y * k4.y, S[i + 1], pa);
-      pa = fmaf(a4.z * k4.z, S[i + 2], pa);
-      pa = fmaf(a4.w * k4.w, S[i + 3], pa);
+    for (int r = 0; r < RT; ++r)
+      *reinterpret_cast<float4 *>(dst + (size_t)(rbase + r) * Dv + col) =
+          make_float4(X[r][0], X[r][1], X[r][2], X[r][3]);
+  };
+  // The 4 columns' sums over all Dk rows of a per-thread part p (one value
+  // per column): reduce-scatter over the warp's row groups, then the four
+  // warps' parts meet in buf.  Returns the thread's 4 column sums.
+  auto col_sums_post = [&](float (&p)[4], float *buf) {
+    buf[w * kCols + c4 + rg] = reduce_scatter<4, 16, 8>(p, lane);
+  };
+  auto col_sums_read = [&](const float *buf, float (&o)[4]) {
+    float x0[4], x1[4], x2[4], x3[4];
+    lds4(buf + c4, x0);
+    lds4(buf + kCols + c4, x1);
+    lds4(buf + 2 * kCols + c4, x2);
+    lds4(buf + 3 * kCols + c4, x3);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) o[c] = (x0[c] + x1[c]) + (x2[c] + x3[c]);
+  };
+  // One forward step of token slot s: S <- Diag(alpha) S + k u^T, with
+  // y_j = sum_c alpha_c k_c S_cj and u = beta (v - y).
+  auto fwd_step = [&](int s) {
+    float kr[RT], ar[RT], vv[4];
+    lds_rows<RT>(tk + s * Dk + rbase, kr);
+    lds_rows<RT>(ta + s * Dk + rbase, ar);
+    float yp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int r = 0; r < RT; ++r) {
+      const float ak = ar[r] * kr[r];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) yp[c] = fmaf(ak, S[r][c], yp[c]);
     }
     float *pp = py + par * 4 * kCols;
-    pp[w * kCols + j] = pa;
+    col_sums_post(yp, pp);
     __syncthreads();
-    const float y = (pp[j] + pp[kCols + j]) + (pp[2 * kCols + j] + pp[3 * kCols + j]);
+    float y[4];
+    col_sums_read(pp, y);
     par ^= 1;
-    const float u = tb[s] * (tv[s * kCols + j] - y);
+    lds4(tv + s * kCols + c4, vv);
+    const float bt = tb[s];
+    float u[4];
 #pragma unroll
-    for (int i = 0; i < RPW; i += 4) {
-      const float4 k4 = *reinterpret_cast<const float4 *>(k_s + i);
-      const float4 a4 = *reinterpret_cast<const float4 *>(a_s + i);
-      S[i] = fmaf(a4.x, S[i], k4.x * u);
-      S[i + 1] = fmaf(a4.y, S[i + 1], k4.y * u);
-      S[i + 2] = fmaf(a4.z, S[i + 2], k4.z * u);
-      S[i + 3] = fmaf(a4.w, S[i + 3], k4.w * u);
-    }
+    for (int c = 0; c < 4; ++c) u[c] = bt * (vv[c] - y[c]);
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) S[r][c] = fmaf(ar[r], S[r][c], kr[r] * u[c]);
   };
   // Backward step of token slot s (token t): S holds S_{t-1}, dS the gradient
   // w.r.t. S_t from later tokens.
   auto bwd_step = [&](int s, int64_t t) {
-    const float *k_s = tk + s * Dk + row0, *a_s = ta + s * Dk + row0, *q_s = tq + s * Dk + row0;
-    const float doj = tdo[s * kCols + j];
-    float pa = 0.f, pd = 0.f;
+    float kr[RT], ar[RT], qr[RT], dov[4], vv[4];
+    lds_rows<RT>(tk + s * Dk + rbase, kr);
+    lds_rows<RT>(ta + s * Dk + rbase, ar);
+    lds_rows<RT>(tq + s * Dk + rbase, qr);
+    lds4(tdo + s * kCols + c4, dov);
+    float yp[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int i = 0; i < RPW; i += 4) {
-      const float4 k4 = *reinterpret_cast<const float4 *>(k_s + i);
-      const float4 a4 = *reinterpret_cast<const float4 *>(a_s + i);
-      const float4 q4 = *reinterpret_cast<const float4 *>(q_s + i);
-      pa = fmaf(a4.x * k4.x, S[i], pa);
-      pa = fmaf(a4.y * k4.y, S[i + 1], pa);
-      pa = fmaf(a4.z * k4.z, S[i + 2], pa);
-      pa = fmaf(a4.w * k4.w, S[i + 3], pa);
-      dS[i] = fmaf(q4.x, doj, dS[i]);
-      dS[i + 1] = fmaf(q4.y, doj, dS[i + 1]);
-      dS[i + 2] = fmaf(q4.z, doj, dS[i + 2]);
-      dS[i + 3] = fmaf(q4.w, doj, dS[i + 3]);
-      pd = fmaf(k4.x, dS[i], pd);
-      pd = fmaf(k4.y, dS[i + 1], pd);
-      pd = fmaf(k4.z, dS[i + 2], pd);
-      pd = fmaf(k4.w, dS[i + 3], pd);
+    for (int r = 0; r < RT; ++r) {
+      const float ak = ar[r] * kr[r];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        yp[c] = fmaf(ak, S[r][c], yp[c]);
+        dS[r][c] = fmaf(qr[r], dov[c], dS[r][c]);
+        dp[c] = fmaf(kr[r], dS[r][c], dp[c]);
+      }
     }
     float *pp = py + par * 4 * kCols, *pq = pdu + par * 4 * kCols;
-    pp[w * kCols + j] = pa;
-    pq[w * kCols + j] = pd;
+    col_sums_post(yp, pp);
+    col_sums_post(dp, pq);
     __syncthreads();
-    const float y = (pp[j] + pp[kCols + j]) + (pp[2 * kCols + j] + pp[3 * kCols + j]);
-    const float du = (pq[j] + pq[kCols + j]) + (pq[2 * kCols + j] + pq[3 * kCols + j]);
+    float y[4], du[4];
+    col_sums_read(pp, y);
+    col_sums_read(pq, du);
     par ^= 1;
-    const float bt = tb[s], vj = tv[s * kCols + j];
-    const float u = bt * (vj - y);
-    const size_t th = (size_t)(t_begin + t) * H + h;
-    if (w == 0) a.dv[th * Dv + col] = bt * du;
-    // this slice's parts of du.(v - y) and u.do
-    float db = du * (vj - y), ud = u * doj;
+    lds4(tv + s * kCols + c4, vv);
+    const float bt = tb[s];
+    float u[4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+    for (int c = 0; c < 4; ++c) u[c] = bt * (vv[c] - y[c]);
+    const size_t th = (size_t)(t_begin + t) * H + h;
+    if (w == 0 && rg == 0)
+      *reinterpret_cast<float4 *>(a.dv + th * Dv + col) =
+          make_float4(bt * du[0], bt * du[1], bt * du[2], bt * du[3]);
+    // this slice's parts of du.(v - y) and u.do: the 4 columns, then across cg
+    float db = 0.f, ud = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      db = fmaf(du[c], vv[c] - y[c], db);
+      ud = fmaf(u[c], dov[c], ud);
+    }
+#pragma unroll
+    for (int o = 4; o > 0; o >>= 1) {
       db += __shfl_xor_sync(kFull, db, o);
       ud += __shfl_xor_sync(kFull, ud, o);
     }
     if (tid == 0) ob[th] = db;
     // row sums over the slice: r1 = S do, r3 = S du, r2 = dS u, r4 = sum_j dS_cj S_cj
-    float tmp[RPW];
+    float tmp[RT];
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) tmp[i] = S[i] * doj;
-    const float r1 = reduce_scatter<RPW>(tmp, j);
+    for (int r = 0; r < RT; ++r)
+      tmp[r] = fmaf(S[r][3], dov[3], fmaf(S[r][2], dov[2], fmaf(S[r][1], dov[1], S[r][0] * dov[0])));
+    const float r1 = reduce_scatter<RT, 4, 1>(tmp, lane);
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) tmp[i] = S[i] * du;
-    const float r3 = reduce_scatter<RPW>(tmp, j);
+    for (int r = 0; r < RT; ++r)
+      tmp[r] = fmaf(S[r][3], du[3], fmaf(S[r][2], du[2], fmaf(S[r][1], du[1], S[r][0] * du[0])));
+    const float r3 = reduce_scatter<RT, 4, 1>(tmp, lane);
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) tmp[i] = dS[i] * u;
-    const float r2 = reduce_scatter<RPW>(tmp, j);
+    for (int r = 0; r < RT; ++r)
+      tmp[r] = fmaf(dS[r][3], u[3], fmaf(dS[r][2], u[2], fmaf(dS[r][1], u[1], dS[r][0] * u[0])));
+    const float r2 = reduce_scatter<RT, 4, 1>(tmp, lane);
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) tmp[i] = dS[i] * S[i];
-    const float r4 = reduce_scatter<RPW>(tmp, j);
-    if ((j & ((1 << SHIFT) - 1)) == 0) {
-      const int c = row0 + (j >> SHIFT);
+    for (int r = 0; r < RT; ++r)
+      tmp[r] = fmaf(dS[r][3], S[r][3], fmaf(dS[r][2], S[r][2], fmaf(dS[r][1], S[r][1], dS[r][0] * S[r][0])));
+    const float r4 = reduce_scatter<RT, 4, 1>(tmp, lane);
+    if ((cg & ((1 << RSH) - 1)) == 0) {
+      const int c = rbase + (cg >> RSH);
       const float al = ta[s * Dk + c], kc = tk[s * Dk + c];
       const size_t o = th * Dk + c;
       // S_t = Diag(alpha) S_{t-1} + k u^T, so S_t do = alpha (S_{t-1} do) + k (u . do)
@@ -253,29 +329,43 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
       okk[o] = r2 - bt * al * r3;
       og[o] = al * (r4 - bt * kc * r3);
     }
-    // dS <- Diag(alpha) (dS - beta k du^T)
-    const float nbd = -bt * du;
+    // dS <- Diag(alpha) (dS - beta k du^T); k and alpha read again rather
+    // than held through the row sums, which keeps the step within 128 registers
+    lds_rows<RT>(tk + s * Dk + rbase, kr);
+    lds_rows<RT>(ta + s * Dk + rbase, ar);
 #pragma unroll
-    for (int i = 0; i < RPW; i += 4) {
-      const float4 k4 = *reinterpret_cast<const float4 *>(k_s + i);
-      const float4 a4 = *reinterpret_cast<const float4 *>(a_s + i);
-      dS[i] = a4.x * fmaf(k4.x, nbd, dS[i]);
-      dS[i + 1] = a4.y * fmaf(k4.y, nbd, dS[i + 1]);
-      dS[i + 2] = a4.z * fmaf(k4.z, nbd, dS[i + 2]);
-      dS[i + 3] = a4.w * fmaf(k4.w, nbd, dS[i + 3]);
-    }
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) dS[r][c] = ar[r] * fmaf(kr[r], -bt * du[c], dS[r][c]);
+  };
+  auto st_slot = [&](int slot) {
+    float *p = st + (size_t)slot * RPW * kBThreads;
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) p[(r * 4 + c) * kBThreads + tid] = S[r][c];
+  };
+  auto ld_slot = [&](int slot) {
+    const float *p = st + (size_t)slot * RPW * kBThreads;
+#pragma unroll
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) S[r][c] = p[(r * 4 + c) * kBThreads + tid];
   };
 
   // ---------------- forward sweep: the state at the start of every block ----------------
+  if (a.init) {
+    ld_tile(a.init + (size_t)unit * DD, S);
+  } else {
 #pragma unroll
-  for (int i = 0; i < RPW; ++i)
-    S[i] = a.init ? a.init[(size_t)unit * DD + (row0 + i) * Dv + col] : 0.f;
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) S[r][c] = 0.f;
+  }
   for (int64_t b = 0; b < nb; ++b) {
     const int64_t t_lo = b * kBlk;
     const int cnt = (int)((T - t_lo) < kBlk ? (T - t_lo) : kBlk);
-    float *dst = ck + (size_t)b * DD;
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) dst[(row0 + i) * Dv + col] = S[i];
+    st_tile(ck + (size_t)b * DD, S);
     __syncthreads();   // the previous block's tokens are no longer read
     load_tokens(t_lo, cnt, false);
     __syncthreads();
@@ -283,42 +373,36 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
   }
 
   // ---------------- reverse sweep ----------------
+  if (a.dfin) {
+    ld_tile(a.dfin + (size_t)unit * DD, dS);
+  } else {
 #pragma unroll
-  for (int i = 0; i < RPW; ++i)
-    dS[i] = a.dfin ? a.dfin[(size_t)unit * DD + (row0 + i) * Dv + col] : 0.f;
+    for (int r = 0; r < RT; ++r)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) dS[r][c] = 0.f;
+  }
   for (int64_t b = nb - 1; b >= 0; --b) {
     const int64_t t_lo = b * kBlk;
     const int cnt = (int)((T - t_lo) < kBlk ? (T - t_lo) : kBlk);
     __syncthreads();
     load_tokens(t_lo, cnt, true);
-    load_state(b);
+    ld_tile(ck + (size_t)b * DD, S);
     __syncthreads();
     // replay: S becomes the state before token slot cnt-1; the states before
-    // slots 1 .. cnt-2 are kept, each thread its own entries
+    // slots 1 .. cnt-2 are kept in slots 0 .. cnt-3, each thread its own entries
     for (int s = 0; s + 1 < cnt; ++s) {
       fwd_step(s);
-      if (s + 1 < cnt - 1) {
-        float *slot = st + (size_t)s * RPW * kBThreads;
-#pragma unroll
-        for (int i = 0; i < RPW; ++i) slot[i * kBThreads + tid] = S[i];
-      }
+      if (s + 1 < cnt - 1) st_slot(s);
     }
     for (int s = cnt - 1; s >= 0; --s) {
       if (s < cnt - 1) {
-        if (s >= 1) {
-          const float *slot = st + (size_t)(s - 1) * RPW * kBThreads;
-#pragma unroll
-          for (int i = 0; i < RPW; ++i) S[i] = slot[i * kBThreads + tid];
-        } else {
-          load_state(b);
-        }
+        if (s >= 1) ld_slot(s - 1);
+        else ld_tile(ck + (size_t)b * DD, S);
       }
       bwd_step(s, t_lo + s);
     }
   }
-  if (a.dinit)
-#pragma unroll
-    for (int i = 0; i < RPW; ++i) a.dinit[(size_t)unit * DD + (row0 + i) * Dv + col] = dS[i];
+  if (a.dinit) st_tile(a.dinit + (size_t)unit * DD, dS);
 }
 
 // dq, dk, dg, dbeta += the parts of slices 1..ns-1, in slice order.
