@@ -59,6 +59,21 @@ __device__ __forceinline__ float ld_in(const void *p, size_t i) {
   return to_f32(reinterpret_cast<const TIn *>(p)[i]);
 }
 
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Reduce-scatter across lanes: v[i] (i < M) is summed over the lanes that
 // differ in the lane bits OHI, OHI/2, ..., OLO; on return the lane holds the
 // sum for one i, i = the lane's bits OHI .. (OHI >> (log2 M - 1)) read as a
@@ -118,8 +133,8 @@ __device__ __forceinline__ void lds4(const float *p, float (&o)[4]) {
   o[3] = x.w;
 }
 
-// Shared memory, in floats.
-template <int Dk>
+// Shared memory, in floats.  ES is the byte size of a q, k, v element.
+template <int Dk, int ES>
 struct BwdSmem {
   static constexpr int PER_THREAD = Dk / 4;           // state entries per thread
   static constexpr int TK = 0;                        // k        [kBlk][Dk]
@@ -131,7 +146,14 @@ struct BwdSmem {
   static constexpr int PY = TB + 4;                   // y parts  [2][4][32]
   static constexpr int PD = PY + 2 * 4 * kCols;       // du parts [2][4][32]
   static constexpr int ST = PD + 2 * 4 * kCols;       // states   [kBlk-2][PER_THREAD][128]
-  static constexpr int TOTAL = ST + (kBlk - 2) * PER_THREAD * kBThreads;
+  // staging of the next block's tokens as they sit in global memory (bytes):
+  // k, q [kBlk][Dk] x ES; g [kBlk][Dk] x 4; v slice [kBlk][32] x ES;
+  // do slice [kBlk][32] x 4; beta [kBlk] x 4
+  static constexpr int SK = 0, SQ = SK + kBlk * Dk * ES, SG = SQ + kBlk * Dk * ES;
+  static constexpr int SV = SG + kBlk * Dk * 4, SD = SV + kBlk * kCols * ES;
+  static constexpr int SB = SD + kBlk * kCols * 4, S_BYTES = SB + 16;
+  static constexpr int STAGE = ST + (kBlk - 2) * PER_THREAD * kBThreads;
+  static constexpr int TOTAL = STAGE + S_BYTES / 4;
 };
 
 // Thread layout: warp w owns rows [w Dk/4, (w+1) Dk/4) of the slice; lane
@@ -141,7 +163,7 @@ struct BwdSmem {
 // slice's columns across cg (lane bits 4, 2, 1).
 template <typename TIn, int Dk, int Dv>
 __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a) {
-  using L = BwdSmem<Dk>;
+  using L = BwdSmem<Dk, (int)sizeof(TIn)>;
   constexpr int RPW = Dk / 4, RT = Dk / 16, NS = Dv / kCols, DD = Dk * Dv;
   constexpr int RSH = 3 - Log2<RT>::value;   // row sums: lanes sharing a row differ in cg's low RSH bits
   extern __shared__ __align__(16) float smem[];
@@ -176,21 +198,62 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
   float S[RT][4], dS[RT][4];
   int par = 0;
 
-  auto load_tokens = [&](int64_t t_lo, int cnt, bool full) {
+  char *stage = reinterpret_cast<char *>(smem + L::STAGE);
+  // Start the copies of the tokens [t_lo, t_lo + cnt) into the staging area
+  // (q and do only when full); they land while the current block computes.
+  auto issue_tokens = [&](int64_t t_lo, int cnt, bool full) {
+    constexpr int KCH = Dk * (int)sizeof(TIn) / 16, GCH = Dk * 4 / 16;
+    constexpr int VCH = kCols * (int)sizeof(TIn) / 16, DCH = kCols * 4 / 16;
+    const size_t th0 = (size_t)(t_begin + t_lo) * H + h;   // (token, head) row of t_lo
+    for (int e = tid; e < cnt * KCH; e += kBThreads) {
+      const int s = e / KCH, x = e - s * KCH;
+      const size_t off = ((th0 + (size_t)s * H) * Dk) * sizeof(TIn) + (size_t)x * 16;
+      cp_async16(stage + L::SK + e * 16, reinterpret_cast<const char *>(a.k) + off);
+      if (full) cp_async16(stage + L::SQ + e * 16, reinterpret_cast<const char *>(a.q) + off);
+    }
+    for (int e = tid; e < cnt * GCH; e += kBThreads) {
+      const int s = e / GCH, x = e - s * GCH;
+      cp_async16(stage + L::SG + e * 16,
+                 reinterpret_cast<const char *>(a.g) + ((th0 + (size_t)s * H) * Dk) * 4 + (size_t)x * 16);
+    }
+    for (int e = tid; e < cnt * VCH; e += kBThreads) {
+      const int s = e / VCH, x = e - s * VCH;
+      cp_async16(stage + L::SV + e * 16,
+                 reinterpret_cast<const char *>(a.v) +
+                     ((th0 + (size_t)s * H) * Dv + slice * kCols) * sizeof(TIn) + (size_t)x * 16);
+    }
+    if (full)
+      for (int e = tid; e < cnt * DCH; e += kBThreads) {
+        const int s = e / DCH, x = e - s * DCH;
+        cp_async16(stage + L::SD + e * 16,
+                   reinterpret_cast<const char *>(a.dout) +
+                       ((th0 + (size_t)s * H) * Dv + slice * kCols) * 4 + (size_t)x * 16);
+      }
+    if (tid < cnt) cp_async4(stage + L::SB + tid * 4, a.beta + th0 + (size_t)tid * H);
+    cp_async_commit();
+  };
+  // Staged tokens -> FP32 token arrays (alpha = exp(g)).  Called between two
+  // barriers, after every thread's copies have landed.
+  auto unpack_tokens = [&](int cnt, bool full) {
+    const TIn *sk = reinterpret_cast<const TIn *>(stage + L::SK);
+    const TIn *sq = reinterpret_cast<const TIn *>(stage + L::SQ);
+    const float *sg = reinterpret_cast<const float *>(stage + L::SG);
     for (int e = tid; e < cnt * Dk; e += kBThreads) {
-      const int s = e / Dk, c = e - s * Dk;
-      const size_t ix = ((size_t)(t_begin + t_lo + s) * H + h) * Dk + c;
-      tk[s * Dk + c] = ld_in<TIn>(a.k, ix);
-      ta[s * Dk + c] = __expf(a.g[ix]);
-      if (full) tq[s * Dk + c] = ld_in<TIn>(a.q, ix);
+      tk[e] = to_f32(sk[e]);
+      ta[e] = __expf(sg[e]);
+      if (full) tq[e] = to_f32(sq[e]);
     }
+    const TIn *sv = reinterpret_cast<const TIn *>(stage + L::SV);
+    const float *sd = reinterpret_cast<const float *>(stage + L::SD);
     for (int e = tid; e < cnt * kCols; e += kBThreads) {
-      const int s = e >> 5, jj = e & 31;
-      const size_t ix = ((size_t)(t_begin + t_lo + s) * H + h) * Dv + slice * kCols + jj;
-      tv[s * kCols + jj] = ld_in<TIn>(a.v, ix);
-      if (full) tdo[s * kCols + jj] = a.dout[ix];
+      tv[e] = to_f32(sv[e]);
+      if (full) tdo[e] = sd[e];
     }
-    if (tid < cnt) tb[tid] = a.beta[(size_t)(t_begin + t_lo + tid) * H + h];
+    if (tid < cnt) tb[tid] = reinterpret_cast<const float *>(stage + L::SB)[tid];
+  };
+  // L2 prefetch of a stored state's slice: one 128-byte line per row.
+  auto prefetch_state = [&](int64_t b) {
+    if (tid < Dk) prefetch_l2(ck + (size_t)b * DD + (size_t)tid * Dv + slice * kCols);
   };
   // a [Dk][Dv] FP32 matrix in global memory <-> the thread's tile
   auto ld_tile = [&](const float *src, float (&X)[RT][4]) {
@@ -362,13 +425,16 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
 #pragma unroll
       for (int c = 0; c < 4; ++c) S[r][c] = 0.f;
   }
+  auto block_len = [&](int64_t b) { return (int)((T - b * kBlk) < kBlk ? (T - b * kBlk) : kBlk); };
+  if (nb > 0) issue_tokens(0, block_len(0), false);
   for (int64_t b = 0; b < nb; ++b) {
-    const int64_t t_lo = b * kBlk;
-    const int cnt = (int)((T - t_lo) < kBlk ? (T - t_lo) : kBlk);
+    const int cnt = block_len(b);
     st_tile(ck + (size_t)b * DD, S);
-    __syncthreads();   // the previous block's tokens are no longer read
-    load_tokens(t_lo, cnt, false);
-    __syncthreads();
+    cp_async_wait_all();
+    __syncthreads();   // staged tokens visible; the previous block's tokens no longer read
+    unpack_tokens(cnt, false);
+    __syncthreads();   // tokens visible; staging free
+    if (b + 1 < nb) issue_tokens((b + 1) * kBlk, block_len(b + 1), false);
     for (int s = 0; s < cnt; ++s) fwd_step(s);
   }
 
@@ -381,13 +447,22 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
 #pragma unroll
       for (int c = 0; c < 4; ++c) dS[r][c] = 0.f;
   }
+  if (nb > 0) {
+    issue_tokens((nb - 1) * kBlk, block_len(nb - 1), true);
+    prefetch_state(nb - 1);
+  }
   for (int64_t b = nb - 1; b >= 0; --b) {
     const int64_t t_lo = b * kBlk;
-    const int cnt = (int)((T - t_lo) < kBlk ? (T - t_lo) : kBlk);
+    const int cnt = block_len(b);
+    cp_async_wait_all();
     __syncthreads();
-    load_tokens(t_lo, cnt, true);
+    unpack_tokens(cnt, true);
+    __syncthreads();
+    if (b > 0) {
+      issue_tokens((b - 1) * kBlk, kBlk, true);
+      prefetch_state(b - 1);
+    }
     ld_tile(ck + (size_t)b * DD, S);
-    __syncthreads();
     // replay: S becomes the state before token slot cnt-1; the states before
     // slots 1 .. cnt-2 are kept in slots 0 .. cnt-3, each thread its own entries
     for (int s = 0; s + 1 < cnt; ++s) {
@@ -438,11 +513,12 @@ __global__ void __launch_bounds__(256) backward_sum_kernel(float *__restrict__ d
 
 }  // namespace
 
-size_t backward_smem_bytes(int Dk) {
+template <int ES>
+static size_t backward_smem_bytes(int Dk) {
   switch (Dk) {
-    case 32: return sizeof(float) * BwdSmem<32>::TOTAL;
-    case 64: return sizeof(float) * BwdSmem<64>::TOTAL;
-    default: return sizeof(float) * BwdSmem<128>::TOTAL;
+    case 32: return sizeof(float) * BwdSmem<32, ES>::TOTAL;
+    case 64: return sizeof(float) * BwdSmem<64, ES>::TOTAL;
+    default: return sizeof(float) * BwdSmem<128, ES>::TOTAL;
   }
 }
 
@@ -458,7 +534,7 @@ size_t backward_workspace_bytes(int N, int H, int64_t T, int Dk, int Dv) {
 
 template <typename TIn, int DK, int DV>
 static cudaError_t launch_backward_t(const BwdArgs &args, int N, cudaStream_t stream) {
-  const size_t smem = backward_smem_bytes(DK);
+  const size_t smem = backward_smem_bytes<(int)sizeof(TIn)>(DK);
   cudaError_t e = cudaFuncSetAttribute(backward_kernel<TIn, DK, DV>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
