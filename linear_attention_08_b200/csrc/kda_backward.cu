@@ -435,7 +435,12 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     unpack_tokens(cnt, false);
     __syncthreads();   // tokens visible; staging free
     if (b + 1 < nb) issue_tokens((b + 1) * kBlk, block_len(b + 1), false);
-    for (int s = 0; s < cnt; ++s) fwd_step(s);
+    if (cnt == kBlk) {
+#pragma unroll
+      for (int s = 0; s < kBlk; ++s) fwd_step(s);
+    } else {
+      for (int s = 0; s < cnt; ++s) fwd_step(s);
+    }
   }
 
   // ---------------- reverse sweep ----------------
@@ -465,16 +470,32 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     ld_tile(ck + (size_t)b * DD, S);
     // replay: S becomes the state before token slot cnt-1; the states before
     // slots 1 .. cnt-2 are kept in slots 0 .. cnt-3, each thread its own entries
-    for (int s = 0; s + 1 < cnt; ++s) {
-      fwd_step(s);
-      if (s + 1 < cnt - 1) st_slot(s);
-    }
-    for (int s = cnt - 1; s >= 0; --s) {
-      if (s < cnt - 1) {
-        if (s >= 1) ld_slot(s - 1);
-        else ld_tile(ck + (size_t)b * DD, S);
+    if (cnt == kBlk) {   // full block: token slots are compile-time constants
+#pragma unroll
+      for (int s = 0; s + 1 < kBlk; ++s) {
+        fwd_step(s);
+        if (s + 1 < kBlk - 1) st_slot(s);
       }
-      bwd_step(s, t_lo + s);
+#pragma unroll
+      for (int s = kBlk - 1; s >= 0; --s) {
+        if (s < kBlk - 1) {
+          if (s >= 1) ld_slot(s - 1);
+          else ld_tile(ck + (size_t)b * DD, S);
+        }
+        bwd_step(s, t_lo + s);
+      }
+    } else {
+      for (int s = 0; s + 1 < cnt; ++s) {
+        fwd_step(s);
+        if (s + 1 < cnt - 1) st_slot(s);
+      }
+      for (int s = cnt - 1; s >= 0; --s) {
+        if (s < cnt - 1) {
+          if (s >= 1) ld_slot(s - 1);
+          else ld_tile(ck + (size_t)b * DD, S);
+        }
+        bwd_step(s, t_lo + s);
+      }
     }
   }
   if (a.dinit) st_tile(a.dinit + (size_t)unit * DD, dS);
