@@ -171,6 +171,22 @@ def test_prefill_at_requires_all_position_pointers():
                               None) == kda.KDA_ERR_INVALID_ARGUMENT
 
 
+@pytest.mark.parametrize("Dk,Dv", [(32, 32), (64, 64), (128, 128), (128, 32)])
+def test_backward_workspace_covers_states_and_slice_parts(Dk, Dv):
+    """A stored state per 4-token block of every sequence (ragged lengths round
+    up), plus, for each 32-column value slice after the first, the slice's
+    dq, dk, dg and dbeta parts."""
+    lib = kda.load()
+    lengths = [5, 0, 8, 1]
+    T, N, H = sum(lengths), len(lengths), 3
+    s = kda.make_shape(N, T, H, Dk, Dv, 0, kda.KDA_DTYPE_F32)
+    need = lib.kda_backward_workspace_bytes(ctypes.byref(s))
+    bound_blocks = (T + 3 * N) // 4            # >= sum of ceil(T_n / 4) = 2 + 0 + 2 + 1
+    assert bound_blocks >= sum((L + 3) // 4 for L in lengths)
+    extra = Dv // 32 - 1
+    assert need == bound_blocks * H * Dk * Dv * 4 + extra * T * H * (3 * Dk + 1) * 4
+
+
 def test_backward_workspace_and_validation():
     lib = kda.load()
     s = kda.make_shape(2, 1000, 4, 128, 64, 0, kda.KDA_DTYPE_BF16)
