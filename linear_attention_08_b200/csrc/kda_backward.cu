@@ -16,20 +16,22 @@
 // Column j of S only ever meets column j of dS, v, do, u and du: the
 // recurrence and its reverse split by value columns.  Only dq, dk, dg and
 // dbeta sum over columns, and those sums are linear.  So one CTA of 128
-// threads takes one (sequence, head, slice of 32 value columns): lane j owns
-// column j of the slice, warp w the rows [w D_k/4, (w+1) D_k/4), and the
-// thread keeps its D_k/4 entries of S and of dS in registers.  Column sums
-// (y, du) cross the four warps through a small shared array; row sums (the
-// parts of dq, dk, dg) are reduce-scattered across the warp's lanes by
-// shuffles, so each lane ends with one row's sum.  Slice 0 writes dq, dk, dg,
-// dbeta; slices 1.. write their parts to the workspace, and a second kernel
-// adds them in slice order.
+// threads takes one (sequence, head, slice of 32 value columns).  Warp w owns
+// the rows [w D_k/4, (w+1) D_k/4); each thread keeps a tile of D_k/16 rows x
+// 4 columns of S and of dS in registers.  Column sums (y, du) are summed over
+// the tile's rows, reduce-scattered over the warp's row groups, and the four
+// warps' parts meet in a small shared array (one barrier per step).  Row sums
+// (the parts of dq, dk, dg) are summed over the tile's 4 columns and
+// reduce-scattered over the warp's 8 column groups, so each lane ends with one
+// row's sum.  Slice 0 writes dq, dk, dg, dbeta; slices 1.. write their parts
+// to the workspace, and a second kernel adds them in slice order.
 //
 // A forward sweep stores the state at the start of every block of kBlk
 // tokens in the workspace.  The reverse sweep walks the blocks backwards:
 // it reloads the block's state, replays the block once (keeping the states
 // before its middle tokens in shared memory, the last one in registers), and
-// then takes the backward steps from the last token down.
+// then takes the backward steps from the last token down.  The next block's
+// tokens are staged by cp.async while the current block computes.
 #include <stdint.h>
 
 #include "kda_common.cuh"
