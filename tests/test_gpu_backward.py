@@ -53,3 +53,30 @@ def test_backward_without_init_or_final_gradient():
 def test_backward_empty_sequence_passes_final_gradient_through():
     errs = run_both([0, 20, 0], 1, 32, 32, torch.float32, seed=7)
     assert errs["d_init"] <= 1e-6
+
+
+def test_backward_bench_shape_sampled_heads():
+    """The bench's backward workload (4 sequences x 1024 tokens, H = 32, D = 128,
+    BF16 q/k/v, FP32 state N(0, 0.02^2), N(0, 1) upstream gradients), run whole
+    on the GPU in the launch configuration the bench times (4 column slices per
+    head plus the slice-sum kernel).  Three heads are recomputed by the oracle
+    and compared in full."""
+    lengths, H, D = [1024] * 4, 32, 128
+    d = make_case(lengths, H, D, D, torch.bfloat16, seed=11, state_std=0.02)
+    dd = to_device(d)
+    rng = np.random.default_rng(111)
+    T = sum(lengths)
+    d_out = torch.tensor(rng.normal(size=(T, H, D)), dtype=torch.float32)
+    d_fin = torch.tensor(rng.normal(size=(len(lengths), H, D, D)), dtype=torch.float32)
+    got = kda.kda_backward(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu_dev"],
+                           d_out.cuda(), init_state=dd["init_state"], d_final=d_fin.cuda())
+    torch.cuda.synchronize()
+    got = [x.cpu() for x in got]
+    for h in (0, 13, 31):
+        hs = slice(h, h + 1)
+        ref = oracle.backward(d["q"][:, hs], d["k"][:, hs], d["v"][:, hs], d["g"][:, hs],
+                              d["beta"][:, hs], d["cu_seqlens"], d_out[:, hs],
+                              init_state=d["init_state"][:, hs], d_final=d_fin[:, hs])
+        for name, x, r in zip(NAMES, got, ref):
+            e = rel_l2(x[:, hs], r)
+            assert e <= 1e-4, f"head {h} {name}: rel-L2 {e:.3e}"
