@@ -197,7 +197,9 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     ob = a.part + 3 * (NS - 1) * n_k + s1 * (size_t)a.T * H;
   }
 
-  float S[RT][4], dS[RT][4];
+  // the thread's tile of S and dS: per row, columns (0, 1) and (2, 3) as
+  // pairs for the paired FP32 units
+  float2 S[RT][2], dS[RT][2];
   int par = 0;
 
   char *stage = reinterpret_cast<char *>(smem + L::STAGE);
@@ -258,27 +260,26 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     if (tid < Dk) prefetch_l2(ck + (size_t)b * DD + (size_t)tid * Dv + slice * kCols);
   };
   // a [Dk][Dv] FP32 matrix in global memory <-> the thread's tile
-  auto ld_tile = [&](const float *src, float (&X)[RT][4]) {
+  auto ld_tile = [&](const float *src, float2 (&X)[RT][2]) {
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
       const float4 x = *reinterpret_cast<const float4 *>(src + (size_t)(rbase + r) * Dv + col);
-      X[r][0] = x.x;
-      X[r][1] = x.y;
-      X[r][2] = x.z;
-      X[r][3] = x.w;
+      X[r][0] = make_float2(x.x, x.y);
+      X[r][1] = make_float2(x.z, x.w);
     }
   };
-  auto st_tile = [&](float *dst, const float (&X)[RT][4]) {
+  auto st_tile = [&](float *dst, const float2 (&X)[RT][2]) {
 #pragma unroll
     for (int r = 0; r < RT; ++r)
       *reinterpret_cast<float4 *>(dst + (size_t)(rbase + r) * Dv + col) =
-          make_float4(X[r][0], X[r][1], X[r][2], X[r][3]);
+          make_float4(X[r][0].x, X[r][0].y, X[r][1].x, X[r][1].y);
   };
   // The 4 columns' sums over all Dk rows of a per-thread part p (one value
   // per column): reduce-scatter over the warp's row groups, then the four
-  // warps' parts meet in buf.  Returns the thread's 4 column sums.
-  auto col_sums_post = [&](float (&p)[4], float *buf) {
-    buf[w * kCols + c4 + rg] = reduce_scatter<4, 16, 8>(p, lane);
+  // warps' parts meet in buf.
+  auto col_sums_post = [&](const float2 (&p)[2], float *buf) {
+    float v[4] = {p[0].x, p[0].y, p[1].x, p[1].y};
+    buf[w * kCols + c4 + rg] = reduce_scatter<4, 16, 8>(v, lane);
   };
   auto col_sums_read = [&](const float *buf, float (&o)[4]) {
     float x0[4], x1[4], x2[4], x3[4];
@@ -295,12 +296,13 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     float kr[RT], ar[RT], vv[4];
     lds_rows<RT>(tk + s * Dk + rbase, kr);
     lds_rows<RT>(ta + s * Dk + rbase, ar);
-    float yp[4] = {0.f, 0.f, 0.f, 0.f};
+    float2 yp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
       const float ak = ar[r] * kr[r];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) yp[c] = fmaf(ak, S[r][c], yp[c]);
+      const float2 ak2 = make_float2(ak, ak);
+      yp[0] = __ffma2_rn(ak2, S[r][0], yp[0]);
+      yp[1] = __ffma2_rn(ak2, S[r][1], yp[1]);
     }
     float *pp = py + par * 4 * kCols;
     col_sums_post(yp, pp);
@@ -310,56 +312,69 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     par ^= 1;
     lds4(tv + s * kCols + c4, vv);
     const float bt = tb[s];
-    float u[4];
+    const float2 u[2] = {make_float2(bt * (vv[0] - y[0]), bt * (vv[1] - y[1])),
+                         make_float2(bt * (vv[2] - y[2]), bt * (vv[3] - y[3]))};
 #pragma unroll
-    for (int c = 0; c < 4; ++c) u[c] = bt * (vv[c] - y[c]);
+    for (int r = 0; r < RT; ++r) {
+      const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
+      S[r][0] = __ffma2_rn(a2, S[r][0], __fmul2_rn(k2, u[0]));
+      S[r][1] = __ffma2_rn(a2, S[r][1], __fmul2_rn(k2, u[1]));
+    }
+  };
+  // sum over the thread's 4 columns of X[r][.] * Y[.], for every row r
+  auto row_dots = [&](const float2 (&X)[RT][2], const float2 (&Y)[2], float (&o)[RT]) {
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) S[r][c] = fmaf(ar[r], S[r][c], kr[r] * u[c]);
+    for (int r = 0; r < RT; ++r) {
+      const float2 t = __ffma2_rn(X[r][1], Y[1], __fmul2_rn(X[r][0], Y[0]));
+      o[r] = t.x + t.y;
+    }
   };
   // Backward step of token slot s (token t): S holds S_{t-1}, dS the gradient
   // w.r.t. S_t from later tokens.
   auto bwd_step = [&](int s, int64_t t) {
-    float kr[RT], ar[RT], qr[RT], dov[4], vv[4];
+    float kr[RT], ar[RT], qr[RT], dov4[4], vv[4];
     lds_rows<RT>(tk + s * Dk + rbase, kr);
     lds_rows<RT>(ta + s * Dk + rbase, ar);
     lds_rows<RT>(tq + s * Dk + rbase, qr);
-    lds4(tdo + s * kCols + c4, dov);
-    float yp[4] = {0.f, 0.f, 0.f, 0.f}, dp[4] = {0.f, 0.f, 0.f, 0.f};
+    lds4(tdo + s * kCols + c4, dov4);
+    const float2 dov[2] = {make_float2(dov4[0], dov4[1]), make_float2(dov4[2], dov4[3])};
+    float2 yp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}, dp[2] = {yp[0], yp[0]};
 #pragma unroll
     for (int r = 0; r < RT; ++r) {
       const float ak = ar[r] * kr[r];
+      const float2 ak2 = make_float2(ak, ak), q2 = make_float2(qr[r], qr[r]);
+      const float2 k2 = make_float2(kr[r], kr[r]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        yp[c] = fmaf(ak, S[r][c], yp[c]);
-        dS[r][c] = fmaf(qr[r], dov[c], dS[r][c]);
-        dp[c] = fmaf(kr[r], dS[r][c], dp[c]);
+      for (int h2 = 0; h2 < 2; ++h2) {
+        yp[h2] = __ffma2_rn(ak2, S[r][h2], yp[h2]);
+        dS[r][h2] = __ffma2_rn(q2, dov[h2], dS[r][h2]);
+        dp[h2] = __ffma2_rn(k2, dS[r][h2], dp[h2]);
       }
     }
     float *pp = py + par * 4 * kCols, *pq = pdu + par * 4 * kCols;
     col_sums_post(yp, pp);
     col_sums_post(dp, pq);
     __syncthreads();
-    float y[4], du[4];
+    float y[4], du4[4];
     col_sums_read(pp, y);
-    col_sums_read(pq, du);
+    col_sums_read(pq, du4);
     par ^= 1;
     lds4(tv + s * kCols + c4, vv);
     const float bt = tb[s];
-    float u[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) u[c] = bt * (vv[c] - y[c]);
+    const float2 u[2] = {make_float2(bt * (vv[0] - y[0]), bt * (vv[1] - y[1])),
+                         make_float2(bt * (vv[2] - y[2]), bt * (vv[3] - y[3]))};
+    const float2 du[2] = {make_float2(du4[0], du4[1]), make_float2(du4[2], du4[3])};
     const size_t th = (size_t)(t_begin + t) * H + h;
     if (w == 0 && rg == 0)
       *reinterpret_cast<float4 *>(a.dv + th * Dv + col) =
-          make_float4(bt * du[0], bt * du[1], bt * du[2], bt * du[3]);
+          make_float4(bt * du4[0], bt * du4[1], bt * du4[2], bt * du4[3]);
     // this slice's parts of du.(v - y) and u.do: the 4 columns, then across cg
+    const float u4[4] = {u[0].x, u[0].y, u[1].x, u[1].y};
     float db = 0.f, ud = 0.f;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      db = fmaf(du[c], vv[c] - y[c], db);
-      ud = fmaf(u[c], dov[c], ud);
+      db = fmaf(du4[c], vv[c] - y[c], db);
+      ud = fmaf(u4[c], dov4[c], ud);
     }
 #pragma unroll
     for (int o = 4; o > 0; o >>= 1) {
@@ -369,21 +384,17 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     if (tid == 0) ob[th] = db;
     // row sums over the slice: r1 = S do, r3 = S du, r2 = dS u, r4 = sum_j dS_cj S_cj
     float tmp[RT];
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-      tmp[r] = fmaf(S[r][3], dov[3], fmaf(S[r][2], dov[2], fmaf(S[r][1], dov[1], S[r][0] * dov[0])));
+    row_dots(S, dov, tmp);
     const float r1 = reduce_scatter<RT, 4, 1>(tmp, lane);
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-      tmp[r] = fmaf(S[r][3], du[3], fmaf(S[r][2], du[2], fmaf(S[r][1], du[1], S[r][0] * du[0])));
+    row_dots(S, du, tmp);
     const float r3 = reduce_scatter<RT, 4, 1>(tmp, lane);
-#pragma unroll
-    for (int r = 0; r < RT; ++r)
-      tmp[r] = fmaf(dS[r][3], u[3], fmaf(dS[r][2], u[2], fmaf(dS[r][1], u[1], dS[r][0] * u[0])));
+    row_dots(dS, u, tmp);
     const float r2 = reduce_scatter<RT, 4, 1>(tmp, lane);
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-      tmp[r] = fmaf(dS[r][3], S[r][3], fmaf(dS[r][2], S[r][2], fmaf(dS[r][1], S[r][1], dS[r][0] * S[r][0])));
+    for (int r = 0; r < RT; ++r) {
+      const float2 x = __ffma2_rn(dS[r][1], S[r][1], __fmul2_rn(dS[r][0], S[r][0]));
+      tmp[r] = x.x + x.y;
+    }
     const float r4 = reduce_scatter<RT, 4, 1>(tmp, lane);
     if ((cg & ((1 << RSH) - 1)) == 0) {
       const int c = rbase + (cg >> RSH);
@@ -398,24 +409,32 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     // than held through the row sums, which keeps the step within 128 registers
     lds_rows<RT>(tk + s * Dk + rbase, kr);
     lds_rows<RT>(ta + s * Dk + rbase, ar);
+    const float2 nbd[2] = {make_float2(-bt * du4[0], -bt * du4[1]),
+                           make_float2(-bt * du4[2], -bt * du4[3])};
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) dS[r][c] = ar[r] * fmaf(kr[r], -bt * du[c], dS[r][c]);
+    for (int r = 0; r < RT; ++r) {
+      const float2 a2 = make_float2(ar[r], ar[r]), k2 = make_float2(kr[r], kr[r]);
+      dS[r][0] = __fmul2_rn(a2, __ffma2_rn(k2, nbd[0], dS[r][0]));
+      dS[r][1] = __fmul2_rn(a2, __ffma2_rn(k2, nbd[1], dS[r][1]));
+    }
   };
   auto st_slot = [&](int slot) {
     float *p = st + (size_t)slot * RPW * kBThreads;
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) p[(r * 4 + c) * kBThreads + tid] = S[r][c];
+    for (int r = 0; r < RT; ++r) {
+      p[(r * 4 + 0) * kBThreads + tid] = S[r][0].x;
+      p[(r * 4 + 1) * kBThreads + tid] = S[r][0].y;
+      p[(r * 4 + 2) * kBThreads + tid] = S[r][1].x;
+      p[(r * 4 + 3) * kBThreads + tid] = S[r][1].y;
+    }
   };
   auto ld_slot = [&](int slot) {
     const float *p = st + (size_t)slot * RPW * kBThreads;
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) S[r][c] = p[(r * 4 + c) * kBThreads + tid];
+    for (int r = 0; r < RT; ++r) {
+      S[r][0] = make_float2(p[(r * 4 + 0) * kBThreads + tid], p[(r * 4 + 1) * kBThreads + tid]);
+      S[r][1] = make_float2(p[(r * 4 + 2) * kBThreads + tid], p[(r * 4 + 3) * kBThreads + tid]);
+    }
   };
 
   // ---------------- forward sweep: the state at the start of every block ----------------
@@ -423,9 +442,7 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     ld_tile(a.init + (size_t)unit * DD, S);
   } else {
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) S[r][c] = 0.f;
+    for (int r = 0; r < RT; ++r) S[r][0] = S[r][1] = make_float2(0.f, 0.f);
   }
   auto block_len = [&](int64_t b) { return (int)((T - b * kBlk) < kBlk ? (T - b * kBlk) : kBlk); };
   if (nb > 0) issue_tokens(0, block_len(0), false);
@@ -450,9 +467,7 @@ __global__ void __launch_bounds__(kBThreads, 4) backward_kernel(const BwdArgs a)
     ld_tile(a.dfin + (size_t)unit * DD, dS);
   } else {
 #pragma unroll
-    for (int r = 0; r < RT; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) dS[r][c] = 0.f;
+    for (int r = 0; r < RT; ++r) dS[r][0] = dS[r][1] = make_float2(0.f, 0.f);
   }
   if (nb > 0) {
     issue_tokens((nb - 1) * kBlk, block_len(nb - 1), true);

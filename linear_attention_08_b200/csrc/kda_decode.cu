@@ -181,9 +181,14 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
   }
 
   float4 *S4 = reinterpret_cast<float4 *>(state + (size_t)unit * DK * DV);
-  float4 s[ROWS];
+  // the thread's float4 of each row as two pairs, for the paired FP32 units
+  float2 sa[ROWS], sb[ROWS];
 #pragma unroll
-  for (int i = 0; i < ROWS; ++i) s[i] = __ldcs(&S4[(rg + i * RPP) * V4 + cg]);
+  for (int i = 0; i < ROWS; ++i) {
+    const float4 x = __ldcs(&S4[(rg + i * RPP) * V4 + cg]);
+    sa[i] = make_float2(x.x, x.y);
+    sb[i] = make_float2(x.z, x.w);
+  }
 
   for (int t0 = 0; t0 < T_new; t0 += G) {
     const int cnt = T_new - t0 < G ? T_new - t0 : G;
@@ -217,16 +222,19 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 
     for (int j = 0; j < cnt; ++j) {
       const int t = t0 + j, p = t & 1;   // parity-indexed buffers: no third barrier
-      float4 y = make_float4(0.f, 0.f, 0.f, 0.f), z = y;
+      float2 ya = make_float2(0.f, 0.f), yb = ya, za = ya, zb = ya;
 #pragma unroll
       for (int i = 0; i < ROWS; ++i) {
         const int r = rg + i * RPP;
-        const float ka = s_ka[j][r], qa = s_qa[j][r];
-        y.x += ka * s[i].x; y.y += ka * s[i].y; y.z += ka * s[i].z; y.w += ka * s[i].w;
-        z.x += qa * s[i].x; z.y += qa * s[i].y; z.z += qa * s[i].z; z.w += qa * s[i].w;
+        const float2 ka = make_float2(s_ka[j][r], s_ka[j][r]);
+        const float2 qa = make_float2(s_qa[j][r], s_qa[j][r]);
+        ya = __ffma2_rn(ka, sa[i], ya);
+        yb = __ffma2_rn(ka, sb[i], yb);
+        za = __ffma2_rn(qa, sa[i], za);
+        zb = __ffma2_rn(qa, sb[i], zb);
       }
-      s_red[p][0][rg][cg] = y;
-      s_red[p][1][rg][cg] = z;
+      s_red[p][0][rg][cg] = make_float4(ya.x, ya.y, yb.x, yb.y);
+      s_red[p][1][rg][cg] = make_float4(za.x, za.y, zb.x, zb.y);
       __syncthreads();
       if (tid < DV) {
         const int c4 = tid >> 2, lane4 = tid & 3;
@@ -242,18 +250,19 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
       }
       __syncthreads();
       const float4 u4 = reinterpret_cast<const float4 *>(s_u[p])[cg];
+      const float2 ua = make_float2(u4.x, u4.y), ub = make_float2(u4.z, u4.w);
 #pragma unroll
       for (int i = 0; i < ROWS; ++i) {
         const int r = rg + i * RPP;
-        const float a = s_alpha[j][r], kc = s_k[j][r];
-        s[i].x = a * s[i].x + kc * u4.x;
-        s[i].y = a * s[i].y + kc * u4.y;
-        s[i].z = a * s[i].z + kc * u4.z;
-        s[i].w = a * s[i].w + kc * u4.w;
+        const float2 a = make_float2(s_alpha[j][r], s_alpha[j][r]);
+        const float2 kc = make_float2(s_k[j][r], s_k[j][r]);
+        sa[i] = __ffma2_rn(a, sa[i], __fmul2_rn(kc, ua));
+        sb[i] = __ffma2_rn(a, sb[i], __fmul2_rn(kc, ub));
       }
       if (t + 1 == acc)
 #pragma unroll
-        for (int i = 0; i < ROWS; ++i) __stcs(&S4[(rg + i * RPP) * V4 + cg], s[i]);
+        for (int i = 0; i < ROWS; ++i)
+          __stcs(&S4[(rg + i * RPP) * V4 + cg], make_float4(sa[i].x, sa[i].y, sb[i].x, sb[i].y));
     }
     __syncthreads();   // the staged group is overwritten by the next one
   }
