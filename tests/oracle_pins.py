@@ -80,6 +80,32 @@ def pin_pure_decay(lib):
     return float(err)
 
 
+# --- I3: one gate for all channels (gated DeltaNet) is DeltaNet on rescaled values ----
+# With g_t,c = gamma_t for every channel, Diag(alpha_t) = e^{gamma_t} I commutes
+# with (I - b k k^T).  Dividing by P_t = exp(gamma_1 + ... + gamma_t) gives
+# S_t / P_t = (I - b k k^T)(S_{t-1} / P_{t-1}) + b k (v_t / P_t)^T: the g = 0
+# recurrence (DeltaNet) on values v_t / P_t.  A decay applied after the delta
+# step, or a gate taken from the wrong token, breaks the identity.
+def pin_scalar_gate(lib):
+    rng = np.random.default_rng(17)
+    p = rand_problem(rng, [7, 5], 2, 4, 3)
+    T, H = p["q"].shape[:2]
+    gamma = -rng.uniform(0.0, 0.6, (T, H))
+    p["g"] = np.repeat(gamma[:, :, None], 4, axis=2)
+    out, fin, _ = _run(lib, p)
+    P = np.empty((T, H))
+    for n in range(2):
+        a, b = p["cu_seqlens"][n], p["cu_seqlens"][n + 1]
+        P[a:b] = np.exp(np.cumsum(gamma[a:b], axis=0))
+    q = dict(p, g=np.zeros_like(p["g"]), v=p["v"] / P[:, :, None])
+    out0, fin0, _ = _run(lib, q)
+    err = np.abs(out - out0 * P[:, :, None]).max()
+    for n in range(2):
+        last = p["cu_seqlens"][n + 1] - 1
+        err = max(err, np.abs(fin[n] - fin0[n] * P[last][:, None, None]).max())
+    return float(err)
+
+
 # --- I5: the explicit matrix product form (I - b k k^T) Diag(a) S + b k v^T -----------
 def pin_matrix_form(lib):
     rng = np.random.default_rng(14)
@@ -311,6 +337,7 @@ PINS = {
     "identity_tokens": (pin_identity_tokens, 1e-15),
     "delta_retrieval": (pin_delta_retrieval, 1e-12),
     "pure_decay": (pin_pure_decay, 1e-12),
+    "scalar_gate": (pin_scalar_gate, 1e-12),
     "matrix_form": (pin_matrix_form, 1e-12),
     "closed_form_sum": (pin_closed_form_sum, 1e-12),
     "exact_rational": (pin_exact_rational, 1e-14),

@@ -17,6 +17,9 @@ MUTATIONS = {
     "delta_sign": ("S[c * Dv + j] += bt * kt[c] * (vt[j] - y[j]);",
                    "S[c * Dv + j] += bt * kt[c] * (vt[j] + y[j]);"),
     "retrieve_with_q": ("y[j] += S[c * Dv + j] * kt[c];", "y[j] += S[c * Dv + j] * qt[c];"),
+    # the delta rule applied to the state before its decay (retrieval from S_{t-1})
+    "retrieve_before_decay": ("y[j] += S[c * Dv + j] * kt[c];",
+                              "y[j] += S[c * Dv + j] * kt[c] / exp(gt[c]);"),
     "drop_beta": ("S[c * Dv + j] += bt * kt[c] * (vt[j] - y[j])", "S[c * Dv + j] += kt[c] * (vt[j] - y[j])"),
     "output_with_k": ("ot[j] += S[c * Dv + j] * qt[c];", "ot[j] += S[c * Dv + j] * kt[c];"),
     "ckpt_off_by_one": ("(t + 1 - t0) % p->ckpt_interval", "(t + 2 - t0) % p->ckpt_interval"),
