@@ -12,6 +12,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -106,21 +107,26 @@ def _worker(rank, world, port, bounds, q):
     dist.destroy_process_group()
 
 
-def test_prefill_cp_two_ranks_gloo():
-    bounds = [0, 192, 250]
+@pytest.mark.parametrize("bounds", [[0, 192, 250], [0, 64, 192, 250]],
+                         ids=["two_ranks", "three_ranks"])
+def test_prefill_cp_gloo(bounds):
+    """Consecutive segments on 2 or 3 gloo ranks; the last segment is ragged
+    and the three-rank case folds two incoming transitions."""
+    world = len(bounds) - 1
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, bounds, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, bounds, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = dict((r, (o, f, c)) for r, o, f, c in (q.get(timeout=120) for _ in range(2)))
+    res = dict((r, (o, f, c)) for r, o, f, c in (q.get(timeout=120) for _ in range(world)))
     for p in procs:
         p.join(timeout=120)
         assert p.exitcode == 0
     x = _sequence(bounds[-1], 2, 8, 6, seed=2)
     ro, rf, rc = _whole(x, 64)
-    out = np.concatenate([res[0][0], res[1][0]])
+    out = np.concatenate([res[r][0] for r in range(world)])
     np.testing.assert_allclose(out, ro, rtol=1e-9, atol=1e-9)
-    np.testing.assert_allclose(res[1][1], rf[0], rtol=1e-9, atol=1e-9)
-    np.testing.assert_allclose(np.concatenate([res[0][2], res[1][2]]), rc, rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(res[world - 1][1], rf[0], rtol=1e-9, atol=1e-9)
+    np.testing.assert_allclose(np.concatenate([res[r][2] for r in range(world)]), rc,
+                               rtol=1e-9, atol=1e-9)
