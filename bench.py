@@ -80,6 +80,7 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "decode": ("kda_decode.cu", "kda_common.cuh"),
+    "decode_multi": ("kda_decode_multi.cu", "kda_common.cuh"),
     "prefill_tc": ("kda_prefill_tc.cu", "kda_tc_util.cuh", "kda_tma.cuh", "kda_common.cuh"),
     # two-pass path: intra-chunk pass + chain pass, one prefill call = one launch of each
     "prefill_split": ("kda_prefill_split.cu", "kda_tc_util.cuh", "kda_tma.cuh", "kda_common.cuh"),
