@@ -130,3 +130,46 @@ def test_prefill_cp_gloo(bounds):
     np.testing.assert_allclose(res[world - 1][1], rf[0], rtol=1e-9, atol=1e-9)
     np.testing.assert_allclose(np.concatenate([res[r][2] for r in range(world)]), rc,
                                rtol=1e-9, atol=1e-9)
+
+
+
+def _worker_bad_interval(rank, world, port, q):
+    import datetime
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world))
+    import torch.distributed as dist
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=5))
+    x = _sequence(100, 1, 4, 4, seed=3)
+    a, b = (0, 50) if rank == 0 else (50, 100)
+    try:
+        cp.prefill_cp(x["q"][a:b], x["k"][a:b], x["v"][a:b], x["g"][a:b], x["beta"][a:b],
+                      chunk=16, ckpt_interval=16, ops=OracleOps())
+        q.put((rank, "ok"))
+    except ValueError:
+        q.put((rank, "ValueError"))
+    except Exception:   # the last rank's all-gather times out: its peer never joined
+        q.put((rank, "collective error"))
+    try:
+        dist.destroy_process_group()
+    except Exception:
+        pass
+
+
+def test_prefill_cp_rejects_unaligned_segment():
+    """Checkpoint positions stay global only if every segment but the last is a
+    multiple of ckpt_interval.  Rank 0's 50 tokens are not a multiple of 16, so
+    it refuses before the collective.  The last rank may be ragged; its
+    all-gather then ends with the process group's short timeout instead of
+    waiting for good."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker_bad_interval, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=120) for _ in range(2))
+    for p in procs:
+        p.join(timeout=120)
+    assert res[0] == "ValueError"
+    assert res[1] == "collective error"
