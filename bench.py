@@ -3,10 +3,13 @@
 Default: one GPU, the prefill workload B=4, H=32, T=8192, D_k=D_v=128, C=64
 (BF16 q/k/v, FP32 g/beta/state, zero initial state) as the headline, plus the
 decode workload (512 sequences x 32 heads, 256 steps captured in one CUDA
-graph, FP32 state N(0, 0.02)) as a second object on the same line.
+graph, FP32 state N(0, 0.02)) as a second object on the same line, and the
+append-prefill (8 sequences of 1K-32K tokens, checkpoints every 4096) and
+1M-token (snapshots every 32K) prefill workloads as two more.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload prefill|decode|append_varlen|long|prefill_small] [--no-decode] [--no-backward]
+                  [--no-extra-prefill]
 
 For N > 1 it is launched by torchrun, one rank per GPU; every rank runs its
 own copy of the workload (the operator's (sequence, head) units are
@@ -97,6 +100,20 @@ def kernel_source_sha(kernel: str) -> str:
         with open(os.path.join(csrc, name), "rb") as fh:
             h.update(name.encode() + fh.read())
     return h.hexdigest()[:16]
+
+
+def scaled_traffic(kernel: str, token_heads: int):
+    """DRAM bytes of one call on another workload, scaled by token-heads from the
+    committed small-case capture of the same kernels (traffic grows in
+    proportion to the chunks processed); None if that capture is stale."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh).get(kernel + "_small")
+    if not rec or rec.get("source_sha") != kernel_source_sha(kernel):
+        return None
+    return rec["bytes_per_launch"] * token_heads / rec["token_heads"]
 
 
 def ncu_traffic(kernel: str):
@@ -203,7 +220,7 @@ def max_over_ranks(x: float, world: int) -> float:
 # --------------------------------------------------------------------------------------
 # Our arm
 # --------------------------------------------------------------------------------------
-def time_prefill(name, steps, warmup, world, local):
+def time_prefill(name, steps, warmup, world, local, e2e=True):
     from linear_attention_08_b200 import kda
     w = kin.WORKLOADS[name]
     d = kin.make_workload(name, device="cuda", seed=local)
@@ -247,6 +264,22 @@ def time_prefill(name, steps, warmup, world, local):
     total_ms = max_over_ranks(total_ms, world)
     launch_ms = max_over_ranks(launch_ms, world)
 
+    tokens = sum(lengths)
+    flops, byts = prefill_algorithmic(lengths, H, Dk, Dv, C, 2 if w["dtype"] == "bf16" else 4,
+                                      interval, init is not None)
+    shape = kda.make_shape(len(lengths), tokens, H, Dk, Dv, C, 1 if w["dtype"] == "bf16" else 0)
+    path = kda.kda_prefill_path(shape)
+    launches = 1
+    if path == 2:   # one intra-chunk pass and one chain pass per window of chunks
+        ws = kda.workspace_for(shape, "meta")
+        launches = 2 * prefill_windows(len(lengths), H, tokens, ws.numel(),
+                                       kda.kda_prefill_workspace_bytes(shape))
+    res = dict(tokens=tokens, steps=steps, total_ms=total_ms, launch_ms=launch_ms,
+               launches_per_step=launches, flops=flops, bytes=byts, clocks=clk.result,
+               kernel=PATH_KERNEL[path], w=w, lengths=lengths, token_heads=tokens * H)
+    if not e2e:
+        return res
+
     # End to end through the public API: pinned host inputs -> device -> kernel -> host.
     host = {x: d[x].to("cpu").pin_memory() for x in ("q", "k", "v", "g", "beta")}
     h_init = init.to("cpu").pin_memory() if init is not None else None
@@ -280,21 +313,39 @@ def time_prefill(name, steps, warmup, world, local):
     b.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(a.elapsed_time(b) / e2e_steps, world)
+    res.update(e2e_ms=e2e_ms, bi=bi, bo=bo)
+    return res
 
-    tokens = sum(lengths)
-    flops, byts = prefill_algorithmic(lengths, H, Dk, Dv, C, 2 if w["dtype"] == "bf16" else 4,
-                                      interval, init is not None)
-    shape = kda.make_shape(len(lengths), tokens, H, Dk, Dv, C, 1 if w["dtype"] == "bf16" else 0)
-    path = kda.kda_prefill_path(shape)
-    launches = 1
-    if path == 2:   # one intra-chunk pass and one chain pass per window of chunks
-        ws = kda.workspace_for(shape, "meta")
-        launches = 2 * prefill_windows(len(lengths), H, tokens, ws.numel(),
-                                       kda.kda_prefill_workspace_bytes(shape))
-    return dict(tokens=tokens, steps=steps, total_ms=total_ms, launch_ms=launch_ms,
-                launches_per_step=launches,
-                e2e_ms=e2e_ms, bi=bi, bo=bo, flops=flops, bytes=byts, clocks=clk.result,
-                kernel=PATH_KERNEL[path], w=w, lengths=lengths)
+
+def prefill_object(r, world, hbm, tflops, peaks_src):
+    """The bench object of one more prefill workload (no end-to-end leg)."""
+    w = r["w"]
+    ms = r["total_ms"] / r["steps"]
+    gbs = r["bytes"] / (r["launch_ms"] / 1e3) / 1e9
+    tfs = r["flops"] / (r["launch_ms"] / 1e3) / 1e12
+    return {
+        "metric": "KDA prefill tokens/s", "value": world * r["tokens"] / (ms / 1e3),
+        "unit": "tokens/s", "ms_per_call": ms, "steps": r["steps"],
+        "config": {"workload": w_name(w), "num_seqs": len(r["lengths"]),
+                   "total_tokens": r["tokens"], "seq_lens": sorted(r["lengths"]),
+                   "heads": w["H"], "d": w["Dk"], "chunk": w["chunk"],
+                   "ckpt_interval": w["ckpt_interval"],
+                   "init_state": "N(0, 0.02)" if w["state_std"] > 0 else "zero"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "traffic": scaled_traffic(r["kernel"], r["token_heads"]),
+                     "kernel": r["kernel"], "peak_source": peaks_src,
+                     "tensor_tflops": tfs, "tensor_frac": tfs / tflops,
+                     "algorithmic_bytes_per_launch": r["bytes"],
+                     "algorithmic_flops_per_launch": r["flops"]},
+        "gpu_launches": r["steps"] * r["launches_per_step"], "clocks": r["clocks"],
+    }
+
+
+def w_name(w):
+    for name, spec in kin.WORKLOADS.items():
+        if spec is w:
+            return name
+    return "?"
 
 
 def prefill_windows(N, H, T, ws_bytes, full_bytes, packet=74240, chunk=64):
@@ -449,6 +500,12 @@ def run_ours(args, rank, world, local):
     spec = None
     if not args.no_decode:
         spec = time_spec_decode(max(args.steps, 5), args.warmup, world, local)
+    extra = {}
+    if name == "prefill" and not args.no_extra_prefill:
+        for other in ("append_varlen", "long"):
+            extra[other] = time_prefill(other, 3 if other == "long" else 10, args.warmup, world,
+                                        local, e2e=False)
+            torch.cuda.empty_cache()
     bwd = None
     if not args.no_backward and name == "prefill":
         bwd = time_backward(max(1, min(args.steps, 3)), args.warmup, world, local)
@@ -488,6 +545,8 @@ def run_ours(args, rank, world, local):
             "gpu_launches": r["steps"] * r["launches_per_step"],
             "clocks": r["clocks"],
         }
+        for other, ro in extra.items():
+            line[other] = prefill_object(ro, world, hbm, tflops, peaks_src)
         if bwd is not None:
             bgbs = bwd["bytes"] / (bwd["ms"] / 1e3) / 1e9
             line["backward"] = {
@@ -611,6 +670,8 @@ def main():
                     choices=["prefill", "decode", "append_varlen", "long", "prefill_small"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-extra-prefill", action="store_true",
+                    help="skip the append-varlen and 1M-token prefill objects")
     ap.add_argument("--decode-steps", type=int, default=0,
                     help="decode steps per graph (default: the workload's 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -22,10 +22,26 @@
  *   checkpoints : [n_ckpt, H, D_k, D_v] FP32, packed sequence by sequence.
  * q, k, v and out share one dtype (FP32 or BF16); g, beta and states are FP32.
  *
- * Ownership and streams: the caller owns every buffer; all pointers are
- * device pointers unless a comment says "host".  Every call is asynchronous
- * on the given stream and never synchronises.  The library keeps no device
- * allocation of its own between calls.
+ * Ownership and streams: the caller owns every buffer it passes; all
+ * pointers are device pointers unless a comment says "host".  Every call is
+ * asynchronous on the given stream and never synchronises.  The library
+ * itself holds device memory in exactly two places:
+ *   - kda_prefill's workspace pool: on the first kda_prefill call on a device
+ *     the library creates a CUDA memory pool for that device.  Each call on
+ *     the two-pass path (kda_prefill_path = 2) takes one workspace from it,
+ *     at most the pool cap (8 GiB unless kda_set_workspace_pool_cap says
+ *     otherwise; longer inputs run in windows of chunks), and gives it back
+ *     at the end of the call, ordered on the call's stream.  The pool keeps
+ *     what it has been given back (release threshold: unlimited), so later
+ *     calls reuse the memory without allocating; kda_release_workspace_pool
+ *     returns it to the device.  When even the smallest window does not fit
+ *     under the cap, or the pool cannot supply it, the call runs the
+ *     single-pass tensor-core kernel instead (same results within the
+ *     tolerances, about 20 % slower); kda_last_prefill_path tells which ran.
+ *   - the fixed array of KDA_NOALLOC_SCRATCH_BYTES behind
+ *     kda_prefill_noalloc, present on every device that loads the library.
+ * kda_prefill_ws, kda_prefill_at, the decode and backward calls and the
+ * affine maps take no device memory of their own.
  *
  * Errors: argument problems return KDA_ERR_INVALID_ARGUMENT or
  * KDA_ERR_UNSUPPORTED before anything is launched.  A failed launch returns
@@ -88,6 +104,16 @@ typedef struct {
  *                      end included when T_i is a multiple).
  *   ckpt_states      : [kda_ckpt_count(...), H, D_k, D_v]; NULL iff interval 0.
  * Every other pointer must be 16-byte aligned; out must not overlap any input.
+ *
+ * Kernels: BF16 with D_k = D_v = 128 runs on the tensor cores (tcgen05) for
+ * chunk 16 and chunk 64 alike.  The tensor-core kernels group tokens in
+ * chunks of 64 with 16-token diagonal blocks inside; the result does not
+ * depend on the chunk size, which the caller names only to fix which
+ * checkpoint intervals are valid.  With up to 1024 sequences and an interval
+ * that is 0 or a multiple of 64 the call runs the two-pass kernels through
+ * the workspace pool; more sequences, or an interval of 16, 32 or 48 modulo
+ * 64, run the single-pass tensor-core kernel.  Other shapes (FP32, smaller
+ * heads) run the FP32 SIMT kernel.
  */
 kda_status kda_prefill(const void *q, const void *k, const void *v, const float *g,
                        const float *beta, const float *init_state, const int32_t *cu_seqlens,
@@ -134,7 +160,10 @@ kda_status kda_prefill_ws(const void *q, const void *k, const void *v, const flo
  * KDA_NOALLOC_SCRATCH_BYTES; longer batches run in windows of chunks.  Other
  * shapes return KDA_ERR_UNSUPPORTED before any work is queued.
  * The first call on a device looks up the array's device address, so make
- * that first call before any stream capture.  All calls share the one array
+ * that first call before any stream capture.  The address is kept for the
+ * life of the process: after cudaDeviceReset (or anything else that tears
+ * down and recreates the device's primary context) this entry point must not
+ * be called again in that process.  All calls share the one array
  * and nothing in it needs to start at zero (each call writes every byte it
  * reads), but calls whose work overlaps on the GPU (other streams, other
  * threads) race on it: order them on one stream or synchronise between them.
@@ -243,7 +272,8 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const float
  *   M : [H, D_k, D_v] FP32.  y must not overlap x or M.
  * kda_affine_state: S_out[h] = A[h] S_in[h] + B[h]
  *   A : [H, D_k, D_k]  S_in, B, S_out : [H, D_k, D_v], all FP32; B may be NULL
- *   (zero); S_out may alias S_in or B but not A.
+ *   (zero); S_out may be exactly S_in or exactly B, but must not overlap A
+ *   and must not partly overlap S_in or B (KDA_ERR_INVALID_ARGUMENT).
  * Only num_heads, head_dim_k, head_dim_v and qkv_dtype of the shape are used.
  */
 kda_status kda_affine_rows(const void *x, const float *M, void *y, int64_t rows, int32_t accumulate,
@@ -269,11 +299,27 @@ size_t kda_prefill_workspace_min_bytes(const kda_shape *shape);
 /* Frees the memory cached by the library's per-device workspace pools. */
 kda_status kda_release_workspace_pool(void);
 
-/* Which prefill kernel a shape runs on without explicit positions:
- * 2 = two-pass tcgen05 tensor-core kernels (intra-chunk pass + chain),
- * 1 = single-pass tcgen05 kernel (also used with explicit positions and
- *     without a workspace), 0 = SIMT FP32 kernel, -1 = invalid shape. */
+/* Largest workspace kda_prefill takes from its pool, in bytes (default
+ * 8 GiB), for calls made after this one on any thread.  Below
+ * kda_prefill_workspace_min_bytes of a shape (with final_state: minus the
+ * carried state), kda_prefill runs that shape on the single-pass kernel and
+ * takes nothing from the pool; 0 therefore keeps the pool unused. */
+kda_status kda_set_workspace_pool_cap(size_t bytes);
+
+/* Which prefill kernel a shape runs on without explicit positions, with a
+ * workspace and an interval that is 0 or a multiple of 64:
+ * 2 = two-pass tcgen05 tensor-core kernels (intra-chunk pass + chain; up to
+ *     1024 sequences per call),
+ * 1 = single-pass tcgen05 kernel (also used with explicit positions, without
+ *     a workspace, for other intervals and for more than 1024 sequences),
+ * 0 = SIMT FP32 kernel, -1 = invalid shape. */
 int kda_prefill_path(const kda_shape *shape);
+
+/* The kernel (2, 1 or 0 as above) that the last kda_prefill,
+ * kda_prefill_ws, kda_prefill_at or kda_prefill_noalloc call on this host
+ * thread launched; -1 before the first launch.  Calls that return an error
+ * before launching leave it unchanged. */
+int kda_last_prefill_path(void);
 
 /* Bounded-wait self-test: launches one CTA that waits on an mbarrier that
  * nothing arrives at, with the same bounded wait the tensor-core kernel

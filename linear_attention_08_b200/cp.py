@@ -8,6 +8,8 @@ and B the state reached from zero; token by token, the outputs from S_in are
 o_t = o_t(B) + S_in^T (A_t^T q_t), and A_t^T q_t is the output of the v = 0,
 identity-start run.  So every rank:
 
+0. all-gathers the segment lengths (a refusal of misaligned segments is
+   then taken by every rank alike);
 1. runs its segment twice, from zero (B and the outputs o(B)) and with v = 0
    from the identity (A and the vectors A_t^T q_t): two ordinary prefill calls;
 2. all-gathers (A, B) of every segment (one collective of
@@ -100,8 +102,16 @@ def prefill_cp(q, k, v, g, beta, *, init_state=None, chunk=64, ckpt_interval=0, 
     rank = dist.get_rank(group)
     T, H, Dk = q.shape
     Dv = v.shape[2]
-    if ckpt_interval > 0 and rank < world - 1 and T % ckpt_interval != 0:
-        raise ValueError("every segment but the last must be a multiple of ckpt_interval")
+    # Every rank learns every segment's length first, so that a refusal is
+    # collective: all ranks raise together and none is left in a collective.
+    mine = torch.tensor([T], dtype=torch.int64, device=q.device)
+    lens = [torch.empty_like(mine) for _ in range(world)]
+    dist.all_gather(lens, mine, group=group)
+    if ckpt_interval > 0:
+        bad = [r for r in range(world - 1) if int(lens[r]) % ckpt_interval != 0]
+        if bad:
+            raise ValueError(f"segments of ranks {bad} are not multiples of ckpt_interval="
+                             f"{ckpt_interval}; every segment but the last must be")
     seg = segment_pass(q, k, v, g, beta, chunk=chunk, ckpt_interval=ckpt_interval, ops=ops)
     ab = torch.cat([seg["A"].reshape(-1), seg["B"].reshape(-1)])
     parts = [torch.empty_like(ab) for _ in range(world)]

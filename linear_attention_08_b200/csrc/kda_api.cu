@@ -2,6 +2,7 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "kda_common.cuh"
@@ -57,9 +58,12 @@ kda_status record_cuda_error(cudaError_t e) {
   return KDA_ERR_CUDA;
 }
 
-// Largest workspace kda_prefill takes from its pool (longer inputs run in windows).
-static const size_t kPoolCap = (size_t)8 << 30;
+// Largest workspace kda_prefill takes from its pool (longer inputs run in
+// windows); kda_set_workspace_pool_cap changes it.
+static std::atomic<size_t> g_pool_cap{(size_t)8 << 30};
 static const int kMaxDevices = 64;
+// Prefill kernel the last prefill call on this thread launched (2, 1, 0; -1 none yet).
+static thread_local int g_last_path = -1;
 static std::mutex g_pool_mu;
 static cudaMemPool_t g_pools[kMaxDevices];
 static int g_num_sms[kMaxDevices];
@@ -92,9 +96,17 @@ static int device_sms(int dev) {
   return g_num_sms[dev];
 }
 
+// BF16, D_k = D_v = 128: the tensor-core kernels.  They run 64-token chunks
+// whatever chunk size the caller names (16 or 64): the result does not depend
+// on the grouping of tokens into chunks, and the pages' 16-token tiles are the
+// diagonal blocks of the kernels' UT transform.
+static bool tc_shape(const kda_shape *s) {
+  return prefill_tc_supported(s->qkv_dtype, s->head_dim_k, s->head_dim_v, 64) &&
+         (s->chunk == 16 || s->chunk == 64);
+}
+
 static bool split_path(const kda_shape *s) {
-  return prefill_tc_supported(s->qkv_dtype, s->head_dim_k, s->head_dim_v, s->chunk) &&
-         prefill_split_supported(s->num_seqs);
+  return tc_shape(s) && prefill_split_supported(s->num_seqs);
 }
 
 static size_t split_min_bytes(const kda_shape *s, bool have_final) {
@@ -192,7 +204,14 @@ kda_status kda_release_workspace_pool(void) {
 int kda_prefill_path(const kda_shape *s) {
   if (check_shape(s, true) != KDA_OK) return -1;
   if (split_path(s)) return 2;
-  return prefill_tc_supported(s->qkv_dtype, s->head_dim_k, s->head_dim_v, s->chunk) ? 1 : 0;
+  return tc_shape(s) ? 1 : 0;
+}
+
+int kda_last_prefill_path(void) { return g_last_path; }
+
+kda_status kda_set_workspace_pool_cap(size_t bytes) {
+  g_pool_cap.store(bytes);
+  return KDA_OK;
 }
 
 // Workspace modes of prefill_impl.
@@ -254,38 +273,48 @@ static kda_status prefill_impl(const void *q, const void *k, const void *v, cons
   cudaError_t e;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
-  if (T > 0 && !positions && ws_mode != WS_NONE && split_path(s)) {
+  // The two-pass kernels store checkpoints at 64-token chunk ends: an interval
+  // that is not a multiple of 64 (possible with chunk 16) runs the single pass,
+  // which cuts its chunks at every checkpoint.
+  if (T > 0 && !positions && ws_mode != WS_NONE && split_path(s) && ckpt_interval % 64 == 0) {
     // Two-pass path when a large enough workspace is at hand.
     const size_t need_min = split_min_bytes(s, final_state != nullptr);
-    if (ws_mode == WS_CALLER && workspace && ws_bytes >= need_min)
+    if (ws_mode == WS_CALLER && workspace && ws_bytes >= need_min) {
+      g_last_path = 2;
       return cuda_status(launch_prefill_split(q, k, v, g, beta, init_state, cu_seqlens, out,
                                               final_state, ckpt_interval, ckpt_states, N, H, T,
                                               workspace, ws_bytes, s->dev_status, cs,
                                               device_sms(dev)));
-    if (ws_mode == WS_POOL) {
+    }
+    const size_t cap = g_pool_cap.load();
+    if (ws_mode == WS_POOL && cap >= need_min) {
       cudaMemPool_t pool;
       size_t want = split_workspace_full(N, H, T, final_state != nullptr);
-      if (want > kPoolCap) want = kPoolCap > need_min ? kPoolCap : need_min;
+      if (want > cap) want = cap;
       void *ws = nullptr;
       if (device_pool(dev, &pool) == cudaSuccess &&
           cudaMallocFromPoolAsync(&ws, want, pool, cs) == cudaSuccess) {
+        g_last_path = 2;
         e = launch_prefill_split(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
                                  ckpt_interval, ckpt_states, N, H, T, ws, want, s->dev_status, cs,
                                  device_sms(dev));
         const cudaError_t f = cudaFreeAsync(ws, cs);
         return cuda_status(e != cudaSuccess ? e : f);
       }
-      cudaGetLastError();   // an allocation that failed falls back to the single pass
+      cudaGetLastError();   // an allocation that failed runs the single pass (see kda_last_prefill_path)
     }
   }
-  if (T > 0 && prefill_tc_supported(s->qkv_dtype, DK, DV, s->chunk))
+  if (T > 0 && tc_shape(s)) {
+    g_last_path = 1;
     e = launch_prefill_tc(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,
                           ckpt_interval, ckpt_states, pos_cu, positions, pos_states, N, H, T,
                           s->dev_status, cs);
-  else
+  } else {
+    g_last_path = 0;
     e = launch_prefill_simt(s->qkv_dtype, DK, DV, q, k, v, g, beta, init_state, cu_seqlens, out,
                             final_state, ckpt_interval, ckpt_states, pos_cu, positions,
                             pos_states, N, H, cs);
+  }
   return cuda_status(e);
 }
 
@@ -344,7 +373,12 @@ kda_status kda_affine_state(const float *A, const float *S_in, const float *B, f
   for (const void *p : ptrs)
     if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
   if (B && !aligned16(B)) return KDA_ERR_INVALID_ARGUMENT;
-  if (overlaps(S_out, (size_t)H * DK * DV * 4, A, (size_t)H * DK * DK * 4)) return KDA_ERR_INVALID_ARGUMENT;
+  const size_t n_s = (size_t)H * DK * DV * 4;
+  if (overlaps(S_out, n_s, A, (size_t)H * DK * DK * 4)) return KDA_ERR_INVALID_ARGUMENT;
+  // Each CTA reads its own head of S_in and B before writing that head of
+  // S_out: exact aliasing is safe, a partial overlap would race across heads.
+  if ((S_out != S_in && overlaps(S_out, n_s, S_in, n_s)) || (B && S_out != B && overlaps(S_out, n_s, B, n_s)))
+    return KDA_ERR_INVALID_ARGUMENT;
   return cuda_status(launch_affine_state(A, S_in, B, S_out, H, DK, DV,
                                          reinterpret_cast<cudaStream_t>(stream)));
 }

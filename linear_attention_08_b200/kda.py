@@ -21,7 +21,8 @@ EXPORTED = ("kda_prefill", "kda_prefill_ws", "kda_prefill_at", "kda_decode", "kd
             "kda_ckpt_count", "kda_prefill_workspace_bytes", "kda_prefill_workspace_min_bytes",
             "kda_release_workspace_pool", "kda_prefill_path", "kda_selftest_bounded_wait",
             "kda_last_cuda_error", "kda_status_string", "kda_version", "kda_backward",
-            "kda_backward_workspace_bytes", "kda_affine_rows", "kda_affine_state")
+            "kda_backward_workspace_bytes", "kda_affine_rows", "kda_affine_state",
+            "kda_last_prefill_path", "kda_set_workspace_pool_cap")
 
 # Largest workspace the binding allocates for the two-pass prefill; longer
 # inputs run in windows of chunks.
@@ -91,6 +92,9 @@ def load(path: str | None = None):
     lib.kda_release_workspace_pool.restype = ctypes.c_int
     lib.kda_prefill_path.argtypes = [SP]
     lib.kda_prefill_path.restype = ctypes.c_int
+    lib.kda_last_prefill_path.restype = ctypes.c_int
+    lib.kda_set_workspace_pool_cap.argtypes = [ctypes.c_size_t]
+    lib.kda_set_workspace_pool_cap.restype = ctypes.c_int
     lib.kda_selftest_bounded_wait.argtypes = [P, I64, P]
     lib.kda_selftest_bounded_wait.restype = ctypes.c_int
     lib.kda_last_cuda_error.restype = ctypes.c_int
@@ -135,6 +139,17 @@ def kda_ckpt_count(cu_seqlens_host, ckpt_interval: int) -> int:
 
 def kda_prefill_path(shape: KdaShape) -> int:
     return int(load().kda_prefill_path(ctypes.byref(shape)))
+
+
+def kda_last_prefill_path() -> int:
+    """Kernel the last prefill call on this thread launched (2, 1, 0; -1 none)."""
+    return int(load().kda_last_prefill_path())
+
+
+def kda_set_workspace_pool_cap(nbytes: int) -> None:
+    st = load().kda_set_workspace_pool_cap(int(nbytes))
+    if st != KDA_OK:
+        raise KdaError(st, "kda_set_workspace_pool_cap")
 
 
 def kda_prefill_workspace_bytes(shape: KdaShape) -> int:
@@ -192,7 +207,8 @@ def kda_prefill(q, k, v, g, beta, cu_seqlens, *, init_state=None, chunk: int = 6
     if positions is None:
         if isinstance(workspace, str):
             assert workspace == "auto"
-            workspace = workspace_for(shape, q.device)
+            # the two-pass kernels take intervals that are multiples of 64 only
+            workspace = workspace_for(shape, q.device) if ckpt_interval % 64 == 0 else None
         nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
         st = lib.kda_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(init_state),
                                 _ptr(cu_seqlens), _ptr(out), _ptr(final_state),

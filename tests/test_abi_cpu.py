@@ -118,6 +118,48 @@ def test_workspace_and_path_queries():
     s3 = kda.make_shape(2000, 4000, 4, 128, 128, 64, kda.KDA_DTYPE_BF16)
     assert kda.kda_prefill_path(s3) == 1          # too many sequences for the two-pass path
     assert lib.kda_prefill_workspace_bytes(ctypes.byref(s3)) == 0
+    # chunk 16 names the same tensor-core kernels (64-token chunks inside)
+    s4 = kda.make_shape(2, 1000, 4, 128, 128, 16, kda.KDA_DTYPE_BF16)
+    assert kda.kda_prefill_path(s4) == 2
+    assert lib.kda_prefill_workspace_bytes(ctypes.byref(s4)) == \
+        lib.kda_prefill_workspace_bytes(ctypes.byref(s2))
+    s5 = kda.make_shape(2000, 4000, 4, 128, 128, 16, kda.KDA_DTYPE_BF16)
+    assert kda.kda_prefill_path(s5) == 1
+    assert kda.kda_prefill_path(kda.make_shape(2, 1000, 4, 128, 128, 16, kda.KDA_DTYPE_F32)) == 0
+
+
+def test_last_path_and_pool_cap():
+    """The last-path query is untouched by a call that fails validation; the pool
+    cap setter accepts any size (0 keeps the pool unused)."""
+    lib = kda.load()
+    before = kda.kda_last_prefill_path()
+    assert before in (-1, 0, 1, 2)
+    s = kda.make_shape(2, 1000, 4, 128, 128, 64, kda.KDA_DTYPE_BF16)
+    a = ctypes.c_void_p(1 << 20)
+    assert lib.kda_prefill(None, a, a, a, a, None, a, a, None, 0, None, ctypes.byref(s),
+                           None) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert kda.kda_last_prefill_path() == before
+    for cap in (0, 1 << 20, 8 << 30):
+        kda.kda_set_workspace_pool_cap(cap)
+    assert kda.kda_last_prefill_path() == before
+
+
+def test_affine_state_rejects_partial_overlap():
+    """S_out may be exactly S_in or B; shifted by one head it would race across CTAs."""
+    lib = kda.load()
+    s = kda.make_shape(1, 1, 4, 64, 64, 0, kda.KDA_DTYPE_F32)
+    head = 64 * 64 * 4
+    A = ctypes.c_void_p(1 << 30)
+    S = ctypes.c_void_p(1 << 32)
+    B = ctypes.c_void_p(1 << 34)
+    shifted_S = ctypes.c_void_p((1 << 32) + head)
+    shifted_B = ctypes.c_void_p((1 << 34) - head)
+    call = lambda out: lib.kda_affine_state(A, S, B, out, ctypes.byref(s), None)
+    assert call(shifted_S) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert call(shifted_B) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert call(A) == kda.KDA_ERR_INVALID_ARGUMENT
+    assert lib.kda_affine_state(A, S, None, shifted_S, ctypes.byref(s), None) == \
+        kda.KDA_ERR_INVALID_ARGUMENT
 
 
 def test_prefill_ws_rejects_bad_workspace():

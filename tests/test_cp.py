@@ -138,38 +138,38 @@ def _worker_bad_interval(rank, world, port, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world))
     import torch.distributed as dist
+    # A long timeout: the refusal must not need one to end.
     dist.init_process_group("gloo", rank=rank, world_size=world,
-                            timeout=datetime.timedelta(seconds=5))
+                            timeout=datetime.timedelta(seconds=60))
     x = _sequence(100, 1, 4, 4, seed=3)
     a, b = (0, 50) if rank == 0 else (50, 100)
+    import time
+    t0 = time.monotonic()
     try:
         cp.prefill_cp(x["q"][a:b], x["k"][a:b], x["v"][a:b], x["g"][a:b], x["beta"][a:b],
                       chunk=16, ckpt_interval=16, ops=OracleOps())
-        q.put((rank, "ok"))
+        q.put((rank, "ok", time.monotonic() - t0))
     except ValueError:
-        q.put((rank, "ValueError"))
-    except Exception:   # the last rank's all-gather times out: its peer never joined
-        q.put((rank, "collective error"))
-    try:
-        dist.destroy_process_group()
-    except Exception:
-        pass
+        q.put((rank, "ValueError", time.monotonic() - t0))
+    except Exception as e:
+        q.put((rank, f"other: {e!r}", time.monotonic() - t0))
+    dist.destroy_process_group()
 
 
 def test_prefill_cp_rejects_unaligned_segment():
     """Checkpoint positions stay global only if every segment but the last is a
-    multiple of ckpt_interval.  Rank 0's 50 tokens are not a multiple of 16, so
-    it refuses before the collective.  The last rank may be ragged; its
-    all-gather then ends with the process group's short timeout instead of
-    waiting for good."""
+    multiple of ckpt_interval.  Rank 0's 50 tokens are not a multiple of 16: both
+    ranks learn it from the gathered lengths and both raise ValueError at once,
+    long before the process group's timeout, with no collective left pending."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
     procs = [ctx.Process(target=_worker_bad_interval, args=(r, 2, port, q)) for r in range(2)]
     for p in procs:
         p.start()
-    res = dict(q.get(timeout=120) for _ in range(2))
+    res = {r: (what, dt) for r, what, dt in (q.get(timeout=120) for _ in range(2))}
     for p in procs:
         p.join(timeout=120)
-    assert res[0] == "ValueError"
-    assert res[1] == "collective error"
+        assert p.exitcode == 0
+    assert res[0][0] == "ValueError" and res[1][0] == "ValueError", res
+    assert max(res[0][1], res[1][1]) < 30.0, res

@@ -200,10 +200,16 @@ def test_full_workload_sampled(name):
             assert rel_l2(ck[base:base + rc.shape[0], h:h + 1], rc) <= 1e-2
 
 
-def test_long_context_segments():
-    """T = 1,048,576 with snapshots every 32,768 tokens.  The oracle replays sampled
-    32K-token segments of sampled heads from the GPU's own snapshot before each one
-    (a property that holds at any length), plus the first segment from zero."""
+def test_long_context_against_oracle_from_token_zero():
+    """T = 1,048,576 with snapshots every 32,768 tokens, in the benchmark's launch
+    configuration.  Heads 0 and 31 are run by the FP64 oracle over the whole
+    sequence from the zero state, and all their outputs, all 32 snapshots and the
+    final state are compared (rel-L2 per tensor, and the worst snapshot).  Then a
+    32K-token segment of head 5 is replayed from the GPU's own snapshot before
+    it, a property that holds at any length."""
+    import concurrent.futures as cf
+
+    import oracle
     w = kin.WORKLOADS["long"]
     d = kin.make_workload("long", device="cuda")
     cu_dev = torch.tensor(d["cu_seqlens"], dtype=torch.int32, device="cuda")
@@ -214,16 +220,37 @@ def test_long_context_segments():
     torch.cuda.synchronize()
     T = d["cu_seqlens"][-1]
     assert ck.shape[0] == T // I == 32
+    assert torch.isfinite(out.float()).all() and torch.isfinite(fin).all()
+
+    def head_inputs(h, a=0, b=T):
+        return {n: d[n][a:b, h:h + 1].to("cpu") for n in ("q", "k", "v", "g", "beta")}
+
+    heads = (0, 31)
+    host = {h: head_inputs(h) for h in heads}
+
+    def run_oracle(h):
+        x = host[h]
+        return oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], [0, T], None, I, 0, 1)
+
+    with cf.ThreadPoolExecutor(len(heads)) as ex:   # the oracle call releases the GIL
+        refs = dict(zip(heads, ex.map(run_oracle, heads)))
+    for h in heads:
+        ro, rf, rc = refs[h]
+        e_o = rel_l2(out[:, h:h + 1], ro)
+        e_f = rel_l2(fin[:, h:h + 1], rf)
+        e_c = rel_l2(ck[:, h:h + 1], rc)
+        e_cmax = max(rel_l2(ck[j:j + 1, h:h + 1], rc[j:j + 1]) for j in range(rc.shape[0]))
+        print(f"long context, head {h}: rel-L2 o {e_o:.3e}, final state {e_f:.3e}, "
+              f"snapshots {e_c:.3e} (worst single snapshot {e_cmax:.3e})")
+        assert e_o <= 1e-2 and e_f <= 1e-2 and e_c <= 1e-2 and e_cmax <= 1e-2
     assert torch.equal(ck[-1], fin[0])
-    import oracle
-    for seg, h in [(0, 0), (17, 5), (31, 31)]:
-        a, b = seg * I, (seg + 1) * I
-        cpu = lambda t: t[a:b, h:h + 1].to("cpu")
-        init = None if seg == 0 else ck[seg - 1:seg, h:h + 1].to("cpu")
-        ro, rf, _ = oracle.prefill(cpu(d["q"]), cpu(d["k"]), cpu(d["v"]), cpu(d["g"]),
-                                   cpu(d["beta"]), [0, I], init, 0, 0, 1)
-        assert rel_l2(out[a:b, h:h + 1], ro) <= 1e-2
-        assert rel_l2(ck[seg:seg + 1, h:h + 1], rf) <= 1e-2
+    seg, h = 17, 5
+    a, b = seg * I, (seg + 1) * I
+    x = head_inputs(h, a, b)
+    ro, rf, _ = oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], [0, I],
+                               ck[seg - 1:seg, h:h + 1].to("cpu"), 0, 0, 1)
+    assert rel_l2(out[a:b, h:h + 1], ro) <= 1e-2
+    assert rel_l2(ck[seg:seg + 1, h:h + 1], rf) <= 1e-2
 
 
 def test_bounded_wait_reports_timeout():

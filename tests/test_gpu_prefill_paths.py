@@ -41,7 +41,9 @@ def test_path_query():
     d = to_device(make_case(LENGTHS, 3, 128, 128, torch.bfloat16, seed=3))
     assert kda.kda_prefill_path(shape_of(d)) == 2
     s = shape_of(d)
-    s.chunk = 16
+    s.chunk = 16      # the same tensor-core kernels (64-token chunks inside)
+    assert kda.kda_prefill_path(s) == 2
+    s.qkv_dtype = kda.KDA_DTYPE_F32
     assert kda.kda_prefill_path(s) == 0
     s = shape_of(d)
     s.num_seqs = 4096   # too many sequences for the two-pass path
@@ -112,3 +114,48 @@ def test_many_sequences_single_pass():
     out, fin, _ = run(dd, 0, "auto")
     torch.cuda.synchronize()
     check(d, out, fin, None, 0)
+
+
+@pytest.mark.parametrize("interval,path", [(0, 2), (64, 2), (128, 2), (32, 1), (48, 1)])
+def test_chunk16_runs_on_tensor_cores(interval, path):
+    """A BF16, D = 128 request for 16-token chunks runs the tensor-core kernels:
+    the two-pass ones when the checkpoint interval is a multiple of 64, the
+    single-pass one (which cuts its chunks at every checkpoint) otherwise."""
+    d = make_case(LENGTHS, 3, 128, 128, torch.bfloat16, seed=8, state_std=0.05)
+    dd = to_device(d)
+    out, fin, ck = kda.kda_prefill(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu_dev"],
+                                   init_state=dd["init_state"], chunk=16, ckpt_interval=interval,
+                                   cu_seqlens_host=dd["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert kda.kda_last_prefill_path() == path
+    check(d, out, fin, ck, interval)
+
+
+def test_pool_cap_fallback_is_visible():
+    """With the pool cap below the smallest window kda_prefill takes nothing from
+    the pool and runs the single-pass kernel; kda_last_prefill_path says so, and
+    the result still matches the oracle.  Restoring the cap restores the path."""
+    d = make_case(LENGTHS, 3, 128, 128, torch.bfloat16, seed=9, state_std=0.05)
+    dd = to_device(d)
+    lib = kda.load()
+    T, H, _ = dd["q"].shape
+    N = len(LENGTHS)
+    shape = shape_of(dd)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    try:
+        for cap, path in ((0, 1), (kda.kda_prefill_workspace_min_bytes(shape) - 1, 1),
+                          (8 << 30, 2)):
+            kda.kda_set_workspace_pool_cap(cap)
+            out = torch.empty(T, H, 128, dtype=torch.bfloat16, device="cuda")
+            fin = torch.empty(N, H, 128, 128, device="cuda")
+            ck = torch.empty(kda.kda_ckpt_count(dd["cu_seqlens"], 128), H, 128, 128, device="cuda")
+            st = lib.kda_prefill(P(dd["q"]), P(dd["k"]), P(dd["v"]), P(dd["g"]), P(dd["beta"]),
+                                 P(dd["init_state"]), P(dd["cu_dev"]), P(out), None, 128, P(ck),
+                                 ctypes.byref(shape), stream)
+            assert st == kda.KDA_OK
+            assert kda.kda_last_prefill_path() == path, cap
+            torch.cuda.synchronize()
+            check(d, out, None, ck, 128)
+    finally:
+        kda.kda_set_workspace_pool_cap(8 << 30)
