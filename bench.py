@@ -484,11 +484,13 @@ def time_backward(steps, warmup, world, local, N=4, H=32, T=1024, D=128):
     b.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    path = kda.kda_last_backward_path()
     # algorithmic bytes per token-head: q, k, v (BF16), g, d_out, the five
     # FP32 gradients and beta; plus three states per unit (init, d_final, d_init)
     per_th = 3 * D * 2 + D * 4 + D * 4 + 4 + 3 * D * 4 + D * 4 + 4
     byts = N * T * H * per_th + 3 * N * H * D * D * 4
-    return dict(tokens=N * T, ms=ms, bytes=byts, N=N, H=H, T=T, D=D)
+    return dict(tokens=N * T, ms=ms, bytes=byts, N=N, H=H, T=T, D=D,
+                kernel="backward_tc" if path == 1 else "backward_simt")
 
 
 def run_ours(args, rank, world, local):
@@ -555,14 +557,15 @@ def run_ours(args, rank, world, local):
                 "ms_per_call": bwd["ms"],
                 "config": {"num_seqs": bwd["N"], "seq_len": bwd["T"], "heads": bwd["H"],
                            "d": bwd["D"], "dtype": "bf16 inputs, fp32 gradients"},
-                "roofline": {"bound": "latency", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
-                             "frac": bgbs / hbm, "kernel": "backward",
-                             "note": "SIMT, one CTA per (sequence, head, 32 value columns), one replay per 4-token block"}}
+                "roofline": {"bound": "hbm", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
+                             "frac": bgbs / hbm, "kernel": bwd["kernel"],
+                             "note": "operator bytes (inputs, upstream gradients, gradients, states) over the whole call"}}
     if dec is not None:
         dgbs = dec["bytes"] / (dec["ms"] / dec["launches"] / 1e3) / 1e9 / dec["launches"]
         dobj = {
             "metric": "KDA decode tokens/s", "value": world * dec["tokens"] / (dec["ms"] / 1e3),
-            "unit": "tokens/s", "ms_per_step": dec["ms"], "steps_per_graph": dec["launches"],
+            "unit": "tokens/s", "ms_per_step": dec["ms"] / dec["launches"], "ms_per_graph": dec["ms"],
+            "steps_per_graph": dec["launches"],
             "config": {"workload": "decode", "num_seqs": 512, "heads": 32, "d": 128,
                        "steps": dec["launches"], "l2": "state 2.1 GB > L2"},
             "roofline": {"bound": "hbm", "achieved": dgbs, "peak": hbm, "unit": "GB/s",

@@ -236,21 +236,37 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const f
 /*
  * Backward pass of the recurrence, for training (the pages name training work
  * but give no detail; the gradients follow from the forward definition above
- * by reverse-mode differentiation, token by token in FP32).
+ * by reverse-mode differentiation).
+ *
+ * BF16 q/k/v with D_k = D_v = 128 and at most 1024 sequences run the chunked
+ * form on the tensor cores when the workspace is at least
+ * kda_backward_workspace_bytes(shape) (what that query returns for such
+ * shapes): the forward is recomputed by the two-pass prefill (its intra-chunk
+ * packets and a state every 64 tokens kept in the workspace), then a chain
+ * kernel carries the state gradient backwards chunk by chunk and two parallel
+ * kernels form every chunk's gradients from 64 x 64 and 64 x 128 tcgen05
+ * products.  The workspace then holds about 300 KB per (64-token chunk, head).
+ * Other shapes, or a smaller workspace that still covers the SIMT kernel's
+ * need, run the FP32 SIMT kernel token by token; kda_last_backward_path tells
+ * which ran.
  *
  *   q, k, v, g, beta, init_state, cu_seqlens : the forward call's inputs
  *   d_out         : [T_tot, H, D_v] FP32, gradient of the loss w.r.t. out
  *   d_final_state : [N, H, D_k, D_v] FP32 or NULL (zero), w.r.t. the final state
  *   dq, dk, dg    : [T_tot, H, D_k] FP32 outputs     dv : [T_tot, H, D_v] FP32
  *   dbeta         : [T_tot, H] FP32                 d_init_state : [N, H, D_k, D_v] or NULL
- *   workspace     : at least kda_backward_workspace_bytes(shape) bytes (the
- *                   state at every 4th token of every unit and, for D_v > 32,
- *                   the dq, dk, dg, dbeta parts of value-column slices 2..)
+ *   workspace     : at least kda_backward_workspace_bytes(shape) bytes (for
+ *                   the SIMT kernel: the state at every 4th token of every
+ *                   unit and, for D_v > 32, the dq, dk, dg, dbeta parts of
+ *                   value-column slices 2..)
  * q, k, v are BF16 or FP32 (shape->qkv_dtype); D_k, D_v in {32, 64, 128};
  * shape->chunk is ignored.  Every pointer 16-byte aligned; outputs must not
  * overlap inputs or each other.
  */
 size_t kda_backward_workspace_bytes(const kda_shape *shape);
+/* The backward kernel the last kda_backward call on this host thread
+ * launched: 1 = chunked tensor-core, 0 = SIMT, -1 before the first launch. */
+int kda_last_backward_path(void);
 kda_status kda_backward(const void *q, const void *k, const void *v, const float *g,
                         const float *beta, const float *init_state, const int32_t *cu_seqlens,
                         const float *d_out, const float *d_final_state, float *dq, float *dk,

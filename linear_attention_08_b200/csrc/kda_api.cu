@@ -20,7 +20,7 @@ cudaError_t launch_prefill_simt(int dtype, int dk, int dv, const void *q, const 
 cudaError_t launch_decode_multi(int dtype, int dk, int dv, const void *q, const void *k,
                                 const void *v, const float *g, const float *beta, float *state,
                                 void *out, const int32_t *accept_len, int T_new, int64_t units,
-                                int H, cudaStream_t stream);
+                                int H, int32_t *dev_status, cudaStream_t stream);
 bool prefill_tc_supported(int dtype, int dk, int dv, int chunk);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const float *init, const int32_t *cu,
@@ -49,7 +49,19 @@ cudaError_t launch_backward(int dtype, const void *q, const void *k, const void 
                             float *dg, float *dbeta, float *dinit, float *ws, int N, int H, int Dk,
                             int Dv, int64_t T, cudaStream_t stream);
 
+bool backward_tc_supported(int dtype, int dk, int dv, int N);
+size_t backward_tc_workspace_bytes(int N, int H, int64_t T);
+cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *init, const int32_t *cu,
+                               const float *dout, const float *dfin, float *dq, float *dk,
+                               float *dv, float *dg, float *dbeta, float *dinit, void *workspace,
+                               int N, int H, int64_t T, int32_t *dev_status, cudaStream_t stream,
+                               int num_sms);
+
 static thread_local int g_last_cuda_error = 0;
+// Backward kernel the last kda_backward call on this thread launched (1 chunked
+// tensor-core, 0 SIMT; -1 none yet).
+static thread_local int g_last_bwd_path = -1;
 
 // For entry points defined in other files of the library.
 kda_status record_cuda_error(cudaError_t e) {
@@ -385,9 +397,13 @@ kda_status kda_affine_state(const float *A, const float *S_in, const float *B, f
 
 size_t kda_backward_workspace_bytes(const kda_shape *s) {
   if (check_shape(s, false) != KDA_OK) return (size_t)-1;
+  if (s->total_tokens > 0 && backward_tc_supported(s->qkv_dtype, s->head_dim_k, s->head_dim_v, s->num_seqs))
+    return backward_tc_workspace_bytes(s->num_seqs, s->num_heads, s->total_tokens);
   return backward_workspace_bytes(s->num_seqs, s->num_heads, s->total_tokens, s->head_dim_k,
                                   s->head_dim_v);
 }
+
+int kda_last_backward_path(void) { return g_last_bwd_path; }
 
 kda_status kda_backward(const void *q, const void *k, const void *v, const float *g,
                         const float *beta, const float *init_state, const int32_t *cu_seqlens,
@@ -404,12 +420,18 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const float
   const size_t n_qk = (size_t)T * H * DK * es, n_v = (size_t)T * H * DV * es;
   const size_t n_k4 = (size_t)T * H * DK * 4, n_v4 = (size_t)T * H * DV * 4, n_b = (size_t)T * H * 4;
   const size_t n_state = (size_t)N * H * DK * DV * 4;
+  bool chunked = false;
   if (T > 0) {
     const void *ptrs[] = {q, k, v, g, beta, d_out, dq, dk, dv, dg, dbeta};
     for (const void *p : ptrs)
       if (!p || !aligned16(p)) return KDA_ERR_INVALID_ARGUMENT;
+    // The chunked tensor-core backward when its (larger or smaller) workspace
+    // is granted, else the SIMT one.
+    chunked = backward_tc_supported(s->qkv_dtype, DK, DV, N) && workspace &&
+              workspace_bytes >= backward_tc_workspace_bytes(N, H, T);
     const size_t need = backward_workspace_bytes(N, H, T, DK, DV);
-    if (!workspace || !aligned16(workspace) || workspace_bytes < need) return KDA_ERR_INVALID_ARGUMENT;
+    if (!workspace || !aligned16(workspace) || (!chunked && workspace_bytes < need))
+      return KDA_ERR_INVALID_ARGUMENT;
   }
   const void *sp[] = {init_state, d_final_state, d_init_state};
   for (const void *p : sp)
@@ -425,10 +447,19 @@ kda_status kda_backward(const void *q, const void *k, const void *v, const float
     for (int j = i + 1; j < 7; ++j)
       if (overlaps(outs[i], out_n[i], outs[j], out_n[j])) return KDA_ERR_INVALID_ARGUMENT;
   }
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (chunked) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    g_last_bwd_path = 1;
+    return cuda_status(launch_backward_tc(q, k, v, g, beta, init_state, cu_seqlens, d_out,
+                                         d_final_state, dq, dk, dv, dg, dbeta, d_init_state,
+                                         workspace, N, H, T, s->dev_status, cs, device_sms(dev)));
+  }
+  g_last_bwd_path = 0;
   return cuda_status(launch_backward(s->qkv_dtype, q, k, v, g, beta, init_state, cu_seqlens, d_out,
                                      d_final_state, dq, dk, dv, dg, dbeta, d_init_state,
-                                     reinterpret_cast<float *>(workspace), N, H, DK, DV, T,
-                                     reinterpret_cast<cudaStream_t>(stream)));
+                                     reinterpret_cast<float *>(workspace), N, H, DK, DV, T, cs));
 }
 
 kda_status kda_decode(const void *q, const void *k, const void *v, const float *g,
@@ -480,7 +511,7 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const f
     return KDA_ERR_INVALID_ARGUMENT;
   return cuda_status(launch_decode_multi(s->qkv_dtype, s->head_dim_k, s->head_dim_v, q, k, v, g,
                                          beta, state_inout, out, accept_len, tokens_per_seq,
-                                         units, s->num_heads,
+                                         units, s->num_heads, s->dev_status,
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 

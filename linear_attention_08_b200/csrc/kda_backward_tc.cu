@@ -1,0 +1,1392 @@
+// Backward pass of KDA on the 5th-generation tensor cores (tcgen05, sm_100a),
+// for BF16 q/k/v with D_k = D_v = 128: the chunked form of the gradients.
+//
+// The pages name training work without detail ("MoonshotAI/Kimi-K3 딥다이브",
+// section 4-1); the gradients below follow from the chunked forward
+// ("LLM - Semianalysis, Kimi K3 아키텍처", Methods 1: intra-chunk matrix
+// products plus a recurrence between chunks) by reverse-mode differentiation.
+// For one chunk (64 tokens, padded with identity tokens) starting from S0,
+// with Gam_r the inclusive cumulative log-decay inside the chunk,
+// Ktilde = k e^Gam, Qtilde = q e^Gam, Khat = k e^(Gam_63 - Gam), d = e^Gam_63,
+// the gated Gram G_ij = sum_c k_ic k_jc e^(Gam_ic - Gam_jc) (j < i),
+// P_ri = sum_c q_rc k_ic e^(Gam_rc - Gam_ic) (i <= r), A = I + diag(beta) G,
+// Ai = A^-1, T = Ai diag(beta):
+//
+//   R = V - Ktilde S0,  U = T R,  O = Qtilde S0 + P U,
+//   S_L = Diag(d) S0 + Khat^T U.
+//
+// Given dO and dS_L (the gradient of the state at the chunk's end):
+//
+//   dU  = P^T dO + Khat dS_L          dR = T^T dU = dV        dT = dU R^T
+//   dP  = dO U^T                      dQtilde = dO S0^T       dKtilde = -dR S0^T
+//   dKhat = U dS_L^T                  dd_c = sum_j dS_L[c,j] S0[c,j]
+//   dS0 = Diag(d) dS_L + Qtilde^T dO - Ktilde^T dR
+//       = Diag(d) dS_L + Qtilde^T dO - W^T dU        (W = T Ktilde)
+//   Y1 = Ai^T dT: dbeta_j += Y1_jj;   dA = -Y1 T^T, dM = strict lower part,
+//   dbeta_i += sum_j dM_ij G_ij,  dG_ij = beta_i dM_ij,
+//
+// and the gated products G, P, Qtilde, Ktilde, Khat, d pass their gradients to
+// q, k and Gam; dg is the reverse cumulative sum of dGam inside the chunk.
+//
+// Three launches after the forward recomputation (the two-pass prefill run
+// with a state stored at every chunk end, its intra-chunk packets kept):
+//  1. bwd_chain_kernel: one CTA per (sequence, head) walks the chunks
+//     backwards carrying dS in tensor memory: per chunk dU = [Khat | P^T]
+//     [dS; dO] and dS <- d dS + [W^T | Qtilde^T] [-dU; dO], two tcgen05 MMAs.
+//     It stores dS_L per chunk and the BF16 tile [-dU; dO] for the others.
+//  2. bwd_state_kernel (per (chunk, head), in parallel): recomputes the gates,
+//     the Gram products and T, then R, U, dR (= dv), dT, dP, dQtilde,
+//     dKtilde, dKhat on the tensor cores; writes dv and the parts of dq, dk and
+//     dg those terms give, and the BF16 tiles dT and dP.
+//  3. bwd_gram_kernel (per (chunk, head)): recomputes the gates, G and Ai,
+//     then Y1, dA, dG and the gated products of dG and dP on the tensor
+//     cores; adds the rest of dq, dk, dg and writes dbeta.
+#include <cuda.h>
+
+#include "kda_common.cuh"
+#include "kda_tc_util.cuh"
+#include "kda_tma.cuh"
+
+namespace kda {
+
+cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *init, const int32_t *cu, void *out,
+                                 float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
+                                 void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 cudaStream_t stream, int num_sms);
+size_t split_packet_bytes();
+bool prefill_split_supported(int N);
+
+namespace {
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+constexpr int kThreads = 256;
+
+// The packet the forward intra-chunk pass writes per (chunk, head): operand
+// tiles in the 128-byte-swizzled row-tile layout of kda_tc_util.cuh.
+struct Pk {
+  static constexpr uint32_t WQ = 0;        // [128][128]: W rows 0..63, Qtilde rows 64..127
+  static constexpr uint32_t KH = 32768;    // [64][128] Khat (tokens x key channels)
+  static constexpr uint32_t P = 65536;     // [64][64] P, lower triangle with diagonal, then
+                                           // float[128] exp(Gam_63) at 73728
+  static constexpr uint32_t BYTES = 74240;
+};
+
+// Chunks of sequence n.
+__device__ __forceinline__ int64_t seq_chunks(const int32_t *cu, int n) {
+  return ((int64_t)cu[n + 1] - cu[n] + kC - 1) / kC;
+}
+
+// ---------------------------------------------------------------------------
+// 1. The backward chain
+// ---------------------------------------------------------------------------
+struct BChainLayout {
+  static constexpr uint32_t S_T = 0;         // [128 ch][128 v] bf16 dS, MN-major B
+  static constexpr uint32_t BT = 32768;      // [128 tok][128 v] bf16: rows 0..63 -dU, 64..127 dO
+  static constexpr uint32_t DOF = 65536;     // float [64][128] dO staging (TMA)
+  static constexpr uint32_t STAGE0 = 98304;  // packet stages
+  // Inside a stage.  Khat and P come first: the M = 128 MMAs that read them as
+  // 64-row operands also read the 8 KB after each (rows 64..127 of the
+  // product, never used), which must stay inside the allocation.
+  static constexpr uint32_t SKH = 0;         // [64][128] Khat
+  static constexpr uint32_t SP = 16384;      // [64][64] P
+  static constexpr uint32_t SD = 24576;      // float[128] d
+  static constexpr uint32_t SWQ = 25600;     // [128][128] [W; Qtilde]
+  static constexpr uint32_t STAGE = SWQ + 32768;
+  static constexpr int NST = 2;
+  static constexpr uint32_t FULL = STAGE0 + NST * STAGE;   // [NST] packet landed
+  static constexpr uint32_t DOBAR = FULL + 8 * NST;        // dO landed
+  static constexpr uint32_t BAR1 = DOBAR + 8;              // dU product done
+  static constexpr uint32_t BAR2 = BAR1 + 8;               // dS product done
+  static constexpr uint32_t SCAL = BAR2 + 8;               // int64 first packet of the unit
+  static constexpr uint32_t TMEM_SLOT = SCAL + 8;
+  static constexpr uint32_t TOTAL = TMEM_SLOT + 8;
+  static constexpr uint32_t ACC1 = 0, ACC2 = 128, SCOL = 256;   // TMEM columns
+  static_assert(SKH + 16384 + 8192 <= STAGE && SP + 8192 + 8192 <= STAGE, "junk rows leave the stage");
+  static_assert(STAGE % 1024 == 0 && SWQ % 1024 == 0, "tile alignment");
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_chain_kernel(const __grid_constant__ CUtensorMap dout_map, const uint8_t *__restrict__ pk,
+                 const int32_t *__restrict__ cu, const float *__restrict__ dfin,
+                 float *__restrict__ dinit, float *__restrict__ dsl, uint8_t *__restrict__ dudo,
+                 int N, int H, int32_t *dev_status, uint64_t wait_ns) {
+  using Lay = BChainLayout;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sb = (sraw + 1023u) & ~1023u;
+  uint8_t *sp = smem_raw + (sb - sraw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hw = warp >> 2;
+  const int unit = blockIdx.x, n = unit / H, h = unit % H;
+  const int crow = 32 * qd + lane;   // TMEM lane of this thread: a key channel
+  const int64_t nch = seq_chunks(cu, n);
+  const int64_t tseq = cu[n];
+  const int64_t T_n = (int64_t)cu[n + 1] - cu[n];
+
+  if (warp == 0) {   // first packet of sequence n (packets: sequence, head, chunk)
+    int64_t before = 0;
+    for (int m = lane; m < n; m += 32) before += seq_chunks(cu, m);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+    if (lane == 0) *reinterpret_cast<int64_t *>(sp + Lay::SCAL) = before;
+  }
+  uint64_t *full = reinterpret_cast<uint64_t *>(sp + Lay::FULL);
+  uint64_t *dobar = reinterpret_cast<uint64_t *>(sp + Lay::DOBAR);
+  uint64_t *bar1 = reinterpret_cast<uint64_t *>(sp + Lay::BAR1);
+  uint64_t *bar2 = reinterpret_cast<uint64_t *>(sp + Lay::BAR2);
+  if (tid == 0) {
+    for (int s = 0; s < Lay::NST; ++s) mbar_init(full + s, 1);
+    mbar_init(dobar, 1);
+    mbar_init(bar1, 1);
+    mbar_init(bar2, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&dout_map)) : "memory");
+  }
+  if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, 512);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
+  const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+  const int64_t p0 = *reinterpret_cast<const int64_t *>(sp + Lay::SCAL) * H + (int64_t)h * nch;
+
+  auto issue_packet = [&](int64_t c, int s) {
+    const uint8_t *src = pk + (size_t)(p0 + c) * Pk::BYTES;
+    const uint32_t st = sb + Lay::STAGE0 + s * Lay::STAGE;
+    const uint32_t fb = sb + Lay::FULL + 8 * s;
+    mbar_expect_tx(fb, 16384 + 8704 + 32768);
+    bulk_load(st + Lay::SKH, src + Pk::KH, 16384, fb);
+    bulk_load(st + Lay::SP, src + Pk::P, 8704, fb);      // P and d
+    bulk_load(st + Lay::SWQ, src + Pk::WQ, 32768, fb);
+  };
+  auto issue_dout = [&](int64_t c) {
+    mbar_expect_tx(sb + Lay::DOBAR, 64 * 512);
+    tma_load_3d(sb + Lay::DOF, &dout_map, 0, h, (int)(tseq + kC * c), sb + Lay::DOBAR);
+  };
+  if (tid == 32 && nch > 0) {
+    issue_dout(nch - 1);
+    for (int s = 0; s < Lay::NST && s < nch; ++s) issue_packet(nch - 1 - s, s);
+  }
+
+  // dS = dS_final, FP32 in tensor memory (lane = key channel), BF16 copy in S_T.
+  const uint32_t s_tm = tl + Lay::SCOL + hw * 64;
+  auto row_ptr = [&](float *base, int64_t slot) {
+    return base + ((size_t)slot * kD + crow) * kD + hw * 64;
+  };
+  {
+    const float *src = dfin ? dfin + ((size_t)unit * kD + crow) * kD + hw * 64 : nullptr;
+    float *dst0 = nch > 0 ? row_ptr(dsl, p0 + nch - 1) : (dinit ? row_ptr(dinit, unit) : nullptr);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float x[32];
+#pragma unroll
+      for (int j = 0; j < 32; j += 4) {
+        const float4 v4 = src ? *reinterpret_cast<const float4 *>(src + 32 * u + j)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        x[j] = v4.x; x[j + 1] = v4.y; x[j + 2] = v4.z; x[j + 3] = v4.w;
+        if (dst0) *reinterpret_cast<float4 *>(dst0 + 32 * u + j) = v4;
+      }
+      tc::tmem_st32(s_tm + 32 * u, x);
+#pragma unroll
+      for (int j = 0; j < 32; j += 8)
+        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * 64 + 32 * u + j) >> 3), x + j);
+    }
+    tc::tmem_wait_st();
+  }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+
+  uint32_t fphase = 0, dphase = 0, ph1 = 0, ph2 = 0;
+  bool aborted = false;
+  for (int64_t i = 0; i < nch; ++i) {
+    const int64_t c = nch - 1 - i;
+    const int s = (int)(i % Lay::NST);
+    const uint32_t st = sb + Lay::STAGE0 + s * Lay::STAGE;
+    const int L = (int)(T_n - kC * c < kC ? T_n - kC * c : kC);
+    if (__syncthreads_or(!wait_timed(dobar, dphase, wait_ns) ||
+                         !wait_timed(full + s, (fphase >> s) & 1u, wait_ns))) { aborted = true; break; }
+    dphase ^= 1;
+    fphase ^= 1u << s;
+    // dO (FP32 staging) -> BF16 rows 64..127 of BT; rows past the chunk's end are zero.
+    {
+      const int r = tid >> 2, c0 = (tid & 3) * 32;
+      const float *srow = reinterpret_cast<const float *>(sp + Lay::DOF) + r * kD + c0;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = r < L ? srow[j + e] : 0.f;
+        tc::st_chunk(sb + Lay::BT + tc::tile_offset(128, 64 + r, (c0 + j) >> 3), x);
+      }
+    }
+    tc::fence_smem_to_async();
+    __syncthreads();
+    if (tid == 32 && c > 0) issue_dout(c - 1);
+    // acc1 = Khat dS + P^T dO  (rows 0..63: dU)
+    if (tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t idk = tc::idesc_bf16(128, 128, 0, 1);
+      constexpr uint32_t idm = tc::idesc_bf16(128, 128, 1, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + Lay::ACC1, tc::desc_kmajor(st + Lay::SKH, 64, s2),
+                     tc::desc_mnmajor(sb + Lay::S_T, 128, s2), idk, s2 > 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + Lay::ACC1, tc::desc_mnmajor(st + Lay::SP, 64, s2),
+                     tc::desc_mnmajor(sb + Lay::BT + 8192, 128, s2), idm, 1);
+      tc::mma_commit(sb + Lay::BAR1);
+    }
+    if (__syncthreads_or(!wait_timed(bar1, ph1, wait_ns))) { aborted = true; break; }
+    ph1 ^= 1;
+    tc::fence_after_sync();
+    if (qd < 2) {   // -dU -> rows 0..63 of BT
+      const int r = 32 * qd + lane;
+      float a[64];
+      tc::tmem_ld32(tl + Lay::ACC1 + hw * 64, *reinterpret_cast<float(*)[32]>(a));
+      tc::tmem_ld32(tl + Lay::ACC1 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(a + 32));
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 64; ++j) a[j] = -a[j];
+#pragma unroll
+      for (int j = 0; j < 64; j += 8)
+        tc::st_chunk(sb + Lay::BT + tc::tile_offset(128, r, (hw * 64 + j) >> 3), a + j);
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // [-dU; dO] goes to the workspace; acc2 = W^T (-dU) + Qtilde^T dO
+    if (tid == 0) {
+      tc::fence_after_sync();
+      bulk_store(dudo + (size_t)(p0 + c) * 32768, sb + Lay::BT, 32768);
+      bulk_commit();
+      constexpr uint32_t id = tc::idesc_bf16(128, 128, 1, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + Lay::ACC2, tc::desc_mnmajor(st + Lay::SWQ, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::BT, 128, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR2);
+    }
+    const float dch = reinterpret_cast<const float *>(sp + (st - sb) + Lay::SD)[crow];
+    if (__syncthreads_or(!wait_timed(bar2, ph2, wait_ns))) { aborted = true; break; }
+    ph2 ^= 1;
+    tc::fence_after_sync();
+    {   // dS <- d dS + acc2: the gradient of the state at the end of chunk c - 1
+      float a[64], sv[64];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        tc::tmem_ld32(tl + Lay::ACC2 + hw * 64 + 32 * u, *reinterpret_cast<float(*)[32]>(a + 32 * u));
+        tc::tmem_ld32(s_tm + 32 * u, *reinterpret_cast<float(*)[32]>(sv + 32 * u));
+      }
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 64; ++j) sv[j] = fmaf(dch, sv[j], a[j]);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) tc::tmem_st32(s_tm + 32 * u, *reinterpret_cast<float(*)[32]>(sv + 32 * u));
+#pragma unroll
+      for (int j = 0; j < 64; j += 8)
+        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * 64 + j) >> 3), sv + j);
+      float *dst = c > 0 ? row_ptr(dsl, p0 + c - 1) : (dinit ? row_ptr(dinit, unit) : nullptr);
+      if (dst)
+#pragma unroll
+        for (int j = 0; j < 64; j += 4)
+          *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+      tc::tmem_wait_st();
+    }
+    if (tid == 0) bulk_wait_read();   // BT is rewritten by the next chunk
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 32 && c - Lay::NST >= 0) issue_packet(c - Lay::NST, s);
+  }
+  if (tid == 0) bulk_wait_all();
+  if (aborted) {
+    report(dev_status, KDA_ERR_TIMEOUT);
+    wait_timed(bar1, ph1, wait_ns);
+    wait_timed(bar2, ph2, wait_ns);
+    wait_timed(dobar, dphase, wait_ns);
+    for (int s = 0; s < Lay::NST; ++s) wait_timed(full + s, (fphase >> s) & 1u, wait_ns);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+}  // namespace kda
+
+namespace kda {
+namespace {
+
+// ---------------------------------------------------------------------------
+// 2, 3. Per (chunk, head): the state part (PART 0) and the Gram part (PART 1)
+// ---------------------------------------------------------------------------
+struct BItemLayout {
+  static constexpr uint32_t GA = 0;          // [128][128] Gram A: k x rows 0..63, q x rows 64..127
+  static constexpr uint32_t S0T = GA;        //   PART 0, after the Gram: S0 [ch][v] bf16
+  static constexpr uint32_t GB = 32768;      // [96][128] Gram B: k y (ref 1) | k y (ref 2), first half | k y, second half
+  static constexpr uint32_t RU = 32768;      //   PART 0, after the Gram: [R; U] [tok][v] bf16 (128 rows)
+  static constexpr uint32_t GST = 65536;     // float [64][128]: g, then Gam in place
+  static constexpr uint32_t KT = 98304;      // [64][128] Ktilde (PART 0)
+  static constexpr uint32_t VT = 114688;     // [64][128] V (PART 0)
+  static constexpr uint32_t BT2 = KT;        //   PART 0, after R: [-dU; dO] from the chain, then [-dR; dO]
+  static constexpr uint32_t XA = KT;         //   PART 1: [dG; dP] placed against Gram B (K = 96)
+  static constexpr uint32_t MM = 131072;     // float [64][68] M = diag(beta) G
+  static constexpr uint32_t XM = MM + 17408; // float [64][68] (I + M)^-1
+  static constexpr uint32_t CST = XM;        //   gate factors during the prep: float [2][6][128]
+  static constexpr uint32_t DST = MM;        //   PART 0, after T: dS_L [ch][v] bf16
+  static constexpr uint32_t YA = MM;         //   PART 1, after T: [dG^T | dP^T] placed against Gram A
+  static constexpr uint32_t YS = XM + 17408; // float [2][16][17]
+  static constexpr uint32_t ZS = YS + 2176;  // float [32][36]
+  static constexpr uint32_t MT = ZS + 4608;  // float [32][33] M_(1,0)^T
+  static constexpr uint32_t GG = MT + 4224;  // float [64][68] G (PART 1)
+  static constexpr uint32_t TT = 194560;     // [64][64] T (row r, column i) bf16
+  static constexpr uint32_t RED = TT;        //   scan partials during the prep: float [8][128]
+  static constexpr uint32_t AIT = TT + 8192; // [64][64] (I + M)^-1 bf16 (PART 1)
+  static constexpr uint32_t Y1T = AIT + 8192;// [64][64] Y1 = Ai^T dT bf16 (PART 1)
+  static constexpr uint32_t DTT = Y1T + 8192;// [64][64] dT bf16 (PART 1)
+  static constexpr uint32_t BETA = DTT + 8192;            // float [64]
+  static constexpr uint32_t DD = BETA + 256;              // float [128] sum_j dS_L S0 (PART 0), dbeta [64] (PART 1)
+  static constexpr uint32_t EXTRA = DD + 512;             // float [128] dGam_63 extras (PART 0)
+  static constexpr uint32_t BAR = EXTRA + 512;            // MMA done
+  static constexpr uint32_t TBAR = BAR + 8;               // inputs landed
+  static constexpr uint32_t CBAR = BAR + 16;              // [-dU; dO] landed (PART 0)
+  static constexpr uint32_t TMEM_SLOT = BAR + 24;
+  static constexpr uint32_t TOTAL = BAR + 32;
+  // PART 0 final partials (after the last MMAs): float [64][128] each
+  static constexpr uint32_t PKM = GA, PDG = RU;
+  // PART 1 final partials: float [64][128] and [32][128]
+  static constexpr uint32_t QDG = XA, KMC = YA;
+  static_assert(GG + 17408 <= TT && MT + 4224 <= GG, "solve scratch");
+  static_assert(GB + 24576 <= RU + 32768 && RU + 32768 <= GST, "[R; U] stays clear of Gam");
+  static_assert(CST + 6144 <= XM + 17408, "gate factors");
+  static_assert(TOTAL + 1024 <= 232448, "shared memory");
+};
+
+__device__ __forceinline__ void st_chunk_s(uint8_t *dst, const float *x) {
+  *reinterpret_cast<uint4 *>(dst) = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                                               tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+}
+
+struct BwdItemArgs {
+  const float *beta, *init, *ck;
+  const int32_t *cu;
+  const int64_t *pref;         // [N+1] chunks before sequence n
+  const int64_t *prefck;       // [N+1] full chunks (stored states) before sequence n
+  const float *dsl;            // dS_L per packet (FP32 [128][128])
+  const uint8_t *dudo;         // [-dU; dO] tile per packet
+  float *dtp;                  // dT, dP per packet: FP32 [64][64] each
+  const void *q, *k;           // raw BF16 inputs (re-read by the final epilogues)
+  float *dq, *dk, *dv, *dg, *dbeta;
+  int N, H;
+  int32_t *dev_status;
+  uint64_t wait_ns;
+};
+
+template <int PART>
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
+  using Lay = BItemLayout;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t sraw = smem_u32(smem_raw);
+  const uint32_t sb = (sraw + 1023u) & ~1023u;
+  uint8_t *sp = smem_raw + (sb - sraw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hw = warp >> 2;
+  const int H = a.H;
+
+  float *s_beta = reinterpret_cast<float *>(sp + Lay::BETA);
+  float *s_red = reinterpret_cast<float *>(sp + Lay::RED);
+  float *s_cst = reinterpret_cast<float *>(sp + Lay::CST);
+  float *s_M = reinterpret_cast<float *>(sp + Lay::MM);
+  float *s_X = reinterpret_cast<float *>(sp + Lay::XM);
+  float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
+  float *s_Z = reinterpret_cast<float *>(sp + Lay::ZS);
+  float *s_MT = reinterpret_cast<float *>(sp + Lay::MT);
+  float *s_G = reinterpret_cast<float *>(sp + Lay::GG);
+  float *s_gam = reinterpret_cast<float *>(sp + Lay::GST);
+  float *s_dd = reinterpret_cast<float *>(sp + Lay::DD);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sp + Lay::BAR);
+  uint64_t *tbar = reinterpret_cast<uint64_t *>(sp + Lay::TBAR);
+  uint64_t *cbar = reinterpret_cast<uint64_t *>(sp + Lay::CBAR);
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(tbar, 1);
+    mbar_init(cbar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, 512);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
+  const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+  uint32_t phase = 0, tphase = 0, cphase = 0;
+  bool aborted = false;
+  const int N = a.N;
+  const int64_t total = a.pref[N] * H;
+
+  // Items (sequence, head, chunk) in packet order: p = H pref[n] + h c_n + j.
+  for (int64_t p = blockIdx.x; p < total && !aborted; p += gridDim.x) {
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {   // last sequence whose first packet is at or before p
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.pref[mid] * H <= p) lo = mid; else hi = mid - 1;
+  }
+  const int n = lo;
+  const int64_t nch = a.pref[n + 1] - a.pref[n];
+  const int64_t rem = p - a.pref[n] * H;
+  const int h = (int)(rem / nch);
+  const int64_t j = rem - (int64_t)h * nch;
+  const int unit = n * H + h;
+  const int64_t ckb = a.prefck[n];
+  const int64_t t0 = (int64_t)a.cu[n] + kC * j;
+  const int64_t T_n = (int64_t)a.cu[n + 1] - a.cu[n];
+  const int L = (int)(T_n - kC * j < kC ? T_n - kC * j : kC);
+
+  // Inputs: q, k into the Gram A tile, g into its staging rows, v (PART 0).
+  if (tid == 32) {
+    mbar_expect_tx(sb + Lay::TBAR, 65536 + (PART == 0 ? 16384 : 0));
+    tma_load_3d(sb + Lay::GST, &maps.g, 0, h, (int)t0, sb + Lay::TBAR);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h, (int)t0, sb + Lay::TBAR);
+      tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h, (int)t0, sb + Lay::TBAR);
+      if (PART == 0) tma_load_3d(sb + Lay::VT + b * 8192, &maps.v, 64 * b, h, (int)t0, sb + Lay::TBAR);
+    }
+  }
+  if (tid >= 64 && tid < 64 + kC) {
+    const int r = tid - 64;
+    const bool ok = r < L;
+    cp_async4(sb + Lay::BETA + 4 * r, a.beta + (ok ? (size_t)(t0 + r) * H + h : 0), ok);
+  }
+  cp_async_commit();
+  // The per-chunk states and gradients come from L2 later; start them now.
+  const float *S0src = j == 0 ? (a.init ? a.init + (size_t)unit * kD * kD : nullptr)
+                              : a.ck + ((size_t)(ckb + j - 1) * H + h) * kD * kD;
+  const float *dSsrc = a.dsl + (size_t)p * kD * kD;
+  if (PART == 0) {
+    for (int e = tid; e < 512; e += kThreads) {
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(dSsrc + 32 * e));
+      if (S0src) asm volatile("prefetch.global.L2 [%0];" ::"l"(S0src + 32 * e));
+    }
+  } else {
+    const float *dtp = a.dtp + (size_t)p * 8192;
+    for (int e = tid; e < 256; e += kThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(dtp + 32 * e));
+  }
+
+  cp_async_wait_all();
+  if (__syncthreads_or(!wait_timed(tbar, tphase, a.wait_ns))) aborted = true;
+  tphase ^= 1;
+
+  // ---------------- gate prep ----------------
+  // Warp w owns rows 8w..8w+7 (half hf = w / 4), lane l owns channels 4l..4l+3.
+  if (!aborted) {
+    const int hf = warp >> 2, cq = lane >> 1, sub = (lane & 1) * 8;
+    float2 gm[8][2];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 8 * warp + i;
+      const float4 x = r < L ? *reinterpret_cast<const float4 *>(sp + Lay::GST + r * 512 + lane * 16)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      gm[i][0] = make_float2(x.x, x.y);
+      gm[i][1] = make_float2(x.z, x.w);
+    }
+#pragma unroll
+    for (int i = 1; i < 8; ++i)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) gm[i][c] = __fadd2_rn(gm[i][c], gm[i - 1][c]);
+    *reinterpret_cast<float4 *>(s_red + warp * 128 + 4 * lane) =
+        make_float4(gm[7][0].x, gm[7][0].y, gm[7][1].x, gm[7][1].y);
+    __syncthreads();
+    if (tid < 128) {
+      const int ch = tid;
+      float t[8], run = 0.f, incl[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) t[i] = s_red[i * 128 + ch];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { run += t[i]; incl[i] = run; }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s_red[i * 128 + ch] = incl[i] - t[i];
+      const float G15 = incl[1], G31 = incl[3], G47 = incl[5], G63 = incl[7];
+      // Slots per half: -ref, fk, fk2, fh, fh2, cb (as in the forward's prep).
+      float f[12];
+      f[0] = -G15; f[1] = 1.f; f[2] = __expf(G15);
+      f[3] = __expf(G31 - G15); f[4] = __expf(G63 - G31); f[5] = __expf(G47 - G15);
+      f[6] = -G47; f[7] = __expf(G47 - G31); f[8] = __expf(G31);
+      f[9] = __expf(G63 - G47); f[10] = 1.f; f[11] = 0.f;
+#pragma unroll
+      for (int q2 = 0; q2 < 12; ++q2) s_cst[q2 * 128 + ch] = f[q2];
+    }
+    __syncthreads();
+    float2 nref[2], fk[2], fk2[2], cb[2];
+    {
+      auto ld4 = [&](int slot, float2 *d) {
+        const float4 x = *reinterpret_cast<const float4 *>(s_cst + (hf * 6 + slot) * 128 + 4 * lane);
+        d[0] = make_float2(x.x, x.y);
+        d[1] = make_float2(x.z, x.w);
+      };
+      float2 base[2];
+      const float4 bv = *reinterpret_cast<const float4 *>(s_red + warp * 128 + 4 * lane);
+      base[0] = make_float2(bv.x, bv.y);
+      base[1] = make_float2(bv.z, bv.w);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) gm[i][c] = __fadd2_rn(gm[i][c], base[c]);
+      ld4(0, nref); ld4(1, fk); ld4(2, fk2); ld4(5, cb);
+    }
+    auto st4 = [&](uint8_t *dst, const float2 *x) {
+      *reinterpret_cast<uint2 *>(dst) = make_uint2(tc::pack_bf16(x[0].x, x[0].y), tc::pack_bf16(x[1].x, x[1].y));
+    };
+    auto un4 = [&](const uint2 &u, float2 *x) {
+      x[0] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+      x[1] = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+    };
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 8 * warp + i;
+      float2 kk[2], qq[2], x[2], y[2], t[2];
+      {
+        const bool in = r < L;
+        const uint2 z2 = make_uint2(0, 0);
+        const uint2 kv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub) : z2;
+        const uint2 qv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub) : z2;
+        un4(kv, kk);
+        un4(qv, qq);
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float2 d = __fadd2_rn(gm[i][c], nref[c]);
+        x[c] = make_float2(__expf(d.x), __expf(d.y));   // exp(Gam_r - ref), within [e^-80, e^80]
+        y[c] = make_float2(__expf(-d.x), __expf(-d.y)); // exp(ref - Gam_r)
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], x[c]);
+      st4(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub, t);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(qq[c], x[c]);
+      st4(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub, t);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], y[c]);
+      st4(sp + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, cq) + sub, t);
+      if (!hf) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], __fmul2_rn(y[c], cb[c]));
+        st4(sp + Lay::GB + tc::tile_offset(96, 32 + r, cq) + sub, t);
+      }
+      if (PART == 0) {   // Ktilde = k exp(Gam_r) = k (x fk) fk2
+#pragma unroll
+        for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], __fmul2_rn(__fmul2_rn(x[c], fk[c]), fk2[c]));
+        st4(sp + Lay::KT + tc::tile_offset(64, r, cq) + sub, t);
+      }
+    }
+    // Gam stays for the final epilogue, in place of g.
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<float4 *>(sp + Lay::GST + (8 * warp + i) * 512 + lane * 16) =
+          make_float4(gm[i][0].x, gm[i][0].y, gm[i][1].x, gm[i][1].y);
+    tc::fence_smem_to_async();
+    __syncthreads();
+  }
+
+  // ---------------- gated Gram products: one [128 x 96 x 128] MMA ----------------
+  if (!aborted && tid == 0) {
+    tc::fence_after_sync();
+    constexpr uint32_t id = tc::idesc_bf16(128, 96, 0, 0);
+#pragma unroll
+    for (int s2 = 0; s2 < 8; ++s2)
+      tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::GA, 128, s2), tc::desc_kmajor(sb + Lay::GB, 96, s2),
+                   id, s2 > 0);
+    tc::mma_commit(sb + Lay::BAR);
+  }
+  if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+  phase ^= 1;
+  tc::fence_after_sync();
+  // Gram rows (lane m = row m, k rows only): M (scaled by beta_r, strictly lower),
+  // and for PART 1 G unscaled.
+  if (!aborted) {
+    const int m = 32 * qd + lane, part = m >> 6, r = m & 63, second = r >> 5;
+    const int i0 = second ? 32 * hw : (hw ? 32 : 0);
+    float acc[32];
+    if (second || hw == 0) {
+      tc::tmem_ld32(tl + (second ? 32 + 32 * hw : 0), acc);
+      tc::tmem_wait_ld();
+    }
+    const bool zero = !second && hw;
+    if (part == 0) {
+      const float br = s_beta[r];
+      float4 *dst = reinterpret_cast<float4 *>(s_M + r * 68 + i0);
+      auto mv = [&](int jj) { return (!zero && i0 + jj < r) ? br * acc[jj] : 0.f; };
+#pragma unroll
+      for (int jj = 0; jj < 32; jj += 4) dst[jj >> 2] = make_float4(mv(jj), mv(jj + 1), mv(jj + 2), mv(jj + 3));
+      if (PART == 1) {
+        float4 *gdst = reinterpret_cast<float4 *>(s_G + r * 68 + i0);
+        auto gv = [&](int jj) { return (!zero && i0 + jj < r) ? acc[jj] : 0.f; };
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 4) gdst[jj >> 2] = make_float4(gv(jj), gv(jj + 1), gv(jj + 2), gv(jj + 3));
+      }
+      if (second && i0 == 0)
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) s_MT[jj * 33 + (r - 32)] = br * acc[jj];
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+
+  // ---------------- (I + M)^-1: 16x16 diagonal blocks, then the 32 and 64 levels ----------------
+  if (!aborted) {
+    if (qd >= 2) {
+      const int blk = (qd - 2) + 2 * hw;
+      const int o = 16 * blk, c = lane & 15, hf = lane >> 4;
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = (8 * hf + i == c) ? 1.f : 0.f;
+      const float *mrow = s_M + (o + 8 * hf) * 68 + o;
+#pragma unroll
+      for (int sidx = 0; sidx < 15; ++sidx) {
+        float mm[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mm[i] = mrow[i * 68 + sidx];
+        const float xs = __shfl_sync(0xffffffffu, x[sidx & 7], c + 16 * (sidx >> 3));
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = fmaf(-mm[i], xs, x[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * 68 + o + c] = x[i];
+      if ((blk & 1) == 0)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * 68 + o + 16 + c] = 0.f;
+    }
+    __syncthreads();
+    {
+      const int hh = tid >> 7, rr = (tid >> 3) & 15, c0 = (tid & 7) * 2;
+      const int ro = 32 * hh + 16, co = 32 * hh;
+      float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) {
+        const float mm = s_M[(ro + rr) * 68 + co + s2];
+        const float2 xv = *reinterpret_cast<const float2 *>(s_X + (co + s2) * 68 + co + c0);
+        y0 = fmaf(mm, xv.x, y0);
+        y1 = fmaf(mm, xv.y, y1);
+      }
+      s_Y[(hh * 16 + rr) * 17 + c0] = y0;
+      s_Y[(hh * 16 + rr) * 17 + c0 + 1] = y1;
+      __syncthreads();
+      float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int s2 = 0; s2 < 16; ++s2) {
+        const float av = s_X[(ro + rr) * 68 + ro + s2];
+        x0 = fmaf(av, s_Y[(hh * 16 + s2) * 17 + c0], x0);
+        x1 = fmaf(av, s_Y[(hh * 16 + s2) * 17 + c0 + 1], x1);
+      }
+      *reinterpret_cast<float2 *>(s_X + (ro + rr) * 68 + co + c0) = make_float2(-x0, -x1);
+      __syncthreads();
+    }
+    {
+      const int rr = lane, cq4 = 4 * warp;
+      float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s2 = cq4; s2 < 32; ++s2) {
+        const float mm = s_MT[s2 * 33 + rr];
+        const float4 xv = *reinterpret_cast<const float4 *>(s_X + s2 * 68 + cq4);
+        z.x = fmaf(mm, xv.x, z.x); z.y = fmaf(mm, xv.y, z.y);
+        z.z = fmaf(mm, xv.z, z.z); z.w = fmaf(mm, xv.w, z.w);
+      }
+      *reinterpret_cast<float4 *>(s_Z + rr * 36 + cq4) = z;
+      __syncthreads();
+      const int r2 = 4 * warp + (lane >> 3), c2 = 4 * (lane & 7);
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int s2 = 0; s2 < 4 * warp + 4; ++s2) {
+        const float av = s_X[(32 + r2) * 68 + 32 + s2];
+        const float4 zv = *reinterpret_cast<const float4 *>(s_Z + s2 * 36 + c2);
+        w.x = fmaf(av, zv.x, w.x); w.y = fmaf(av, zv.y, w.y);
+        w.z = fmaf(av, zv.z, w.z); w.w = fmaf(av, zv.w, w.w);
+      }
+      *reinterpret_cast<float4 *>(s_X + (32 + r2) * 68 + c2) = make_float4(-w.x, -w.y, -w.z, -w.w);
+      __syncthreads();
+    }
+    // T_ri = X_ri beta_i (i <= r) and, for PART 1, X itself, as [64][64] bf16 tiles.
+    for (int e = tid; e < 64 * 8; e += kThreads) {
+      const int row = e >> 3, chk = e & 7;
+      float tv[8], xv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = 8 * chk + u;
+        xv[u] = i <= row ? s_X[row * 68 + i] : 0.f;
+        tv[u] = xv[u] * s_beta[i];
+      }
+      st_chunk_s(sp + Lay::TT + tc::tile_offset(64, row, chk), tv);
+      if (PART == 1) st_chunk_s(sp + Lay::AIT + tc::tile_offset(64, row, chk), xv);
+    }
+    tc::fence_smem_to_async();
+    __syncthreads();
+  }
+  const size_t row_stride = (size_t)H * kD;   // elements between tokens in [T][H][128]
+  const size_t base_row = ((size_t)t0 * H + h) * kD;
+  if constexpr (PART == 0) {
+    // ---- S0 and dS_L as BF16 [ch][v] tiles; dd_c = sum_v dS_L[c, v] S0[c, v] ----
+    // S0T lies over the consumed Gram A tile, DST over the consumed M, (I+M)^-1.
+    if (!aborted) {
+      const int c = tid >> 1, h2 = tid & 1;
+      const float *s0r = S0src ? S0src + (size_t)c * kD + 64 * h2 : nullptr;
+      const float *dsr = dSsrc + (size_t)c * kD + 64 * h2;
+      float dot = 0.f;
+#pragma unroll
+      for (int jj = 0; jj < 64; jj += 8) {
+        float xs[8], xd[8];
+#pragma unroll
+        for (int e = 0; e < 8; e += 4) {
+          const float4 u4 = s0r ? *reinterpret_cast<const float4 *>(s0r + jj + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 w4 = *reinterpret_cast<const float4 *>(dsr + jj + e);
+          xs[e] = u4.x; xs[e + 1] = u4.y; xs[e + 2] = u4.z; xs[e + 3] = u4.w;
+          xd[e] = w4.x; xd[e + 1] = w4.y; xd[e + 2] = w4.z; xd[e + 3] = w4.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dot = fmaf(xs[e], xd[e], dot);
+        st_chunk_s(sp + Lay::S0T + tc::tile_offset(128, c, (64 * h2 + jj) >> 3), xs);
+        st_chunk_s(sp + Lay::DST + tc::tile_offset(128, c, (64 * h2 + jj) >> 3), xd);
+      }
+      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      if (h2 == 0) s_dd[c] = dot;
+      tc::fence_smem_to_async();
+      __syncthreads();
+    }
+    // ---- R = V - Ktilde S0 (TMEM columns 128..255) ----
+    if (!aborted && tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + 128, tc::desc_kmajor(sb + Lay::KT, 64, s2),
+                     tc::desc_mnmajor(sb + Lay::S0T, 128, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+    phase ^= 1;
+    tc::fence_after_sync();
+    if (!aborted && qd < 2) {   // rows 0..63 of [R; U]; V rows past the chunk's end are zero
+      const int r = 32 * qd + lane;
+      float acc[64];
+      tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(acc));
+      tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc) {
+        const int chunk = hw * 8 + cc;
+        float xv[8];
+        unpack8(*reinterpret_cast<const uint4 *>(sp + Lay::VT + tc::tile_offset(64, r, chunk)), xv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xv[e] = (r < L ? xv[e] : 0.f) - acc[8 * cc + e];
+        st_chunk_s(sp + Lay::RU + tc::tile_offset(128, r, chunk), xv);
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- U = T R (columns 256..383); the chain's [-dU; dO] tile lands over Ktilde, V ----
+    if (!aborted && tid == 32) {
+      mbar_expect_tx(sb + Lay::CBAR, 32768);
+      bulk_load(sb + Lay::BT2, a.dudo + (size_t)p * 32768, 32768, sb + Lay::CBAR);
+    }
+    if (!aborted && tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::TT, 64, s2),
+                     tc::desc_mnmajor(sb + Lay::RU, 128, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+    phase ^= 1;
+    tc::fence_after_sync();
+    if (!aborted && qd < 2) {   // rows 64..127 of [R; U]
+      const int r = 32 * qd + lane;
+      float acc[64];
+      tc::tmem_ld32(tl + 256 + hw * 64, *reinterpret_cast<float(*)[32]>(acc));
+      tc::tmem_ld32(tl + 256 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        st_chunk_s(sp + Lay::RU + tc::tile_offset(128, 64 + r, hw * 8 + cc), acc + 8 * cc);
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    if (!aborted && __syncthreads_or(!wait_timed(cbar, cphase, a.wait_ns))) aborted = true;
+    cphase ^= 1;
+    // ---- dR = T^T (-dU) -> -dR (columns 0..127);  [-dU; dO] [R; U]^T (384..511):
+    //      rows 0..63 x 0..63 = -dT, rows 64..127 x 64..127 = dP;  [R; U] dS_L^T (256..383):
+    //      rows 64..127 = dKhat ----
+    if (!aborted && tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t idr = tc::idesc_bf16(128, 128, 1, 1);
+      constexpr uint32_t idk = tc::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + 0, tc::desc_mnmajor(sb + Lay::TT, 64, s2),
+                     tc::desc_mnmajor(sb + Lay::BT2, 128, s2), idr, s2 > 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + 384, tc::desc_kmajor(sb + Lay::BT2, 128, s2),
+                     tc::desc_kmajor(sb + Lay::RU, 128, s2), idk, s2 > 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::RU, 128, s2),
+                     tc::desc_kmajor(sb + Lay::DST, 128, s2), idk, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+    phase ^= 1;
+    tc::fence_after_sync();
+    float *dtp = a.dtp + (size_t)p * 8192;
+    if (!aborted) {
+      if (qd < 2) {
+        const int r = 32 * qd + lane;
+        float acc[64];
+        tc::tmem_ld32(tl + 0 + hw * 64, *reinterpret_cast<float(*)[32]>(acc));
+        tc::tmem_ld32(tl + 0 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
+        tc::tmem_wait_ld();
+        if (r < L) {   // dv = dR
+          float *dst = a.dv + base_row + (size_t)r * row_stride + hw * 64;
+#pragma unroll
+          for (int e = 0; e < 64; e += 4)
+            *reinterpret_cast<float4 *>(dst + e) = make_float4(-acc[e], -acc[e + 1], -acc[e + 2], -acc[e + 3]);
+        }
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc)   // -dR replaces -dU in rows 0..63
+          st_chunk_s(sp + Lay::BT2 + tc::tile_offset(128, r, hw * 8 + cc), acc + 8 * cc);
+        float d2[32];
+        tc::tmem_ld32(tl + 384 + hw * 32, d2);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const int i = 32 * hw + e;
+          *reinterpret_cast<float4 *>(dtp + r * 64 + i) =
+              make_float4(i <= r ? -d2[e] : 0.f, i + 1 <= r ? -d2[e + 1] : 0.f,
+                          i + 2 <= r ? -d2[e + 2] : 0.f, i + 3 <= r ? -d2[e + 3] : 0.f);
+        }
+      } else {
+        const int r = 32 * (qd - 2) + lane;
+        float d2[32];
+        tc::tmem_ld32(tl + 448 + hw * 32, d2);
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const int i = 32 * hw + e;
+          *reinterpret_cast<float4 *>(dtp + 4096 + r * 64 + i) =
+              make_float4(i <= r ? d2[e] : 0.f, i + 1 <= r ? d2[e + 1] : 0.f,
+                          i + 2 <= r ? d2[e + 2] : 0.f, i + 3 <= r ? d2[e + 3] : 0.f);
+        }
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- [dKtilde; dQtilde] = [-dR; dO] S0^T (columns 128..255) ----
+    if (!aborted && tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + 128, tc::desc_kmajor(sb + Lay::BT2, 128, s2),
+                     tc::desc_kmajor(sb + Lay::S0T, 128, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+    phase ^= 1;
+    tc::fence_after_sync();
+    // ---- final epilogue: dq, dk and dGam from Qtilde, Ktilde, Khat and d ----
+    float *pkm = reinterpret_cast<float *>(sp + Lay::PKM);   // dk from Khat
+    float *pdg = reinterpret_cast<float *>(sp + Lay::PDG);   // dGam
+    float *pkk = reinterpret_cast<float *>(sp + Lay::BT2);   // k (dk from Khat): the dGam_63 extra
+    const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+    const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(a.k);
+    if (!aborted && qd >= 2) {
+      const int r = 32 * (qd - 2) + lane;
+      const bool in = r < L;
+      float aq[64], ak[64];
+      tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(aq));
+      tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(aq + 32));
+      tc::tmem_ld32(tl + 256 + hw * 64, *reinterpret_cast<float(*)[32]>(ak));
+      tc::tmem_ld32(tl + 256 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ak + 32));
+      tc::tmem_wait_ld();
+      const size_t off = base_row + (size_t)r * row_stride + hw * 64;
+#pragma unroll
+      for (int cc = 0; cc < 64; cc += 8) {
+        float qv[8], kv[8], dq8[8];
+        if (in) {
+          unpack8(*reinterpret_cast<const uint4 *>(qb + off + cc), qv);
+          unpack8(*reinterpret_cast<const uint4 *>(kb + off + cc), kv);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) qv[e] = kv[e] = 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int ch = hw * 64 + cc + e;
+          const float gam = s_gam[r * 128 + ch], g63 = s_gam[63 * 128 + ch];
+          const float dqa = __expf(gam) * aq[cc + e];
+          const float dkm = __expf(g63 - gam) * ak[cc + e];
+          dq8[e] = dqa;
+          pkm[r * 128 + ch] = dkm;
+          pkk[r * 128 + ch] = kv[e] * dkm;
+          pdg[r * 128 + ch] = qv[e] * dqa - kv[e] * dkm;
+        }
+        if (in) {
+          float *dst = a.dq + off + cc;
+          *reinterpret_cast<float4 *>(dst) = make_float4(dq8[0], dq8[1], dq8[2], dq8[3]);
+          *reinterpret_cast<float4 *>(dst + 4) = make_float4(dq8[4], dq8[5], dq8[6], dq8[7]);
+        }
+      }
+    }
+    __syncthreads();
+    if (!aborted && qd < 2) {
+      const int r = 32 * qd + lane;
+      const bool in = r < L;
+      float ak[64];
+      tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(ak));
+      tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ak + 32));
+      tc::tmem_wait_ld();
+      const size_t off = base_row + (size_t)r * row_stride + hw * 64;
+#pragma unroll
+      for (int cc = 0; cc < 64; cc += 8) {
+        float kv[8], dk8[8];
+        if (in) unpack8(*reinterpret_cast<const uint4 *>(kb + off + cc), kv);
+        else
+#pragma unroll
+          for (int e = 0; e < 8; ++e) kv[e] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int ch = hw * 64 + cc + e;
+          const float dkp = __expf(s_gam[r * 128 + ch]) * ak[cc + e];
+          dk8[e] = dkp + pkm[r * 128 + ch];
+          pdg[r * 128 + ch] += kv[e] * dkp;
+        }
+        if (in) {
+          float *dst = a.dk + off + cc;
+          *reinterpret_cast<float4 *>(dst) = make_float4(dk8[0], dk8[1], dk8[2], dk8[3]);
+          *reinterpret_cast<float4 *>(dst + 4) = make_float4(dk8[4], dk8[5], dk8[6], dk8[7]);
+        }
+      }
+    }
+    __syncthreads();
+    if (!aborted && tid < 128) {   // dg = reverse cumulative sum of dGam (+ the Gam_63 terms)
+      const int ch = tid;
+      float suffix = __expf(s_gam[63 * 128 + ch]) * s_dd[ch];
+      for (int r = 0; r < 64; ++r) suffix += pkk[r * 128 + ch];
+      for (int r = 63; r >= 0; --r) {
+        suffix += pdg[r * 128 + ch];
+        if (r < L) a.dg[base_row + (size_t)r * row_stride + ch] = suffix;
+      }
+    }
+  } else {
+    // ---- PART 1: dT, dP from the state part ----
+    const float *dT = a.dtp + (size_t)p * 8192, *dP = dT + 4096;
+    float *s_db = s_dd;   // dbeta [64]
+    if (!aborted) {
+      for (int e = tid; e < 64 * 8; e += kThreads) {
+        const int row = e >> 3, chk = e & 7;
+        float x8[8];
+        const float4 u0 = *reinterpret_cast<const float4 *>(dT + row * 64 + 8 * chk);
+        const float4 u1 = *reinterpret_cast<const float4 *>(dT + row * 64 + 8 * chk + 4);
+        x8[0] = u0.x; x8[1] = u0.y; x8[2] = u0.z; x8[3] = u0.w;
+        x8[4] = u1.x; x8[5] = u1.y; x8[6] = u1.z; x8[7] = u1.w;
+        st_chunk_s(sp + Lay::DTT + tc::tile_offset(64, row, chk), x8);
+      }
+      tc::fence_smem_to_async();
+      __syncthreads();
+    }
+    // ---- Y1 = Ai^T dT (columns 128..191) ----
+    if (!aborted && tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 64, 1, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + 128, tc::desc_mnmajor(sb + Lay::AIT, 64, s2),
+                     tc::desc_mnmajor(sb + Lay::DTT, 64, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+    phase ^= 1;
+    tc::fence_after_sync();
+    if (!aborted && qd < 2) {   // dbeta_j = Y1_jj (the T part); Y1 as a K-major operand
+      const int jr = 32 * qd + lane;
+      float y[32];
+      tc::tmem_ld32(tl + 128 + hw * 32, y);
+      tc::tmem_wait_ld();
+      if ((jr >> 5) == hw) {
+        float dgl = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) dgl = e == (jr & 31) ? y[e] : dgl;
+        s_db[jr] = dgl;
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) st_chunk_s(sp + Lay::Y1T + tc::tile_offset(64, jr, hw * 4 + cc), y + 8 * cc);
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- dA = -Y1 T^T (columns 256..319) and its transpose (384..447) ----
+    if (!aborted && tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 64, 0, 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::Y1T, 64, s2),
+                     tc::desc_kmajor(sb + Lay::TT, 64, s2), id, s2 > 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 4; ++s2)
+        tc::mma_bf16(tmem + 384, tc::desc_kmajor(sb + Lay::TT, 64, s2),
+                     tc::desc_kmajor(sb + Lay::Y1T, 64, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    // While they run: dP into rows 64..127 of XA (against Gram B) and columns
+    // 64..127 of YA (against the q x rows of Gram A).  XA row rho: first-half
+    // rows take column kappa = i, second-half rows kappa = 32 + i (Gram B rows
+    // 32..95 are k y against the second half's reference for every key).
+    // YA row i (second index, own reference): dP_ri for r in i's half; row
+    // 64 + i (i in the first half, second-half reference): dP_ri for r in the
+    // second half; rows 96..127 zero.
+    if (!aborted) {
+      {
+        const int r = tid >> 2, kq = (tid & 3) * 24;   // 24 columns of kappa each
+        float x8[8];
+#pragma unroll
+        for (int cc = 0; cc < 3; ++cc) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int kap = kq + 8 * cc + e;
+            const int i = r < 32 ? kap : kap - 32;
+            const bool ok = (r < 32 ? kap < 32 : kap >= 32) && i <= r;
+            x8[e] = ok ? dP[r * 64 + i] : 0.f;
+          }
+          st_chunk_s(sp + Lay::XA + tc::tile_offset(128, 64 + r, (kq >> 3) + cc), x8);
+        }
+      }
+      {
+        const int m = tid >> 1, rh = (tid & 1) * 32;   // YA row m, P columns r = rh..rh+31
+        float x8[8];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int r = rh + 8 * cc + e;
+            float val = 0.f;
+            if (m < 64) {
+              if ((m >> 5) == (r >> 5) && r >= m) val = dP[r * 64 + m];
+            } else if (m < 96) {
+              if (r >= 32) val = dP[r * 64 + (m - 64)];
+            }
+            x8[e] = val;
+          }
+          st_chunk_s(sp + Lay::YA + tc::tile_offset(128, m, 8 + (rh >> 3) + cc), x8);
+        }
+      }
+    }
+    if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+    phase ^= 1;
+    tc::fence_after_sync();
+    if (!aborted) {
+      if (qd < 2) {   // row rho of dA: dM, dbeta (the M part), dG into rows 0..63 of XA
+        const int rho = 32 * qd + lane;
+        float x[32];
+        tc::tmem_ld32(tl + 256 + hw * 32, x);
+        tc::tmem_wait_ld();
+        const float br = s_beta[rho];
+        float db = 0.f, vals[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int sig = 32 * hw + e;
+          const float dm = sig < rho ? -x[e] : 0.f;
+          db = fmaf(dm, s_G[rho * 68 + sig], db);
+          vals[e] = br * dm;
+        }
+        atomicAdd(&s_db[rho], db);
+        const int kbase = (rho < 32 ? 0 : 32) + 32 * hw;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_chunk_s(sp + Lay::XA + tc::tile_offset(128, rho, (kbase >> 3) + cc), vals + 8 * cc);
+        if ((rho < 32) == (hw == 1)) {   // the four chunks of kappa this row leaves zero
+          float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          const int kz = rho < 32 ? 64 : 0;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc) st_chunk_s(sp + Lay::XA + tc::tile_offset(128, rho, (kz >> 3) + cc), z);
+        }
+      } else {        // column sig of dA (from the transposed product): dG^T into YA
+        const int sig = 32 * (qd - 2) + lane;
+        float x[32];
+        tc::tmem_ld32(tl + 384 + hw * 32, x);
+        tc::tmem_wait_ld();
+        float vals[32], z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int rho = 32 * hw + e;
+          vals[e] = rho > sig ? s_beta[rho] * (-x[e]) : 0.f;
+        }
+        const bool cross = sig < 32 && hw == 1;   // second-half rho against a first-half sig
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          st_chunk_s(sp + Lay::YA + tc::tile_offset(128, sig, hw * 4 + cc), cross ? z : vals + 8 * cc);
+          st_chunk_s(sp + Lay::YA + tc::tile_offset(128, 64 + sig, hw * 4 + cc), cross ? vals + 8 * cc : z);
+        }
+      }
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    // ---- [X; Xq] = [dG; dP] Gram B (columns 0..127), Y = [dG^T | dP^T] Gram A (128..255) ----
+    if (!aborted && tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+      for (int s2 = 0; s2 < 6; ++s2)
+        tc::mma_bf16(tmem + 0, tc::desc_kmajor(sb + Lay::XA, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::GB, 96, s2), id, s2 > 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + 128, tc::desc_kmajor(sb + Lay::YA, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::GA, 128, s2), id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+    phase ^= 1;
+    tc::fence_after_sync();
+    // ---- final epilogue: the rest of dq, dk, dGam; dbeta ----
+    float *qdg = reinterpret_cast<float *>(sp + Lay::QDG);   // q dq, then dGam
+    float *kmc = reinterpret_cast<float *>(sp + Lay::KMC);   // dk from first-half keys, second-half reference
+    const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(a.q);
+    const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(a.k);
+    if (!aborted && qd >= 2) {
+      const int r = 32 * (qd - 2) + lane;
+      const bool in = r < L;
+      float xq[64], yc[64];
+      tc::tmem_ld32(tl + 0 + hw * 64, *reinterpret_cast<float(*)[32]>(xq));
+      tc::tmem_ld32(tl + 0 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(xq + 32));
+      tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(yc));
+      tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(yc + 32));
+      tc::tmem_wait_ld();
+      const size_t off = base_row + (size_t)r * row_stride + hw * 64;
+      const int ref = r < 32 ? 15 : 47;
+#pragma unroll
+      for (int cc = 0; cc < 64; cc += 8) {
+        float qv[8], add[8];
+        if (in) unpack8(*reinterpret_cast<const uint4 *>(qb + off + cc), qv);
+        else
+#pragma unroll
+          for (int e = 0; e < 8; ++e) qv[e] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int ch = hw * 64 + cc + e;
+          const float gam = s_gam[r * 128 + ch];
+          const float dqb = __expf(gam - s_gam[ref * 128 + ch]) * xq[cc + e];
+          add[e] = dqb;
+          qdg[r * 128 + ch] = qv[e] * dqb;
+          if (r < 32) kmc[r * 128 + ch] = __expf(s_gam[47 * 128 + ch] - gam) * yc[cc + e];
+        }
+        if (in) {
+          float *dst = a.dq + off + cc;
+          float4 o0 = *reinterpret_cast<float4 *>(dst), o1 = *reinterpret_cast<float4 *>(dst + 4);
+          o0.x += add[0]; o0.y += add[1]; o0.z += add[2]; o0.w += add[3];
+          o1.x += add[4]; o1.y += add[5]; o1.z += add[6]; o1.w += add[7];
+          *reinterpret_cast<float4 *>(dst) = o0;
+          *reinterpret_cast<float4 *>(dst + 4) = o1;
+        }
+      }
+    }
+    __syncthreads();
+    if (!aborted && qd < 2) {
+      const int t = 32 * qd + lane;
+      const bool in = t < L;
+      float xk[64], yo[64];
+      tc::tmem_ld32(tl + 0 + hw * 64, *reinterpret_cast<float(*)[32]>(xk));
+      tc::tmem_ld32(tl + 0 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(xk + 32));
+      tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(yo));
+      tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(yo + 32));
+      tc::tmem_wait_ld();
+      const size_t off = base_row + (size_t)t * row_stride + hw * 64;
+      const int ref = t < 32 ? 15 : 47;
+#pragma unroll
+      for (int cc = 0; cc < 64; cc += 8) {
+        float kv[8], add[8];
+        if (in) unpack8(*reinterpret_cast<const uint4 *>(kb + off + cc), kv);
+        else
+#pragma unroll
+          for (int e = 0; e < 8; ++e) kv[e] = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int ch = hw * 64 + cc + e;
+          const float dlt = s_gam[t * 128 + ch] - s_gam[ref * 128 + ch];
+          const float dkp = __expf(dlt) * xk[cc + e];
+          const float dkm = __expf(-dlt) * yo[cc + e] + (t < 32 ? kmc[t * 128 + ch] : 0.f);
+          add[e] = dkp + dkm;
+          qdg[t * 128 + ch] += kv[e] * (dkp - dkm);
+        }
+        if (in) {
+          float *dst = a.dk + off + cc;
+          float4 o0 = *reinterpret_cast<float4 *>(dst), o1 = *reinterpret_cast<float4 *>(dst + 4);
+          o0.x += add[0]; o0.y += add[1]; o0.z += add[2]; o0.w += add[3];
+          o1.x += add[4]; o1.y += add[5]; o1.z += add[6]; o1.w += add[7];
+          *reinterpret_cast<float4 *>(dst) = o0;
+          *reinterpret_cast<float4 *>(dst + 4) = o1;
+        }
+      }
+    }
+    __syncthreads();
+    if (!aborted && tid < 128) {
+      const int ch = tid;
+      float suffix = 0.f;
+      for (int r = 63; r >= 0; --r) {
+        suffix += qdg[r * 128 + ch];
+        if (r < L) a.dg[base_row + (size_t)r * row_stride + ch] += suffix;
+      }
+    }
+    if (!aborted && tid < L) a.dbeta[(size_t)(t0 + tid) * H + h] = s_db[tid];
+  }
+  // Every reader of this item's shared memory and tensor memory is done
+  // before the next item's copies land.
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  }   // items
+
+  if (aborted) {
+    report(a.dev_status, KDA_ERR_TIMEOUT);
+    wait_timed(bar, phase, a.wait_ns);
+    wait_timed(tbar, tphase, a.wait_ns);
+    if (PART == 0) wait_timed(cbar, cphase, a.wait_ns);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+}  // namespace kda
+
+namespace kda {
+namespace {
+
+// pref[n] = chunks of the sequences before n, prefck[n] = their full chunks
+// (the states the forward stores every 64 tokens); one warp.
+__global__ void bwd_prefix_kernel(const int32_t *__restrict__ cu, int N, int64_t *pref,
+                                  int64_t *prefck) {
+  const int lane = threadIdx.x;
+  int64_t carry = 0, carryck = 0;
+  if (lane == 0) { pref[0] = 0; prefck[0] = 0; }
+  for (int base = 0; base < N; base += 32) {
+    const int i = base + lane;
+    const int64_t len = i < N ? (int64_t)cu[i + 1] - cu[i] : 0;
+    int64_t v = (len + kC - 1) / kC, w = len / kC;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int64_t tv = __shfl_up_sync(0xffffffffu, v, o), tw = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) { v += tv; w += tw; }
+    }
+    if (i < N) { pref[i + 1] = carry + v; prefck[i + 1] = carryck + w; }
+    carry += __shfl_sync(0xffffffffu, v, 31);
+    carryck += __shfl_sync(0xffffffffu, w, 31);
+  }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct BwdWs {
+  size_t pk, ck, dsl, dudo, dtp, oscr, pref, prefck, total;
+};
+
+BwdWs bwd_ws_layout(int N, int H, int64_t T) {
+  const size_t P = (size_t)H * (size_t)((T + (int64_t)(kC - 1) * N) / kC);   // packets, upper bound
+  BwdWs w;
+  size_t off = 0;
+  w.pk = off;     off += align256(P * Pk::BYTES + 256);
+  w.ck = off;     off += align256((size_t)(T / kC) * H * kD * kD * 4);
+  w.dsl = off;    off += align256(P * kD * kD * 4);
+  w.dudo = off;   off += align256(P * 32768);
+  w.dtp = off;    off += align256(P * 8192 * 4);
+  w.oscr = off;   off += align256((size_t)T * H * kD * 2);
+  w.pref = off;   off += align256((size_t)(N + 1) * 8);
+  w.prefck = off; off += align256((size_t)(N + 1) * 8);
+  w.total = off + 256;
+  return w;
+}
+
+}  // namespace
+
+bool backward_tc_supported(int dtype, int dk, int dv, int N) {
+  return dtype == KDA_DTYPE_BF16 && dk == kD && dv == kD && prefill_split_supported(N);
+}
+
+size_t backward_tc_workspace_bytes(int N, int H, int64_t T) { return bwd_ws_layout(N, H, T).total; }
+
+cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, const float *init, const int32_t *cu,
+                               const float *dout, const float *dfin, float *dq, float *dk,
+                               float *dv, float *dg, float *dbeta, float *dinit, void *workspace,
+                               int N, int H, int64_t T, int32_t *dev_status, cudaStream_t stream,
+                               int num_sms) {
+  if (split_packet_bytes() != Pk::BYTES) return cudaErrorInvalidValue;
+  const BwdWs w = bwd_ws_layout(N, H, T);
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(workspace) + 255) & ~(uintptr_t)255);
+  uint8_t *pk = base + w.pk;
+  float *ck = reinterpret_cast<float *>(base + w.ck);
+  float *dsl = reinterpret_cast<float *>(base + w.dsl);
+  uint8_t *dudo = base + w.dudo;
+  float *dtp = reinterpret_cast<float *>(base + w.dtp);
+  void *oscr = base + w.oscr;
+  int64_t *pref = reinterpret_cast<int64_t *>(base + w.pref);
+  int64_t *prefck = reinterpret_cast<int64_t *>(base + w.prefck);
+  const uint64_t wait_ns = 2000000000ull;
+
+  // Forward recomputation: the two-pass prefill in one window keeps every
+  // intra-chunk packet in the workspace and stores the state every 64 tokens.
+  cudaError_t e = launch_prefill_split(q, k, v, g, beta, init, cu, oscr, nullptr, kC, ck, N, H, T,
+                                       pk, w.ck - w.pk, dev_status, stream, num_sms);
+  if (e != cudaSuccess) return e;
+  bwd_prefix_kernel<<<1, 32, 0, stream>>>(cu, N, pref, prefck);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  CUtensorMap dout_map;
+  TmaMaps maps;
+  if (!make_map(&dout_map, dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kD, H, T, kD, kC,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_input_maps(&maps, q, k, v, g, H, T) ||
+      !make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, H, T, 64, 64,
+                CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, H, T, 64, 64,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+
+  const size_t smem_c = BChainLayout::TOTAL + 1024;
+  e = cudaFuncSetAttribute(bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
+  if (e != cudaSuccess) return e;
+  bwd_chain_kernel<<<(unsigned)((int64_t)N * H), kThreads, smem_c, stream>>>(
+      dout_map, pk, cu, dfin, dinit, dsl, dudo, N, H, dev_status, wait_ns);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  BwdItemArgs a;
+  a.beta = beta; a.init = init; a.ck = ck; a.cu = cu; a.pref = pref; a.prefck = prefck;
+  a.dsl = dsl; a.dudo = dudo; a.dtp = dtp; a.q = q; a.k = k;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
+  a.N = N; a.H = H; a.dev_status = dev_status; a.wait_ns = wait_ns;
+  const size_t smem_i = BItemLayout::TOTAL + 1024;
+  e = cudaFuncSetAttribute(bwd_item_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_i);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_item_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_i);
+  if (e != cudaSuccess) return e;
+  bwd_item_kernel<0><<<num_sms, kThreads, smem_i, stream>>>(maps, a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  bwd_item_kernel<1><<<num_sms, kThreads, smem_i, stream>>>(maps, a);
+  return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -5,6 +5,7 @@
 //   y = A^T k, z = A^T q with A = Diag(alpha) S_{t-1};  u = beta (v - y);
 //   S_t = A + k u^T;  o = z + (q . k) u.
 #include "kda_common.cuh"
+#include "kda_tma.cuh"
 
 namespace kda {
 
@@ -12,11 +13,31 @@ namespace kda {
 // head) runs T_new tokens through the recurrence with its state held in
 // registers, writes the output of every token, and stores the state reached
 // after the first accept_len[n] tokens (all T_new when accept_len is null).
-// One HBM round trip of the state serves all T_new tokens.  Tokens are staged
-// in shared memory in groups of kMultiGroup with one batched load, and their
-// gates are formed for the whole group before the token loop, so each token
-// costs two block barriers and no global-memory latency.
+// One HBM round trip of the state serves all T_new tokens.
+//
+// The kernel is persistent: two CTAs per SM walk the (sequence, head) units,
+// and while a CTA runs the token loop of one unit, the next unit's FP32 state
+// (one bulk copy into shared memory, completing on an mbarrier) and the raw
+// inputs of its first kMultiGroup tokens (16-byte async copies) are already on
+// their way, so the SM's share of HBM bandwidth stays busy during the serial
+// token loop.  Tokens are prepared in groups of kMultiGroup (gates and q . k
+// for the whole group before the token loop), so each token costs two block
+// barriers and no global-memory latency.
 constexpr int kMultiGroup = 8;
+
+template <int DK, int DV, typename TIn>
+struct MultiLayout {
+  static constexpr int G = kMultiGroup;
+  static constexpr uint32_t STATE = 0;                                    // float [DK][DV]
+  static constexpr uint32_t RAW_Q = DK * DV * 4;                          // TIn [G][DK]
+  static constexpr uint32_t RAW_K = RAW_Q + G * DK * sizeof(TIn);         // TIn [G][DK]
+  static constexpr uint32_t RAW_V = RAW_K + G * DK * sizeof(TIn);         // TIn [G][DV]
+  static constexpr uint32_t RAW_G = RAW_V + G * DV * sizeof(TIn);         // float [G][DK]
+  static constexpr uint32_t RAW_B = RAW_G + G * DK * 4;                   // float [G]
+  static constexpr uint32_t BAR = RAW_B + 64;                             // mbarrier
+  static constexpr uint32_t TOTAL = BAR + 16;
+  static_assert(RAW_Q % 16 == 0 && RAW_G % 16 == 0 && BAR % 8 == 0, "alignment");
+};
 
 template <int DK, int DV, int THREADS, typename TIn>
 __global__ void __launch_bounds__(THREADS, 2)
@@ -24,124 +45,233 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
                     const TIn *__restrict__ v, const float *__restrict__ g,
                     const float *__restrict__ beta, float *__restrict__ state,
                     TIn *__restrict__ out, const int32_t *__restrict__ accept_len, int T_new,
-                    int H) {
+                    int H, int64_t units, int32_t *dev_status, uint64_t wait_ns) {
+  using Lay = MultiLayout<DK, DV, TIn>;
   constexpr int V4 = DV / 4;
   constexpr int RPP = THREADS / V4;
   constexpr int ROWS = DK / RPP;
   constexpr int G = kMultiGroup;
   static_assert(THREADS % V4 == 0 && DK % RPP == 0, "tile mismatch");
 
+  extern __shared__ __align__(16) uint8_t smem_raw[];
   __shared__ float s_ka[G][DK], s_qa[G][DK], s_alpha[G][DK], s_k[G][DK];
   __shared__ float s_v[G][DV], s_beta[G], s_qk[G];
   __shared__ float s_u[2][DV];
   __shared__ float4 s_red[2][2][RPP][V4];
 
-  const int unit = blockIdx.x, n = unit / H, h = unit % H;
   const int tid = threadIdx.x, cg = tid % V4, rg = tid / V4;
   const int lane = tid & 31, warp = tid >> 5;
-  int acc = T_new;
-  if (accept_len) {
-    acc = accept_len[n];
-    acc = acc < 0 ? 0 : (acc > T_new ? T_new : acc);
+  const uint32_t sb = smem_u32(smem_raw);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(smem_raw + Lay::BAR);
+  int64_t u = blockIdx.x;
+  if (u >= units) return;
+
+  // Next unit's state: one bulk copy (tid 0); its first group's raw inputs:
+  // 16-byte async copies spread over the block, beta by 4-byte copies.
+  auto prefetch = [&](int64_t unit) {
+    const int n = (int)(unit / H), h = (int)(unit % H);
+    if (tid == 0) {
+      mbar_expect_tx(sb + Lay::BAR, DK * DV * 4);
+      bulk_load(sb + Lay::STATE, state + (size_t)unit * DK * DV, DK * DV * 4, sb + Lay::BAR);
+    }
+    constexpr int QCH = DK * (int)sizeof(TIn) / 16, VCH = DV * (int)sizeof(TIn) / 16;
+    constexpr int GCH = DK * 4 / 16, PER = 2 * QCH + VCH + GCH;
+    const int cnt = T_new < G ? T_new : G;
+    for (int e = tid; e < cnt * PER; e += THREADS) {
+      const int j = e / PER, r = e % PER;
+      const size_t tok = ((size_t)n * T_new + j) * H + h;
+      const uint8_t *src;
+      uint32_t dst;
+      if (r < QCH) {
+        src = reinterpret_cast<const uint8_t *>(q + tok * DK) + 16 * r;
+        dst = Lay::RAW_Q + j * DK * sizeof(TIn) + 16 * r;
+      } else if (r < 2 * QCH) {
+        src = reinterpret_cast<const uint8_t *>(k + tok * DK) + 16 * (r - QCH);
+        dst = Lay::RAW_K + j * DK * sizeof(TIn) + 16 * (r - QCH);
+      } else if (r < 2 * QCH + VCH) {
+        src = reinterpret_cast<const uint8_t *>(v + tok * DV) + 16 * (r - 2 * QCH);
+        dst = Lay::RAW_V + j * DV * sizeof(TIn) + 16 * (r - 2 * QCH);
+      } else {
+        src = reinterpret_cast<const uint8_t *>(g + tok * DK) + 16 * (r - 2 * QCH - VCH);
+        dst = Lay::RAW_G + j * DK * 4 + 16 * (r - 2 * QCH - VCH);
+      }
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sb + dst), "l"(src) : "memory");
+    }
+    if (tid < cnt) cp_async4(sb + Lay::RAW_B + 4 * tid, beta + ((size_t)n * T_new + tid) * H + h, true);
+    cp_async_commit();
+  };
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  __syncthreads();
+  prefetch(u);
+  uint32_t phase = 0;
+  bool aborted = false;
 
-  float4 *S4 = reinterpret_cast<float4 *>(state + (size_t)unit * DK * DV);
-  // the thread's float4 of each row as two pairs, for the paired FP32 units
-  float2 sa[ROWS], sb[ROWS];
-#pragma unroll
-  for (int i = 0; i < ROWS; ++i) {
-    const float4 x = __ldcs(&S4[(rg + i * RPP) * V4 + cg]);
-    sa[i] = make_float2(x.x, x.y);
-    sb[i] = make_float2(x.z, x.w);
-  }
-
-  for (int t0 = 0; t0 < T_new; t0 += G) {
-    const int cnt = T_new - t0 < G ? T_new - t0 : G;
-    // Stage the group: gates and products for every token at once.
-    for (int e = tid; e < cnt * DK; e += THREADS) {
-      const int j = e / DK, c = e % DK;
-      const size_t off = (((size_t)n * T_new + t0 + j) * H + h) * DK + c;
-      const float kc = to_f32(k[off]), qc = to_f32(q[off]);
-      const float a = __expf(g[off]);
-      s_alpha[j][c] = a;
-      s_k[j][c] = kc;
-      s_ka[j][c] = a * kc;
-      s_qa[j][c] = qc;     // q for now; becomes alpha * q below
+  for (; u < units; u += gridDim.x) {
+    const int n = (int)(u / H), h = (int)(u % H);
+    int acc = T_new;
+    if (accept_len) {
+      acc = accept_len[n];
+      acc = acc < 0 ? 0 : (acc > T_new ? T_new : acc);
     }
-    for (int e = tid; e < cnt * DV; e += THREADS) {
-      const int j = e / DV, c = e % DV;
-      s_v[j][c] = to_f32(v[(((size_t)n * T_new + t0 + j) * H + h) * DV + c]);
-    }
-    if (tid < cnt) s_beta[tid] = beta[((size_t)n * T_new + t0 + tid) * H + h];
-    __syncthreads();
-    // q . k per token (one warp per token), then q <- alpha * q
-    for (int j = warp; j < cnt; j += THREADS / 32) {
-      float qk = 0.f;
-      for (int c = lane; c < DK; c += 32) qk += s_qa[j][c] * s_k[j][c];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
-      if (lane == 0) s_qk[j] = qk;
-      for (int c = lane; c < DK; c += 32) s_qa[j][c] *= s_alpha[j][c];
-    }
-    __syncthreads();
-
-    for (int j = 0; j < cnt; ++j) {
-      const int t = t0 + j, p = t & 1;   // parity-indexed buffers: no third barrier
-      float2 ya = make_float2(0.f, 0.f), yb = ya, za = ya, zb = ya;
+    if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
+    phase ^= 1;
+    // the thread's float4 of each row as two pairs, for the paired FP32 units
+    float2 sa[ROWS], sb2[ROWS];
+    {
+      const float4 *S4s = reinterpret_cast<const float4 *>(smem_raw + Lay::STATE);
 #pragma unroll
       for (int i = 0; i < ROWS; ++i) {
-        const int r = rg + i * RPP;
-        const float2 ka = make_float2(s_ka[j][r], s_ka[j][r]);
-        const float2 qa = make_float2(s_qa[j][r], s_qa[j][r]);
-        ya = __ffma2_rn(ka, sa[i], ya);
-        yb = __ffma2_rn(ka, sb[i], yb);
-        za = __ffma2_rn(qa, sa[i], za);
-        zb = __ffma2_rn(qa, sb[i], zb);
+        const float4 x = S4s[(rg + i * RPP) * V4 + cg];
+        sa[i] = make_float2(x.x, x.y);
+        sb2[i] = make_float2(x.z, x.w);
       }
-      s_red[p][0][rg][cg] = make_float4(ya.x, ya.y, yb.x, yb.y);
-      s_red[p][1][rg][cg] = make_float4(za.x, za.y, zb.x, zb.y);
-      __syncthreads();
-      if (tid < DV) {
-        const int c4 = tid >> 2, lane4 = tid & 3;
-        float yy = 0.f, zz = 0.f;
-#pragma unroll 8
-        for (int r = 0; r < RPP; ++r) {
-          yy += reinterpret_cast<const float *>(&s_red[p][0][r][c4])[lane4];
-          zz += reinterpret_cast<const float *>(&s_red[p][1][r][c4])[lane4];
+    }
+    cp_async_wait_all();
+    // Every thread has read the state and its token copies have landed: the
+    // buffers may be refilled once the raw group is converted below.
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    float4 *S4 = reinterpret_cast<float4 *>(state + (size_t)u * DK * DV);
+
+    for (int t0 = 0; t0 < T_new; t0 += G) {
+      const int cnt = T_new - t0 < G ? T_new - t0 : G;
+      // Stage the group: gates and products for every token at once.  The
+      // first group comes from the prefetched raw copies, later ones (drafts
+      // longer than a group) straight from global memory.
+      if (t0 == 0) {
+        const TIn *rq = reinterpret_cast<const TIn *>(smem_raw + Lay::RAW_Q);
+        const TIn *rk = reinterpret_cast<const TIn *>(smem_raw + Lay::RAW_K);
+        const TIn *rv = reinterpret_cast<const TIn *>(smem_raw + Lay::RAW_V);
+        const float *rg_ = reinterpret_cast<const float *>(smem_raw + Lay::RAW_G);
+        for (int e = tid; e < cnt * DK; e += THREADS) {
+          const int j = e / DK, c = e % DK;
+          const float kc = to_f32(rk[j * DK + c]), qc = to_f32(rq[j * DK + c]);
+          const float a = __expf(rg_[j * DK + c]);
+          s_alpha[j][c] = a;
+          s_k[j][c] = kc;
+          s_ka[j][c] = a * kc;
+          s_qa[j][c] = qc;     // q for now; becomes alpha * q below
         }
-        const float u = s_beta[j] * (s_v[j][tid] - yy);
-        s_u[p][tid] = u;
-        out[(((size_t)n * T_new + t) * H + h) * DV + tid] = from_f32<TIn>(zz + s_qk[j] * u);
+        for (int e = tid; e < cnt * DV; e += THREADS) {
+          const int j = e / DV, c = e % DV;
+          s_v[j][c] = to_f32(rv[j * DV + c]);
+        }
+        if (tid < cnt) s_beta[tid] = reinterpret_cast<const float *>(smem_raw + Lay::RAW_B)[tid];
+        __syncthreads();
+        const int64_t nx = u + gridDim.x;   // the raw and state buffers are free now
+        if (nx < units) prefetch(nx);
+      } else {
+        for (int e = tid; e < cnt * DK; e += THREADS) {
+          const int j = e / DK, c = e % DK;
+          const size_t off = (((size_t)n * T_new + t0 + j) * H + h) * DK + c;
+          const float kc = to_f32(k[off]), qc = to_f32(q[off]);
+          const float a = __expf(g[off]);
+          s_alpha[j][c] = a;
+          s_k[j][c] = kc;
+          s_ka[j][c] = a * kc;
+          s_qa[j][c] = qc;
+        }
+        for (int e = tid; e < cnt * DV; e += THREADS) {
+          const int j = e / DV, c = e % DV;
+          s_v[j][c] = to_f32(v[(((size_t)n * T_new + t0 + j) * H + h) * DV + c]);
+        }
+        if (tid < cnt) s_beta[tid] = beta[((size_t)n * T_new + t0 + tid) * H + h];
+        __syncthreads();
+      }
+      // q . k per token (one warp per token), then q <- alpha * q
+      for (int j = warp; j < cnt; j += THREADS / 32) {
+        float qk = 0.f;
+        for (int c = lane; c < DK; c += 32) qk += s_qa[j][c] * s_k[j][c];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
+        if (lane == 0) s_qk[j] = qk;
+        for (int c = lane; c < DK; c += 32) s_qa[j][c] *= s_alpha[j][c];
       }
       __syncthreads();
-      const float4 u4 = reinterpret_cast<const float4 *>(s_u[p])[cg];
-      const float2 ua = make_float2(u4.x, u4.y), ub = make_float2(u4.z, u4.w);
+
+      for (int j = 0; j < cnt; ++j) {
+        const int t = t0 + j, p = t & 1;   // parity-indexed buffers: no third barrier
+        float2 ya = make_float2(0.f, 0.f), yb = ya, za = ya, zb = ya;
 #pragma unroll
-      for (int i = 0; i < ROWS; ++i) {
-        const int r = rg + i * RPP;
-        const float2 a = make_float2(s_alpha[j][r], s_alpha[j][r]);
-        const float2 kc = make_float2(s_k[j][r], s_k[j][r]);
-        sa[i] = __ffma2_rn(a, sa[i], __fmul2_rn(kc, ua));
-        sb[i] = __ffma2_rn(a, sb[i], __fmul2_rn(kc, ub));
+        for (int i = 0; i < ROWS; ++i) {
+          const int r = rg + i * RPP;
+          const float2 ka = make_float2(s_ka[j][r], s_ka[j][r]);
+          const float2 qa = make_float2(s_qa[j][r], s_qa[j][r]);
+          ya = __ffma2_rn(ka, sa[i], ya);
+          yb = __ffma2_rn(ka, sb2[i], yb);
+          za = __ffma2_rn(qa, sa[i], za);
+          zb = __ffma2_rn(qa, sb2[i], zb);
+        }
+        s_red[p][0][rg][cg] = make_float4(ya.x, ya.y, yb.x, yb.y);
+        s_red[p][1][rg][cg] = make_float4(za.x, za.y, zb.x, zb.y);
+        __syncthreads();
+        if (tid < DV) {
+          const int c4 = tid >> 2, lane4 = tid & 3;
+          float yy = 0.f, zz = 0.f;
+#pragma unroll 8
+          for (int r = 0; r < RPP; ++r) {
+            yy += reinterpret_cast<const float *>(&s_red[p][0][r][c4])[lane4];
+            zz += reinterpret_cast<const float *>(&s_red[p][1][r][c4])[lane4];
+          }
+          const float uu = s_beta[j] * (s_v[j][tid] - yy);
+          s_u[p][tid] = uu;
+          out[(((size_t)n * T_new + t) * H + h) * DV + tid] = from_f32<TIn>(zz + s_qk[j] * uu);
+        }
+        __syncthreads();
+        const float4 u4 = reinterpret_cast<const float4 *>(s_u[p])[cg];
+        const float2 ua = make_float2(u4.x, u4.y), ub = make_float2(u4.z, u4.w);
+#pragma unroll
+        for (int i = 0; i < ROWS; ++i) {
+          const int r = rg + i * RPP;
+          const float2 a = make_float2(s_alpha[j][r], s_alpha[j][r]);
+          const float2 kc = make_float2(s_k[j][r], s_k[j][r]);
+          sa[i] = __ffma2_rn(a, sa[i], __fmul2_rn(kc, ua));
+          sb2[i] = __ffma2_rn(a, sb2[i], __fmul2_rn(kc, ub));
+        }
+        if (t + 1 == acc)
+#pragma unroll
+          for (int i = 0; i < ROWS; ++i)
+            __stcs(&S4[(rg + i * RPP) * V4 + cg], make_float4(sa[i].x, sa[i].y, sb2[i].x, sb2[i].y));
       }
-      if (t + 1 == acc)
-#pragma unroll
-        for (int i = 0; i < ROWS; ++i)
-          __stcs(&S4[(rg + i * RPP) * V4 + cg], make_float4(sa[i].x, sa[i].y, sb[i].x, sb[i].y));
+      __syncthreads();   // the staged group is overwritten by the next one
     }
-    __syncthreads();   // the staged group is overwritten by the next one
   }
+  cp_async_wait_all();
+  if (aborted) {
+    report(dev_status, KDA_ERR_TIMEOUT);
+    wait_timed(bar, phase, wait_ns);   // the state copy in flight, if any
+  }
+}
+
+static int multi_num_sms() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    v = 148;
+  return v;
 }
 
 template <int DK, int DV, typename TIn>
 static cudaError_t launch_decode_multi_t(const void *q, const void *k, const void *v,
                                          const float *g, const float *beta, float *state,
                                          void *out, const int32_t *accept_len, int T_new,
-                                         int64_t units, int H, cudaStream_t stream) {
+                                         int64_t units, int H, int32_t *dev_status,
+                                         cudaStream_t stream) {
   constexpr int THREADS = 256;
-  decode_multi_kernel<DK, DV, THREADS, TIn><<<(unsigned)units, THREADS, 0, stream>>>(
-      (const TIn *)q, (const TIn *)k, (const TIn *)v, g, beta, state, (TIn *)out, accept_len,
-      T_new, H);
+  if (units <= 0) return cudaSuccess;
+  auto kern = decode_multi_kernel<DK, DV, THREADS, TIn>;
+  const size_t smem = MultiLayout<DK, DV, TIn>::TOTAL;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int64_t slots = 2 * (int64_t)multi_num_sms();
+  const unsigned grid = (unsigned)(units < slots ? units : slots);
+  kern<<<grid, THREADS, smem, stream>>>((const TIn *)q, (const TIn *)k, (const TIn *)v, g, beta,
+                                        state, (TIn *)out, accept_len, T_new, H, units, dev_status,
+                                        2000000000ull);
   return cudaGetLastError();
 }
 
@@ -149,11 +279,12 @@ template <typename TIn>
 static cudaError_t launch_decode_multi_d(int dk, int dv, const void *q, const void *k,
                                          const void *v, const float *g, const float *beta,
                                          float *state, void *out, const int32_t *accept_len,
-                                         int T_new, int64_t units, int H, cudaStream_t stream) {
+                                         int T_new, int64_t units, int H, int32_t *dev_status,
+                                         cudaStream_t stream) {
 #define KDA_DECM(DK_, DV_)                                                                  \
   if (dk == DK_ && dv == DV_)                                                               \
     return launch_decode_multi_t<DK_, DV_, TIn>(q, k, v, g, beta, state, out, accept_len,   \
-                                                T_new, units, H, stream);
+                                                T_new, units, H, dev_status, stream);
   KDA_DECM(32, 32) KDA_DECM(32, 64) KDA_DECM(32, 128)
   KDA_DECM(64, 32) KDA_DECM(64, 64) KDA_DECM(64, 128)
   KDA_DECM(128, 32) KDA_DECM(128, 64) KDA_DECM(128, 128)
@@ -164,12 +295,12 @@ static cudaError_t launch_decode_multi_d(int dk, int dv, const void *q, const vo
 cudaError_t launch_decode_multi(int dtype, int dk, int dv, const void *q, const void *k,
                                 const void *v, const float *g, const float *beta, float *state,
                                 void *out, const int32_t *accept_len, int T_new, int64_t units,
-                                int H, cudaStream_t stream) {
+                                int H, int32_t *dev_status, cudaStream_t stream) {
   if (dtype == KDA_DTYPE_BF16)
     return launch_decode_multi_d<__nv_bfloat16>(dk, dv, q, k, v, g, beta, state, out,
-                                                accept_len, T_new, units, H, stream);
+                                                accept_len, T_new, units, H, dev_status, stream);
   return launch_decode_multi_d<float>(dk, dv, q, k, v, g, beta, state, out, accept_len, T_new,
-                                      units, H, stream);
+                                      units, H, dev_status, stream);
 }
 
 }  // namespace kda

@@ -22,7 +22,7 @@ EXPORTED = ("kda_prefill", "kda_prefill_ws", "kda_prefill_at", "kda_decode", "kd
             "kda_release_workspace_pool", "kda_prefill_path", "kda_selftest_bounded_wait",
             "kda_last_cuda_error", "kda_status_string", "kda_version", "kda_backward",
             "kda_backward_workspace_bytes", "kda_affine_rows", "kda_affine_state",
-            "kda_last_prefill_path", "kda_set_workspace_pool_cap")
+            "kda_last_prefill_path", "kda_set_workspace_pool_cap", "kda_last_backward_path")
 
 # Largest workspace the binding allocates for the two-pass prefill; longer
 # inputs run in windows of chunks.
@@ -93,6 +93,7 @@ def load(path: str | None = None):
     lib.kda_prefill_path.argtypes = [SP]
     lib.kda_prefill_path.restype = ctypes.c_int
     lib.kda_last_prefill_path.restype = ctypes.c_int
+    lib.kda_last_backward_path.restype = ctypes.c_int
     lib.kda_set_workspace_pool_cap.argtypes = [ctypes.c_size_t]
     lib.kda_set_workspace_pool_cap.restype = ctypes.c_int
     lib.kda_selftest_bounded_wait.argtypes = [P, I64, P]
@@ -144,6 +145,12 @@ def kda_prefill_path(shape: KdaShape) -> int:
 def kda_last_prefill_path() -> int:
     """Kernel the last prefill call on this thread launched (2, 1, 0; -1 none)."""
     return int(load().kda_last_prefill_path())
+
+
+def kda_last_backward_path() -> int:
+    """Backward kernel the last kda_backward on this thread launched (1 chunked
+    tensor-core, 0 SIMT; -1 none)."""
+    return int(load().kda_last_backward_path())
 
 
 def kda_set_workspace_pool_cap(nbytes: int) -> None:

@@ -13,8 +13,24 @@ pytestmark = pytest.mark.gpu
 NAMES = ("dq", "dk", "dv", "dg", "dbeta", "d_init")
 
 
-def run_both(lengths, H, Dk, Dv, dtype, seed, use_init=True, use_dfin=True, tol=1e-4):
+def chunked_path(dtype, Dk, Dv):
+    """BF16 with D_k = D_v = 128 runs the chunked tensor-core backward."""
+    return dtype == torch.bfloat16 and Dk == 128 and Dv == 128
+
+
+def bound(dtype, Dk, Dv):
+    """FP32 SIMT: the FP32 bound for either input dtype (it reads the exact bits
+    the oracle reads).  Chunked tensor-core path: the BF16 bound of the forward,
+    since its products take BF16 operands with FP32 accumulation."""
+    return 1e-2 if chunked_path(dtype, Dk, Dv) else 1e-4
+
+
+def run_both(lengths, H, Dk, Dv, dtype, seed, use_init=True, use_dfin=True, tol=None,
+             mutate=None):
     d = make_case(lengths, H, Dk, Dv, dtype, seed=seed, state_std=0.1)
+    if mutate is not None:
+        mutate(d)
+    tol = tol or bound(dtype, Dk, Dv)
     dd = to_device(d)
     rng = np.random.default_rng(seed + 100)
     T = sum(lengths)
@@ -25,6 +41,8 @@ def run_both(lengths, H, Dk, Dv, dtype, seed, use_init=True, use_dfin=True, tol=
                            d_out.cuda(), init_state=init,
                            d_final=d_fin.cuda() if use_dfin else None)
     torch.cuda.synchronize()
+    if sum(lengths) > 0:
+        assert kda.kda_last_backward_path() == (1 if chunked_path(dtype, Dk, Dv) else 0)
     ref = oracle.backward(d["q"], d["k"], d["v"], d["g"], d["beta"], d["cu_seqlens"], d_out,
                           init_state=d["init_state"] if use_init else None,
                           d_final=d_fin if use_dfin else None)
@@ -40,10 +58,44 @@ def test_backward_matches_oracle(dtype, dims):
     """Ragged sequences around the 4-token replay blocks (last blocks of 1, 2, 3 and 4
     tokens), nonzero initial state and final-state gradient.  D_v of 64 and 128 run
     2 and 4 column slices whose row-sum parts are added by the second kernel.  The
-    GPU reads the same bits as the oracle, so the bound is the FP32 one for both
-    input dtypes."""
+    SIMT kernel reads the same bits as the oracle, so its bound is the FP32 one for
+    both input dtypes; BF16 at D = 128 runs the chunked tensor-core kernels."""
     Dk, Dv = dims
     run_both([1, 2, 15, 16, 17, 42], 2, Dk, Dv, dtype, seed=5)
+
+
+@pytest.mark.parametrize("lengths", [[1, 63, 64, 65], [130, 200, 7], [256]],
+                         ids=["around_one_chunk", "ragged_multi_chunk", "four_chunks"])
+def test_chunked_backward_ragged(lengths):
+    """The chunked tensor-core backward on ragged sequences: partial last chunks
+    (identity-token padding), several chunks per sequence (the chain carries dS
+    across chunk ends), three heads."""
+    run_both(lengths, 3, 128, 128, torch.bfloat16, seed=len(lengths) + lengths[0])
+
+
+@pytest.mark.parametrize("case", ["g_floor", "g_zero", "beta_zero", "beta_one",
+                                  "strong_decay_16_32", "alternate_8"])
+def test_chunked_backward_gate_extremes(case):
+    """Gates at the floor (g = -5: the cumulative decay spans e^-320 inside a chunk,
+    so every gated product needs its factored form), no decay, beta at 0 and 1,
+    and strong decay confined to parts of each chunk."""
+    def mutate(d):
+        T = d["g"].shape[0]
+        pos = torch.cat([torch.arange(n) for n in d["lengths"]]) % 64
+        if case == "g_floor":
+            d["g"].fill_(-5.0)
+        elif case == "g_zero":
+            d["g"].zero_()
+        elif case == "beta_zero":
+            d["beta"].zero_()
+        elif case == "beta_one":
+            d["beta"].fill_(1.0)
+        else:
+            mask = ((pos >= 16) & (pos < 32)) if case == "strong_decay_16_32" else ((pos // 8) % 2 == 0)
+            d["g"] = torch.where(mask[:, None, None], torch.full_like(d["g"], -5.0),
+                                 torch.zeros_like(d["g"])).contiguous()
+        assert d["g"].shape[0] == T
+    run_both([150, 64], 2, 128, 128, torch.bfloat16, seed=31, mutate=mutate)
 
 
 def test_backward_without_init_or_final_gradient():
@@ -58,9 +110,9 @@ def test_backward_empty_sequence_passes_final_gradient_through():
 def test_backward_bench_shape_sampled_heads():
     """The bench's backward workload (4 sequences x 1024 tokens, H = 32, D = 128,
     BF16 q/k/v, FP32 state N(0, 0.02^2), N(0, 1) upstream gradients), run whole
-    on the GPU in the launch configuration the bench times (4 column slices per
-    head plus the slice-sum kernel).  Three heads are recomputed by the oracle
-    and compared in full."""
+    on the GPU in the launch configuration the bench times (the chunked
+    tensor-core backward).  Three heads are recomputed by the oracle and
+    compared in full."""
     lengths, H, D = [1024] * 4, 32, 128
     d = make_case(lengths, H, D, D, torch.bfloat16, seed=11, state_std=0.02)
     dd = to_device(d)
@@ -71,6 +123,7 @@ def test_backward_bench_shape_sampled_heads():
     got = kda.kda_backward(dd["q"], dd["k"], dd["v"], dd["g"], dd["beta"], dd["cu_dev"],
                            d_out.cuda(), init_state=dd["init_state"], d_final=d_fin.cuda())
     torch.cuda.synchronize()
+    assert kda.kda_last_backward_path() == 1
     got = [x.cpu() for x in got]
     for h in (0, 13, 31):
         hs = slice(h, h + 1)
@@ -79,4 +132,5 @@ def test_backward_bench_shape_sampled_heads():
                               init_state=d["init_state"][:, hs], d_final=d_fin[:, hs])
         for name, x, r in zip(NAMES, got, ref):
             e = rel_l2(x[:, hs], r)
-            assert e <= 1e-4, f"head {h} {name}: rel-L2 {e:.3e}"
+            print(f"backward, head {h}, {name}: rel-L2 {e:.3e}")
+            assert e <= 1e-2, f"head {h} {name}: rel-L2 {e:.3e}"
