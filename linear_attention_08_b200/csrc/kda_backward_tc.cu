@@ -369,6 +369,11 @@ struct BItemLayout {
   static_assert(TOTAL + 1024 <= 232448, "shared memory");
 };
 
+// FP32 [64 tokens][128 channels] arrays read with one token per lane: the
+// channel index is XOR-ed with the token's low five bits, so a warp reading
+// one channel of 32 tokens touches 32 banks.
+__device__ __forceinline__ int sw(int r, int ch) { return r * 128 + (ch ^ (r & 31)); }
+
 __device__ __forceinline__ void st_chunk_s(uint8_t *dst, const float *x) {
   *reinterpret_cast<uint4 *>(dst) = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
                                                tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
@@ -588,11 +593,16 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         st4(sp + Lay::KT + tc::tile_offset(64, r, cq) + sub, t);
       }
     }
-    // Gam stays for the final epilogue, in place of g.
+    // Gam stays for the final epilogue, in place of g (every thread has read
+    // its g rows before the first barrier of the prep).
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      *reinterpret_cast<float4 *>(sp + Lay::GST + (8 * warp + i) * 512 + lane * 16) =
-          make_float4(gm[i][0].x, gm[i][0].y, gm[i][1].x, gm[i][1].y);
+    for (int i = 0; i < 8; ++i) {
+      const int r = 8 * warp + i;
+      s_gam[sw(r, 4 * lane)] = gm[i][0].x;
+      s_gam[sw(r, 4 * lane + 1)] = gm[i][0].y;
+      s_gam[sw(r, 4 * lane + 2)] = gm[i][1].x;
+      s_gam[sw(r, 4 * lane + 3)] = gm[i][1].y;
+    }
     tc::fence_smem_to_async();
     __syncthreads();
   }
@@ -739,19 +749,22 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       const float *dsr = dSsrc + (size_t)c * kD + 64 * h2;
       float dot = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < 64; jj += 8) {
-        float xs[8], xd[8];
+      for (int half = 0; half < 2; ++half) {   // 32 columns: all loads first, then the stores
+        float xs[32], xd[32];
 #pragma unroll
-        for (int e = 0; e < 8; e += 4) {
-          const float4 u4 = s0r ? *reinterpret_cast<const float4 *>(s0r + jj + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 w4 = *reinterpret_cast<const float4 *>(dsr + jj + e);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 u4 = s0r ? *reinterpret_cast<const float4 *>(s0r + 32 * half + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+          const float4 w4 = *reinterpret_cast<const float4 *>(dsr + 32 * half + e);
           xs[e] = u4.x; xs[e + 1] = u4.y; xs[e + 2] = u4.z; xs[e + 3] = u4.w;
           xd[e] = w4.x; xd[e + 1] = w4.y; xd[e + 2] = w4.z; xd[e + 3] = w4.w;
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dot = fmaf(xs[e], xd[e], dot);
-        st_chunk_s(sp + Lay::S0T + tc::tile_offset(128, c, (64 * h2 + jj) >> 3), xs);
-        st_chunk_s(sp + Lay::DST + tc::tile_offset(128, c, (64 * h2 + jj) >> 3), xd);
+        for (int e = 0; e < 32; ++e) dot = fmaf(xs[e], xd[e], dot);
+#pragma unroll
+        for (int jj = 0; jj < 32; jj += 8) {
+          st_chunk_s(sp + Lay::S0T + tc::tile_offset(128, c, (64 * h2 + 32 * half + jj) >> 3), xs + jj);
+          st_chunk_s(sp + Lay::DST + tc::tile_offset(128, c, (64 * h2 + 32 * half + jj) >> 3), xd + jj);
+        }
       }
       dot += __shfl_xor_sync(0xffffffffu, dot, 1);
       if (h2 == 0) s_dd[c] = dot;
@@ -918,26 +931,27 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       tc::tmem_ld32(tl + 256 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ak + 32));
       tc::tmem_wait_ld();
       const size_t off = base_row + (size_t)r * row_stride + hw * 64;
+      uint4 qraw[8], kraw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        qraw[u] = in ? *reinterpret_cast<const uint4 *>(qb + off + 8 * u) : make_uint4(0, 0, 0, 0);
+        kraw[u] = in ? *reinterpret_cast<const uint4 *>(kb + off + 8 * u) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
       for (int cc = 0; cc < 64; cc += 8) {
         float qv[8], kv[8], dq8[8];
-        if (in) {
-          unpack8(*reinterpret_cast<const uint4 *>(qb + off + cc), qv);
-          unpack8(*reinterpret_cast<const uint4 *>(kb + off + cc), kv);
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) qv[e] = kv[e] = 0.f;
-        }
+        unpack8(qraw[cc >> 3], qv);
+        unpack8(kraw[cc >> 3], kv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int ch = hw * 64 + cc + e;
-          const float gam = s_gam[r * 128 + ch], g63 = s_gam[63 * 128 + ch];
+          const float gam = s_gam[sw(r, ch)], g63 = s_gam[sw(63, ch)];
           const float dqa = __expf(gam) * aq[cc + e];
           const float dkm = __expf(g63 - gam) * ak[cc + e];
           dq8[e] = dqa;
-          pkm[r * 128 + ch] = dkm;
-          pkk[r * 128 + ch] = kv[e] * dkm;
-          pdg[r * 128 + ch] = qv[e] * dqa - kv[e] * dkm;
+          pkm[sw(r, ch)] = dkm;
+          pkk[sw(r, ch)] = kv[e] * dkm;
+          pdg[sw(r, ch)] = qv[e] * dqa - kv[e] * dkm;
         }
         if (in) {
           float *dst = a.dq + off + cc;
@@ -955,19 +969,20 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ak + 32));
       tc::tmem_wait_ld();
       const size_t off = base_row + (size_t)r * row_stride + hw * 64;
+      uint4 kraw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        kraw[u] = in ? *reinterpret_cast<const uint4 *>(kb + off + 8 * u) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int cc = 0; cc < 64; cc += 8) {
         float kv[8], dk8[8];
-        if (in) unpack8(*reinterpret_cast<const uint4 *>(kb + off + cc), kv);
-        else
-#pragma unroll
-          for (int e = 0; e < 8; ++e) kv[e] = 0.f;
+        unpack8(kraw[cc >> 3], kv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int ch = hw * 64 + cc + e;
-          const float dkp = __expf(s_gam[r * 128 + ch]) * ak[cc + e];
-          dk8[e] = dkp + pkm[r * 128 + ch];
-          pdg[r * 128 + ch] += kv[e] * dkp;
+          const float dkp = __expf(s_gam[sw(r, ch)]) * ak[cc + e];
+          dk8[e] = dkp + pkm[sw(r, ch)];
+          pdg[sw(r, ch)] += kv[e] * dkp;
         }
         if (in) {
           float *dst = a.dk + off + cc;
@@ -979,10 +994,10 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     __syncthreads();
     if (!aborted && tid < 128) {   // dg = reverse cumulative sum of dGam (+ the Gam_63 terms)
       const int ch = tid;
-      float suffix = __expf(s_gam[63 * 128 + ch]) * s_dd[ch];
-      for (int r = 0; r < 64; ++r) suffix += pkk[r * 128 + ch];
+      float suffix = __expf(s_gam[sw(63, ch)]) * s_dd[ch];
+      for (int r = 0; r < 64; ++r) suffix += pkk[sw(r, ch)];
       for (int r = 63; r >= 0; --r) {
-        suffix += pdg[r * 128 + ch];
+        suffix += pdg[sw(r, ch)];
         if (r < L) a.dg[base_row + (size_t)r * row_stride + ch] = suffix;
       }
     }
@@ -1055,39 +1070,37 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     // 64 + i (i in the first half, second-half reference): dP_ri for r in the
     // second half; rows 96..127 zero.
     if (!aborted) {
-      {
+      {   // all loads first, then the stores
         const int r = tid >> 2, kq = (tid & 3) * 24;   // 24 columns of kappa each
-        float x8[8];
+        float xv[24];
 #pragma unroll
-        for (int cc = 0; cc < 3; ++cc) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int kap = kq + 8 * cc + e;
-            const int i = r < 32 ? kap : kap - 32;
-            const bool ok = (r < 32 ? kap < 32 : kap >= 32) && i <= r;
-            x8[e] = ok ? dP[r * 64 + i] : 0.f;
-          }
-          st_chunk_s(sp + Lay::XA + tc::tile_offset(128, 64 + r, (kq >> 3) + cc), x8);
+        for (int e = 0; e < 24; ++e) {
+          const int kap = kq + e;
+          const int i = r < 32 ? kap : kap - 32;
+          const bool ok = (r < 32 ? kap < 32 : kap >= 32) && i <= r;
+          xv[e] = ok ? dP[r * 64 + i] : 0.f;
         }
+#pragma unroll
+        for (int cc = 0; cc < 3; ++cc)
+          st_chunk_s(sp + Lay::XA + tc::tile_offset(128, 64 + r, (kq >> 3) + cc), xv + 8 * cc);
       }
       {
         const int m = tid >> 1, rh = (tid & 1) * 32;   // YA row m, P columns r = rh..rh+31
-        float x8[8];
+        float xv[32];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int r = rh + 8 * cc + e;
-            float val = 0.f;
-            if (m < 64) {
-              if ((m >> 5) == (r >> 5) && r >= m) val = dP[r * 64 + m];
-            } else if (m < 96) {
-              if (r >= 32) val = dP[r * 64 + (m - 64)];
-            }
-            x8[e] = val;
+        for (int e = 0; e < 32; ++e) {
+          const int r = rh + e;
+          float val = 0.f;
+          if (m < 64) {
+            if ((m >> 5) == (r >> 5) && r >= m) val = dP[r * 64 + m];
+          } else if (m < 96) {
+            if (r >= 32) val = dP[r * 64 + (m - 64)];
           }
-          st_chunk_s(sp + Lay::YA + tc::tile_offset(128, m, 8 + (rh >> 3) + cc), x8);
+          xv[e] = val;
         }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+          st_chunk_s(sp + Lay::YA + tc::tile_offset(128, m, 8 + (rh >> 3) + cc), xv + 8 * cc);
       }
     }
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
@@ -1119,18 +1132,18 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) st_chunk_s(sp + Lay::XA + tc::tile_offset(128, rho, (kz >> 3) + cc), z);
         }
-      } else {        // column sig of dA (from the transposed product): dG^T into YA
-        const int sig = 32 * (qd - 2) + lane;
-        float x[32];
+        // Column sig = rho of dA, from the transposed product (its A operand has
+        // 64 rows, so it too lands in TMEM lanes 0..63): dG^T into YA.
+        const int sig = rho;
         tc::tmem_ld32(tl + 384 + hw * 32, x);
         tc::tmem_wait_ld();
-        float vals[32], z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const int rho = 32 * hw + e;
-          vals[e] = rho > sig ? s_beta[rho] * (-x[e]) : 0.f;
+          const int r2 = 32 * hw + e;
+          vals[e] = r2 > sig ? s_beta[r2] * (-x[e]) : 0.f;
         }
-        const bool cross = sig < 32 && hw == 1;   // second-half rho against a first-half sig
+        const bool cross = sig < 32 && hw == 1;   // second-half rows against a first-half sig
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           st_chunk_s(sp + Lay::YA + tc::tile_offset(128, sig, hw * 4 + cc), cross ? z : vals + 8 * cc);
@@ -1159,44 +1172,53 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     phase ^= 1;
     tc::fence_after_sync();
     // ---- final epilogue: the rest of dq, dk, dGam; dbeta ----
-    float *qdg = reinterpret_cast<float *>(sp + Lay::QDG);   // q dq, then dGam
+    // dGam takes each gated pair's two sides from the very BF16 operands the
+    // products used (Gram A rows for the sides where Gam enters with a plus
+    // sign, Gram B rows for the others), so that the pair's terms, which the
+    // reverse cumulative sum below sets against each other, cancel to FP32
+    // accumulation precision.
+    float *qdg = reinterpret_cast<float *>(sp + Lay::QDG);   // dGam
     float *kmc = reinterpret_cast<float *>(sp + Lay::KMC);   // dk from first-half keys, second-half reference
-    const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(a.q);
-    const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(a.k);
+    auto tile_val = [&](uint32_t tile, int rows, int row, int ch) {
+      return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+          sp + tile + tc::tile_offset(rows, row, ch >> 3) + 2 * (ch & 7)));
+    };
+    float *dqp = a.dq, *dkp_ = a.dk;
     if (!aborted && qd >= 2) {
       const int r = 32 * (qd - 2) + lane;
       const bool in = r < L;
-      float xq[64], yc[64];
-      tc::tmem_ld32(tl + 0 + hw * 64, *reinterpret_cast<float(*)[32]>(xq));
-      tc::tmem_ld32(tl + 0 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(xq + 32));
-      tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(yc));
-      tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(yc + 32));
-      tc::tmem_wait_ld();
-      const size_t off = base_row + (size_t)r * row_stride + hw * 64;
       const int ref = r < 32 ? 15 : 47;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const int c0 = hw * 64 + 32 * half;
+        float xq[32], yc[32];
+        tc::tmem_ld32(tl + 0 + c0, xq);
+        tc::tmem_ld32(tl + 128 + c0, yc);
+        tc::tmem_wait_ld();
+        const size_t off = base_row + (size_t)r * row_stride + c0;
+        float4 old[8];
+        if (in)
 #pragma unroll
-      for (int cc = 0; cc < 64; cc += 8) {
-        float qv[8], add[8];
-        if (in) unpack8(*reinterpret_cast<const uint4 *>(qb + off + cc), qv);
-        else
+          for (int e = 0; e < 8; ++e) old[e] = *reinterpret_cast<const float4 *>(dqp + off + 4 * e);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) qv[e] = 0.f;
+        for (int e4 = 0; e4 < 8; ++e4) {
+          float add[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int ch = hw * 64 + cc + e;
-          const float gam = s_gam[r * 128 + ch];
-          const float dqb = __expf(gam - s_gam[ref * 128 + ch]) * xq[cc + e];
-          add[e] = dqb;
-          qdg[r * 128 + ch] = qv[e] * dqb;
-          if (r < 32) kmc[r * 128 + ch] = __expf(s_gam[47 * 128 + ch] - gam) * yc[cc + e];
-        }
-        if (in) {
-          float *dst = a.dq + off + cc;
-          float4 o0 = *reinterpret_cast<float4 *>(dst), o1 = *reinterpret_cast<float4 *>(dst + 4);
-          o0.x += add[0]; o0.y += add[1]; o0.z += add[2]; o0.w += add[3];
-          o1.x += add[4]; o1.y += add[5]; o1.z += add[6]; o1.w += add[7];
-          *reinterpret_cast<float4 *>(dst) = o0;
-          *reinterpret_cast<float4 *>(dst + 4) = o1;
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * e4 + e, ch = c0 + c;
+            const float gam = s_gam[sw(r, ch)];
+            add[e] = __expf(gam - s_gam[sw(ref, ch)]) * xq[c];
+            float dgm = tile_val(Lay::GA, 128, 64 + r, ch) * xq[c];
+            if (r < 32) {
+              dgm -= tile_val(Lay::GB, 96, 32 + r, ch) * yc[c];
+              kmc[sw(r, ch)] = __expf(s_gam[sw(47, ch)] - gam) * yc[c];
+            }
+            qdg[sw(r, ch)] = dgm;
+          }
+          if (in) {
+            old[e4].x += add[0]; old[e4].y += add[1]; old[e4].z += add[2]; old[e4].w += add[3];
+            *reinterpret_cast<float4 *>(dqp + off + 4 * e4) = old[e4];
+          }
         }
       }
     }
@@ -1204,47 +1226,59 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     if (!aborted && qd < 2) {
       const int t = 32 * qd + lane;
       const bool in = t < L;
-      float xk[64], yo[64];
-      tc::tmem_ld32(tl + 0 + hw * 64, *reinterpret_cast<float(*)[32]>(xk));
-      tc::tmem_ld32(tl + 0 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(xk + 32));
-      tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(yo));
-      tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(yo + 32));
-      tc::tmem_wait_ld();
-      const size_t off = base_row + (size_t)t * row_stride + hw * 64;
       const int ref = t < 32 ? 15 : 47;
+      const int gbrow = t < 32 ? t : 32 + t;
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const int c0 = hw * 64 + 32 * half;
+        float xk[32], yo[32];
+        tc::tmem_ld32(tl + 0 + c0, xk);
+        tc::tmem_ld32(tl + 128 + c0, yo);
+        tc::tmem_wait_ld();
+        const size_t off = base_row + (size_t)t * row_stride + c0;
+        float4 old[8];
+        if (in)
 #pragma unroll
-      for (int cc = 0; cc < 64; cc += 8) {
-        float kv[8], add[8];
-        if (in) unpack8(*reinterpret_cast<const uint4 *>(kb + off + cc), kv);
-        else
+          for (int e = 0; e < 8; ++e) old[e] = *reinterpret_cast<const float4 *>(dkp_ + off + 4 * e);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) kv[e] = 0.f;
+        for (int e4 = 0; e4 < 8; ++e4) {
+          float add[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int ch = hw * 64 + cc + e;
-          const float dlt = s_gam[t * 128 + ch] - s_gam[ref * 128 + ch];
-          const float dkp = __expf(dlt) * xk[cc + e];
-          const float dkm = __expf(-dlt) * yo[cc + e] + (t < 32 ? kmc[t * 128 + ch] : 0.f);
-          add[e] = dkp + dkm;
-          qdg[t * 128 + ch] += kv[e] * (dkp - dkm);
-        }
-        if (in) {
-          float *dst = a.dk + off + cc;
-          float4 o0 = *reinterpret_cast<float4 *>(dst), o1 = *reinterpret_cast<float4 *>(dst + 4);
-          o0.x += add[0]; o0.y += add[1]; o0.z += add[2]; o0.w += add[3];
-          o1.x += add[4]; o1.y += add[5]; o1.z += add[6]; o1.w += add[7];
-          *reinterpret_cast<float4 *>(dst) = o0;
-          *reinterpret_cast<float4 *>(dst + 4) = o1;
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * e4 + e, ch = c0 + c;
+            const float gam = s_gam[sw(t, ch)];
+            const float dlt = gam - s_gam[sw(ref, ch)];
+            float dkm = __expf(-dlt) * yo[c];
+            if (t < 32) dkm += kmc[sw(t, ch)];
+            add[e] = __expf(dlt) * xk[c] + dkm;
+            qdg[sw(t, ch)] += tile_val(Lay::GA, 128, t, ch) * xk[c] - tile_val(Lay::GB, 96, gbrow, ch) * yo[c];
+          }
+          if (in) {
+            old[e4].x += add[0]; old[e4].y += add[1]; old[e4].z += add[2]; old[e4].w += add[3];
+            *reinterpret_cast<float4 *>(dkp_ + off + 4 * e4) = old[e4];
+          }
         }
       }
     }
     __syncthreads();
     if (!aborted && tid < 128) {
       const int ch = tid;
+      float *dgp = a.dg;
       float suffix = 0.f;
-      for (int r = 63; r >= 0; --r) {
-        suffix += qdg[r * 128 + ch];
-        if (r < L) a.dg[base_row + (size_t)r * row_stride + ch] += suffix;
+#pragma unroll 1
+      for (int blk = 3; blk >= 0; --blk) {   // 16 rows at a time: their loads issue together
+        float prev[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int r = 16 * blk + u;
+          prev[u] = r < L ? dgp[base_row + (size_t)r * row_stride + ch] : 0.f;
+        }
+#pragma unroll
+        for (int u = 15; u >= 0; --u) {
+          const int r = 16 * blk + u;
+          suffix += qdg[sw(r, ch)];
+          if (r < L) dgp[base_row + (size_t)r * row_stride + ch] = prev[u] + suffix;
+        }
       }
     }
     if (!aborted && tid < L) a.dbeta[(size_t)(t0 + tid) * H + h] = s_db[tid];

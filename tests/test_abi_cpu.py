@@ -256,3 +256,24 @@ def test_backward_workspace_and_validation():
     # head size outside {32, 64, 128}
     s_bad = kda.make_shape(2, 1000, 4, 96, 64, 0, kda.KDA_DTYPE_BF16)
     assert lib.kda_backward(*args, ws, need, ctypes.byref(s_bad), None) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_chunked_backward_workspace():
+    """BF16, D_k = D_v = 128: the chunked tensor-core backward's workspace holds, per
+    (64-token chunk, head) of an upper bound of the chunk count, the forward's
+    74,240-byte packet, dS at the chunk's end (64 KiB), the [-dU; dO] tile (32 KiB)
+    and dT, dP (32 KiB); per full chunk the stored forward state (64 KiB); the
+    forward's output (BF16); two prefix tables."""
+    lib = kda.load()
+    al = lambda x: (x + 255) // 256 * 256
+    for lengths, H in (([1024] * 4, 32), ([5, 0, 130, 64], 3)):
+        N, T = len(lengths), sum(lengths)
+        s = kda.make_shape(N, T, H, 128, 128, 0, kda.KDA_DTYPE_BF16)
+        P = H * ((T + 63 * N) // 64)
+        assert P >= H * sum(-(-L // 64) for L in lengths)
+        want = (al(P * 74240 + 256) + al((T // 64) * H * 65536) + al(P * 65536) + al(P * 32768)
+                + al(P * 32768) + al(T * H * 256) + 2 * al((N + 1) * 8) + 256)
+        assert lib.kda_backward_workspace_bytes(ctypes.byref(s)) == want
+    # FP32 inputs keep the SIMT kernel's workspace
+    s = kda.make_shape(4, 4096, 32, 128, 128, 0, kda.KDA_DTYPE_F32)
+    assert lib.kda_backward_workspace_bytes(ctypes.byref(s)) == (4096 + 12) // 4 * 32 * 128 * 128 * 4 + 3 * 4096 * 32 * 385 * 4

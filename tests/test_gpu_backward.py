@@ -48,8 +48,42 @@ def run_both(lengths, H, Dk, Dv, dtype, seed, use_init=True, use_dfin=True, tol=
                           d_final=d_fin if use_dfin else None)
     errs = {n: rel_l2(x, r) for n, x, r in zip(NAMES, got, ref)}
     for n, e in errs.items():
+        if n == "dg" and chunked_path(dtype, Dk, Dv):
+            check_dg(got[3], ref, d, lengths)
+            continue
         assert e <= tol, f"{n}: rel-L2 {e:.3e} > {tol:.0e} ({errs})"
     return errs
+
+
+def dg_term_scale(ref, d, lengths):
+    """dg is the reverse cumulative sum, inside each 64-token chunk, of
+    dGam = q * dq + k * (dk_plus - dk_minus): products that largely cancel.
+    This returns that sum taken over the magnitudes |q * dq| + |k * dk|
+    instead (FP64, from the oracle's dq and dk), the scale against which a
+    cancelling sum's rounding error is measured."""
+    q = d["q"].double().numpy()
+    k = d["k"].double().numpy()
+    mag = np.abs(q * ref[0]) + np.abs(k * ref[1])
+    out = np.zeros_like(mag)
+    cu = d["cu_seqlens"]
+    for a, b in zip(cu[:-1], cu[1:]):
+        for c0 in range(a, b, 64):
+            blk = mag[c0:min(c0 + 64, b)]
+            out[c0:c0 + blk.shape[0]] = np.cumsum(blk[::-1], axis=0)[::-1]
+    return out
+
+
+def check_dg(dg, ref, d, lengths):
+    """dg on the chunked tensor-core path: rel-L2 1e-2 of dg, plus 2e-5 (a
+    hundredth of the BF16 unit roundoff 2^-9) of the scale of the terms it
+    is summed from.  For ordinary gates that scale is about 60x |dg| and the
+    second part adds about 1e-3; at the decay floor (g = -5 everywhere) dg is
+    about 5000x smaller than its terms, and a bound on dg alone would ask the
+    BF16 products for more digits than they carry."""
+    err = float(np.linalg.norm(dg.detach().double().cpu().numpy() - ref[3]))
+    scale = float(np.linalg.norm(dg_term_scale(ref, d, lengths)))
+    bound = 1e-2 * float(np.linalg.norm(ref[3])) + 2e-5 * scale
+    assert err <= bound, f"dg: |err| {err:.3e} > {bound:.3e} (|dg| {np.linalg.norm(ref[3]):.3e}, term scale {scale:.3e})"
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
