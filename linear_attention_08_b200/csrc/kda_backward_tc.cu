@@ -82,35 +82,73 @@ __device__ __forceinline__ int64_t seq_chunks(const int32_t *cu, int n) {
 // 1. The backward chain
 // ---------------------------------------------------------------------------
 struct BChainLayout {
-  static constexpr uint32_t S_T = 0;         // [128 ch][128 v] bf16 dS, MN-major B
-  static constexpr uint32_t BT = 32768;      // [128 tok][128 v] bf16: rows 0..63 -dU, 64..127 dO
-  static constexpr uint32_t DOF = 65536;     // float [64][128] dO staging (TMA)
-  static constexpr uint32_t STAGE0 = 98304;  // packet stages
+  static constexpr uint32_t S_T = 0;         // [128 ch][128 v] bf16 dS, MN-major B (stored as dS_L)
+  static constexpr uint32_t NDU = 32768;     // [64 tok][128 v] bf16 -dU, MN-major B (stored)
+  static constexpr uint32_t STAGE0 = 49152;  // stages: a chunk's packet and its dO tile
   // Inside a stage.  Khat and P come first: the M = 128 MMAs that read them as
   // 64-row operands also read the 8 KB after each (rows 64..127 of the
-  // product, never used), which must stay inside the allocation.
+  // product, never used), which must stay inside the stage.
   static constexpr uint32_t SKH = 0;         // [64][128] Khat
   static constexpr uint32_t SP = 16384;      // [64][64] P
   static constexpr uint32_t SD = 24576;      // float[128] d
   static constexpr uint32_t SWQ = 25600;     // [128][128] [W; Qtilde]
-  static constexpr uint32_t STAGE = SWQ + 32768;
+  static constexpr uint32_t SDO = SWQ + 32768;   // [64 tok][128 v] bf16 dO, MN-major B
+  static constexpr uint32_t STAGE = SDO + 16384;
   static constexpr int NST = 2;
-  static constexpr uint32_t FULL = STAGE0 + NST * STAGE;   // [NST] packet landed
-  static constexpr uint32_t DOBAR = FULL + 8 * NST;        // dO landed
-  static constexpr uint32_t BAR1 = DOBAR + 8;              // dU product done
+  static constexpr uint32_t FULL = STAGE0 + NST * STAGE;   // [NST] stage landed
+  static constexpr uint32_t BAR1 = FULL + 8 * NST;         // dU product done
   static constexpr uint32_t BAR2 = BAR1 + 8;               // dS product done
   static constexpr uint32_t SCAL = BAR2 + 8;               // int64 first packet of the unit
   static constexpr uint32_t TMEM_SLOT = SCAL + 8;
   static constexpr uint32_t TOTAL = TMEM_SLOT + 8;
+  static constexpr uint32_t TX = 16384 + 8704 + 32768 + 16384;   // bytes landing per stage
   static constexpr uint32_t ACC1 = 0, ACC2 = 128, SCOL = 256;   // TMEM columns
   static_assert(SKH + 16384 + 8192 <= STAGE && SP + 8192 + 8192 <= STAGE, "junk rows leave the stage");
-  static_assert(STAGE % 1024 == 0 && SWQ % 1024 == 0, "tile alignment");
+  static_assert(STAGE % 1024 == 0 && SWQ % 1024 == 0 && SDO % 1024 == 0, "tile alignment");
+  static_assert(TOTAL + 1024 <= 232448, "shared memory");
 };
 
+// The chunk's dO as the BF16 operand tile [64 tokens][128 value columns]
+// (rows past the sequence's end zero), for every packet: one CTA per packet.
+__global__ void __launch_bounds__(kThreads)
+bwd_dout_tiles_kernel(const float *__restrict__ dout, const int32_t *__restrict__ cu,
+                      const int64_t *__restrict__ pref, int N, int H, uint8_t *__restrict__ tiles) {
+  const int64_t total = pref[N] * H;
+  const int64_t p = blockIdx.x;
+  if (p >= total) return;
+  int lo = 0, hi = N - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (pref[mid] * H <= p) lo = mid; else hi = mid - 1;
+  }
+  const int n = lo;
+  const int64_t nch = pref[n + 1] - pref[n];
+  const int64_t rem = p - pref[n] * H;
+  const int h = (int)(rem / nch);
+  const int64_t j = rem - (int64_t)h * nch;
+  const int64_t t0 = (int64_t)cu[n] + kC * j;
+  const int64_t T_n = (int64_t)cu[n + 1] - cu[n];
+  const int L = (int)(T_n - kC * j < kC ? T_n - kC * j : kC);
+  const int tid = threadIdx.x, r = tid >> 2, c0 = (tid & 3) * 32;
+  float x[32];
+  const float *src = dout + ((size_t)(t0 + r) * H + h) * kD + c0;
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    const float4 v4 = r < L ? *reinterpret_cast<const float4 *>(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    x[e] = v4.x; x[e + 1] = v4.y; x[e + 2] = v4.z; x[e + 3] = v4.w;
+  }
+  uint8_t *dst = tiles + (size_t)p * 16384;
+#pragma unroll
+  for (int e = 0; e < 32; e += 8)
+    *reinterpret_cast<uint4 *>(dst + tc::tile_offset(64, r, (c0 + e) >> 3)) =
+        make_uint4(tc::pack_bf16(x[e], x[e + 1]), tc::pack_bf16(x[e + 2], x[e + 3]),
+                   tc::pack_bf16(x[e + 4], x[e + 5]), tc::pack_bf16(x[e + 6], x[e + 7]));
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_chain_kernel(const __grid_constant__ CUtensorMap dout_map, const uint8_t *__restrict__ pk,
+bwd_chain_kernel(const uint8_t *__restrict__ pk, const uint8_t *__restrict__ dotiles,
                  const int32_t *__restrict__ cu, const float *__restrict__ dfin,
-                 float *__restrict__ dinit, float *__restrict__ dsl, uint8_t *__restrict__ dudo,
+                 float *__restrict__ dinit, uint8_t *__restrict__ dsl, uint8_t *__restrict__ ndu,
                  int N, int H, int32_t *dev_status, uint64_t wait_ns) {
   using Lay = BChainLayout;
   extern __shared__ uint8_t smem_raw[];
@@ -122,8 +160,6 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap dout_map, const uint8_t *__
   const int unit = blockIdx.x, n = unit / H, h = unit % H;
   const int crow = 32 * qd + lane;   // TMEM lane of this thread: a key channel
   const int64_t nch = seq_chunks(cu, n);
-  const int64_t tseq = cu[n];
-  const int64_t T_n = (int64_t)cu[n + 1] - cu[n];
 
   if (warp == 0) {   // first packet of sequence n (packets: sequence, head, chunk)
     int64_t before = 0;
@@ -133,16 +169,13 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap dout_map, const uint8_t *__
     if (lane == 0) *reinterpret_cast<int64_t *>(sp + Lay::SCAL) = before;
   }
   uint64_t *full = reinterpret_cast<uint64_t *>(sp + Lay::FULL);
-  uint64_t *dobar = reinterpret_cast<uint64_t *>(sp + Lay::DOBAR);
   uint64_t *bar1 = reinterpret_cast<uint64_t *>(sp + Lay::BAR1);
   uint64_t *bar2 = reinterpret_cast<uint64_t *>(sp + Lay::BAR2);
   if (tid == 0) {
     for (int s = 0; s < Lay::NST; ++s) mbar_init(full + s, 1);
-    mbar_init(dobar, 1);
     mbar_init(bar1, 1);
     mbar_init(bar2, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&dout_map)) : "memory");
   }
   if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, 512);
   tc::fence_before_sync();
@@ -152,79 +185,57 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap dout_map, const uint8_t *__
   const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
   const int64_t p0 = *reinterpret_cast<const int64_t *>(sp + Lay::SCAL) * H + (int64_t)h * nch;
 
-  auto issue_packet = [&](int64_t c, int s) {
+  auto issue_stage = [&](int64_t c, int s) {
     const uint8_t *src = pk + (size_t)(p0 + c) * Pk::BYTES;
     const uint32_t st = sb + Lay::STAGE0 + s * Lay::STAGE;
     const uint32_t fb = sb + Lay::FULL + 8 * s;
-    mbar_expect_tx(fb, 16384 + 8704 + 32768);
+    mbar_expect_tx(fb, Lay::TX);
     bulk_load(st + Lay::SKH, src + Pk::KH, 16384, fb);
     bulk_load(st + Lay::SP, src + Pk::P, 8704, fb);      // P and d
     bulk_load(st + Lay::SWQ, src + Pk::WQ, 32768, fb);
+    bulk_load(st + Lay::SDO, dotiles + (size_t)(p0 + c) * 16384, 16384, fb);
   };
-  auto issue_dout = [&](int64_t c) {
-    mbar_expect_tx(sb + Lay::DOBAR, 64 * 512);
-    tma_load_3d(sb + Lay::DOF, &dout_map, 0, h, (int)(tseq + kC * c), sb + Lay::DOBAR);
-  };
-  if (tid == 32 && nch > 0) {
-    issue_dout(nch - 1);
-    for (int s = 0; s < Lay::NST && s < nch; ++s) issue_packet(nch - 1 - s, s);
-  }
+  if (tid == 32)
+    for (int s = 0; s < Lay::NST && s < nch; ++s) issue_stage(nch - 1 - s, s);
 
   // dS = dS_final, FP32 in tensor memory (lane = key channel), BF16 copy in S_T.
   const uint32_t s_tm = tl + Lay::SCOL + hw * 64;
-  auto row_ptr = [&](float *base, int64_t slot) {
-    return base + ((size_t)slot * kD + crow) * kD + hw * 64;
-  };
   {
     const float *src = dfin ? dfin + ((size_t)unit * kD + crow) * kD + hw * 64 : nullptr;
-    float *dst0 = nch > 0 ? row_ptr(dsl, p0 + nch - 1) : (dinit ? row_ptr(dinit, unit) : nullptr);
+    float *dst0 = (nch == 0 && dinit) ? dinit + ((size_t)unit * kD + crow) * kD + hw * 64 : nullptr;
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       float x[32];
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const float4 v4 = src ? *reinterpret_cast<const float4 *>(src + 32 * u + j)
+      for (int jj = 0; jj < 32; jj += 4) {
+        const float4 v4 = src ? *reinterpret_cast<const float4 *>(src + 32 * u + jj)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
-        x[j] = v4.x; x[j + 1] = v4.y; x[j + 2] = v4.z; x[j + 3] = v4.w;
-        if (dst0) *reinterpret_cast<float4 *>(dst0 + 32 * u + j) = v4;
+        x[jj] = v4.x; x[jj + 1] = v4.y; x[jj + 2] = v4.z; x[jj + 3] = v4.w;
+        if (dst0) *reinterpret_cast<float4 *>(dst0 + 32 * u + jj) = v4;
       }
       tc::tmem_st32(s_tm + 32 * u, x);
 #pragma unroll
-      for (int j = 0; j < 32; j += 8)
-        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * 64 + 32 * u + j) >> 3), x + j);
+      for (int jj = 0; jj < 32; jj += 8)
+        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * 64 + 32 * u + jj) >> 3), x + jj);
     }
     tc::tmem_wait_st();
   }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
   __syncthreads();
+  if (tid == 0 && nch > 0) {   // dS_L of the last chunk
+    bulk_store(dsl + (size_t)(p0 + nch - 1) * 32768, sb + Lay::S_T, 32768);
+    bulk_commit();
+  }
 
-  uint32_t fphase = 0, dphase = 0, ph1 = 0, ph2 = 0;
+  uint32_t fphase = 0, ph1 = 0, ph2 = 0;
   bool aborted = false;
   for (int64_t i = 0; i < nch; ++i) {
     const int64_t c = nch - 1 - i;
     const int s = (int)(i % Lay::NST);
     const uint32_t st = sb + Lay::STAGE0 + s * Lay::STAGE;
-    const int L = (int)(T_n - kC * c < kC ? T_n - kC * c : kC);
-    if (__syncthreads_or(!wait_timed(dobar, dphase, wait_ns) ||
-                         !wait_timed(full + s, (fphase >> s) & 1u, wait_ns))) { aborted = true; break; }
-    dphase ^= 1;
+    if (__syncthreads_or(!wait_timed(full + s, (fphase >> s) & 1u, wait_ns))) { aborted = true; break; }
     fphase ^= 1u << s;
-    // dO (FP32 staging) -> BF16 rows 64..127 of BT; rows past the chunk's end are zero.
-    {
-      const int r = tid >> 2, c0 = (tid & 3) * 32;
-      const float *srow = reinterpret_cast<const float *>(sp + Lay::DOF) + r * kD + c0;
-#pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        float x[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = r < L ? srow[j + e] : 0.f;
-        tc::st_chunk(sb + Lay::BT + tc::tile_offset(128, 64 + r, (c0 + j) >> 3), x);
-      }
-    }
-    tc::fence_smem_to_async();
-    __syncthreads();
-    if (tid == 32 && c > 0) issue_dout(c - 1);
     // acc1 = Khat dS + P^T dO  (rows 0..63: dU)
     if (tid == 0) {
       tc::fence_after_sync();
@@ -237,37 +248,42 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap dout_map, const uint8_t *__
 #pragma unroll
       for (int s2 = 0; s2 < 4; ++s2)
         tc::mma_bf16(tmem + Lay::ACC1, tc::desc_mnmajor(st + Lay::SP, 64, s2),
-                     tc::desc_mnmajor(sb + Lay::BT + 8192, 128, s2), idm, 1);
+                     tc::desc_mnmajor(st + Lay::SDO, 64, s2), idm, 1);
       tc::mma_commit(sb + Lay::BAR1);
+      bulk_wait_read();   // the previous -dU and dS_L stores have left NDU and S_T
     }
     if (__syncthreads_or(!wait_timed(bar1, ph1, wait_ns))) { aborted = true; break; }
     ph1 ^= 1;
     tc::fence_after_sync();
-    if (qd < 2) {   // -dU -> rows 0..63 of BT
+    if (qd < 2) {   // -dU -> NDU
       const int r = 32 * qd + lane;
       float a[64];
       tc::tmem_ld32(tl + Lay::ACC1 + hw * 64, *reinterpret_cast<float(*)[32]>(a));
       tc::tmem_ld32(tl + Lay::ACC1 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(a + 32));
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 64; ++j) a[j] = -a[j];
+      for (int jj = 0; jj < 64; ++jj) a[jj] = -a[jj];
 #pragma unroll
-      for (int j = 0; j < 64; j += 8)
-        tc::st_chunk(sb + Lay::BT + tc::tile_offset(128, r, (hw * 64 + j) >> 3), a + j);
+      for (int jj = 0; jj < 64; jj += 8)
+        tc::st_chunk(sb + Lay::NDU + tc::tile_offset(64, r, (hw * 64 + jj) >> 3), a + jj);
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
-    // [-dU; dO] goes to the workspace; acc2 = W^T (-dU) + Qtilde^T dO
+    // -dU goes to the workspace; acc2 = W^T (-dU) + Qtilde^T dO
     if (tid == 0) {
       tc::fence_after_sync();
-      bulk_store(dudo + (size_t)(p0 + c) * 32768, sb + Lay::BT, 32768);
+      bulk_store(ndu + (size_t)(p0 + c) * 16384, sb + Lay::NDU, 16384);
       bulk_commit();
       constexpr uint32_t id = tc::idesc_bf16(128, 128, 1, 1);
 #pragma unroll
-      for (int s2 = 0; s2 < 8; ++s2)
+      for (int s2 = 0; s2 < 4; ++s2)
         tc::mma_bf16(tmem + Lay::ACC2, tc::desc_mnmajor(st + Lay::SWQ, 128, s2),
-                     tc::desc_mnmajor(sb + Lay::BT, 128, s2), id, s2 > 0);
+                     tc::desc_mnmajor(sb + Lay::NDU, 64, s2), id, s2 > 0);
+#pragma unroll
+      for (int s2 = 4; s2 < 8; ++s2)
+        tc::mma_bf16(tmem + Lay::ACC2, tc::desc_mnmajor(st + Lay::SWQ, 128, s2),
+                     tc::desc_mnmajor(st + Lay::SDO, 64, s2 - 4), id, 1);
       tc::mma_commit(sb + Lay::BAR2);
     }
     const float dch = reinterpret_cast<const float *>(sp + (st - sb) + Lay::SD)[crow];
@@ -283,31 +299,34 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap dout_map, const uint8_t *__
       }
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 64; ++j) sv[j] = fmaf(dch, sv[j], a[j]);
+      for (int jj = 0; jj < 64; ++jj) sv[jj] = fmaf(dch, sv[jj], a[jj]);
 #pragma unroll
       for (int u = 0; u < 2; ++u) tc::tmem_st32(s_tm + 32 * u, *reinterpret_cast<float(*)[32]>(sv + 32 * u));
 #pragma unroll
-      for (int j = 0; j < 64; j += 8)
-        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * 64 + j) >> 3), sv + j);
-      float *dst = c > 0 ? row_ptr(dsl, p0 + c - 1) : (dinit ? row_ptr(dinit, unit) : nullptr);
-      if (dst)
+      for (int jj = 0; jj < 64; jj += 8)
+        tc::st_chunk(sb + Lay::S_T + tc::tile_offset(128, crow, (hw * 64 + jj) >> 3), sv + jj);
+      if (c == 0 && dinit) {
+        float *dst = dinit + ((size_t)unit * kD + crow) * kD + hw * 64;
 #pragma unroll
-        for (int j = 0; j < 64; j += 4)
-          *reinterpret_cast<float4 *>(dst + j) = make_float4(sv[j], sv[j + 1], sv[j + 2], sv[j + 3]);
+        for (int jj = 0; jj < 64; jj += 4)
+          *reinterpret_cast<float4 *>(dst + jj) = make_float4(sv[jj], sv[jj + 1], sv[jj + 2], sv[jj + 3]);
+      }
       tc::tmem_wait_st();
     }
-    if (tid == 0) bulk_wait_read();   // BT is rewritten by the next chunk
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
-    if (tid == 32 && c - Lay::NST >= 0) issue_packet(c - Lay::NST, s);
+    if (tid == 0 && c > 0) {   // dS_L of chunk c - 1, as the BF16 tile
+      bulk_store(dsl + (size_t)(p0 + c - 1) * 32768, sb + Lay::S_T, 32768);
+      bulk_commit();
+    }
+    if (tid == 32 && c - Lay::NST >= 0) issue_stage(c - Lay::NST, s);
   }
   if (tid == 0) bulk_wait_all();
   if (aborted) {
     report(dev_status, KDA_ERR_TIMEOUT);
     wait_timed(bar1, ph1, wait_ns);
     wait_timed(bar2, ph2, wait_ns);
-    wait_timed(dobar, dphase, wait_ns);
     for (int s = 0; s < Lay::NST; ++s) wait_timed(full + s, (fphase >> s) & 1u, wait_ns);
   }
   tc::fence_before_sync();
@@ -384,8 +403,9 @@ struct BwdItemArgs {
   const int32_t *cu;
   const int64_t *pref;         // [N+1] chunks before sequence n
   const int64_t *prefck;       // [N+1] full chunks (stored states) before sequence n
-  const float *dsl;            // dS_L per packet (FP32 [128][128])
-  const uint8_t *dudo;         // [-dU; dO] tile per packet
+  const uint8_t *dsl;          // dS_L per packet: BF16 [128 ch][128 v] tile
+  const uint8_t *ndu;          // -dU per packet: BF16 [64 tok][128 v] tile
+  const uint8_t *dot;          // dO per packet: BF16 [64 tok][128 v] tile
   float *dtp;                  // dT, dP per packet: FP32 [64][64] each
   const void *q, *k;           // raw BF16 inputs (re-read by the final epilogues)
   float *dq, *dk, *dv, *dg, *dbeta;
@@ -476,12 +496,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   // The per-chunk states and gradients come from L2 later; start them now.
   const float *S0src = j == 0 ? (a.init ? a.init + (size_t)unit * kD * kD : nullptr)
                               : a.ck + ((size_t)(ckb + j - 1) * H + h) * kD * kD;
-  const float *dSsrc = a.dsl + (size_t)p * kD * kD;
   if (PART == 0) {
-    for (int e = tid; e < 512; e += kThreads) {
-      asm volatile("prefetch.global.L2 [%0];" ::"l"(dSsrc + 32 * e));
-      if (S0src) asm volatile("prefetch.global.L2 [%0];" ::"l"(S0src + 32 * e));
-    }
+    if (S0src)
+      for (int e = tid; e < 512; e += kThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(S0src + 32 * e));
   } else {
     const float *dtp = a.dtp + (size_t)p * 8192;
     for (int e = tid; e < 256; e += kThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(dtp + 32 * e));
@@ -741,33 +758,22 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   const size_t row_stride = (size_t)H * kD;   // elements between tokens in [T][H][128]
   const size_t base_row = ((size_t)t0 * H + h) * kD;
   if constexpr (PART == 0) {
-    // ---- S0 and dS_L as BF16 [ch][v] tiles; dd_c = sum_v dS_L[c, v] S0[c, v] ----
-    // S0T lies over the consumed Gram A tile, DST over the consumed M, (I+M)^-1.
+    // ---- S0 as the BF16 [ch][v] tile over the consumed Gram A tile ----
     if (!aborted) {
       const int c = tid >> 1, h2 = tid & 1;
       const float *s0r = S0src ? S0src + (size_t)c * kD + 64 * h2 : nullptr;
-      const float *dsr = dSsrc + (size_t)c * kD + 64 * h2;
-      float dot = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {   // 32 columns: all loads first, then the stores
-        float xs[32], xd[32];
+        float xs[32];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 u4 = s0r ? *reinterpret_cast<const float4 *>(s0r + 32 * half + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-          const float4 w4 = *reinterpret_cast<const float4 *>(dsr + 32 * half + e);
           xs[e] = u4.x; xs[e + 1] = u4.y; xs[e + 2] = u4.z; xs[e + 3] = u4.w;
-          xd[e] = w4.x; xd[e + 1] = w4.y; xd[e + 2] = w4.z; xd[e + 3] = w4.w;
         }
 #pragma unroll
-        for (int e = 0; e < 32; ++e) dot = fmaf(xs[e], xd[e], dot);
-#pragma unroll
-        for (int jj = 0; jj < 32; jj += 8) {
+        for (int jj = 0; jj < 32; jj += 8)
           st_chunk_s(sp + Lay::S0T + tc::tile_offset(128, c, (64 * h2 + 32 * half + jj) >> 3), xs + jj);
-          st_chunk_s(sp + Lay::DST + tc::tile_offset(128, c, (64 * h2 + 32 * half + jj) >> 3), xd + jj);
-        }
       }
-      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-      if (h2 == 0) s_dd[c] = dot;
       tc::fence_smem_to_async();
       __syncthreads();
     }
@@ -804,9 +810,16 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     tc::fence_before_sync();
     __syncthreads();
     // ---- U = T R (columns 256..383); the chain's [-dU; dO] tile lands over Ktilde, V ----
+    // [-dU; dO] lands over Ktilde and V as one 128-row tile (each 64-row
+    // tile's column blocks interleaved), dS_L over the consumed M, (I+M)^-1.
     if (!aborted && tid == 32) {
-      mbar_expect_tx(sb + Lay::CBAR, 32768);
-      bulk_load(sb + Lay::BT2, a.dudo + (size_t)p * 32768, 32768, sb + Lay::CBAR);
+      mbar_expect_tx(sb + Lay::CBAR, 65536);
+      const uint8_t *nd = a.ndu + (size_t)p * 16384, *dd = a.dot + (size_t)p * 16384;
+      bulk_load(sb + Lay::BT2, nd, 8192, sb + Lay::CBAR);
+      bulk_load(sb + Lay::BT2 + 16384, nd + 8192, 8192, sb + Lay::CBAR);
+      bulk_load(sb + Lay::BT2 + 8192, dd, 8192, sb + Lay::CBAR);
+      bulk_load(sb + Lay::BT2 + 24576, dd + 8192, 8192, sb + Lay::CBAR);
+      bulk_load(sb + Lay::DST, a.dsl + (size_t)p * 32768, 32768, sb + Lay::CBAR);
     }
     if (!aborted && tid == 0) {
       tc::fence_after_sync();
@@ -994,7 +1007,22 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     __syncthreads();
     if (!aborted && tid < 128) {   // dg = reverse cumulative sum of dGam (+ the Gam_63 terms)
       const int ch = tid;
-      float suffix = __expf(s_gam[sw(63, ch)]) * s_dd[ch];
+      float ddc = 0.f;   // sum_v dS_L[ch, v] S0[ch, v]
+      if (S0src) {
+        const float *s0r = S0src + (size_t)ch * kD;
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) {
+          float dv8[8];
+          unpack8(*reinterpret_cast<const uint4 *>(sp + Lay::DST + tc::tile_offset(128, ch, cc)), dv8);
+          const float4 u0 = *reinterpret_cast<const float4 *>(s0r + 8 * cc);
+          const float4 u1 = *reinterpret_cast<const float4 *>(s0r + 8 * cc + 4);
+          ddc = fmaf(dv8[0], u0.x, ddc); ddc = fmaf(dv8[1], u0.y, ddc);
+          ddc = fmaf(dv8[2], u0.z, ddc); ddc = fmaf(dv8[3], u0.w, ddc);
+          ddc = fmaf(dv8[4], u1.x, ddc); ddc = fmaf(dv8[5], u1.y, ddc);
+          ddc = fmaf(dv8[6], u1.z, ddc); ddc = fmaf(dv8[7], u1.w, ddc);
+        }
+      }
+      float suffix = __expf(s_gam[sw(63, ch)]) * ddc;
       for (int r = 0; r < 64; ++r) suffix += pkk[sw(r, ch)];
       for (int r = 63; r >= 0; --r) {
         suffix += pdg[sw(r, ch)];
@@ -1335,7 +1363,7 @@ __global__ void bwd_prefix_kernel(const int32_t *__restrict__ cu, int N, int64_t
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdWs {
-  size_t pk, ck, dsl, dudo, dtp, oscr, pref, prefck, total;
+  size_t pk, ck, dsl, ndu, dot, dtp, oscr, pref, prefck, total;
 };
 
 BwdWs bwd_ws_layout(int N, int H, int64_t T) {
@@ -1344,8 +1372,9 @@ BwdWs bwd_ws_layout(int N, int H, int64_t T) {
   size_t off = 0;
   w.pk = off;     off += align256(P * Pk::BYTES + 256);
   w.ck = off;     off += align256((size_t)(T / kC) * H * kD * kD * 4);
-  w.dsl = off;    off += align256(P * kD * kD * 4);
-  w.dudo = off;   off += align256(P * 32768);
+  w.dsl = off;    off += align256(P * 32768);
+  w.ndu = off;    off += align256(P * 16384);
+  w.dot = off;    off += align256(P * 16384);
   w.dtp = off;    off += align256(P * 8192 * 4);
   w.oscr = off;   off += align256((size_t)T * H * kD * 2);
   w.pref = off;   off += align256((size_t)(N + 1) * 8);
@@ -1373,8 +1402,9 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(workspace) + 255) & ~(uintptr_t)255);
   uint8_t *pk = base + w.pk;
   float *ck = reinterpret_cast<float *>(base + w.ck);
-  float *dsl = reinterpret_cast<float *>(base + w.dsl);
-  uint8_t *dudo = base + w.dudo;
+  uint8_t *dsl = base + w.dsl;
+  uint8_t *ndu = base + w.ndu;
+  uint8_t *dot = base + w.dot;
   float *dtp = reinterpret_cast<float *>(base + w.dtp);
   void *oscr = base + w.oscr;
   int64_t *pref = reinterpret_cast<int64_t *>(base + w.pref);
@@ -1389,11 +1419,12 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   bwd_prefix_kernel<<<1, 32, 0, stream>>>(cu, N, pref, prefck);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  CUtensorMap dout_map;
+  const int64_t P_max = (int64_t)H * ((T + (int64_t)(kC - 1) * N) / kC);
+  bwd_dout_tiles_kernel<<<(unsigned)P_max, kThreads, 0, stream>>>(dout, cu, pref, N, H, dot);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
   TmaMaps maps;
-  if (!make_map(&dout_map, dout, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kD, H, T, kD, kC,
-                CU_TENSOR_MAP_SWIZZLE_NONE) ||
-      !make_input_maps(&maps, q, k, v, g, H, T) ||
+  if (!make_input_maps(&maps, q, k, v, g, H, T) ||
       !make_map(&maps.q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, H, T, 64, 64,
                 CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map(&maps.k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, kD, H, T, 64, 64,
@@ -1404,12 +1435,12 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   e = cudaFuncSetAttribute(bwd_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_c);
   if (e != cudaSuccess) return e;
   bwd_chain_kernel<<<(unsigned)((int64_t)N * H), kThreads, smem_c, stream>>>(
-      dout_map, pk, cu, dfin, dinit, dsl, dudo, N, H, dev_status, wait_ns);
+      pk, dot, cu, dfin, dinit, dsl, ndu, N, H, dev_status, wait_ns);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   BwdItemArgs a;
   a.beta = beta; a.init = init; a.ck = ck; a.cu = cu; a.pref = pref; a.prefck = prefck;
-  a.dsl = dsl; a.dudo = dudo; a.dtp = dtp; a.q = q; a.k = k;
+  a.dsl = dsl; a.ndu = ndu; a.dot = dot; a.dtp = dtp; a.q = q; a.k = k;
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
   a.N = N; a.H = H; a.dev_status = dev_status; a.wait_ns = wait_ns;
   const size_t smem_i = BItemLayout::TOTAL + 1024;
