@@ -383,15 +383,21 @@ struct BItemLayout {
   // PART 1 final partials: float [64][128] and [32][128]
   static constexpr uint32_t QDG = XA, KMC = YA;
   static_assert(GG + 17408 <= TT && MT + 4224 <= GG, "solve scratch");
+  static_assert(YS + 2048 <= ZS && DST + 32768 <= YS, "scan scratch clears dS_L");
   static_assert(GB + 24576 <= RU + 32768 && RU + 32768 <= GST, "[R; U] stays clear of Gam");
   static_assert(CST + 6144 <= XM + 17408, "gate factors");
   static_assert(TOTAL + 1024 <= 232448, "shared memory");
 };
 
-// FP32 [64 tokens][128 channels] arrays read with one token per lane: the
-// channel index is XOR-ed with the token's low five bits, so a warp reading
-// one channel of 32 tokens touches 32 banks.
-__device__ __forceinline__ int sw(int r, int ch) { return r * 128 + (ch ^ (r & 31)); }
+// FP32 [64 tokens][128 channels] arrays read both with one token per lane
+// (float4 groups of channels) and with one channel per thread: the float4
+// slot of channels 4f..4f+3 of token r is XOR-ed with the token's low five
+// bits, so a warp reading one group of 32 tokens, or one token's channels,
+// touches every bank.
+__device__ __forceinline__ int sw4(int r, int f) { return r * 32 + (f ^ (r & 31)); }
+__device__ __forceinline__ int sw(int r, int ch) { return 4 * sw4(r, ch >> 2) + (ch & 3); }
+__device__ __forceinline__ float4 f4mul(float4 a, float4 b) { return make_float4(a.x * b.x, a.y * b.y, a.z * b.z, a.w * b.w); }
+__device__ __forceinline__ float4 f4exp(float4 a) { return make_float4(__expf(a.x), __expf(a.y), __expf(a.z), __expf(a.w)); }
 
 __device__ __forceinline__ void st_chunk_s(uint8_t *dst, const float *x) {
   *reinterpret_cast<uint4 *>(dst) = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
@@ -613,13 +619,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     // Gam stays for the final epilogue, in place of g (every thread has read
     // its g rows before the first barrier of the prep).
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int r = 8 * warp + i;
-      s_gam[sw(r, 4 * lane)] = gm[i][0].x;
-      s_gam[sw(r, 4 * lane + 1)] = gm[i][0].y;
-      s_gam[sw(r, 4 * lane + 2)] = gm[i][1].x;
-      s_gam[sw(r, 4 * lane + 3)] = gm[i][1].y;
-    }
+    for (int i = 0; i < 8; ++i)
+      reinterpret_cast<float4 *>(s_gam)[sw4(8 * warp + i, lane)] =
+          make_float4(gm[i][0].x, gm[i][0].y, gm[i][1].x, gm[i][1].y);
     tc::fence_smem_to_async();
     __syncthreads();
   }
@@ -790,7 +792,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
     phase ^= 1;
     tc::fence_after_sync();
-    if (!aborted && qd < 2) {   // rows 0..63 of [R; U]; V rows past the chunk's end are zero
+    if (!aborted && qd < 2) {   // rows 64..127 of [U; R]; V rows past the chunk's end are zero
       const int r = 32 * qd + lane;
       float acc[64];
       tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(acc));
@@ -803,7 +805,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         unpack8(*reinterpret_cast<const uint4 *>(sp + Lay::VT + tc::tile_offset(64, r, chunk)), xv);
 #pragma unroll
         for (int e = 0; e < 8; ++e) xv[e] = (r < L ? xv[e] : 0.f) - acc[8 * cc + e];
-        st_chunk_s(sp + Lay::RU + tc::tile_offset(128, r, chunk), xv);
+        st_chunk_s(sp + Lay::RU + tc::tile_offset(128, 64 + r, chunk), xv);
       }
     }
     tc::fence_smem_to_async();
@@ -827,13 +829,13 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll
       for (int s2 = 0; s2 < 4; ++s2)
         tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::TT, 64, s2),
-                     tc::desc_mnmajor(sb + Lay::RU, 128, s2), id, s2 > 0);
+                     tc::desc_mnmajor(sb + Lay::RU + 8192, 128, s2), id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
     phase ^= 1;
     tc::fence_after_sync();
-    if (!aborted && qd < 2) {   // rows 64..127 of [R; U]
+    if (!aborted && qd < 2) {   // rows 0..63 of [U; R]
       const int r = 32 * qd + lane;
       float acc[64];
       tc::tmem_ld32(tl + 256 + hw * 64, *reinterpret_cast<float(*)[32]>(acc));
@@ -841,15 +843,15 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       tc::tmem_wait_ld();
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc)
-        st_chunk_s(sp + Lay::RU + tc::tile_offset(128, 64 + r, hw * 8 + cc), acc + 8 * cc);
+        st_chunk_s(sp + Lay::RU + tc::tile_offset(128, r, hw * 8 + cc), acc + 8 * cc);
     }
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     if (!aborted && __syncthreads_or(!wait_timed(cbar, cphase, a.wait_ns))) aborted = true;
     cphase ^= 1;
-    // ---- dR = T^T (-dU) -> -dR (columns 0..127);  [-dU; dO] [R; U]^T (384..511):
-    //      rows 0..63 x 0..63 = -dT, rows 64..127 x 64..127 = dP;  [R; U] dS_L^T (256..383):
-    //      rows 64..127 = dKhat ----
+    // ---- dR = T^T (-dU) -> -dR (columns 0..127);  [-dU; dO] [U; R]^T (384..511):
+    //      rows 0..63 x 64..127 = -dT, rows 64..127 x 0..63 = dP;  [U; R] dS_L^T (256..383):
+    //      rows 0..63 = dKhat ----
     if (!aborted && tid == 0) {
       tc::fence_after_sync();
       constexpr uint32_t idr = tc::idesc_bf16(128, 128, 1, 1);
@@ -889,7 +891,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         for (int cc = 0; cc < 8; ++cc)   // -dR replaces -dU in rows 0..63
           st_chunk_s(sp + Lay::BT2 + tc::tile_offset(128, r, hw * 8 + cc), acc + 8 * cc);
         float d2[32];
-        tc::tmem_ld32(tl + 384 + hw * 32, d2);
+        tc::tmem_ld32(tl + 448 + hw * 32, d2);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -901,7 +903,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       } else {
         const int r = 32 * (qd - 2) + lane;
         float d2[32];
-        tc::tmem_ld32(tl + 448 + hw * 32, d2);
+        tc::tmem_ld32(tl + 384 + hw * 32, d2);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
@@ -929,57 +931,46 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     phase ^= 1;
     tc::fence_after_sync();
     // ---- final epilogue: dq, dk and dGam from Qtilde, Ktilde, Khat and d ----
-    float *pkm = reinterpret_cast<float *>(sp + Lay::PKM);   // dk from Khat
-    float *pdg = reinterpret_cast<float *>(sp + Lay::PDG);   // dGam
-    float *pkk = reinterpret_cast<float *>(sp + Lay::BT2);   // k (dk from Khat): the dGam_63 extra
+    // Token r's dQtilde sits in TMEM lane 64 + r, its dKtilde and dKhat in lane
+    // r: the two halves of the CTA work at once, each on its own dGam part.
+    float4 *pdq4 = reinterpret_cast<float4 *>(sp + Lay::PKM);   // q (dq from Qtilde)
+    float4 *pdk4 = reinterpret_cast<float4 *>(sp + Lay::PDG);   // k (dk+ - dk-)
+    float4 *pkk4 = reinterpret_cast<float4 *>(sp + Lay::BT2);   // k (dk from Khat): the dGam_63 extra
     const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(a.q);
     const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(a.k);
+    const float4 *g4 = reinterpret_cast<const float4 *>(s_gam);
     if (!aborted && qd >= 2) {
       const int r = 32 * (qd - 2) + lane;
       const bool in = r < L;
-      float aq[64], ak[64];
+      float aq[64];
       tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(aq));
       tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(aq + 32));
-      tc::tmem_ld32(tl + 256 + hw * 64, *reinterpret_cast<float(*)[32]>(ak));
-      tc::tmem_ld32(tl + 256 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ak + 32));
       tc::tmem_wait_ld();
       const size_t off = base_row + (size_t)r * row_stride + hw * 64;
-      uint4 qraw[8], kraw[8];
+      uint4 qraw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        qraw[u] = in ? *reinterpret_cast<const uint4 *>(qb + off + 8 * u) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        qraw[u] = in ? *reinterpret_cast<const uint4 *>(qb + off + 8 * u) : make_uint4(0, 0, 0, 0);
-        kraw[u] = in ? *reinterpret_cast<const uint4 *>(kb + off + 8 * u) : make_uint4(0, 0, 0, 0);
-      }
+        float qv[8];
+        unpack8(qraw[u], qv);
 #pragma unroll
-      for (int cc = 0; cc < 64; cc += 8) {
-        float qv[8], kv[8], dq8[8];
-        unpack8(qraw[cc >> 3], qv);
-        unpack8(kraw[cc >> 3], kv);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int ch = hw * 64 + cc + e;
-          const float gam = s_gam[sw(r, ch)], g63 = s_gam[sw(63, ch)];
-          const float dqa = __expf(gam) * aq[cc + e];
-          const float dkm = __expf(g63 - gam) * ak[cc + e];
-          dq8[e] = dqa;
-          pkm[sw(r, ch)] = dkm;
-          pkk[sw(r, ch)] = kv[e] * dkm;
-          pdg[sw(r, ch)] = qv[e] * dqa - kv[e] * dkm;
-        }
-        if (in) {
-          float *dst = a.dq + off + cc;
-          *reinterpret_cast<float4 *>(dst) = make_float4(dq8[0], dq8[1], dq8[2], dq8[3]);
-          *reinterpret_cast<float4 *>(dst + 4) = make_float4(dq8[4], dq8[5], dq8[6], dq8[7]);
+        for (int hf = 0; hf < 2; ++hf) {   // channels hw*64 + 8u + 4hf .. +3
+          const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
+          const float4 dqa = f4mul(f4exp(g4[sw4(r, F)]), make_float4(aq[c], aq[c + 1], aq[c + 2], aq[c + 3]));
+          pdq4[sw4(r, F)] = f4mul(make_float4(qv[4 * hf], qv[4 * hf + 1], qv[4 * hf + 2], qv[4 * hf + 3]), dqa);
+          if (in) *reinterpret_cast<float4 *>(a.dq + off + c) = dqa;
         }
       }
-    }
-    __syncthreads();
-    if (!aborted && qd < 2) {
+    } else if (!aborted) {
       const int r = 32 * qd + lane;
       const bool in = r < L;
-      float ak[64];
+      float ak[64], ah[64];
       tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(ak));
       tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ak + 32));
+      tc::tmem_ld32(tl + 256 + hw * 64, *reinterpret_cast<float(*)[32]>(ah));
+      tc::tmem_ld32(tl + 256 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ah + 32));
       tc::tmem_wait_ld();
       const size_t off = base_row + (size_t)r * row_stride + hw * 64;
       uint4 kraw[8];
@@ -987,45 +978,64 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       for (int u = 0; u < 8; ++u)
         kraw[u] = in ? *reinterpret_cast<const uint4 *>(kb + off + 8 * u) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int cc = 0; cc < 64; cc += 8) {
-        float kv[8], dk8[8];
-        unpack8(kraw[cc >> 3], kv);
+      for (int u = 0; u < 8; ++u) {
+        float kv[8];
+        unpack8(kraw[u], kv);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int ch = hw * 64 + cc + e;
-          const float dkp = __expf(s_gam[sw(r, ch)]) * ak[cc + e];
-          dk8[e] = dkp + pkm[sw(r, ch)];
-          pdg[sw(r, ch)] += kv[e] * dkp;
-        }
-        if (in) {
-          float *dst = a.dk + off + cc;
-          *reinterpret_cast<float4 *>(dst) = make_float4(dk8[0], dk8[1], dk8[2], dk8[3]);
-          *reinterpret_cast<float4 *>(dst + 4) = make_float4(dk8[4], dk8[5], dk8[6], dk8[7]);
+        for (int hf = 0; hf < 2; ++hf) {
+          const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
+          const float4 gam = g4[sw4(r, F)], g63 = g4[sw4(63, F)];
+          const float4 dkp = f4mul(f4exp(gam), make_float4(ak[c], ak[c + 1], ak[c + 2], ak[c + 3]));
+          const float4 dkm = f4mul(f4exp(make_float4(g63.x - gam.x, g63.y - gam.y, g63.z - gam.z, g63.w - gam.w)),
+                                   make_float4(ah[c], ah[c + 1], ah[c + 2], ah[c + 3]));
+          const float4 k4 = make_float4(kv[4 * hf], kv[4 * hf + 1], kv[4 * hf + 2], kv[4 * hf + 3]);
+          const float4 kp = f4mul(k4, dkp), km = f4mul(k4, dkm);
+          pdk4[sw4(r, F)] = make_float4(kp.x - km.x, kp.y - km.y, kp.z - km.z, kp.w - km.w);
+          pkk4[sw4(r, F)] = km;
+          if (in)
+            *reinterpret_cast<float4 *>(a.dk + off + c) =
+                make_float4(dkp.x + dkm.x, dkp.y + dkm.y, dkp.z + dkm.z, dkp.w + dkm.w);
         }
       }
     }
     __syncthreads();
-    if (!aborted && tid < 128) {   // dg = reverse cumulative sum of dGam (+ the Gam_63 terms)
-      const int ch = tid;
-      float ddc = 0.f;   // sum_v dS_L[ch, v] S0[ch, v]
-      if (S0src) {
-        const float *s0r = S0src + (size_t)ch * kD;
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc) {
-          float dv8[8];
-          unpack8(*reinterpret_cast<const uint4 *>(sp + Lay::DST + tc::tile_offset(128, ch, cc)), dv8);
-          const float4 u0 = *reinterpret_cast<const float4 *>(s0r + 8 * cc);
-          const float4 u1 = *reinterpret_cast<const float4 *>(s0r + 8 * cc + 4);
-          ddc = fmaf(dv8[0], u0.x, ddc); ddc = fmaf(dv8[1], u0.y, ddc);
-          ddc = fmaf(dv8[2], u0.z, ddc); ddc = fmaf(dv8[3], u0.w, ddc);
-          ddc = fmaf(dv8[4], u1.x, ddc); ddc = fmaf(dv8[5], u1.y, ddc);
-          ddc = fmaf(dv8[6], u1.z, ddc); ddc = fmaf(dv8[7], u1.w, ddc);
-        }
+    // dg = reverse cumulative sum of dGam plus the Gam_63 terms (sum_r k dk-_r from
+    // Khat, d * sum_v dS_L S0).  Two threads per channel, 32 rows each.
+    float *sred = s_Y;   // [2][128] partial sums, [2][128] partial extras (the solve scratch)
+    if (!aborted) {
+      const int ch = tid & 127, hf = tid >> 7;
+      const float *pdq = reinterpret_cast<const float *>(pdq4), *pdk = reinterpret_cast<const float *>(pdk4);
+      const float *pkk = reinterpret_cast<const float *>(pkk4);
+      float part = 0.f, extra = 0.f;
+#pragma unroll 8
+      for (int r = 32 * hf; r < 32 * hf + 32; ++r) {
+        part += pdq[sw(r, ch)] + pdk[sw(r, ch)];
+        extra += pkk[sw(r, ch)];
       }
-      float suffix = __expf(s_gam[sw(63, ch)]) * ddc;
-      for (int r = 0; r < 64; ++r) suffix += pkk[sw(r, ch)];
-      for (int r = 63; r >= 0; --r) {
-        suffix += pdg[sw(r, ch)];
+      if (S0src) {   // sum over this thread's half of the value columns
+        const float *s0r = S0src + (size_t)ch * kD + 64 * hf;
+        float4 s4[16];
+#pragma unroll
+        for (int cc = 0; cc < 16; ++cc) s4[cc] = *reinterpret_cast<const float4 *>(s0r + 4 * cc);
+        float dd = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          float dv8[8];
+          unpack8(*reinterpret_cast<const uint4 *>(sp + Lay::DST + tc::tile_offset(128, ch, 8 * hf + cc)), dv8);
+          dd = fmaf(dv8[0], s4[2 * cc].x, dd); dd = fmaf(dv8[1], s4[2 * cc].y, dd);
+          dd = fmaf(dv8[2], s4[2 * cc].z, dd); dd = fmaf(dv8[3], s4[2 * cc].w, dd);
+          dd = fmaf(dv8[4], s4[2 * cc + 1].x, dd); dd = fmaf(dv8[5], s4[2 * cc + 1].y, dd);
+          dd = fmaf(dv8[6], s4[2 * cc + 1].z, dd); dd = fmaf(dv8[7], s4[2 * cc + 1].w, dd);
+        }
+        extra = fmaf(__expf(s_gam[sw(63, ch)]), dd, extra);
+      }
+      sred[hf * 128 + ch] = part;
+      sred[256 + hf * 128 + ch] = extra;
+      __syncthreads();
+      float suffix = sred[256 + ch] + sred[384 + ch] + (hf == 0 ? sred[128 + ch] : 0.f);
+#pragma unroll 8
+      for (int r = 32 * hf + 31; r >= 32 * hf; --r) {
+        suffix += pdq[sw(r, ch)] + pdk[sw(r, ch)];
         if (r < L) a.dg[base_row + (size_t)r * row_stride + ch] = suffix;
       }
     }
@@ -1182,7 +1192,8 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
-    // ---- [X; Xq] = [dG; dP] Gram B (columns 0..127), Y = [dG^T | dP^T] Gram A (128..255) ----
+    // ---- [X; Xq] = [dG; dP] Gram B (columns 0..127), Y = [dG^T | dP^T] Gram A (128..255),
+    //      and rows 64..127 of YA again (256..383) so that the cross rows land in lanes 0..31 ----
     if (!aborted && tid == 0) {
       tc::fence_after_sync();
       constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 1);
@@ -1194,6 +1205,10 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       for (int s2 = 0; s2 < 8; ++s2)
         tc::mma_bf16(tmem + 128, tc::desc_kmajor(sb + Lay::YA, 128, s2),
                      tc::desc_mnmajor(sb + Lay::GA, 128, s2), id, s2 > 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)   // rows 64..127 of YA as rows 0..63 (the rest read past them)
+        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::YA + 8192, 128, s2),
+                     tc::desc_mnmajor(sb + Lay::GA, 128, s2), id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
@@ -1204,12 +1219,14 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     // products used (Gram A rows for the sides where Gam enters with a plus
     // sign, Gram B rows for the others), so that the pair's terms, which the
     // reverse cumulative sum below sets against each other, cancel to FP32
-    // accumulation precision.
-    float *qdg = reinterpret_cast<float *>(sp + Lay::QDG);   // dGam
-    float *kmc = reinterpret_cast<float *>(sp + Lay::KMC);   // dk from first-half keys, second-half reference
-    auto tile_val = [&](uint32_t tile, int rows, int row, int ch) {
-      return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-          sp + tile + tc::tile_offset(rows, row, ch >> 3) + 2 * (ch & 7)));
+    // accumulation precision.  Lanes 64..127 (Xq) and lanes 0..63 (X, Y and the
+    // cross rows) work at once, each half on its own dGam part.
+    float4 *qdg4 = reinterpret_cast<float4 *>(sp + Lay::QDG);   // dGam from the q side
+    float4 *kdg4 = reinterpret_cast<float4 *>(sp + Lay::KMC);   // dGam from the k sides
+    const float4 *g4 = reinterpret_cast<const float4 *>(s_gam);
+    // 8 BF16 values of a tile row (one 16-byte chunk) as floats
+    auto tile8 = [&](uint32_t tile, int rows, int row, int chunk, float *x) {
+      unpack8(*reinterpret_cast<const uint4 *>(sp + tile + tc::tile_offset(rows, row, chunk)), x);
     };
     float *dqp = a.dq, *dkp_ = a.dk;
     if (!aborted && qd >= 2) {
@@ -1219,9 +1236,8 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         const int c0 = hw * 64 + 32 * half;
-        float xq[32], yc[32];
+        float xq[32];
         tc::tmem_ld32(tl + 0 + c0, xq);
-        tc::tmem_ld32(tl + 128 + c0, yc);
         tc::tmem_wait_ld();
         const size_t off = base_row + (size_t)r * row_stride + c0;
         float4 old[8];
@@ -1229,29 +1245,25 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) old[e] = *reinterpret_cast<const float4 *>(dqp + off + 4 * e);
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          float add[4];
+        for (int u = 0; u < 4; ++u) {   // 8 channels: one tile chunk
+          float ga[8];
+          tile8(Lay::GA, 128, 64 + r, (c0 >> 3) + u, ga);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * e4 + e, ch = c0 + c;
-            const float gam = s_gam[sw(r, ch)];
-            add[e] = __expf(gam - s_gam[sw(ref, ch)]) * xq[c];
-            float dgm = tile_val(Lay::GA, 128, 64 + r, ch) * xq[c];
-            if (r < 32) {
-              dgm -= tile_val(Lay::GB, 96, 32 + r, ch) * yc[c];
-              kmc[sw(r, ch)] = __expf(s_gam[sw(47, ch)] - gam) * yc[c];
-            }
-            qdg[sw(r, ch)] = dgm;
-          }
-          if (in) {
-            old[e4].x += add[0]; old[e4].y += add[1]; old[e4].z += add[2]; old[e4].w += add[3];
-            *reinterpret_cast<float4 *>(dqp + off + 4 * e4) = old[e4];
+          for (int hf = 0; hf < 2; ++hf) {
+            const int F = (c0 >> 2) + 2 * u + hf, c = 8 * u + 4 * hf;
+            const float4 gam = g4[sw4(r, F)], gref = g4[sw4(ref, F)];
+            const float4 xqv = make_float4(xq[c], xq[c + 1], xq[c + 2], xq[c + 3]);
+            const float4 add = f4mul(f4exp(make_float4(gam.x - gref.x, gam.y - gref.y, gam.z - gref.z, gam.w - gref.w)), xqv);
+            qdg4[sw4(r, F)] = f4mul(make_float4(ga[4 * hf], ga[4 * hf + 1], ga[4 * hf + 2], ga[4 * hf + 3]), xqv);
+            const int e = 2 * u + hf;
+            old[e].x += add.x; old[e].y += add.y; old[e].z += add.z; old[e].w += add.w;
           }
         }
+        if (in)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) *reinterpret_cast<float4 *>(dqp + off + 4 * e) = old[e];
       }
-    }
-    __syncthreads();
-    if (!aborted && qd < 2) {
+    } else if (!aborted) {
       const int t = 32 * qd + lane;
       const bool in = t < L;
       const int ref = t < 32 ? 15 : 47;
@@ -1259,9 +1271,10 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         const int c0 = hw * 64 + 32 * half;
-        float xk[32], yo[32];
+        float xk[32], yo[32], yc[32];
         tc::tmem_ld32(tl + 0 + c0, xk);
         tc::tmem_ld32(tl + 128 + c0, yo);
+        tc::tmem_ld32(tl + 256 + c0, yc);   // cross rows (first-half keys, second-half reference)
         tc::tmem_wait_ld();
         const size_t off = base_row + (size_t)t * row_stride + c0;
         float4 old[8];
@@ -1269,42 +1282,66 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) old[e] = *reinterpret_cast<const float4 *>(dkp_ + off + 4 * e);
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          float add[4];
+        for (int u = 0; u < 4; ++u) {
+          float ga[8], gb[8], gc[8];
+          tile8(Lay::GA, 128, t, (c0 >> 3) + u, ga);
+          tile8(Lay::GB, 96, gbrow, (c0 >> 3) + u, gb);
+          if (t < 32) tile8(Lay::GB, 96, 32 + t, (c0 >> 3) + u, gc);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 4 * e4 + e, ch = c0 + c;
-            const float gam = s_gam[sw(t, ch)];
-            const float dlt = gam - s_gam[sw(ref, ch)];
-            float dkm = __expf(-dlt) * yo[c];
-            if (t < 32) dkm += kmc[sw(t, ch)];
-            add[e] = __expf(dlt) * xk[c] + dkm;
-            qdg[sw(t, ch)] += tile_val(Lay::GA, 128, t, ch) * xk[c] - tile_val(Lay::GB, 96, gbrow, ch) * yo[c];
-          }
-          if (in) {
-            old[e4].x += add[0]; old[e4].y += add[1]; old[e4].z += add[2]; old[e4].w += add[3];
-            *reinterpret_cast<float4 *>(dkp_ + off + 4 * e4) = old[e4];
+          for (int hf = 0; hf < 2; ++hf) {
+            const int F = (c0 >> 2) + 2 * u + hf, c = 8 * u + 4 * hf;
+            const float4 gam = g4[sw4(t, F)], gref = g4[sw4(ref, F)];
+            const float4 dlt = make_float4(gam.x - gref.x, gam.y - gref.y, gam.z - gref.z, gam.w - gref.w);
+            const float4 xkv = make_float4(xk[c], xk[c + 1], xk[c + 2], xk[c + 3]);
+            const float4 yov = make_float4(yo[c], yo[c + 1], yo[c + 2], yo[c + 3]);
+            const float4 dkp = f4mul(f4exp(dlt), xkv);
+            float4 dkm = f4mul(f4exp(make_float4(-dlt.x, -dlt.y, -dlt.z, -dlt.w)), yov);
+            const float4 pa = f4mul(make_float4(ga[4 * hf], ga[4 * hf + 1], ga[4 * hf + 2], ga[4 * hf + 3]), xkv);
+            float4 pb = f4mul(make_float4(gb[4 * hf], gb[4 * hf + 1], gb[4 * hf + 2], gb[4 * hf + 3]), yov);
+            if (t < 32) {
+              const float4 ycv = make_float4(yc[c], yc[c + 1], yc[c + 2], yc[c + 3]);
+              const float4 g47 = g4[sw4(47, F)];
+              const float4 km = f4mul(f4exp(make_float4(g47.x - gam.x, g47.y - gam.y, g47.z - gam.z, g47.w - gam.w)), ycv);
+              dkm = make_float4(dkm.x + km.x, dkm.y + km.y, dkm.z + km.z, dkm.w + km.w);
+              const float4 pc = f4mul(make_float4(gc[4 * hf], gc[4 * hf + 1], gc[4 * hf + 2], gc[4 * hf + 3]), ycv);
+              pb = make_float4(pb.x + pc.x, pb.y + pc.y, pb.z + pc.z, pb.w + pc.w);
+            }
+            kdg4[sw4(t, F)] = make_float4(pa.x - pb.x, pa.y - pb.y, pa.z - pb.z, pa.w - pb.w);
+            const int e = 2 * u + hf;
+            old[e].x += dkp.x + dkm.x; old[e].y += dkp.y + dkm.y;
+            old[e].z += dkp.z + dkm.z; old[e].w += dkp.w + dkm.w;
           }
         }
+        if (in)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) *reinterpret_cast<float4 *>(dkp_ + off + 4 * e) = old[e];
       }
     }
     __syncthreads();
-    if (!aborted && tid < 128) {
-      const int ch = tid;
+    // dg += reverse cumulative sum of dGam: two threads per channel, 32 rows each.
+    if (!aborted) {
+      const int ch = tid & 127, hf = tid >> 7;
+      const float *qdg = reinterpret_cast<const float *>(qdg4), *kdg = reinterpret_cast<const float *>(kdg4);
+      float *sred = s_Y;
+      float part = 0.f;
+#pragma unroll 8
+      for (int r = 32 * hf; r < 32 * hf + 32; ++r) part += qdg[sw(r, ch)] + kdg[sw(r, ch)];
+      sred[hf * 128 + ch] = part;
+      __syncthreads();
       float *dgp = a.dg;
-      float suffix = 0.f;
+      float suffix = hf == 0 ? sred[128 + ch] : 0.f;
 #pragma unroll 1
-      for (int blk = 3; blk >= 0; --blk) {   // 16 rows at a time: their loads issue together
+      for (int blk = 1; blk >= 0; --blk) {   // 16 rows at a time: their loads issue together
         float prev[16];
 #pragma unroll
         for (int u = 0; u < 16; ++u) {
-          const int r = 16 * blk + u;
+          const int r = 32 * hf + 16 * blk + u;
           prev[u] = r < L ? dgp[base_row + (size_t)r * row_stride + ch] : 0.f;
         }
 #pragma unroll
         for (int u = 15; u >= 0; --u) {
-          const int r = 16 * blk + u;
-          suffix += qdg[sw(r, ch)];
+          const int r = 32 * hf + 16 * blk + u;
+          suffix += qdg[sw(r, ch)] + kdg[sw(r, ch)];
           if (r < L) dgp[base_row + (size_t)r * row_stride + ch] = prev[u] + suffix;
         }
       }

@@ -22,8 +22,27 @@ namespace kda {
 // their way, so the SM's share of HBM bandwidth stays busy during the serial
 // token loop.  Tokens are prepared in groups of kMultiGroup (gates and q . k
 // for the whole group before the token loop), so each token costs two block
-// barriers and no global-memory latency.
+// barriers and no global-memory latency.  Each thread keeps four columns of a
+// block of consecutive state rows, held as (row 2i, row 2i+1) pairs so that
+// the paired FP32 instructions take a token's per-row gate values in pairs
+// straight from 16-byte shared-memory loads.
 constexpr int kMultiGroup = 8;
+
+// ROWS consecutive shared-memory floats (the same for every lane of a warp):
+// 16-byte loads when ROWS is a multiple of 4.
+template <int ROWS>
+__device__ __forceinline__ void load_rows(const float *src, float *dst) {
+  if constexpr (ROWS % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < ROWS; i += 4) {
+      const float4 v = *reinterpret_cast<const float4 *>(src + i);
+      dst[i] = v.x; dst[i + 1] = v.y; dst[i + 2] = v.z; dst[i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < ROWS; ++i) dst[i] = src[i];
+  }
+}
 
 template <int DK, int DV, typename TIn>
 struct MultiLayout {
@@ -51,10 +70,11 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
   constexpr int RPP = THREADS / V4;
   constexpr int ROWS = DK / RPP;
   constexpr int G = kMultiGroup;
-  static_assert(THREADS % V4 == 0 && DK % RPP == 0, "tile mismatch");
+  static_assert(THREADS % V4 == 0 && DK % RPP == 0 && ROWS % 2 == 0, "tile mismatch");
+  constexpr int RP = ROWS / 2;   // row pairs per thread
 
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  __shared__ float s_ka[G][DK], s_qa[G][DK], s_alpha[G][DK], s_k[G][DK];
+  __shared__ __align__(16) float s_ka[G][DK], s_qa[G][DK], s_alpha[G][DK], s_k[G][DK];
   __shared__ float s_v[G][DV], s_beta[G], s_qk[G];
   __shared__ float s_u[2][DV];
   __shared__ float4 s_red[2][2][RPP][V4];
@@ -119,15 +139,19 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
     }
     if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
     phase ^= 1;
-    // the thread's float4 of each row as two pairs, for the paired FP32 units
-    float2 sa[ROWS], sb2[ROWS];
+    // The thread's four columns of each pair of consecutive rows, as
+    // (row 2i, row 2i+1) pairs for the paired FP32 units: sp[i][c].
+    float2 sp[RP][4];
     {
       const float4 *S4s = reinterpret_cast<const float4 *>(smem_raw + Lay::STATE);
 #pragma unroll
-      for (int i = 0; i < ROWS; ++i) {
-        const float4 x = S4s[(rg + i * RPP) * V4 + cg];
-        sa[i] = make_float2(x.x, x.y);
-        sb2[i] = make_float2(x.z, x.w);
+      for (int i = 0; i < RP; ++i) {
+        const float4 x0 = S4s[(rg * ROWS + 2 * i) * V4 + cg];
+        const float4 x1 = S4s[(rg * ROWS + 2 * i + 1) * V4 + cg];
+        sp[i][0] = make_float2(x0.x, x1.x);
+        sp[i][1] = make_float2(x0.y, x1.y);
+        sp[i][2] = make_float2(x0.z, x1.z);
+        sp[i][3] = make_float2(x0.w, x1.w);
       }
     }
     cp_async_wait_all();
@@ -195,19 +219,24 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 
       for (int j = 0; j < cnt; ++j) {
         const int t = t0 + j, p = t & 1;   // parity-indexed buffers: no third barrier
-        float2 ya = make_float2(0.f, 0.f), yb = ya, za = ya, zb = ya;
+        float kar[ROWS], qar[ROWS];
+        load_rows<ROWS>(&s_ka[j][rg * ROWS], kar);
+        load_rows<ROWS>(&s_qa[j][rg * ROWS], qar);
+        float2 yp[4], zp[4];   // (even rows, odd rows) partial sums per column
 #pragma unroll
-        for (int i = 0; i < ROWS; ++i) {
-          const int r = rg + i * RPP;
-          const float2 ka = make_float2(s_ka[j][r], s_ka[j][r]);
-          const float2 qa = make_float2(s_qa[j][r], s_qa[j][r]);
-          ya = __ffma2_rn(ka, sa[i], ya);
-          yb = __ffma2_rn(ka, sb2[i], yb);
-          za = __ffma2_rn(qa, sa[i], za);
-          zb = __ffma2_rn(qa, sb2[i], zb);
+        for (int c = 0; c < 4; ++c) yp[c] = zp[c] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < RP; ++i) {
+          const float2 ka = make_float2(kar[2 * i], kar[2 * i + 1]);
+          const float2 qa = make_float2(qar[2 * i], qar[2 * i + 1]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            yp[c] = __ffma2_rn(ka, sp[i][c], yp[c]);
+            zp[c] = __ffma2_rn(qa, sp[i][c], zp[c]);
+          }
         }
-        s_red[p][0][rg][cg] = make_float4(ya.x, ya.y, yb.x, yb.y);
-        s_red[p][1][rg][cg] = make_float4(za.x, za.y, zb.x, zb.y);
+        s_red[p][0][rg][cg] = make_float4(yp[0].x + yp[0].y, yp[1].x + yp[1].y, yp[2].x + yp[2].y, yp[3].x + yp[3].y);
+        s_red[p][1][rg][cg] = make_float4(zp[0].x + zp[0].y, zp[1].x + zp[1].y, zp[2].x + zp[2].y, zp[3].x + zp[3].y);
         __syncthreads();
         if (tid < DV) {
           const int c4 = tid >> 2, lane4 = tid & 3;
@@ -223,19 +252,24 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
         }
         __syncthreads();
         const float4 u4 = reinterpret_cast<const float4 *>(s_u[p])[cg];
-        const float2 ua = make_float2(u4.x, u4.y), ub = make_float2(u4.z, u4.w);
+        const float2 uu[4] = {make_float2(u4.x, u4.x), make_float2(u4.y, u4.y),
+                              make_float2(u4.z, u4.z), make_float2(u4.w, u4.w)};
+        float alr[ROWS], kr[ROWS];
+        load_rows<ROWS>(&s_alpha[j][rg * ROWS], alr);
+        load_rows<ROWS>(&s_k[j][rg * ROWS], kr);
 #pragma unroll
-        for (int i = 0; i < ROWS; ++i) {
-          const int r = rg + i * RPP;
-          const float2 a = make_float2(s_alpha[j][r], s_alpha[j][r]);
-          const float2 kc = make_float2(s_k[j][r], s_k[j][r]);
-          sa[i] = __ffma2_rn(a, sa[i], __fmul2_rn(kc, ua));
-          sb2[i] = __ffma2_rn(a, sb2[i], __fmul2_rn(kc, ub));
+        for (int i = 0; i < RP; ++i) {
+          const float2 a = make_float2(alr[2 * i], alr[2 * i + 1]);
+          const float2 kc = make_float2(kr[2 * i], kr[2 * i + 1]);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) sp[i][c] = __ffma2_rn(a, sp[i][c], __fmul2_rn(kc, uu[c]));
         }
         if (t + 1 == acc)
 #pragma unroll
-          for (int i = 0; i < ROWS; ++i)
-            __stcs(&S4[(rg + i * RPP) * V4 + cg], make_float4(sa[i].x, sa[i].y, sb2[i].x, sb2[i].y));
+          for (int i = 0; i < RP; ++i) {
+            __stcs(&S4[(rg * ROWS + 2 * i) * V4 + cg], make_float4(sp[i][0].x, sp[i][1].x, sp[i][2].x, sp[i][3].x));
+            __stcs(&S4[(rg * ROWS + 2 * i + 1) * V4 + cg], make_float4(sp[i][0].y, sp[i][1].y, sp[i][2].y, sp[i][3].y));
+          }
       }
       __syncthreads();   // the staged group is overwritten by the next one
     }
@@ -261,7 +295,8 @@ static cudaError_t launch_decode_multi_t(const void *q, const void *k, const voi
                                          void *out, const int32_t *accept_len, int T_new,
                                          int64_t units, int H, int32_t *dev_status,
                                          cudaStream_t stream) {
-  constexpr int THREADS = 256;
+  // Two or more rows per thread (the row pairs of the paired FP32 units).
+  constexpr int THREADS = (DK == 32 && DV == 32) ? 128 : 256;
   if (units <= 0) return cudaSuccess;
   auto kern = decode_multi_kernel<DK, DV, THREADS, TIn>;
   const size_t smem = MultiLayout<DK, DV, TIn>::TOTAL;
