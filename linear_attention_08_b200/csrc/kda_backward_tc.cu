@@ -376,8 +376,10 @@ struct BItemLayout {
   static constexpr uint32_t BAR = EXTRA + 512;            // MMA done
   static constexpr uint32_t TBAR = BAR + 8;               // inputs landed
   static constexpr uint32_t CBAR = BAR + 16;              // [-dU; dO] landed (PART 0)
-  static constexpr uint32_t TMEM_SLOT = BAR + 24;
-  static constexpr uint32_t TOTAL = BAR + 32;
+  static constexpr uint32_t SBAR = BAR + 24;              // S0 (FP32) landed (PART 0)
+  static constexpr uint32_t TMEM_SLOT = BAR + 32;
+  static constexpr uint32_t TOTAL = BAR + 40;
+  static constexpr uint32_t S0F = 0;         //   PART 0, after the Gram: S0 FP32 [128][128] over GA, GB
   // PART 0 final partials (after the last MMAs): float [64][128] each
   static constexpr uint32_t PKM = GA, PDG = RU;
   // PART 1 final partials: float [64][128] and [32][128]
@@ -446,11 +448,13 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   uint64_t *bar = reinterpret_cast<uint64_t *>(sp + Lay::BAR);
   uint64_t *tbar = reinterpret_cast<uint64_t *>(sp + Lay::TBAR);
   uint64_t *cbar = reinterpret_cast<uint64_t *>(sp + Lay::CBAR);
+  uint64_t *s0bar = reinterpret_cast<uint64_t *>(sp + Lay::SBAR);
 
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(tbar, 1);
     mbar_init(cbar, 1);
+    mbar_init(s0bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, 512);
@@ -459,7 +463,8 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   tc::fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
   const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
-  uint32_t phase = 0, tphase = 0, cphase = 0;
+  uint32_t phase = 0, tphase = 0, cphase = 0, s0phase = 0;
+  bool s0pend = false;   // an S0 copy is in flight (PART 0)
   bool aborted = false;
   const int N = a.N;
   const int64_t total = a.pref[N] * H;
@@ -502,10 +507,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   // The per-chunk states and gradients come from L2 later; start them now.
   const float *S0src = j == 0 ? (a.init ? a.init + (size_t)unit * kD * kD : nullptr)
                               : a.ck + ((size_t)(ckb + j - 1) * H + h) * kD * kD;
-  if (PART == 0) {
-    if (S0src)
-      for (int e = tid; e < 512; e += kThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(S0src + 32 * e));
-  } else {
+  if (PART == 1) {
     const float *dtp = a.dtp + (size_t)p * 8192;
     for (int e = tid; e < 256; e += kThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(dtp + 32 * e));
   }
@@ -639,6 +641,15 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
   phase ^= 1;
   tc::fence_after_sync();
+  // The Gram operands are consumed: the state part's S0 (FP32) lands over them
+  // while the inverse is formed.
+  if (PART == 0 && !aborted && S0src) {
+    s0pend = true;
+    if (tid == 32) {
+      mbar_expect_tx(sb + Lay::SBAR, kD * kD * 4);
+      bulk_load(sb + Lay::S0F, S0src, kD * kD * 4, sb + Lay::SBAR);
+    }
+  }
   // Gram rows (lane m = row m, k rows only): M (scaled by beta_r, strictly lower),
   // and for PART 1 G unscaled.
   if (!aborted) {
@@ -760,22 +771,30 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   const size_t row_stride = (size_t)H * kD;   // elements between tokens in [T][H][128]
   const size_t base_row = ((size_t)t0 * H + h) * kD;
   if constexpr (PART == 0) {
-    // ---- S0 as the BF16 [ch][v] tile over the consumed Gram A tile ----
+    // ---- S0 as the BF16 [ch][v] tile (over the first half of its own FP32 copy) ----
+    // Warp w converts rows w, w + 8, ...: one float4 per lane per row, so both the
+    // FP32 reads and the tile writes are free of bank conflicts.
     if (!aborted) {
-      const int c = tid >> 1, h2 = tid & 1;
-      const float *s0r = S0src ? S0src + (size_t)c * kD + 64 * h2 : nullptr;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {   // 32 columns: all loads first, then the stores
-        float xs[32];
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 u4 = s0r ? *reinterpret_cast<const float4 *>(s0r + 32 * half + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-          xs[e] = u4.x; xs[e + 1] = u4.y; xs[e + 2] = u4.z; xs[e + 3] = u4.w;
+      float4 v4[16];
+      if (S0src) {
+        if (__syncthreads_or(!wait_timed(s0bar, s0phase, a.wait_ns))) {
+          aborted = true;
+        } else {
+          s0pend = false;
+          s0phase ^= 1;
         }
+        const float4 *src4 = reinterpret_cast<const float4 *>(sp + Lay::S0F);
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 8)
-          st_chunk_s(sp + Lay::S0T + tc::tile_offset(128, c, (64 * h2 + 32 * half + jj) >> 3), xs + jj);
+        for (int i = 0; i < 16; ++i) v4[i] = src4[(warp + 8 * i) * 32 + lane];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      __syncthreads();   // every FP32 row is in registers before the tile overwrites it
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        *reinterpret_cast<uint2 *>(sp + Lay::S0T + tc::tile_offset(128, warp + 8 * i, lane >> 1) + 8 * (lane & 1)) =
+            make_uint2(tc::pack_bf16(v4[i].x, v4[i].y), tc::pack_bf16(v4[i].z, v4[i].w));
       tc::fence_smem_to_async();
       __syncthreads();
     }
@@ -868,12 +887,25 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       for (int s2 = 0; s2 < 8; ++s2)
         tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::RU, 128, s2),
                      tc::desc_kmajor(sb + Lay::DST, 128, s2), idk, s2 > 0);
+#pragma unroll
+      for (int s2 = 0; s2 < 8; ++s2)   // dS_L S0^T: its diagonal is dd_c = sum_v dS_L[c, v] S0[c, v]
+        tc::mma_bf16(tmem + 128, tc::desc_kmajor(sb + Lay::DST, 128, s2),
+                     tc::desc_kmajor(sb + Lay::S0T, 128, s2), idk, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
     phase ^= 1;
     tc::fence_after_sync();
     float *dtp = a.dtp + (size_t)p * 8192;
+    if (!aborted && hw == 0) {   // the diagonal of dS_L S0^T: lane c takes column c
+      float x[32];
+      tc::tmem_ld32(tl + 128 + 32 * qd, x);
+      tc::tmem_wait_ld();
+      float dd = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e) dd = e == lane ? x[e] : dd;
+      s_dd[32 * qd + lane] = dd;
+    }
     if (!aborted) {
       if (qd < 2) {
         const int r = 32 * qd + lane;
@@ -1012,23 +1044,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         part += pdq[sw(r, ch)] + pdk[sw(r, ch)];
         extra += pkk[sw(r, ch)];
       }
-      if (S0src) {   // sum over this thread's half of the value columns
-        const float *s0r = S0src + (size_t)ch * kD + 64 * hf;
-        float4 s4[16];
-#pragma unroll
-        for (int cc = 0; cc < 16; ++cc) s4[cc] = *reinterpret_cast<const float4 *>(s0r + 4 * cc);
-        float dd = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-          float dv8[8];
-          unpack8(*reinterpret_cast<const uint4 *>(sp + Lay::DST + tc::tile_offset(128, ch, 8 * hf + cc)), dv8);
-          dd = fmaf(dv8[0], s4[2 * cc].x, dd); dd = fmaf(dv8[1], s4[2 * cc].y, dd);
-          dd = fmaf(dv8[2], s4[2 * cc].z, dd); dd = fmaf(dv8[3], s4[2 * cc].w, dd);
-          dd = fmaf(dv8[4], s4[2 * cc + 1].x, dd); dd = fmaf(dv8[5], s4[2 * cc + 1].y, dd);
-          dd = fmaf(dv8[6], s4[2 * cc + 1].z, dd); dd = fmaf(dv8[7], s4[2 * cc + 1].w, dd);
-        }
-        extra = fmaf(__expf(s_gam[sw(63, ch)]), dd, extra);
-      }
+      if (hf == 0) extra = fmaf(__expf(s_gam[sw(63, ch)]), s_dd[ch], extra);
       sred[hf * 128 + ch] = part;
       sred[256 + hf * 128 + ch] = extra;
       __syncthreads();
@@ -1360,6 +1376,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     wait_timed(bar, phase, a.wait_ns);
     wait_timed(tbar, tphase, a.wait_ns);
     if (PART == 0) wait_timed(cbar, cphase, a.wait_ns);
+    if (PART == 0 && s0pend) wait_timed(s0bar, s0phase, a.wait_ns);
   }
   tc::fence_before_sync();
   __syncthreads();
