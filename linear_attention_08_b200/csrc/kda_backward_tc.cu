@@ -49,11 +49,12 @@
 
 namespace kda {
 
-cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
-                                 const float *beta, const float *init, const int32_t *cu, void *out,
-                                 float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
-                                 void *workspace, size_t ws_bytes, int32_t *dev_status,
-                                 cudaStream_t stream, int num_sms);
+cudaError_t launch_prefill_split_ex(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const float *init, const int32_t *cu,
+                                    void *out, float *fin, int64_t interval, float *ck,
+                                    uint8_t *ck_tiles, int N, int H, int64_t T, void *workspace,
+                                    size_t ws_bytes, int32_t *dev_status, cudaStream_t stream,
+                                    int num_sms);
 size_t split_packet_bytes();
 bool prefill_split_supported(int N);
 
@@ -379,7 +380,6 @@ struct BItemLayout {
   static constexpr uint32_t SBAR = BAR + 24;              // S0 (FP32) landed (PART 0)
   static constexpr uint32_t TMEM_SLOT = BAR + 32;
   static constexpr uint32_t TOTAL = BAR + 40;
-  static constexpr uint32_t S0F = 0;         //   PART 0, after the Gram: S0 FP32 [128][128] over GA, GB
   // PART 0 final partials (after the last MMAs): float [64][128] each
   static constexpr uint32_t PKM = GA, PDG = RU;
   // PART 1 final partials: float [64][128] and [32][128]
@@ -407,7 +407,9 @@ __device__ __forceinline__ void st_chunk_s(uint8_t *dst, const float *x) {
 }
 
 struct BwdItemArgs {
-  const float *beta, *init, *ck;
+  const float *beta;
+  const uint8_t *s0_init;      // BF16 state tiles [N*H] of the initial states, or null
+  const uint8_t *s0_ck;        // BF16 state tiles at every full chunk end, [chunk][H]
   const int32_t *cu;
   const int64_t *pref;         // [N+1] chunks before sequence n
   const int64_t *prefck;       // [N+1] full chunks (stored states) before sequence n
@@ -505,8 +507,8 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   }
   cp_async_commit();
   // The per-chunk states and gradients come from L2 later; start them now.
-  const float *S0src = j == 0 ? (a.init ? a.init + (size_t)unit * kD * kD : nullptr)
-                              : a.ck + ((size_t)(ckb + j - 1) * H + h) * kD * kD;
+  const uint8_t *S0src = j == 0 ? (a.s0_init ? a.s0_init + (size_t)unit * 32768 : nullptr)
+                                : a.s0_ck + ((size_t)(ckb + j - 1) * H + h) * 32768;
   if (PART == 1) {
     const float *dtp = a.dtp + (size_t)p * 8192;
     for (int e = tid; e < 256; e += kThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(dtp + 32 * e));
@@ -641,13 +643,13 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
   phase ^= 1;
   tc::fence_after_sync();
-  // The Gram operands are consumed: the state part's S0 (FP32) lands over them
-  // while the inverse is formed.
+  // The Gram A tile is consumed: the state part's S0 (the BF16 operand tile)
+  // lands over it while the inverse is formed.
   if (PART == 0 && !aborted && S0src) {
     s0pend = true;
     if (tid == 32) {
-      mbar_expect_tx(sb + Lay::SBAR, kD * kD * 4);
-      bulk_load(sb + Lay::S0F, S0src, kD * kD * 4, sb + Lay::SBAR);
+      mbar_expect_tx(sb + Lay::SBAR, 32768);
+      bulk_load(sb + Lay::S0T, S0src, 32768, sb + Lay::SBAR);
     }
   }
   // Gram rows (lane m = row m, k rows only): M (scaled by beta_r, strictly lower),
@@ -771,11 +773,8 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   const size_t row_stride = (size_t)H * kD;   // elements between tokens in [T][H][128]
   const size_t base_row = ((size_t)t0 * H + h) * kD;
   if constexpr (PART == 0) {
-    // ---- S0 as the BF16 [ch][v] tile (over the first half of its own FP32 copy) ----
-    // Warp w converts rows w, w + 8, ...: one float4 per lane per row, so both the
-    // FP32 reads and the tile writes are free of bank conflicts.
+    // ---- S0 as the BF16 [ch][v] tile: copied in, or zero without an initial state ----
     if (!aborted) {
-      float4 v4[16];
       if (S0src) {
         if (__syncthreads_or(!wait_timed(s0bar, s0phase, a.wait_ns))) {
           aborted = true;
@@ -783,20 +782,12 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
           s0pend = false;
           s0phase ^= 1;
         }
-        const float4 *src4 = reinterpret_cast<const float4 *>(sp + Lay::S0F);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v4[i] = src4[(warp + 8 * i) * 32 + lane];
       } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int e = tid; e < 2048; e += kThreads)
+          reinterpret_cast<uint4 *>(sp + Lay::S0T)[e] = make_uint4(0, 0, 0, 0);
+        tc::fence_smem_to_async();
+        __syncthreads();
       }
-      __syncthreads();   // every FP32 row is in registers before the tile overwrites it
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        *reinterpret_cast<uint2 *>(sp + Lay::S0T + tc::tile_offset(128, warp + 8 * i, lane >> 1) + 8 * (lane & 1)) =
-            make_uint2(tc::pack_bf16(v4[i].x, v4[i].y), tc::pack_bf16(v4[i].z, v4[i].w));
-      tc::fence_smem_to_async();
-      __syncthreads();
     }
     // ---- R = V - Ktilde S0 (TMEM columns 128..255) ----
     if (!aborted && tid == 0) {
@@ -1414,10 +1405,24 @@ __global__ void bwd_prefix_kernel(const int32_t *__restrict__ cu, int N, int64_t
   }
 }
 
+// The initial states as BF16 operand tiles, in the layout of the forward's
+// checkpoint tiles (128-byte swizzled [key channel][value column]).
+__global__ void __launch_bounds__(kThreads)
+bwd_init_tiles_kernel(const float *__restrict__ init, uint8_t *__restrict__ tiles) {
+  const int unit = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float *src = init + (size_t)unit * kD * kD;
+  uint8_t *dst = tiles + (size_t)unit * 32768;
+  for (int row = warp; row < kD; row += kThreads / 32) {
+    const float4 x = reinterpret_cast<const float4 *>(src + (size_t)row * kD)[lane];
+    *reinterpret_cast<uint2 *>(dst + tc::tile_offset(128, row, lane >> 1) + 8 * (lane & 1)) =
+        make_uint2(tc::pack_bf16(x.x, x.y), tc::pack_bf16(x.z, x.w));
+  }
+}
+
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdWs {
-  size_t pk, ck, dsl, ndu, dot, dtp, oscr, pref, prefck, total;
+  size_t pk, ck, s0i, dsl, ndu, dot, dtp, oscr, pref, prefck, total;
 };
 
 BwdWs bwd_ws_layout(int N, int H, int64_t T) {
@@ -1425,7 +1430,8 @@ BwdWs bwd_ws_layout(int N, int H, int64_t T) {
   BwdWs w;
   size_t off = 0;
   w.pk = off;     off += align256(P * Pk::BYTES + 256);
-  w.ck = off;     off += align256((size_t)(T / kC) * H * kD * kD * 4);
+  w.ck = off;     off += align256((size_t)(T / kC) * H * 32768);      // BF16 state tiles
+  w.s0i = off;    off += align256((size_t)N * H * 32768);             // initial states, same layout
   w.dsl = off;    off += align256(P * 32768);
   w.ndu = off;    off += align256(P * 16384);
   w.dot = off;    off += align256(P * 16384);
@@ -1455,7 +1461,8 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   const BwdWs w = bwd_ws_layout(N, H, T);
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(workspace) + 255) & ~(uintptr_t)255);
   uint8_t *pk = base + w.pk;
-  float *ck = reinterpret_cast<float *>(base + w.ck);
+  uint8_t *ck = base + w.ck;
+  uint8_t *s0i = base + w.s0i;
   uint8_t *dsl = base + w.dsl;
   uint8_t *ndu = base + w.ndu;
   uint8_t *dot = base + w.dot;
@@ -1467,9 +1474,13 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
 
   // Forward recomputation: the two-pass prefill in one window keeps every
   // intra-chunk packet in the workspace and stores the state every 64 tokens.
-  cudaError_t e = launch_prefill_split(q, k, v, g, beta, init, cu, oscr, nullptr, kC, ck, N, H, T,
-                                       pk, w.ck - w.pk, dev_status, stream, num_sms);
+  cudaError_t e = launch_prefill_split_ex(q, k, v, g, beta, init, cu, oscr, nullptr, kC, nullptr,
+                                          ck, N, H, T, pk, w.ck - w.pk, dev_status, stream, num_sms);
   if (e != cudaSuccess) return e;
+  if (init) {
+    bwd_init_tiles_kernel<<<(unsigned)((int64_t)N * H), kThreads, 0, stream>>>(init, s0i);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   bwd_prefix_kernel<<<1, 32, 0, stream>>>(cu, N, pref, prefck);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -1493,7 +1504,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   BwdItemArgs a;
-  a.beta = beta; a.init = init; a.ck = ck; a.cu = cu; a.pref = pref; a.prefck = prefck;
+  a.beta = beta; a.s0_init = init ? s0i : nullptr; a.s0_ck = ck; a.cu = cu; a.pref = pref; a.prefck = prefck;
   a.dsl = dsl; a.ndu = ndu; a.dot = dot; a.dtp = dtp; a.q = q; a.k = k;
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
   a.N = N; a.H = H; a.dev_status = dev_status; a.wait_ns = wait_ns;

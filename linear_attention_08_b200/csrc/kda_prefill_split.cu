@@ -632,8 +632,8 @@ template <int DVS>
 __global__ void __launch_bounds__(kThreads, 1)
 chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *__restrict__ cu,
              __nv_bfloat16 *__restrict__ out, float *carry, int64_t interval, float *__restrict__ ck,
-             int N, int H, int64_t jw0, int64_t wc, int first_window, int32_t *dev_status,
-             uint64_t wait_ns) {
+             uint8_t *__restrict__ ck_tiles, int N, int H, int64_t jw0, int64_t wc, int first_window,
+             int32_t *dev_status, uint64_t wait_ns) {
   using Lay = ChainLayout<DVS>;
   constexpr int NCOL = DVS / 2;
   constexpr int NST = Lay::NST;
@@ -776,6 +776,7 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
   };
   int64_t t0_prev = 0;
   int L_prev = 0;
+  int64_t tile_slot = -1;   // a checkpoint to copy out of S_T (BF16 tile mode)
   for (int64_t jl = 0; jl < cnt; ++jl) {
     const int s = (int)(jl % NST);
     const uint32_t st = sb + Lay::STAGE0 + s * Lay::STAGE;
@@ -852,6 +853,7 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
       tc::mma_commit(sb + Lay::OBAR);
     }
     const float d = reinterpret_cast<const float *>(sp + (st - sb) + Lay::D)[crow];
+    if (tid == 32) bulk_wait_read();   // the last checkpoint copy has left S_T
     if (__syncthreads_or(!wait_timed(sbar, sphase, wait_ns))) { aborted = true; break; }
     sphase ^= 1;
     tc::fence_after_sync();
@@ -874,7 +876,8 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
       tc::tmem_wait_st();
       since_ck += L;
       if (interval > 0 && since_ck == interval) {
-        store_state(ck, ck_slot++);
+        if (ck_tiles) tile_slot = ck_slot++;
+        else store_state(ck, ck_slot++);
         since_ck = 0;
       }
     }
@@ -883,7 +886,16 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
     tc::fence_smem_to_async();
     tc::fence_before_sync();
     __syncthreads();
+    if (tile_slot >= 0) {   // the BF16 state tile (this CTA's column block) as the checkpoint
+      if (tid == 32) {
+        bulk_store(ck_tiles + ((size_t)tile_slot * H + h) * (kDK * kDV * 2) + (size_t)y * (128 * DVS * 2),
+                   sb + Lay::S_T, 128 * DVS * 2);
+        bulk_commit();
+      }
+      tile_slot = -1;
+    }
   }
+  if (tid == 32) bulk_wait_all();
   if (!aborted && cnt > 0) {
     if (__syncthreads_or(!wait_timed(obar, ophase, wait_ns))) aborted = true;
     else {
@@ -912,15 +924,16 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
 
 template <int DVS>
 cudaError_t launch_chain(const uint8_t *ws, const float *init, const int32_t *cu, void *out,
-                         float *carry, int64_t interval, float *ck, int N, int H, int64_t jw0,
-                         int64_t wc, int first, int32_t *dev_status, cudaStream_t stream) {
+                         float *carry, int64_t interval, float *ck, uint8_t *ck_tiles, int N, int H,
+                         int64_t jw0, int64_t wc, int first, int32_t *dev_status,
+                         cudaStream_t stream) {
   const size_t smem = ChainLayout<DVS>::TOTAL + 1024;
   auto kern = chain_kernel<DVS>;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   dim3 grid((unsigned)((int64_t)N * H), (unsigned)(kDV / DVS));
-  kern<<<grid, kThreads, smem, stream>>>(ws, init, cu, (__nv_bfloat16 *)out, carry, interval, ck, N,
-                                         H, jw0, wc, first, dev_status, 2000000000ull);
+  kern<<<grid, kThreads, smem, stream>>>(ws, init, cu, (__nv_bfloat16 *)out, carry, interval, ck,
+                                         ck_tiles, N, H, jw0, wc, first, dev_status, 2000000000ull);
   return cudaGetLastError();
 }
 
@@ -942,11 +955,15 @@ size_t split_workspace_full(int N, int H, int64_t T, bool have_final) {
 // Two-pass prefill over windows of chunks.  Packets of a window are stored
 // sequence by sequence, head by head, chunk by chunk: packet (n, h, j) sits at
 // index H * sum_{m<n} c_m + h * c_n + (j - jw0), c_m = chunks of m in the window.
-cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
-                                 const float *beta, const float *init, const int32_t *cu, void *out,
-                                 float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
-                                 void *workspace, size_t ws_bytes, int32_t *dev_status,
-                                 cudaStream_t stream, int num_sms) {
+// Checkpoints go to `ck` as FP32 [128][128] states, or, with `ck_tiles` set
+// (and `ck` null), as the chain's BF16 state tiles (32 KB each, the 128-byte
+// swizzled [key channel][value column] MMA operand layout).
+cudaError_t launch_prefill_split_ex(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const float *init, const int32_t *cu,
+                                    void *out, float *fin, int64_t interval, float *ck,
+                                    uint8_t *ck_tiles, int N, int H, int64_t T, void *workspace,
+                                    size_t ws_bytes, int32_t *dev_status, cudaStream_t stream,
+                                    int num_sms) {
   if (!prefill_split_supported(N)) return cudaErrorNotSupported;
   uintptr_t base = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~(uintptr_t)255;
   const size_t lost = base - reinterpret_cast<uintptr_t>(workspace);
@@ -991,13 +1008,22 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
     }
     // One window: no carry needed unless the caller wants the final state.
     float *c = (windows == 1) ? fin : carry;
-    err = narrow ? launch_chain<64>(ws, init, cu, out, c, interval, ck, N, H, jw0, wc, w == 0,
-                                    dev_status, stream)
-                 : launch_chain<128>(ws, init, cu, out, c, interval, ck, N, H, jw0, wc, w == 0,
-                                     dev_status, stream);
+    err = narrow ? launch_chain<64>(ws, init, cu, out, c, interval, ck, ck_tiles, N, H, jw0, wc,
+                                    w == 0, dev_status, stream)
+                 : launch_chain<128>(ws, init, cu, out, c, interval, ck, ck_tiles, N, H, jw0, wc,
+                                     w == 0, dev_status, stream);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *init, const int32_t *cu, void *out,
+                                 float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
+                                 void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                 cudaStream_t stream, int num_sms) {
+  return launch_prefill_split_ex(q, k, v, g, beta, init, cu, out, fin, interval, ck, nullptr, N, H,
+                                 T, workspace, ws_bytes, dev_status, stream, num_sms);
 }
 
 }  // namespace kda
