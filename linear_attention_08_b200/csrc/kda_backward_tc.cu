@@ -1227,7 +1227,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     // sign, Gram B rows for the others), so that the pair's terms, which the
     // reverse cumulative sum below sets against each other, cancel to FP32
     // accumulation precision.  Lanes 64..127 (Xq) and lanes 0..63 (X, Y and the
-    // cross rows) work at once, each half on its own dGam part.
+    // cross rows) work at once, each half on its own dGam part.  The parts of
+    // dq, dk and dg go onto what the state part wrote as reductions in global
+    // memory (no load, so no wait for the earlier values).
     float4 *qdg4 = reinterpret_cast<float4 *>(sp + Lay::QDG);   // dGam from the q side
     float4 *kdg4 = reinterpret_cast<float4 *>(sp + Lay::KMC);   // dGam from the k sides
     const float4 *g4 = reinterpret_cast<const float4 *>(s_gam);
@@ -1246,11 +1248,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         float xq[32];
         tc::tmem_ld32(tl + 0 + c0, xq);
         tc::tmem_wait_ld();
-        const size_t off = base_row + (size_t)r * row_stride + c0;
-        float4 old[8];
-        if (in)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) old[e] = *reinterpret_cast<const float4 *>(dqp + off + 4 * e);
+        float4 *dst = reinterpret_cast<float4 *>(dqp + base_row + (size_t)r * row_stride + c0);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {   // 8 channels: one tile chunk
           float ga[8];
@@ -1262,13 +1260,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
             const float4 xqv = make_float4(xq[c], xq[c + 1], xq[c + 2], xq[c + 3]);
             const float4 add = f4mul(f4exp(make_float4(gam.x - gref.x, gam.y - gref.y, gam.z - gref.z, gam.w - gref.w)), xqv);
             qdg4[sw4(r, F)] = f4mul(make_float4(ga[4 * hf], ga[4 * hf + 1], ga[4 * hf + 2], ga[4 * hf + 3]), xqv);
-            const int e = 2 * u + hf;
-            old[e].x += add.x; old[e].y += add.y; old[e].z += add.z; old[e].w += add.w;
+            if (in) atomicAdd(dst + 2 * u + hf, add);   // onto the state part's dq, no read back
           }
         }
-        if (in)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) *reinterpret_cast<float4 *>(dqp + off + 4 * e) = old[e];
       }
     } else if (!aborted) {
       const int t = 32 * qd + lane;
@@ -1283,11 +1277,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         tc::tmem_ld32(tl + 128 + c0, yo);
         tc::tmem_ld32(tl + 256 + c0, yc);   // cross rows (first-half keys, second-half reference)
         tc::tmem_wait_ld();
-        const size_t off = base_row + (size_t)t * row_stride + c0;
-        float4 old[8];
-        if (in)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) old[e] = *reinterpret_cast<const float4 *>(dkp_ + off + 4 * e);
+        float4 *dst = reinterpret_cast<float4 *>(dkp_ + base_row + (size_t)t * row_stride + c0);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           float ga[8], gb[8], gc[8];
@@ -1314,14 +1304,10 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
               pb = make_float4(pb.x + pc.x, pb.y + pc.y, pb.z + pc.z, pb.w + pc.w);
             }
             kdg4[sw4(t, F)] = make_float4(pa.x - pb.x, pa.y - pb.y, pa.z - pb.z, pa.w - pb.w);
-            const int e = 2 * u + hf;
-            old[e].x += dkp.x + dkm.x; old[e].y += dkp.y + dkm.y;
-            old[e].z += dkp.z + dkm.z; old[e].w += dkp.w + dkm.w;
+            if (in)
+              atomicAdd(dst + 2 * u + hf, make_float4(dkp.x + dkm.x, dkp.y + dkm.y, dkp.z + dkm.z, dkp.w + dkm.w));
           }
         }
-        if (in)
-#pragma unroll
-          for (int e = 0; e < 8; ++e) *reinterpret_cast<float4 *>(dkp_ + off + 4 * e) = old[e];
       }
     }
     __syncthreads();
@@ -1337,20 +1323,10 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       __syncthreads();
       float *dgp = a.dg;
       float suffix = hf == 0 ? sred[128 + ch] : 0.f;
-#pragma unroll 1
-      for (int blk = 1; blk >= 0; --blk) {   // 16 rows at a time: their loads issue together
-        float prev[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const int r = 32 * hf + 16 * blk + u;
-          prev[u] = r < L ? dgp[base_row + (size_t)r * row_stride + ch] : 0.f;
-        }
-#pragma unroll
-        for (int u = 15; u >= 0; --u) {
-          const int r = 32 * hf + 16 * blk + u;
-          suffix += qdg[sw(r, ch)] + kdg[sw(r, ch)];
-          if (r < L) dgp[base_row + (size_t)r * row_stride + ch] = prev[u] + suffix;
-        }
+#pragma unroll 8
+      for (int r = 32 * hf + 31; r >= 32 * hf; --r) {
+        suffix += qdg[sw(r, ch)] + kdg[sw(r, ch)];
+        if (r < L) atomicAdd(dgp + base_row + (size_t)r * row_stride + ch, suffix);
       }
     }
     if (!aborted && tid < L) a.dbeta[(size_t)(t0 + tid) * H + h] = s_db[tid];
