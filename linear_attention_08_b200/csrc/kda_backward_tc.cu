@@ -471,41 +471,73 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   const int N = a.N;
   const int64_t total = a.pref[N] * H;
 
-  // Items (sequence, head, chunk) in packet order: p = H pref[n] + h c_n + j.
-  for (int64_t p = blockIdx.x; p < total && !aborted; p += gridDim.x) {
-  int lo = 0, hi = N - 1;
-  while (lo < hi) {   // last sequence whose first packet is at or before p
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.pref[mid] * H <= p) lo = mid; else hi = mid - 1;
-  }
-  const int n = lo;
-  const int64_t nch = a.pref[n + 1] - a.pref[n];
-  const int64_t rem = p - a.pref[n] * H;
-  const int h = (int)(rem / nch);
-  const int64_t j = rem - (int64_t)h * nch;
-  const int unit = n * H + h;
-  const int64_t ckb = a.prefck[n];
-  const int64_t t0 = (int64_t)a.cu[n] + kC * j;
-  const int64_t T_n = (int64_t)a.cu[n + 1] - a.cu[n];
-  const int L = (int)(T_n - kC * j < kC ? T_n - kC * j : kC);
-
-  // Inputs: q, k into the Gram A tile, g into its staging rows, v (PART 0).
-  if (tid == 32) {
-    mbar_expect_tx(sb + Lay::TBAR, 65536 + (PART == 0 ? 16384 : 0));
-    tma_load_3d(sb + Lay::GST, &maps.g, 0, h, (int)t0, sb + Lay::TBAR);
+  // Item pp (sequence, head, chunk) in packet order: pp = H pref[n] + h c_n + j.
+  auto locate = [&](int64_t pp, int &n_, int &h_, int64_t &j_, int64_t &t0_, int &L_) {
+    int lo = 0, hi = N - 1;
+    while (lo < hi) {   // last sequence whose first packet is at or before pp
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.pref[mid] * H <= pp) lo = mid; else hi = mid - 1;
+    }
+    n_ = lo;
+    const int64_t nch = a.pref[lo + 1] - a.pref[lo];
+    const int64_t rem = pp - a.pref[lo] * H;
+    h_ = (int)(rem / nch);
+    j_ = rem - (int64_t)h_ * nch;
+    t0_ = (int64_t)a.cu[lo] + kC * j_;
+    const int64_t T_n = (int64_t)a.cu[lo + 1] - a.cu[lo];
+    L_ = (int)(T_n - kC * j_ < kC ? T_n - kC * j_ : kC);
+  };
+  // Inputs: g into its staging rows and beta (both parts), q, k into the Gram A
+  // tile, v (the state part).  `arrive`: this issue completes the barrier
+  // phase's arrival (the other only adds its bytes).
+  auto issue_g = [&](int h_, int64_t t0_, int L_, bool arrive, uint32_t bytes) {
+    if (tid == 32) {
+      if (arrive) mbar_expect_tx(sb + Lay::TBAR, bytes);
+      else mbar_add_tx(sb + Lay::TBAR, bytes);
+      tma_load_3d(sb + Lay::GST, &maps.g, 0, h_, (int)t0_, sb + Lay::TBAR);
+    }
+    if (tid >= 64 && tid < 64 + kC) {
+      const int r = tid - 64;
+      const bool ok = r < L_;
+      cp_async4(sb + Lay::BETA + 4 * r, a.beta + (ok ? (size_t)(t0_ + r) * H + h_ : 0), ok);
+    }
+    cp_async_commit();
+  };
+  auto issue_kqv = [&](int h_, int64_t t0_) {   // tid 32, after its expect_tx
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h, (int)t0, sb + Lay::TBAR);
-      tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h, (int)t0, sb + Lay::TBAR);
-      if (PART == 0) tma_load_3d(sb + Lay::VT + b * 8192, &maps.v, 64 * b, h, (int)t0, sb + Lay::TBAR);
+      tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
+      tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
+      if (PART == 0) tma_load_3d(sb + Lay::VT + b * 8192, &maps.v, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
+    }
+  };
+  // Issued during the previous item's reverse scan: g and beta (state part),
+  // all inputs (Gram part).
+  bool pre = false;
+  int n2 = 0, h2 = 0, L2 = 0;   // the next item, located while the current one's inputs land
+  int64_t j2 = 0, t02 = 0;
+  if ((int64_t)blockIdx.x < total) locate(blockIdx.x, n2, h2, j2, t02, L2);
+
+  for (int64_t p = blockIdx.x; p < total && !aborted; p += gridDim.x) {
+  const int n = n2, h = h2, L = L2;
+  const int64_t j = j2, t0 = t02;
+  const int unit = n * H + h;
+  const int64_t ckb = a.prefck[n];
+
+  if (PART == 1 && !pre) {
+    issue_g(h, t0, L, true, 65536);
+    if (tid == 32) issue_kqv(h, t0);
+  }
+  if (PART == 0) {
+    if (!pre) issue_g(h, t0, L, false, 32768);
+    if (tid == 32) {
+      mbar_expect_tx(sb + Lay::TBAR, 32768 + 16384);
+      issue_kqv(h, t0);
     }
   }
-  if (tid >= 64 && tid < 64 + kC) {
-    const int r = tid - 64;
-    const bool ok = r < L;
-    cp_async4(sb + Lay::BETA + 4 * r, a.beta + (ok ? (size_t)(t0 + r) * H + h : 0), ok);
-  }
-  cp_async_commit();
+  pre = false;
+  const bool has_next = p + gridDim.x < total;
+  if (has_next) locate(p + gridDim.x, n2, h2, j2, t02, L2);
   // The per-chunk states and gradients come from L2 later; start them now.
   const uint8_t *S0src = j == 0 ? (a.s0_init ? a.s0_init + (size_t)unit * 32768 : nullptr)
                                 : a.s0_ck + ((size_t)(ckb + j - 1) * H + h) * 32768;
@@ -1021,7 +1053,14 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         }
       }
     }
+    // Gam leaves its rows for the next item's g; the scan keeps exp(Gam_63).
+    const float e63 = tid < 128 ? __expf(s_gam[sw(63, tid)]) : 0.f;
+    tc::fence_smem_to_async();
     __syncthreads();
+    if (!aborted && has_next) {
+      issue_g(h2, t02, L2, false, 32768);
+      pre = true;
+    }
     // dg = reverse cumulative sum of dGam plus the Gam_63 terms (sum_r k dk-_r from
     // Khat, d * sum_v dS_L S0).  Two threads per channel, 32 rows each.
     float *sred = s_Y;   // [2][128] partial sums, [2][128] partial extras (the solve scratch)
@@ -1035,7 +1074,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         part += pdq[sw(r, ch)] + pdk[sw(r, ch)];
         extra += pkk[sw(r, ch)];
       }
-      if (hf == 0) extra = fmaf(__expf(s_gam[sw(63, ch)]), s_dd[ch], extra);
+      if (hf == 0) extra = fmaf(e63, s_dd[ch], extra);
       sred[hf * 128 + ch] = part;
       sred[256 + hf * 128 + ch] = extra;
       __syncthreads();
@@ -1310,7 +1349,14 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         }
       }
     }
+    tc::fence_smem_to_async();
     __syncthreads();
+    // The Gram tiles and Gam are consumed: the next item's inputs land during the scan.
+    if (!aborted && has_next) {
+      issue_g(h2, t02, L2, true, 65536);
+      if (tid == 32) issue_kqv(h2, t02);
+      pre = true;
+    }
     // dg += reverse cumulative sum of dGam: two threads per channel, 32 rows each.
     if (!aborted) {
       const int ch = tid & 127, hf = tid >> 7;
