@@ -982,6 +982,17 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
                      tc::desc_kmajor(sb + Lay::S0T, 128, s2), id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
+    // The raw q (lanes 64..127) or k (lanes 0..63) of this thread's token and
+    // channel half, loaded while the product runs.
+    uint4 raw[8];
+    {
+      const int rr = qd >= 2 ? 32 * (qd - 2) + lane : 32 * qd + lane;
+      const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(qd >= 2 ? a.q : a.k) +
+                                 base_row + (size_t)rr * row_stride + hw * 64;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        raw[u] = rr < L ? *reinterpret_cast<const uint4 *>(src + 8 * u) : make_uint4(0, 0, 0, 0);
+    }
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
     phase ^= 1;
     tc::fence_after_sync();
@@ -991,8 +1002,6 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     float4 *pdq4 = reinterpret_cast<float4 *>(sp + Lay::PKM);   // q (dq from Qtilde)
     float4 *pdk4 = reinterpret_cast<float4 *>(sp + Lay::PDG);   // k (dk+ - dk-)
     float4 *pkk4 = reinterpret_cast<float4 *>(sp + Lay::BT2);   // k (dk from Khat): the dGam_63 extra
-    const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(a.q);
-    const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(a.k);
     const float4 *g4 = reinterpret_cast<const float4 *>(s_gam);
     if (!aborted && qd >= 2) {
       const int r = 32 * (qd - 2) + lane;
@@ -1002,14 +1011,10 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(aq + 32));
       tc::tmem_wait_ld();
       const size_t off = base_row + (size_t)r * row_stride + hw * 64;
-      uint4 qraw[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        qraw[u] = in ? *reinterpret_cast<const uint4 *>(qb + off + 8 * u) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         float qv[8];
-        unpack8(qraw[u], qv);
+        unpack8(raw[u], qv);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {   // channels hw*64 + 8u + 4hf .. +3
           const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
@@ -1028,14 +1033,10 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       tc::tmem_ld32(tl + 256 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ah + 32));
       tc::tmem_wait_ld();
       const size_t off = base_row + (size_t)r * row_stride + hw * 64;
-      uint4 kraw[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        kraw[u] = in ? *reinterpret_cast<const uint4 *>(kb + off + 8 * u) : make_uint4(0, 0, 0, 0);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         float kv[8];
-        unpack8(kraw[u], kv);
+        unpack8(raw[u], kv);
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
