@@ -88,6 +88,10 @@ KERNEL_SOURCES = {
     # two-pass path: intra-chunk pass + chain pass, one prefill call = one launch of each
     "prefill_split": ("kda_prefill_split.cu", "kda_tc_util.cuh", "kda_tma.cuh", "kda_common.cuh"),
     "prefill_simt": ("kda_prefill_simt.cu", "kda_common.cuh"),
+    # chunked tensor-core backward: the forward recomputation (two-pass prefill)
+    # and the backward's own kernels, one call
+    "backward_tc": ("kda_backward_tc.cu", "kda_prefill_split.cu", "kda_tc_util.cuh", "kda_tma.cuh",
+                    "kda_common.cuh"),
 }
 PATH_KERNEL = {2: "prefill_split", 1: "prefill_tc", 0: "prefill_simt"}
 
@@ -559,7 +563,9 @@ def run_ours(args, rank, world, local):
                            "d": bwd["D"], "dtype": "bf16 inputs, fp32 gradients"},
                 "roofline": {"bound": "hbm", "achieved": bgbs, "peak": hbm, "unit": "GB/s",
                              "frac": bgbs / hbm, "kernel": bwd["kernel"],
-                             "note": "operator bytes (inputs, upstream gradients, gradients, states) over the whole call"}}
+                             "traffic": ncu_traffic(bwd["kernel"]) if bwd["kernel"] == "backward_tc" else None,
+                             "note": "operator bytes (inputs, upstream gradients, gradients, states) over the whole call; "
+                                     "traffic = DRAM bytes of all eight kernels of one call"}}
     if dec is not None:
         dgbs = dec["bytes"] / (dec["ms"] / dec["launches"] / 1e3) / 1e9 / dec["launches"]
         dobj = {
