@@ -44,6 +44,15 @@ __device__ __forceinline__ void load_rows(const float *src, float *dst) {
   }
 }
 
+// Four consecutive values as floats (8- or 16-byte aligned).
+__device__ __forceinline__ float4 load4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 load4(const __nv_bfloat16 *p) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(p);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
 template <int DK, int DV, typename TIn>
 struct MultiLayout {
   static constexpr int G = kMultiGroup;
@@ -163,59 +172,60 @@ decode_multi_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k,
 
     for (int t0 = 0; t0 < T_new; t0 += G) {
       const int cnt = T_new - t0 < G ? T_new - t0 : G;
-      // Stage the group: gates and products for every token at once.  The
-      // first group comes from the prefetched raw copies, later ones (drafts
-      // longer than a group) straight from global memory.
-      if (t0 == 0) {
+      // Stage the group: gates, alpha k, alpha q and q . k for every token at
+      // once, four consecutive channels per thread (the QK lanes holding one
+      // token reduce q . k by shuffles).  The first group comes from the
+      // prefetched raw copies, later ones (drafts longer than a group)
+      // straight from global memory.
+      {
+        constexpr int QK = DK / 4, QV = DV / 4;   // channel quads per token row
+        static_assert(QK <= 32 && 32 % QK == 0, "a token's quads share one warp");
         const TIn *rq = reinterpret_cast<const TIn *>(smem_raw + Lay::RAW_Q);
         const TIn *rk = reinterpret_cast<const TIn *>(smem_raw + Lay::RAW_K);
         const TIn *rv = reinterpret_cast<const TIn *>(smem_raw + Lay::RAW_V);
-        const float *rg_ = reinterpret_cast<const float *>(smem_raw + Lay::RAW_G);
-        for (int e = tid; e < cnt * DK; e += THREADS) {
-          const int j = e / DK, c = e % DK;
-          const float kc = to_f32(rk[j * DK + c]), qc = to_f32(rq[j * DK + c]);
-          const float a = __expf(rg_[j * DK + c]);
-          s_alpha[j][c] = a;
-          s_k[j][c] = kc;
-          s_ka[j][c] = a * kc;
-          s_qa[j][c] = qc;     // q for now; becomes alpha * q below
-        }
-        for (int e = tid; e < cnt * DV; e += THREADS) {
-          const int j = e / DV, c = e % DV;
-          s_v[j][c] = to_f32(rv[j * DV + c]);
-        }
-        if (tid < cnt) s_beta[tid] = reinterpret_cast<const float *>(smem_raw + Lay::RAW_B)[tid];
-        __syncthreads();
-        const int64_t nx = u + gridDim.x;   // the raw and state buffers are free now
-        if (nx < units) prefetch(nx);
-      } else {
-        for (int e = tid; e < cnt * DK; e += THREADS) {
-          const int j = e / DK, c = e % DK;
-          const size_t off = (((size_t)n * T_new + t0 + j) * H + h) * DK + c;
-          const float kc = to_f32(k[off]), qc = to_f32(q[off]);
-          const float a = __expf(g[off]);
-          s_alpha[j][c] = a;
-          s_k[j][c] = kc;
-          s_ka[j][c] = a * kc;
-          s_qa[j][c] = qc;
-        }
-        for (int e = tid; e < cnt * DV; e += THREADS) {
-          const int j = e / DV, c = e % DV;
-          s_v[j][c] = to_f32(v[(((size_t)n * T_new + t0 + j) * H + h) * DV + c]);
-        }
-        if (tid < cnt) s_beta[tid] = beta[((size_t)n * T_new + t0 + tid) * H + h];
-        __syncthreads();
-      }
-      // q . k per token (one warp per token), then q <- alpha * q
-      for (int j = warp; j < cnt; j += THREADS / 32) {
-        float qk = 0.f;
-        for (int c = lane; c < DK; c += 32) qk += s_qa[j][c] * s_k[j][c];
+        const float *rgp = reinterpret_cast<const float *>(smem_raw + Lay::RAW_G);
+        const size_t tok0 = ((size_t)n * T_new + t0) * H + h;   // token (t0 + j): tok0 + j H
+        for (int base = warp * 32; base < cnt * QK; base += THREADS) {   // whole warps: shuffles below
+          const int e = base + lane;
+          const bool ok = e < cnt * QK;
+          const int j = ok ? e / QK : 0, c = 4 * (e % QK);
+          float4 kc, qc, gc;
+          if (t0 == 0) {
+            kc = load4(rk + j * DK + c);
+            qc = load4(rq + j * DK + c);
+            gc = *reinterpret_cast<const float4 *>(rgp + j * DK + c);
+          } else {
+            const size_t off = (tok0 + (size_t)j * H) * DK + c;
+            kc = load4(k + off);
+            qc = load4(q + off);
+            gc = *reinterpret_cast<const float4 *>(g + off);
+          }
+          const float4 al = make_float4(__expf(gc.x), __expf(gc.y), __expf(gc.z), __expf(gc.w));
+          float qk = qc.x * kc.x + qc.y * kc.y + qc.z * kc.z + qc.w * kc.w;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
-        if (lane == 0) s_qk[j] = qk;
-        for (int c = lane; c < DK; c += 32) s_qa[j][c] *= s_alpha[j][c];
+          for (int o = QK / 2; o > 0; o >>= 1) qk += __shfl_xor_sync(0xffffffffu, qk, o);
+          if (ok) {
+            *reinterpret_cast<float4 *>(&s_alpha[j][c]) = al;
+            *reinterpret_cast<float4 *>(&s_k[j][c]) = kc;
+            *reinterpret_cast<float4 *>(&s_ka[j][c]) = make_float4(al.x * kc.x, al.y * kc.y, al.z * kc.z, al.w * kc.w);
+            *reinterpret_cast<float4 *>(&s_qa[j][c]) = make_float4(al.x * qc.x, al.y * qc.y, al.z * qc.z, al.w * qc.w);
+            if (c == 0) s_qk[j] = qk;
+          }
+        }
+        for (int e = tid; e < cnt * QV; e += THREADS) {
+          const int j = e / QV, c = 4 * (e % QV);
+          *reinterpret_cast<float4 *>(&s_v[j][c]) =
+              t0 == 0 ? load4(rv + j * DV + c) : load4(v + (tok0 + (size_t)j * H) * DV + c);
+        }
+        if (tid < cnt)
+          s_beta[tid] = t0 == 0 ? reinterpret_cast<const float *>(smem_raw + Lay::RAW_B)[tid]
+                                : beta[tok0 + (size_t)tid * H];
+        __syncthreads();
+        if (t0 == 0) {
+          const int64_t nx = u + gridDim.x;   // the raw and state buffers are free now
+          if (nx < units) prefetch(nx);
+        }
       }
-      __syncthreads();
 
       for (int j = 0; j < cnt; ++j) {
         const int t = t0 + j, p = t & 1;   // parity-indexed buffers: no third barrier
