@@ -601,18 +601,23 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
 // ---------------------------------------------------------------------------
 // Pass 2: the inter-chunk chain
 // ---------------------------------------------------------------------------
+// DVS = 128, 64 or 32 value columns per CTA.  The MN-major operand tiles of
+// a 32-column slice keep the 64-column (128-byte) rows of the swizzle atom,
+// half of each row used.
 template <int DVS>
 struct ChainLayout {
   static constexpr int NST = 2;                                   // packet buffers
+  static constexpr int TW = DVS < 64 ? 64 : DVS;                  // tile width in columns
   static constexpr uint32_t S_T = 0;                              // [128][DVS] bf16 state, MN-major B
-  static constexpr uint32_t VN = S_T + 128 * DVS * 2;             // [64][DVS] bf16 V_new, MN-major B
-  static constexpr uint32_t OBUF = VN + 64 * DVS * 2;             // [64][DVS] bf16 O, rows of DVS*2 bytes
-  static constexpr uint32_t STAGE0 = OBUF + 64 * DVS * 2;
+  static constexpr uint32_t VN = S_T + 128 * TW * 2;              // [64][DVS] bf16 V_new, MN-major B
+  static constexpr uint32_t OBUF = VN + 64 * TW * 2;              // [64][DVS] bf16 O, rows of DVS*2 bytes
+  static constexpr uint32_t STAGE0 = OBUF + 64 * TW * 2;
   // inside a stage
   static constexpr uint32_t WQ = 0;                               // [128][128] [W; Qtilde], K-major A
   static constexpr uint32_t KH = 32768;                           // [64][128] Khat, MN-major A
-  static constexpr uint32_t U = 49152;                            // [64][DVS] U slice
-  static constexpr uint32_t P = U + 64 * DVS * 2;                 // [64][64] P = rows 64..127 of the A tile at P - 8192
+  static constexpr uint32_t U = 49152;                            // [64][TW] U column block (the slice's columns)
+  static constexpr uint32_t UB = 64 * TW * 2;                     // its bytes
+  static constexpr uint32_t P = U + UB;                           // [64][64] P = rows 64..127 of the A tile at P - 8192
   static constexpr uint32_t D = P + 8192;                         // float[128]
   static constexpr uint32_t STAGE = (D + 512 + 1023) & ~1023u;
   static constexpr uint32_t BAR = STAGE0 + NST * STAGE;           // first product done
@@ -622,10 +627,11 @@ struct ChainLayout {
   static constexpr uint32_t SCAL = FULL + 8 * NST;                // int64 [2]: first packet, checkpoint slot
   static constexpr uint32_t TMEM_SLOT = SCAL + 16;
   static constexpr uint32_t TOTAL = TMEM_SLOT + 8;
-  static constexpr uint32_t TMEM_COLS = DVS == 128 ? 512 : 256;
+  static constexpr uint32_t TMEM_COLS = DVS == 128 ? 512 : (DVS == 64 ? 256 : 128);
   // TMEM columns: acc1 in two buffers (chunk parity), acc2, the FP32 state
   static constexpr uint32_t ACC1 = 0, ACC2 = DVS, SCOL = 2 * DVS, ACC1B = 3 * DVS;
-  static constexpr uint32_t TX_BYTES = 49152 + 64 * DVS * 2 + 8704;
+  static constexpr uint32_t TX_BYTES = 49152 + UB + 8704;
+  static constexpr int UCOL = 0;   // first column of the slice inside the U block: (y & 1) * 32 for DVS = 32
 };
 
 template <int DVS>
@@ -635,7 +641,8 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
              uint8_t *__restrict__ ck_tiles, int N, int H, int64_t jw0, int64_t wc, int first_window,
              int32_t *dev_status, uint64_t wait_ns) {
   using Lay = ChainLayout<DVS>;
-  constexpr int NCOL = DVS / 2;
+  constexpr int NCOL = DVS / 2;           // columns per warp half
+  constexpr int CW = NCOL < 32 ? NCOL : 32;   // columns per TMEM load or store
   constexpr int NST = Lay::NST;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
@@ -700,7 +707,7 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
     const uint32_t fb = sb + Lay::FULL + 8 * s;
     mbar_expect_tx(fb, Lay::TX_BYTES);
     bulk_load(st + Lay::WQ, pk + Packet::WQ, 49152, fb);                    // [W; Qtilde] and Khat
-    bulk_load(st + Lay::U, pk + Packet::U + (DVS == 64 ? 8192 * y : 0), 64 * DVS * 2, fb);
+    bulk_load(st + Lay::U, pk + Packet::U + (DVS == 128 ? 0 : 8192 * (DVS == 64 ? y : y >> 1)), Lay::UB, fb);
     bulk_load(st + Lay::P, pk + Packet::P, 8704, fb);                       // P and d
   };
   if (tid == 32)
@@ -712,31 +719,31 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
   {
     const size_t soff = ((size_t)unit * kDK + crow) * kDV + col0 + hw * NCOL;
 #pragma unroll
-    for (int u = 0; u < NCOL / 32; ++u) {
-      float x[32];
+    for (int u = 0; u < NCOL / CW; ++u) {
+      float x[CW];
 #pragma unroll
-      for (int j = 0; j < 32; j += 4) {
-        const float4 v4 = src ? *reinterpret_cast<const float4 *>(src + soff + 32 * u + j)
+      for (int j = 0; j < CW; j += 4) {
+        const float4 v4 = src ? *reinterpret_cast<const float4 *>(src + soff + CW * u + j)
                               : make_float4(0.f, 0.f, 0.f, 0.f);
         x[j] = v4.x; x[j + 1] = v4.y; x[j + 2] = v4.z; x[j + 3] = v4.w;
       }
-      tc::tmem_st32(s_tm + 32 * u, x);
+      tc::tmem_stw<CW>(s_tm + CW * u, x);
 #pragma unroll
-      for (int j = 0; j < 32; j += 8)
-        st_chunk_s(sp + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + 32 * u + j) >> 3), x + j);
+      for (int j = 0; j < CW; j += 8)
+        st_chunk_s(sp + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + CW * u + j) >> 3), x + j);
     }
     tc::tmem_wait_st();
   }
   auto store_state = [&](float *base_ptr, int64_t slot) {
     float *dst = base_ptr + ((size_t)slot * H + h) * kDK * kDV + (size_t)crow * kDV + col0 + hw * NCOL;
 #pragma unroll
-    for (int u = 0; u < NCOL / 32; ++u) {
-      float x[32];
-      tc::tmem_ld32(s_tm + 32 * u, x);
+    for (int u = 0; u < NCOL / CW; ++u) {
+      float x[CW];
+      tc::tmem_ldw<CW>(s_tm + CW * u, x);
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; j += 4)
-        *reinterpret_cast<float4 *>(dst + 32 * u + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
+      for (int j = 0; j < CW; j += 4)
+        *reinterpret_cast<float4 *>(dst + CW * u + j) = make_float4(x[j], x[j + 1], x[j + 2], x[j + 3]);
     }
   };
   tc::fence_smem_to_async();
@@ -750,18 +757,18 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
   // Only the four warps on TMEM lanes 64..127 call it: they stage O (bf16) in
   // OBUF, 16-byte chunks of row r permuted by r % 8, then write whole rows.
   constexpr int CH = DVS / 8;   // 16-byte chunks per O row
+  constexpr int CHM = (CH < 8 ? CH : 8) - 1;   // chunk permutation mask
   auto write_o = [&](uint32_t acc, int64_t t0, int L) {
     tc::fence_after_sync();
     const int r = 32 * (qd - 2) + lane;
     float a[NCOL];
 #pragma unroll
-    for (int u = 0; u < NCOL / 32; ++u)
-      tc::tmem_ld32(tl + acc + hw * NCOL + 32 * u, *reinterpret_cast<float(*)[32]>(a + 32 * u));
+    for (int u = 0; u < NCOL / CW; ++u) tc::tmem_ldw<CW>(tl + acc + hw * NCOL + CW * u, a + CW * u);
     tc::tmem_wait_ld();
 #pragma unroll
     for (int cc = 0; cc < NCOL / 8; ++cc) {
       const int c = hw * (NCOL / 8) + cc;
-      st_chunk_s(sp + Lay::OBUF + r * (DVS * 2) + ((c ^ (r & 7)) << 4), a + 8 * cc);
+      st_chunk_s(sp + Lay::OBUF + r * (DVS * 2) + ((c ^ (r & CHM)) << 4), a + 8 * cc);
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");   // the four O warps
     const int t = 32 * ((qd - 2) + 2 * hw) + lane;
@@ -769,7 +776,7 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
     for (int e = t; e < 64 * CH; e += 128) {
       const int row = e / CH, c = e % CH;
       if (row < L) {
-        const uint4 v4 = *reinterpret_cast<const uint4 *>(sp + Lay::OBUF + row * (DVS * 2) + ((c ^ (row & 7)) << 4));
+        const uint4 v4 = *reinterpret_cast<const uint4 *>(sp + Lay::OBUF + row * (DVS * 2) + ((c ^ (row & CHM)) << 4));
         *reinterpret_cast<uint4 *>(out + ((size_t)(t0 + row) * H + h) * kDV + col0 + 8 * c) = v4;
       }
     }
@@ -817,13 +824,13 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
       const int r = 32 * qd + lane;
       float a[NCOL];
 #pragma unroll
-      for (int u = 0; u < NCOL / 32; ++u)
-        tc::tmem_ld32(tl + acc1 + hw * NCOL + 32 * u, *reinterpret_cast<float(*)[32]>(a + 32 * u));
+      for (int u = 0; u < NCOL / CW; ++u) tc::tmem_ldw<CW>(tl + acc1 + hw * NCOL + CW * u, a + CW * u);
       tc::tmem_wait_ld();
+      const int uc0 = DVS == 32 ? 4 * (y & 1) : 0;   // the slice's first chunk in the U block
 #pragma unroll
       for (int cc = 0; cc < NCOL / 8; ++cc) {
         const int chunk = hw * (NCOL / 8) + cc;
-        const uint4 uu = *reinterpret_cast<const uint4 *>(sp + (st - sb) + Lay::U + tc::tile_offset(64, r, chunk));
+        const uint4 uu = *reinterpret_cast<const uint4 *>(sp + (st - sb) + Lay::U + tc::tile_offset(64, r, uc0 + chunk));
         float xv[8];
         unpack8(uu, xv);
 #pragma unroll
@@ -860,16 +867,15 @@ chain_kernel(const uint8_t *__restrict__ ws, const float *init, const int32_t *_
     {
       float a[NCOL], sv[NCOL];
 #pragma unroll
-      for (int u = 0; u < NCOL / 32; ++u) {
-        tc::tmem_ld32(tl + Lay::ACC2 + hw * NCOL + 32 * u, *reinterpret_cast<float(*)[32]>(a + 32 * u));
-        tc::tmem_ld32(s_tm + 32 * u, *reinterpret_cast<float(*)[32]>(sv + 32 * u));
+      for (int u = 0; u < NCOL / CW; ++u) {
+        tc::tmem_ldw<CW>(tl + Lay::ACC2 + hw * NCOL + CW * u, a + CW * u);
+        tc::tmem_ldw<CW>(s_tm + CW * u, sv + CW * u);
       }
       tc::tmem_wait_ld();
 #pragma unroll
       for (int i = 0; i < NCOL; ++i) sv[i] = fmaf(d, sv[i], a[i]);
 #pragma unroll
-      for (int u = 0; u < NCOL / 32; ++u)
-        tc::tmem_st32(s_tm + 32 * u, *reinterpret_cast<float(*)[32]>(sv + 32 * u));
+      for (int u = 0; u < NCOL / CW; ++u) tc::tmem_stw<CW>(s_tm + CW * u, sv + CW * u);
 #pragma unroll
       for (int jj = 0; jj < NCOL; jj += 8)
         st_chunk_s(sp + Lay::S_T + tc::tile_offset(128, crow, (hw * NCOL + jj) >> 3), sv + jj);
@@ -996,7 +1002,9 @@ cudaError_t launch_prefill_split_ex(const void *q, const void *k, const void *v,
   const size_t smem1 = IntraLayout::TOTAL + 1024;
   cudaError_t err = cudaFuncSetAttribute(intra_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (err != cudaSuccess) return err;
-  const bool narrow = (int64_t)N * H * 2 <= num_sms;       // few units: split the value columns
+  // Few units: split the value columns over 2 or 4 CTAs per unit (not with
+  // state tiles as checkpoints, which a 32-column slice does not fill whole).
+  const int slices = ((int64_t)N * H * 4 <= num_sms && !ck_tiles) ? 4 : ((int64_t)N * H * 2 <= num_sms ? 2 : 1);
   const int64_t windows = max_chunks > 0 ? (max_chunks + wc - 1) / wc : 1;
   for (int64_t w = 0; w < windows; ++w) {
     const int64_t jw0 = w * wc;
@@ -1008,10 +1016,12 @@ cudaError_t launch_prefill_split_ex(const void *q, const void *k, const void *v,
     }
     // One window: no carry needed unless the caller wants the final state.
     float *c = (windows == 1) ? fin : carry;
-    err = narrow ? launch_chain<64>(ws, init, cu, out, c, interval, ck, ck_tiles, N, H, jw0, wc,
-                                    w == 0, dev_status, stream)
-                 : launch_chain<128>(ws, init, cu, out, c, interval, ck, ck_tiles, N, H, jw0, wc,
-                                     w == 0, dev_status, stream);
+    err = slices == 4 ? launch_chain<32>(ws, init, cu, out, c, interval, ck, ck_tiles, N, H, jw0, wc,
+                                         w == 0, dev_status, stream)
+        : slices == 2 ? launch_chain<64>(ws, init, cu, out, c, interval, ck, ck_tiles, N, H, jw0, wc,
+                                         w == 0, dev_status, stream)
+                      : launch_chain<128>(ws, init, cu, out, c, interval, ck, ck_tiles, N, H, jw0, wc,
+                                          w == 0, dev_status, stream);
     if (err != cudaSuccess) return err;
   }
   return cudaSuccess;

@@ -72,6 +72,20 @@ def test_two_pass_windows(windows_of, want_final):
     check(d, out, fin if want_final else None, ck, 128)
 
 
+@pytest.mark.parametrize("H", [3, 12, 16])
+def test_chain_value_slices(H):
+    """The chain pass splits each (sequence, head)'s value columns over 4, 2 or 1
+    CTAs when N*H is at most a quarter, a half, or more than half the SM count:
+    5 sequences x H = 3, 12, 16 reach all three widths on a 148-SM B200.  Each
+    against the oracle, with checkpoints every 64 tokens and the final state."""
+    d = make_case(LENGTHS, H, 128, 128, torch.bfloat16, seed=40 + H)
+    dd = to_device(d)
+    out, fin, ck = run(dd, 64, "auto")
+    torch.cuda.synchronize()
+    assert kda.kda_last_prefill_path() == 2
+    check(d, out, fin, ck, 64)
+
+
 def test_single_pass_and_two_pass_agree():
     d = make_case(LENGTHS, 4, 128, 128, torch.bfloat16, seed=5, state_std=0.05)
     dd = to_device(d)
