@@ -52,9 +52,9 @@ namespace kda {
 cudaError_t launch_prefill_split_ex(const void *q, const void *k, const void *v, const float *g,
                                     const float *beta, const float *init, const int32_t *cu,
                                     void *out, float *fin, int64_t interval, float *ck,
-                                    uint8_t *ck_tiles, int N, int H, int64_t T, void *workspace,
-                                    size_t ws_bytes, int32_t *dev_status, cudaStream_t stream,
-                                    int num_sms);
+                                    uint8_t *ck_tiles, uint8_t *tt_out, int N, int H, int64_t T,
+                                    void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                    cudaStream_t stream, int num_sms);
 size_t split_packet_bytes();
 bool prefill_split_supported(int N);
 
@@ -357,8 +357,8 @@ struct BItemLayout {
   static constexpr uint32_t VT = 114688;     // [64][128] V (PART 0)
   static constexpr uint32_t BT2 = KT;        //   PART 0, after R: [-dU; dO] from the chain, then [-dR; dO]
   static constexpr uint32_t XA = KT;         //   PART 1: [dG; dP] placed against Gram B (K = 96)
-  static constexpr uint32_t MM = 131072;     // float [64][68] M = diag(beta) G
-  static constexpr uint32_t XM = MM + 17408; // float [64][68] (I + M)^-1
+  static constexpr uint32_t MM = 131072;     // prep scan partials, then dS_L (PART 0) or [dG^T | dP^T] (PART 1)
+  static constexpr uint32_t XM = MM + 17408; // gate factors during the prep
   static constexpr uint32_t CST = XM;        //   gate factors during the prep: float [2][6][128]
   static constexpr uint32_t DST = MM;        //   PART 0, after T: dS_L [ch][v] bf16
   static constexpr uint32_t YA = MM;         //   PART 1, after T: [dG^T | dP^T] placed against Gram A
@@ -367,7 +367,7 @@ struct BItemLayout {
   static constexpr uint32_t MT = ZS + 4608;  // float [32][33] M_(1,0)^T
   static constexpr uint32_t GG = MT + 4224;  // float [64][68] G (PART 1)
   static constexpr uint32_t TT = 194560;     // [64][64] T (row r, column i) bf16
-  static constexpr uint32_t RED = TT;        //   scan partials during the prep: float [8][128]
+  static constexpr uint32_t RED = MM;        //   scan partials during the prep: float [8][128]
   static constexpr uint32_t AIT = TT + 8192; // [64][64] (I + M)^-1 bf16 (PART 1)
   static constexpr uint32_t Y1T = AIT + 8192;// [64][64] Y1 = Ai^T dT bf16 (PART 1)
   static constexpr uint32_t DTT = Y1T + 8192;// [64][64] dT bf16 (PART 1)
@@ -417,6 +417,7 @@ struct BwdItemArgs {
   const uint8_t *ndu;          // -dU per packet: BF16 [64 tok][128 v] tile
   const uint8_t *dot;          // dO per packet: BF16 [64 tok][128 v] tile
   float *dtp;                  // dT, dP per packet: FP32 [64][64] each
+  const uint8_t *tt;           // T and (I + M)^-1 per packet from the forward: BF16 [64][64] tiles
   const void *q, *k;           // raw BF16 inputs (re-read by the final epilogues)
   float *dq, *dk, *dv, *dg, *dbeta;
   int N, H;
@@ -439,11 +440,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   float *s_beta = reinterpret_cast<float *>(sp + Lay::BETA);
   float *s_red = reinterpret_cast<float *>(sp + Lay::RED);
   float *s_cst = reinterpret_cast<float *>(sp + Lay::CST);
-  float *s_M = reinterpret_cast<float *>(sp + Lay::MM);
-  float *s_X = reinterpret_cast<float *>(sp + Lay::XM);
   float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
-  float *s_Z = reinterpret_cast<float *>(sp + Lay::ZS);
-  float *s_MT = reinterpret_cast<float *>(sp + Lay::MT);
   float *s_G = reinterpret_cast<float *>(sp + Lay::GG);
   float *s_gam = reinterpret_cast<float *>(sp + Lay::GST);
   float *s_dd = reinterpret_cast<float *>(sp + Lay::DD);
@@ -488,13 +485,18 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     L_ = (int)(T_n - kC * j_ < kC ? T_n - kC * j_ : kC);
   };
   // Inputs: g into its staging rows and beta (both parts), q, k into the Gram A
-  // tile, v (the state part).  `arrive`: this issue completes the barrier
-  // phase's arrival (the other only adds its bytes).
-  auto issue_g = [&](int h_, int64_t t0_, int L_, bool arrive, uint32_t bytes) {
+  // tile, v (the state part); with g, the item's T (and for the Gram part
+  // (I + M)^-1) as the forward formed them.  `arrive`: this issue completes
+  // the barrier phase's arrival (the other only adds its bytes).
+  constexpr uint32_t kTtBytes = PART == 0 ? 8192 : 16384;
+  constexpr uint32_t kGBytes = 32768 + kTtBytes;                 // g, T (, Ai)
+  constexpr uint32_t kKqvBytes = PART == 0 ? 16384 + 16384 : 32768;   // k, v | k, q
+  auto issue_g = [&](int h_, int64_t t0_, int L_, int64_t pp, bool arrive, uint32_t bytes) {
     if (tid == 32) {
       if (arrive) mbar_expect_tx(sb + Lay::TBAR, bytes);
       else mbar_add_tx(sb + Lay::TBAR, bytes);
       tma_load_3d(sb + Lay::GST, &maps.g, 0, h_, (int)t0_, sb + Lay::TBAR);
+      bulk_load(sb + Lay::TT, a.tt + (size_t)pp * 16384, kTtBytes, sb + Lay::TBAR);
     }
     if (tid >= 64 && tid < 64 + kC) {
       const int r = tid - 64;
@@ -507,7 +509,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
-      tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
+      if (PART == 1) tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
       if (PART == 0) tma_load_3d(sb + Lay::VT + b * 8192, &maps.v, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
     }
   };
@@ -525,13 +527,13 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   const int64_t ckb = a.prefck[n];
 
   if (PART == 1 && !pre) {
-    issue_g(h, t0, L, true, 65536);
+    issue_g(h, t0, L, p, true, kGBytes + kKqvBytes);
     if (tid == 32) issue_kqv(h, t0);
   }
   if (PART == 0) {
-    if (!pre) issue_g(h, t0, L, false, 32768);
+    if (!pre) issue_g(h, t0, L, p, false, kGBytes);
     if (tid == 32) {
-      mbar_expect_tx(sb + Lay::TBAR, 32768 + 16384);
+      mbar_expect_tx(sb + Lay::TBAR, kKqvBytes);
       issue_kqv(h, t0);
     }
   }
@@ -622,29 +624,33 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         const bool in = r < L;
         const uint2 z2 = make_uint2(0, 0);
         const uint2 kv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub) : z2;
-        const uint2 qv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub) : z2;
         un4(kv, kk);
-        un4(qv, qq);
+        if (PART == 1) {
+          const uint2 qv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub) : z2;
+          un4(qv, qq);
+        }
       }
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const float2 d = __fadd2_rn(gm[i][c], nref[c]);
         x[c] = make_float2(__expf(d.x), __expf(d.y));   // exp(Gam_r - ref), within [e^-80, e^80]
-        y[c] = make_float2(__expf(-d.x), __expf(-d.y)); // exp(ref - Gam_r)
+        if (PART == 1) y[c] = make_float2(__expf(-d.x), __expf(-d.y)); // exp(ref - Gam_r)
       }
+      if (PART == 1) {   // the gated Gram operands (the state part takes T from the forward)
 #pragma unroll
-      for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], x[c]);
-      st4(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub, t);
+        for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], x[c]);
+        st4(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub, t);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(qq[c], x[c]);
-      st4(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub, t);
+        for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(qq[c], x[c]);
+        st4(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub, t);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], y[c]);
-      st4(sp + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, cq) + sub, t);
-      if (!hf) {
+        for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], y[c]);
+        st4(sp + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, cq) + sub, t);
+        if (!hf) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], __fmul2_rn(y[c], cb[c]));
-        st4(sp + Lay::GB + tc::tile_offset(96, 32 + r, cq) + sub, t);
+          for (int c = 0; c < 2; ++c) t[c] = __fmul2_rn(kk[c], __fmul2_rn(y[c], cb[c]));
+          st4(sp + Lay::GB + tc::tile_offset(96, 32 + r, cq) + sub, t);
+        }
       }
       if (PART == 0) {   // Ktilde = k exp(Gam_r) = k (x fk) fk2
 #pragma unroll
@@ -662,21 +668,8 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     __syncthreads();
   }
 
-  // ---------------- gated Gram products: one [128 x 96 x 128] MMA ----------------
-  if (!aborted && tid == 0) {
-    tc::fence_after_sync();
-    constexpr uint32_t id = tc::idesc_bf16(128, 96, 0, 0);
-#pragma unroll
-    for (int s2 = 0; s2 < 8; ++s2)
-      tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::GA, 128, s2), tc::desc_kmajor(sb + Lay::GB, 96, s2),
-                   id, s2 > 0);
-    tc::mma_commit(sb + Lay::BAR);
-  }
-  if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
-  phase ^= 1;
-  tc::fence_after_sync();
-  // The Gram A tile is consumed: the state part's S0 (the BF16 operand tile)
-  // lands over it while the inverse is formed.
+  // The state part takes T from the forward; the raw k rows are consumed, and
+  // S0 (the BF16 operand tile) lands over them.
   if (PART == 0 && !aborted && S0src) {
     s0pend = true;
     if (tid == 32) {
@@ -684,122 +677,39 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       bulk_load(sb + Lay::S0T, S0src, 32768, sb + Lay::SBAR);
     }
   }
-  // Gram rows (lane m = row m, k rows only): M (scaled by beta_r, strictly lower),
-  // and for PART 1 G unscaled.
-  if (!aborted) {
-    const int m = 32 * qd + lane, part = m >> 6, r = m & 63, second = r >> 5;
-    const int i0 = second ? 32 * hw : (hw ? 32 : 0);
-    float acc[32];
-    if (second || hw == 0) {
-      tc::tmem_ld32(tl + (second ? 32 + 32 * hw : 0), acc);
-      tc::tmem_wait_ld();
-    }
-    const bool zero = !second && hw;
-    if (part == 0) {
-      const float br = s_beta[r];
-      float4 *dst = reinterpret_cast<float4 *>(s_M + r * 68 + i0);
-      auto mv = [&](int jj) { return (!zero && i0 + jj < r) ? br * acc[jj] : 0.f; };
+  // ---------------- the Gram part: gated Gram products, one [128 x 96 x 128] MMA ----------------
+  // (T and (I + M)^-1 come from the forward, so only G is read back.)
+  if (PART == 1) {
+    if (!aborted && tid == 0) {
+      tc::fence_after_sync();
+      constexpr uint32_t id = tc::idesc_bf16(128, 96, 0, 0);
 #pragma unroll
-      for (int jj = 0; jj < 32; jj += 4) dst[jj >> 2] = make_float4(mv(jj), mv(jj + 1), mv(jj + 2), mv(jj + 3));
-      if (PART == 1) {
+      for (int s2 = 0; s2 < 8; ++s2)
+        tc::mma_bf16(tmem, tc::desc_kmajor(sb + Lay::GA, 128, s2), tc::desc_kmajor(sb + Lay::GB, 96, s2),
+                     id, s2 > 0);
+      tc::mma_commit(sb + Lay::BAR);
+    }
+    if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
+    phase ^= 1;
+    tc::fence_after_sync();
+    // Gram rows (lane m = row m, k rows only): G, strictly lower.
+    if (!aborted) {
+      const int m = 32 * qd + lane, part = m >> 6, r = m & 63, second = r >> 5;
+      const int i0 = second ? 32 * hw : (hw ? 32 : 0);
+      float acc[32];
+      if (second || hw == 0) {
+        tc::tmem_ld32(tl + (second ? 32 + 32 * hw : 0), acc);
+        tc::tmem_wait_ld();
+      }
+      const bool zero = !second && hw;
+      if (part == 0) {
         float4 *gdst = reinterpret_cast<float4 *>(s_G + r * 68 + i0);
         auto gv = [&](int jj) { return (!zero && i0 + jj < r) ? acc[jj] : 0.f; };
 #pragma unroll
         for (int jj = 0; jj < 32; jj += 4) gdst[jj >> 2] = make_float4(gv(jj), gv(jj + 1), gv(jj + 2), gv(jj + 3));
       }
-      if (second && i0 == 0)
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) s_MT[jj * 33 + (r - 32)] = br * acc[jj];
     }
-  }
-  tc::fence_before_sync();
-  __syncthreads();
-
-  // ---------------- (I + M)^-1: 16x16 diagonal blocks, then the 32 and 64 levels ----------------
-  if (!aborted) {
-    if (qd >= 2) {
-      const int blk = (qd - 2) + 2 * hw;
-      const int o = 16 * blk, c = lane & 15, hf = lane >> 4;
-      float x[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = (8 * hf + i == c) ? 1.f : 0.f;
-      const float *mrow = s_M + (o + 8 * hf) * 68 + o;
-#pragma unroll
-      for (int sidx = 0; sidx < 15; ++sidx) {
-        float mm[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mm[i] = mrow[i * 68 + sidx];
-        const float xs = __shfl_sync(0xffffffffu, x[sidx & 7], c + 16 * (sidx >> 3));
-#pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = fmaf(-mm[i], xs, x[i]);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * 68 + o + c] = x[i];
-      if ((blk & 1) == 0)
-#pragma unroll
-        for (int i = 0; i < 8; ++i) s_X[(o + 8 * hf + i) * 68 + o + 16 + c] = 0.f;
-    }
-    __syncthreads();
-    {
-      const int hh = tid >> 7, rr = (tid >> 3) & 15, c0 = (tid & 7) * 2;
-      const int ro = 32 * hh + 16, co = 32 * hh;
-      float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2) {
-        const float mm = s_M[(ro + rr) * 68 + co + s2];
-        const float2 xv = *reinterpret_cast<const float2 *>(s_X + (co + s2) * 68 + co + c0);
-        y0 = fmaf(mm, xv.x, y0);
-        y1 = fmaf(mm, xv.y, y1);
-      }
-      s_Y[(hh * 16 + rr) * 17 + c0] = y0;
-      s_Y[(hh * 16 + rr) * 17 + c0 + 1] = y1;
-      __syncthreads();
-      float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2) {
-        const float av = s_X[(ro + rr) * 68 + ro + s2];
-        x0 = fmaf(av, s_Y[(hh * 16 + s2) * 17 + c0], x0);
-        x1 = fmaf(av, s_Y[(hh * 16 + s2) * 17 + c0 + 1], x1);
-      }
-      *reinterpret_cast<float2 *>(s_X + (ro + rr) * 68 + co + c0) = make_float2(-x0, -x1);
-      __syncthreads();
-    }
-    {
-      const int rr = lane, cq4 = 4 * warp;
-      float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s2 = cq4; s2 < 32; ++s2) {
-        const float mm = s_MT[s2 * 33 + rr];
-        const float4 xv = *reinterpret_cast<const float4 *>(s_X + s2 * 68 + cq4);
-        z.x = fmaf(mm, xv.x, z.x); z.y = fmaf(mm, xv.y, z.y);
-        z.z = fmaf(mm, xv.z, z.z); z.w = fmaf(mm, xv.w, z.w);
-      }
-      *reinterpret_cast<float4 *>(s_Z + rr * 36 + cq4) = z;
-      __syncthreads();
-      const int r2 = 4 * warp + (lane >> 3), c2 = 4 * (lane & 7);
-      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int s2 = 0; s2 < 4 * warp + 4; ++s2) {
-        const float av = s_X[(32 + r2) * 68 + 32 + s2];
-        const float4 zv = *reinterpret_cast<const float4 *>(s_Z + s2 * 36 + c2);
-        w.x = fmaf(av, zv.x, w.x); w.y = fmaf(av, zv.y, w.y);
-        w.z = fmaf(av, zv.z, w.z); w.w = fmaf(av, zv.w, w.w);
-      }
-      *reinterpret_cast<float4 *>(s_X + (32 + r2) * 68 + c2) = make_float4(-w.x, -w.y, -w.z, -w.w);
-      __syncthreads();
-    }
-    // T_ri = X_ri beta_i (i <= r) and, for PART 1, X itself, as [64][64] bf16 tiles.
-    for (int e = tid; e < 64 * 8; e += kThreads) {
-      const int row = e >> 3, chk = e & 7;
-      float tv[8], xv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = 8 * chk + u;
-        xv[u] = i <= row ? s_X[row * 68 + i] : 0.f;
-        tv[u] = xv[u] * s_beta[i];
-      }
-      st_chunk_s(sp + Lay::TT + tc::tile_offset(64, row, chk), tv);
-      if (PART == 1) st_chunk_s(sp + Lay::AIT + tc::tile_offset(64, row, chk), xv);
-    }
-    tc::fence_smem_to_async();
+    tc::fence_before_sync();
     __syncthreads();
   }
   const size_t row_stride = (size_t)H * kD;   // elements between tokens in [T][H][128]
@@ -1059,7 +969,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     tc::fence_smem_to_async();
     __syncthreads();
     if (!aborted && has_next) {
-      issue_g(h2, t02, L2, false, 32768);
+      issue_g(h2, t02, L2, p + gridDim.x, false, kGBytes);
       pre = true;
     }
     // dg = reverse cumulative sum of dGam plus the Gam_63 terms (sum_r k dk-_r from
@@ -1354,7 +1264,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     __syncthreads();
     // The Gram tiles and Gam are consumed: the next item's inputs land during the scan.
     if (!aborted && has_next) {
-      issue_g(h2, t02, L2, true, 65536);
+      issue_g(h2, t02, L2, p + gridDim.x, true, kGBytes + kKqvBytes);
       if (tid == 32) issue_kqv(h2, t02);
       pre = true;
     }
@@ -1445,7 +1355,7 @@ bwd_init_tiles_kernel(const float *__restrict__ init, uint8_t *__restrict__ tile
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdWs {
-  size_t pk, ck, s0i, dsl, ndu, dot, dtp, oscr, pref, prefck, total;
+  size_t pk, ck, s0i, tt, dsl, ndu, dot, dtp, oscr, pref, prefck, total;
 };
 
 BwdWs bwd_ws_layout(int N, int H, int64_t T) {
@@ -1455,6 +1365,7 @@ BwdWs bwd_ws_layout(int N, int H, int64_t T) {
   w.pk = off;     off += align256(P * Pk::BYTES + 256);
   w.ck = off;     off += align256((size_t)(T / kC) * H * 32768);      // BF16 state tiles
   w.s0i = off;    off += align256((size_t)N * H * 32768);             // initial states, same layout
+  w.tt = off;     off += align256(P * 16384);                         // T, (I + M)^-1 per packet
   w.dsl = off;    off += align256(P * 32768);
   w.ndu = off;    off += align256(P * 16384);
   w.dot = off;    off += align256(P * 16384);
@@ -1486,6 +1397,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   uint8_t *pk = base + w.pk;
   uint8_t *ck = base + w.ck;
   uint8_t *s0i = base + w.s0i;
+  uint8_t *tt = base + w.tt;
   uint8_t *dsl = base + w.dsl;
   uint8_t *ndu = base + w.ndu;
   uint8_t *dot = base + w.dot;
@@ -1498,7 +1410,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   // Forward recomputation: the two-pass prefill in one window keeps every
   // intra-chunk packet in the workspace and stores the state every 64 tokens.
   cudaError_t e = launch_prefill_split_ex(q, k, v, g, beta, init, cu, oscr, nullptr, kC, nullptr,
-                                          ck, N, H, T, pk, w.ck - w.pk, dev_status, stream, num_sms);
+                                          ck, tt, N, H, T, pk, w.ck - w.pk, dev_status, stream, num_sms);
   if (e != cudaSuccess) return e;
   if (init) {
     bwd_init_tiles_kernel<<<(unsigned)((int64_t)N * H), kThreads, 0, stream>>>(init, s0i);
@@ -1528,7 +1440,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
 
   BwdItemArgs a;
   a.beta = beta; a.s0_init = init ? s0i : nullptr; a.s0_ck = ck; a.cu = cu; a.pref = pref; a.prefck = prefck;
-  a.dsl = dsl; a.ndu = ndu; a.dot = dot; a.dtp = dtp; a.q = q; a.k = k;
+  a.dsl = dsl; a.ndu = ndu; a.dot = dot; a.dtp = dtp; a.tt = tt; a.q = q; a.k = k;
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
   a.N = N; a.H = H; a.dev_status = dev_status; a.wait_ns = wait_ns;
   const size_t smem_i = BItemLayout::TOTAL + 1024;

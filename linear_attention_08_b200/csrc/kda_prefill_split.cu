@@ -175,7 +175,8 @@ __device__ __forceinline__ Item decode_item(int p, const int32_t *s_pref, const 
 __global__ void __launch_bounds__(kThreads, 2)
 intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ beta,
              const int32_t *__restrict__ cu, int N, int H, int64_t jw0, int64_t wc,
-             uint8_t *__restrict__ ws, int32_t *dev_status, uint64_t wait_ns) {
+             uint8_t *__restrict__ ws, uint8_t *__restrict__ tt_out, int32_t *dev_status,
+             uint64_t wait_ns) {
   using Lay = IntraLayout;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t sraw = smem_u32(smem_raw);
@@ -522,16 +523,26 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
     }
     // T_ri = X_ri beta_i (i <= r), in rows 0..63 and again in rows 64..127 of the
     // K-major A tile, so that the product rows reach all four TMEM lane quadrants.
+    // With `tt_out` (the backward's forward recomputation) T and (I + M)^-1
+    // also go to global memory as [64][64] BF16 tiles, 16 KB per item.
     for (int e = tid; e < 64 * 8; e += kThreads) {
       const int row = e >> 3, ch = e & 7;
-      float val[8];
+      float val[8], xv[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int i = 8 * ch + u;
-        val[u] = i <= row ? s_X[row * kLd + i] * s_beta[i] : 0.f;
+        xv[u] = i <= row ? s_X[row * kLd + i] : 0.f;
+        val[u] = xv[u] * s_beta[i];
       }
       st_chunk_s(sp + Lay::TP + tc::tile_offset(128, row, ch), val);
       st_chunk_s(sp + Lay::TP + tc::tile_offset(128, 64 + row, ch), val);
+      if (tt_out) {
+        uint8_t *tt = tt_out + (size_t)p * 16384 + tc::tile_offset(64, row, ch);
+        *reinterpret_cast<uint4 *>(tt) = make_uint4(tc::pack_bf16(val[0], val[1]), tc::pack_bf16(val[2], val[3]),
+                                                    tc::pack_bf16(val[4], val[5]), tc::pack_bf16(val[6], val[7]));
+        *reinterpret_cast<uint4 *>(tt + 8192) = make_uint4(tc::pack_bf16(xv[0], xv[1]), tc::pack_bf16(xv[2], xv[3]),
+                                                           tc::pack_bf16(xv[4], xv[5]), tc::pack_bf16(xv[6], xv[7]));
+      }
     }
     tc::fence_smem_to_async();
     if (__syncthreads_or(!wait_timed(vbar, vphase, wait_ns))) { aborted = true; break; }
@@ -631,7 +642,6 @@ struct ChainLayout {
   // TMEM columns: acc1 in two buffers (chunk parity), acc2, the FP32 state
   static constexpr uint32_t ACC1 = 0, ACC2 = DVS, SCOL = 2 * DVS, ACC1B = 3 * DVS;
   static constexpr uint32_t TX_BYTES = 49152 + UB + 8704;
-  static constexpr int UCOL = 0;   // first column of the slice inside the U block: (y & 1) * 32 for DVS = 32
 };
 
 template <int DVS>
@@ -963,13 +973,14 @@ size_t split_workspace_full(int N, int H, int64_t T, bool have_final) {
 // index H * sum_{m<n} c_m + h * c_n + (j - jw0), c_m = chunks of m in the window.
 // Checkpoints go to `ck` as FP32 [128][128] states, or, with `ck_tiles` set
 // (and `ck` null), as the chain's BF16 state tiles (32 KB each, the 128-byte
-// swizzled [key channel][value column] MMA operand layout).
+// swizzled [key channel][value column] MMA operand layout).  `tt_out` (one
+// window only) receives each packet's T and (I + M)^-1 as BF16 tiles.
 cudaError_t launch_prefill_split_ex(const void *q, const void *k, const void *v, const float *g,
                                     const float *beta, const float *init, const int32_t *cu,
                                     void *out, float *fin, int64_t interval, float *ck,
-                                    uint8_t *ck_tiles, int N, int H, int64_t T, void *workspace,
-                                    size_t ws_bytes, int32_t *dev_status, cudaStream_t stream,
-                                    int num_sms) {
+                                    uint8_t *ck_tiles, uint8_t *tt_out, int N, int H, int64_t T,
+                                    void *workspace, size_t ws_bytes, int32_t *dev_status,
+                                    cudaStream_t stream, int num_sms) {
   if (!prefill_split_supported(N)) return cudaErrorNotSupported;
   uintptr_t base = (reinterpret_cast<uintptr_t>(workspace) + 255) & ~(uintptr_t)255;
   const size_t lost = base - reinterpret_cast<uintptr_t>(workspace);
@@ -1010,7 +1021,7 @@ cudaError_t launch_prefill_split_ex(const void *q, const void *k, const void *v,
     const int64_t jw0 = w * wc;
     if (max_chunks > 0) {
       intra_kernel<<<2 * num_sms, kThreads, smem1, stream>>>(maps, beta, cu, N, H, jw0, wc, ws,
-                                                            dev_status, 2000000000ull);
+                                                            tt_out, dev_status, 2000000000ull);
       err = cudaGetLastError();
       if (err != cudaSuccess) return err;
     }
@@ -1032,8 +1043,8 @@ cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, co
                                  float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
                                  void *workspace, size_t ws_bytes, int32_t *dev_status,
                                  cudaStream_t stream, int num_sms) {
-  return launch_prefill_split_ex(q, k, v, g, beta, init, cu, out, fin, interval, ck, nullptr, N, H,
-                                 T, workspace, ws_bytes, dev_status, stream, num_sms);
+  return launch_prefill_split_ex(q, k, v, g, beta, init, cu, out, fin, interval, ck, nullptr, nullptr,
+                                 N, H, T, workspace, ws_bytes, dev_status, stream, num_sms);
 }
 
 }  // namespace kda

@@ -264,7 +264,8 @@ def test_chunked_backward_workspace():
     74,240-byte packet, dS at the chunk's end as a BF16 tile (32 KiB), the -dU and
     dO tiles (16 KiB each) and dT, dP (FP32, 32 KiB); per full chunk the stored
     forward state as a BF16 operand tile (32 KiB); per (sequence, head) the initial
-    state as such a tile; the forward's output (BF16); two prefix tables."""
+    state as such a tile; per (chunk, head) the forward's T and (I + M)^-1 as BF16
+    tiles (16 KiB); the forward's output (BF16); two prefix tables."""
     lib = kda.load()
     al = lambda x: (x + 255) // 256 * 256
     for lengths, H in (([1024] * 4, 32), ([5, 0, 130, 64], 3)):
@@ -272,7 +273,7 @@ def test_chunked_backward_workspace():
         s = kda.make_shape(N, T, H, 128, 128, 0, kda.KDA_DTYPE_BF16)
         P = H * ((T + 63 * N) // 64)
         assert P >= H * sum(-(-L // 64) for L in lengths)
-        want = (al(P * 74240 + 256) + al((T // 64) * H * 32768) + al(N * H * 32768)
+        want = (al(P * 74240 + 256) + al((T // 64) * H * 32768) + al(N * H * 32768) + al(P * 16384)
                 + al(P * 32768) + al(P * 16384)
                 + al(P * 16384) + al(P * 32768) + al(T * H * 256) + 2 * al((N + 1) * 8) + 256)
         assert lib.kda_backward_workspace_bytes(ctypes.byref(s)) == want
