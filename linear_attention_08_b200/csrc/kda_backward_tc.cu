@@ -508,8 +508,12 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   auto issue_kqv = [&](int h_, int64_t t0_) {   // tid 32, after its expect_tx
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
-      if (PART == 1) tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
+      if (PART == 1) {   // k and q into the rows of the Gram A tile their scaled versions replace
+        tma_load_3d(sb + Lay::GA + b * 16384, &maps.k, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
+        tma_load_3d(sb + Lay::GA + b * 16384 + 8192, &maps.q, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
+      } else {           // k into the Ktilde tile, scaled in place by the prep
+        tma_load_3d(sb + Lay::KT + b * 8192, &maps.k, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
+      }
       if (PART == 0) tma_load_3d(sb + Lay::VT + b * 8192, &maps.v, 64 * b, h_, (int)t0_, sb + Lay::TBAR);
     }
   };
@@ -543,6 +547,15 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   // The per-chunk states and gradients come from L2 later; start them now.
   const uint8_t *S0src = j == 0 ? (a.s0_init ? a.s0_init + (size_t)unit * 32768 : nullptr)
                                 : a.s0_ck + ((size_t)(ckb + j - 1) * H + h) * 32768;
+  // The state part takes T from the forward and needs no Gram tiles: S0 (the
+  // BF16 operand tile) lands in the Gram A tile's space from the start.
+  if (PART == 0 && S0src) {
+    s0pend = true;
+    if (tid == 32) {
+      mbar_expect_tx(sb + Lay::SBAR, 32768);
+      bulk_load(sb + Lay::S0T, S0src, 32768, sb + Lay::SBAR);
+    }
+  }
   if (PART == 1) {
     const float *dtp = a.dtp + (size_t)p * 8192;
     for (int e = tid; e < 256; e += kThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(dtp + 32 * e));
@@ -623,7 +636,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       {
         const bool in = r < L;
         const uint2 z2 = make_uint2(0, 0);
-        const uint2 kv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub) : z2;
+        const uint2 kv = !in ? z2
+                         : PART == 1 ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, r, cq) + sub)
+                                     : *reinterpret_cast<const uint2 *>(sp + Lay::KT + tc::tile_offset(64, r, cq) + sub);
         un4(kv, kk);
         if (PART == 1) {
           const uint2 qv = in ? *reinterpret_cast<const uint2 *>(sp + Lay::GA + tc::tile_offset(128, 64 + r, cq) + sub) : z2;
@@ -668,15 +683,6 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     __syncthreads();
   }
 
-  // The state part takes T from the forward; the raw k rows are consumed, and
-  // S0 (the BF16 operand tile) lands over them.
-  if (PART == 0 && !aborted && S0src) {
-    s0pend = true;
-    if (tid == 32) {
-      mbar_expect_tx(sb + Lay::SBAR, 32768);
-      bulk_load(sb + Lay::S0T, S0src, 32768, sb + Lay::SBAR);
-    }
-  }
   // ---------------- the Gram part: gated Gram products, one [128 x 96 x 128] MMA ----------------
   // (T and (I + M)^-1 come from the forward, so only G is read back.)
   if (PART == 1) {
