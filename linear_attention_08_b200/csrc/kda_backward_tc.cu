@@ -846,31 +846,15 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       s_dd[32 * qd + lane] = dd;
     }
     if (!aborted) {
-      if (qd < 2) {
+      if (qd < 2) {   // -dR replaces -dU in rows 0..63: the next product's operand first
         const int r = 32 * qd + lane;
         float acc[64];
         tc::tmem_ld32(tl + 0 + hw * 64, *reinterpret_cast<float(*)[32]>(acc));
         tc::tmem_ld32(tl + 0 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(acc + 32));
         tc::tmem_wait_ld();
-        if (r < L) {   // dv = dR
-          float *dst = a.dv + base_row + (size_t)r * row_stride + hw * 64;
 #pragma unroll
-          for (int e = 0; e < 64; e += 4)
-            *reinterpret_cast<float4 *>(dst + e) = make_float4(-acc[e], -acc[e + 1], -acc[e + 2], -acc[e + 3]);
-        }
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc)   // -dR replaces -dU in rows 0..63
+        for (int cc = 0; cc < 8; ++cc)
           st_chunk_s(sp + Lay::BT2 + tc::tile_offset(128, r, hw * 8 + cc), acc + 8 * cc);
-        float d2[32];
-        tc::tmem_ld32(tl + 448 + hw * 32, d2);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const int i = 32 * hw + e;
-          *reinterpret_cast<float4 *>(dtp + r * 64 + i) =
-              make_float4(i <= r ? -d2[e] : 0.f, i + 1 <= r ? -d2[e + 1] : 0.f,
-                          i + 2 <= r ? -d2[e + 2] : 0.f, i + 3 <= r ? -d2[e + 3] : 0.f);
-        }
       } else {
         const int r = 32 * (qd - 2) + lane;
         float d2[32];
@@ -898,8 +882,33 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
                      tc::desc_kmajor(sb + Lay::S0T, 128, s2), id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
-    // The raw q (lanes 64..127) or k (lanes 0..63) of this thread's token and
-    // channel half, loaded while the product runs.
+    // While the product runs: dv (= dR) and dT leave for global memory (their
+    // TMEM columns are not the product's), and the raw q (lanes 64..127) or k
+    // (lanes 0..63) of this thread's token and channel half is loaded.
+    if (!aborted && qd < 2) {
+      const int r = 32 * qd + lane;
+      float *dst = a.dv + base_row + (size_t)r * row_stride + hw * 64;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {   // warp-wide TMEM loads; stores for tokens inside the chunk
+        float acc[32];
+        tc::tmem_ld32(tl + 0 + hw * 64 + 32 * half, acc);
+        tc::tmem_wait_ld();
+        if (r < L)
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4 *>(dst + 32 * half + e) = make_float4(-acc[e], -acc[e + 1], -acc[e + 2], -acc[e + 3]);
+      }
+      float d2[32];
+      tc::tmem_ld32(tl + 448 + hw * 32, d2);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const int i = 32 * hw + e;
+        *reinterpret_cast<float4 *>(dtp + r * 64 + i) =
+            make_float4(i <= r ? -d2[e] : 0.f, i + 1 <= r ? -d2[e + 1] : 0.f,
+                        i + 2 <= r ? -d2[e + 2] : 0.f, i + 3 <= r ? -d2[e + 3] : 0.f);
+      }
+    }
     uint4 raw[8];
     {
       const int rr = qd >= 2 ? 32 * (qd - 2) + lane : 32 * qd + lane;
