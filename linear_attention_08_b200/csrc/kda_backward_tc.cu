@@ -28,19 +28,22 @@
 // and the gated products G, P, Qtilde, Ktilde, Khat, d pass their gradients to
 // q, k and Gam; dg is the reverse cumulative sum of dGam inside the chunk.
 //
-// Three launches after the forward recomputation (the two-pass prefill run
-// with a state stored at every chunk end, its intra-chunk packets kept):
+// The forward is recomputed first (the two-pass prefill, keeping its
+// intra-chunk packets, each chunk's T and Ai as BF16 tiles, and the state at
+// every chunk end as a BF16 tile); small launches then build the item prefix
+// and the BF16 tiles of dO and of the initial states.  Then:
 //  1. bwd_chain_kernel: one CTA per (sequence, head) walks the chunks
 //     backwards carrying dS in tensor memory: per chunk dU = [Khat | P^T]
 //     [dS; dO] and dS <- d dS + [W^T | Qtilde^T] [-dU; dO], two tcgen05 MMAs.
-//     It stores dS_L per chunk and the BF16 tile [-dU; dO] for the others.
-//  2. bwd_state_kernel (per (chunk, head), in parallel): recomputes the gates,
-//     the Gram products and T, then R, U, dR (= dv), dT, dP, dQtilde,
-//     dKtilde, dKhat on the tensor cores; writes dv and the parts of dq, dk and
-//     dg those terms give, and the BF16 tiles dT and dP.
-//  3. bwd_gram_kernel (per (chunk, head)): recomputes the gates, G and Ai,
-//     then Y1, dA, dG and the gated products of dG and dP on the tensor
-//     cores; adds the rest of dq, dk, dg and writes dbeta.
+//     It stores dS_L and -dU per chunk as BF16 tiles.
+//  2. bwd_item_kernel<0>, the state part (per (chunk, head), persistent):
+//     recomputes Gam and Ktilde, takes T from the forward, then R, U,
+//     dR (= dv), dT, dP, dQtilde, dKtilde, dKhat and dd on the tensor cores;
+//     writes dv and the parts of dq, dk and dg those terms give, and dT, dP.
+//  3. bwd_item_kernel<1>, the Gram part: recomputes the gates and G, takes T
+//     and Ai from the forward, then Y1, dA, dG and the gated products of dG
+//     and dP on the tensor cores; adds the rest of dq, dk, dg (global
+//     reductions) and writes dbeta.
 #include <cuda.h>
 
 #include "kda_common.cuh"
@@ -349,26 +352,26 @@ namespace {
 // ---------------------------------------------------------------------------
 struct BItemLayout {
   static constexpr uint32_t GA = 0;          // [128][128] Gram A: k x rows 0..63, q x rows 64..127
-  static constexpr uint32_t S0T = GA;        //   PART 0, after the Gram: S0 [ch][v] bf16
+  static constexpr uint32_t S0T = GA;        //   PART 0 (no Gram tiles): S0 [ch][v] bf16
   static constexpr uint32_t GB = 32768;      // [96][128] Gram B: k y (ref 1) | k y (ref 2), first half | k y, second half
-  static constexpr uint32_t RU = 32768;      //   PART 0, after the Gram: [R; U] [tok][v] bf16 (128 rows)
+  static constexpr uint32_t RU = 32768;      //   PART 0: [U; R] [tok][v] bf16 (128 rows)
   static constexpr uint32_t GST = 65536;     // float [64][128]: g, then Gam in place
-  static constexpr uint32_t KT = 98304;      // [64][128] Ktilde (PART 0)
+  static constexpr uint32_t KT = 98304;      // [64][128] k, then Ktilde in place (PART 0)
   static constexpr uint32_t VT = 114688;     // [64][128] V (PART 0)
   static constexpr uint32_t BT2 = KT;        //   PART 0, after R: [-dU; dO] from the chain, then [-dR; dO]
   static constexpr uint32_t XA = KT;         //   PART 1: [dG; dP] placed against Gram B (K = 96)
   static constexpr uint32_t MM = 131072;     // prep scan partials, then dS_L (PART 0) or [dG^T | dP^T] (PART 1)
   static constexpr uint32_t XM = MM + 17408; // gate factors during the prep
   static constexpr uint32_t CST = XM;        //   gate factors during the prep: float [2][6][128]
-  static constexpr uint32_t DST = MM;        //   PART 0, after T: dS_L [ch][v] bf16
-  static constexpr uint32_t YA = MM;         //   PART 1, after T: [dG^T | dP^T] placed against Gram A
-  static constexpr uint32_t YS = XM + 17408; // float [2][16][17]
-  static constexpr uint32_t ZS = YS + 2176;  // float [32][36]
-  static constexpr uint32_t MT = ZS + 4608;  // float [32][33] M_(1,0)^T
+  static constexpr uint32_t DST = MM;        //   PART 0: dS_L [ch][v] bf16
+  static constexpr uint32_t YA = MM;         //   PART 1: [dG^T | dP^T] placed against Gram A
+  static constexpr uint32_t YS = XM + 17408; // float [2][256]: the reverse scan's partial sums
+  static constexpr uint32_t ZS = YS + 2176;  // (free)
+  static constexpr uint32_t MT = ZS + 4608;  // (free)
   static constexpr uint32_t GG = MT + 4224;  // float [64][68] G (PART 1)
-  static constexpr uint32_t TT = 194560;     // [64][64] T (row r, column i) bf16
+  static constexpr uint32_t TT = 194560;     // [64][64] T (row r, column i) bf16, from the forward
   static constexpr uint32_t RED = MM;        //   scan partials during the prep: float [8][128]
-  static constexpr uint32_t AIT = TT + 8192; // [64][64] (I + M)^-1 bf16 (PART 1)
+  static constexpr uint32_t AIT = TT + 8192; // [64][64] (I + M)^-1 bf16, from the forward (PART 1)
   static constexpr uint32_t Y1T = AIT + 8192;// [64][64] Y1 = Ai^T dT bf16 (PART 1)
   static constexpr uint32_t DTT = Y1T + 8192;// [64][64] dT bf16 (PART 1)
   static constexpr uint32_t BETA = DTT + 8192;            // float [64]
@@ -377,14 +380,14 @@ struct BItemLayout {
   static constexpr uint32_t BAR = EXTRA + 512;            // MMA done
   static constexpr uint32_t TBAR = BAR + 8;               // inputs landed
   static constexpr uint32_t CBAR = BAR + 16;              // [-dU; dO] landed (PART 0)
-  static constexpr uint32_t SBAR = BAR + 24;              // S0 (FP32) landed (PART 0)
+  static constexpr uint32_t SBAR = BAR + 24;              // S0 (BF16 tile) landed (PART 0)
   static constexpr uint32_t TMEM_SLOT = BAR + 32;
   static constexpr uint32_t TOTAL = BAR + 40;
   // PART 0 final partials (after the last MMAs): float [64][128] each
   static constexpr uint32_t PKM = GA, PDG = RU;
   // PART 1 final partials: float [64][128] and [32][128]
   static constexpr uint32_t QDG = XA, KMC = YA;
-  static_assert(GG + 17408 <= TT && MT + 4224 <= GG, "solve scratch");
+  static_assert(GG + 17408 <= TT && MT + 4224 <= GG, "G");
   static_assert(YS + 2048 <= ZS && DST + 32768 <= YS, "scan scratch clears dS_L");
   static_assert(GB + 24576 <= RU + 32768 && RU + 32768 <= GST, "[R; U] stays clear of Gam");
   static_assert(CST + 6144 <= XM + 17408, "gate factors");
@@ -989,7 +992,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     }
     // dg = reverse cumulative sum of dGam plus the Gam_63 terms (sum_r k dk-_r from
     // Khat, d * sum_v dS_L S0).  Two threads per channel, 32 rows each.
-    float *sred = s_Y;   // [2][128] partial sums, [2][128] partial extras (the solve scratch)
+    float *sred = s_Y;   // [2][128] partial sums, [2][128] partial extras
     if (!aborted) {
       const int ch = tid & 127, hf = tid >> 7;
       const float *pdq = reinterpret_cast<const float *>(pdq4), *pdk = reinterpret_cast<const float *>(pdk4);
