@@ -426,11 +426,11 @@ def time_decode(steps_graph, warmup, world, local, decode_steps=None):
                 flops=token_heads * decode_flops_per_token_head(Dk), clocks=clk.result)
 
 
-def time_spec_decode(steps, warmup, world, local, T_new=8):
-    """Multi-token decode: 512 sequences x 32 heads, T_new draft tokens each, all
-    accepted.  One call moves the FP32 state once for T_new tokens."""
+def time_spec_decode(steps, warmup, world, local, T_new=8, N=512):
+    """Multi-token decode: N (512) sequences x 32 heads, T_new draft tokens each,
+    all accepted.  One call moves the FP32 state once for T_new tokens."""
     from linear_attention_08_b200 import kda
-    N, H, D = 512, 32, 128
+    H, D = 32, 128
     d = kin.make_inputs((N, T_new), H, D, D, torch.bfloat16, local, num_states=N,
                         state_std=0.02, device="cuda")
     state = d["init_state"].clone()
@@ -454,7 +454,7 @@ def time_spec_decode(steps, warmup, world, local, T_new=8):
     ms = max_over_ranks(a.elapsed_time(b) / steps, world)
     byts = N * H * (decode_state_bytes_per_token_head(D, D)
                     + T_new * prefill_io_bytes_per_token_head(D, D, 2))
-    return dict(tokens=N * T_new, ms=ms, bytes=byts, T_new=T_new)
+    return dict(tokens=N * T_new, ms=ms, bytes=byts, T_new=T_new, N=N)
 
 
 def time_backward(steps, warmup, world, local, N=4, H=32, T=1024, D=128):
@@ -684,6 +684,9 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=0,
                     help="decode steps per graph (default: the workload's 256)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--spec-only", type=int, default=0, metavar="NUM_SEQS",
+                    help="time only the multi-token decode (8 draft tokens) on NUM_SEQS "
+                         "sequences x 32 heads (a small case for profiling); prints its object alone")
     ap.add_argument("--backward-only", type=int, default=0, metavar="SEQ_LEN",
                     help="time only the backward pass on 4 sequences of SEQ_LEN tokens "
                          "(a small case for profiling); prints its object alone")
@@ -696,6 +699,19 @@ def main():
             print(json.dumps(line), flush=True)
         return
     rank, world, local = dist_setup(args.gpus)
+    if args.spec_only > 0:
+        spec = time_spec_decode(args.steps, args.warmup, world, local, N=args.spec_only)
+        if rank == 0:
+            print(json.dumps({"metric": "KDA multi-token decode tokens/s", "unit": "tokens/s",
+                              "value": world * spec["tokens"] / (spec["ms"] / 1e3),
+                              "ms_per_call": spec["ms"], "n_gpus": world,
+                              "config": {"num_seqs": spec["N"], "heads": 32, "d": 128,
+                                         "draft_tokens": spec["T_new"]}}), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     if args.backward_only > 0:
         bwd = time_backward(args.steps, args.warmup, world, local, T=args.backward_only)
         if rank == 0:
