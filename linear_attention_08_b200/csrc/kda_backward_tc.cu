@@ -379,7 +379,7 @@ struct BItemLayout {
   static constexpr uint32_t EXTRA = DD + 512;             // float [128] dGam_63 extras (PART 0)
   static constexpr uint32_t BAR = EXTRA + 512;            // MMA done
   static constexpr uint32_t TBAR = BAR + 8;               // inputs landed
-  static constexpr uint32_t CBAR = BAR + 16;              // [-dU; dO] landed (PART 0)
+  static constexpr uint32_t CBAR = BAR + 16;              // [-dU; dO] landed (PART 0); dT, placed dP (PART 1)
   static constexpr uint32_t SBAR = BAR + 24;              // S0 (BF16 tile) landed (PART 0)
   static constexpr uint32_t TMEM_SLOT = BAR + 32;
   static constexpr uint32_t TOTAL = BAR + 40;
@@ -419,7 +419,9 @@ struct BwdItemArgs {
   const uint8_t *dsl;          // dS_L per packet: BF16 [128 ch][128 v] tile
   const uint8_t *ndu;          // -dU per packet: BF16 [64 tok][128 v] tile
   const uint8_t *dot;          // dO per packet: BF16 [64 tok][128 v] tile
-  float *dtp;                  // dT, dP per packet: FP32 [64][64] each
+  uint8_t *dtp;                // per packet, from the state part to the Gram part (kDtpBytes):
+                               //   dT as the BF16 [64][64] operand tile, rows 64..127 of the
+                               //   [dG; dP] tile (dP placed, BF16, 2 x 8 KB), dP^T FP32 [64][64]
   const uint8_t *tt;           // T and (I + M)^-1 per packet from the forward: BF16 [64][64] tiles
   const void *q, *k;           // raw BF16 inputs (re-read by the final epilogues)
   float *dq, *dk, *dv, *dg, *dbeta;
@@ -427,6 +429,8 @@ struct BwdItemArgs {
   int32_t *dev_status;
   uint64_t wait_ns;
 };
+
+constexpr uint32_t kDtpBytes = 8192 + 16384 + 16384;
 
 template <int PART>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -559,9 +563,12 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       bulk_load(sb + Lay::S0T, S0src, 32768, sb + Lay::SBAR);
     }
   }
-  if (PART == 1) {
-    const float *dtp = a.dtp + (size_t)p * 8192;
-    for (int e = tid; e < 256; e += kThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(dtp + 32 * e));
+  if (PART == 1 && tid == 32) {   // dT's operand tile and the placed dP rows of [dG; dP]
+    const uint8_t *dt = a.dtp + (size_t)p * kDtpBytes;
+    mbar_expect_tx(sb + Lay::CBAR, 24576);
+    bulk_load(sb + Lay::DTT, dt, 8192, sb + Lay::CBAR);
+    bulk_load(sb + Lay::XA + 8192, dt + 8192, 8192, sb + Lay::CBAR);
+    bulk_load(sb + Lay::XA + 16384 + 8192, dt + 16384, 8192, sb + Lay::CBAR);
   }
 
   cp_async_wait_all();
@@ -838,7 +845,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
     phase ^= 1;
     tc::fence_after_sync();
-    float *dtp = a.dtp + (size_t)p * 8192;
+    uint8_t *dtp = a.dtp + (size_t)p * kDtpBytes;
     if (!aborted && hw == 0) {   // the diagonal of dS_L S0^T: lane c takes column c
       float x[32];
       tc::tmem_ld32(tl + 128 + 32 * qd, x);
@@ -858,18 +865,6 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll
         for (int cc = 0; cc < 8; ++cc)
           st_chunk_s(sp + Lay::BT2 + tc::tile_offset(128, r, hw * 8 + cc), acc + 8 * cc);
-      } else {
-        const int r = 32 * (qd - 2) + lane;
-        float d2[32];
-        tc::tmem_ld32(tl + 384 + hw * 32, d2);
-        tc::tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const int i = 32 * hw + e;
-          *reinterpret_cast<float4 *>(dtp + 4096 + r * 64 + i) =
-              make_float4(i <= r ? d2[e] : 0.f, i + 1 <= r ? d2[e + 1] : 0.f,
-                          i + 2 <= r ? d2[e + 2] : 0.f, i + 3 <= r ? d2[e + 3] : 0.f);
-        }
       }
     }
     tc::fence_smem_to_async();
@@ -901,16 +896,49 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
           for (int e = 0; e < 32; e += 4)
             *reinterpret_cast<float4 *>(dst + 32 * half + e) = make_float4(-acc[e], -acc[e + 1], -acc[e + 2], -acc[e + 3]);
       }
-      float d2[32];
+      float d2[32];   // dT row r, columns 32 hw .. +31 (kept on and below the diagonal)
       tc::tmem_ld32(tl + 448 + hw * 32, d2);
       tc::tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const int i = 32 * hw + e;
-        *reinterpret_cast<float4 *>(dtp + r * 64 + i) =
-            make_float4(i <= r ? -d2[e] : 0.f, i + 1 <= r ? -d2[e + 1] : 0.f,
-                        i + 2 <= r ? -d2[e + 2] : 0.f, i + 3 <= r ? -d2[e + 3] : 0.f);
+      for (int e = 0; e < 32; ++e) d2[e] = 32 * hw + e <= r ? -d2[e] : 0.f;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {   // the Gram part's dT operand tile
+        const float *x = d2 + 8 * cc;
+        *reinterpret_cast<uint4 *>(dtp + tc::tile_offset(64, r, 4 * hw + cc)) =
+            make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                       tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
       }
+    } else if (!aborted) {
+      // dP row r, columns i = 32 hw .. +31 (i <= r): placed against Gram B as
+      // rows 64..127 of [dG; dP] (first-half rows at kappa = i, second-half rows
+      // at kappa = 32 + i, zeros elsewhere; K = 96), and transposed (FP32) for
+      // the placement against Gram A.
+      const int r = 32 * (qd - 2) + lane;
+      float d2[32];
+      tc::tmem_ld32(tl + 384 + hw * 32, d2);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) d2[e] = 32 * hw + e <= r ? d2[e] : 0.f;
+      uint8_t *xa = dtp + 8192;   // [2 blocks][rows 64..127][128 B]
+      auto put = [&](int ch, const float *x) {
+        *reinterpret_cast<uint4 *>(xa + (ch >> 3) * 8192 + r * 128 + (((ch & 7) ^ (r & 7)) << 4)) =
+            make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
+                       tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+      };
+      const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      if (hw == 0) {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          put((r < 32 ? 0 : 4) + cc, d2 + 8 * cc);
+          put((r < 32 ? 4 : 0) + cc, z);
+        }
+      } else {
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) put(8 + cc, d2 + 8 * cc);
+      }
+      float *dpt = reinterpret_cast<float *>(dtp + 24576);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) dpt[(32 * hw + e) * 64 + r] = d2[e];
     }
     uint4 raw[8];
     {
@@ -1015,22 +1043,11 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       }
     }
   } else {
-    // ---- PART 1: dT, dP from the state part ----
-    const float *dT = a.dtp + (size_t)p * 8192, *dP = dT + 4096;
+    // ---- PART 1: dT (its operand tile) and dP from the state part ----
+    const float *dPT = reinterpret_cast<const float *>(a.dtp + (size_t)p * kDtpBytes + 24576);
     float *s_db = s_dd;   // dbeta [64]
-    if (!aborted) {
-      for (int e = tid; e < 64 * 8; e += kThreads) {
-        const int row = e >> 3, chk = e & 7;
-        float x8[8];
-        const float4 u0 = *reinterpret_cast<const float4 *>(dT + row * 64 + 8 * chk);
-        const float4 u1 = *reinterpret_cast<const float4 *>(dT + row * 64 + 8 * chk + 4);
-        x8[0] = u0.x; x8[1] = u0.y; x8[2] = u0.z; x8[3] = u0.w;
-        x8[4] = u1.x; x8[5] = u1.y; x8[6] = u1.z; x8[7] = u1.w;
-        st_chunk_s(sp + Lay::DTT + tc::tile_offset(64, row, chk), x8);
-      }
-      tc::fence_smem_to_async();
-      __syncthreads();
-    }
+    if (!aborted && __syncthreads_or(!wait_timed(cbar, cphase, a.wait_ns))) aborted = true;
+    cphase ^= 1;
     // ---- Y1 = Ai^T dT (columns 128..191) ----
     if (!aborted && tid == 0) {
       tc::fence_after_sync();
@@ -1075,46 +1092,30 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
                      tc::desc_kmajor(sb + Lay::Y1T, 64, s2), id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
-    // While they run: dP into rows 64..127 of XA (against Gram B) and columns
-    // 64..127 of YA (against the q x rows of Gram A).  XA row rho: first-half
-    // rows take column kappa = i, second-half rows kappa = 32 + i (Gram B rows
-    // 32..95 are k y against the second half's reference for every key).
-    // YA row i (second index, own reference): dP_ri for r in i's half; row
-    // 64 + i (i in the first half, second-half reference): dP_ri for r in the
-    // second half; rows 96..127 zero.
+    // While they run: dP into columns 64..127 of YA (against the q x rows of
+    // Gram A; rows 64..127 of XA came placed from the state part).  YA row i
+    // (second index, own reference): dP_ri for r in i's half; row 64 + i (i in
+    // the first half, second-half reference): dP_ri for r in the second half;
+    // rows 96..127 zero.
     if (!aborted) {
-      {   // all loads first, then the stores
-        const int r = tid >> 2, kq = (tid & 3) * 24;   // 24 columns of kappa each
-        float xv[24];
+      const int m = tid >> 1, rh = (tid & 1) * 32;   // YA row m, P columns r = rh..rh+31
+      float xv[32];
+      const int src = m < 64 ? m : (m < 96 ? m - 64 : 0);
 #pragma unroll
-        for (int e = 0; e < 24; ++e) {
-          const int kap = kq + e;
-          const int i = r < 32 ? kap : kap - 32;
-          const bool ok = (r < 32 ? kap < 32 : kap >= 32) && i <= r;
-          xv[e] = ok ? dP[r * 64 + i] : 0.f;
-        }
-#pragma unroll
-        for (int cc = 0; cc < 3; ++cc)
-          st_chunk_s(sp + Lay::XA + tc::tile_offset(128, 64 + r, (kq >> 3) + cc), xv + 8 * cc);
+      for (int e = 0; e < 32; e += 4) {
+        const float4 v4 = m < 96 ? *reinterpret_cast<const float4 *>(dPT + src * 64 + rh + e)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+        xv[e] = v4.x; xv[e + 1] = v4.y; xv[e + 2] = v4.z; xv[e + 3] = v4.w;
       }
-      {
-        const int m = tid >> 1, rh = (tid & 1) * 32;   // YA row m, P columns r = rh..rh+31
-        float xv[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int r = rh + e;
-          float val = 0.f;
-          if (m < 64) {
-            if ((m >> 5) == (r >> 5) && r >= m) val = dP[r * 64 + m];
-          } else if (m < 96) {
-            if (r >= 32) val = dP[r * 64 + (m - 64)];
-          }
-          xv[e] = val;
-        }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-          st_chunk_s(sp + Lay::YA + tc::tile_offset(128, m, 8 + (rh >> 3) + cc), xv + 8 * cc);
+      for (int e = 0; e < 32; ++e) {
+        const int r = rh + e;
+        const bool keep = m < 64 ? ((m >> 5) == (r >> 5) && r >= m) : (m < 96 && r >= 32);
+        xv[e] = keep ? xv[e] : 0.f;
       }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc)
+        st_chunk_s(sp + Lay::YA + tc::tile_offset(128, m, 8 + (rh >> 3) + cc), xv + 8 * cc);
     }
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
     phase ^= 1;
@@ -1317,7 +1318,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     report(a.dev_status, KDA_ERR_TIMEOUT);
     wait_timed(bar, phase, a.wait_ns);
     wait_timed(tbar, tphase, a.wait_ns);
-    if (PART == 0) wait_timed(cbar, cphase, a.wait_ns);
+    wait_timed(cbar, cphase, a.wait_ns);
     if (PART == 0 && s0pend) wait_timed(s0bar, s0phase, a.wait_ns);
   }
   tc::fence_before_sync();
@@ -1387,7 +1388,7 @@ BwdWs bwd_ws_layout(int N, int H, int64_t T) {
   w.dsl = off;    off += align256(P * 32768);
   w.ndu = off;    off += align256(P * 16384);
   w.dot = off;    off += align256(P * 16384);
-  w.dtp = off;    off += align256(P * 8192 * 4);
+  w.dtp = off;    off += align256(P * kDtpBytes);
   w.oscr = off;   off += align256((size_t)T * H * kD * 2);
   w.pref = off;   off += align256((size_t)(N + 1) * 8);
   w.prefck = off; off += align256((size_t)(N + 1) * 8);
@@ -1419,7 +1420,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   uint8_t *dsl = base + w.dsl;
   uint8_t *ndu = base + w.ndu;
   uint8_t *dot = base + w.dot;
-  float *dtp = reinterpret_cast<float *>(base + w.dtp);
+  uint8_t *dtp = base + w.dtp;
   void *oscr = base + w.oscr;
   int64_t *pref = reinterpret_cast<int64_t *>(base + w.pref);
   int64_t *prefck = reinterpret_cast<int64_t *>(base + w.prefck);

@@ -262,7 +262,8 @@ def test_chunked_backward_workspace():
     """BF16, D_k = D_v = 128: the chunked tensor-core backward's workspace holds, per
     (64-token chunk, head) of an upper bound of the chunk count, the forward's
     74,240-byte packet, dS at the chunk's end as a BF16 tile (32 KiB), the -dU and
-    dO tiles (16 KiB each) and dT, dP (FP32, 32 KiB); per full chunk the stored
+    dO tiles (16 KiB each), dT as a BF16 tile, dP placed as BF16 tile rows and dP^T in
+    FP32 (40 KiB together); per full chunk the stored
     forward state as a BF16 operand tile (32 KiB); per (sequence, head) the initial
     state as such a tile; per (chunk, head) the forward's T and (I + M)^-1 as BF16
     tiles (16 KiB); the forward's output (BF16); two prefix tables."""
@@ -275,7 +276,7 @@ def test_chunked_backward_workspace():
         assert P >= H * sum(-(-L // 64) for L in lengths)
         want = (al(P * 74240 + 256) + al((T // 64) * H * 32768) + al(N * H * 32768) + al(P * 16384)
                 + al(P * 32768) + al(P * 16384)
-                + al(P * 16384) + al(P * 32768) + al(T * H * 256) + 2 * al((N + 1) * 8) + 256)
+                + al(P * 16384) + al(P * 40960) + al(T * H * 256) + 2 * al((N + 1) * 8) + 256)
         assert lib.kda_backward_workspace_bytes(ctypes.byref(s)) == want
     # FP32 inputs keep the SIMT kernel's workspace
     s = kda.make_shape(4, 4096, 32, 128, 128, 0, kda.KDA_DTYPE_F32)
