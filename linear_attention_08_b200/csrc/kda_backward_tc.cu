@@ -390,7 +390,7 @@ struct BItemLayout {
   static_assert(GG + 17408 <= TT && MT + 4224 <= GG, "G");
   static_assert(YS + 2048 <= ZS && DST + 32768 <= YS, "scan scratch clears dS_L");
   static_assert(GB + 24576 <= RU + 32768 && RU + 32768 <= GST, "[R; U] stays clear of Gam");
-  static_assert(CST + 6144 <= XM + 17408, "gate factors");
+  static_assert(CST + 6144 <= XM + 17408 && ZS + 6144 <= GG, "gate factors");
   static_assert(TOTAL + 1024 <= 232448, "shared memory");
 };
 
@@ -446,7 +446,8 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 
   float *s_beta = reinterpret_cast<float *>(sp + Lay::BETA);
   float *s_red = reinterpret_cast<float *>(sp + Lay::RED);
-  float *s_cst = reinterpret_cast<float *>(sp + Lay::CST);
+  // gate factors during the prep (the Gram part keeps YA's second block free for dP^T)
+  float *s_cst = reinterpret_cast<float *>(sp + (PART == 0 ? Lay::CST : Lay::ZS));
   float *s_Y = reinterpret_cast<float *>(sp + Lay::YS);
   float *s_G = reinterpret_cast<float *>(sp + Lay::GG);
   float *s_gam = reinterpret_cast<float *>(sp + Lay::GST);
@@ -565,10 +566,11 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   }
   if (PART == 1 && tid == 32) {   // dT's operand tile and the placed dP rows of [dG; dP]
     const uint8_t *dt = a.dtp + (size_t)p * kDtpBytes;
-    mbar_expect_tx(sb + Lay::CBAR, 24576);
+    mbar_expect_tx(sb + Lay::CBAR, 40960);
     bulk_load(sb + Lay::DTT, dt, 8192, sb + Lay::CBAR);
     bulk_load(sb + Lay::XA + 8192, dt + 8192, 8192, sb + Lay::CBAR);
     bulk_load(sb + Lay::XA + 16384 + 8192, dt + 16384, 8192, sb + Lay::CBAR);
+    bulk_load(sb + Lay::YA + 16384, dt + 24576, 16384, sb + Lay::CBAR);   // dP^T (FP32) where its tile goes
   }
 
   cp_async_wait_all();
@@ -936,9 +938,14 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) put(8 + cc, d2 + 8 * cc);
       }
+      // dP^T row i (64 floats): float4 slot f stored at f ^ (i & 15), so that the
+      // Gram part's reads of one slot of 16 consecutive rows spread over the banks
       float *dpt = reinterpret_cast<float *>(dtp + 24576);
 #pragma unroll
-      for (int e = 0; e < 32; ++e) dpt[(32 * hw + e) * 64 + r] = d2[e];
+      for (int e = 0; e < 32; ++e) {
+        const int i = 32 * hw + e;
+        dpt[i * 64 + ((((r >> 2) ^ (i & 15))) << 2) + (r & 3)] = d2[e];
+      }
     }
     uint4 raw[8];
     {
@@ -1044,7 +1051,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     }
   } else {
     // ---- PART 1: dT (its operand tile) and dP from the state part ----
-    const float *dPT = reinterpret_cast<const float *>(a.dtp + (size_t)p * kDtpBytes + 24576);
+    const float *dPT = reinterpret_cast<const float *>(sp + Lay::YA + 16384);   // FP32 [64][64], copied in
     float *s_db = s_dd;   // dbeta [64]
     if (!aborted && __syncthreads_or(!wait_timed(cbar, cphase, a.wait_ns))) aborted = true;
     cphase ^= 1;
@@ -1097,13 +1104,14 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     // (second index, own reference): dP_ri for r in i's half; row 64 + i (i in
     // the first half, second-half reference): dP_ri for r in the second half;
     // rows 96..127 zero.
-    if (!aborted) {
+    if (!aborted) {   // read every FP32 value, then write the tile over them
       const int m = tid >> 1, rh = (tid & 1) * 32;   // YA row m, P columns r = rh..rh+31
       float xv[32];
       const int src = m < 64 ? m : (m < 96 ? m - 64 : 0);
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
-        const float4 v4 = m < 96 ? *reinterpret_cast<const float4 *>(dPT + src * 64 + rh + e)
+        const int f = (rh + e) >> 2;   // float4 slot of columns r = rh + e .. +3, stored at f ^ (src & 15)
+        const float4 v4 = m < 96 ? *reinterpret_cast<const float4 *>(dPT + src * 64 + ((f ^ (src & 15)) << 2))
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
         xv[e] = v4.x; xv[e + 1] = v4.y; xv[e + 2] = v4.z; xv[e + 3] = v4.w;
       }
@@ -1113,6 +1121,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         const bool keep = m < 64 ? ((m >> 5) == (r >> 5) && r >= m) : (m < 96 && r >= 32);
         xv[e] = keep ? xv[e] : 0.f;
       }
+      __syncthreads();
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc)
         st_chunk_s(sp + Lay::YA + tc::tile_offset(128, m, 8 + (rh >> 3) + cc), xv + 8 * cc);
