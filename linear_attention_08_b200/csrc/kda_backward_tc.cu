@@ -1373,11 +1373,15 @@ bwd_init_tiles_kernel(const float *__restrict__ init, uint8_t *__restrict__ tile
   const int unit = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float *src = init + (size_t)unit * kD * kD;
   uint8_t *dst = tiles + (size_t)unit * 32768;
-  for (int row = warp; row < kD; row += kThreads / 32) {
-    const float4 x = reinterpret_cast<const float4 *>(src + (size_t)row * kD)[lane];
-    *reinterpret_cast<uint2 *>(dst + tc::tile_offset(128, row, lane >> 1) + 8 * (lane & 1)) =
-        make_uint2(tc::pack_bf16(x.x, x.y), tc::pack_bf16(x.z, x.w));
-  }
+  constexpr int kRows = kD / (kThreads / 32);   // rows per warp: all loads first, then the stores
+  float4 x[kRows];
+#pragma unroll
+  for (int i = 0; i < kRows; ++i)
+    x[i] = reinterpret_cast<const float4 *>(src + (size_t)(warp + 8 * i) * kD)[lane];
+#pragma unroll
+  for (int i = 0; i < kRows; ++i)
+    *reinterpret_cast<uint2 *>(dst + tc::tile_offset(128, warp + 8 * i, lane >> 1) + 8 * (lane & 1)) =
+        make_uint2(tc::pack_bf16(x[i].x, x[i].y), tc::pack_bf16(x[i].z, x[i].w));
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
