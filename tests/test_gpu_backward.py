@@ -107,6 +107,17 @@ def test_chunked_backward_ragged(lengths):
     run_both(lengths, 3, 128, 128, torch.bfloat16, seed=len(lengths) + lengths[0])
 
 
+def test_chunked_backward_many_items_per_cta():
+    """More (chunk, head) items than CTAs (one per SM), over ragged sequences:
+    every CTA walks several items, so the next item's inputs are copied in
+    during the current item's reverse scan, across sequence boundaries, partial
+    chunks and first chunks (initial state); the state part's S0 then comes
+    from the initial-state tiles and the forward's chunk-end tiles alike."""
+    rng = np.random.default_rng(77)
+    lengths = [int(x) for x in rng.integers(1, 400, size=24)] + [64, 128, 1]
+    run_both(lengths, 8, 128, 128, torch.bfloat16, seed=78)
+
+
 @pytest.mark.parametrize("case", ["g_floor", "g_zero", "beta_zero", "beta_one",
                                   "strong_decay_16_32", "alternate_8"])
 def test_chunked_backward_gate_extremes(case):
