@@ -107,6 +107,14 @@ def test_chunked_backward_ragged(lengths):
     run_both(lengths, 3, 128, 128, torch.bfloat16, seed=len(lengths) + lengths[0])
 
 
+def test_chunked_backward_with_empty_sequences():
+    """Empty sequences inside a batch on the chunked path: they own no chunk,
+    so their d_init is the final-state gradient passed through, and the
+    sequences around them keep their packet, state and item numbering."""
+    errs = run_both([0, 70, 0, 5, 0], 2, 128, 128, torch.bfloat16, seed=79)
+    assert errs["d_init"] <= 1e-2
+
+
 def test_chunked_backward_many_items_per_cta():
     """More (chunk, head) items than CTAs (one per SM), over ragged sequences:
     every CTA walks several items, so the next item's inputs are copied in
