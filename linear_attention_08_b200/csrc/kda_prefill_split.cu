@@ -312,7 +312,7 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
       // q and k must have landed too before the rows are scaled.
       if (__syncthreads_or(!wait_timed(tbar, tphase, wait_ns))) { aborted = true; break; }
       tphase ^= 1;
-      float2 nref[2], fk[2], fk2[2], fh[2], fh2[2], cb[2];
+      float2 nref[2], fk[2], fk2[2];   // fh, fh2, cb (used once per row) stay in shared memory
       {
         auto ld4 = [&](int j, float2 *d) {
           const float4 v = *reinterpret_cast<const float4 *>(s_cst + (hf * 6 + j) * 128 + 4 * lane);
@@ -327,7 +327,7 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
         for (int i = 0; i < 8; ++i)
 #pragma unroll
           for (int j = 0; j < 2; ++j) gm[i][j] = __fadd2_rn(gm[i][j], base[j]);
-        ld4(0, nref); ld4(1, fk); ld4(2, fk2); ld4(3, fh); ld4(4, fh2); ld4(5, cb);
+        ld4(0, nref); ld4(1, fk); ld4(2, fk2);
       }
       auto st4 = [&](uint8_t *dst, const float2 *x) {
         *reinterpret_cast<uint2 *>(dst) = make_uint2(tc::pack_bf16(x[0].x, x[0].y), tc::pack_bf16(x[1].x, x[1].y));
@@ -370,7 +370,10 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
         st4(sp + Lay::GB + tc::tile_offset(96, hf ? 32 + r : r, cq) + sub, t);
         if (!hf) {
 #pragma unroll
-          for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], __fmul2_rn(y[j], cb[j]));
+          for (int j = 0; j < 2; ++j) {
+            const float2 cb = reinterpret_cast<const float2 *>(s_cst + (hf * 6 + 5) * 128 + 4 * lane)[j];
+            t[j] = __fmul2_rn(kk[j], __fmul2_rn(y[j], cb));
+          }
           st4(sp + Lay::GB + tc::tile_offset(96, 32 + r, cq) + sub, t);
         }
         // Ktilde, Qtilde: exp(Gam_r) = (x fk) fk2.
@@ -384,7 +387,11 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
         st4(pk + Packet::WQ + tc::tile_offset(128, 64 + r, cq) + sub, t);
         // Khat: exp(Gam_last - Gam_r) = (y fh) fh2.
 #pragma unroll
-        for (int j = 0; j < 2; ++j) t[j] = __fmul2_rn(kk[j], __fmul2_rn(__fmul2_rn(y[j], fh[j]), fh2[j]));
+        for (int j = 0; j < 2; ++j) {
+          const float2 fh = reinterpret_cast<const float2 *>(s_cst + (hf * 6 + 3) * 128 + 4 * lane)[j];
+          const float2 fh2 = reinterpret_cast<const float2 *>(s_cst + (hf * 6 + 4) * 128 + 4 * lane)[j];
+          t[j] = __fmul2_rn(kk[j], __fmul2_rn(__fmul2_rn(y[j], fh), fh2));
+        }
         st4(pk + Packet::KH + tc::tile_offset(64, r, cq) + sub, t);
       }
       tc::fence_smem_to_async();
