@@ -113,40 +113,53 @@ struct BChainLayout {
 };
 
 // The chunk's dO as the BF16 operand tile [64 tokens][128 value columns]
-// (rows past the sequence's end zero), for every packet: one CTA per packet.
+// (rows past the sequence's end zero), for every packet: two packets per CTA.
 __global__ void __launch_bounds__(kThreads)
 bwd_dout_tiles_kernel(const float *__restrict__ dout, const int32_t *__restrict__ cu,
                       const int64_t *__restrict__ pref, int N, int H, uint8_t *__restrict__ tiles) {
+  // Two items per CTA: both items' rows are loaded before any store.
   const int64_t total = pref[N] * H;
-  const int64_t p = blockIdx.x;
-  if (p >= total) return;
-  int lo = 0, hi = N - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (pref[mid] * H <= p) lo = mid; else hi = mid - 1;
-  }
-  const int n = lo;
-  const int64_t nch = pref[n + 1] - pref[n];
-  const int64_t rem = p - pref[n] * H;
-  const int h = (int)(rem / nch);
-  const int64_t j = rem - (int64_t)h * nch;
-  const int64_t t0 = (int64_t)cu[n] + kC * j;
-  const int64_t T_n = (int64_t)cu[n + 1] - cu[n];
-  const int L = (int)(T_n - kC * j < kC ? T_n - kC * j : kC);
   const int tid = threadIdx.x, r = tid >> 2, c0 = (tid & 3) * 32;
-  float x[32];
-  const float *src = dout + ((size_t)(t0 + r) * H + h) * kD + c0;
+  float x[2][32];
+  int64_t pp[2];
 #pragma unroll
-  for (int e = 0; e < 32; e += 4) {
-    const float4 v4 = r < L ? *reinterpret_cast<const float4 *>(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-    x[e] = v4.x; x[e + 1] = v4.y; x[e + 2] = v4.z; x[e + 3] = v4.w;
+  for (int it = 0; it < 2; ++it) {
+    const int64_t p = 2 * (int64_t)blockIdx.x + it;
+    pp[it] = p;
+    int L = 0;
+    const float *src = dout;
+    if (p < total) {
+      int lo = 0, hi = N - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pref[mid] * H <= p) lo = mid; else hi = mid - 1;
+      }
+      const int n = lo;
+      const int64_t nch = pref[n + 1] - pref[n];
+      const int64_t rem = p - pref[n] * H;
+      const int h = (int)(rem / nch);
+      const int64_t j = rem - (int64_t)h * nch;
+      const int64_t t0 = (int64_t)cu[n] + kC * j;
+      const int64_t T_n = (int64_t)cu[n + 1] - cu[n];
+      L = (int)(T_n - kC * j < kC ? T_n - kC * j : kC);
+      src = dout + ((size_t)(t0 + r) * H + h) * kD + c0;
+    }
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      const float4 v4 = r < L ? *reinterpret_cast<const float4 *>(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+      x[it][e] = v4.x; x[it][e + 1] = v4.y; x[it][e + 2] = v4.z; x[it][e + 3] = v4.w;
+    }
   }
-  uint8_t *dst = tiles + (size_t)p * 16384;
 #pragma unroll
-  for (int e = 0; e < 32; e += 8)
-    *reinterpret_cast<uint4 *>(dst + tc::tile_offset(64, r, (c0 + e) >> 3)) =
-        make_uint4(tc::pack_bf16(x[e], x[e + 1]), tc::pack_bf16(x[e + 2], x[e + 3]),
-                   tc::pack_bf16(x[e + 4], x[e + 5]), tc::pack_bf16(x[e + 6], x[e + 7]));
+  for (int it = 0; it < 2; ++it) {
+    if (pp[it] >= total) continue;
+    uint8_t *dst = tiles + (size_t)pp[it] * 16384;
+#pragma unroll
+    for (int e = 0; e < 32; e += 8)
+      *reinterpret_cast<uint4 *>(dst + tc::tile_offset(64, r, (c0 + e) >> 3)) =
+          make_uint4(tc::pack_bf16(x[it][e], x[it][e + 1]), tc::pack_bf16(x[it][e + 2], x[it][e + 3]),
+                     tc::pack_bf16(x[it][e + 4], x[it][e + 5]), tc::pack_bf16(x[it][e + 6], x[it][e + 7]));
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1452,7 +1465,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const int64_t P_max = (int64_t)H * ((T + (int64_t)(kC - 1) * N) / kC);
-  bwd_dout_tiles_kernel<<<(unsigned)P_max, kThreads, 0, stream>>>(dout, cu, pref, N, H, dot);
+  bwd_dout_tiles_kernel<<<(unsigned)((P_max + 1) / 2), kThreads, 0, stream>>>(dout, cu, pref, N, H, dot);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   TmaMaps maps;
