@@ -426,6 +426,49 @@ def time_decode(steps_graph, warmup, world, local, decode_steps=None):
                 flops=token_heads * decode_flops_per_token_head(Dk), clocks=clk.result)
 
 
+def time_prefill_at(steps, warmup, world, local, positions=(1000, 3000, 5000, 7777)):
+    """Prefill with states at explicit positions (prompt boundaries): the
+    headline workload (4 x 8192 tokens, H=32, D=128, BF16) with the state also
+    taken after each of `positions` tokens of every sequence (kda_prefill_at)."""
+    from linear_attention_08_b200 import kda
+    w = kin.WORKLOADS["prefill"]
+    d = kin.make_workload("prefill", device="cuda", seed=local)
+    lengths, cu = d["lengths"], d["cu_seqlens"]
+    N, H, Dk, Dv, C = len(lengths), w["H"], w["Dk"], w["Dv"], w["chunk"]
+    cu_dev = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    pos_cu = torch.tensor([len(positions) * n for n in range(N + 1)], dtype=torch.int32, device="cuda")
+    pos = torch.tensor(list(positions) * N, dtype=torch.int32, device="cuda")
+    out = torch.empty_like(d["v"])
+    fin = torch.empty(N, H, Dk, Dv, device="cuda")
+    pos_states = torch.empty(N * len(positions), H, Dk, Dv, device="cuda")
+    lib = kda.load()
+    shape = kda.make_shape(N, sum(lengths), H, Dk, Dv, C, kda.KDA_DTYPE_BF16)
+    stream = torch.cuda.current_stream()
+    P = kda._ptr
+
+    def step():
+        st = lib.kda_prefill_at(P(d["q"]), P(d["k"]), P(d["v"]), P(d["g"]), P(d["beta"]), None,
+                                P(cu_dev), P(out), P(fin), 0, None, P(pos_cu), P(pos),
+                                P(pos_states), kda.ctypes.byref(shape), kda._stream(stream))
+        assert st == kda.KDA_OK, st
+
+    for _ in range(max(warmup, 1)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b) / steps, world)
+    flops, byts = prefill_algorithmic(lengths, H, Dk, Dv, C, 2, 0, False)
+    byts += N * len(positions) * H * Dk * Dv * 4
+    return dict(tokens=sum(lengths), ms=ms, bytes=byts, flops=flops, positions=list(positions), N=N,
+                H=H, T=lengths[0])
+
+
 def time_spec_decode(steps, warmup, world, local, T_new=8, N=512):
     """Multi-token decode: N (512) sequences x 32 heads, T_new draft tokens each,
     all accepted.  One call moves the FP32 state once for T_new tokens."""
@@ -512,6 +555,9 @@ def run_ours(args, rank, world, local):
             extra[other] = time_prefill(other, 3 if other == "long" else 10, args.warmup, world,
                                         local, e2e=False)
             torch.cuda.empty_cache()
+    pat = None
+    if name == "prefill" and not args.no_extra_prefill:
+        pat = time_prefill_at(10, args.warmup, world, local)
     bwd = None
     if not args.no_backward and name == "prefill":
         bwd = time_backward(max(1, min(args.steps, 3)), args.warmup, world, local)
@@ -553,6 +599,17 @@ def run_ours(args, rank, world, local):
         }
         for other, ro in extra.items():
             line[other] = prefill_object(ro, world, hbm, tflops, peaks_src)
+        if pat is not None:
+            pgbs = pat["bytes"] / (pat["ms"] / 1e3) / 1e9
+            line["prefill_at"] = {
+                "metric": "KDA prefill tokens/s, states at prompt boundaries",
+                "value": world * pat["tokens"] / (pat["ms"] / 1e3), "unit": "tokens/s",
+                "ms_per_call": pat["ms"],
+                "config": {"workload": "prefill_at", "num_seqs": pat["N"], "seq_len": pat["T"],
+                           "heads": pat["H"], "d": 128, "positions_per_seq": pat["positions"]},
+                "roofline": {"bound": "hbm", "achieved": pgbs, "peak": hbm, "unit": "GB/s",
+                             "frac": pgbs / hbm, "kernel": "prefill_tc", "traffic": None,
+                             "note": "single-pass kernel (explicit positions); operator bytes incl. the position states"}}
         if bwd is not None:
             bgbs = bwd["bytes"] / (bwd["ms"] / 1e3) / 1e9
             line["backward"] = {
