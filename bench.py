@@ -83,7 +83,9 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "decode": ("kda_decode.cu", "kda_common.cuh"),
-    "decode_multi": ("kda_decode_multi.cu", "kda_common.cuh"),
+    # BF16, D = 128, drafts up to 16 tokens: the tensor-core form; others: CUDA cores
+    "decode_multi": ("kda_decode_multi.cu", "kda_decode_multi_tc.cu", "kda_tc_util.cuh",
+                     "kda_tma.cuh", "kda_common.cuh"),
     "prefill_tc": ("kda_prefill_tc.cu", "kda_tc_util.cuh", "kda_tma.cuh", "kda_common.cuh"),
     # two-pass path: intra-chunk pass + chain pass, one prefill call = one launch of each
     "prefill_split": ("kda_prefill_split.cu", "kda_tc_util.cuh", "kda_tma.cuh", "kda_common.cuh"),
@@ -647,7 +649,8 @@ def run_ours(args, rank, world, local):
                 "config": {"num_seqs": 512, "heads": 32, "d": 128, "tokens_per_seq": spec["T_new"],
                            "accepted": "all"},
                 "roofline": {"bound": "hbm", "achieved": sgbs, "peak": hbm, "unit": "GB/s",
-                             "frac": sgbs / hbm, "kernel": "decode_multi"}}
+                             "frac": sgbs / hbm, "traffic": ncu_traffic("decode_multi"),
+                             "kernel": "decode_multi", "peak_source": peaks_src}}
         if res is None:
             line = dict(dobj)
             line.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
