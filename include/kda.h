@@ -223,10 +223,14 @@ kda_status kda_decode(const void *q, const void *k, const void *v, const float *
  *   beta    : [N, tokens_per_seq, H]         accept_len : device int32[N] or NULL
  *   state_inout : [N, H, D_k, D_v]
  * shape->total_tokens must equal N * tokens_per_seq; 1 <= tokens_per_seq <= 64.
- * Values of accept_len outside [0, tokens_per_seq] are clamped.  This is the
- * recurrence of the decode step applied token by token (the first page,
- * Methods 1: decode runs the recurrence directly); the serving side that
- * decides acceptance is not part of this library.
+ * Values of accept_len outside [0, tokens_per_seq] are clamped.  The result
+ * is the recurrence of the decode step applied token by token (the first
+ * page, Methods 1: decode runs the recurrence directly).  BF16 inputs with
+ * D_k = D_v = 128 and at most 16 tokens compute it as one chunk of the
+ * chunked form (Methods 1, FlashKDA) on the tensor cores, with S0 rounded to
+ * BF16 as an operand and the state updated in FP32; other shapes run the
+ * recurrence on the CUDA cores.  The serving side that decides acceptance is
+ * not part of this library.
  */
 kda_status kda_decode_multi(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, float *state_inout, void *out,
