@@ -186,10 +186,9 @@ decode_multi_tc_kernel(const __grid_constant__ MtcMaps maps, const float *__rest
 
     // ---- the unit's rows; Gam (in place), beta and exp(Gam_a) ----
     if (__syncthreads_or(!wait_timed(bars + 1, rph, wait_ns))) { aborted = true; break; }
-    if (warp == 0) cp_async_wait_all();   // beta
+    if (warp == 0) cp_async_wait_all();   // beta, published by the barrier below
     rph ^= 1;
     pend &= ~2u;
-    __syncthreads();
     if (tid < kMD) {
       float gv[MC];
 #pragma unroll
@@ -313,14 +312,13 @@ decode_multi_tc_kernel(const __grid_constant__ MtcMaps maps, const float *__rest
       }
     }
     tc::fence_smem_to_async();   // operand tiles for the products; raw rows refilled below
-    __syncthreads();
-    if (u + G < units) load_raw(u + G);
 
     // ---- S0 -> TMEM (scaled by exp(Gam_a)) and -> the BF16 operand S0^T, which
     //      takes the place of the FP32 rows once every thread has read its column ----
     if (__syncthreads_or(!wait_timed(bars + 0, sph, wait_ns))) { aborted = true; break; }
     sph ^= 1;
     pend &= ~1u;
+    if (u + G < units) load_raw(u + G);   // every thread is past its last read of the rows
     {
       const float *sf = reinterpret_cast<const float *>(sp + Lay::SF);
       uint32_t pk[32];   // the thread's 64 values of S0 as BF16 pairs
@@ -423,8 +421,9 @@ decode_multi_tc_kernel(const __grid_constant__ MtcMaps maps, const float *__rest
         for (int e = 0; e < 32; ++e) __stcs(so + (size_t)(k0 + e) * kMD, y[e]);
       }
     }
+    // No barrier here: the next unit's first wait is one, and every thread
+    // reads (state out) and later writes (state in) the same TMEM columns.
     tc::fence_before_sync();
-    __syncthreads();   // TMEM and the operand tiles are reused by the next unit
   }
 
   if (aborted) {
