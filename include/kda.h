@@ -109,9 +109,11 @@ typedef struct {
  * chunk 16 and chunk 64 alike.  The tensor-core kernels group tokens in
  * chunks of 64 with 16-token diagonal blocks inside; the result does not
  * depend on the chunk size, which the caller names only to fix which
- * checkpoint intervals are valid.  With up to 1024 sequences and an interval
- * that is 0 or a multiple of 64 the call runs the two-pass kernels through
- * the workspace pool; more sequences, or an interval of 16, 32 or 48 modulo
+ * checkpoint intervals are valid.  With up to 1024 sequences and 2048
+ * (sequence, head) units and an interval that is 0 or a multiple of 64 the
+ * call runs the two-pass kernels through the workspace pool, unless the
+ * windows that workspace allows would cost more than the work (see
+ * kda_prefill_path); larger batches, or an interval of 16, 32 or 48 modulo
  * 64, run the single-pass tensor-core kernel.  Other shapes (FP32, smaller
  * heads) run the FP32 SIMT kernel.
  */
@@ -127,7 +129,8 @@ kda_status kda_prefill(const void *q, const void *k, const void *v, const float 
  * chain over them.  workspace_bytes >= kda_prefill_workspace_bytes(shape)
  * runs the whole batch in one window; a smaller workspace (at least
  * kda_prefill_workspace_min_bytes) runs it in several windows of chunks.
- * A NULL or too small workspace, or a shape off the two-pass path, runs the
+ * A NULL or too small workspace, a shape off the two-pass path, or windows
+ * that would cost more than the work (see kda_prefill_path) run the
  * single-pass kernels, which need none.  The workspace must be 16-byte
  * aligned (256 is best), must not overlap any argument, and is free again
  * when the work queued on `stream` completes.  kda_prefill itself takes its
@@ -157,8 +160,10 @@ kda_status kda_prefill_ws(const void *q, const void *k, const void *v, const flo
  * (kda_prefill_path = 2) are accepted, and only when one chunk of every
  * (sequence, head) fits the array: num_seqs * num_heads * 74240 bytes, plus
  * num_seqs * num_heads * 65536 when final_state is NULL, plus 256, at most
- * KDA_NOALLOC_SCRATCH_BYTES; longer batches run in windows of chunks.  Other
- * shapes return KDA_ERR_UNSUPPORTED before any work is queued.
+ * KDA_NOALLOC_SCRATCH_BYTES; longer batches run in windows of chunks, or on
+ * the single-pass kernel (which needs no workspace) where those windows would
+ * cost more than the work, as in kda_prefill_ws.  Other shapes return
+ * KDA_ERR_UNSUPPORTED before any work is queued.
  * The first call on a device looks up the array's device address, so make
  * that first call before any stream capture.  The address is kept for the
  * life of the process: after cudaDeviceReset (or anything else that tears
@@ -327,13 +332,23 @@ kda_status kda_release_workspace_pool(void);
  * takes nothing from the pool; 0 therefore keeps the pool unused. */
 kda_status kda_set_workspace_pool_cap(size_t bytes);
 
-/* Which prefill kernel a shape runs on without explicit positions, with a
- * workspace and an interval that is 0 or a multiple of 64:
- * 2 = two-pass tcgen05 tensor-core kernels (intra-chunk pass + chain; up to
- *     1024 sequences per call),
+/* Which prefill kernel kda_prefill runs a shape on without explicit
+ * positions, with an interval that is 0 or a multiple of 64 and the workspace
+ * its pool cap allows:
+ * 2 = two-pass tcgen05 tensor-core kernels (intra-chunk pass + chain): at most
+ *     1024 sequences and 2048 (sequence, head) units, and only when the
+ *     windows of chunks the workspace allows are worth it (below),
  * 1 = single-pass tcgen05 kernel (also used with explicit positions, without
- *     a workspace, for other intervals and for more than 1024 sequences),
- * 0 = SIMT FP32 kernel, -1 = invalid shape. */
+ *     a workspace, for other intervals, and for larger batches, where its
+ *     one CTA per (sequence, head) has the parallelism: from 4096 units on
+ *     B200 it is the faster of the two),
+ * 0 = SIMT FP32 kernel, -1 = invalid shape.
+ * Windows: the host does not know the longest sequence, so a batch that does
+ * not fit its workspace runs windows up to ceil(T_tot / 64) chunks, and those
+ * past the longest sequence still cost both launches (about 5 us plus 6 ns
+ * per unit each).  When that cost is over 5 % of the work (at about 35 M
+ * tokens/s) and over 1 ms, kda_prefill and kda_prefill_ws run the single
+ * pass instead. */
 int kda_prefill_path(const kda_shape *shape);
 
 /* The kernel (2, 1 or 0 as above) that the last kda_prefill,

@@ -32,6 +32,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
 bool prefill_split_supported(int N);
 size_t split_packet_bytes();
 size_t split_workspace_full(int N, int H, int64_t T, bool have_final);
+int64_t split_windows(int N, int H, int64_t T, size_t ws_bytes, bool have_final);
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const float *init, const int32_t *cu, void *out,
                                  float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
@@ -117,8 +118,31 @@ static bool tc_shape(const kda_shape *s) {
          (s->chunk == 16 || s->chunk == 64);
 }
 
+// Up to 2048 (sequence, head) units the two-pass kernels are faster (34.9 vs
+// 31.8 M tokens/s at 128 units on B200, BF16, D = 128, H = 32; equal at
+// 2048); from 4096 units the single-pass grid has the parallelism and is 3 %
+// faster.
+constexpr int64_t kSplitMaxUnits = 2048;
+
 static bool split_path(const kda_shape *s) {
-  return tc_shape(s) && prefill_split_supported(s->num_seqs);
+  return tc_shape(s) && prefill_split_supported(s->num_seqs) &&
+         (int64_t)s->num_seqs * s->num_heads <= kSplitMaxUnits;
+}
+
+// Whether the windows the two-pass path would run with ws_bytes of workspace
+// are worth it.  A window the host cannot rule out (past the longest
+// sequence) still costs both launches, about 5 us + 6 ns per (sequence, head)
+// unit; with 1024 x 1024 tokens (H = 32) and an 8 GiB workspace that was 5461
+// windows, 1050 ms against 29 ms for the single pass.  The path is kept
+// unless those windows cost both more than 5 % of the work (at about 35 M
+// tokens/s) and more than 1 ms.
+static bool split_worthwhile(const kda_shape *s, size_t ws_bytes, bool have_final) {
+  const int64_t units = (int64_t)s->num_seqs * s->num_heads;
+  const int64_t w = split_windows(s->num_seqs, s->num_heads, s->total_tokens, ws_bytes, have_final);
+  if (w < 1) return false;
+  const double idle_us = (double)(w - 1) * (5.0 + 0.006 * (double)units);
+  const double work_us = (double)s->total_tokens / 35.0;
+  return idle_us <= 0.05 * work_us || idle_us <= 1000.0;
 }
 
 static size_t split_min_bytes(const kda_shape *s, bool have_final) {
@@ -215,7 +239,12 @@ kda_status kda_release_workspace_pool(void) {
 
 int kda_prefill_path(const kda_shape *s) {
   if (check_shape(s, true) != KDA_OK) return -1;
-  if (split_path(s)) return 2;
+  if (split_path(s)) {   // as kda_prefill would run it, with a workspace from the pool
+    size_t want = split_workspace_full(s->num_seqs, s->num_heads, s->total_tokens, false);
+    const size_t cap = g_pool_cap.load();
+    if (want > cap) want = cap;
+    if (want >= split_min_bytes(s, false) && split_worthwhile(s, want, false)) return 2;
+  }
   return tc_shape(s) ? 1 : 0;
 }
 
@@ -291,7 +320,8 @@ static kda_status prefill_impl(const void *q, const void *k, const void *v, cons
   if (T > 0 && !positions && ws_mode != WS_NONE && split_path(s) && ckpt_interval % 64 == 0) {
     // Two-pass path when a large enough workspace is at hand.
     const size_t need_min = split_min_bytes(s, final_state != nullptr);
-    if (ws_mode == WS_CALLER && workspace && ws_bytes >= need_min) {
+    if (ws_mode == WS_CALLER && workspace && ws_bytes >= need_min &&
+        split_worthwhile(s, ws_bytes, final_state != nullptr)) {
       g_last_path = 2;
       return cuda_status(launch_prefill_split(q, k, v, g, beta, init_state, cu_seqlens, out,
                                               final_state, ckpt_interval, ckpt_states, N, H, T,
@@ -304,7 +334,8 @@ static kda_status prefill_impl(const void *q, const void *k, const void *v, cons
       size_t want = split_workspace_full(N, H, T, final_state != nullptr);
       if (want > cap) want = cap;
       void *ws = nullptr;
-      if (device_pool(dev, &pool) == cudaSuccess &&
+      if (split_worthwhile(s, want, final_state != nullptr) &&
+          device_pool(dev, &pool) == cudaSuccess &&
           cudaMallocFromPoolAsync(&ws, want, pool, cs) == cudaSuccess) {
         g_last_path = 2;
         e = launch_prefill_split(q, k, v, g, beta, init_state, cu_seqlens, out, final_state,

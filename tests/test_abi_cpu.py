@@ -128,6 +128,34 @@ def test_workspace_and_path_queries():
     assert kda.kda_prefill_path(kda.make_shape(2, 1000, 4, 128, 128, 16, kda.KDA_DTYPE_F32)) == 0
 
 
+def test_path_rules_units_and_windows():
+    """The two-pass path takes at most 2048 (sequence, head) units, and only
+    when the windows its workspace allows do not cost more than the work."""
+    lib = kda.load()
+    bf = kda.KDA_DTYPE_BF16
+    # 600 x 4 = 2400 units: the single pass, and no workspace is asked for
+    many = kda.make_shape(600, 600 * 64, 4, 128, 128, 64, bf)
+    assert kda.kda_prefill_path(many) == 1
+    assert lib.kda_prefill_workspace_bytes(ctypes.byref(many)) == 0
+    assert lib.kda_prefill_workspace_min_bytes(ctypes.byref(many)) == 0
+    # exactly 2048 units in one window: the two-pass path
+    assert kda.kda_prefill_path(kda.make_shape(64, 64 * 256, 32, 128, 128, 64, bf)) == 2
+    # one 1M-token sequence, 32 heads: five windows of an 8 GiB workspace, all of them real
+    assert kda.kda_prefill_path(kda.make_shape(1, 1 << 20, 32, 128, 128, 64, bf)) == 2
+    # 1000 sequences x 2 heads over 10^8 tokens: ~27K windows, most past the
+    # longest sequence, against ~2.9 s of work
+    assert kda.kda_prefill_path(kda.make_shape(1000, 100_000_000, 2, 128, 128, 64, bf)) == 1
+    # the pool cap bounds the workspace kda_prefill takes: at the minimum, the
+    # 64 x 256-token batch would run 256 one-chunk windows
+    small = kda.make_shape(64, 64 * 256, 32, 128, 128, 64, bf)
+    try:
+        kda.kda_set_workspace_pool_cap(lib.kda_prefill_workspace_min_bytes(ctypes.byref(small)))
+        assert kda.kda_prefill_path(small) == 1
+    finally:
+        kda.kda_set_workspace_pool_cap(8 << 30)
+    assert kda.kda_prefill_path(small) == 2
+
+
 def test_last_path_and_pool_cap():
     """The last-path query is untouched by a call that fails validation; the pool
     cap setter accepts any size (0 keeps the pool unused)."""

@@ -173,3 +173,24 @@ def test_pool_cap_fallback_is_visible():
             check(d, out, None, ck, 128)
     finally:
         kda.kda_set_workspace_pool_cap(8 << 30)
+
+
+def test_many_windows_run_the_single_pass():
+    """64 sequences x 256 tokens x 32 heads with the smallest caller workspace:
+    the two-pass path would run 256 one-chunk windows (most of them past every
+    sequence), so the single-pass kernel runs; with room for one window the
+    two-pass path runs.  Both against the oracle."""
+    lengths = [256] * 64
+    d = make_case(lengths, 32, 128, 128, torch.bfloat16, seed=41, state_std=0.02)
+    dd = to_device(d)
+    shape = shape_of(dd)
+    ws = torch.empty(kda.kda_prefill_workspace_min_bytes(shape), dtype=torch.uint8, device="cuda")
+    out, fin, _ = run(dd, 0, ws)
+    torch.cuda.synchronize()
+    assert kda.kda_last_prefill_path() == 1
+    check(d, out, fin, None, 0)
+    ws = torch.empty(kda.kda_prefill_workspace_bytes(shape), dtype=torch.uint8, device="cuda")
+    out, fin, _ = run(dd, 0, ws)
+    torch.cuda.synchronize()
+    assert kda.kda_last_prefill_path() == 2
+    check(d, out, fin, None, 0)
