@@ -8,7 +8,7 @@ append-prefill (8 sequences of 1K-32K tokens, checkpoints every 4096) and
 1M-token (snapshots every 32K) prefill workloads as two more.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload prefill|decode|append_varlen|long|prefill_small] [--no-decode] [--no-backward]
+                  [--workload prefill|decode|append_varlen|long|many_seqs|prefill_small] [--no-decode] [--no-backward]
                   [--no-extra-prefill]
 
 For N > 1 it is launched by torchrun, one rank per GPU; every rank runs its
@@ -333,7 +333,9 @@ def prefill_object(r, world, hbm, tflops, peaks_src):
         "metric": "KDA prefill tokens/s", "value": world * r["tokens"] / (ms / 1e3),
         "unit": "tokens/s", "ms_per_call": ms, "steps": r["steps"],
         "config": {"workload": w_name(w), "num_seqs": len(r["lengths"]),
-                   "total_tokens": r["tokens"], "seq_lens": sorted(r["lengths"]),
+                   "total_tokens": r["tokens"],
+                   "seq_lens": sorted(r["lengths"]) if len(r["lengths"]) <= 16 else
+                   {"min": min(r["lengths"]), "max": max(r["lengths"])},
                    "heads": w["H"], "d": w["Dk"], "chunk": w["chunk"],
                    "ckpt_interval": w["ckpt_interval"],
                    "init_state": "N(0, 0.02)" if w["state_std"] > 0 else "zero"},
@@ -553,7 +555,7 @@ def run_ours(args, rank, world, local):
         spec = time_spec_decode(max(args.steps, 5), args.warmup, world, local)
     extra = {}
     if name == "prefill" and not args.no_extra_prefill:
-        for other in ("append_varlen", "long"):
+        for other in ("append_varlen", "long", "many_seqs"):
             extra[other] = time_prefill(other, 3 if other == "long" else 10, args.warmup, world,
                                         local, e2e=False)
             torch.cuda.empty_cache()
@@ -736,7 +738,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill",
-                    choices=["prefill", "decode", "append_varlen", "long", "prefill_small"])
+                    choices=["prefill", "decode", "append_varlen", "long", "many_seqs",
+                             "prefill_small"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-extra-prefill", action="store_true",

@@ -95,6 +95,10 @@ WORKLOADS = {
                           ckpt_interval=4096),
     "long": dict(kind="prefill", num_seqs=1, seq_len=1048576, H=32, Dk=128, Dv=128,
                  chunk=64, dtype="bf16", state_std=0.0, ckpt_interval=32768),
+    # many short sequences: 32,768 (sequence, head) units, past the 2048 the
+    # two-pass path takes, so the single-pass kernel runs
+    "many_seqs": dict(kind="prefill", num_seqs=1024, seq_len=1024, H=32, Dk=128, Dv=128,
+                      chunk=64, dtype="bf16", state_std=0.0, ckpt_interval=0),
     # a smaller case of the prefill kernels, in the same launch configuration as
     # "prefill" (more than 74 (sequence, head) units), for profiler captures
     "prefill_small": dict(kind="prefill", num_seqs=2, seq_len=4096, H=40, Dk=128, Dv=128,
