@@ -32,7 +32,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
 bool prefill_split_supported(int N);
 size_t split_packet_bytes();
 size_t split_workspace_full(int N, int H, int64_t T, bool have_final);
-int64_t split_windows(int N, int H, int64_t T, size_t ws_bytes, bool have_final);
+
 cudaError_t launch_prefill_split(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const float *init, const int32_t *cu, void *out,
                                  float *fin, int64_t interval, float *ck, int N, int H, int64_t T,
@@ -127,6 +127,28 @@ constexpr int64_t kSplitMaxUnits = 2048;
 static bool split_path(const kda_shape *s) {
   return tc_shape(s) && prefill_split_supported(s->num_seqs) &&
          (int64_t)s->num_seqs * s->num_heads <= kSplitMaxUnits;
+}
+
+// Windows the two-pass prefill (launch_prefill_split) runs with ws_bytes of
+// workspace, 0 if it cannot run: the same count as its launcher makes.  The
+// host does not know the longest sequence, so windows are counted up to
+// ceil(T / 64) chunks; those past the longest sequence launch both passes with
+// nothing to do.
+static int64_t split_windows(int N, int H, int64_t T, size_t ws_bytes, bool have_final) {
+  if (!prefill_split_supported(N) || ws_bytes < 256) return 0;
+  const size_t packet = split_packet_bytes();
+  size_t avail = ws_bytes - 256;   // at most this much is lost to the 256-byte alignment
+  const int64_t max_chunks = (T + 63) / 64;
+  const size_t all_packets = (size_t)H * (size_t)((T + (int64_t)63 * N) / 64);
+  if (all_packets * packet <= avail) return 1;
+  const size_t state_bytes = (size_t)N * H * 128 * 128 * 4;
+  if (!have_final) {
+    if (avail < state_bytes) return 0;
+    avail -= state_bytes;
+  }
+  const int64_t wc = (int64_t)(avail / ((size_t)N * H * packet));
+  if (wc < 1) return 0;
+  return max_chunks > 0 ? (max_chunks + wc - 1) / wc : 1;
 }
 
 // Whether the windows the two-pass path would run with ws_bytes of workspace

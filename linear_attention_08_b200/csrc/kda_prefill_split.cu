@@ -967,26 +967,6 @@ size_t split_packet_bytes() { return Packet::BYTES; }
 
 bool prefill_split_supported(int N) { return N >= 1 && N <= kMaxSeqs; }
 
-// Windows launch_prefill_split runs with ws_bytes of workspace (0 if it cannot
-// run).  The host does not know the longest sequence, so windows are counted
-// up to ceil(T / 64) chunks; those past the longest sequence launch both passes
-// with nothing to do.
-int64_t split_windows(int N, int H, int64_t T, size_t ws_bytes, bool have_final) {
-  if (!prefill_split_supported(N) || ws_bytes < 256) return 0;
-  size_t avail = ws_bytes - 256;   // at most this much is lost to the 256-byte alignment
-  const int64_t max_chunks = (T + kC - 1) / kC;
-  const size_t all_packets = (size_t)H * (size_t)((T + (int64_t)(kC - 1) * N) / kC);
-  if (all_packets * Packet::BYTES <= avail) return 1;
-  const size_t state_bytes = (size_t)N * H * kDK * kDV * 4;
-  if (!have_final) {
-    if (avail < state_bytes) return 0;
-    avail -= state_bytes;
-  }
-  const int64_t wc = (int64_t)(avail / ((size_t)N * H * Packet::BYTES));
-  if (wc < 1) return 0;
-  return max_chunks > 0 ? (max_chunks + wc - 1) / wc : 1;
-}
-
 // Workspace that runs the whole batch as a single window (an upper bound:
 // every sequence may end in a partial chunk), plus the FP32 state carried
 // between windows when the caller keeps no final state.
