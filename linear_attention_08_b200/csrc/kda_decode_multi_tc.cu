@@ -207,11 +207,14 @@ decode_multi_tc_kernel(const __grid_constant__ MtcMaps maps, const float *__rest
     }
     __syncthreads();
 
-    // ---- gated Gram products L (s < t) and P (s <= t): 8 lanes per pair ----
+    // ---- gated Gram products L (s < t) and P (s <= t): 4 lanes per pair, 64
+    //      pairs per pass (one pass up to 8 tokens); group grp walks the 16-
+    //      channel blocks in the order i ^ grp, so the 8 groups of a warp read 8
+    //      different blocks of their rows at each step (no bank conflicts) ----
     {
-      const int np = C * (C + 1) / 2, grp = lane >> 3, sub = lane & 7;
-      for (int base = 0; base < np; base += 4 * (kMThreads / 32)) {
-        const int p = base + 4 * warp + grp;
+      const int np = C * (C + 1) / 2, grp = lane >> 2, sub = lane & 3;
+      for (int base = 0; base < np; base += 8 * (kMThreads / 32)) {
+        const int p = base + 8 * warp + grp;
         const bool ok = p < np;
         int t = 0, s = 0;
         if (ok) {
@@ -220,9 +223,9 @@ decode_multi_tc_kernel(const __grid_constant__ MtcMaps maps, const float *__rest
         }
         float kk = 0.f, qq = 0.f;
         if (ok) {
-#pragma unroll 2
-          for (int i = 0; i < 4; ++i) {
-            const int c = 4 * sub + 32 * i;
+#pragma unroll 4
+          for (int i = 0; i < 8; ++i) {
+            const int c = 16 * (i ^ grp) + 4 * sub;
             const float4 gt = *reinterpret_cast<const float4 *>(gam + t * kMD + c);
             const float4 gs = *reinterpret_cast<const float4 *>(gam + s * kMD + c);
             const float4 kt = ld4_bf16(rk + t * kMD + c), ks = ld4_bf16(rk + s * kMD + c);
@@ -235,7 +238,7 @@ decode_multi_tc_kernel(const __grid_constant__ MtcMaps maps, const float *__rest
           }
         }
 #pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
+        for (int o = 1; o < 4; o <<= 1) {
           kk += __shfl_xor_sync(0xffffffffu, kk, o);
           qq += __shfl_xor_sync(0xffffffffu, qq, o);
         }
