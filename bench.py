@@ -8,7 +8,7 @@ append-prefill (8 sequences of 1K-32K tokens, checkpoints every 4096) and
 1M-token (snapshots every 32K) prefill workloads as two more.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                  [--workload prefill|decode|append_varlen|long|many_seqs|prefill_small] [--no-decode] [--no-backward]
+                  [--workload prefill|decode|append_varlen|long|many_seqs|many_seqs_small|prefill_small] [--no-decode] [--no-backward]
                   [--no-extra-prefill]
 
 For N > 1 it is launched by torchrun, one rank per GPU; every rank runs its
@@ -739,7 +739,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="prefill",
                     choices=["prefill", "decode", "append_varlen", "long", "many_seqs",
-                             "prefill_small"])
+                             "many_seqs_small", "prefill_small"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-backward", action="store_true")
     ap.add_argument("--no-extra-prefill", action="store_true",

@@ -99,6 +99,10 @@ WORKLOADS = {
     # two-pass path takes, so the single-pass kernel runs
     "many_seqs": dict(kind="prefill", num_seqs=1024, seq_len=1024, H=32, Dk=128, Dv=128,
                       chunk=64, dtype="bf16", state_std=0.0, ckpt_interval=0),
+    # the single-pass kernel on 128 x 1024 tokens (4096 units), for profiler
+    # captures whose traffic is scaled to many_seqs
+    "many_seqs_small": dict(kind="prefill", num_seqs=128, seq_len=1024, H=32, Dk=128, Dv=128,
+                            chunk=64, dtype="bf16", state_std=0.0, ckpt_interval=0),
     # a smaller case of the prefill kernels, in the same launch configuration as
     # "prefill" (more than 74 (sequence, head) units), for profiler captures
     "prefill_small": dict(kind="prefill", num_seqs=2, seq_len=4096, H=40, Dk=128, Dv=128,
