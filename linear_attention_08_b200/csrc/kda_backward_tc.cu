@@ -117,10 +117,12 @@ struct BChainLayout {
 __global__ void __launch_bounds__(kThreads)
 bwd_dout_tiles_kernel(const float *__restrict__ dout, const int32_t *__restrict__ cu,
                       const int64_t *__restrict__ pref, int N, int H, uint8_t *__restrict__ tiles) {
-  // Two items per CTA: both items' rows are loaded before any store.
+  // Two items per CTA: both items' rows are loaded before any store.  Warp w
+  // takes rows w, w + 8, .., lane l columns 4l .. 4l + 3: every load is one
+  // whole 512-byte row of dO.
   const int64_t total = pref[N] * H;
-  const int tid = threadIdx.x, r = tid >> 2, c0 = (tid & 3) * 32;
-  float x[2][32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, c = 4 * lane;
+  float4 x[2][8];
   int64_t pp[2];
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
@@ -128,6 +130,7 @@ bwd_dout_tiles_kernel(const float *__restrict__ dout, const int32_t *__restrict_
     pp[it] = p;
     int L = 0;
     const float *src = dout;
+    size_t stride = 0;
     if (p < total) {
       int lo = 0, hi = N - 1;
       while (lo < hi) {
@@ -142,23 +145,24 @@ bwd_dout_tiles_kernel(const float *__restrict__ dout, const int32_t *__restrict_
       const int64_t t0 = (int64_t)cu[n] + kC * j;
       const int64_t T_n = (int64_t)cu[n + 1] - cu[n];
       L = (int)(T_n - kC * j < kC ? T_n - kC * j : kC);
-      src = dout + ((size_t)(t0 + r) * H + h) * kD + c0;
+      src = dout + ((size_t)t0 * H + h) * kD + c;
+      stride = (size_t)H * kD;
     }
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-      const float4 v4 = r < L ? *reinterpret_cast<const float4 *>(src + e) : make_float4(0.f, 0.f, 0.f, 0.f);
-      x[it][e] = v4.x; x[it][e + 1] = v4.y; x[it][e + 2] = v4.z; x[it][e + 3] = v4.w;
+    for (int i = 0; i < 8; ++i) {
+      const int r = warp + 8 * i;
+      x[it][i] = r < L ? *reinterpret_cast<const float4 *>(src + (size_t)r * stride)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 #pragma unroll
   for (int it = 0; it < 2; ++it) {
     if (pp[it] >= total) continue;
-    uint8_t *dst = tiles + (size_t)pp[it] * 16384;
+    uint8_t *dst = tiles + (size_t)pp[it] * 16384 + 2 * (c & 7);
 #pragma unroll
-    for (int e = 0; e < 32; e += 8)
-      *reinterpret_cast<uint4 *>(dst + tc::tile_offset(64, r, (c0 + e) >> 3)) =
-          make_uint4(tc::pack_bf16(x[it][e], x[it][e + 1]), tc::pack_bf16(x[it][e + 2], x[it][e + 3]),
-                     tc::pack_bf16(x[it][e + 4], x[it][e + 5]), tc::pack_bf16(x[it][e + 6], x[it][e + 7]));
+    for (int i = 0; i < 8; ++i)
+      *reinterpret_cast<uint2 *>(dst + tc::tile_offset(64, warp + 8 * i, c >> 3)) =
+          make_uint2(tc::pack_bf16(x[it][i].x, x[it][i].y), tc::pack_bf16(x[it][i].z, x[it][i].w));
   }
 }
 
