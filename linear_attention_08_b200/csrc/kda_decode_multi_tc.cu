@@ -439,6 +439,7 @@ decode_multi_tc_kernel(const __grid_constant__ MtcMaps maps, const float *__rest
     if (pend & 4u) wait_timed(bars + 2, m1ph, wait_ns);
     if (pend & 8u) wait_timed(bars + 3, m2ph, wait_ns);
   }
+  cp_async_wait_all();   // beta's copies of a unit the loop did not reach
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
