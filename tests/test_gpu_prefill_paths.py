@@ -194,3 +194,29 @@ def test_many_windows_run_the_single_pass():
     torch.cuda.synchronize()
     assert kda.kda_last_prefill_path() == 2
     check(d, out, fin, None, 0)
+
+
+def test_many_units_take_the_single_pass_from_the_pool():
+    """600 sequences x 4 heads = 2400 (sequence, head) units through the plain C
+    entry (workspace from the library's pool): the single-pass kernel runs and
+    nothing is taken from the pool; against the oracle."""
+    lengths = [8, 1, 17, 64] * 150
+    d = make_case(lengths, 4, 128, 128, torch.bfloat16, seed=42, state_std=0.05)
+    dd = to_device(d)
+    lib = kda.load()
+    T, H, _ = dd["q"].shape
+    N = len(lengths)
+    out = torch.empty(T, H, 128, dtype=torch.bfloat16, device="cuda")
+    fin = torch.empty(N, H, 128, 128, device="cuda")
+    shape = shape_of(dd)
+    assert kda.kda_prefill_path(shape) == 1
+    assert kda.kda_prefill_workspace_bytes(shape) == 0
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    st = lib.kda_prefill(P(dd["q"]), P(dd["k"]), P(dd["v"]), P(dd["g"]), P(dd["beta"]),
+                         P(dd["init_state"]), P(dd["cu_dev"]), P(out), P(fin), 0, None,
+                         ctypes.byref(shape), stream)
+    assert st == kda.KDA_OK
+    assert kda.kda_last_prefill_path() == 1
+    torch.cuda.synchronize()
+    check(d, out, fin, None, 0)
