@@ -404,11 +404,20 @@ struct BItemLayout {
   static constexpr uint32_t PKM = GA, PDG = RU;
   // PART 1 final partials: float [64][128] and [32][128]
   static constexpr uint32_t QDG = XA, KMC = YA;
+  // Store slabs, 4 KB per warp: PART 0 over dS_L (read only by products that
+  // are done when dv and the final epilogue write), PART 1 over T, (I+M)^-1,
+  // Y1 and dT (consumed; the next item's copies are issued after the final
+  // epilogue).
+  static constexpr uint32_t SLAB0 = DST, SLAB1 = TT;
   static_assert(GG + 17408 <= TT && MT + 4224 <= GG, "G");
   static_assert(YS + 2048 <= ZS && DST + 32768 <= YS, "scan scratch clears dS_L");
   static_assert(GB + 24576 <= RU + 32768 && RU + 32768 <= GST, "[R; U] stays clear of Gam");
   static_assert(CST + 6144 <= XM + 17408 && ZS + 6144 <= GG, "gate factors");
   static_assert(TOTAL + 1024 <= 232448, "shared memory");
+  static_assert(SLAB0 + 32768 <= YS && (SLAB0 >= PDG + 32768 || SLAB0 + 32768 <= PKM) &&
+                    (SLAB0 >= BT2 + 32768 || SLAB0 + 32768 <= BT2), "PART 0 slabs clear of the live partials and scan scratch");
+  static_assert(SLAB1 >= KMC + 32768 && SLAB1 >= GG + 17408 && SLAB1 + 32768 <= BETA,
+                "PART 1 slabs clear of the partials, G and beta");
 };
 
 // FP32 [64 tokens][128 channels] arrays read both with one token per lane
@@ -424,6 +433,34 @@ __device__ __forceinline__ float4 f4exp(float4 a) { return make_float4(__expf(a.
 __device__ __forceinline__ void st_chunk_s(uint8_t *dst, const float *x) {
   *reinterpret_cast<uint4 *>(dst) = make_uint4(tc::pack_bf16(x[0], x[1]), tc::pack_bf16(x[2], x[3]),
                                                tc::pack_bf16(x[4], x[5]), tc::pack_bf16(x[6], x[7]));
+}
+
+// Gradient rows leave through a warp's 4 KB slab of shared memory.  Lane l
+// holds token row l of a [32 rows][32 FP32 columns] block; it puts its eight
+// float4 pieces into row l of the slab, piece j at slot j ^ (l & 7), and the
+// block then leaves four whole 128-byte rows per warp instruction (lane l
+// takes row 4i + (l >> 3), piece l & 7) instead of 32 rows of 16 bytes each.
+// Both sides touch every bank once per quarter warp.
+__device__ __forceinline__ void slab_put(float4 *slab, int lane, int j, float4 v) {
+  slab[lane * 8 + (j ^ (lane & 7))] = v;
+}
+// Rows at or past `rows` are not written; ADD: FP32 reductions onto global memory.
+template <bool ADD>
+__device__ __forceinline__ void slab_rows_out(const float4 *slab, float *dst, size_t row_stride, int rows,
+                                              int lane) {
+  __syncwarp();
+  const int j = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int R = 4 * i + (lane >> 3);
+    const float4 v = slab[R * 8 + (j ^ (R & 7))];
+    float4 *d = reinterpret_cast<float4 *>(dst + (size_t)R * row_stride) + j;
+    if (R < rows) {
+      if (ADD) atomicAdd(d, v);
+      else *d = v;
+    }
+  }
+  __syncwarp();   // every lane has read the slab before it is filled again
 }
 
 struct BwdItemArgs {
@@ -904,16 +941,17 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     // (lanes 0..63) of this thread's token and channel half is loaded.
     if (!aborted && qd < 2) {
       const int r = 32 * qd + lane;
-      float *dst = a.dv + base_row + (size_t)r * row_stride + hw * 64;
+      float4 *slab = reinterpret_cast<float4 *>(sp + Lay::SLAB0) + warp * 256;
+      float *dst = a.dv + base_row + (size_t)(32 * qd) * row_stride + hw * 64;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {   // warp-wide TMEM loads; stores for tokens inside the chunk
         float acc[32];
         tc::tmem_ld32(tl + 0 + hw * 64 + 32 * half, acc);
         tc::tmem_wait_ld();
-        if (r < L)
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4 *>(dst + 32 * half + e) = make_float4(-acc[e], -acc[e + 1], -acc[e + 2], -acc[e + 3]);
+        for (int e = 0; e < 32; e += 4)
+          slab_put(slab, lane, e >> 2, make_float4(-acc[e], -acc[e + 1], -acc[e + 2], -acc[e + 3]));
+        slab_rows_out<false>(slab, dst + 32 * half, row_stride, L - 32 * qd, lane);
       }
       float d2[32];   // dT row r, columns 32 hw .. +31 (kept on and below the diagonal)
       tc::tmem_ld32(tl + 448 + hw * 32, d2);
@@ -983,55 +1021,60 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     float4 *pdk4 = reinterpret_cast<float4 *>(sp + Lay::PDG);   // k (dk+ - dk-)
     float4 *pkk4 = reinterpret_cast<float4 *>(sp + Lay::BT2);   // k (dk from Khat): the dGam_63 extra
     const float4 *g4 = reinterpret_cast<const float4 *>(s_gam);
+    float4 *slab = reinterpret_cast<float4 *>(sp + Lay::SLAB0) + warp * 256;
     if (!aborted && qd >= 2) {
       const int r = 32 * (qd - 2) + lane;
-      const bool in = r < L;
       float aq[64];
       tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(aq));
       tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(aq + 32));
       tc::tmem_wait_ld();
-      const size_t off = base_row + (size_t)r * row_stride + hw * 64;
+      float *dst = a.dq + base_row + (size_t)(32 * (qd - 2)) * row_stride + hw * 64;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float qv[8];
-        unpack8(raw[u], qv);
+      for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {   // channels hw*64 + 8u + 4hf .. +3
-          const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
-          const float4 dqa = f4mul(f4exp(g4[sw4(r, F)]), make_float4(aq[c], aq[c + 1], aq[c + 2], aq[c + 3]));
-          pdq4[sw4(r, F)] = f4mul(make_float4(qv[4 * hf], qv[4 * hf + 1], qv[4 * hf + 2], qv[4 * hf + 3]), dqa);
-          if (in) *reinterpret_cast<float4 *>(a.dq + off + c) = dqa;
+        for (int u = 4 * half; u < 4 * half + 4; ++u) {
+          float qv[8];
+          unpack8(raw[u], qv);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {   // channels hw*64 + 8u + 4hf .. +3
+            const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
+            const float4 dqa = f4mul(f4exp(g4[sw4(r, F)]), make_float4(aq[c], aq[c + 1], aq[c + 2], aq[c + 3]));
+            pdq4[sw4(r, F)] = f4mul(make_float4(qv[4 * hf], qv[4 * hf + 1], qv[4 * hf + 2], qv[4 * hf + 3]), dqa);
+            slab_put(slab, lane, (2 * u + hf) & 7, dqa);
+          }
         }
+        slab_rows_out<false>(slab, dst + 32 * half, row_stride, L - 32 * (qd - 2), lane);
       }
     } else if (!aborted) {
       const int r = 32 * qd + lane;
-      const bool in = r < L;
       float ak[64], ah[64];
       tc::tmem_ld32(tl + 128 + hw * 64, *reinterpret_cast<float(*)[32]>(ak));
       tc::tmem_ld32(tl + 128 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ak + 32));
       tc::tmem_ld32(tl + 256 + hw * 64, *reinterpret_cast<float(*)[32]>(ah));
       tc::tmem_ld32(tl + 256 + hw * 64 + 32, *reinterpret_cast<float(*)[32]>(ah + 32));
       tc::tmem_wait_ld();
-      const size_t off = base_row + (size_t)r * row_stride + hw * 64;
+      float *dst = a.dk + base_row + (size_t)(32 * qd) * row_stride + hw * 64;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        float kv[8];
-        unpack8(raw[u], kv);
+      for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
-          const float4 gam = g4[sw4(r, F)], g63 = g4[sw4(63, F)];
-          const float4 dkp = f4mul(f4exp(gam), make_float4(ak[c], ak[c + 1], ak[c + 2], ak[c + 3]));
-          const float4 dkm = f4mul(f4exp(make_float4(g63.x - gam.x, g63.y - gam.y, g63.z - gam.z, g63.w - gam.w)),
-                                   make_float4(ah[c], ah[c + 1], ah[c + 2], ah[c + 3]));
-          const float4 k4 = make_float4(kv[4 * hf], kv[4 * hf + 1], kv[4 * hf + 2], kv[4 * hf + 3]);
-          const float4 kp = f4mul(k4, dkp), km = f4mul(k4, dkm);
-          pdk4[sw4(r, F)] = make_float4(kp.x - km.x, kp.y - km.y, kp.z - km.z, kp.w - km.w);
-          pkk4[sw4(r, F)] = km;
-          if (in)
-            *reinterpret_cast<float4 *>(a.dk + off + c) =
-                make_float4(dkp.x + dkm.x, dkp.y + dkm.y, dkp.z + dkm.z, dkp.w + dkm.w);
+        for (int u = 4 * half; u < 4 * half + 4; ++u) {
+          float kv[8];
+          unpack8(raw[u], kv);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
+            const float4 gam = g4[sw4(r, F)], g63 = g4[sw4(63, F)];
+            const float4 dkp = f4mul(f4exp(gam), make_float4(ak[c], ak[c + 1], ak[c + 2], ak[c + 3]));
+            const float4 dkm = f4mul(f4exp(make_float4(g63.x - gam.x, g63.y - gam.y, g63.z - gam.z, g63.w - gam.w)),
+                                     make_float4(ah[c], ah[c + 1], ah[c + 2], ah[c + 3]));
+            const float4 k4 = make_float4(kv[4 * hf], kv[4 * hf + 1], kv[4 * hf + 2], kv[4 * hf + 3]);
+            const float4 kp = f4mul(k4, dkp), km = f4mul(k4, dkm);
+            pdk4[sw4(r, F)] = make_float4(kp.x - km.x, kp.y - km.y, kp.z - km.z, kp.w - km.w);
+            pkk4[sw4(r, F)] = km;
+            slab_put(slab, lane, (2 * u + hf) & 7, make_float4(dkp.x + dkm.x, dkp.y + dkm.y, dkp.z + dkm.z, dkp.w + dkm.w));
+          }
         }
+        slab_rows_out<false>(slab, dst + 32 * half, row_stride, L - 32 * qd, lane);
       }
     }
     // Gam leaves its rows for the next item's g; the scan keeps exp(Gam_63).
@@ -1233,9 +1276,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       unpack8(*reinterpret_cast<const uint4 *>(sp + tile + tc::tile_offset(rows, row, chunk)), x);
     };
     float *dqp = a.dq, *dkp_ = a.dk;
+    float4 *slab = reinterpret_cast<float4 *>(sp + Lay::SLAB1) + warp * 256;
     if (!aborted && qd >= 2) {
       const int r = 32 * (qd - 2) + lane;
-      const bool in = r < L;
       const int ref = r < 32 ? 15 : 47;
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
@@ -1243,7 +1286,6 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         float xq[32];
         tc::tmem_ld32(tl + 0 + c0, xq);
         tc::tmem_wait_ld();
-        float4 *dst = reinterpret_cast<float4 *>(dqp + base_row + (size_t)r * row_stride + c0);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {   // 8 channels: one tile chunk
           float ga[8];
@@ -1255,13 +1297,15 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
             const float4 xqv = make_float4(xq[c], xq[c + 1], xq[c + 2], xq[c + 3]);
             const float4 add = f4mul(f4exp(make_float4(gam.x - gref.x, gam.y - gref.y, gam.z - gref.z, gam.w - gref.w)), xqv);
             qdg4[sw4(r, F)] = f4mul(make_float4(ga[4 * hf], ga[4 * hf + 1], ga[4 * hf + 2], ga[4 * hf + 3]), xqv);
-            if (in) atomicAdd(dst + 2 * u + hf, add);   // onto the state part's dq, no read back
+            slab_put(slab, lane, 2 * u + hf, add);
           }
         }
+        // onto the state part's dq, no read back
+        slab_rows_out<true>(slab, dqp + base_row + (size_t)(32 * (qd - 2)) * row_stride + c0, row_stride,
+                            L - 32 * (qd - 2), lane);
       }
     } else if (!aborted) {
       const int t = 32 * qd + lane;
-      const bool in = t < L;
       const int ref = t < 32 ? 15 : 47;
       const int gbrow = t < 32 ? t : 32 + t;
 #pragma unroll 1
@@ -1272,7 +1316,6 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         tc::tmem_ld32(tl + 128 + c0, yo);
         tc::tmem_ld32(tl + 256 + c0, yc);   // cross rows (first-half keys, second-half reference)
         tc::tmem_wait_ld();
-        float4 *dst = reinterpret_cast<float4 *>(dkp_ + base_row + (size_t)t * row_stride + c0);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           float ga[8], gb[8], gc[8];
@@ -1299,10 +1342,11 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
               pb = make_float4(pb.x + pc.x, pb.y + pc.y, pb.z + pc.z, pb.w + pc.w);
             }
             kdg4[sw4(t, F)] = make_float4(pa.x - pb.x, pa.y - pb.y, pa.z - pb.z, pa.w - pb.w);
-            if (in)
-              atomicAdd(dst + 2 * u + hf, make_float4(dkp.x + dkm.x, dkp.y + dkm.y, dkp.z + dkm.z, dkp.w + dkm.w));
+            slab_put(slab, lane, 2 * u + hf, make_float4(dkp.x + dkm.x, dkp.y + dkm.y, dkp.z + dkm.z, dkp.w + dkm.w));
           }
         }
+        slab_rows_out<true>(slab, dkp_ + base_row + (size_t)(32 * qd) * row_stride + c0, row_stride, L - 32 * qd,
+                            lane);
       }
     }
     tc::fence_smem_to_async();
