@@ -398,8 +398,9 @@ struct BItemLayout {
   static constexpr uint32_t TBAR = BAR + 8;               // inputs landed
   static constexpr uint32_t CBAR = BAR + 16;              // [-dU; dO] landed (PART 0); dT, placed dP (PART 1)
   static constexpr uint32_t SBAR = BAR + 24;              // S0 (BF16 tile) landed (PART 0)
-  static constexpr uint32_t TMEM_SLOT = BAR + 32;
-  static constexpr uint32_t TOTAL = BAR + 40;
+  static constexpr uint32_t RBAR = BAR + 32;              // raw q and k tiles landed (PART 0)
+  static constexpr uint32_t TMEM_SLOT = BAR + 40;
+  static constexpr uint32_t TOTAL = BAR + 48;
   // PART 0 final partials (after the last MMAs): float [64][128] each
   static constexpr uint32_t PKM = GA, PDG = RU;
   // PART 1 final partials: float [64][128] and [32][128]
@@ -409,6 +410,9 @@ struct BItemLayout {
   // Y1 and dT (consumed; the next item's copies are issued after the final
   // epilogue).
   static constexpr uint32_t SLAB0 = DST, SLAB1 = TT;
+  // PART 0: the raw q and k tiles [64 tok][128 ch] for the final epilogue, in
+  // space only the Gram part uses (its gate factors, G, and its Ai, Y1, dT tiles).
+  static constexpr uint32_t RAWQ = 168960, RAWK = AIT;
   static_assert(GG + 17408 <= TT && MT + 4224 <= GG, "G");
   static_assert(YS + 2048 <= ZS && DST + 32768 <= YS, "scan scratch clears dS_L");
   static_assert(GB + 24576 <= RU + 32768 && RU + 32768 <= GST, "[R; U] stays clear of Gam");
@@ -416,6 +420,8 @@ struct BItemLayout {
   static_assert(TOTAL + 1024 <= 232448, "shared memory");
   static_assert(SLAB0 + 32768 <= YS && (SLAB0 >= PDG + 32768 || SLAB0 + 32768 <= PKM) &&
                     (SLAB0 >= BT2 + 32768 || SLAB0 + 32768 <= BT2), "PART 0 slabs clear of the live partials and scan scratch");
+  static_assert(RAWQ >= YS + 2048 && RAWQ + 16384 <= TT && RAWK + 16384 <= BETA && RAWQ % 1024 == 0 &&
+                    RAWK % 1024 == 0, "PART 0 raw q, k tiles: clear of the scan scratch, T and beta; swizzle alignment");
   static_assert(SLAB1 >= KMC + 32768 && SLAB1 >= GG + 17408 && SLAB1 + 32768 <= BETA,
                 "PART 1 slabs clear of the partials, G and beta");
 };
@@ -477,7 +483,6 @@ struct BwdItemArgs {
                                //   dT as the BF16 [64][64] operand tile, rows 64..127 of the
                                //   [dG; dP] tile (dP placed, BF16, 2 x 8 KB), dP^T FP32 [64][64]
   const uint8_t *tt;           // T and (I + M)^-1 per packet from the forward: BF16 [64][64] tiles
-  const void *q, *k;           // raw BF16 inputs (re-read by the final epilogues)
   float *dq, *dk, *dv, *dg, *dbeta;
   int N, H;
   int32_t *dev_status;
@@ -510,12 +515,14 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   uint64_t *tbar = reinterpret_cast<uint64_t *>(sp + Lay::TBAR);
   uint64_t *cbar = reinterpret_cast<uint64_t *>(sp + Lay::CBAR);
   uint64_t *s0bar = reinterpret_cast<uint64_t *>(sp + Lay::SBAR);
+  uint64_t *rbar = reinterpret_cast<uint64_t *>(sp + Lay::RBAR);
 
   if (tid == 0) {
     mbar_init(bar, 1);
     mbar_init(tbar, 1);
     mbar_init(cbar, 1);
     mbar_init(s0bar, 1);
+    mbar_init(rbar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) tc::tmem_alloc(sb + Lay::TMEM_SLOT, 512);
@@ -524,8 +531,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
   tc::fence_after_sync();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(sp + Lay::TMEM_SLOT);
   const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
-  uint32_t phase = 0, tphase = 0, cphase = 0, s0phase = 0;
+  uint32_t phase = 0, tphase = 0, cphase = 0, s0phase = 0, rphase = 0;
   bool s0pend = false;   // an S0 copy is in flight (PART 0)
+  bool rpend = false;    // raw q, k copies are in flight (PART 0)
   bool aborted = false;
   const int N = a.N;
   const int64_t total = a.pref[N] * H;
@@ -601,7 +609,15 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     if (tid == 32) {
       mbar_expect_tx(sb + Lay::TBAR, kKqvBytes);
       issue_kqv(h, t0);
+      // The raw q and k tiles, read only by the final epilogue.
+      mbar_expect_tx(sb + Lay::RBAR, 32768);
+#pragma unroll
+      for (int b = 0; b < 2; ++b) {
+        tma_load_3d(sb + Lay::RAWQ + b * 8192, &maps.q, 64 * b, h, (int)t0, sb + Lay::RBAR);
+        tma_load_3d(sb + Lay::RAWK + b * 8192, &maps.k, 64 * b, h, (int)t0, sb + Lay::RBAR);
+      }
     }
+    rpend = true;
   }
   pre = false;
   const bool has_next = p + gridDim.x < total;
@@ -936,9 +952,8 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
                      tc::desc_kmajor(sb + Lay::S0T, 128, s2), id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
-    // While the product runs: dv (= dR) and dT leave for global memory (their
-    // TMEM columns are not the product's), and the raw q (lanes 64..127) or k
-    // (lanes 0..63) of this thread's token and channel half is loaded.
+    // While the product runs: dv (= dR), dT and dP leave for global memory
+    // (their TMEM columns are not the product's).
     if (!aborted && qd < 2) {
       const int r = 32 * qd + lane;
       float4 *slab = reinterpret_cast<float4 *>(sp + Lay::SLAB0) + warp * 256;
@@ -1002,18 +1017,17 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
         dpt[i * 64 + ((((r >> 2) ^ (i & 15))) << 2) + (r & 3)] = d2[e];
       }
     }
-    uint4 raw[8];
-    {
-      const int rr = qd >= 2 ? 32 * (qd - 2) + lane : 32 * qd + lane;
-      const __nv_bfloat16 *src = reinterpret_cast<const __nv_bfloat16 *>(qd >= 2 ? a.q : a.k) +
-                                 base_row + (size_t)rr * row_stride + hw * 64;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        raw[u] = rr < L ? *reinterpret_cast<const uint4 *>(src + 8 * u) : make_uint4(0, 0, 0, 0);
-    }
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
     phase ^= 1;
     tc::fence_after_sync();
+    if (!aborted) {
+      if (__syncthreads_or(!wait_timed(rbar, rphase, a.wait_ns))) {
+        aborted = true;
+      } else {
+        rpend = false;
+        rphase ^= 1;
+      }
+    }
     // ---- final epilogue: dq, dk and dGam from Qtilde, Ktilde, Khat and d ----
     // Token r's dQtilde sits in TMEM lane 64 + r, its dKtilde and dKhat in lane
     // r: the two halves of the CTA work at once, each on its own dGam part.
@@ -1033,8 +1047,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       for (int half = 0; half < 2; ++half) {
 #pragma unroll
         for (int u = 4 * half; u < 4 * half + 4; ++u) {
-          float qv[8];
-          unpack8(raw[u], qv);
+          float qv[8];   // raw q of token r (zero past the chunk's end)
+          unpack8(r < L ? *reinterpret_cast<const uint4 *>(sp + Lay::RAWQ + tc::tile_offset(64, r, hw * 8 + u))
+                        : make_uint4(0, 0, 0, 0), qv);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {   // channels hw*64 + 8u + 4hf .. +3
             const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
@@ -1058,8 +1073,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       for (int half = 0; half < 2; ++half) {
 #pragma unroll
         for (int u = 4 * half; u < 4 * half + 4; ++u) {
-          float kv[8];
-          unpack8(raw[u], kv);
+          float kv[8];   // raw k of token r (zero past the chunk's end)
+          unpack8(r < L ? *reinterpret_cast<const uint4 *>(sp + Lay::RAWK + tc::tile_offset(64, r, hw * 8 + u))
+                        : make_uint4(0, 0, 0, 0), kv);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
             const int F = hw * 16 + 2 * u + hf, c = 8 * u + 4 * hf;
@@ -1390,6 +1406,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     wait_timed(tbar, tphase, a.wait_ns);
     wait_timed(cbar, cphase, a.wait_ns);
     if (PART == 0 && s0pend) wait_timed(s0bar, s0phase, a.wait_ns);
+    if (PART == 0 && rpend) wait_timed(rbar, rphase, a.wait_ns);
   }
   tc::fence_before_sync();
   __syncthreads();
@@ -1533,7 +1550,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
 
   BwdItemArgs a;
   a.beta = beta; a.s0_init = init ? s0i : nullptr; a.s0_ck = ck; a.cu = cu; a.pref = pref; a.prefck = prefck;
-  a.dsl = dsl; a.ndu = ndu; a.dot = dot; a.dtp = dtp; a.tt = tt; a.q = q; a.k = k;
+  a.dsl = dsl; a.ndu = ndu; a.dot = dot; a.dtp = dtp; a.tt = tt;
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
   a.N = N; a.H = H; a.dev_status = dev_status; a.wait_ns = wait_ns;
   const size_t smem_i = BItemLayout::TOTAL + 1024;
