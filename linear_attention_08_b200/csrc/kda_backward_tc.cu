@@ -1108,10 +1108,12 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       const int ch = tid & 127, hf = tid >> 7;
       const float *pdq = reinterpret_cast<const float *>(pdq4), *pdk = reinterpret_cast<const float *>(pdk4);
       const float *pkk = reinterpret_cast<const float *>(pkk4);
-      float part = 0.f, extra = 0.f;
-#pragma unroll 8
-      for (int r = 32 * hf; r < 32 * hf + 32; ++r) {
-        part += pdq[sw(r, ch)] + pdk[sw(r, ch)];
+      float dgam[32], part = 0.f, extra = 0.f;   // dGam of rows 32 hf + i, kept for the suffix sums
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * hf + i;
+        dgam[i] = pdq[sw(r, ch)] + pdk[sw(r, ch)];
+        part += dgam[i];
         extra += pkk[sw(r, ch)];
       }
       if (hf == 0) extra = fmaf(e63, s_dd[ch], extra);
@@ -1119,9 +1121,10 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       sred[256 + hf * 128 + ch] = extra;
       __syncthreads();
       float suffix = sred[256 + ch] + sred[384 + ch] + (hf == 0 ? sred[128 + ch] : 0.f);
-#pragma unroll 8
-      for (int r = 32 * hf + 31; r >= 32 * hf; --r) {
-        suffix += pdq[sw(r, ch)] + pdk[sw(r, ch)];
+#pragma unroll
+      for (int i = 31; i >= 0; --i) {
+        const int r = 32 * hf + i;
+        suffix += dgam[i];
         if (r < L) a.dg[base_row + (size_t)r * row_stride + ch] = suffix;
       }
     }
@@ -1378,16 +1381,21 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       const int ch = tid & 127, hf = tid >> 7;
       const float *qdg = reinterpret_cast<const float *>(qdg4), *kdg = reinterpret_cast<const float *>(kdg4);
       float *sred = s_Y;
-      float part = 0.f;
-#pragma unroll 8
-      for (int r = 32 * hf; r < 32 * hf + 32; ++r) part += qdg[sw(r, ch)] + kdg[sw(r, ch)];
+      float dgam[32], part = 0.f;   // dGam of rows 32 hf + i, kept for the suffix sums
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int r = 32 * hf + i;
+        dgam[i] = qdg[sw(r, ch)] + kdg[sw(r, ch)];
+        part += dgam[i];
+      }
       sred[hf * 128 + ch] = part;
       __syncthreads();
       float *dgp = a.dg;
       float suffix = hf == 0 ? sred[128 + ch] : 0.f;
-#pragma unroll 8
-      for (int r = 32 * hf + 31; r >= 32 * hf; --r) {
-        suffix += qdg[sw(r, ch)] + kdg[sw(r, ch)];
+#pragma unroll
+      for (int i = 31; i >= 0; --i) {
+        const int r = 32 * hf + i;
+        suffix += dgam[i];
         if (r < L) atomicAdd(dgp + base_row + (size_t)r * row_stride + ch, suffix);
       }
     }
