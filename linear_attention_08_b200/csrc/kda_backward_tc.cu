@@ -1257,7 +1257,7 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     tc::fence_before_sync();
     __syncthreads();
     // ---- [X; Xq] = [dG; dP] Gram B (columns 0..127), Y = [dG^T | dP^T] Gram A (128..255),
-    //      and rows 64..127 of YA again (256..383) so that the cross rows land in lanes 0..31 ----
+    //      whose lanes 64..95 hold the cross rows (first-half keys, second-half reference) ----
     if (!aborted && tid == 0) {
       tc::fence_after_sync();
       constexpr uint32_t id = tc::idesc_bf16(128, 128, 0, 1);
@@ -1269,10 +1269,6 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
       for (int s2 = 0; s2 < 8; ++s2)
         tc::mma_bf16(tmem + 128, tc::desc_kmajor(sb + Lay::YA, 128, s2),
                      tc::desc_mnmajor(sb + Lay::GA, 128, s2), id, s2 > 0);
-#pragma unroll
-      for (int s2 = 0; s2 < 8; ++s2)   // rows 64..127 of YA as rows 0..63 (the rest read past them)
-        tc::mma_bf16(tmem + 256, tc::desc_kmajor(sb + Lay::YA + 8192, 128, s2),
-                     tc::desc_mnmajor(sb + Lay::GA, 128, s2), id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
     if (!aborted && __syncthreads_or(!wait_timed(bar, phase, a.wait_ns))) aborted = true;
@@ -1283,8 +1279,11 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
     // products used (Gram A rows for the sides where Gam enters with a plus
     // sign, Gram B rows for the others), so that the pair's terms, which the
     // reverse cumulative sum below sets against each other, cancel to FP32
-    // accumulation precision.  Lanes 64..127 (Xq) and lanes 0..63 (X, Y and the
-    // cross rows) work at once, each half on its own dGam part.  The parts of
+    // accumulation precision.  Lanes 64..127 (Xq, and in lanes 64..95 the
+    // cross rows of Y) and lanes 0..63 (X, Y) work at once, each half on its
+    // own dGam part; the cross rows' terms of dk and dGam (keys 0..31) fall to
+    // the warps of lanes 64..95, which have only dq otherwise, so that the
+    // exponentials split evenly over the four lane quarters.  The parts of
     // dq, dk and dg go onto what the state part wrote as reductions in global
     // memory (no load, so no wait for the earlier values).
     float4 *qdg4 = reinterpret_cast<float4 *>(sp + Lay::QDG);   // dGam from the q side
@@ -1302,26 +1301,43 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         const int c0 = hw * 64 + 32 * half;
-        float xq[32];
+        const bool cross = qd == 2;   // key r < 32 also has a cross row (TMEM lane 64 + r of Y)
+        float xq[32], yc[32];
+        float4 km[8];
         tc::tmem_ld32(tl + 0 + c0, xq);
+        if (cross) tc::tmem_ld32(tl + 128 + c0, yc);
         tc::tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 4; ++u) {   // 8 channels: one tile chunk
-          float ga[8];
+          float ga[8], gc[8];
           tile8(Lay::GA, 128, 64 + r, (c0 >> 3) + u, ga);
+          if (cross) tile8(Lay::GB, 96, 32 + r, (c0 >> 3) + u, gc);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
             const int F = (c0 >> 2) + 2 * u + hf, c = 8 * u + 4 * hf;
             const float4 gam = g4[sw4(r, F)], gref = g4[sw4(ref, F)];
             const float4 xqv = make_float4(xq[c], xq[c + 1], xq[c + 2], xq[c + 3]);
             const float4 add = f4mul(f4exp(make_float4(gam.x - gref.x, gam.y - gref.y, gam.z - gref.z, gam.w - gref.w)), xqv);
-            qdg4[sw4(r, F)] = f4mul(make_float4(ga[4 * hf], ga[4 * hf + 1], ga[4 * hf + 2], ga[4 * hf + 3]), xqv);
+            float4 qa = f4mul(make_float4(ga[4 * hf], ga[4 * hf + 1], ga[4 * hf + 2], ga[4 * hf + 3]), xqv);
+            if (cross) {   // key r against the second half's reference: its dk term and -(its dGam side)
+              const float4 ycv = make_float4(yc[c], yc[c + 1], yc[c + 2], yc[c + 3]);
+              const float4 g47 = g4[sw4(47, F)];
+              km[2 * u + hf] = f4mul(f4exp(make_float4(g47.x - gam.x, g47.y - gam.y, g47.z - gam.z, g47.w - gam.w)), ycv);
+              const float4 pc = f4mul(make_float4(gc[4 * hf], gc[4 * hf + 1], gc[4 * hf + 2], gc[4 * hf + 3]), ycv);
+              qa = make_float4(qa.x - pc.x, qa.y - pc.y, qa.z - pc.z, qa.w - pc.w);
+            }
+            qdg4[sw4(r, F)] = qa;
             slab_put(slab, lane, 2 * u + hf, add);
           }
         }
         // onto the state part's dq, no read back
         slab_rows_out<true>(slab, dqp + base_row + (size_t)(32 * (qd - 2)) * row_stride + c0, row_stride,
                             L - 32 * (qd - 2), lane);
+        if (cross) {   // the cross rows' part of dk for keys 0..31
+#pragma unroll
+          for (int j = 0; j < 8; ++j) slab_put(slab, lane, j, km[j]);
+          slab_rows_out<true>(slab, dkp_ + base_row + c0, row_stride, L, lane);
+        }
       }
     } else if (!aborted) {
       const int t = 32 * qd + lane;
@@ -1330,17 +1346,15 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         const int c0 = hw * 64 + 32 * half;
-        float xk[32], yo[32], yc[32];
+        float xk[32], yo[32];
         tc::tmem_ld32(tl + 0 + c0, xk);
         tc::tmem_ld32(tl + 128 + c0, yo);
-        tc::tmem_ld32(tl + 256 + c0, yc);   // cross rows (first-half keys, second-half reference)
         tc::tmem_wait_ld();
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          float ga[8], gb[8], gc[8];
+          float ga[8], gb[8];
           tile8(Lay::GA, 128, t, (c0 >> 3) + u, ga);
           tile8(Lay::GB, 96, gbrow, (c0 >> 3) + u, gb);
-          if (t < 32) tile8(Lay::GB, 96, 32 + t, (c0 >> 3) + u, gc);
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
             const int F = (c0 >> 2) + 2 * u + hf, c = 8 * u + 4 * hf;
@@ -1349,17 +1363,9 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
             const float4 xkv = make_float4(xk[c], xk[c + 1], xk[c + 2], xk[c + 3]);
             const float4 yov = make_float4(yo[c], yo[c + 1], yo[c + 2], yo[c + 3]);
             const float4 dkp = f4mul(f4exp(dlt), xkv);
-            float4 dkm = f4mul(f4exp(make_float4(-dlt.x, -dlt.y, -dlt.z, -dlt.w)), yov);
+            const float4 dkm = f4mul(f4exp(make_float4(-dlt.x, -dlt.y, -dlt.z, -dlt.w)), yov);
             const float4 pa = f4mul(make_float4(ga[4 * hf], ga[4 * hf + 1], ga[4 * hf + 2], ga[4 * hf + 3]), xkv);
-            float4 pb = f4mul(make_float4(gb[4 * hf], gb[4 * hf + 1], gb[4 * hf + 2], gb[4 * hf + 3]), yov);
-            if (t < 32) {
-              const float4 ycv = make_float4(yc[c], yc[c + 1], yc[c + 2], yc[c + 3]);
-              const float4 g47 = g4[sw4(47, F)];
-              const float4 km = f4mul(f4exp(make_float4(g47.x - gam.x, g47.y - gam.y, g47.z - gam.z, g47.w - gam.w)), ycv);
-              dkm = make_float4(dkm.x + km.x, dkm.y + km.y, dkm.z + km.z, dkm.w + km.w);
-              const float4 pc = f4mul(make_float4(gc[4 * hf], gc[4 * hf + 1], gc[4 * hf + 2], gc[4 * hf + 3]), ycv);
-              pb = make_float4(pb.x + pc.x, pb.y + pc.y, pb.z + pc.z, pb.w + pc.w);
-            }
+            const float4 pb = f4mul(make_float4(gb[4 * hf], gb[4 * hf + 1], gb[4 * hf + 2], gb[4 * hf + 3]), yov);
             kdg4[sw4(t, F)] = make_float4(pa.x - pb.x, pa.y - pb.y, pa.z - pb.z, pa.w - pb.w);
             slab_put(slab, lane, 2 * u + hf, make_float4(dkp.x + dkm.x, dkp.y + dkm.y, dkp.z + dkm.z, dkp.w + dkm.w));
           }
