@@ -85,7 +85,8 @@ struct IntraLayout {
   static constexpr uint32_t VBAR = BAR + 16;                      // v landed
   static constexpr uint32_t GBAR = BAR + 24;                      // g landed
   static constexpr uint32_t TMEM_SLOT = BAR + 32;
-  static constexpr uint32_t TOTAL = BAR + 40;
+  static constexpr uint32_t NEXT = BAR + 40;                      // int64 [2][2]: the next item's t0, (L, h)
+  static constexpr uint32_t TOTAL = NEXT + 32;
   static_assert(MT + 32 * 33 * 4 <= VT, "solve scratch overlaps the V tile");
   static_assert(VT >= GA && VT + 16384 <= GA + 32768, "the V tile must lie in the consumed Gram A tile");
   static_assert(MT + 32 * 33 * 4 <= 65536 && STG_G + 32768 <= GA, "g staging and the solve scratch");
@@ -242,17 +243,26 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
   uint32_t phase = 0, tphase = 0, vphase = 0, gphase = 0;
   bool aborted = false;
   int p = blockIdx.x;
+  // The next item's place is found by one thread while the Gram product runs
+  // (its search and divisions are off every other thread's path) and handed
+  // over through shared memory, in two slots used in turn.
+  int64_t *s_next = reinterpret_cast<int64_t *>(sp + Lay::NEXT);
+  int slot = 0;
+  int64_t cur_t0;
+  int cur_L, cur_h;
   {
     const Item it = decode_item(p, s_pref, s_cu, N, H, jw0);
     intra_issue_g(sb, maps, beta, it.t0, it.L, H, it.h, tid);
     intra_issue_qk(sb, maps, it.t0, it.h, tid);
+    cur_t0 = it.t0;
+    cur_L = it.L;
+    cur_h = it.h;
   }
 
   for (; p < total; p += gridDim.x) {
-    const Item it = decode_item(p, s_pref, s_cu, N, H, jw0);
     const bool more = p + (int)gridDim.x < total;
-    const Item nx = decode_item(more ? p + (int)gridDim.x : p, s_pref, s_cu, N, H, jw0);
-    const int L = it.L, h = it.h;
+    const int L = cur_L, h = cur_h;
+    const int64_t t0 = cur_t0;
     uint8_t *pk = ws + (size_t)p * Packet::BYTES;
 
     cp_async_wait_all();
@@ -408,6 +418,11 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
                      id, s2 > 0);
       tc::mma_commit(sb + Lay::BAR);
     }
+    if (tid == 224 && more) {
+      const Item nx = decode_item(p + (int)gridDim.x, s_pref, s_cu, N, H, jw0);
+      s_next[2 * (slot ^ 1)] = nx.t0;
+      s_next[2 * (slot ^ 1) + 1] = ((int64_t)nx.h << 32) | (uint32_t)nx.L;
+    }
     if (__syncthreads_or(!wait_timed(bar, phase, wait_ns))) { aborted = true; break; }
     phase ^= 1;
     tc::fence_after_sync();
@@ -415,8 +430,8 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
     if (tid == 32) {
       const uint32_t vb = sb + Lay::VBAR;
       mbar_expect_tx(vb, 64 * 256);
-      tma_load_3d(sb + Lay::VT, &maps.v, 0, h, (int)it.t0, vb);
-      tma_load_3d(sb + Lay::VT + 8192, &maps.v, 64, h, (int)it.t0, vb);
+      tma_load_3d(sb + Lay::VT, &maps.v, 0, h, (int)t0, vb);
+      tma_load_3d(sb + Lay::VT + 8192, &maps.v, 64, h, (int)t0, vb);
     }
 
     // Gram rows: lane m = row m.  k rows -> FP32 M (scaled by beta_r, strictly
@@ -555,7 +570,9 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
     if (__syncthreads_or(!wait_timed(vbar, vphase, wait_ns))) { aborted = true; break; }
     vphase ^= 1;
     // The solve scratch and beta are consumed: the next item's g and beta may land.
-    if (more) intra_issue_g(sb, maps, beta, nx.t0, nx.L, H, nx.h, tid);
+    const int64_t nx_t0 = s_next[2 * (slot ^ 1)], nx_lh = s_next[2 * (slot ^ 1) + 1];
+    const int nx_L = (int)(uint32_t)nx_lh, nx_h = (int)(nx_lh >> 32);
+    if (more) intra_issue_g(sb, maps, beta, nx_t0, nx_L, H, nx_h, tid);
 
     // ---------------- W = T Ktilde (columns 0..127), U = T V (128..255) ----------------
     // Rows 64..127 of the A tile repeat T: TMEM lanes 64..127 get a copy of the product.
@@ -576,7 +593,7 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
     phase ^= 1;
     tc::fence_after_sync();
     // The V tile is consumed: the next item's q and k may land in the Gram A tile.
-    if (more) intra_issue_qk(sb, maps, nx.t0, nx.h, tid);
+    if (more) intra_issue_qk(sb, maps, nx_t0, nx_h, tid);
     {   // Each warp takes one 64-column quarter of [W | U] (W -> KT tile, U -> TP tile)
         // for 32 tokens: quadrants 0, 1 read lanes 0..63, quadrants 2, 3 the copy.
       const int r = 32 * (qd & 1) + lane, quarter = 2 * (qd >> 1) + hw;
@@ -597,6 +614,10 @@ intra_kernel(const __grid_constant__ TmaMaps maps, const float *__restrict__ bet
       bulk_store(pk + Packet::U, sb + Lay::TP, 16384);
       bulk_commit();
     }
+    cur_t0 = nx_t0;
+    cur_L = nx_L;
+    cur_h = nx_h;
+    slot ^= 1;
   }
   if (tid == 0) bulk_wait_all();
 
