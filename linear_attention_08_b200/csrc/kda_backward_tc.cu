@@ -77,6 +77,14 @@ struct Pk {
   static constexpr uint32_t BYTES = 74240;
 };
 
+// Where packet p sits: written by the dO tile conversion, which locates every
+// packet anyway, and read by the per-chunk kernels with one independent load
+// instead of a search and divisions on each item's path.
+struct ItemRec {
+  int64_t t0, j;   // first token, chunk index in the sequence
+  int32_t n, h, L, pad;
+};
+
 // Chunks of sequence n.
 __device__ __forceinline__ int64_t seq_chunks(const int32_t *cu, int n) {
   return ((int64_t)cu[n + 1] - cu[n] + kC - 1) / kC;
@@ -116,7 +124,8 @@ struct BChainLayout {
 // (rows past the sequence's end zero), for every packet: two packets per CTA.
 __global__ void __launch_bounds__(kThreads)
 bwd_dout_tiles_kernel(const float *__restrict__ dout, const int32_t *__restrict__ cu,
-                      const int64_t *__restrict__ pref, int N, int H, uint8_t *__restrict__ tiles) {
+                      const int64_t *__restrict__ pref, int N, int H, uint8_t *__restrict__ tiles,
+                      ItemRec *__restrict__ items) {
   // Two items per CTA: both items' rows are loaded before any store.  Warp w
   // takes rows w, w + 8, .., lane l columns 4l .. 4l + 3: every load is one
   // whole 512-byte row of dO.
@@ -145,6 +154,11 @@ bwd_dout_tiles_kernel(const float *__restrict__ dout, const int32_t *__restrict_
       const int64_t t0 = (int64_t)cu[n] + kC * j;
       const int64_t T_n = (int64_t)cu[n + 1] - cu[n];
       L = (int)(T_n - kC * j < kC ? T_n - kC * j : kC);
+      if (tid == 0) {
+        ItemRec rec;
+        rec.t0 = t0; rec.j = j; rec.n = n; rec.h = h; rec.L = L; rec.pad = 0;
+        items[p] = rec;
+      }
       src = dout + ((size_t)t0 * H + h) * kD + c;
       stride = (size_t)H * kD;
     }
@@ -483,6 +497,7 @@ struct BwdItemArgs {
                                //   dT as the BF16 [64][64] operand tile, rows 64..127 of the
                                //   [dG; dP] tile (dP placed, BF16, 2 x 8 KB), dP^T FP32 [64][64]
   const uint8_t *tt;           // T and (I + M)^-1 per packet from the forward: BF16 [64][64] tiles
+  const ItemRec *items;        // where each packet sits (from the dO tile conversion)
   float *dq, *dk, *dv, *dg, *dbeta;
   int N, H;
   int32_t *dev_status;
@@ -540,19 +555,12 @@ bwd_item_kernel(const __grid_constant__ TmaMaps maps, const BwdItemArgs a) {
 
   // Item pp (sequence, head, chunk) in packet order: pp = H pref[n] + h c_n + j.
   auto locate = [&](int64_t pp, int &n_, int &h_, int64_t &j_, int64_t &t0_, int &L_) {
-    int lo = 0, hi = N - 1;
-    while (lo < hi) {   // last sequence whose first packet is at or before pp
-      const int mid = (lo + hi + 1) >> 1;
-      if (a.pref[mid] * H <= pp) lo = mid; else hi = mid - 1;
-    }
-    n_ = lo;
-    const int64_t nch = a.pref[lo + 1] - a.pref[lo];
-    const int64_t rem = pp - a.pref[lo] * H;
-    h_ = (int)(rem / nch);
-    j_ = rem - (int64_t)h_ * nch;
-    t0_ = (int64_t)a.cu[lo] + kC * j_;
-    const int64_t T_n = (int64_t)a.cu[lo + 1] - a.cu[lo];
-    L_ = (int)(T_n - kC * j_ < kC ? T_n - kC * j_ : kC);
+    const ItemRec rec = a.items[pp];
+    n_ = rec.n;
+    h_ = rec.h;
+    j_ = rec.j;
+    t0_ = rec.t0;
+    L_ = rec.L;
   };
   // Inputs: g into its staging rows and beta (both parts), q, k into the Gram A
   // tile, v (the state part); with g, the item's T (and for the Gram part
@@ -1479,7 +1487,7 @@ bwd_init_tiles_kernel(const float *__restrict__ init, uint8_t *__restrict__ tile
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 struct BwdWs {
-  size_t pk, ck, s0i, tt, dsl, ndu, dot, dtp, oscr, pref, prefck, total;
+  size_t pk, ck, s0i, tt, dsl, ndu, dot, dtp, oscr, pref, prefck, items, total;
 };
 
 BwdWs bwd_ws_layout(int N, int H, int64_t T) {
@@ -1497,6 +1505,7 @@ BwdWs bwd_ws_layout(int N, int H, int64_t T) {
   w.oscr = off;   off += align256((size_t)T * H * kD * 2);
   w.pref = off;   off += align256((size_t)(N + 1) * 8);
   w.prefck = off; off += align256((size_t)(N + 1) * 8);
+  w.items = off;  off += align256(P * sizeof(ItemRec));
   w.total = off + 256;
   return w;
 }
@@ -1529,6 +1538,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   void *oscr = base + w.oscr;
   int64_t *pref = reinterpret_cast<int64_t *>(base + w.pref);
   int64_t *prefck = reinterpret_cast<int64_t *>(base + w.prefck);
+  ItemRec *items = reinterpret_cast<ItemRec *>(base + w.items);
   const uint64_t wait_ns = 2000000000ull;
 
   // Forward recomputation: the two-pass prefill in one window keeps every
@@ -1544,7 +1554,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const int64_t P_max = (int64_t)H * ((T + (int64_t)(kC - 1) * N) / kC);
-  bwd_dout_tiles_kernel<<<(unsigned)((P_max + 1) / 2), kThreads, 0, stream>>>(dout, cu, pref, N, H, dot);
+  bwd_dout_tiles_kernel<<<(unsigned)((P_max + 1) / 2), kThreads, 0, stream>>>(dout, cu, pref, N, H, dot, items);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   TmaMaps maps;
@@ -1564,7 +1574,7 @@ cudaError_t launch_backward_tc(const void *q, const void *k, const void *v, cons
 
   BwdItemArgs a;
   a.beta = beta; a.s0_init = init ? s0i : nullptr; a.s0_ck = ck; a.cu = cu; a.pref = pref; a.prefck = prefck;
-  a.dsl = dsl; a.ndu = ndu; a.dot = dot; a.dtp = dtp; a.tt = tt;
+  a.dsl = dsl; a.ndu = ndu; a.dot = dot; a.dtp = dtp; a.tt = tt; a.items = items;
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbeta = dbeta;
   a.N = N; a.H = H; a.dev_status = dev_status; a.wait_ns = wait_ns;
   const size_t smem_i = BItemLayout::TOTAL + 1024;
