@@ -252,10 +252,11 @@ kda_status kda_decode_multi(const void *q, const void *k, const void *v, const f
  * kda_backward_workspace_bytes(shape) (what that query returns for such
  * shapes): the forward is recomputed by the two-pass prefill (its intra-chunk
  * packets and, every 64 tokens, the state as a BF16 tile kept in the
- * workspace), then a chain
- * kernel carries the state gradient backwards chunk by chunk and two kernels,
- * one after the other and each over all (chunk, head) items at once, form
- * every chunk's gradients from 64 x 64 and 64 x 128 tcgen05 products.  The workspace then holds about 250 KB per (64-token chunk, head).
+ * workspace), then a chain kernel carries the state gradient backwards chunk
+ * by chunk and two kernels, one after the other and each over all (chunk,
+ * head) items at once, form every chunk's gradients from 64 x 64 and
+ * 64 x 128 tcgen05 products.  The workspace then holds about 250 KB per
+ * (64-token chunk, head).
  * Other shapes, or a smaller workspace that still covers the SIMT kernel's
  * need, run the FP32 SIMT kernel token by token; kda_last_backward_path tells
  * which ran.

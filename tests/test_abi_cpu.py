@@ -294,7 +294,8 @@ def test_chunked_backward_workspace():
     FP32 (40 KiB together); per full chunk the stored
     forward state as a BF16 operand tile (32 KiB); per (sequence, head) the initial
     state as such a tile; per (chunk, head) the forward's T and (I + M)^-1 as BF16
-    tiles (16 KiB); the forward's output (BF16); two prefix tables."""
+    tiles (16 KiB); the forward's output (BF16); two prefix tables; per (chunk,
+    head) a 32-byte record of where it sits."""
     lib = kda.load()
     al = lambda x: (x + 255) // 256 * 256
     for lengths, H in (([1024] * 4, 32), ([5, 0, 130, 64], 3)):
@@ -304,7 +305,7 @@ def test_chunked_backward_workspace():
         assert P >= H * sum(-(-L // 64) for L in lengths)
         want = (al(P * 74240 + 256) + al((T // 64) * H * 32768) + al(N * H * 32768) + al(P * 16384)
                 + al(P * 32768) + al(P * 16384)
-                + al(P * 16384) + al(P * 40960) + al(T * H * 256) + 2 * al((N + 1) * 8) + 256)
+                + al(P * 16384) + al(P * 40960) + al(T * H * 256) + 2 * al((N + 1) * 8) + al(P * 32) + 256)
         assert lib.kda_backward_workspace_bytes(ctypes.byref(s)) == want
     # FP32 inputs keep the SIMT kernel's workspace
     s = kda.make_shape(4, 4096, 32, 128, 128, 0, kda.KDA_DTYPE_F32)
